@@ -1,0 +1,322 @@
+"""CPU fp64 oracle of the token-choice top-k MoE layer forward.
+
+TEST INFRASTRUCTURE ONLY: this package is the checker the CUDA library is
+compared against.  Only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import it; the library itself never does, and
+it imports nothing from the library.
+
+The arithmetic lives in ``moe_oracle.c`` (plain loops, double precision); this
+module builds it with gcc, marshals numpy arrays in and out through ctypes, and
+strings the steps together in the order the pages give them
+("Lab: build a tiny MoE in PyTorch", section "Full implementation" and
+"Add a capacity limit").
+
+Inputs may be numpy arrays or CPU torch tensors: fp32 arrays, or bf16 data
+given either as a torch bfloat16 tensor or as raw uint16 words.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle_moe.so")
+_lib = None
+_lock = threading.Lock()
+
+F32, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle_moe.so (gcc, OpenMP, -O2)."""
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P = ctypes.c_void_p
+            i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+            lib.oracle_router_logits.argtypes = [i64, i32, i32, P, i32, P, P, P, P]
+            lib.oracle_router_logits.restype = None
+            lib.oracle_route.argtypes = [i64, i32, i32, P, P, P, P, P]
+            lib.oracle_route.restype = i32
+            lib.oracle_router_stats.argtypes = [i64, i32, i32, P, P, P, P, P, P, P]
+            lib.oracle_router_stats.restype = None
+            lib.oracle_capacity.argtypes = [i64, i32, i32, f64]
+            lib.oracle_capacity.restype = i64
+            lib.oracle_dispatch.argtypes = [i64, i32, i32, P, i64, P, P, P, P, P]
+            lib.oracle_dispatch.restype = None
+            lib.oracle_gather.argtypes = [i64, i32, i32, P, i32, P, P]
+            lib.oracle_gather.restype = None
+            lib.oracle_expert_rows.argtypes = [i64, i32, i32, P, P, P, P, i32, P]
+            lib.oracle_expert_rows.restype = None
+            lib.oracle_combine.argtypes = [i64, i32, i32, P, P, P, P]
+            lib.oracle_combine.restype = None
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _elem_array(a):
+    """Return (contiguous numpy array, element-type code) for fp32 / bf16 data."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach()
+            if a.device.type != "cpu":
+                raise ValueError("oracle inputs must be CPU tensors")
+            if a.dtype == torch.bfloat16:
+                return np.ascontiguousarray(a.contiguous().view(torch.int16).numpy().view(np.uint16)), BF16
+            a = a.contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray(a), BF16
+    if a.dtype == np.float32:
+        return np.ascontiguousarray(a), F32
+    raise TypeError(f"unsupported element type {a.dtype}")
+
+
+def _f32(a):
+    if a is None:
+        return None
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu().contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(np.asarray(a))
+    if a.dtype != np.float32:
+        raise TypeError("expected fp32 data")
+    return a
+
+
+def _i32(a):
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu().contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _f64(a):
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().cpu()
+            if a.dtype == torch.bfloat16:
+                a = a.double()  # exact widening
+            a = a.contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def router_logits(x, w_router, bias=None, noise=None) -> np.ndarray:
+    """L[t,e] = x[t] . W_r[:, e] (+ b[e]) (+ noise[t,e]) in fp64, shape (T, E)."""
+    lib = _load()
+    xa, xd = _elem_array(x)
+    w = _f32(w_router)
+    b, nz = _f32(bias), _f32(noise)
+    T, D = xa.shape
+    E = w.shape[1]
+    out = np.empty((T, E), dtype=np.float64)
+    lib.oracle_router_logits(T, D, E, _ptr(xa), xd, _ptr(w), _ptr(b), _ptr(nz), _ptr(out))
+    return out
+
+
+def route(logits, K: int):
+    """Softmax, top-K on (logit desc, id asc) and renormalised weights.
+
+    ``logits`` is (T, E), any real type (fp32 logits convert exactly).
+    Returns ids (T,K) int32, weights (T,K) f64, probs (T,E) f64, lse (T,) f64.
+    """
+    lib = _load()
+    L = _f64(logits)
+    T, E = L.shape
+    if not 1 <= K <= E:
+        raise ValueError("top_k must be in [1, n_experts]")
+    ids = np.empty((T, K), dtype=np.int32)
+    w = np.empty((T, K), dtype=np.float64)
+    probs = np.empty((T, E), dtype=np.float64)
+    lse = np.empty((T,), dtype=np.float64)
+    rc = lib.oracle_route(T, E, K, _ptr(L), _ptr(ids), _ptr(w), _ptr(probs), _ptr(lse))
+    if rc != 0:
+        raise ValueError("non-finite router logit")
+    return ids, w, probs, lse
+
+
+def router_stats(ids, probs, lse, E: int):
+    """counts (E,) int64, mean_prob (E,), z_loss, balance_loss."""
+    lib = _load()
+    ids = _i32(ids)
+    probs, lse = _f64(probs), _f64(lse)
+    T, K = ids.shape
+    counts = np.empty((E,), dtype=np.int64)
+    mp = np.empty((E,), dtype=np.float64)
+    z = ctypes.c_double()
+    bal = ctypes.c_double()
+    lib.oracle_router_stats(T, E, K, _ptr(ids), _ptr(probs), _ptr(lse), _ptr(counts), _ptr(mp),
+                            ctypes.byref(z), ctypes.byref(bal))
+    return counts, mp, z.value, bal.value
+
+
+def capacity(T: int, K: int, E: int, capacity_factor: float) -> int:
+    return int(_load().oracle_capacity(T, K, E, float(capacity_factor)))
+
+
+def dispatch(ids, E: int, C: int) -> dict:
+    """counts, kept, offsets (E+1), perm (sum kept), row_of (T*K) -- all int32."""
+    lib = _load()
+    ids = _i32(ids)
+    T, K = ids.shape
+    counts = np.empty((E,), np.int32)
+    kept = np.empty((E,), np.int32)
+    offsets = np.empty((E + 1,), np.int32)
+    perm = np.full((T * K,), -1, np.int32)
+    row_of = np.empty((T * K,), np.int32)
+    lib.oracle_dispatch(T, K, E, _ptr(ids), int(C), _ptr(counts), _ptr(kept), _ptr(offsets),
+                        _ptr(perm), _ptr(row_of))
+    R = int(offsets[-1])
+    return dict(counts=counts, kept=kept, offsets=offsets, perm=perm[:R].copy(), row_of=row_of)
+
+
+def gather(x, perm, K: int) -> np.ndarray:
+    lib = _load()
+    xa, xd = _elem_array(x)
+    perm = _i32(perm)
+    R = perm.shape[0]
+    D = xa.shape[1]
+    out = np.empty((R, D), np.float64)
+    lib.oracle_gather(R, D, K, _ptr(xa), xd, _ptr(perm), _ptr(out))
+    return out
+
+
+def expert_rows(rows, w_gate_e, w_up_e, w_down_e) -> np.ndarray:
+    """Unweighted SwiGLU expert output for each row of ``rows`` (n, D)."""
+    lib = _load()
+    rows = _f64(rows)
+    wg, wdt = _elem_array(w_gate_e)
+    wu, wdt2 = _elem_array(w_up_e)
+    wd, wdt3 = _elem_array(w_down_e)
+    if not (wdt == wdt2 == wdt3):
+        raise TypeError("expert weights must share one element type")
+    n, D = rows.shape
+    F = wg.shape[1]
+    assert wg.shape == (D, F) and wu.shape == (D, F) and wd.shape == (F, D)
+    out = np.empty((n, D), np.float64)
+    if n:
+        lib.oracle_expert_rows(n, D, F, _ptr(rows), _ptr(wg), _ptr(wu), _ptr(wd), wdt, _ptr(out))
+    return out
+
+
+def combine(o, row_of, weights, T: int, K: int) -> np.ndarray:
+    lib = _load()
+    o = _f64(o)
+    row_of = _i32(row_of)
+    w = _f64(weights)
+    D = o.shape[1] if o.ndim == 2 and o.shape[0] else None
+    if D is None:
+        raise ValueError("combine needs the row width: pass o with shape (R, D), R >= 1")
+    y = np.empty((T, D), np.float64)
+    lib.oracle_combine(T, K, D, _ptr(o), _ptr(row_of), _ptr(w), _ptr(y))
+    return y
+
+
+def _expert_slice(w, e):
+    return w[e]
+
+
+def forward(x, w_router, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
+            bias=None, noise=None, logits=None) -> dict:
+    """The whole layer: route -> dispatch -> experts -> combine.
+
+    When ``logits`` is given (T, E) the router GEMM is skipped and the layer is
+    routed from those logits (parity mode: the CUDA path's fp32 logits).
+    Returns every intermediate: logits, ids, weights, probs, lse, counts,
+    mean_prob, z_loss, balance_loss, capacity, kept, offsets, perm, row_of,
+    o (unweighted expert outputs per row), row_weight (w per row), y.
+    """
+    xa, _ = _elem_array(x)
+    T, D = xa.shape
+    E = _f32(w_router).shape[1]
+    L = router_logits(x, w_router, bias, noise) if logits is None else _f64(logits)
+    ids, w, probs, lse = route(L, K)
+    counts64, mean_prob, z, bal = router_stats(ids, probs, lse, E)
+    C = capacity(T, K, E, capacity_factor)
+    dsp = dispatch(ids, E, C)
+    perm, offsets = dsp["perm"], dsp["offsets"]
+    x_perm = gather(x, perm, K)
+    R = perm.shape[0]
+    o = np.zeros((R, D), np.float64)
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b > a:
+            o[a:b] = expert_rows(x_perm[a:b], _expert_slice(w_gate, e), _expert_slice(w_up, e),
+                                 _expert_slice(w_down, e))
+    wflat = w.reshape(-1)
+    row_weight = wflat[perm] if R else np.zeros((0,), np.float64)
+    y = combine(o, dsp["row_of"], w, T, K) if R else np.zeros((T, D), np.float64)
+    return dict(logits=L, ids=ids, weights=w, probs=probs, lse=lse, counts=dsp["counts"],
+                mean_prob=mean_prob, z_loss=z, balance_loss=bal, capacity=C, kept=dsp["kept"],
+                offsets=offsets, perm=perm, row_of=dsp["row_of"], x_perm=x_perm, o=o,
+                row_weight=row_weight, y=y)
+
+
+def token_outputs(x_rows, slot_ids, slot_weights, slot_kept, get_expert) -> np.ndarray:
+    """Direct per-token layer output for a few tokens ("Trace one token by hand").
+
+    x_rows (n, D) token activations; slot_ids / slot_weights / slot_kept (n, K).
+    get_expert(e) -> (w_gate_e, w_up_e, w_down_e) host arrays of one expert.
+    y[i] = sum over kept slots, in slot order, of w * expert(x_i).
+    Experts are visited one at a time so a caller can stream large weights.
+    """
+    xr = _f64(x_rows)
+    n, D = xr.shape
+    ids = np.asarray(slot_ids)
+    ws = np.asarray(slot_weights, dtype=np.float64)
+    kp = np.asarray(slot_kept, dtype=bool)
+    K = ids.shape[1]
+    outs = np.zeros((n, K, D), np.float64)
+    for e in sorted(set(int(v) for v in ids[kp].reshape(-1))):
+        sel = [(i, k) for i in range(n) for k in range(K) if kp[i, k] and int(ids[i, k]) == e]
+        wg, wu, wd = get_expert(e)
+        o = expert_rows(xr[[i for i, _ in sel]], wg, wu, wd)
+        for j, (i, k) in enumerate(sel):
+            outs[i, k] = o[j]
+    y = np.zeros((n, D), np.float64)
+    for i in range(n):
+        for k in range(K):
+            if kp[i, k]:
+                y[i] += ws[i, k] * outs[i, k]
+    return y

@@ -1,0 +1,339 @@
+/*
+ * moe_oracle.c -- plain CPU fp64 oracle of the token-choice top-k
+ * Mixture-of-Experts layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker that the CUDA library is
+ * compared against.  It shares no code, header, table or helper with the CUDA
+ * path and must never be linked into it.  Only the tests, the smoke check and
+ * the CPU-baseline leg of the benchmark load it.
+ *
+ * Every step is written as plain nested loops in double precision, in the order
+ * the sources give it; OpenMP only splits independent tokens (or rows) across
+ * threads and never changes the order of any sum.
+ *
+ * Sources (web pages; cited by page title and section):
+ *   [TinyMoE]  "Lab: build a tiny MoE in PyTorch" (open-llm-engineering),
+ *              sections "Full implementation", "Add a capacity limit",
+ *              "Trace one token by hand", "Required correctness tests".
+ *   [LLMBook]  "2.9 Mixture-of-Experts (MoE) Architectures" (llm-stack-book),
+ *              sections "The Router: Gating, Top-k, and the Softmax-Then-Select
+ *              Question", "A Toy MoE Layer From Scratch", "The auxiliary
+ *              load-balancing loss", "Capacity Factor, Token Dropping, and the
+ *              Worked Numbers".
+ *
+ * Element types of inputs: 0 = IEEE fp32, 1 = bf16 given as raw 16-bit words.
+ * Both convert exactly to double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_F32 0
+#define ORC_BF16 1
+
+static double elem(const void *p, int32_t dtype, int64_t i)
+{
+    if (dtype == ORC_F32)
+        return (double)((const float *)p)[i];
+    uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/*
+ * Router logits, [TinyMoE] "Full implementation" (router = bias-free linear
+ * layer evaluated in fp32; here in fp64) and [LLMBook] "The Router" (one
+ * logit per expert from a single linear map):
+ *     L[t,e] = sum_d x[t,d] * W_r[d,e]  (+ bias[e])  (+ noise[t,e])
+ * W_r is (D, E) row-major.  bias (E) and noise (T, E) may be NULL.  The bias
+ * is a plain linear bias; the noise is noisy top-k gating's additive logit
+ * noise ([LLMBook] "Noisy / top-k gating"), drawn by the caller.
+ */
+void oracle_router_logits(int64_t T, int32_t D, int32_t E, const void *x, int32_t x_dtype,
+                          const float *w_r, const float *bias, const float *noise,
+                          double *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int32_t d = 0; d < D; ++d)
+                acc += elem(x, x_dtype, t * D + d) * (double)w_r[(int64_t)d * E + e];
+            if (bias)
+                acc += (double)bias[e];
+            if (noise)
+                acc += (double)noise[t * E + e];
+            logits[t * E + e] = acc;
+        }
+    }
+}
+
+/*
+ * Softmax over all E experts, top-K selection and renormalised weights,
+ * [TinyMoE] "Full implementation" (softmax, topk, divide by the sum of the
+ * selected) and [LLMBook] "The Router" (top-k-then-softmax gives the same
+ * weights once renormalised).
+ *
+ * Selection is made on the logits: expert a ranks before expert b iff
+ * L[a] > L[b], or L[a] == L[b] and a < b.  Slot k holds the (k+1)-th expert in
+ * that order.  Since softmax is monotone this is the same choice as ranking
+ * the probabilities.
+ *
+ *     m    = max_e L[t,e]
+ *     p_e  = exp(L_e - m) / sum_e' exp(L_e' - m)
+ *     lse  = m + log sum_e exp(L_e - m)
+ *     w_k  = p[id_k] / sum_j p[id_j]
+ *
+ * probs (T, E) may be NULL.  Returns 0, or -1 if a logit is not finite.
+ */
+int32_t oracle_route(int64_t T, int32_t E, int32_t K, const double *logits, int32_t *ids,
+                     double *weights, double *probs, double *lse)
+{
+    int32_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int64_t t = 0; t < T; ++t) {
+        const double *L = logits + t * E;
+        double m = L[0];
+        for (int32_t e = 0; e < E; ++e) {
+            if (!isfinite(L[e]))
+                bad = 1;
+            if (L[e] > m)
+                m = L[e];
+        }
+        double s = 0.0;
+        for (int32_t e = 0; e < E; ++e)
+            s += exp(L[e] - m);
+        if (lse)
+            lse[t] = m + log(s);
+        if (probs)
+            for (int32_t e = 0; e < E; ++e)
+                probs[t * E + e] = exp(L[e] - m) / s;
+
+        /* K passes, each picking the best expert not yet taken. */
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                int32_t taken = 0;
+                for (int32_t j = 0; j < k; ++j)
+                    if (ids[t * K + j] == e)
+                        taken = 1;
+                if (taken)
+                    continue;
+                if (best < 0 || L[e] > L[best])
+                    best = e; /* strict '>' keeps the lower id on ties */
+            }
+            ids[t * K + k] = best;
+        }
+        double sel = 0.0;
+        for (int32_t k = 0; k < K; ++k)
+            sel += exp(L[ids[t * K + k]] - m) / s;
+        for (int32_t k = 0; k < K; ++k)
+            weights[t * K + k] = (exp(L[ids[t * K + k]] - m) / s) / sel;
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Router statistics, [TinyMoE] "Full implementation" (Switch-style top-k
+ * balance loss and ST-MoE z-loss) and [LLMBook] "The auxiliary load-balancing
+ * loss":
+ *     counts_e = #{(t,k) : ids[t,k] = e}          (before any capacity drop)
+ *     f_e      = counts_e / (T*K)
+ *     P_e      = (1/T) sum_t p[t,e]
+ *     balance  = E * sum_e f_e * P_e
+ *     z        = (1/T) sum_t lse_t^2
+ * The raw, unweighted values (the loss coefficients are the caller's).
+ */
+void oracle_router_stats(int64_t T, int32_t E, int32_t K, const int32_t *ids, const double *probs,
+                         const double *lse, int64_t *counts, double *mean_prob, double *z_loss,
+                         double *balance_loss)
+{
+    for (int32_t e = 0; e < E; ++e) {
+        counts[e] = 0;
+        mean_prob[e] = 0.0;
+    }
+    for (int64_t i = 0; i < T * K; ++i)
+        counts[ids[i]] += 1;
+    for (int32_t e = 0; e < E; ++e) {
+        double s = 0.0;
+        for (int64_t t = 0; t < T; ++t)
+            s += probs[t * E + e];
+        mean_prob[e] = s / (double)T;
+    }
+    double bal = 0.0;
+    for (int32_t e = 0; e < E; ++e)
+        bal += ((double)counts[e] / (double)(T * K)) * mean_prob[e];
+    *balance_loss = (double)E * bal;
+    double z = 0.0;
+    for (int64_t t = 0; t < T; ++t)
+        z += lse[t] * lse[t];
+    *z_loss = z / (double)T;
+}
+
+/*
+ * Expert capacity, [TinyMoE] "Add a capacity limit" and [LLMBook] "A Toy MoE
+ * Layer From Scratch": C = max(1, ceil(cf * T * K / E)), evaluated in double.
+ * cf <= 0 means dropless; then C = T*K, which no expert can exceed.
+ */
+int64_t oracle_capacity(int64_t T, int32_t K, int32_t E, double cf)
+{
+    if (!(cf > 0.0))
+        return T * (int64_t)K;
+    double c = ceil(cf * (double)T * (double)K / (double)E);
+    if (c < 1.0)
+        c = 1.0;
+    return (int64_t)c;
+}
+
+/*
+ * Dispatch layout, [TinyMoE] "Add a capacity limit" (first-come keep mask:
+ * walk tokens in order and their slots in order; an assignment is kept while
+ * its expert has used fewer than C places) and "From local loop to expert
+ * parallelism" (group rows by expert).
+ *
+ *   counts[e]  assignments that chose e (before drops)
+ *   kept[e]    assignments of e that were kept
+ *   offsets    exclusive prefix sum of kept, E+1 entries
+ *   perm[row]  = t*K + k for the assignment stored at that row; the rows of
+ *              expert e are offsets[e] .. offsets[e+1]-1 and hold its kept
+ *              assignments in increasing token order
+ *   row_of[t*K+k] = its row, or -1 when the assignment was dropped
+ */
+void oracle_dispatch(int64_t T, int32_t K, int32_t E, const int32_t *ids, int64_t C,
+                     int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *perm,
+                     int32_t *row_of)
+{
+    int64_t *used = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    unsigned char *keep = (unsigned char *)calloc((size_t)(T * K), 1);
+    for (int32_t e = 0; e < E; ++e) {
+        counts[e] = 0;
+        kept[e] = 0;
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t e = ids[t * K + k];
+            counts[e] += 1;
+            if (used[e] < C) {
+                keep[t * K + k] = 1;
+                used[e] += 1;
+            }
+        }
+    }
+    for (int32_t e = 0; e < E; ++e)
+        kept[e] = (int32_t)used[e];
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + kept[e];
+    int64_t *cursor = used; /* reuse: next free row of each expert */
+    for (int32_t e = 0; e < E; ++e)
+        cursor[e] = offsets[e];
+    for (int64_t i = 0; i < T * K; ++i) {
+        if (keep[i]) {
+            int32_t e = ids[i];
+            int64_t row = cursor[e]++;
+            perm[row] = (int32_t)i;
+            row_of[i] = (int32_t)row;
+        } else {
+            row_of[i] = -1;
+        }
+    }
+    free(keep);
+    free(used);
+}
+
+/*
+ * Gather each expert's token rows, [TinyMoE] "Full implementation"
+ * (flat[token_index]): x_perm[row, :] = x[perm[row] / K, :].
+ */
+void oracle_gather(int64_t R, int32_t D, int32_t K, const void *x, int32_t x_dtype,
+                   const int32_t *perm, double *x_perm)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        int64_t t = perm[r] / K;
+        for (int32_t d = 0; d < D; ++d)
+            x_perm[r * D + d] = elem(x, x_dtype, t * D + d);
+    }
+}
+
+/*
+ * One SwiGLU expert on a block of rows, [TinyMoE] "Full implementation"
+ * (SwiGLUExpert: down(silu(gate(x)) * up(x)), no biases):
+ *     g_f = sum_d x_d Wg[d,f],  u_f = sum_d x_d Wu[d,f]
+ *     h_f = g_f / (1 + exp(-g_f)) * u_f
+ *     o_j = sum_f h_f Wd[f,j]
+ * wg, wu point at this expert's (D, F) matrices, wd at its (F, D) matrix, all
+ * row-major, element type w_dtype.  rows_in (n, D), rows_out (n, D).
+ */
+void oracle_expert_rows(int64_t n, int32_t D, int32_t F, const double *rows_in, const void *wg,
+                        const void *wu, const void *wd, int32_t w_dtype, double *rows_out)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+        double *g = (double *)malloc(sizeof(double) * (size_t)F);
+        double *u = (double *)malloc(sizeof(double) * (size_t)F);
+        const double *xr = rows_in + r * D;
+        for (int32_t f = 0; f < F; ++f) {
+            g[f] = 0.0;
+            u[f] = 0.0;
+        }
+        for (int32_t d = 0; d < D; ++d) {
+            double xd = xr[d];
+            for (int32_t f = 0; f < F; ++f) {
+                g[f] += xd * elem(wg, w_dtype, (int64_t)d * F + f);
+                u[f] += xd * elem(wu, w_dtype, (int64_t)d * F + f);
+            }
+        }
+        for (int32_t f = 0; f < F; ++f)
+            g[f] = g[f] / (1.0 + exp(-g[f])) * u[f]; /* h_f */
+        double *o = rows_out + r * D;
+        for (int32_t j = 0; j < D; ++j)
+            o[j] = 0.0;
+        for (int32_t f = 0; f < F; ++f) {
+            double hf = g[f];
+            for (int32_t j = 0; j < D; ++j)
+                o[j] += hf * elem(wd, w_dtype, (int64_t)f * D + j);
+        }
+        free(g);
+        free(u);
+    }
+}
+
+/*
+ * Weighted combine back to token order, [TinyMoE] "Full implementation"
+ * (index_add_ of weight * expert output) and "Add a capacity limit" (a dropped
+ * assignment adds nothing; an all-dropped token gets zero):
+ *     y[t, :] = sum over kept slots k, in slot order, of w[t,k] * o[row_of[t*K+k], :]
+ * o holds the unweighted expert outputs in row order (R, D).
+ */
+void oracle_combine(int64_t T, int32_t K, int32_t D, const double *o, const int32_t *row_of,
+                    const double *weights, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double *yt = y + t * D;
+        for (int32_t j = 0; j < D; ++j)
+            yt[j] = 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t row = row_of[t * K + k];
+            if (row < 0)
+                continue;
+            double w = weights[t * K + k];
+            for (int32_t j = 0; j < D; ++j)
+                yt[j] += w * o[(int64_t)row * D + j];
+        }
+    }
+}
+
+/* Threads OpenMP will use (1 when built without OpenMP). */
+int32_t oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return (int32_t)omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
