@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward: routed tokens/s on B200.
+
+One step = one whole layer forward (router, dispatch, grouped SwiGLU experts,
+combine) over one batch of T tokens, through moe_forward.  Default workload:
+the Mixtral-shaped dropless layer (T=8192, D=4096, F=14336, E=8, K=2, bf16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+N > 1 runs under torchrun: one independent replica per GPU (the layer is
+per-token, so ranks share nothing on the data path); value = all ranks'
+tokens / the slowest rank's device time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, Workload, make_inputs, make_tokens  # noqa: E402
+
+METRIC = "routed tokens/s per MoE layer fwd on 1 B200; % bf16 tensor peak / % HBM BW"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# kernels this library launches per moe_forward (router 3, dispatch 3, gather 1,
+# expert GEMMs 2, combine 1)
+LAUNCHES_PER_STEP = 10
+
+
+# ------------------------------------------------------------------ ranks --
+
+def rank_info():
+    r = int(os.environ.get("RANK", "0"))
+    w = int(os.environ.get("WORLD_SIZE", "1"))
+    lr = int(os.environ.get("LOCAL_RANK", str(r)))
+    return r, w, lr
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_token_seed(rank: int) -> int:
+    """Each replica routes its own batch of tokens (weights are shared)."""
+    return 1000 + rank
+
+
+# ------------------------------------------------------------------ peaks --
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sms.append(float(parts[0]))
+                maxs.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ------------------------------------------------------------- the layer --
+
+def algorithmic(wl: Workload, counts, kept_rows: int):
+    """Algorithmic work of one step (the units of the roofline)."""
+    s = wl.elem_bytes
+    R = kept_rows
+    return {
+        "gateup_flop": 4.0 * R * wl.D * wl.F,
+        "down_flop": 2.0 * R * wl.F * wl.D,
+        "dispatch_bytes": float(wl.T * wl.D * s + R * wl.D * s),
+        "combine_bytes": float(R * wl.D * s + wl.T * wl.D * s),
+        "active_weight_bytes": float(sum(1 for c in counts if c > 0) * 3 * wl.D * wl.F * s),
+    }
+
+
+def kernel_source_hash() -> str:
+    csrc = os.path.join(ROOT, "mixture_experts_layer_55_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernels have
+    not changed since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_gpu(args):
+    import mixture_experts_layer_55_b200 as M
+
+    rank, world, local_rank = rank_info()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    init_dist(world, "nccl")
+    wl = WORKLOADS[args.workload]
+
+    inp = make_inputs(wl, device=dev)
+    layer = M.MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
+                       wl.capacity_factor, router_bias=inp["bias"])
+    noise = inp["noise"]
+    # a few batches of tokens, rotated between steps
+    nbuf = 3
+    xs = [make_tokens(wl, device=dev, seed=rank_token_seed(rank) * 16 + i) for i in range(nbuf)]
+    y = torch.empty_like(xs[0])
+    stream = torch.cuda.current_stream(dev)
+
+    # ---------------- device-resident timing (value) ----------------
+    for i in range(args.warmup):
+        layer.forward(xs[i % nbuf], y, logit_noise=noise)
+    torch.cuda.synchronize(dev)
+    nb = M._binding.lib().moe_trace_boundary_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(args.steps):
+        M.moe_trace_attach(evs[i])
+        layer.forward(xs[i % nbuf], y, logit_noise=noise)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    M.moe_trace_attach([])
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(stop)
+    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_step = ms_total / args.steps
+    value = world * wl.T / (ms_step / 1e3)
+
+    names = M.trace_stage_names()
+    stage_ms = {}
+    for j in range(1, nb):
+        d = [evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(args.steps)]
+        stage_ms[names[j]] = sum(d) / len(d)
+
+    counts = layer.counts.cpu().tolist()
+    kept_rows = int(min(sum(min(c, M.capacity(layer.cfg)) for c in counts), M.max_rows(layer.cfg)))
+    alg = algorithmic(wl, counts, kept_rows)
+
+    # ---------------- end to end from pinned host memory (e2e) ----------------
+    x_host = xs[0].cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(xs[0])
+    y_dev = torch.empty_like(xs[0])
+    for _ in range(max(1, args.warmup)):
+        layer.forward_host(x_host, y_host, x_dev, y_dev, logit_noise=noise)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward_host(x_host, y_host, x_dev, y_dev, logit_noise=noise)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    io_bytes = wl.T * wl.D * wl.elem_bytes
+
+    flags = M.moe_get_device_status(layer.workspace)
+    if flags:
+        raise RuntimeError(f"device status flags {flags:#x} after the benchmark")
+
+    if rank != 0:
+        _finish(world)
+        return
+
+    peaks, peak_src = load_peaks()
+    long_region = ms_total > 1000.0
+    if wl.dtype == "bf16":
+        key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
+        gu_ms = stage_ms["expert_gate_up"]
+        achieved = alg["gateup_flop"] / (gu_ms / 1e3) / 1e12
+        roofline = {"kernel": "expert_gate_up (grouped GEMM + SwiGLU)", "bound": "tensor",
+                    "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4),
+                    "peak_source": f"{key} of {peak_src}",
+                    "traffic": recorded_traffic(wl.name, "expert_gate_up")}
+    else:
+        # fp32 layer: SIMT FMA pipes; peak from unit counts and the clock:
+        # 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock
+        sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+        gu_ms = stage_ms["expert_gate_up"]
+        achieved = alg["gateup_flop"] / (gu_ms / 1e3) / 1e12
+        roofline = {"kernel": "expert_gate_up (fp32 SIMT)", "bound": "alu",
+                    "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "peak_source": "148 SMs x 128 FMA x 2 x max clock",
+                    "traffic": recorded_traffic(wl.name, "expert_gate_up")}
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    stages = {}
+    for name, ms in stage_ms.items():
+        ent = {"ms": round(ms, 4)}
+        if name == "gather":
+            gbs = alg["dispatch_bytes"] / (ms / 1e3) / 1e9
+            ent.update(GBs=round(gbs, 1), hbm_frac=round(gbs / hbm, 4))
+        elif name == "combine":
+            gbs = alg["combine_bytes"] / (ms / 1e3) / 1e9
+            ent.update(GBs=round(gbs, 1), hbm_frac=round(gbs / hbm, 4))
+        elif name == "expert_gate_up":
+            ent.update(TFLOPs=round(alg["gateup_flop"] / (ms / 1e3) / 1e12, 1))
+        elif name == "expert_down":
+            ent.update(TFLOPs=round(alg["down_flop"] / (ms / 1e3) / 1e12, 1))
+        stages[name] = ent
+    ffn_ms = stage_ms["expert_gate_up"] + stage_ms["expert_down"]
+    weights_gbs = alg["active_weight_bytes"] / (ffn_ms / 1e3) / 1e9
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) random-init weights)",
+        "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
+                   "capacity_factor": wl.capacity_factor, "router_bias": wl.bias,
+                   "logit_noise": wl.noise, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (expert weights "
+                         f"{3 * wl.E * wl.D * wl.F * wl.elem_bytes / 1e9:.2f} GB read per step)"},
+        "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io_bytes,
+                "d2h_bytes_per_step": io_bytes},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "roofline": roofline,
+        "stages": stages,
+        "layer": {"assignments_per_s": round(world * wl.T * wl.K / (ms_step / 1e3), 1),
+                  "kept_rows": kept_rows, "max_over_mean_load": round(
+                      max(counts) / (sum(counts) / len(counts)), 3),
+                  "expert_weights_GBs": round(weights_gbs, 1),
+                  "expert_tflops": round((alg["gateup_flop"] + alg["down_flop"]) / (ffn_ms / 1e3) / 1e12, 1)},
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if args.warmup < 3:
+        line["note"] = "fewer than 3 warm-up steps: not a valid measurement"
+
+    print(json.dumps(line), flush=True)
+    _finish(world)
+
+
+def _finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def cpu_baseline(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
+    """Time the oracle as it stands on a bounded sample of the workload.
+
+    Router logits + routing + dispatch layout for all T tokens, then the expert
+    FFN and combine for a sample of tokens (grown until the time budget is
+    used).  value = tokens/s extrapolated from the per-token costs.
+    """
+    import numpy as np
+
+    import oracle
+    torch.manual_seed(seed)
+    cpu_inp = _cpu_inputs_for_sample(wl)
+    t0 = time.perf_counter()
+    L = oracle.router_logits(cpu_inp["x"], cpu_inp["w_router"], cpu_inp["bias"], cpu_inp["noise"])
+    ids, w, probs, lse = oracle.route(L, wl.K)
+    oracle.router_stats(ids, probs, lse, wl.E)
+    C = oracle.capacity(wl.T, wl.K, wl.E, wl.capacity_factor)
+    d = oracle.dispatch(ids, wl.E, C)
+    t_route = time.perf_counter() - t0
+    kept = d["row_of"].reshape(wl.T, wl.K) >= 0
+    get = cpu_inp["get_expert"]
+    n, t_ffn = 0, 0.0
+    budget = max(1.0, seconds - t_route)
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(wl.T)
+    batch = 1
+    while t_ffn < budget and n < wl.T:
+        toks = sorted(order[n:n + batch].tolist())
+        t1 = time.perf_counter()
+        oracle.token_outputs(cpu_inp["x"][toks], ids[toks], w[toks], kept[toks], get)
+        t_ffn += time.perf_counter() - t1
+        n += len(toks)
+        batch = min(batch * 2, 64)
+    per_token = t_route / wl.T + t_ffn / n
+    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"router + routing + dispatch layout on all {wl.T} tokens "
+                       f"({t_route:.2f} s), expert FFN + combine on {n} sampled tokens "
+                       f"({t_ffn:.2f} s); value extrapolated per token")}
+
+
+def _cpu_inputs_for_sample(wl: Workload):
+    """Host inputs for the CPU baseline: the activations, router and, for the
+    experts, one expert at a time (generated on demand, seeded per expert)."""
+    small = wl.E * wl.D * wl.F * wl.elem_bytes * 3 < (2 << 30)
+    if small:
+        inp = make_inputs(wl, device="cpu")
+        get = (lambda e: (inp["w_gate"][e], inp["w_up"][e], inp["w_down"][e]))
+        return dict(inp, get_expert=get)
+    # large layers: same shapes and distributions; experts drawn on demand
+    x = make_tokens(wl, device="cpu", seed=7)
+    g = torch.Generator().manual_seed(wl.seed)
+    w_router = (torch.randn(wl.D, wl.E, generator=g) * wl.w_std).float()
+    from workloads import zipf_bias
+    bias = zipf_bias(wl.E) if wl.bias == "zipf" else None
+    noise = None
+    if wl.noise:
+        noise = torch.randn(wl.T, wl.E, generator=torch.Generator().manual_seed(wl.seed + 1)) / wl.E
+    cache = {}
+
+    def get(e):
+        if e not in cache:
+            cache.clear()
+            ge = torch.Generator().manual_seed(10_000 + e)
+            mk = (lambda *s: (torch.randn(*s, generator=ge) * wl.w_std).to(wl.torch_dtype))
+            cache[e] = (mk(wl.D, wl.F), mk(wl.D, wl.F), mk(wl.F, wl.D))
+        return cache[e]
+    return dict(x=x, w_router=w_router, bias=bias, noise=noise, get_expert=get)
+
+
+def run_reference(args):
+    """The oracle on the host cores, timed per step on a bounded sample."""
+    rank, world, _ = rank_info()
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    per_step = max(2.0, args.cpu_seconds / 2)
+    if args.warmup > 0:
+        cpu_baseline(wl, min(per_step, 4.0) / 2)
+    vals = []
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        vals.append(cpu_baseline(wl, per_step, seed=i))
+        if time.perf_counter() - t0 > 240:
+            break
+    value = statistics.median(v["value"] for v in vals)
+    ms_step = 1e3 * wl.T / value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": len(vals), "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
+                   "capacity_factor": wl.capacity_factor, "parallelism": "host cores (oracle)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_8x", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

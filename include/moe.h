@@ -1,0 +1,251 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: the forward pass of a token-choice top-k
+ * Mixture-of-Experts layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources cited by page title and section):
+ *   "Lab: build a tiny MoE in PyTorch" (open-llm-engineering), sections
+ *   "The contract", "Full implementation", "Add a capacity limit";
+ *   "2.9 Mixture-of-Experts (MoE) Architectures" (llm-stack-book), sections
+ *   "The Router", "A Toy MoE Layer From Scratch", "Capacity Factor, Token
+ *   Dropping, and the Worked Numbers".
+ *
+ *   y = sum over the K experts a token selects of w_k * Expert_{id_k}(x),
+ *   Expert_e(x) = (silu(x Wg_e) * (x Wu_e)) Wd_e,
+ *   ids = top-K of the router logits x W_r (+ bias) (+ noise), ties to the
+ *   lower expert id; w = softmax probabilities of the selected experts,
+ *   renormalised to sum to one; with a capacity factor, each expert keeps its
+ *   first C assignments in token order and the rest contribute zero.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument named as a buffer is a DEVICE pointer unless
+ *     stated otherwise; the caller allocates and owns every buffer.  The
+ *     library allocates no device or host memory and never synchronises the
+ *     host, except moe_get_device_status.
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued on it, asynchronously.
+ *   - Layouts are row-major and dense:
+ *       x (T, D), y (T, D), w_router (D, E) fp32, router_bias (E) fp32,
+ *       logit_noise (T, E) fp32, w_gate / w_up (E, D, F), w_down (E, F, D),
+ *       x_perm / y_perm (max_rows, D), h (max_rows, F),
+ *       topk_ids (T, K) int32, topk_w (T, K) fp32, probs (T, E) fp32.
+ *     dtype (moe_config.dtype) is the element type of x, y, the expert
+ *     weights, x_perm, h and y_perm; router arithmetic is always fp32.
+ *   - Alignment: D and F must be multiples of 8, and every buffer must start
+ *     on a 16-byte boundary (MOE_ERR_ALIGN otherwise).
+ *   - Errors in the arguments are reported before anything is enqueued, and
+ *     nothing is enqueued then.  A failure in the CUDA runtime returns
+ *     MOE_ERR_CUDA.  Faults found on the device (an index out of range, a
+ *     wait that gave up) are recorded in the workspace status word and read
+ *     with moe_get_device_status.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_ARG = -1,            /* K outside [1, min(E, 8)], E > 256, a NULL required pointer, a bad enum */
+    MOE_ERR_SHAPE = -2,          /* T, D, F or E below 1, or T*K beyond 2^31 - 1 */
+    MOE_ERR_UNSUPPORTED = -3,    /* an option this build does not implement */
+    MOE_ERR_ALIGN = -4,          /* D or F not a multiple of 8, or a buffer not 16-byte aligned */
+    MOE_ERR_CUDA = -5,           /* a CUDA runtime call failed */
+    MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel gave up a bounded wait (device status) */
+    MOE_ERR_DEVICE_BOUNDS = -7,  /* a kernel met an index out of range (device status) */
+    MOE_ERR_WORKSPACE = -8       /* workspace NULL or smaller than the size query returned */
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Router score function.  Only the softmax router of the sources is built. */
+typedef enum moe_score_func { MOE_SCORE_SOFTMAX = 0 } moe_score_func;
+
+/* Device status flags (bit set), as read by moe_get_device_status. */
+#define MOE_DEVFLAG_TIMEOUT 0x1
+#define MOE_DEVFLAG_BOUNDS 0x2
+
+typedef struct moe_config {
+    int64_t T;             /* tokens = batch * sequence, >= 1 */
+    int32_t D;             /* d_model, multiple of 8 */
+    int32_t F;             /* expert hidden size d_hidden, multiple of 8 */
+    int32_t E;             /* number of experts, 1..256 */
+    int32_t K;             /* experts per token (top-k), 1..min(E, 8) */
+    float capacity_factor; /* <= 0: dropless; > 0: C = max(1, ceil(cf * T * K / E)) */
+    int32_t score_func;    /* moe_score_func; MOE_SCORE_SOFTMAX */
+    int32_t renormalize;   /* 1: selected weights renormalised to sum to one (only value) */
+    int32_t dtype;         /* moe_dtype */
+} moe_config;
+
+/* Returns a static, NUL-terminated description of a status code. */
+MOE_API const char *moe_status_string(int32_t status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+MOE_API int32_t moe_version(void);
+
+/* Validates a configuration (no device work).  MOE_OK or the error code. */
+MOE_API moe_status moe_check_config(const moe_config *cfg);
+
+/*
+ * Expert capacity C ("Lab: build a tiny MoE in PyTorch", section "Add a
+ * capacity limit"): max(1, ceil(cf * T * K / E)) computed in double; T*K when
+ * dropless.  Host-only.
+ */
+MOE_API moe_status moe_capacity(const moe_config *cfg, int64_t *capacity);
+
+/*
+ * Upper bound on the kept assignments R: T*K dropless, else min(T*K, E*C).
+ * Rows of x_perm, h and y_perm must be allocated for this many.  Host-only.
+ */
+MOE_API moe_status moe_max_rows(const moe_config *cfg, int64_t *rows);
+
+/*
+ * Bytes of device workspace that moe_route, moe_dispatch and moe_expert_ffn
+ * need (the same buffer serves all three; it holds the device status word and
+ * per-block partials).  The workspace must be 256-byte aligned and zeroed
+ * once before first use (the status word must start at zero).
+ */
+MOE_API moe_status moe_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/*
+ * Bytes of device workspace moe_forward needs: the above plus every
+ * intermediate of the layer (routing, dispatch layout, x_perm, h, y_perm).
+ */
+MOE_API moe_status moe_forward_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/*
+ * Router: "Lab: build a tiny MoE in PyTorch", section "Full implementation"
+ * (fp32 router logits, softmax, top-k, renormalised weights, balance loss and
+ * router z-loss) and "2.9 Mixture-of-Experts (MoE) Architectures", section
+ * "The Router" (noisy top-k gating adds noise to the logits before top-k).
+ *
+ *   L[t,e]  = sum_d x[t,d] W_r[d,e] + router_bias[e] + logit_noise[t,e]   (fp32)
+ *   p[t,:]  = softmax(L[t,:])
+ *   ids[t,:]= the K experts of largest L[t,e], ties to the lower id, in
+ *             descending order
+ *   w[t,k]  = p[t,ids[t,k]] / sum_j p[t,ids[t,j]]
+ *   mean_prob[e] = (1/T) sum_t p[t,e]
+ *   losses[0] = z-loss = (1/T) sum_t (logsumexp_e L[t,e])^2
+ *   losses[1] = balance = E * sum_e (counts_e / (T*K)) * mean_prob[e],
+ *               counts_e = assignments to e before any capacity drop.
+ *
+ * x (T, D) dtype; w_router (D, E) fp32.  router_bias (E) and logit_noise
+ * (T, E) may be NULL.  logits_in (T, E), if not NULL, are taken as the
+ * complete routing logits: x, w_router, bias and noise are then not read and
+ * may be NULL.  logits_out (T, E) and probs_out (T, E) may be NULL.
+ * topk_ids (T, K) and topk_w (T, K) are required.  mean_prob (E) and
+ * losses (2) may be NULL; the statistics are then skipped.
+ * The reductions behind mean_prob and losses run in a fixed order
+ * (deterministic run to run).
+ */
+MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router,
+                     const float *router_bias, const float *logit_noise, const float *logits_in,
+                     float *logits_out, float *probs_out, int32_t *topk_ids, float *topk_w,
+                     float *mean_prob, float *losses, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
+/*
+ * Dispatch: per-expert histogram, capacity drop, exclusive-scan offsets and a
+ * stable expert-major permutation, then the gather of token rows.
+ * "Lab: build a tiny MoE in PyTorch", sections "Full implementation" (bincount,
+ * gather flat[token_index]) and "Add a capacity limit" (first C assignments of
+ * each expert in token order are kept).
+ *
+ *   counts[e]  = #{(t,k) : topk_ids[t,k] = e}                    (E)
+ *   kept[e]    = min(counts[e], C)                                (E)
+ *   offsets    = exclusive prefix sum of kept, offsets[E] = R     (E+1)
+ *   perm[row]  = t*K + k of the assignment stored at row; the rows of expert e
+ *                are offsets[e] .. offsets[e+1]-1, in increasing t  (max_rows)
+ *   row_of[t*K+k] = its row, or -1 if dropped                     (T*K)
+ *   x_perm[row, :] = x[perm[row] / K, :]                          (max_rows, D)
+ *
+ * Every output is fully determined (bit-exact run to run).  x and x_perm may
+ * both be NULL: only the index arrays are then produced.  Entries of perm and
+ * rows of x_perm at and beyond R are left untouched.
+ */
+MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_ids,
+                        int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *perm,
+                        int32_t *row_of, void *x_perm, void *workspace, size_t workspace_bytes,
+                        void *stream);
+
+/*
+ * Grouped SwiGLU experts over each expert's contiguous row block, with the
+ * routing weight applied to the output.  "Lab: build a tiny MoE in PyTorch",
+ * section "Full implementation" (SwiGLUExpert: down(silu(gate x) * up x), no
+ * biases; each expert output scaled by its combine weight).
+ *
+ * For every row r < offsets[E] of expert e (offsets[e] <= r < offsets[e+1]):
+ *   h[r, :]      = silu(x_perm[r] Wg_e) * (x_perm[r] Wu_e)        (dtype)
+ *   y_perm[r, :] = topk_w[perm[r]] * (h[r] Wd_e)                  (dtype)
+ * with fp32 accumulation, silu(z) = z / (1 + exp(-z)).  bf16 runs on tcgen05
+ * tensor cores; fp32 runs in true fp32 (no TF32).
+ * h is a caller-provided intermediate of max_rows x F elements.  offsets,
+ * perm and topk_w are device arrays as produced by moe_dispatch / moe_route.
+ */
+MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                          const int32_t *perm, const float *topk_w, const void *w_gate,
+                          const void *w_up, const void *w_down, void *h, void *y_perm,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Combine back to token order.  "Lab: build a tiny MoE in PyTorch", sections
+ * "Full implementation" (index_add_ of weighted expert outputs) and "Add a
+ * capacity limit" (an all-dropped token returns zero).
+ *
+ *   y[t, :] = sum over k = 0..K-1 with row_of[t*K+k] >= 0 of y_perm[row_of[t*K+k], :]
+ * summed in slot order in fp32 and rounded once to dtype (deterministic; the
+ * routing weight was applied by moe_expert_ffn).
+ */
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *row_of, void *y,
+                       void *stream);
+
+/*
+ * The whole layer: moe_route -> moe_dispatch -> moe_expert_ffn -> moe_combine
+ * on one stream, every intermediate in the workspace
+ * (moe_forward_workspace_size bytes).  y (T, D) dtype is required; losses (2),
+ * mean_prob (E), counts (E, before drops), topk_ids (T, K) and topk_w (T, K)
+ * are optional copies of the routing results (NULL to skip).
+ */
+MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *w_router,
+                       const float *router_bias, const float *logit_noise, const void *w_gate,
+                       const void *w_up, const void *w_down, void *y, float *losses,
+                       float *mean_prob, int32_t *counts, int32_t *topk_ids, float *topk_w,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Device status of a workspace: synchronises the stream, then reads the
+ * status word.  *flags receives MOE_DEVFLAG_* bits (0 when clean).  Returns
+ * MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BOUNDS when a flag is set, MOE_OK
+ * otherwise.  moe_clear_device_status enqueues a reset of the word.
+ */
+MOE_API moe_status moe_get_device_status(const void *workspace, void *stream, int32_t *flags);
+MOE_API moe_status moe_clear_device_status(void *workspace, void *stream);
+
+/*
+ * Kernel-boundary tracing for timing.  After moe_trace_attach(events, n),
+ * moe_forward records events[i] (cudaEvent_t values passed as void*) on its
+ * stream at each of the first n stage boundaries: 0 before the first kernel,
+ * then after the router, the dispatch index pass, the gather, the gate/up
+ * GEMM, the down GEMM and the combine (7 boundaries; moe_trace_stage_name
+ * names the stage that ends at boundary i).  moe_trace_attach(NULL, 0)
+ * detaches.  The table is process-wide and not thread-safe.
+ */
+MOE_API moe_status moe_trace_attach(void *const *events, int32_t n_events);
+MOE_API int32_t moe_trace_boundary_count(void);
+MOE_API const char *moe_trace_stage_name(int32_t boundary);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

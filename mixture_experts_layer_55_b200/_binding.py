@@ -1,0 +1,246 @@
+"""ctypes binding of libmoe_b200.so (the C ABI declared in include/moe.h).
+
+Argument marshalling only: tensors become device pointers, the current torch
+stream becomes the cudaStream_t, and a non-OK status becomes MoEError.  Every
+step of the layer runs in the library's CUDA kernels; nothing here computes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "moe.h")
+
+MOE_OK = 0
+MOE_ERR_ARG = -1
+MOE_ERR_SHAPE = -2
+MOE_ERR_UNSUPPORTED = -3
+MOE_ERR_ALIGN = -4
+MOE_ERR_CUDA = -5
+MOE_ERR_DEVICE_TIMEOUT = -6
+MOE_ERR_DEVICE_BOUNDS = -7
+MOE_ERR_WORKSPACE = -8
+
+MOE_F32 = 0
+MOE_BF16 = 1
+MOE_SCORE_SOFTMAX = 0
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int64),
+        ("D", ctypes.c_int32),
+        ("F", ctypes.c_int32),
+        ("E", ctypes.c_int32),
+        ("K", ctypes.c_int32),
+        ("capacity_factor", ctypes.c_float),
+        ("score_func", ctypes.c_int32),
+        ("renormalize", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+    @classmethod
+    def make(cls, T, D, F, E, K, dtype="bf16", capacity_factor=0.0, score_func=MOE_SCORE_SOFTMAX,
+             renormalize=1):
+        dt = {"bf16": MOE_BF16, "f32": MOE_F32, MOE_BF16: MOE_BF16, MOE_F32: MOE_F32}[dtype]
+        return cls(int(T), int(D), int(F), int(E), int(K), float(capacity_factor), int(score_func),
+                   int(renormalize), dt)
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_SIG = {
+    "moe_status_string": ([ctypes.c_int32], ctypes.c_char_p),
+    "moe_version": ([], ctypes.c_int32),
+    "moe_check_config": ([_P], ctypes.c_int32),
+    "moe_capacity": ([_P, _P], ctypes.c_int32),
+    "moe_max_rows": ([_P, _P], ctypes.c_int32),
+    "moe_workspace_size": ([_P, _P], ctypes.c_int32),
+    "moe_forward_workspace_size": ([_P, _P], ctypes.c_int32),
+    "moe_route": ([_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_dispatch": ([_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_expert_ffn": ([_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_combine": ([_P] * 5, ctypes.c_int32),
+    "moe_forward": ([_P] * 15 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_get_device_status": ([_P, _P, _P], ctypes.c_int32),
+    "moe_clear_device_status": ([_P, _P], ctypes.c_int32),
+    "moe_trace_attach": ([_P, ctypes.c_int32], ctypes.c_int32),
+    "moe_trace_boundary_count": ([], ctypes.c_int32),
+    "moe_trace_stage_name": ([ctypes.c_int32], ctypes.c_char_p),
+}
+
+
+def header_symbols() -> list[str]:
+    """Names of every function include/moe.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"^MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M)
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (fails loudly when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build the CUDA library first "
+                "(python -m mixture_experts_layer_55_b200.build or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIG.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().moe_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - library unavailable
+        return "unknown"
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+# ----------------------------------------------------------- marshalling --
+
+def _ptr(t):
+    """Device (or host) address of a tensor, or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        return torch.cuda.current_stream().cuda_stream
+    return None
+
+
+def _cfg(cfg: MoeConfig):
+    return ctypes.byref(cfg)
+
+
+def check_config(cfg: MoeConfig) -> int:
+    return int(lib().moe_check_config(_cfg(cfg)))
+
+
+def capacity(cfg: MoeConfig) -> int:
+    v = ctypes.c_int64()
+    _check(lib().moe_capacity(_cfg(cfg), ctypes.byref(v)), "moe_capacity")
+    return v.value
+
+
+def max_rows(cfg: MoeConfig) -> int:
+    v = ctypes.c_int64()
+    _check(lib().moe_max_rows(_cfg(cfg), ctypes.byref(v)), "moe_max_rows")
+    return v.value
+
+
+def workspace_size(cfg: MoeConfig) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().moe_workspace_size(_cfg(cfg), ctypes.byref(v)), "moe_workspace_size")
+    return v.value
+
+
+def forward_workspace_size(cfg: MoeConfig) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().moe_forward_workspace_size(_cfg(cfg), ctypes.byref(v)),
+           "moe_forward_workspace_size")
+    return v.value
+
+
+def moe_route(cfg, x, w_router, topk_ids, topk_w, workspace, router_bias=None, logit_noise=None,
+              logits_in=None, logits_out=None, probs_out=None, mean_prob=None, losses=None,
+              stream=None):
+    st = lib().moe_route(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
+                         _ptr(logit_noise), _ptr(logits_in), _ptr(logits_out), _ptr(probs_out),
+                         _ptr(topk_ids), _ptr(topk_w), _ptr(mean_prob), _ptr(losses),
+                         _ptr(workspace), _nbytes(workspace), _stream(stream))
+    _check(st, "moe_route")
+
+
+def moe_dispatch(cfg, x, topk_ids, counts, kept, offsets, perm, row_of, x_perm, workspace,
+                 stream=None):
+    st = lib().moe_dispatch(_cfg(cfg), _ptr(x), _ptr(topk_ids), _ptr(counts), _ptr(kept),
+                            _ptr(offsets), _ptr(perm), _ptr(row_of), _ptr(x_perm), _ptr(workspace),
+                            _nbytes(workspace), _stream(stream))
+    _check(st, "moe_dispatch")
+
+
+def moe_expert_ffn(cfg, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h, y_perm, workspace,
+                   stream=None):
+    st = lib().moe_expert_ffn(_cfg(cfg), _ptr(x_perm), _ptr(offsets), _ptr(perm), _ptr(topk_w),
+                              _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(h), _ptr(y_perm),
+                              _ptr(workspace), _nbytes(workspace), _stream(stream))
+    _check(st, "moe_expert_ffn")
+
+
+def moe_combine(cfg, y_perm, row_of, y, stream=None):
+    st = lib().moe_combine(_cfg(cfg), _ptr(y_perm), _ptr(row_of), _ptr(y), _stream(stream))
+    _check(st, "moe_combine")
+
+
+def moe_forward(cfg, x, w_router, w_gate, w_up, w_down, y, workspace, router_bias=None,
+                logit_noise=None, losses=None, mean_prob=None, counts=None, topk_ids=None,
+                topk_w=None, stream=None):
+    st = lib().moe_forward(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
+                           _ptr(logit_noise), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y),
+                           _ptr(losses), _ptr(mean_prob), _ptr(counts), _ptr(topk_ids),
+                           _ptr(topk_w), _ptr(workspace), _nbytes(workspace), _stream(stream))
+    _check(st, "moe_forward")
+
+
+def moe_get_device_status(workspace, stream=None) -> int:
+    """Flags word of a workspace (synchronises the stream); raises on a set flag."""
+    flags = ctypes.c_int32()
+    st = lib().moe_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(flags))
+    if st not in (MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS):
+        _check(st, "moe_get_device_status")
+    return flags.value
+
+
+def moe_clear_device_status(workspace, stream=None):
+    _check(lib().moe_clear_device_status(_ptr(workspace), _stream(stream)),
+           "moe_clear_device_status")
+
+
+def moe_trace_attach(events):
+    """Attach torch.cuda.Event objects (or raw cudaEvent_t ints); [] detaches."""
+    handles = [e if isinstance(e, int) else e.cuda_event for e in events]
+    arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
+    _check(lib().moe_trace_attach(arr if handles else None, len(handles)), "moe_trace_attach")
+
+
+def trace_stage_names() -> list[str]:
+    n = lib().moe_trace_boundary_count()
+    return [lib().moe_trace_stage_name(i).decode() for i in range(n)]
+
+
+def _nbytes(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        raise ValueError("pass the workspace as a tensor so its size is known")
+    return t.numel() * t.element_size()

@@ -1,0 +1,368 @@
+// api.cu -- the extern "C" boundary of libmoe_b200.so (declared in moe.h):
+// argument validation, workspace layout, and the launch sequence of each
+// entry point.  No allocation, no host synchronisation (except the device
+// status query).
+#include <math.h>
+#include <string.h>
+
+#include "internal.h"
+
+namespace moe {
+
+cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const void* x_perm,
+                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                                const void* w_gate, const void* w_up, const void* w_down, void* h,
+                                void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                                void* mid_ctx);
+cudaError_t launch_ffn_simt_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
+                                 const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                                 const void* w_gate, const void* w_up, const void* w_down, void* h,
+                                 void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                                 void* mid_ctx);
+
+int64_t capacity_of(const moe_config& c)
+{
+    const int64_t tk = c.T * (int64_t)c.K;
+    if (!(c.capacity_factor > 0.0f)) return tk;
+    double v = ceil((double)c.capacity_factor * (double)c.T * (double)c.K / (double)c.E);
+    if (v < 1.0) v = 1.0;
+    if (v > (double)tk) v = (double)tk;  // no expert can receive more than T*K
+    return (int64_t)v;
+}
+
+int64_t max_rows_of(const moe_config& c)
+{
+    const int64_t tk = c.T * (int64_t)c.K;
+    const int64_t cap = capacity_of(c) * (int64_t)c.E;
+    return cap < tk ? cap : tk;
+}
+
+WsLayout ws_layout(const moe_config& c)
+{
+    const RouterPlan rp = router_plan(c);
+    const int64_t nch = dispatch_chunks(c);
+    WsLayout L;
+    size_t o = 0;
+    L.status = o;
+    o += align_up(64 * sizeof(int));
+    L.r_part = o;
+    o += align_up((size_t)rp.splits * (size_t)c.T * c.E * sizeof(float));
+    L.r_mp = o;
+    o += align_up((size_t)rp.nb_topk * c.E * sizeof(float));
+    L.r_z = o;
+    o += align_up((size_t)rp.nb_topk * sizeof(float));
+    L.r_cnt = o;
+    o += align_up((size_t)rp.nb_topk * c.E * sizeof(int32_t));
+    L.d_cnt = o;
+    o += align_up((size_t)nch * c.E * sizeof(int32_t));
+    L.d_base = o;
+    o += align_up((size_t)nch * c.E * sizeof(int32_t));
+    L.total = o;
+    return L;
+}
+
+FwdLayout fwd_layout(const moe_config& c, int64_t max_rows)
+{
+    FwdLayout F;
+    F.ws = ws_layout(c);
+    const size_t es = c.dtype == MOE_BF16 ? 2 : 4;
+    const size_t tk = (size_t)c.T * c.K;
+    size_t o = F.ws.total;
+    F.ids = o;       o += align_up(tk * sizeof(int32_t));
+    F.w = o;         o += align_up(tk * sizeof(float));
+    F.counts = o;    o += align_up((size_t)c.E * sizeof(int32_t));
+    F.kept = o;      o += align_up((size_t)c.E * sizeof(int32_t));
+    F.offsets = o;   o += align_up((size_t)(c.E + 1) * sizeof(int32_t));
+    F.perm = o;      o += align_up((size_t)max_rows * sizeof(int32_t));
+    F.row_of = o;    o += align_up(tk * sizeof(int32_t));
+    F.mean_prob = o; o += align_up((size_t)c.E * sizeof(float));
+    F.losses = o;    o += align_up(2 * sizeof(float));
+    F.x_perm = o;    o += align_up((size_t)max_rows * c.D * es);
+    F.h = o;         o += align_up((size_t)max_rows * c.F * es);
+    F.y_perm = o;    o += align_up((size_t)max_rows * c.D * es);
+    F.total = o;
+    return F;
+}
+
+static moe_status check_config(const moe_config* c)
+{
+    if (c == nullptr) return MOE_ERR_ARG;
+    if (c->T < 1 || c->D < 1 || c->F < 1 || c->E < 1) return MOE_ERR_SHAPE;
+    if (c->E > 256) return MOE_ERR_ARG;
+    if (c->K < 1 || c->K > c->E || c->K > 8) return MOE_ERR_ARG;
+    if (c->T * (int64_t)c->K > (int64_t)INT32_MAX) return MOE_ERR_SHAPE;
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_ARG;
+    if (c->score_func != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+    if (c->renormalize != 1) return MOE_ERR_UNSUPPORTED;
+    if (c->D % 8 != 0 || c->F % 8 != 0) return MOE_ERR_ALIGN;
+    if (!isfinite(c->capacity_factor)) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ------------------------------------------------------------- tracing --
+static void* g_trace[16];
+static int g_trace_n = 0;
+static const char* kStageNames[7] = {"start", "route", "dispatch_index", "gather",
+                                     "expert_gate_up", "expert_down", "combine"};
+
+static void trace(int boundary, cudaStream_t s)
+{
+    if (boundary < g_trace_n && g_trace[boundary] != nullptr)
+        cudaEventRecord(static_cast<cudaEvent_t>(g_trace[boundary]), s);
+}
+
+static void trace_mid_ffn(void*, cudaStream_t s) { trace(4, s); }
+
+cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
+                              const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                              const void* w_gate, const void* w_up, const void* w_down, void* h,
+                              void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                              void* mid_ctx)
+{
+    if (c.dtype == MOE_F32)
+        return launch_ffn_simt_f32(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up,
+                                   w_down, h, y_perm, status, s, mid, mid_ctx);
+    return launch_ffn_simt_bf16(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down,
+                                h, y_perm, status, s, mid, mid_ctx);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int32_t st)
+{
+    switch (st) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_SHAPE: return "invalid shape";
+        case MOE_ERR_UNSUPPORTED: return "unsupported option";
+        case MOE_ERR_ALIGN: return "misaligned size or buffer";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_DEVICE_BOUNDS: return "device index out of range";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int32_t moe_version(void) { return 100; }
+
+moe_status moe_check_config(const moe_config* cfg) { return check_config(cfg); }
+
+moe_status moe_capacity(const moe_config* cfg, int64_t* capacity)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (capacity == nullptr) return MOE_ERR_ARG;
+    *capacity = capacity_of(*cfg);
+    return MOE_OK;
+}
+
+moe_status moe_max_rows(const moe_config* cfg, int64_t* rows)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (rows == nullptr) return MOE_ERR_ARG;
+    *rows = max_rows_of(*cfg);
+    return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_ARG;
+    *bytes = ws_layout(*cfg).total;
+    return MOE_OK;
+}
+
+moe_status moe_forward_workspace_size(const moe_config* cfg, size_t* bytes)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_ARG;
+    *bytes = fwd_layout(*cfg, max_rows_of(*cfg)).total;
+    return MOE_OK;
+}
+
+static moe_status check_ws(const moe_config* cfg, const void* ws, size_t bytes, size_t need)
+{
+    (void)cfg;
+    if (ws == nullptr || bytes < need) return MOE_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_ALIGN;
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router,
+                     const float* router_bias, const float* logit_noise, const float* logits_in,
+                     float* logits_out, float* probs_out, int32_t* topk_ids, float* topk_w,
+                     float* mean_prob, float* losses, void* workspace, size_t workspace_bytes,
+                     void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_ARG;
+    if (logits_in == nullptr && (x == nullptr || w_router == nullptr)) return MOE_ERR_ARG;
+    if (logits_in == nullptr && !aligned16(x)) return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(*cfg);
+    st = check_ws(cfg, workspace, workspace_bytes, L.total);
+    if (st != MOE_OK) return st;
+    const RouterPlan rp = router_plan(*cfg);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(launch_router(*cfg, rp, x, w_router, router_bias, logit_noise, logits_in,
+                                     logits_out, probs_out, topk_ids, topk_w, mean_prob, losses,
+                                     static_cast<char*>(workspace), L, s));
+}
+
+moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* topk_ids,
+                        int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* perm,
+                        int32_t* row_of, void* x_perm, void* workspace, size_t workspace_bytes,
+                        void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!topk_ids || !counts || !kept || !offsets || !perm || !row_of) return MOE_ERR_ARG;
+    if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_ARG;
+    if (x && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(*cfg);
+    st = check_ws(cfg, workspace, workspace_bytes, L.total);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    cudaError_t e = launch_dispatch_index(*cfg, capacity_of(*cfg), topk_ids, counts, kept, offsets,
+                                          perm, row_of, ws, L, s);
+    if (e == cudaSuccess && x)
+        e = launch_gather(*cfg, x, row_of, x_perm, max_rows_of(*cfg),
+                          reinterpret_cast<int*>(ws + L.status), s);
+    return cuda_status(e);
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                          const int32_t* perm, const float* topk_w, const void* w_gate,
+                          const void* w_up, const void* w_down, void* h, void* y_perm,
+                          void* workspace, size_t workspace_bytes, void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!x_perm || !offsets || !perm || !topk_w || !w_gate || !w_up || !w_down || !h || !y_perm)
+        return MOE_ERR_ARG;
+    if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+        !aligned16(h) || !aligned16(y_perm))
+        return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(*cfg);
+    st = check_ws(cfg, workspace, workspace_bytes, L.total);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + L.status);
+    return cuda_status(launch_expert_ffn(*cfg, max_rows_of(*cfg), x_perm, offsets, perm, topk_w,
+                                         w_gate, w_up, w_down, h, y_perm, status, s, nullptr,
+                                         nullptr));
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of, void* y,
+                       void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!y_perm || !row_of || !y) return MOE_ERR_ARG;
+    if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(launch_combine(*cfg, y_perm, row_of, y, max_rows_of(*cfg), s));
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
+                       const float* router_bias, const float* logit_noise, const void* w_gate,
+                       const void* w_up, const void* w_down, void* y, float* losses,
+                       float* mean_prob, int32_t* counts, int32_t* topk_ids, float* topk_w,
+                       void* workspace, size_t workspace_bytes, void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !y) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(w_gate) || !aligned16(w_up) ||
+        !aligned16(w_down))
+        return MOE_ERR_ALIGN;
+    const moe_config& c = *cfg;
+    const int64_t max_rows = max_rows_of(c);
+    const FwdLayout F = fwd_layout(c, max_rows);
+    st = check_ws(cfg, workspace, workspace_bytes, F.total);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    int* status = reinterpret_cast<int*>(ws + F.ws.status);
+    int32_t* ids = topk_ids ? topk_ids : reinterpret_cast<int32_t*>(ws + F.ids);
+    float* w = topk_w ? topk_w : reinterpret_cast<float*>(ws + F.w);
+    int32_t* cnt = counts ? counts : reinterpret_cast<int32_t*>(ws + F.counts);
+    int32_t* kept = reinterpret_cast<int32_t*>(ws + F.kept);
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + F.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + F.perm);
+    int32_t* row_of = reinterpret_cast<int32_t*>(ws + F.row_of);
+    void* x_perm = ws + F.x_perm;
+    void* h = ws + F.h;
+    void* y_perm = ws + F.y_perm;
+
+    trace(0, s);
+    const RouterPlan rp = router_plan(c);
+    cudaError_t e = launch_router(c, rp, x, w_router, router_bias, logit_noise, nullptr, nullptr,
+                                  nullptr, ids, w, mean_prob, losses, ws, F.ws, s);
+    trace(1, s);
+    if (e == cudaSuccess)
+        e = launch_dispatch_index(c, capacity_of(c), ids, cnt, kept, offsets, perm, row_of, ws,
+                                  F.ws, s);
+    trace(2, s);
+    if (e == cudaSuccess) e = launch_gather(c, x, row_of, x_perm, max_rows, status, s);
+    trace(3, s);
+    if (e == cudaSuccess)
+        e = launch_expert_ffn(c, max_rows, x_perm, offsets, perm, w, w_gate, w_up, w_down, h,
+                              y_perm, status, s, trace_mid_ffn, nullptr);
+    trace(5, s);
+    if (e == cudaSuccess) e = launch_combine(c, y_perm, row_of, y, max_rows, s);
+    trace(6, s);
+    return cuda_status(e);
+}
+
+moe_status moe_get_device_status(const void* workspace, void* stream, int32_t* flags)
+{
+    if (workspace == nullptr || flags == nullptr) return MOE_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t word[2] = {0, 0};
+    cudaError_t e = cudaMemcpyAsync(word, workspace, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    *flags = word[0];
+    if (word[0] & MOE_DEVFLAG_TIMEOUT) return MOE_ERR_DEVICE_TIMEOUT;
+    if (word[0] & MOE_DEVFLAG_BOUNDS) return MOE_ERR_DEVICE_BOUNDS;
+    return MOE_OK;
+}
+
+moe_status moe_clear_device_status(void* workspace, void* stream)
+{
+    if (workspace == nullptr) return MOE_ERR_ARG;
+    return cuda_status(
+        cudaMemsetAsync(workspace, 0, 64 * sizeof(int), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_trace_attach(void* const* events, int32_t n_events)
+{
+    if (n_events < 0 || n_events > 16 || (n_events > 0 && events == nullptr)) return MOE_ERR_ARG;
+    for (int i = 0; i < 16; ++i) g_trace[i] = i < n_events ? events[i] : nullptr;
+    g_trace_n = n_events;
+    return MOE_OK;
+}
+
+int32_t moe_trace_boundary_count(void) { return 7; }
+
+const char* moe_trace_stage_name(int32_t boundary)
+{
+    if (boundary < 0 || boundary >= 7) return "";
+    return kStageNames[boundary];
+}
+
+}  // extern "C"

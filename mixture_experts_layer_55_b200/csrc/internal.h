@@ -1,0 +1,87 @@
+// internal.h -- host-side plan and launch declarations shared by the C ABI
+// (api.cu) and the kernel files.  Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------ router plan --
+struct RouterPlan {
+    int be;          // experts per logits block (8, 16, 32 or 64)
+    int grid_t;      // token blocks of the logits GEMM (64 tokens each)
+    int grid_e;      // expert blocks
+    int splits;      // d_model splits of the logits GEMM
+    int d_per_split; // multiple of 32
+    int nb_topk;     // blocks of the softmax/top-k kernel (64 tokens each)
+};
+RouterPlan router_plan(const moe_config& c);
+
+// ---------------------------------------------------------- dispatch plan --
+constexpr int kDispatchChunk = 2048;  // assignments per dispatch block
+inline int64_t dispatch_chunks(const moe_config& c)
+{
+    return (c.T * c.K + kDispatchChunk - 1) / kDispatchChunk;
+}
+
+// ------------------------------------------------------ workspace layout --
+struct WsLayout {
+    size_t status;      // int32[64]
+    size_t r_part;      // splits * T * E fp32 partial logits
+    size_t r_mp;        // nb_topk * E fp32
+    size_t r_z;         // nb_topk fp32
+    size_t r_cnt;       // nb_topk * E int32
+    size_t d_cnt;       // chunks * E int32
+    size_t d_base;      // chunks * E int32
+    size_t total;
+};
+WsLayout ws_layout(const moe_config& c);
+
+struct FwdLayout {
+    WsLayout ws;        // scratch at offset 0
+    size_t ids, w, counts, kept, offsets, perm, row_of, mean_prob, losses;
+    size_t x_perm, h, y_perm;
+    size_t total;
+};
+FwdLayout fwd_layout(const moe_config& c, int64_t max_rows);
+
+int64_t capacity_of(const moe_config& c);
+int64_t max_rows_of(const moe_config& c);
+
+// ---------------------------------------------------------------- launches --
+// Each returns cudaSuccess or the launch error.
+cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void* x,
+                          const float* w_router, const float* bias, const float* noise,
+                          const float* logits_in, float* logits_out, float* probs_out,
+                          int32_t* ids, float* w, float* mean_prob, float* losses, char* ws,
+                          const WsLayout& L, cudaStream_t s);
+
+cudaError_t launch_dispatch_index(const moe_config& c, int64_t C, const int32_t* ids,
+                                  int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* perm,
+                                  int32_t* row_of, char* ws, const WsLayout& L, cudaStream_t s);
+
+cudaError_t launch_gather(const moe_config& c, const void* x, const int32_t* row_of, void* x_perm,
+                          int64_t max_rows, int* status, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
+                           void* y, int64_t max_rows, cudaStream_t s);
+
+// Expert FFN: gate/up (+SwiGLU) into h, then down (+routing weight) into y_perm.
+// The stage boundary between the two GEMMs is reported through `mid` (may be
+// null): it is called after the gate/up launch.
+typedef void (*StageHook)(void* ctx, cudaStream_t s);
+cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
+                              const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                              const void* w_gate, const void* w_up, const void* w_down, void* h,
+                              void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                              void* mid_ctx);
+
+}  // namespace moe

@@ -293,18 +293,17 @@ def forward(x, w_router, w_gate, w_up, w_down, K: int, capacity_factor: float = 
                 row_weight=row_weight, y=y)
 
 
-def token_outputs(x_rows, slot_ids, slot_weights, slot_kept, get_expert) -> np.ndarray:
-    """Direct per-token layer output for a few tokens ("Trace one token by hand").
+def slot_outputs(x_rows, slot_ids, slot_kept, get_expert) -> np.ndarray:
+    """Unweighted expert output of every kept (token, slot) of a few tokens.
 
-    x_rows (n, D) token activations; slot_ids / slot_weights / slot_kept (n, K).
-    get_expert(e) -> (w_gate_e, w_up_e, w_down_e) host arrays of one expert.
-    y[i] = sum over kept slots, in slot order, of w * expert(x_i).
-    Experts are visited one at a time so a caller can stream large weights.
+    x_rows (n, D); slot_ids / slot_kept (n, K); get_expert(e) -> (w_gate_e,
+    w_up_e, w_down_e) host arrays of one expert.  Returns (n, K, D), zero rows
+    for dropped slots.  Experts are visited one at a time so a caller can
+    stream large weights.
     """
     xr = _f64(x_rows)
     n, D = xr.shape
     ids = np.asarray(slot_ids)
-    ws = np.asarray(slot_weights, dtype=np.float64)
     kp = np.asarray(slot_kept, dtype=bool)
     K = ids.shape[1]
     outs = np.zeros((n, K, D), np.float64)
@@ -314,6 +313,20 @@ def token_outputs(x_rows, slot_ids, slot_weights, slot_kept, get_expert) -> np.n
         o = expert_rows(xr[[i for i, _ in sel]], wg, wu, wd)
         for j, (i, k) in enumerate(sel):
             outs[i, k] = o[j]
+    return outs
+
+
+def token_outputs(x_rows, slot_ids, slot_weights, slot_kept, get_expert, outs=None) -> np.ndarray:
+    """Direct per-token layer output for a few tokens ("Trace one token by hand").
+
+    y[i] = sum over kept slots, in slot order, of w * expert(x_i).  ``outs``
+    may pass precomputed slot_outputs.
+    """
+    ws = np.asarray(slot_weights, dtype=np.float64)
+    kp = np.asarray(slot_kept, dtype=bool)
+    if outs is None:
+        outs = slot_outputs(x_rows, slot_ids, kp, get_expert)
+    n, K, D = outs.shape
     y = np.zeros((n, D), np.float64)
     for i in range(n):
         for k in range(K):

@@ -1,0 +1,192 @@
+"""Helpers of the GPU parity tests: run the library through its C ABI on
+seeded inputs and compare with the CPU oracle.
+
+Tolerances (from the acceptance bar of the layer):
+  * routing ids, counts, kept, offsets, perm, row_of: bit-exact, the oracle
+    routed on the CUDA path's own fp32 logits;
+  * probabilities and combine weights: 1e-5 absolute;
+  * losses and mean probabilities: 1e-5 relative / absolute;
+  * bf16 outputs: |gpu - oracle| <= 1e-2 * max|oracle| + 1e-3 per element;
+  * fp32 outputs: |gpu - oracle| <= 1e-4 * max|oracle| per element.
+The fp32 logits themselves are checked against the fp64 logits with the
+classical bound for a length-n floating-point sum, gamma_n * sum|terms|.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_layer_55_b200 import _binding as B
+from workloads import Workload, make_inputs
+
+U32 = 2.0 ** -24
+
+
+def out_tol(wl: Workload, ref: np.ndarray) -> np.ndarray:
+    m = float(np.abs(ref).max()) if ref.size else 0.0
+    return 1e-4 * m if wl.dtype == "f32" else 1e-2 * m + 1e-3
+
+
+def assert_close_out(wl, got, ref, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    err = np.abs(got - ref)
+    tol = out_tol(wl, ref)
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements out of tolerance; "
+                           f"max err {err.max():.3e} > tol {tol:.3e}")
+    return float(err.max()), tol
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        t = t.double()
+    return t.numpy()
+
+
+class Bufs:
+    """Every buffer of the op-by-op path, allocated through torch."""
+
+    def __init__(self, wl: Workload, device="cuda"):
+        self.wl = wl
+        self.cfg = B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K, wl.dtype, wl.capacity_factor)
+        T, D, F, E, K = wl.T, wl.D, wl.F, wl.E, wl.K
+        dt = wl.torch_dtype
+        self.max_rows = B.max_rows(self.cfg)
+        R = self.max_rows
+        i32, f32 = torch.int32, torch.float32
+        self.ws = torch.zeros(B.workspace_size(self.cfg), dtype=torch.uint8, device=device)
+        self.logits = torch.empty(T, E, dtype=f32, device=device)
+        self.probs = torch.empty(T, E, dtype=f32, device=device)
+        self.ids = torch.empty(T, K, dtype=i32, device=device)
+        self.w = torch.empty(T, K, dtype=f32, device=device)
+        self.mean_prob = torch.empty(E, dtype=f32, device=device)
+        self.losses = torch.empty(2, dtype=f32, device=device)
+        self.counts = torch.empty(E, dtype=i32, device=device)
+        self.kept = torch.empty(E, dtype=i32, device=device)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=device)
+        self.perm = torch.full((R,), -7, dtype=i32, device=device)
+        self.row_of = torch.empty(T * K, dtype=i32, device=device)
+        self.x_perm = torch.empty(R, D, dtype=dt, device=device)
+        self.h = torch.empty(R, F, dtype=dt, device=device)
+        self.y_perm = torch.empty(R, D, dtype=dt, device=device)
+        self.y = torch.empty(T, D, dtype=dt, device=device)
+
+    def run_ops(self, inp, logits_in=None):
+        c = self.cfg
+        B.moe_route(c, inp["x"], inp["w_router"], self.ids, self.w, self.ws,
+                    router_bias=inp["bias"], logit_noise=inp["noise"], logits_in=logits_in,
+                    logits_out=self.logits if logits_in is None else None, probs_out=self.probs,
+                    mean_prob=self.mean_prob, losses=self.losses)
+        if logits_in is not None:
+            self.logits.copy_(logits_in)
+        B.moe_dispatch(c, inp["x"], self.ids, self.counts, self.kept, self.offsets, self.perm,
+                       self.row_of, self.x_perm, self.ws)
+        B.moe_expert_ffn(c, self.x_perm, self.offsets, self.perm, self.w, inp["w_gate"],
+                         inp["w_up"], inp["w_down"], self.h, self.y_perm, self.ws)
+        B.moe_combine(c, self.y_perm, self.row_of, self.y)
+        torch.cuda.synchronize()
+        flags = B.moe_get_device_status(self.ws)
+        assert flags == 0, f"device status flags {flags:#x}"
+
+
+def check_logits(wl, inp_cpu, logits_gpu):
+    """fp32 logits against the fp64 ones, within gamma_n * sum|terms|."""
+    L64 = oracle.router_logits(inp_cpu["x"], inp_cpu["w_router"], inp_cpu["bias"],
+                               inp_cpu["noise"])
+    ax = inp_cpu["x"].double().abs()
+    aw = inp_cpu["w_router"].double().abs()
+    mag = (ax @ aw).numpy()
+    if inp_cpu["bias"] is not None:
+        mag = mag + inp_cpu["bias"].double().abs().numpy()[None, :]
+    if inp_cpu["noise"] is not None:
+        mag = mag + inp_cpu["noise"].double().abs().numpy()
+    n = wl.D + 4
+    gamma = n * U32 / (1 - n * U32)
+    err = np.abs(logits_gpu.astype(np.float64) - L64)
+    assert (err <= gamma * mag + 1e-30).all(), f"logit error {err.max():.3e} beyond the fp32 bound"
+    return float((err / np.maximum(mag, 1e-30)).max())
+
+
+def check_routing(wl, b: Bufs):
+    """Everything the router and the dispatch index pass produce."""
+    L = b.logits.cpu().numpy()
+    ids, w, probs, lse = oracle.route(L, wl.K)
+    counts64, mp, z, bal = oracle.router_stats(ids, probs, lse, wl.E)
+    np.testing.assert_array_equal(b.ids.cpu().numpy(), ids)
+    np.testing.assert_allclose(b.w.cpu().numpy(), w, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(b.probs.cpu().numpy(), probs, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(b.mean_prob.cpu().numpy(), mp, rtol=0, atol=1e-5)
+    lg = b.losses.cpu().numpy().astype(np.float64)
+    assert abs(lg[0] - z) <= 1e-5 * abs(z) + 1e-7, (lg[0], z)
+    assert abs(lg[1] - bal) <= 1e-5 * abs(bal) + 1e-7, (lg[1], bal)
+    C = oracle.capacity(wl.T, wl.K, wl.E, wl.capacity_factor)
+    assert C == B.capacity(b.cfg)
+    d = oracle.dispatch(ids, wl.E, C)
+    np.testing.assert_array_equal(b.counts.cpu().numpy(), d["counts"])
+    assert int(counts64.sum()) == wl.T * wl.K
+    np.testing.assert_array_equal(b.kept.cpu().numpy(), d["kept"])
+    np.testing.assert_array_equal(b.offsets.cpu().numpy(), d["offsets"])
+    R = int(d["offsets"][-1])
+    np.testing.assert_array_equal(b.perm[:R].cpu().numpy(), d["perm"])
+    np.testing.assert_array_equal(b.row_of.cpu().numpy(), d["row_of"])
+    return dict(ids=ids, w=w, probs=probs, lse=lse, z=z, bal=bal, C=C, **d)
+
+
+def expert_getter(inp):
+    """Host copies of one expert's weights (fetched one expert at a time)."""
+    def get(e):
+        return (inp["w_gate"][e].cpu(), inp["w_up"][e].cpu(), inp["w_down"][e].cpu())
+    return get
+
+
+def sample_tokens(wl, rt, n_random=16, seed=0):
+    """Token sample: first, last, random, hottest/coldest experts' tokens, and
+    any token with a dropped slot."""
+    rng = np.random.default_rng(seed)
+    T, K = wl.T, wl.K
+    toks = {0, T - 1}
+    toks.update(int(t) for t in rng.choice(T, size=min(n_random, T), replace=False))
+    ids = rt["ids"]
+    counts = rt["counts"]
+    nz = np.nonzero(counts)[0]
+    for e in (int(np.argmax(counts)), int(nz[np.argmin(counts[nz])])):
+        tt = np.nonzero((ids == e).any(1))[0]
+        toks.update(int(t) for t in tt[:2])
+        toks.update(int(t) for t in tt[-1:])
+    dropped = np.nonzero((rt["row_of"].reshape(T, K) < 0).any(1))[0]
+    toks.update(int(t) for t in dropped[:3])
+    toks.update(int(t) for t in dropped[-2:])
+    return sorted(toks)
+
+
+def check_tokens(wl, inp, rt, tokens, y_gpu, y_perm=None, x_perm=None):
+    """Sampled tokens: the direct per-token computation against y, and (when
+    given) each kept slot's y_perm row against w * expert(x) and its x_perm
+    row against the token row (an exact copy)."""
+    T, K = wl.T, wl.K
+    row_of = rt["row_of"].reshape(T, K)
+    kept = row_of >= 0
+    x_rows = inp["x"][tokens].cpu()
+    outs = oracle.slot_outputs(x_rows, rt["ids"][tokens], kept[tokens], expert_getter(inp))
+    ref = oracle.token_outputs(x_rows, rt["ids"][tokens], rt["w"][tokens], kept[tokens], None,
+                               outs=outs)
+    err, tol = assert_close_out(wl, to_np(y_gpu[tokens]), ref, "y (sampled tokens)")
+    if y_perm is not None:
+        rows, refs = [], []
+        for i, t in enumerate(tokens):
+            for k in range(K):
+                r = int(row_of[t, k])
+                if r >= 0:
+                    rows.append(r)
+                    refs.append(rt["w"][t, k] * outs[i, k])
+        if rows:
+            assert_close_out(wl, to_np(y_perm[rows]), np.stack(refs), "y_perm (sampled rows)")
+    if x_perm is not None:
+        for t in tokens:
+            for k in range(K):
+                r = int(row_of[t, k])
+                if r >= 0:
+                    assert torch.equal(x_perm[r].cpu(), inp["x"][t].cpu()), f"x_perm[{r}] != x[{t}]"
+    return err, tol

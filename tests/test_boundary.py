@@ -1,0 +1,127 @@
+"""The C ABI library loads, exports every symbol include/moe.h declares, and
+rejects bad arguments on the host before any device work (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from mixture_experts_layer_55_b200 import build as build_mod
+from mixture_experts_layer_55_b200 import _binding as B
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = B.header_symbols()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moe.h but not exported"
+    assert set(B._SIG) == set(names), "binding signatures out of sync with moe.h"
+    assert lib.moe_version() == 100
+
+
+def _cfg(**kw):
+    base = dict(T=64, D=128, F=256, E=8, K=2, dtype="bf16", capacity_factor=0.0)
+    base.update(kw)
+    return B.MoeConfig.make(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(), B.MOE_OK),
+    (dict(K=0), B.MOE_ERR_ARG),
+    (dict(K=9, E=16), B.MOE_ERR_ARG),       # register top-k bound
+    (dict(K=5, E=4), B.MOE_ERR_ARG),        # K > E
+    (dict(E=257, K=2), B.MOE_ERR_ARG),
+    (dict(T=0), B.MOE_ERR_SHAPE),
+    (dict(D=0), B.MOE_ERR_SHAPE),
+    (dict(F=-8), B.MOE_ERR_SHAPE),
+    (dict(D=100), B.MOE_ERR_ALIGN),         # 16-byte rows
+    (dict(F=12), B.MOE_ERR_ALIGN),
+    (dict(T=2**31, K=2), B.MOE_ERR_SHAPE),  # T*K beyond int32
+    (dict(score_func=1), B.MOE_ERR_UNSUPPORTED),
+    (dict(renormalize=0), B.MOE_ERR_UNSUPPORTED),
+    (dict(capacity_factor=float("nan")), B.MOE_ERR_ARG),
+])
+def test_check_config(lib, kw, code):
+    assert B.check_config(_cfg(**kw)) == code
+
+
+def test_capacity_and_rows(lib):
+    c = _cfg(T=32768, D=1024, F=4096, E=32, K=2, capacity_factor=1.25)
+    assert B.capacity(c) == 2560
+    assert B.max_rows(c) == min(32768 * 2, 2560 * 32)
+    c = _cfg(T=4096, E=16, K=2, capacity_factor=1.5)
+    assert B.capacity(c) == 768
+    c = _cfg(T=100, E=8, K=2)  # dropless
+    assert B.capacity(c) == 200 and B.max_rows(c) == 200
+    c = _cfg(T=3, E=8, K=1, capacity_factor=0.5)
+    assert B.capacity(c) == 1 and B.max_rows(c) == 3
+    c = _cfg(T=10, E=2, K=1, capacity_factor=100.0)  # never above T*K
+    assert B.capacity(c) == 10
+
+
+def test_workspace_sizes_grow_with_problem(lib):
+    small = B.workspace_size(_cfg(T=64))
+    big = B.workspace_size(_cfg(T=65536))
+    assert 0 < small < big
+    fwd = B.forward_workspace_size(_cfg(T=64))
+    assert fwd > small
+
+
+FAKE = 0x10000  # an aligned address the library never dereferences here
+
+
+def _call_route(lib, cfg, x=FAKE, w=FAKE, ids=FAKE, tw=FAKE, ws=FAKE, nbytes=None):
+    nb = B.workspace_size(cfg) if nbytes is None else nbytes
+    return lib.moe_route(ctypes.byref(cfg), x, w, None, None, None, None, None, ids, tw, None,
+                         None, ws, nb, None)
+
+
+def test_route_argument_errors(lib):
+    c = _cfg()
+    assert _call_route(lib, c, ids=None) == B.MOE_ERR_ARG
+    assert _call_route(lib, c, tw=None) == B.MOE_ERR_ARG
+    assert _call_route(lib, c, x=None) == B.MOE_ERR_ARG
+    assert _call_route(lib, c, x=FAKE + 8) == B.MOE_ERR_ALIGN
+    assert _call_route(lib, c, ws=None) == B.MOE_ERR_WORKSPACE
+    assert _call_route(lib, c, nbytes=16) == B.MOE_ERR_WORKSPACE
+    assert _call_route(lib, c, ws=FAKE + 16) == B.MOE_ERR_ALIGN  # workspace wants 256 B
+    bad = _cfg(K=9, E=8)
+    assert _call_route(lib, bad, nbytes=1 << 20) == B.MOE_ERR_ARG
+
+
+def test_dispatch_ffn_combine_forward_argument_errors(lib):
+    c = _cfg()
+    nb = B.workspace_size(c)
+    cr = ctypes.byref(c)
+    # x and x_perm must be both given or both NULL
+    assert lib.moe_dispatch(cr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, nb,
+                            None) == B.MOE_ERR_ARG
+    assert lib.moe_dispatch(cr, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, nb,
+                            None) == B.MOE_ERR_ARG
+    assert lib.moe_dispatch(cr, FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nb,
+                            None) == B.MOE_ERR_ALIGN
+    assert lib.moe_expert_ffn(cr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, nb,
+                              None) == B.MOE_ERR_ARG
+    assert lib.moe_expert_ffn(cr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE,
+                              nb, None) == B.MOE_ERR_ALIGN
+    assert lib.moe_combine(cr, FAKE, None, FAKE, None) == B.MOE_ERR_ARG
+    assert lib.moe_combine(cr, FAKE, FAKE, FAKE + 8, None) == B.MOE_ERR_ALIGN
+    fb = B.forward_workspace_size(c)
+    assert lib.moe_forward(cr, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, None, None, None,
+                           None, None, FAKE, fb - 1, None) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(cr, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, None, None, None,
+                           None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+
+
+def test_status_strings_and_trace_table(lib):
+    assert B.status_string(0) == "ok"
+    assert "workspace" in B.status_string(B.MOE_ERR_WORKSPACE)
+    names = B.trace_stage_names()
+    assert names[0] == "start" and names[-1] == "combine" and len(names) == 7
+    assert lib.moe_trace_attach(None, 0) == B.MOE_OK
+    assert lib.moe_trace_attach(None, 3) == B.MOE_ERR_ARG
+    assert lib.moe_trace_attach(None, 17) == B.MOE_ERR_ARG

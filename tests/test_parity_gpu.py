@@ -1,0 +1,162 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Small cases compare every output element by element; they span several
+tiles and ragged tails.  The five full-size layer shapes compare the routing
+and dispatch results in full and the layer output on a token sample (tokens
+of the hottest and coldest experts and tokens with dropped slots included),
+through moe_forward, the call the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_55_b200 import _binding as B
+from tests.gpu_common import (Bufs, assert_close_out, check_logits, check_routing, check_tokens,
+                              sample_tokens, to_np)
+from workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(name, **kw):
+    base = dict(T=300, D=136, F=200, E=8, K=2, dtype="bf16", seed=1)
+    base.update(kw)
+    return Workload(name, **base)
+
+
+SMALL = [
+    _wl("ragged_bf16"),
+    _wl("ragged_f32", dtype="f32"),
+    _wl("tiles_bf16", T=700, D=264, F=392, E=6, K=3, seed=2),  # several 128-row tiles, K/N tails
+    _wl("fine_bias", T=512, D=128, F=72, E=64, K=6, bias="zipf", seed=3),
+    _wl("capacity_drops", T=400, D=64, F=96, E=8, K=2, capacity_factor=0.5, noise=True, seed=4),
+    _wl("capacity_f32", T=257, D=64, F=64, E=4, K=2, capacity_factor=0.3, dtype="f32", seed=5),
+    _wl("k_equals_e", T=96, D=64, F=64, E=4, K=4, seed=6),
+    _wl("e256_k8", T=40, D=256, F=128, E=256, K=8, seed=7),
+    _wl("one_token", T=1, D=64, F=64, E=8, K=2, seed=8),
+    _wl("top1", T=130, D=72, F=80, E=5, K=1, seed=9),
+    _wl("one_expert", T=33, D=32, F=48, E=1, K=1, seed=10),
+]
+
+
+def _to_dev(inp):
+    return {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
+def test_small_layers_elementwise(cuda_ok, wl):
+    inp_cpu = make_inputs(wl, device="cpu")
+    inp = _to_dev(inp_cpu)
+    b = Bufs(wl)
+    b.run_ops(inp)
+    check_logits(wl, inp_cpu, b.logits.cpu().numpy())
+    rt = check_routing(wl, b)
+    ref = oracle.forward(inp_cpu["x"], inp_cpu["w_router"], inp_cpu["w_gate"], inp_cpu["w_up"],
+                         inp_cpu["w_down"], wl.K, wl.capacity_factor, inp_cpu["bias"],
+                         inp_cpu["noise"], logits=b.logits.cpu().numpy())
+    R = int(ref["offsets"][-1])
+    # dispatch gather: exact copies
+    assert torch.equal(b.x_perm[:R].cpu().to(torch.float64),
+                       torch.from_numpy(ref["x_perm"])), "x_perm differs"
+    # expert outputs with the routing weight applied
+    assert_close_out(wl, to_np(b.y_perm[:R]), ref["o"] * ref["row_weight"][:, None], "y_perm")
+    assert_close_out(wl, to_np(b.y), ref["y"], "y")
+    # dropped-everything tokens are exactly zero
+    kept = ref["row_of"].reshape(wl.T, wl.K) >= 0
+    none = np.nonzero(~kept.any(1))[0]
+    if none.size:
+        assert (to_np(b.y[none]) == 0).all()
+    # the whole layer in one call gives the same bits as the op-by-op path
+    ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
+    y2 = torch.empty_like(b.y)
+    losses = torch.empty(2, device="cuda")
+    counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y2,
+                  ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses,
+                  counts=counts)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, b.y)
+    assert torch.equal(losses, b.losses)
+    assert torch.equal(counts, b.counts)
+    assert B.moe_get_device_status(ws) == 0
+
+
+def test_parity_mode_routes_given_logits(cuda_ok):
+    """logits_in: the router kernel routes exactly the logits it is given,
+    ties included (tie rule: lower expert id)."""
+    wl = _wl("given_logits", T=200, E=16, K=4, seed=11)
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    g = torch.Generator().manual_seed(3)
+    L = torch.round(torch.randn(wl.T, wl.E, generator=g) * 2) / 2  # many exact ties
+    L[:5] = 0.0  # all-equal rows
+    b = Bufs(wl)
+    b.run_ops(inp, logits_in=L.cuda())
+    rt = check_routing(wl, b)
+    assert (rt["ids"][:5] == np.arange(4)[None, :]).all()
+
+
+def test_determinism_bitwise(cuda_ok):
+    wl = _wl("det", T=1000, D=128, F=128, E=16, K=4, bias="zipf", seed=12)
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    outs = []
+    for _ in range(2):
+        b = Bufs(wl)
+        b.run_ops(inp)
+        outs.append((b.y.clone(), b.losses.clone(), b.mean_prob.clone(), b.perm.clone()))
+    for a, c in zip(*outs):
+        assert torch.equal(a, c)
+
+
+def test_out_of_range_ids_raise_bounds_flag(cuda_ok):
+    """Corrupt ids are caught by the dispatch kernels' own bounds checks: the
+    status word gets the bounds flag and nothing is written out of range."""
+    wl = _wl("bad_ids", T=64, E=8, K=2)
+    b = Bufs(wl)
+    ids = torch.randint(0, 8, (wl.T, wl.K), dtype=torch.int32)
+    ids[5, 1] = 11
+    ids[9, 0] = -3
+    b.ids.copy_(ids)
+    B.moe_dispatch(b.cfg, None, b.ids, b.counts, b.kept, b.offsets, b.perm, b.row_of, None, b.ws)
+    flags = B.moe_get_device_status(b.ws)
+    assert flags & 0x2
+    row_of = b.row_of.cpu().numpy().reshape(wl.T, wl.K)
+    assert row_of[5, 1] == -1 and row_of[9, 0] == -1
+    assert int(b.counts.sum()) == wl.T * wl.K - 2
+    B.moe_clear_device_status(b.ws)
+    assert B.moe_get_device_status(b.ws) == 0
+
+
+# ------------------------------------------------------------- full sizes --
+
+FULL = ["tiny_fp32", "mixtral_8x", "fine_skewed", "stmoe_capacity", "decode_e256"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_layer(cuda_ok, name):
+    wl = WORKLOADS[name]
+    torch.manual_seed(0)
+    inp = make_inputs(wl, device="cuda")
+    b = Bufs(wl)
+    b.run_ops(inp)
+    rt = check_routing(wl, b)
+    # the benchmark's call: the whole layer through moe_forward
+    ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(b.y)
+    losses = torch.empty(2, device="cuda")
+    B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y,
+                  ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses)
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status(ws) == 0
+    assert torch.equal(y, b.y), "moe_forward differs from the op-by-op path"
+    if wl.T <= 512:
+        tokens = list(range(wl.T)) if wl.name == "tiny_fp32" else sample_tokens(wl, rt, 6)
+    else:
+        tokens = sample_tokens(wl, rt, 12)
+    if wl.name == "decode_e256":
+        tokens = tokens[:6]
+    check_tokens(wl, inp, rt, tokens, y, y_perm=b.y_perm, x_perm=b.x_perm)
+    if wl.capacity_factor > 0:
+        assert rt["C"] == 2560
+    del inp
+    torch.cuda.empty_cache()
