@@ -227,8 +227,15 @@ def moe_clear_device_status(workspace, stream=None):
 
 
 def moe_trace_attach(events):
-    """Attach torch.cuda.Event objects (or raw cudaEvent_t ints); [] detaches."""
-    handles = [e if isinstance(e, int) else e.cuda_event for e in events]
+    """Attach torch.cuda.Event objects (or raw cudaEvent_t ints); [] detaches.
+
+    torch creates an event's CUDA handle lazily, at its first record; events
+    without a handle are recorded once here so that one exists."""
+    handles = []
+    for e in events:
+        if not isinstance(e, int) and not e.cuda_event:
+            e.record()
+        handles.append(e if isinstance(e, int) else e.cuda_event)
     arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
     _check(lib().moe_trace_attach(arr if handles else None, len(handles)), "moe_trace_attach")
 

@@ -14,11 +14,11 @@ cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const voi
                                 const void* w_gate, const void* w_up, const void* w_down, void* h,
                                 void* y_perm, int* status, cudaStream_t s, StageHook mid,
                                 void* mid_ctx);
-cudaError_t launch_ffn_simt_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
-                                 const int32_t* offsets, const int32_t* perm, const float* topk_w,
-                                 const void* w_gate, const void* w_up, const void* w_down, void* h,
-                                 void* y_perm, int* status, cudaStream_t s, StageHook mid,
-                                 void* mid_ctx);
+cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
+                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                               const void* w_gate, const void* w_up, const void* w_down, void* h,
+                               void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                               void* mid_ctx);
 
 int64_t capacity_of(const moe_config& c)
 {
@@ -126,8 +126,8 @@ cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void*
     if (c.dtype == MOE_F32)
         return launch_ffn_simt_f32(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up,
                                    w_down, h, y_perm, status, s, mid, mid_ctx);
-    return launch_ffn_simt_bf16(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down,
-                                h, y_perm, status, s, mid, mid_ctx);
+    return launch_ffn_tc_bf16(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h,
+                              y_perm, status, s, mid, mid_ctx);
 }
 
 }  // namespace moe

@@ -1,0 +1,441 @@
+// ffn_tc.cu -- grouped SwiGLU expert FFN on the 5th-generation tensor cores
+// (tcgen05 MMA, accumulators in tensor memory, operands staged by TMA).
+//
+// "Lab: build a tiny MoE in PyTorch", section "Full implementation":
+// SwiGLUExpert computes down(silu(gate x) * up x) with no biases, and each
+// expert output is scaled by its combine weight before the scatter-add.  The
+// experts' rows are contiguous blocks of x_perm (expert-major), so each
+// expert is one dense GEMM over its block; both contractions run here:
+//
+//   gate/up:  [G | U] = x_perm[block] . [Wg_e | Wu_e]   (K = D, two fp32 accumulators)
+//             h = bf16(silu(G) * U)                     (epilogue)
+//   down:     Y = h[block] . Wd_e                       (K = F)
+//             y_perm = bf16(topk_w[perm[row]] * Y)      (epilogue)
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0      TMA producer: A tile 128 x 64 (K-major, 128-byte swizzle) and
+//               B tiles 64 x 64 (N-major, 128-byte swizzle) into a 4-stage ring
+//   warp 1      MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M = 128,
+//               N = 128 (x2 for gate/up) or 256 (down), K = 16 per instruction;
+//               it also owns the 512-column tensor-memory allocation
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (lane = row), the
+//               SwiGLU or routing-weight step, bf16 stores to global memory
+// Accumulators are double-buffered in tensor memory (2 x 256 columns), so the
+// epilogue of one tile overlaps the MMAs of the next.  Tiles are ordered
+// (expert, n-tile, m-tile) with m fastest: concurrently running CTAs share an
+// expert's weight tile through L2.  The tile -> (expert, rows) map is built
+// on the device from the dispatch offsets; rows past an expert's block are
+// computed but never stored.  Every wait is bounded (device status flag).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;               // rows per tile (UMMA M)
+constexpr int BK = 64;                // K per stage: one 128-byte swizzle row of bf16
+constexpr int UK = 16;                // K per tcgen05.mma (bf16)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BK * 256 * 2; // 32 KB: [gate 128 | up 128] or down 256 columns
+constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64 x 64 B box
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = 256;         // tensor-memory columns per accumulator buffer
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 192;
+constexpr int MAX_E = 256;
+
+struct Misc {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int row0[MAX_E];
+    int rowend[MAX_E];
+    int pref[MAX_E + 1];  // first tile index of each expert; pref[E] = total tiles
+};
+
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Misc);
+
+struct Args {
+    const int32_t* offsets;
+    const int32_t* perm;
+    const float* topk_w;
+    __nv_bfloat16* out;  // h (gate/up) or y_perm (down), row-major (max_rows, N)
+    int E;
+    int Kdim;            // D for gate/up, F for down
+    int N;               // F for gate/up, D for down
+    int n_tiles;         // ceil(N / BN)
+    int64_t max_rows;
+    int64_t nk;          // T * K (range of perm values)
+    int* status;
+};
+
+template <bool GATEUP> struct Cfg {
+    static constexpr int BN = GATEUP ? 128 : 256;  // output columns per tile
+};
+
+MOE_DEVICE void decode_tile(const Misc* m, int E, int n_tiles, int bn, int t, int& e, int& m_row0,
+                            int& row_end, int& n0)
+{
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {  // largest e with pref[e] <= t (its block is non-empty)
+        const int mid = (lo + hi + 1) >> 1;
+        if (m->pref[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    e = lo;
+    const int mt = (m->rowend[e] - m->row0[e] + BM - 1) / BM;
+    const int local = t - m->pref[e];
+    const int n = local / mt, mm = local - n * mt;
+    m_row0 = m->row0[e] + mm * BM;
+    row_end = m->rowend[e];
+    n0 = n * bn;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                  const __grid_constant__ CUtensorMap tmB1, const Args a)
+{
+    constexpr int BN = Cfg<GATEUP>::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&m->tfull[b], 1);
+            mbar_init(&m->tempty[b], 128);
+        }
+        mbar_init(&m->drain, 1);
+        m->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB0);
+        if (GATEUP) prefetch_tmap(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(&m->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    // tile table from the offsets (validated: a malformed block is treated as empty)
+    for (int e = threadIdx.x; e < E; e += NUM_THREADS) {
+        m->row0[e] = a.offsets[e];
+        m->rowend[e] = a.offsets[e + 1];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0, prev = 0;
+        for (int e = 0; e < E; ++e) {
+            int r0 = m->row0[e], r1 = m->rowend[e];
+            if (r0 < prev || r1 < r0 || (int64_t)r1 > a.max_rows) {
+                raise_flag(a.status, kFlagBounds, 400);
+                r0 = r1 = prev;
+            }
+            m->row0[e] = r0;
+            m->rowend[e] = r1;
+            prev = r1;
+            m->pref[e] = run;
+            run += (r1 - r0 + BM - 1) / BM * a.n_tiles;
+        }
+        m->pref[E] = run;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = m->tmem_base;
+    const int total = m->pref[E];
+    const int num_kb = (a.Kdim + BK - 1) / BK;
+    volatile int* abort_flag = &m->abort_flag;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int last_phase[STAGES];
+        for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int e, m_row0, row_end, n0;
+            decode_tile(m, E, a.n_tiles, BN, t, e, m_row0, row_end, n0);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 410, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
+                uint8_t* sB = sA + A_BYTES;
+                uint64_t* fb = &m->full[stage];
+                mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                const int k0 = kb * BK;
+                tma_load_2d(sA, &tmA, k0, m_row0, fb);
+                if (GATEUP) {
+                    tma_load_3d(sB, &tmB0, n0, k0, e, fb);
+                    tma_load_3d(sB + BOX_BYTES, &tmB0, n0 + 64, k0, e, fb);
+                    tma_load_3d(sB + 2 * BOX_BYTES, &tmB1, n0, k0, e, fb);
+                    tma_load_3d(sB + 3 * BOX_BYTES, &tmB1, n0 + 64, k0, e, fb);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tma_load_3d(sB + j * BOX_BYTES, &tmB0, n0 + 64 * j, k0, e, fb);
+                }
+                last_phase[stage] = (int)phase;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // never leave the CTA with a copy in flight
+        for (int s = 0; s < STAGES; ++s)
+            if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 411, nullptr);
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = GATEUP ? umma_idesc_bf16(BM, 128, 0, 1) : umma_idesc_bf16(BM, 256, 0, 1);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            if (!mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 420, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + (uint32_t)(acc * ACC_COLS);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(&m->full[stage], phase, a.status, 421, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sA = smem_u32(stages + (size_t)stage * STAGE_BYTES);
+                const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / UK; ++kk) {
+                    const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+                    // A: K-major, 8-row groups 1024 B apart; +32 B per 16-element K step
+                    const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
+                    // B: N-major, 64-column blocks 8 KB apart (LBO), 8-row K groups
+                    // 1024 B apart (SBO); +2048 B per 16-row K step
+                    if (GATEUP) {
+                        const uint64_t bg = umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
+                        const uint64_t bu = umma_desc_sw128(sB + 2 * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
+                        umma_f16_ss(d0, adesc, bg, idesc, accum);
+                        umma_f16_ss(d0 + 128, adesc, bu, idesc, accum);
+                    } else {
+                        const uint64_t bd = umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
+                        umma_f16_ss(d0, adesc, bd, idesc, accum);
+                    }
+                }
+                umma_commit(&m->empty[stage]);  // frees the stage once these MMAs complete
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            umma_commit(&m->tfull[acc]);  // accumulator ready for the epilogue
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        // wait for every MMA issued here before the allocation is released
+        umma_commit(&m->drain);
+        mbar_wait(&m->drain, 0, a.status, 422, nullptr);
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue
+        const int quad = warp & 3;  // tensor-memory lanes this warp may read
+        const int r_in_tile = quad * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            int e, m_row0, row_end, n0;
+            decode_tile(m, E, a.n_tiles, BN, t, e, m_row0, row_end, n0);
+            if (!mbar_wait(&m->tfull[acc], acc_phase, a.status, 430, abort_flag)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)m_row0 + r_in_tile;
+            const bool valid = row < row_end;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            __nv_bfloat16* orow = a.out + row * (int64_t)a.N;
+            if (GATEUP) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, g);
+                    tmem_ld_32x32b_x32(taddr + 128 + c * 32, u);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint32_t p[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float h0 = silu_f32(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
+                            const float h1 =
+                                silu_f32(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
+                            p[j] = pack_bf16x2(h0, h1);
+                        }
+                        const int col = n0 + c * 32;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (col + 8 * q < a.N)
+                                *reinterpret_cast<uint4*>(orow + col + 8 * q) =
+                                    make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                    }
+                }
+            } else {
+                float w = 0.f;
+                if (valid) {
+                    const int32_t pa = a.perm[row];
+                    if (pa >= 0 && (int64_t)pa < a.nk) w = a.topk_w[pa];
+                    else raise_flag(a.status, kFlagBounds, 431);
+                }
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint32_t p[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            p[j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
+                        const int col = n0 + c * 32;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (col + 8 * q < a.N)
+                                *reinterpret_cast<uint4*>(orow + col + 8 * q) =
+                                    make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&m->tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------- host --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encoder()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 map over a row-major (rows, cols) matrix; box = 64 columns x box_rows rows.
+static bool map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over (E, rows, cols) row-major weights; box = 64 cols x 64 rows x 1.
+static bool map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cols, rows, E};
+    cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GATEUP>
+static cudaError_t prepare()
+{
+    static int done_dev_mask = 0;  // devices 0..30 on which the attribute was set
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 31 && (done_dev_mask >> dev) & 1) return cudaSuccess;
+    e = cudaFuncSetAttribute(ffn_tc_kernel<GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES);
+    if (e == cudaSuccess && dev < 31) done_dev_mask |= 1 << dev;
+    return e;
+}
+
+}  // namespace tc
+
+cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
+                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                               const void* w_gate, const void* w_up, const void* w_down, void* h,
+                               void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                               void* mid_ctx)
+{
+    using namespace tc;
+    cudaError_t err = prepare<true>();
+    if (err == cudaSuccess) err = prepare<false>();
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t mtiles_bound = (max_rows + BM - 1) / BM + c.E;
+
+    CUtensorMap mA, mG, mU, mH, mD;
+    if (!map_2d(&mA, x_perm, (uint64_t)c.D, (uint64_t)max_rows, BM) ||
+        !map_3d(&mG, w_gate, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E) ||
+        !map_3d(&mU, w_up, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E) ||
+        !map_2d(&mH, h, (uint64_t)c.F, (uint64_t)max_rows, BM) ||
+        !map_3d(&mD, w_down, (uint64_t)c.D, (uint64_t)c.F, (uint64_t)c.E))
+        return cudaErrorInvalidValue;
+
+    Args a1{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(h), c.E, c.D, c.F,
+            (c.F + Cfg<true>::BN - 1) / Cfg<true>::BN, max_rows, c.T * c.K, status};
+    int64_t g1 = mtiles_bound * a1.n_tiles;
+    if (g1 > sms) g1 = sms;
+    ffn_tc_kernel<true><<<(unsigned)g1, NUM_THREADS, SMEM_BYTES, s>>>(mA, mG, mU, a1);
+    if (mid) mid(mid_ctx, s);
+
+    Args a2{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(y_perm), c.E, c.F, c.D,
+            (c.D + Cfg<false>::BN - 1) / Cfg<false>::BN, max_rows, c.T * c.K, status};
+    int64_t g2 = mtiles_bound * a2.n_tiles;
+    if (g2 > sms) g2 = sms;
+    ffn_tc_kernel<false><<<(unsigned)g2, NUM_THREADS, SMEM_BYTES, s>>>(mH, mD, mD, a2);
+    return cudaGetLastError();
+}
+
+}  // namespace moe
