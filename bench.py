@@ -193,7 +193,7 @@ def run_gpu(args):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     init_dist(world, "nccl")
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
 
     inp = make_inputs(wl, device=dev)
     layer = M.MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
@@ -422,12 +422,27 @@ def _cpu_inputs_for_sample(wl: Workload):
     return dict(x=x, w_router=w_router, bias=bias, noise=noise, get_expert=get)
 
 
+def workload_of(args) -> Workload:
+    """The named workload, with any --override KEY=VALUE applied (a smaller case
+    of the same kernels, for profiler captures; renamed so it is never mistaken
+    for the named workload)."""
+    wl = WORKLOADS[args.workload]
+    if args.override:
+        kw = {}
+        for item in args.override:
+            k, v = item.split("=", 1)
+            kw[k] = type(getattr(wl, k))(v)
+        tag = ",".join(f"{k}={v}" for k, v in kw.items())
+        wl = wl.with_(name=f"{wl.name}[{tag}]", **kw)
+    return wl
+
+
 def run_reference(args):
     """The oracle on the host cores, timed per step on a bounded sample."""
     rank, world, _ = rank_info()
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     per_step = max(2.0, args.cpu_seconds / 2)
     if args.warmup > 0:
         cpu_baseline(wl, min(per_step, 4.0) / 2)
@@ -463,6 +478,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="mixtral_8x", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--override", action="append", default=[],
+                    help="KEY=VALUE change of the workload shape (profiling cases only)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
