@@ -223,6 +223,34 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * moe_dispatch without a workspace, for callers that cannot allocate device
+ * memory: code handed only its input and output buffers by a host framework
+ * (a plugin in an inference engine, a fixed-budget C program) has no
+ * workspace to pass, and cudaMalloc is not open to it because the call can
+ * synchronise the device and lies outside the memory it was budgeted.  The
+ * sources have no counterpart of this entry point; it is a deployment aid.
+ *
+ * Same arguments and results as moe_dispatch, minus the workspace.  Its
+ * scratch (status word, per-chunk counts and rank bases) lives in a static
+ * device array of 256 KiB inside the library, which every GPU that loads the
+ * library holds until the process exits.  A problem whose scratch would not
+ * fit (2 * ceil(T*K / 2048) * E int32 words plus 256 bytes) is rejected with
+ * MOE_ERR_WORKSPACE before anything is enqueued.  Allocates nothing.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call clears what must start at zero.  Calls whose work
+ *     overlaps on the GPU (other streams, other threads) race on the array:
+ *     order them on one stream.
+ *   - Device-side range checks still guard every write, but their flags are
+ *     kept in the shared array and are not reported to the caller.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
+                                        const int32_t *topk_ids, int32_t *counts, int32_t *kept,
+                                        int32_t *offsets, int32_t *perm, int32_t *row_of,
+                                        void *x_perm, void *stream);
+
+/*
  * Device status of a workspace: synchronises the stream, then reads the
  * status word.  *flags receives MOE_DEVFLAG_* bits (0 when clean).  Returns
  * MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BOUNDS when a flag is set, MOE_OK

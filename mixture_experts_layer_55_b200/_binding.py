@@ -69,6 +69,7 @@ _SIG = {
     "moe_forward_workspace_size": ([_P, _P], ctypes.c_int32),
     "moe_route": ([_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_dispatch_noalloc": ([_P] * 10, ctypes.c_int32),
     "moe_expert_ffn": ([_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([_P] * 5, ctypes.c_int32),
     "moe_forward": ([_P] * 15 + [ctypes.c_size_t, _P], ctypes.c_int32),
@@ -187,6 +188,16 @@ def moe_dispatch(cfg, x, topk_ids, counts, kept, offsets, perm, row_of, x_perm, 
                             _ptr(offsets), _ptr(perm), _ptr(row_of), _ptr(x_perm), _ptr(workspace),
                             _nbytes(workspace), _stream(stream))
     _check(st, "moe_dispatch")
+
+
+def moe_dispatch_noalloc(cfg, x, topk_ids, counts, kept, offsets, perm, row_of, x_perm,
+                         stream=None):
+    """moe_dispatch with its scratch in the library's static device array (no
+    workspace argument; for callers that cannot allocate device memory)."""
+    st = lib().moe_dispatch_noalloc(_cfg(cfg), _ptr(x), _ptr(topk_ids), _ptr(counts), _ptr(kept),
+                                    _ptr(offsets), _ptr(perm), _ptr(row_of), _ptr(x_perm),
+                                    _stream(stream))
+    _check(st, "moe_dispatch_noalloc")
 
 
 def moe_expert_ffn(cfg, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h, y_perm, workspace,

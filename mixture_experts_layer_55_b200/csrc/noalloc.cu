@@ -1,0 +1,93 @@
+// noalloc.cu -- moe_dispatch_noalloc: the dispatch with its scratch memory in
+// a static device array instead of a caller-allocated workspace.
+//
+// For callers that are handed only their input and output buffers and may not
+// allocate device memory themselves (for example a plugin enqueued by a host
+// inference framework, or a C program with a fixed memory budget): they have
+// no workspace to pass, and cudaMalloc is not open to them because it can
+// synchronise the device and falls outside the memory they were budgeted.
+//
+// The scratch (device status word, per-chunk expert counts and rank bases)
+// lives in g_noalloc_scratch, kNoallocScratchBytes = 256 KiB, which every GPU
+// that loads the library holds until the process exits.  In host code the
+// array's name is only a host-side stand-in, so its device address is taken
+// with cudaGetSymbolAddress once per device, on that device's first call.
+#include <mutex>
+
+#include "internal.h"
+
+namespace moe {
+
+constexpr size_t kNoallocScratchBytes = 256 * 1024;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static void* g_noalloc_ptr[kMaxDevices];
+static std::mutex g_noalloc_mutex;
+
+// Device address of the static scratch on the current device (set-up on the
+// first call made with that device current).
+static cudaError_t noalloc_scratch(char** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = static_cast<char*>(g_noalloc_ptr[dev]);
+    return cudaSuccess;
+}
+
+// The dispatch kernels' scratch regions packed into the static array.
+static WsLayout noalloc_layout(const moe_config& c)
+{
+    const int64_t nch = dispatch_chunks(c);
+    WsLayout L{};
+    L.status = 0;
+    L.d_cnt = align_up(64 * sizeof(int));
+    L.d_base = L.d_cnt + align_up((size_t)nch * c.E * sizeof(int32_t));
+    L.total = L.d_base + align_up((size_t)nch * c.E * sizeof(int32_t));
+    return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
+                                           const int32_t* topk_ids, int32_t* counts,
+                                           int32_t* kept, int32_t* offsets, int32_t* perm,
+                                           int32_t* row_of, void* x_perm, void* stream)
+{
+    moe_status st = moe_check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!topk_ids || !counts || !kept || !offsets || !perm || !row_of) return MOE_ERR_ARG;
+    if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_ARG;
+    if (x && (((uintptr_t)x & 15u) != 0 || ((uintptr_t)x_perm & 15u) != 0)) return MOE_ERR_ALIGN;
+    const WsLayout L = noalloc_layout(*cfg);
+    if (L.total > kNoallocScratchBytes) return MOE_ERR_WORKSPACE;  // beyond the static array
+    char* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the status word collects flags with atomic OR: it must start at zero
+    cudaError_t e = cudaMemsetAsync(scratch + L.status, 0, 64 * sizeof(int), s);
+    if (e == cudaSuccess) {
+        int64_t C = 0;
+        moe_capacity(cfg, &C);
+        e = launch_dispatch_index(*cfg, C, topk_ids, counts, kept, offsets, perm, row_of, scratch,
+                                  L, s);
+    }
+    if (e == cudaSuccess && x) {
+        int64_t rows = 0;
+        moe_max_rows(cfg, &rows);
+        e = launch_gather(*cfg, x, row_of, x_perm, rows, reinterpret_cast<int*>(scratch + L.status),
+                          s);
+    }
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
