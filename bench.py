@@ -35,9 +35,9 @@ from workloads import WORKLOADS, Workload, make_inputs, make_tokens  # noqa: E40
 METRIC = "routed tokens/s per MoE layer fwd on 1 B200; % bf16 tensor peak / % HBM BW"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# kernels this library launches per moe_forward (router 3, dispatch 3, gather 1,
+# kernels this library launches per moe_forward (router 4, dispatch 3, gather 1,
 # expert GEMMs 2, combine 1)
-LAUNCHES_PER_STEP = 10
+LAUNCHES_PER_STEP = 11
 
 
 # ------------------------------------------------------------------ ranks --

@@ -53,6 +53,8 @@ WsLayout ws_layout(const moe_config& c)
     o += align_up((size_t)rp.nb_topk * sizeof(float));
     L.r_cnt = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(int32_t));
+    L.r_fin = o;
+    o += align_up((size_t)(2 * c.E + 1) * sizeof(double));
     L.d_cnt = o;
     o += align_up((size_t)nch * c.E * sizeof(int32_t));
     L.d_base = o;

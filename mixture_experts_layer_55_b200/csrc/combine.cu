@@ -6,8 +6,8 @@
 // nothing, so an all-dropped token gets zero.
 //
 // The routing weight is already applied by the down GEMM's epilogue, so the
-// combine is a plain gather-sum: one warp per token, 16-byte vector loads of
-// the token's K rows of y_perm, summed in slot order in fp32 and rounded once.
+// combine is a plain gather-sum: 16-byte vector loads of the token's K rows of
+// y_perm, summed in slot order in fp32 and rounded once.
 // No atomics: the result is deterministic.
 #include "common.cuh"
 #include "internal.h"
@@ -48,52 +48,65 @@ template <> struct Vec<__nv_bfloat16> {
     }
 };
 
-constexpr int kCombineUnroll = 2;
-
-template <typename ET>
+// Each thread produces VPT 16-byte vectors of the output, with KS >= K slots
+// per token and VPT * KS = 8, so that about 8 loads are in flight per thread
+// whatever K is: vectors i, i + G, ... of the flattened (T x vec_per_row)
+// output, G = total threads.  row_of is shared by a row's threads through L1.
+// Consecutive threads cover consecutive vectors of a row (coalesced).
+template <typename ET, int KS>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ row_of,
                                                       uint4* __restrict__ y, int64_t T, int K,
                                                       int64_t vec_per_row, int64_t max_rows)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
-         t += warps) {
-        int32_t myrow = -1;
-        if (lane < K) {
-            myrow = row_of[t * K + lane];
-            if (myrow >= max_rows) myrow = -1;  // never read outside y_perm
+    constexpr int VPT = 8 / KS;
+    const int64_t n = T * vec_per_row;
+    const int64_t G = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n; base += G * VPT) {
+        uint4 vals[VPT][KS];
+        int32_t rows[VPT][KS];
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) {
+            const int64_t i = base + (int64_t)u * G;
+            const int64_t t = i < n ? i / vec_per_row : 0, v = i - t * vec_per_row;
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                int32_t r = (i < n && k < K) ? __ldg(row_of + t * K + k) : -1;
+                rows[u][k] = (r >= 0 && r < max_rows) ? r : -1;  // never read outside y_perm
+            }
+#pragma unroll
+            for (int k = 0; k < KS; ++k)
+                vals[u][k] = rows[u][k] >= 0 ? __ldg(y_perm + (int64_t)rows[u][k] * vec_per_row + v)
+                                             : make_uint4(0, 0, 0, 0);
         }
-        int32_t rows[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) rows[k] = __shfl_sync(0xffffffffu, myrow, k);
-        for (int64_t v0 = lane; v0 < vec_per_row; v0 += 32 * kCombineUnroll) {
-            float acc[kCombineUnroll][8];
+        for (int u = 0; u < VPT; ++u) {
+            const int64_t i = base + (int64_t)u * G;
+            if (i >= n) break;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int u = 0; u < kCombineUnroll; ++u)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if (k >= K || rows[k] < 0) continue;
-                const uint4* src = y_perm + (int64_t)rows[k] * vec_per_row;
-                uint4 v[kCombineUnroll];
-#pragma unroll
-                for (int u = 0; u < kCombineUnroll; ++u) {
-                    const int64_t vi = v0 + 32 * u;
-                    v[u] = vi < vec_per_row ? __ldg(src + vi) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < kCombineUnroll; ++u) Vec<ET>::add(acc[u], v[u]);
-            }
-#pragma unroll
-            for (int u = 0; u < kCombineUnroll; ++u) {
-                const int64_t vi = v0 + 32 * u;
-                if (vi < vec_per_row) y[t * vec_per_row + vi] = Vec<ET>::pack(acc[u]);
-            }
+            for (int k = 0; k < KS; ++k)
+                if (rows[u][k] >= 0) Vec<ET>::add(acc, vals[u][k]);  // slot order
+            y[i] = Vec<ET>::pack(acc);
         }
     }
+}
+
+template <typename ET>
+static void launch_combine_t(const moe_config& c, int64_t blocks, const void* y_perm,
+                             const int32_t* row_of, void* y, int64_t vpr, int64_t max_rows,
+                             cudaStream_t s)
+{
+    const uint4* src = static_cast<const uint4*>(y_perm);
+    uint4* dst = static_cast<uint4*>(y);
+    if (c.K <= 1)
+        combine_kernel<ET, 1><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+    else if (c.K == 2)
+        combine_kernel<ET, 2><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+    else if (c.K <= 4)
+        combine_kernel<ET, 4><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+    else
+        combine_kernel<ET, 8><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
 }
 
 cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
@@ -104,17 +117,15 @@ cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t blocks = (c.T + 7) / 8;
-    const int64_t cap = (int64_t)sms * 8;
+    const int vpt = c.K <= 1 ? 8 : c.K == 2 ? 4 : c.K <= 4 ? 2 : 1;
+    int64_t blocks = (c.T * vpr + 256LL * vpt - 1) / (256LL * vpt);
+    const int64_t cap = (int64_t)sms * 16;
     if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
     if (c.dtype == MOE_BF16)
-        combine_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
-            static_cast<const uint4*>(y_perm), row_of, static_cast<uint4*>(y), c.T, c.K, vpr,
-            max_rows);
+        launch_combine_t<__nv_bfloat16>(c, blocks, y_perm, row_of, y, vpr, max_rows, s);
     else
-        combine_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(y_perm),
-                                                               row_of, static_cast<uint4*>(y), c.T,
-                                                               c.K, vpr, max_rows);
+        launch_combine_t<float>(c, blocks, y_perm, row_of, y, vpr, max_rows, s);
     return cudaGetLastError();
 }
 

@@ -58,6 +58,23 @@ MOE_DEVICE float silu_f32(float g)
     return g / (1.0f + __expf(-g));
 }
 
+// silu(g) = g * sigmoid(g), with sigmoid(g) = (1 + tanh(g/2)) / 2, so
+// silu(g) = h + h * tanh(h), h = g/2.  tanh.approx.f32 is one hardware
+// instruction (relative error about 2^-11), well inside a bf16 result's own
+// rounding (2^-9); used where the result is rounded to bf16.
+MOE_DEVICE float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+MOE_DEVICE float silu_bf16_path(float g)
+{
+    const float h = 0.5f * g;
+    return fmaf(h, tanh_approx(h), h);
+}
+
 // --------------------------------------------------------------- mbarrier --
 MOE_DEVICE uint32_t smem_u32(const void* p)
 {
@@ -251,6 +268,100 @@ MOE_DEVICE uint32_t elect_one()
         "selp.u32 %0, 1, 0, P;\n\t}"
         : "=r"(pred));
     return pred;
+}
+
+// ------------------------------------------------------ CTA pairs (2-SM) --
+MOE_DEVICE uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+MOE_DEVICE void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+MOE_DEVICE uint32_t mapa_shared(uint32_t smem_addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
+MOE_DEVICE void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// Tiled TMA load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster
+// address).  No multicast: each CTA loads only its own tile.
+MOE_DEVICE void tma_load_2d_pair(void* smem_dst, const void* tmap, int32_t c0, int32_t c1,
+                                 uint32_t bar_cluster)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(bar_cluster)
+        : "memory");
+}
+
+MOE_DEVICE void tma_load_3d_pair(void* smem_dst, const void* tmap, int32_t c0, int32_t c1,
+                                 int32_t c2, uint32_t bar_cluster)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(bar_cluster)
+        : "memory");
+}
+
+MOE_DEVICE void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+MOE_DEVICE void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+MOE_DEVICE void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// D (256 rows over the pair) (+)= A (128 rows per CTA) * B (N/2 columns per CTA).
+MOE_DEVICE void umma_f16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                 uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier at this shared offset in every CTA of `cta_mask` once
+// the pair's tcgen05 ops issued so far by this thread complete.
+MOE_DEVICE void umma_commit_pair_mc(uint64_t* bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
 }
 
 // --------------------------------------------------- shared-memory layouts --

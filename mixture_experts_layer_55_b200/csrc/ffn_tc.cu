@@ -12,13 +12,19 @@
 //   down:     Y = h[block] . Wd_e                       (K = F)
 //             y_perm = bf16(topk_w[perm[row]] * Y)      (epilogue)
 //
-// One persistent CTA per SM, 6 warps:
+// Persistent kernel, one CTA per SM, either alone (M = 128 rows per tile,
+// cta_group::1) or as a CTA pair on two SMs (M = 256, cta_group::2: each CTA
+// holds its 128 rows of A and half of B's columns, the leader issues the MMAs
+// for both).  10 warps per CTA:
 //   warp 0      TMA producer: A tile 128 x 64 (K-major, 128-byte swizzle) and
-//               B tiles 64 x 64 (N-major, 128-byte swizzle) into a 4-stage ring
-//   warp 1      MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M = 128,
-//               N = 128 (x2 for gate/up) or 256 (down), K = 16 per instruction;
+//               B tiles 64 x 64 (N-major, 128-byte swizzle) into a 4-stage
+//               (single) or 6-stage (pair) ring
+//   warp 1      MMA issuer: tcgen05.mma.kind::f16, N = 256, K = 16 per
+//               instruction (gate/up: gate and up columns interleaved in
+//               64-column blocks, so one MMA feeds both accumulators);
 //               it also owns the 512-column tensor-memory allocation
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (lane = row), the
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (lane = row; two
+//               warps per lane quadrant, each half of the columns), the
 //               SwiGLU or routing-weight step, bf16 stores to global memory
 // Accumulators are double-buffered in tensor memory (2 x 256 columns), so the
 // epilogue of one tile overlaps the MMAs of the next.  Tiles are ordered
@@ -34,22 +40,33 @@
 namespace moe {
 namespace tc {
 
-constexpr int BM = 128;               // rows per tile (UMMA M)
-constexpr int BK = 64;                // K per stage: one 128-byte swizzle row of bf16
-constexpr int UK = 16;                // K per tcgen05.mma (bf16)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BK * 256 * 2; // 32 KB: [gate 128 | up 128] or down 256 columns
-constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64 x 64 B box
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int ACC_COLS = 256;         // tensor-memory columns per accumulator buffer
+constexpr int BK = 64;                 // K per stage: one 128-byte swizzle row of bf16
+constexpr int UK = 16;                 // K per tcgen05.mma (bf16)
+constexpr int BOX_BYTES = 64 * 64 * 2; // one 64 x 64 B box
+constexpr int A_BYTES = 128 * BK * 2;  // this CTA's 128 rows of A per stage: 16 KB
+constexpr int ACC_COLS = 256;          // tensor-memory columns per accumulator buffer
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;      // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int EPI_WARPS = 8;          // two per tensor-memory lane quadrant
 constexpr int MAX_E = 256;
 
+// Tile geometry.  Single CTA: M = 128 rows, all N columns of the tile's B in
+// this CTA (gate/up: 128 gate + 128 up; down: 256).  CTA pair: M = 256 rows,
+// 128 per CTA, and each CTA holds half of every B tile's columns.
+template <bool GATEUP, bool PAIR> struct Geo {
+    static constexpr int CTAS = PAIR ? 2 : 1;
+    static constexpr int BM = 128 * CTAS;                  // rows per tile
+    static constexpr int BN = GATEUP ? 128 : 256;          // output columns per tile
+    static constexpr int B_BOXES = (GATEUP ? 2 * 128 : 256) / 64 / CTAS;  // B boxes per CTA per stage
+    static constexpr int B_BYTES = B_BOXES * BOX_BYTES;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB single, 32 KB pair
+    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;  // one per epilogue warp
+};
+
 struct Misc {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[8];
+    uint64_t empty[8];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -60,7 +77,12 @@ struct Misc {
     int pref[MAX_E + 1];  // first tile index of each expert; pref[E] = total tiles
 };
 
-constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Misc);
+template <bool GATEUP, bool PAIR>
+constexpr size_t smem_bytes()
+{
+    return 1024 /*alignment slack*/ + (size_t)Geo<GATEUP, PAIR>::STAGES * Geo<GATEUP, PAIR>::STAGE_BYTES +
+           sizeof(Misc);
+}
 
 struct Args {
     const int32_t* offsets;
@@ -76,11 +98,7 @@ struct Args {
     int* status;
 };
 
-template <bool GATEUP> struct Cfg {
-    static constexpr int BN = GATEUP ? 128 : 256;  // output columns per tile
-};
-
-MOE_DEVICE void decode_tile(const Misc* m, int E, int n_tiles, int bn, int t, int& e, int& m_row0,
+MOE_DEVICE void decode_tile(const Misc* m, int E, int bm, int bn, int t, int& e, int& m_row0,
                             int& row_end, int& n0)
 {
     int lo = 0, hi = E - 1;
@@ -90,20 +108,21 @@ MOE_DEVICE void decode_tile(const Misc* m, int E, int n_tiles, int bn, int t, in
         else hi = mid - 1;
     }
     e = lo;
-    const int mt = (m->rowend[e] - m->row0[e] + BM - 1) / BM;
+    const int mt = (m->rowend[e] - m->row0[e] + bm - 1) / bm;
     const int local = t - m->pref[e];
     const int n = local / mt, mm = local - n * mt;
-    m_row0 = m->row0[e] + mm * BM;
+    m_row0 = m->row0[e] + mm * bm;
     row_end = m->rowend[e];
     n0 = n * bn;
 }
 
-template <bool GATEUP>
+template <bool GATEUP, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                   const __grid_constant__ CUtensorMap tmB1, const Args a)
 {
-    constexpr int BN = Cfg<GATEUP>::BN;
+    using G = Geo<GATEUP, PAIR>;
+    constexpr int BM = G::BM, BN = G::BN, STAGES = G::STAGES, STAGE_BYTES = G::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -111,6 +130,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = a.E;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader (issues the MMAs)
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // pair (or CTA) index
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -119,7 +141,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&m->tfull[b], 1);
-            mbar_init(&m->tempty[b], 128);
+            mbar_init(&m->tempty[b], G::EPI_ARRIVALS);
         }
         mbar_init(&m->drain, 1);
         m->abort_flag = 0;
@@ -129,8 +151,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (GATEUP) prefetch_tmap(&tmB1);
     }
     if (warp == 1) {
-        tmem_alloc(&m->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&m->tmem_base, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&m->tmem_base, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     // tile table from the offsets (validated: a malformed block is treated as empty)
     for (int e = threadIdx.x; e < E; e += NUM_THREADS) {
@@ -155,7 +182,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         m->pref[E] = run;
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote signal
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
     const int total = m->pref[E];
@@ -163,15 +191,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int* abort_flag = &m->abort_flag;
 
     if (warp == 0 && lane == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (each CTA)
         int stage = 0;
         uint32_t phase = 0;
         int last_phase[STAGES];
         for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = unit; t < total && ok; t += units) {
             int e, m_row0, row_end, n0;
-            decode_tile(m, E, a.n_tiles, BN, t, e, m_row0, row_end, n0);
+            decode_tile(m, E, BM, BN, t, e, m_row0, row_end, n0);
+            const int a_row = m_row0 + (int)rank * 128;
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 410, abort_flag)) {
                     ok = false;
@@ -179,18 +208,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
                 uint8_t* sB = sA + A_BYTES;
-                uint64_t* fb = &m->full[stage];
-                mbar_arrive_expect_tx(fb, STAGE_BYTES);
                 const int k0 = kb * BK;
-                tma_load_2d(sA, &tmA, k0, m_row0, fb);
-                if (GATEUP) {
-                    tma_load_3d(sB, &tmB0, n0, k0, e, fb);
-                    tma_load_3d(sB + BOX_BYTES, &tmB0, n0 + 64, k0, e, fb);
-                    tma_load_3d(sB + 2 * BOX_BYTES, &tmB1, n0, k0, e, fb);
-                    tma_load_3d(sB + 3 * BOX_BYTES, &tmB1, n0 + 64, k0, e, fb);
+                if (PAIR) {
+                    // both CTAs' bytes are counted on the leader's full barrier
+                    if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
+                    tma_load_2d_pair(sA, &tmA, k0, a_row, fb);
+                    if (GATEUP) {  // this CTA's [gate 64 | up 64] columns
+                        tma_load_3d_pair(sB, &tmB0, n0 + 64 * (int)rank, k0, e, fb);
+                        tma_load_3d_pair(sB + BOX_BYTES, &tmB1, n0 + 64 * (int)rank, k0, e, fb);
+                    } else {       // this CTA's 128 down columns
+                        tma_load_3d_pair(sB, &tmB0, n0 + 128 * (int)rank, k0, e, fb);
+                        tma_load_3d_pair(sB + BOX_BYTES, &tmB0, n0 + 128 * (int)rank + 64, k0, e, fb);
+                    }
                 } else {
+                    uint64_t* fb = &m->full[stage];
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(sA, &tmA, k0, a_row, fb);
+                    if (GATEUP) {  // [gate n0 | up n0 | gate n0+64 | up n0+64]
+                        tma_load_3d(sB, &tmB0, n0, k0, e, fb);
+                        tma_load_3d(sB + BOX_BYTES, &tmB1, n0, k0, e, fb);
+                        tma_load_3d(sB + 2 * BOX_BYTES, &tmB0, n0 + 64, k0, e, fb);
+                        tma_load_3d(sB + 3 * BOX_BYTES, &tmB1, n0 + 64, k0, e, fb);
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) tma_load_3d(sB + j * BOX_BYTES, &tmB0, n0 + 64 * j, k0, e, fb);
+                        for (int j = 0; j < 4; ++j)
+                            tma_load_3d(sB + j * BOX_BYTES, &tmB0, n0 + 64 * j, k0, e, fb);
+                    }
                 }
                 last_phase[stage] = (int)phase;
                 if (++stage == STAGES) {
@@ -199,18 +243,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
         }
-        // never leave the CTA with a copy in flight
-        for (int s = 0; s < STAGES; ++s)
-            if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 411, nullptr);
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = GATEUP ? umma_idesc_bf16(BM, 128, 0, 1) : umma_idesc_bf16(BM, 256, 0, 1);
+        // never leave the CTA with a copy in flight (the leader sees every completion)
+        if (!PAIR || rank == 0)
+            for (int s = 0; s < STAGES; ++s)
+                if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 411, nullptr);
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        constexpr uint32_t idesc = umma_idesc_bf16(BM, 256, 0, 1);
+        // B: N-major; 64-column blocks 8 KB apart (LBO), 8-row K groups 1024 B apart (SBO)
         int stage = 0;
         uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = unit; t < total && ok; t += units) {
             if (!mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 420, abort_flag)) break;
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -227,43 +273,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
                     // A: K-major, 8-row groups 1024 B apart; +32 B per 16-element K step
                     const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
-                    // B: N-major, 64-column blocks 8 KB apart (LBO), 8-row K groups
-                    // 1024 B apart (SBO); +2048 B per 16-row K step
-                    if (GATEUP) {
-                        const uint64_t bg = umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
-                        const uint64_t bu = umma_desc_sw128(sB + 2 * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
-                        umma_f16_ss(d0, adesc, bg, idesc, accum);
-                        umma_f16_ss(d0 + 128, adesc, bu, idesc, accum);
-                    } else {
-                        const uint64_t bd = umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
-                        umma_f16_ss(d0, adesc, bd, idesc, accum);
-                    }
+                    // one N = 256 MMA: the 64-column boxes of B (for gate/up,
+                    // gate and up interleaved) are 8 KB apart
+                    const uint64_t bdesc = umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
+                    if (PAIR) umma_f16_ss_pair(d0, adesc, bdesc, idesc, accum);
+                    else umma_f16_ss(d0, adesc, bdesc, idesc, accum);
                 }
-                umma_commit(&m->empty[stage]);  // frees the stage once these MMAs complete
+                // frees the stage (in both CTAs) once these MMAs complete
+                if (PAIR) umma_commit_pair_mc(&m->empty[stage], 0x3);
+                else umma_commit(&m->empty[stage]);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
             if (!ok) break;
-            umma_commit(&m->tfull[acc]);  // accumulator ready for the epilogue
+            // accumulator ready for the epilogue (of both CTAs)
+            if (PAIR) umma_commit_pair_mc(&m->tfull[acc], 0x3);
+            else umma_commit(&m->tfull[acc]);
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
         }
         // wait for every MMA issued here before the allocation is released
-        umma_commit(&m->drain);
+        if (PAIR) umma_commit_pair_mc(&m->drain, 0x1);
+        else umma_commit(&m->drain);
         mbar_wait(&m->drain, 0, a.status, 422, nullptr);
     } else if (warp >= 2) {
-        // ------------------------------------------------ epilogue
-        const int quad = warp & 3;  // tensor-memory lanes this warp may read
-        const int r_in_tile = quad * 32 + lane;
+        // ------------------------------------------------ epilogue (each CTA, its 128 rows)
+        // warp w reads tensor-memory lanes 32*(w%4) .. +31 (rows), and half of
+        // the tile's columns: warps 2..5 the first half, warps 6..9 the second.
+        const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int r_in_tile = (int)rank * 128 + quad * 32 + lane;
+        const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m->tempty[0]), 0);
+        const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m->tempty[1]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        for (int t = unit; t < total; t += units) {
             int e, m_row0, row_end, n0;
-            decode_tile(m, E, a.n_tiles, BN, t, e, m_row0, row_end, n0);
+            decode_tile(m, E, BM, BN, t, e, m_row0, row_end, n0);
             if (!mbar_wait(&m->tfull[acc], acc_phase, a.status, 430, abort_flag)) break;
             tc_fence_after();
             const int64_t row = (int64_t)m_row0 + r_in_tile;
@@ -272,18 +322,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __nv_bfloat16* orow = a.out + row * (int64_t)a.N;
             if (GATEUP) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 2 * half; c < 2 * half + 2; ++c) {
+                    // accumulator columns: [gate 0-63 | up 0-63 | gate 64-127 | up 64-127]
                     uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(taddr + c * 32, g);
-                    tmem_ld_32x32b_x32(taddr + 128 + c * 32, u);
+                    const uint32_t gcol = (c < 2) ? (uint32_t)(c * 32) : (uint32_t)(128 + (c - 2) * 32);
+                    tmem_ld_32x32b_x32(taddr + gcol, g);
+                    tmem_ld_32x32b_x32(taddr + gcol + 64, u);
                     tmem_ld_wait();
                     if (valid) {
                         uint32_t p[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const float h0 = silu_f32(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
+                            const float h0 = silu_bf16_path(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
                             const float h1 =
-                                silu_f32(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
+                                silu_bf16_path(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
                             p[j] = pack_bf16x2(h0, h1);
                         }
                         const int col = n0 + c * 32;
@@ -299,10 +351,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (valid) {
                     const int32_t pa = a.perm[row];
                     if (pa >= 0 && (int64_t)pa < a.nk) w = a.topk_w[pa];
-                    else raise_flag(a.status, kFlagBounds, 431);
+                    else if (half == 0) raise_flag(a.status, kFlagBounds, 431);
                 }
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 4 * half; c < 4 * half + 4; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
                     tmem_ld_wait();
@@ -320,8 +372,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
+            // this warp is done reading the accumulator: one arrival per warp, on
+            // the leader's barrier (the MMA issuer waits there)
             tc_fence_before();
-            mbar_arrive(&m->tempty[acc]);
+            __syncwarp();
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+                else mbar_arrive(&m->tempty[acc]);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -329,10 +387,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync();  // no CTA leaves while its peer may still signal it
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
@@ -384,21 +444,86 @@ static bool map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATEUP>
-static cudaError_t prepare()
+// Per device: dynamic shared memory opted in, and the number of CTAs (or CTA
+// pairs) that can be resident at once, which sizes the persistent grid.
+template <bool GATEUP, bool PAIR>
+static cudaError_t prepare(int* resident_units)
 {
-    static int done_dev_mask = 0;  // devices 0..30 on which the attribute was set
+    static int cached[32];  // 0 = not yet queried on that device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 31 && (done_dev_mask >> dev) & 1) return cudaSuccess;
-    e = cudaFuncSetAttribute(ffn_tc_kernel<GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BYTES);
-    if (e == cudaSuccess && dev < 31) done_dev_mask |= 1 << dev;
-    return e;
+    if (dev < 32 && cached[dev] > 0) {
+        *resident_units = cached[dev];
+        return cudaSuccess;
+    }
+    constexpr size_t smem = smem_bytes<GATEUP, PAIR>();
+    e = cudaFuncSetAttribute(ffn_tc_kernel<GATEUP, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    int units = 0;
+    if (PAIR) {
+        e = cudaFuncSetAttribute(ffn_tc_kernel<GATEUP, PAIR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaOccupancyMaxActiveClusters(&units, ffn_tc_kernel<GATEUP, PAIR>, &cfg);
+        if (e != cudaSuccess) return e;
+    } else {
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        units = sms;  // one CTA per SM (shared memory allows no second)
+    }
+    if (units < 1) return cudaErrorInvalidConfiguration;
+    if (dev < 32) cached[dev] = units;
+    *resident_units = units;
+    return cudaSuccess;
+}
+
+template <bool GATEUP, bool PAIR>
+static cudaError_t launch_one(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
+                              const Args& a, int64_t tiles_bound, cudaStream_t s)
+{
+    int units = 0;
+    cudaError_t e = prepare<GATEUP, PAIR>(&units);
+    if (e != cudaSuccess) return e;
+    int64_t n = tiles_bound < units ? tiles_bound : units;
+    if (n < 1) n = 1;
+    constexpr size_t smem = smem_bytes<GATEUP, PAIR>();
+    if (!PAIR) {
+        ffn_tc_kernel<GATEUP, false><<<(unsigned)n, NUM_THREADS, smem, s>>>(mA, mB0, mB1, a);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * n), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<GATEUP, true>, mA, mB0, mB1, a);
 }
 
 }  // namespace tc
+
+// CTA pairs (256-row tiles) when experts hold 128 rows or more on average;
+// single CTAs (128-row tiles) otherwise, which waste fewer padded rows when
+// each expert has only a few tokens (decode-shaped layers).
+static bool use_pairs(const moe_config& c, int64_t max_rows) { return max_rows >= 128 * (int64_t)c.E; }
 
 cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
@@ -407,35 +532,27 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
                                void* mid_ctx)
 {
     using namespace tc;
-    cudaError_t err = prepare<true>();
-    if (err == cudaSuccess) err = prepare<false>();
-    if (err != cudaSuccess) return err;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t mtiles_bound = (max_rows + BM - 1) / BM + c.E;
-
     CUtensorMap mA, mG, mU, mH, mD;
-    if (!map_2d(&mA, x_perm, (uint64_t)c.D, (uint64_t)max_rows, BM) ||
+    if (!map_2d(&mA, x_perm, (uint64_t)c.D, (uint64_t)max_rows, 128) ||
         !map_3d(&mG, w_gate, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E) ||
         !map_3d(&mU, w_up, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E) ||
-        !map_2d(&mH, h, (uint64_t)c.F, (uint64_t)max_rows, BM) ||
+        !map_2d(&mH, h, (uint64_t)c.F, (uint64_t)max_rows, 128) ||
         !map_3d(&mD, w_down, (uint64_t)c.D, (uint64_t)c.F, (uint64_t)c.E))
         return cudaErrorInvalidValue;
+    const bool pair = use_pairs(c, max_rows);
+    const int64_t bm = pair ? 256 : 128;
+    const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
 
     Args a1{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(h), c.E, c.D, c.F,
-            (c.F + Cfg<true>::BN - 1) / Cfg<true>::BN, max_rows, c.T * c.K, status};
-    int64_t g1 = mtiles_bound * a1.n_tiles;
-    if (g1 > sms) g1 = sms;
-    ffn_tc_kernel<true><<<(unsigned)g1, NUM_THREADS, SMEM_BYTES, s>>>(mA, mG, mU, a1);
+            (c.F + 127) / 128, max_rows, c.T * c.K, status};
+    cudaError_t err = pair ? launch_one<true, true>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<true, false>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s);
+    if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
-
     Args a2{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(y_perm), c.E, c.F, c.D,
-            (c.D + Cfg<false>::BN - 1) / Cfg<false>::BN, max_rows, c.T * c.K, status};
-    int64_t g2 = mtiles_bound * a2.n_tiles;
-    if (g2 > sms) g2 = sms;
-    ffn_tc_kernel<false><<<(unsigned)g2, NUM_THREADS, SMEM_BYTES, s>>>(mH, mD, mD, a2);
-    return cudaGetLastError();
+            (c.D + 255) / 256, max_rows, c.T * c.K, status};
+    return pair ? launch_one<false, true>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s)
+                : launch_one<false, false>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s);
 }
 
 }  // namespace moe

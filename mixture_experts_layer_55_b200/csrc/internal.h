@@ -39,6 +39,7 @@ struct WsLayout {
     size_t r_mp;        // nb_topk * E fp32
     size_t r_z;         // nb_topk fp32
     size_t r_cnt;       // nb_topk * E int32
+    size_t r_fin;       // (2E + 1) fp64: probability sums, z sum, counts
     size_t d_cnt;       // chunks * E int32
     size_t d_base;      // chunks * E int32
     size_t total;

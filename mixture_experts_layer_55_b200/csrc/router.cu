@@ -13,24 +13,29 @@
 //                         fixed order, adds bias and noise, softmax, top-k by
 //                         (logit desc, id asc) with warp shuffles, weights,
 //                         and per-block statistic partials.
-//   router_finalize_kernel fixed-order reduction of the block partials.
+//   router_colsum_kernel  per-expert fixed-order reduction of the block partials.
+//   router_finalize_kernel mean probabilities, z-loss and balance loss.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-constexpr int kLogitsBT = 64;  // tokens per logits block
-constexpr int kLogitsBD = 32;  // d_model per smem step
-constexpr int kTopkTPB = 64;   // tokens per top-k block (8 warps x 8)
+constexpr int kLogitsBD = 32;  // d_model per shared-memory step
+constexpr int kTopkTPB = 16;   // tokens per top-k block (8 warps x 2)
+
+// Tokens per logits block for an expert tile of be columns (see the kernel's
+// thread layout): 128 for be = 8, else 64.
+static int logits_bt(int be) { return be == 8 ? 128 : 64; }
 
 RouterPlan router_plan(const moe_config& c)
 {
     RouterPlan p;
     p.be = c.E <= 8 ? 8 : c.E <= 16 ? 16 : c.E <= 32 ? 32 : 64;
-    p.grid_t = (int)((c.T + kLogitsBT - 1) / kLogitsBT);
+    const int bt = logits_bt(p.be);
+    p.grid_t = (int)((c.T + bt - 1) / bt);
     p.grid_e = (c.E + p.be - 1) / p.be;
     int64_t base = (int64_t)p.grid_t * p.grid_e;
-    int want = (int)((2 * 148 + base - 1) / base);
+    int want = (int)((6 * 148 + base - 1) / base);  // enough blocks to hide load latency
     int max_splits = c.D / 256 > 1 ? c.D / 256 : 1;
     if (want > max_splits) want = max_splits;
     if (want < 1) want = 1;
@@ -42,20 +47,48 @@ RouterPlan router_plan(const moe_config& c)
     return p;
 }
 
-// Thread layout: 256 threads = (BT/TM) token groups x (BE/TE) expert groups.
-// Thread (ty, tx) owns tokens ty + i*(BT/TM) and experts tx + j*(BE/TE), so
-// that neighbouring threads read neighbouring shared-memory words.
+template <typename XT> struct XVec;  // 16-byte vector of x elements
+template <> struct XVec<float> {
+    static constexpr int N = 4;
+    MOE_DEVICE static void to_f32(const uint4& v, float* o)
+    {
+        o[0] = __uint_as_float(v.x); o[1] = __uint_as_float(v.y);
+        o[2] = __uint_as_float(v.z); o[3] = __uint_as_float(v.w);
+    }
+};
+template <> struct XVec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    MOE_DEVICE static void to_f32(const uint4& v, float* o)
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o[2 * i] = __uint_as_float(w[i] << 16);
+            o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+// Logits GEMM partials: part[z][t][e] = sum over this block's d-split of
+// x[t][d] * W_r[d][e].  256 threads = NTY token groups x NTX expert groups;
+// thread (ty, tx) owns tokens ty*TM .. ty*TM+TM-1 (one float4 of the
+// transposed x tile) and experts tx + j*NTX.  x arrives as 16-byte vectors;
+// the next tile is prefetched into registers while the current one is used.
 template <typename XT, int BE, int TM, int TE>
 __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict__ x,
                                                             const float* __restrict__ w,
                                                             float* __restrict__ part, int64_t T,
                                                             int D, int E, int dps)
 {
-    constexpr int BT = kLogitsBT, BD = kLogitsBD;
-    constexpr int NTX = BE / TE, NTY = BT / TM;
-    static_assert(NTX * NTY == 256, "256 threads");
-    __shared__ float xs[BD][BT + 1];
-    __shared__ float wsm[BD][BE];
+    constexpr int BD = kLogitsBD;
+    constexpr int NTX = BE / TE, NTY = 256 / NTX, BT = NTY * TM;
+    static_assert(TM == 4, "float4 token reads");
+    constexpr int VN = XVec<XT>::N;                   // elements per 16-byte vector
+    constexpr int XV = BT * BD / VN / 256;            // x vectors per thread per step
+    constexpr int WV = BD * BE / 256;                 // w scalars per thread per step
+    static_assert(XV >= 1 && WV >= 1, "tile sizes");
+    __shared__ __align__(16) float xs[2][BD][BT + 4];
+    __shared__ float wsm[2][BD][BE];
 
     const int tid = threadIdx.x;
     const int tx = tid % NTX, ty = tid / NTX;
@@ -64,50 +97,82 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict
     const int d_begin = blockIdx.z * dps;
     const int d_end = min(D, d_begin + dps);
 
+    uint4 xr[XV];
+    float wr[WV];
+    auto load = [&](int d0) {
+#pragma unroll
+        for (int i = 0; i < XV; ++i) {
+            const int idx = tid + i * 256;
+            const int tt = idx / (BD / VN), dv = idx % (BD / VN);
+            const int64_t t = t0 + tt;
+            const int d = d0 + dv * VN;
+            xr[i] = (t < T && d < d_end) ? __ldg(reinterpret_cast<const uint4*>(x + t * D + d))
+                                         : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < WV; ++i) {
+            const int idx = tid + i * 256;
+            const int dd = idx / BE, ee = idx % BE;
+            const int d = d0 + dd, e = e0 + ee;
+            wr[i] = (d < d_end && e < E) ? __ldg(w + (int64_t)d * E + e) : 0.f;
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int i = 0; i < XV; ++i) {
+            const int idx = tid + i * 256;
+            const int tt = idx / (BD / VN), dv = idx % (BD / VN);
+            float v[VN];
+            XVec<XT>::to_f32(xr[i], v);
+#pragma unroll
+            for (int k = 0; k < VN; ++k) xs[buf][dv * VN + k][tt] = v[k];
+        }
+#pragma unroll
+        for (int i = 0; i < WV; ++i) {
+            const int idx = tid + i * 256;
+            wsm[buf][idx / BE][idx % BE] = wr[i];
+        }
+    };
+
     float acc[TM][TE];
 #pragma unroll
     for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < TE; ++j) acc[i][j] = 0.f;
 
+    int buf = 0;
+    load(d_begin);
+    store(0);
+    __syncthreads();
     for (int d0 = d_begin; d0 < d_end; d0 += BD) {
-        // x tile: BT tokens x BD columns, stored transposed (d-major).
-        for (int idx = tid; idx < BT * BD; idx += 256) {
-            int tt = idx / BD, dd = idx % BD;
-            int64_t t = t0 + tt;
-            int d = d0 + dd;
-            float v = 0.f;
-            if (t < T && d < d_end) v = to_f32(x[t * D + d]);
-            xs[dd][tt] = v;
-        }
-        for (int idx = tid; idx < BD * BE; idx += 256) {
-            int dd = idx / BE, ee = idx % BE;
-            int d = d0 + dd, e = e0 + ee;
-            wsm[dd][ee] = (d < d_end && e < E) ? w[(int64_t)d * E + e] : 0.f;
-        }
-        __syncthreads();
+        const bool more = d0 + BD < d_end;
+        if (more) load(d0 + BD);
 #pragma unroll 8
         for (int dd = 0; dd < BD; ++dd) {
-            float xv[TM], wv[TE];
+            const float4 xv = *reinterpret_cast<const float4*>(&xs[buf][dd][ty * TM]);
+            float wv[TE];
 #pragma unroll
-            for (int i = 0; i < TM; ++i) xv[i] = xs[dd][ty + i * NTY];
+            for (int j = 0; j < TE; ++j) wv[j] = wsm[buf][dd][tx + j * NTX];
 #pragma unroll
-            for (int j = 0; j < TE; ++j) wv[j] = wsm[dd][tx + j * NTX];
-#pragma unroll
-            for (int i = 0; i < TM; ++i)
-#pragma unroll
-                for (int j = 0; j < TE; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+            for (int j = 0; j < TE; ++j) {
+                acc[0][j] = fmaf(xv.x, wv[j], acc[0][j]);
+                acc[1][j] = fmaf(xv.y, wv[j], acc[1][j]);
+                acc[2][j] = fmaf(xv.z, wv[j], acc[2][j]);
+                acc[3][j] = fmaf(xv.w, wv[j], acc[3][j]);
+            }
         }
+        if (more) store(buf ^ 1);
         __syncthreads();
+        buf ^= 1;
     }
     float* out = part + (size_t)blockIdx.z * (size_t)T * E;
 #pragma unroll
     for (int i = 0; i < TM; ++i) {
-        int64_t t = t0 + ty + i * NTY;
+        const int64_t t = t0 + ty * TM + i;
         if (t >= T) continue;
 #pragma unroll
         for (int j = 0; j < TE; ++j) {
-            int e = e0 + tx + j * NTX;
+            const int e = e0 + tx + j * NTX;
             if (e < E) out[t * E + e] = acc[i][j];
         }
     }
@@ -143,7 +208,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     float z_acc = 0.f;
 
     const int64_t tbase = (int64_t)blockIdx.x * kTopkTPB;
-    for (int i = 0; i < kTopkTPB / 8; ++i) {
+    for (int i = 0; i < kTopkTPB / 8; ++i) {  // tokens warp, warp + 8, ...
         const int64_t t = tbase + warp + 8 * i;
         if (t >= T) break;
         float L[EPL];
@@ -273,12 +338,46 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     }
 }
 
-// One block: mean_prob[e] = (1/T) sum_b blk_mp[b][e]; losses = {z, balance}.
-// Cross-block sums in double, in block order.
-__global__ void __launch_bounds__(256) router_finalize_kernel(const float* __restrict__ blk_mp,
-                                                              const float* __restrict__ blk_z,
-                                                              const int32_t* __restrict__ blk_cnt,
-                                                              int nb, int64_t T, int E, int K,
+// Block e < E reduces column e of the per-block partials (mean probability in
+// double, counts in int64); block E reduces the z partials.  Fixed order:
+// strided per-thread sums, then a tree.
+__global__ void __launch_bounds__(256) router_colsum_kernel(const float* __restrict__ blk_mp,
+                                                            const float* __restrict__ blk_z,
+                                                            const int32_t* __restrict__ blk_cnt,
+                                                            int nb, int E, double* __restrict__ fin)
+{
+    __shared__ double s_a[256];
+    __shared__ long long s_c[256];
+    const int col = blockIdx.x;
+    double a = 0.0;
+    long long cn = 0;
+    for (int b = threadIdx.x; b < nb; b += 256) {
+        if (col < E) {
+            a += (double)blk_mp[(size_t)b * E + col];
+            cn += blk_cnt[(size_t)b * E + col];
+        } else {
+            a += (double)blk_z[b];
+        }
+    }
+    s_a[threadIdx.x] = a;
+    s_c[threadIdx.x] = cn;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (threadIdx.x < o) {
+            s_a[threadIdx.x] += s_a[threadIdx.x + o];
+            s_c[threadIdx.x] += s_c[threadIdx.x + o];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        fin[col] = s_a[0];                                   // sum of probabilities (or z)
+        if (col < E) fin[E + 1 + col] = (double)s_c[0];      // count (exact in double)
+    }
+}
+
+// mean_prob[e] = sum_p[e] / T; losses = {z, E * sum_e (count_e / (T*K)) * mean_prob[e]}.
+__global__ void __launch_bounds__(256) router_finalize_kernel(const double* __restrict__ fin,
+                                                              int64_t T, int E, int K,
                                                               float* __restrict__ mean_prob,
                                                               float* __restrict__ losses)
 {
@@ -286,15 +385,9 @@ __global__ void __launch_bounds__(256) router_finalize_kernel(const float* __res
     const int e = threadIdx.x;
     double term = 0.0;
     if (e < E) {
-        double mp = 0.0;
-        long long cn = 0;
-        for (int b = 0; b < nb; ++b) {
-            mp += (double)blk_mp[(size_t)b * E + e];
-            cn += blk_cnt[(size_t)b * E + e];
-        }
-        mp /= (double)T;
+        const double mp = fin[e] / (double)T;
         if (mean_prob) mean_prob[e] = (float)mp;
-        term = ((double)cn / ((double)T * (double)K)) * mp;
+        term = (fin[E + 1 + e] / ((double)T * (double)K)) * mp;
     }
     s_term[e] = term;
     __syncthreads();
@@ -303,9 +396,7 @@ __global__ void __launch_bounds__(256) router_finalize_kernel(const float* __res
         __syncthreads();
     }
     if (e == 0 && losses) {
-        double z = 0.0;
-        for (int b = 0; b < nb; ++b) z += (double)blk_z[b];
-        losses[0] = (float)(z / (double)T);
+        losses[0] = (float)(fin[E] / (double)T);
         losses[1] = (float)((double)E * s_term[0]);
     }
 }
@@ -317,7 +408,7 @@ static void launch_logits(const moe_config& c, const RouterPlan& rp, const XT* x
     dim3 grid(rp.grid_t, rp.grid_e, rp.splits);
     switch (rp.be) {
         case 8:
-            router_logits_kernel<XT, 8, 2, 1><<<grid, 256, 0, s>>>(x, w, part, c.T, c.D, c.E,
+            router_logits_kernel<XT, 8, 4, 1><<<grid, 256, 0, s>>>(x, w, part, c.T, c.D, c.E,
                                                                    rp.d_per_split);
             break;
         case 16:
@@ -375,9 +466,11 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
         default: MOE_TOPK(8); break;
     }
 #undef MOE_TOPK
-    if (with_stats)
-        router_finalize_kernel<<<1, 256, 0, s>>>(blk_mp, blk_z, blk_cnt, rp.nb_topk, c.T, c.E, c.K,
-                                                 mean_prob, losses);
+    if (with_stats) {
+        double* fin = reinterpret_cast<double*>(ws + L.r_fin);
+        router_colsum_kernel<<<c.E + 1, 256, 0, s>>>(blk_mp, blk_z, blk_cnt, rp.nb_topk, c.E, fin);
+        router_finalize_kernel<<<1, 256, 0, s>>>(fin, c.T, c.E, c.K, mean_prob, losses);
+    }
     return cudaGetLastError();
 }
 

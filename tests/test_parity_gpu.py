@@ -37,6 +37,10 @@ SMALL = [
     _wl("one_token", T=1, D=64, F=64, E=8, K=2, seed=8),
     _wl("top1", T=130, D=72, F=80, E=5, K=1, seed=9),
     _wl("one_expert", T=33, D=32, F=48, E=1, K=1, seed=10),
+    # CTA-pair tiles (256 rows): chosen when experts average >= 128 rows
+    _wl("pair_ragged", T=1200, D=200, F=392, E=4, K=2, seed=13),
+    _wl("pair_skewed", T=1500, D=128, F=136, E=8, K=2, bias="zipf", seed=14),
+    _wl("pair_drops", T=2000, D=64, F=256, E=8, K=2, capacity_factor=0.75, noise=True, seed=15),
 ]
 
 
