@@ -73,6 +73,14 @@ def barrier(world: int):
         dist.barrier()
 
 
+def aggregate(ms_total_local: float, world: int, T: int, steps: int, device) -> tuple:
+    """(ms per step, tokens/s of the whole job): the slowest rank's device time
+    over all ranks' tokens (each rank processes its own T tokens per step)."""
+    ms_total = max_over_ranks(ms_total_local, world, device)
+    ms_step = ms_total / steps
+    return ms_total, ms_step, world * T / (ms_step / 1e3)
+
+
 def rank_token_seed(rank: int) -> int:
     """Each replica routes its own batch of tokens (weights are shared)."""
     return 1000 + rank
@@ -226,10 +234,7 @@ def run_gpu(args):
     barrier(world)
     M.moe_trace_attach([])
     clk = clocks.stop()
-    ms_total = start.elapsed_time(stop)
-    ms_total = max_over_ranks(ms_total, world, dev)
-    ms_step = ms_total / args.steps
-    value = world * wl.T / (ms_step / 1e3)
+    ms_total, ms_step, value = aggregate(start.elapsed_time(stop), world, wl.T, args.steps, dev)
 
     names = M.trace_stage_names()
     stage_ms = {}
