@@ -35,9 +35,6 @@ from workloads import WORKLOADS, Workload, make_inputs, make_tokens  # noqa: E40
 METRIC = "routed tokens/s per MoE layer fwd on 1 B200; % bf16 tensor peak / % HBM BW"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# kernels this library launches per moe_forward (router 4, dispatch 3, gather 1,
-# expert GEMMs 2, combine 1)
-LAUNCHES_PER_STEP = 11
 
 
 # ------------------------------------------------------------------ ranks --
@@ -170,10 +167,15 @@ def algorithmic(wl: Workload, counts, kept_rows: int):
     }
 
 
-def kernel_source_hash() -> str:
+# sources that define the expert GEMM kernels (a recorded traffic figure is
+# only valid while these are unchanged)
+GEMM_SOURCES = ("ffn_tc.cu", "common.cuh", "internal.h")
+
+
+def kernel_source_hash(files=GEMM_SOURCES) -> str:
     csrc = os.path.join(ROOT, "mixture_experts_layer_55_b200", "csrc")
     h = hashlib.sha256()
-    for n in sorted(os.listdir(csrc)):
+    for n in sorted(files):
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(n.encode())
             h.update(f.read())
@@ -331,7 +333,7 @@ def run_gpu(args):
         "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": M.forward_kernel_count(layer.cfg) * args.steps,
         "roofline": roofline,
         "stages": stages,
         "layer": {"assignments_per_s": round(world * wl.T * wl.K / (ms_step / 1e3), 1),

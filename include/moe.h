@@ -260,6 +260,13 @@ MOE_API moe_status moe_get_device_status(const void *workspace, void *stream, in
 MOE_API moe_status moe_clear_device_status(void *workspace, void *stream);
 
 /*
+ * Number of kernels one moe_forward call launches for this configuration
+ * (router 4, plus 1 when its logits GEMM is split over d_model; dispatch 3;
+ * gather 1; expert GEMMs 2; combine 1).  0 for an invalid configuration.
+ */
+MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
+
+/*
  * Kernel-boundary tracing for timing.  After moe_trace_attach(events, n),
  * moe_forward records events[i] (cudaEvent_t values passed as void*) on its
  * stream at each of the first n stage boundaries: 0 before the first kernel,

@@ -75,6 +75,7 @@ _SIG = {
     "moe_forward": ([_P] * 15 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_get_device_status": ([_P, _P, _P], ctypes.c_int32),
     "moe_clear_device_status": ([_P, _P], ctypes.c_int32),
+    "moe_forward_kernel_count": ([_P], ctypes.c_int32),
     "moe_trace_attach": ([_P, ctypes.c_int32], ctypes.c_int32),
     "moe_trace_boundary_count": ([], ctypes.c_int32),
     "moe_trace_stage_name": ([ctypes.c_int32], ctypes.c_char_p),
@@ -235,6 +236,11 @@ def moe_get_device_status(workspace, stream=None) -> int:
 def moe_clear_device_status(workspace, stream=None):
     _check(lib().moe_clear_device_status(_ptr(workspace), _stream(stream)),
            "moe_clear_device_status")
+
+
+def forward_kernel_count(cfg: MoeConfig) -> int:
+    """Kernels one moe_forward launches for this configuration."""
+    return int(lib().moe_forward_kernel_count(_cfg(cfg)))
 
 
 def moe_trace_attach(events):

@@ -351,6 +351,12 @@ moe_status moe_clear_device_status(void* workspace, void* stream)
         cudaMemsetAsync(workspace, 0, 64 * sizeof(int), static_cast<cudaStream_t>(stream)));
 }
 
+int32_t moe_forward_kernel_count(const moe_config* cfg)
+{
+    if (check_config(cfg) != MOE_OK) return 0;
+    return 11 + (router_plan(*cfg).splits > 1 ? 1 : 0);
+}
+
 moe_status moe_trace_attach(void* const* events, int32_t n_events)
 {
     if (n_events < 0 || n_events > 16 || (n_events > 0 && events == nullptr)) return MOE_ERR_ARG;

@@ -9,8 +9,8 @@
 // Kernels:
 //   router_logits_kernel  tiled SIMT fp32 GEMM (T x D) * (D x E), optionally
 //                         split over d_model; partial sums go to scratch.
-//   router_topk_kernel    one warp per token: sums the split partials in a
-//                         fixed order, adds bias and noise, softmax, top-k by
+//   router_splitsum_kernel sums the d-split partials in split order.
+//   router_topk_kernel    one warp per token: adds bias and noise, softmax, top-k by
 //                         (logit desc, id asc) with warp shuffles, weights,
 //                         and per-block statistic partials.
 //   router_colsum_kernel  per-expert fixed-order reduction of the block partials.
@@ -175,6 +175,19 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict
             const int e = e0 + tx + j * NTX;
             if (e < E) out[t * E + e] = acc[i][j];
         }
+    }
+}
+
+// part[0][t][e] = sum over s of part[s][t][e] (in place, in split order), so
+// that the per-token kernel reads one value per logit.  One thread per logit.
+__global__ void __launch_bounds__(256) router_splitsum_kernel(float* __restrict__ part, int splits,
+                                                              int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float v = part[i];
+        for (int sp = 1; sp < splits; ++sp) v += part[(size_t)sp * n + i];
+        part[i] = v;
     }
 }
 
@@ -445,8 +458,14 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
             launch_logits(c, rp, static_cast<const __nv_bfloat16*>(x), w_router, p, s);
         else
             launch_logits(c, rp, static_cast<const float*>(x), w_router, p, s);
+        if (rp.splits > 1) {
+            const int64_t n = c.T * c.E;
+            int64_t blocks = (n + 255) / 256;
+            if (blocks > 148 * 16) blocks = 148 * 16;
+            router_splitsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rp.splits, n);
+        }
         part = p;
-        splits = rp.splits;
+        splits = 1;
     }
     const int with_stats = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
     float* blk_mp = reinterpret_cast<float*>(ws + L.r_mp);

@@ -117,6 +117,12 @@ def test_dispatch_ffn_combine_forward_argument_errors(lib):
                            None, None, FAKE, fb, None) == B.MOE_ERR_ARG
 
 
+def test_forward_kernel_count(lib):
+    assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 11
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 12  # split router
+    assert B.forward_kernel_count(_cfg(K=0)) == 0
+
+
 def test_status_strings_and_trace_table(lib):
     assert B.status_string(0) == "ok"
     assert "workspace" in B.status_string(B.MOE_ERR_WORKSPACE)
