@@ -260,9 +260,12 @@ MOE_API moe_status moe_get_device_status(const void *workspace, void *stream, in
 MOE_API moe_status moe_clear_device_status(void *workspace, void *stream);
 
 /*
- * Number of kernels one moe_forward call launches for this configuration
- * (router 4, plus 1 when its logits GEMM is split over d_model; dispatch 3;
- * gather 1; expert GEMMs 2; combine 1).  0 for an invalid configuration.
+ * Number of kernels one moe_forward call launches for this configuration:
+ * router 4 (bf16 with E <= 128 and T >= 2048: weight split, fused
+ * tensor-core router, two statistic reductions; otherwise logits GEMM, top-k,
+ * two statistic reductions, plus a split-sum when the GEMM is split over
+ * d_model), dispatch 3, gather 1, expert GEMMs 2, combine 1.  0 for an
+ * invalid configuration.
  */
 MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
 

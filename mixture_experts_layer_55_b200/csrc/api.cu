@@ -46,7 +46,10 @@ WsLayout ws_layout(const moe_config& c)
     L.status = o;
     o += align_up(64 * sizeof(int));
     L.r_part = o;
-    o += align_up((size_t)rp.splits * (size_t)c.T * c.E * sizeof(float));
+    size_t part_bytes = (size_t)rp.splits * (size_t)c.T * c.E * sizeof(float);
+    if (router_tc_eligible(c) && router_tc_wsplit_bytes(c) > part_bytes)
+        part_bytes = router_tc_wsplit_bytes(c);
+    o += align_up(part_bytes);
     L.r_mp = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(float));
     L.r_z = o;
@@ -354,6 +357,7 @@ moe_status moe_clear_device_status(void* workspace, void* stream)
 int32_t moe_forward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK) return 0;
+    if (router_tc_eligible(*cfg)) return 11;  // split weights, fused router, colsum, finalize
     return 11 + (router_plan(*cfg).splits > 1 ? 1 : 0);
 }
 

@@ -35,7 +35,8 @@ inline int64_t dispatch_chunks(const moe_config& c)
 // ------------------------------------------------------ workspace layout --
 struct WsLayout {
     size_t status;      // int32[64]
-    size_t r_part;      // splits * T * E fp32 partial logits
+    size_t r_part;      // splits * T * E fp32 partial logits, or the tensor-core
+                        // router's split weights (3 * D * EP bf16), whichever is larger
     size_t r_mp;        // nb_topk * E fp32
     size_t r_z;         // nb_topk fp32
     size_t r_cnt;       // nb_topk * E int32
@@ -56,6 +57,16 @@ FwdLayout fwd_layout(const moe_config& c, int64_t max_rows);
 
 int64_t capacity_of(const moe_config& c);
 int64_t max_rows_of(const moe_config& c);
+
+// Tensor-core router (router_tc.cu): bf16 layers with E <= 128 and T >= 2048.
+bool router_tc_eligible(const moe_config& c);
+int router_tc_blocks(const moe_config& c);
+size_t router_tc_wsplit_bytes(const moe_config& c);
+cudaError_t launch_router_tc(const moe_config& c, const void* x, const float* w_router,
+                             const float* bias, const float* noise, float* logits_out,
+                             float* probs_out, int32_t* ids, float* w, float* blk_mp, float* blk_z,
+                             int32_t* blk_cnt, int with_stats, void* wsplit_scratch, int* status,
+                             cudaStream_t s);
 
 // ---------------------------------------------------------------- launches --
 // Each returns cudaSuccess or the launch error.

@@ -445,6 +445,24 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
                           int32_t* ids, float* w, float* mean_prob, float* losses, char* ws,
                           const WsLayout& L, cudaStream_t s)
 {
+    const int with_stats0 = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
+    if (!logits_in && router_tc_eligible(c)) {
+        // bf16 layers with enough tokens: fused tensor-core router
+        float* blk_mp = reinterpret_cast<float*>(ws + L.r_mp);
+        float* blk_z = reinterpret_cast<float*>(ws + L.r_z);
+        int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
+        cudaError_t e = launch_router_tc(c, x, w_router, bias, noise, logits_out, probs_out, ids, w,
+                                         blk_mp, blk_z, blk_cnt, with_stats0, ws + L.r_part,
+                                         reinterpret_cast<int*>(ws + L.status), s);
+        if (e != cudaSuccess) return e;
+        if (with_stats0) {
+            double* fin = reinterpret_cast<double*>(ws + L.r_fin);
+            router_colsum_kernel<<<c.E + 1, 256, 0, s>>>(blk_mp, blk_z, blk_cnt, router_tc_blocks(c),
+                                                          c.E, fin);
+            router_finalize_kernel<<<1, 256, 0, s>>>(fin, c.T, c.E, c.K, mean_prob, losses);
+        }
+        return cudaGetLastError();
+    }
     const float* part;
     int splits;
     if (logits_in) {

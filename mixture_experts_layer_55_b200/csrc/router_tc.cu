@@ -1,0 +1,402 @@
+// router_tc.cu -- router for bf16 layers on the tensor cores: the logits GEMM,
+// softmax, top-k and renormalised weights fused in one kernel.
+//
+// "Lab: build a tiny MoE in PyTorch", section "Full implementation": fp32
+// router logits, softmax over the experts, top-k, weights divided by the sum
+// of the selected probabilities; the statistics (mean probability, counts,
+// logsumexp) feed the balance loss and the z-loss.
+//
+// fp32 logits on bf16 tensor cores: x is bf16 already, and each fp32 router
+// weight is split exactly into three bf16 terms w = hi + mid + lo (hi =
+// bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid): 3 x 8 significand
+// bits cover fp32's 24).  Every product x*part is exact in fp32, and the
+// three MMAs accumulate in fp32 in tensor memory, so the logits carry fp32
+// accumulation error only (no bf16 rounding of the weights).
+//
+//   router_wsplit_kernel  W_r (D, E) fp32 -> (3, D, EP) bf16, EP = E rounded
+//                         up to 64 (zero columns), N-major for TMA.
+//   router_tc_kernel      one CTA per 128 tokens: warp 0 TMA (x tile 128 x 64,
+//                         three 64 x EP weight tiles per stage), warp 1
+//                         tcgen05.mma M=128, N=EP, three per K step into one
+//                         accumulator; warps 2..5 own one token row each:
+//                         logits (+ bias + noise) staged in shared memory,
+//                         max, top-K by (logit desc, id asc) with an unrolled
+//                         insertion network, sum of exponentials, weights,
+//                         probabilities, and fixed-order per-CTA statistics.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace rtc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int BOX_BYTES = 64 * 64 * 2;     // 8 KB
+constexpr int NUM_THREADS = 192;
+
+template <int EPB> struct Geo {            // EPB = EP / 64 (1 or 2)
+    static constexpr int EP = 64 * EPB;
+    static constexpr int B_BYTES = 3 * EPB * BOX_BYTES;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 40 KB or 64 KB
+    static constexpr int STAGES = EPB == 1 ? 4 : 3;
+    static constexpr int TMEM_COLS = EP;                   // 64 or 128 (powers of two)
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+struct Misc {
+    uint64_t full[4];
+    uint64_t empty[4];
+    uint64_t tfull;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct Args {
+    const float* bias;        // E or null
+    const float* noise;       // T x E or null
+    float* logits_out;        // T x E or null
+    float* probs_out;         // T x E or null
+    int32_t* ids;             // T x K
+    float* wout;              // T x K
+    float* blk_mp;            // grid x E
+    float* blk_z;             // grid
+    int32_t* blk_cnt;         // grid x E
+    int64_t T;
+    int D, E, K;
+    int with_stats;
+    int* status;
+};
+
+__global__ void __launch_bounds__(256) router_wsplit_kernel(const float* __restrict__ w,
+                                                            __nv_bfloat16* __restrict__ out, int D,
+                                                            int E, int EP)
+{
+    const int64_t n = (int64_t)D * EP;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int d = (int)(i / EP), e = (int)(i % EP);
+        const float v = e < E ? w[(int64_t)d * E + e] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+        out[i] = hi;
+        out[n + i] = mid;
+        out[2 * n + i] = lo;
+    }
+}
+
+MOE_DEVICE void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int EPB>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const Args a)
+{
+    using G = Geo<EPB>;
+    constexpr int EP = G::EP, STAGES = G::STAGES, STAGE_BYTES = G::STAGE_BYTES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * BM;
+    const int num_kb = (a.D + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->empty[s], 1);
+        }
+        mbar_init(&m->tfull, 1);
+        m->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmX);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(&m->tmem_base, G::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = m->tmem_base;
+    volatile int* abort_flag = &m->abort_flag;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int last_phase[STAGES];
+        for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+        for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
+            uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
+            uint8_t* sB = sA + A_BYTES;
+            uint64_t* fb = &m->full[stage];
+            mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            const int k0 = kb * BK;
+            tma_load_2d(sA, &tmX, k0, (int32_t)t0, fb);
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int j = 0; j < EPB; ++j)
+                    tma_load_3d(sB + (p * EPB + j) * BOX_BYTES, &tmW, 64 * j, k0, p, fb);
+            last_phase[stage] = (int)phase;
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        for (int s = 0; s < STAGES; ++s)
+            if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = umma_idesc_bf16(BM, EP, 0, 1);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&m->full[stage], phase, a.status, 520, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t sA = smem_u32(stages + (size_t)stage * STAGE_BYTES);
+            const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const uint64_t bdesc =
+                        umma_desc_sw128(sB + p * EPB * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
+                    umma_f16_ss(tmem_base, adesc, bdesc, idesc, (kb | kk | p) != 0 ? 1u : 0u);
+                }
+            }
+            umma_commit(&m->empty[stage]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        umma_commit(&m->tfull);  // also the drain: every MMA done once it fires
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue: one token row per thread
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // row in tile = tensor-memory lane
+        const int64_t t = t0 + r;
+        const bool valid = t < a.T;
+        const int E = a.E, K = a.K;
+        // the pipeline buffers are free once the accumulator is complete
+        float* Ls = reinterpret_cast<float*>(stages);  // [BM][EP + 1] logits, then probabilities
+        constexpr int LDS = EP + 1;
+        const bool ok = mbar_wait(&m->tfull, 0, a.status, 530, abort_flag);
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+        float mx = -INFINITY;
+        float tv[8];
+        int ti[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            tv[k] = -INFINITY;
+            ti[k] = 0x7fffffff;
+        }
+        // pass 1: logits (+ bias + noise) to shared memory, max, top-K insertion
+#pragma unroll 1
+        for (int c = 0; c < EP / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int e = c * 32 + j;
+                float L = -INFINITY;
+                if (e < E && ok) {
+                    L = __uint_as_float(v[j]);
+                    if (a.bias) L += a.bias[e];
+                    if (a.noise && valid) L += a.noise[t * E + e];
+                    if (a.logits_out && valid) a.logits_out[t * E + e] = L;
+                }
+                Ls[r * LDS + e] = L;
+                mx = fmaxf(mx, L);
+                // insertion into the list ordered by (value desc, id asc); a
+                // displaced entry carried further down keeps that order too
+                float x = L;
+                int xi = e;
+                if (e < E) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const bool gt = x > tv[k] || (x == tv[k] && xi < ti[k]);
+                        const float nv = gt ? x : tv[k];
+                        const int ni = gt ? xi : ti[k];
+                        x = gt ? tv[k] : x;
+                        xi = gt ? ti[k] : xi;
+                        tv[k] = nv;
+                        ti[k] = ni;
+                    }
+                }
+            }
+        }
+        // pass 2: sum of exponentials; probabilities back into shared memory
+        float ssum = 0.f;
+        for (int e = 0; e < E; ++e) ssum += expf(Ls[r * LDS + e] - mx);
+        const float inv = 1.0f / ssum;
+        for (int e = 0; e < E; ++e) {
+            const float p = expf(Ls[r * LDS + e] - mx) * inv;
+            Ls[r * LDS + e] = p;
+            if (a.probs_out && valid) a.probs_out[t * E + e] = p;
+        }
+        // selected weights, renormalised in slot order
+        float psum = 0.f;
+        float pk[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            pk[k] = (k < K) ? expf(tv[k] - mx) * inv : 0.f;
+            psum += pk[k];
+        }
+        if (valid) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < K) {
+                    a.ids[t * K + k] = ti[k];
+                    a.wout[t * K + k] = pk[k] / psum;
+                }
+        }
+        if (a.with_stats) {
+            // per-CTA statistics in a fixed order: column sums over the rows
+            const float lse = mx + logf(ssum);
+            epi_sync();
+            // rows past T contribute nothing
+            if (!valid)
+                for (int e = 0; e < E; ++e) Ls[r * LDS + e] = 0.f;
+            int* sid = reinterpret_cast<int*>(Ls + BM * LDS);  // [BM][8]
+            float* sz = reinterpret_cast<float*>(sid + BM * 8);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sid[r * 8 + k] = (valid && k < K) ? ti[k] : -1;
+            sz[r] = valid ? lse * lse : 0.f;
+            epi_sync();
+            const int tid = threadIdx.x - 64;
+            for (int e = tid; e < E; e += 128) {
+                float sp = 0.f;
+                int cn = 0;
+                for (int rr = 0; rr < BM; ++rr) {
+                    sp += Ls[rr * LDS + e];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) cn += sid[rr * 8 + k] == e;
+                }
+                a.blk_mp[(size_t)blockIdx.x * E + e] = sp;
+                a.blk_cnt[(size_t)blockIdx.x * E + e] = cn;
+            }
+            if (tid == 0) {
+                float zs = 0.f;
+                for (int rr = 0; rr < BM; ++rr) zs += sz[rr];
+                a.blk_z[blockIdx.x] = zs;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, G::TMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encoder()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int EPB>
+static cudaError_t launch_t(const moe_config& c, const void* x, const __nv_bfloat16* wsplit,
+                            const Args& a, cudaStream_t s)
+{
+    using G = Geo<EPB>;
+    static int done_mask = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 31 || !((done_mask >> dev) & 1)) {
+        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EPB>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
+        if (e != cudaSuccess) return e;
+        if (dev < 31) done_mask |= 1 << dev;
+    }
+    EncodeTiledFn enc = encoder();
+    if (!enc) return cudaErrorInvalidValue;
+    CUtensorMap mX, mW;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)c.D, (cuuint64_t)c.T};
+        cuuint64_t strides[1] = {(cuuint64_t)c.D * 2};
+        cuuint32_t box[2] = {64, BM};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)G::EP, (cuuint64_t)c.D, 3};
+        cuuint64_t strides[2] = {(cuuint64_t)G::EP * 2, (cuuint64_t)G::EP * c.D * 2};
+        cuuint32_t box[3] = {64, 64, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&mW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(wsplit), dims,
+                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const unsigned grid = (unsigned)((c.T + BM - 1) / BM);
+    router_tc_kernel<EPB><<<grid, NUM_THREADS, G::SMEM, s>>>(mX, mW, a);
+    return cudaGetLastError();
+}
+
+}  // namespace rtc
+
+bool router_tc_eligible(const moe_config& c)
+{
+    return c.dtype == MOE_BF16 && c.E <= 128 && c.T >= 2048;
+}
+
+int router_tc_blocks(const moe_config& c) { return (int)((c.T + rtc::BM - 1) / rtc::BM); }
+
+size_t router_tc_wsplit_bytes(const moe_config& c)
+{
+    const int ep = (c.E + 63) / 64 * 64;
+    return (size_t)3 * c.D * ep * sizeof(__nv_bfloat16);
+}
+
+cudaError_t launch_router_tc(const moe_config& c, const void* x, const float* w_router,
+                             const float* bias, const float* noise, float* logits_out,
+                             float* probs_out, int32_t* ids, float* w, float* blk_mp, float* blk_z,
+                             int32_t* blk_cnt, int with_stats, void* wsplit_scratch, int* status,
+                             cudaStream_t s)
+{
+    using namespace rtc;
+    const int ep = (c.E + 63) / 64 * 64;
+    __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(wsplit_scratch);
+    const int64_t n = (int64_t)c.D * ep;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    router_wsplit_kernel<<<(unsigned)blocks, 256, 0, s>>>(w_router, wsplit, c.D, c.E, ep);
+    Args a{bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_cnt,
+           c.T, c.D, c.E, c.K, with_stats, status};
+    return ep == 64 ? launch_t<1>(c, x, wsplit, a, s) : launch_t<2>(c, x, wsplit, a, s);
+}
+
+}  // namespace moe

@@ -119,7 +119,8 @@ def test_dispatch_ffn_combine_forward_argument_errors(lib):
 
 def test_forward_kernel_count(lib):
     assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 11
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 12  # split router
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 11  # tensor-core router
+    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 12  # split SIMT router
     assert B.forward_kernel_count(_cfg(K=0)) == 0
 
 

@@ -41,6 +41,11 @@ SMALL = [
     _wl("pair_ragged", T=1200, D=200, F=392, E=4, K=2, seed=13),
     _wl("pair_skewed", T=1500, D=128, F=136, E=8, K=2, bias="zipf", seed=14),
     _wl("pair_drops", T=2000, D=64, F=256, E=8, K=2, capacity_factor=0.75, noise=True, seed=15),
+    # tensor-core router (bf16, E <= 128, T >= 2048): ragged 128-token tail, E not
+    # a multiple of 64, bias and noise, K = 8
+    _wl("tcr_ragged", T=2500, D=136, F=64, E=8, K=2, seed=16),
+    _wl("tcr_e100", T=2100, D=264, F=64, E=100, K=4, bias="zipf", noise=True, seed=17),
+    _wl("tcr_e128_k8", T=2048, D=128, F=32, E=128, K=8, seed=18),
 ]
 
 
@@ -98,6 +103,23 @@ def test_parity_mode_routes_given_logits(cuda_ok):
     b.run_ops(inp, logits_in=L.cuda())
     rt = check_routing(wl, b)
     assert (rt["ids"][:5] == np.arange(4)[None, :]).all()
+
+
+def test_tensor_core_router_ties(cuda_ok):
+    """Exact ties through the fused tensor-core router: a zero router weight and
+    a bias with repeated values; the lower expert id must win every tie."""
+    wl = _wl("tcr_ties", T=2048, D=64, F=32, E=16, K=5, seed=19)
+    inp_cpu = make_inputs(wl, device="cpu")
+    inp_cpu["w_router"] = torch.zeros_like(inp_cpu["w_router"])
+    inp_cpu["bias"] = torch.tensor([0., 1, 1, 0, 2, 1, 0, 2, 1, 0, 0, 2, 1, 1, 0, 2])
+    inp = _to_dev(inp_cpu)
+    b = Bufs(wl)
+    b.run_ops(inp)
+    rt = check_routing(wl, b)
+    # bias 2 at experts 4, 7, 11, 15; then bias 1 at 1, 2, 5, ...
+    assert (rt["ids"] == np.array([4, 7, 11, 15, 1])[None, :]).all()
+    np.testing.assert_array_equal(b.logits.cpu().numpy(), np.broadcast_to(
+        inp_cpu["bias"].numpy(), (wl.T, wl.E)))
 
 
 def test_determinism_bitwise(cuda_ok):
