@@ -249,19 +249,18 @@ def run_gpu(args):
     alg = algorithmic(wl, counts, kept_rows)
 
     # ---------------- end to end from pinned host memory (e2e) ----------------
-    x_host = xs[0].cpu().pin_memory()
-    y_host = torch.empty_like(x_host).pin_memory()
-    x_dev = torch.empty_like(xs[0])
-    y_dev = torch.empty_like(xs[0])
-    for _ in range(max(1, args.warmup)):
-        layer.forward_host(x_host, y_host, x_dev, y_dev, logit_noise=noise)
+    # every step copies its batch in from pinned host memory and its result out;
+    # copies of neighbouring steps overlap the forward (MoELayer.forward_host_stream)
+    x_hosts = [xs[i % nbuf].cpu().pin_memory() for i in range(nbuf)]
+    y_hosts = [torch.empty_like(x_hosts[0]).pin_memory() for _ in range(nbuf)]
+    seq_in = [x_hosts[i % nbuf] for i in range(args.steps)]
+    seq_out = [y_hosts[i % nbuf] for i in range(args.steps)]
+    layer.forward_host_stream(seq_in[:max(2, args.warmup)], seq_out[:max(2, args.warmup)],
+                              logit_noise=noise)
     torch.cuda.synchronize(dev)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        layer.forward_host(x_host, y_host, x_dev, y_dev, logit_noise=noise)
-    e1.record(stream)
+    layer.forward_host_stream(seq_in, seq_out, logit_noise=noise, events=(e0, e1))
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
@@ -332,7 +331,9 @@ def run_gpu(args):
                          f"{3 * wl.E * wl.D * wl.F * wl.elem_bytes / 1e9:.2f} GB read per step)"},
         "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io_bytes,
-                "d2h_bytes_per_step": io_bytes},
+                "d2h_bytes_per_step": io_bytes,
+                "how": "MoELayer.forward_host_stream: per step, x in from pinned host memory, "
+                       "moe_forward, y out; copies overlap neighbouring steps' forwards"},
         "gpu_launches": M.forward_kernel_count(layer.cfg) * args.steps,
         "roofline": roofline,
         "stages": stages,

@@ -260,6 +260,19 @@ MOE_API moe_status moe_get_device_status(const void *workspace, void *stream, in
 MOE_API moe_status moe_clear_device_status(void *workspace, void *stream);
 
 /*
+ * Self-test of the device-side failure path.  Launches one kernel whose only
+ * thread waits, with the library's bounded mbarrier wait and a limit of
+ * limit_ns (1 us .. 1 s), on a barrier that nothing arrives at.  The wait gives
+ * up, sets MOE_DEVFLAG_TIMEOUT (location code 900) in the workspace status
+ * word, writes 1 to workspace word 2, and the kernel returns normally: a
+ * following moe_get_device_status returns MOE_ERR_DEVICE_TIMEOUT and the CUDA
+ * context stays usable.  The workspace is any zeroed buffer of >= 256 bytes
+ * (256-byte aligned); clear it with moe_clear_device_status afterwards.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(void *workspace, size_t workspace_bytes,
+                                             int64_t limit_ns, void *stream);
+
+/*
  * Number of kernels one moe_forward call launches for this configuration:
  * router 4 (bf16 with E <= 128 and T >= 2048: weight split, fused
  * tensor-core router, two statistic reductions; otherwise logits GEMM, top-k,

@@ -76,6 +76,7 @@ _SIG = {
     "moe_get_device_status": ([_P, _P, _P], ctypes.c_int32),
     "moe_clear_device_status": ([_P, _P], ctypes.c_int32),
     "moe_forward_kernel_count": ([_P], ctypes.c_int32),
+    "moe_selftest_wait_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
     "moe_trace_attach": ([_P, ctypes.c_int32], ctypes.c_int32),
     "moe_trace_boundary_count": ([], ctypes.c_int32),
     "moe_trace_stage_name": ([ctypes.c_int32], ctypes.c_char_p),
@@ -236,6 +237,11 @@ def moe_get_device_status(workspace, stream=None) -> int:
 def moe_clear_device_status(workspace, stream=None):
     _check(lib().moe_clear_device_status(_ptr(workspace), _stream(stream)),
            "moe_clear_device_status")
+
+
+def moe_selftest_wait_timeout(workspace, limit_ns: int, stream=None):
+    _check(lib().moe_selftest_wait_timeout(_ptr(workspace), _nbytes(workspace), int(limit_ns),
+                                           _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def forward_kernel_count(cfg: MoeConfig) -> int:

@@ -119,10 +119,10 @@ MOE_DEVICE bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the timeout
-// flag) if the phase did not complete within kWaitLimitNs, or if *abort was
-// set by another role of the same CTA.
+// flag) if the phase did not complete within limit_ns (kWaitLimitNs by
+// default), or if *abort was set by another role of the same CTA.
 MOE_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where,
-                          volatile int* abort_flag)
+                          volatile int* abort_flag, uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
@@ -131,7 +131,7 @@ MOE_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where
         if (mbar_try_wait(bar, parity)) return true;
         if (((++spins) & 255u) == 0u) {
             if (abort_flag != nullptr && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 raise_flag(status, kFlagTimeout, where);
                 if (abort_flag != nullptr) *abort_flag = 1;
                 return false;

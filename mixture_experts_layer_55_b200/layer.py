@@ -63,3 +63,47 @@ class MoELayer:
             self.forward(x_dev, y_dev, logit_noise=logit_noise, stream=s)
             y_host.copy_(y_dev, non_blocking=True)
         return y_host
+
+    def forward_host_stream(self, x_hosts, y_hosts, logit_noise=None, nbuf: int = 2,
+                            events=None):
+        """The layer over a sequence of host batches, end to end and pipelined.
+
+        x_hosts / y_hosts: lists of pinned host tensors (T, D).  Three streams:
+        the copy in of batch i+1 and the copy out of batch i-1 overlap the
+        forward of batch i; device batches are double-buffered.  Returns the
+        copy-out stream (synchronise on it, or on `events` when given: a pair of
+        timing events recorded before the first copy in and after the last
+        copy out)."""
+        dev = self.device
+        comp = torch.cuda.current_stream(dev)
+        h2d = torch.cuda.Stream(dev)
+        d2h = torch.cuda.Stream(dev)
+        shape, dt = x_hosts[0].shape, x_hosts[0].dtype
+        xd = [torch.empty(shape, dtype=dt, device=dev) for _ in range(nbuf)]
+        yd = [torch.empty(shape, dtype=dt, device=dev) for _ in range(nbuf)]
+        ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_done = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+        if events is not None:
+            h2d.wait_stream(comp)
+            events[0].record(h2d)
+        for i, (xh, yh) in enumerate(zip(x_hosts, y_hosts)):
+            b = i % nbuf
+            with torch.cuda.stream(h2d):
+                if i >= nbuf:
+                    h2d.wait_event(ev_done[b])  # the forward of batch i-nbuf read xd[b]
+                xd[b].copy_(xh, non_blocking=True)
+                ev_in[b].record(h2d)
+            comp.wait_event(ev_in[b])
+            if i >= nbuf:
+                comp.wait_event(ev_out[b])      # the copy out of batch i-nbuf read yd[b]
+            self.forward(xd[b], yd[b], logit_noise=logit_noise, stream=comp)
+            ev_done[b].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_done[b])
+                yh.copy_(yd[b], non_blocking=True)
+                ev_out[b].record(d2h)
+        if events is not None:
+            events[1].record(d2h)
+        comp.wait_stream(d2h)
+        return d2h

@@ -117,6 +117,14 @@ def test_dispatch_ffn_combine_forward_argument_errors(lib):
                            None, None, FAKE, fb, None) == B.MOE_ERR_ARG
 
 
+def test_selftest_argument_errors(lib):
+    assert lib.moe_selftest_wait_timeout(None, 256, 10_000, None) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_wait_timeout(FAKE, 16, 10_000, None) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_wait_timeout(FAKE + 16, 256, 10_000, None) == B.MOE_ERR_ALIGN
+    assert lib.moe_selftest_wait_timeout(FAKE, 256, 10, None) == B.MOE_ERR_ARG
+    assert lib.moe_selftest_wait_timeout(FAKE, 256, 5_000_000_000, None) == B.MOE_ERR_ARG
+
+
 def test_forward_kernel_count(lib):
     assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 11
     assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 11  # tensor-core router

@@ -186,3 +186,39 @@ def test_full_size_layer(cuda_ok, name):
         assert rt["C"] == 2560
     del inp
     torch.cuda.empty_cache()
+
+
+def test_bounded_wait_gives_up_and_reports(cuda_ok):
+    """The device failure path: a wait on a barrier nothing arrives at gives up
+    after its limit (20 ms here), the status word reports the timeout and its
+    location, and the context keeps working (a layer forward runs after it)."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    B.moe_selftest_wait_timeout(ws, 20_000_000)
+    flags = B.moe_get_device_status(ws)
+    assert flags & 0x1
+    words = ws.view(torch.int32).cpu()
+    assert int(words[1]) == 900 and int(words[2]) == 1
+    B.moe_clear_device_status(ws)
+    assert B.moe_get_device_status(ws) == 0
+    wl = _wl("after_timeout", T=64, E=4, K=2, seed=21)
+    b = Bufs(wl)
+    b.run_ops(_to_dev(make_inputs(wl, device="cpu")))
+
+
+def test_host_stream_matches_device_forward(cuda_ok):
+    """MoELayer.forward_host_stream (pipelined copies in / forward / copies out)
+    returns, for every batch, the same bits as the device-resident forward."""
+    from mixture_experts_layer_55_b200 import MoELayer
+    from workloads import make_tokens
+    wl = _wl("host_stream", T=512, D=128, F=256, E=8, K=2, seed=22)
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    layer = MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K)
+    xs = [make_tokens(wl, seed=100 + i) for i in range(5)]
+    x_hosts = [x.pin_memory() for x in xs]
+    y_hosts = [torch.empty_like(x).pin_memory() for x in xs]
+    layer.forward_host_stream(x_hosts, y_hosts)
+    torch.cuda.synchronize()
+    for x, yh in zip(xs, y_hosts):
+        y = layer.forward(x.cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(y.cpu(), yh)
