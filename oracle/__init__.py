@@ -55,8 +55,10 @@ def _load():
             i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
             lib.oracle_router_logits.argtypes = [i64, i32, i32, P, i32, P, P, P, P]
             lib.oracle_router_logits.restype = None
-            lib.oracle_route.argtypes = [i64, i32, i32, P, P, P, P, P]
+            lib.oracle_route.argtypes = [i64, i32, i32, P, i32, i32, P, i32, i32, f64, P, P, P, P, P]
             lib.oracle_route.restype = i32
+            lib.oracle_update_bias.argtypes = [i32, P, f64, P]
+            lib.oracle_update_bias.restype = None
             lib.oracle_router_stats.argtypes = [i64, i32, i32, P, P, P, P, P, P, P]
             lib.oracle_router_stats.restype = None
             lib.oracle_capacity.argtypes = [i64, i32, i32, f64]
@@ -155,25 +157,51 @@ def router_logits(x, w_router, bias=None, noise=None) -> np.ndarray:
     return out
 
 
-def route(logits, K: int):
-    """Softmax, top-K on (logit desc, id asc) and renormalised weights.
+SCORE_FUNCS = {"softmax": 0, "sigmoid": 1}
+
+
+def route(logits, K: int, score_func: str = "softmax", renormalize: bool = True, sel_bias=None,
+          n_groups: int = 1, topk_groups: int = 1, route_scale: float = 1.0,
+          with_entropy: bool = False):
+    """Scores, (group-limited) top-K on (logit + selection bias desc, id asc),
+    and the weights of the selected experts.
 
     ``logits`` is (T, E), any real type (fp32 logits convert exactly).
-    Returns ids (T,K) int32, weights (T,K) f64, probs (T,E) f64, lse (T,) f64.
+    Returns ids (T,K) int32, weights (T,K) f64, probs (T,E) f64 (the scores
+    normalised per token), lse (T,) f64, and with ``with_entropy`` the
+    per-token entropy (T,) of the softmax probabilities.
     """
     lib = _load()
     L = _f64(logits)
     T, E = L.shape
     if not 1 <= K <= E:
         raise ValueError("top_k must be in [1, n_experts]")
+    if n_groups > 1 and (E % n_groups or not 1 <= topk_groups <= n_groups
+                         or topk_groups * (E // n_groups) < K):
+        raise ValueError("invalid expert groups")
+    b = None if sel_bias is None else _f64(sel_bias)
     ids = np.empty((T, K), dtype=np.int32)
     w = np.empty((T, K), dtype=np.float64)
     probs = np.empty((T, E), dtype=np.float64)
     lse = np.empty((T,), dtype=np.float64)
-    rc = lib.oracle_route(T, E, K, _ptr(L), _ptr(ids), _ptr(w), _ptr(probs), _ptr(lse))
+    ent = np.empty((T,), dtype=np.float64)
+    rc = lib.oracle_route(T, E, K, _ptr(L), SCORE_FUNCS[score_func], int(bool(renormalize)),
+                          _ptr(b), int(n_groups), int(topk_groups), float(route_scale), _ptr(ids),
+                          _ptr(w), _ptr(probs), _ptr(lse), _ptr(ent))
     if rc != 0:
         raise ValueError("non-finite router logit")
+    if with_entropy:
+        return ids, w, probs, lse, ent
     return ids, w, probs, lse
+
+
+def update_bias(bias, counts, gamma: float) -> np.ndarray:
+    """DeepSeek-V3 selection-bias step: b_e += gamma * sign(mean(counts) - counts_e)."""
+    lib = _load()
+    b = _f64(bias).copy()
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.int64))
+    lib.oracle_update_bias(b.shape[0], _ptr(c), float(gamma), _ptr(b))
+    return b
 
 
 def router_stats(ids, probs, lse, E: int):
@@ -258,20 +286,22 @@ def _expert_slice(w, e):
 
 
 def forward(x, w_router, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
-            bias=None, noise=None, logits=None) -> dict:
+            bias=None, noise=None, logits=None, **routing) -> dict:
     """The whole layer: route -> dispatch -> experts -> combine.
 
     When ``logits`` is given (T, E) the router GEMM is skipped and the layer is
     routed from those logits (parity mode: the CUDA path's fp32 logits).
-    Returns every intermediate: logits, ids, weights, probs, lse, counts,
-    mean_prob, z_loss, balance_loss, capacity, kept, offsets, perm, row_of,
-    o (unweighted expert outputs per row), row_weight (w per row), y.
+    ``routing`` passes the router options of ``route`` (score_func,
+    renormalize, sel_bias, n_groups, topk_groups, route_scale).
+    Returns every intermediate: logits, ids, weights, probs, lse, entropy,
+    counts, mean_prob, z_loss, balance_loss, capacity, kept, offsets, perm,
+    row_of, o (unweighted expert outputs per row), row_weight (w per row), y.
     """
     xa, _ = _elem_array(x)
     T, D = xa.shape
     E = _f32(w_router).shape[1]
     L = router_logits(x, w_router, bias, noise) if logits is None else _f64(logits)
-    ids, w, probs, lse = route(L, K)
+    ids, w, probs, lse, ent = route(L, K, with_entropy=True, **routing)
     counts64, mean_prob, z, bal = router_stats(ids, probs, lse, E)
     C = capacity(T, K, E, capacity_factor)
     dsp = dispatch(ids, E, C)
@@ -287,7 +317,8 @@ def forward(x, w_router, w_gate, w_up, w_down, K: int, capacity_factor: float = 
     wflat = w.reshape(-1)
     row_weight = wflat[perm] if R else np.zeros((0,), np.float64)
     y = combine(o, dsp["row_of"], w, T, K) if R else np.zeros((T, D), np.float64)
-    return dict(logits=L, ids=ids, weights=w, probs=probs, lse=lse, counts=dsp["counts"],
+    return dict(logits=L, ids=ids, weights=w, probs=probs, lse=lse, entropy=float(ent.mean()),
+                counts=dsp["counts"],
                 mean_prob=mean_prob, z_loss=z, balance_loss=bal, capacity=C, kept=dsp["kept"],
                 offsets=offsets, perm=perm, row_of=dsp["row_of"], x_perm=x_perm, o=o,
                 row_weight=row_weight, y=y)

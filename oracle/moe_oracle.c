@@ -71,30 +71,45 @@ void oracle_router_logits(int64_t T, int32_t D, int32_t E, const void *x, int32_
 }
 
 /*
- * Softmax over all E experts, top-K selection and renormalised weights,
- * [TinyMoE] "Full implementation" (softmax, topk, divide by the sum of the
- * selected) and [LLMBook] "The Router" (top-k-then-softmax gives the same
- * weights once renormalised).
+ * Routing of one token from its logits.  Sources: [TinyMoE] "Full
+ * implementation" (softmax, top-k, weights divided by the sum of the
+ * selected); [LLMBook] "The Router" (softmax-then-top-k keeps the selected
+ * probabilities as they are, without renormalisation) and "Exercises" 6
+ * (DeepSeek-V3 selection-only bias: top-k on h + b, gate weights from the
+ * unbiased logits over the chosen set); [TinyMoE] "Lab extensions" (sigmoid
+ * top-k, group-limited routing).
  *
- * Selection is made on the logits: expert a ranks before expert b iff
- * L[a] > L[b], or L[a] == L[b] and a < b.  Slot k holds the (k+1)-th expert in
- * that order.  Since softmax is monotone this is the same choice as ranking
- * the probabilities.
+ *   scores      softmax: p_e = exp(L_e - m) / sum_e' exp(L_e' - m)
+ *               sigmoid: s_e = 1 / (1 + exp(-L_e))
+ *   selection   u_e = L_e + sel_bias[e] (sel_bias may be NULL: u = L).
+ *               With n_groups > 1 the experts form n_groups contiguous
+ *               groups; a group's score is the largest u in it; the
+ *               topk_groups groups of largest score (ties: lower group id)
+ *               stay eligible, the others are excluded.  Then the K eligible
+ *               experts ordered by (u desc, id asc) fill slots 0..K-1.
+ *   weights     w_k = score[id_k] / sum_j score[id_j] when renormalize, else
+ *               score[id_k]; then times route_scale.
+ *   norm_scores (T, E): the scores normalised per token to sum to one (the
+ *               softmax probabilities themselves; sigmoid scores / their sum);
+ *               they feed the mean probability of the balance loss.
+ *   lse         m + log sum_e exp(L_e - m)            (the z-loss term)
+ *   entropy     -sum_e p_e log max(p_e, 1e-9) of the softmax probabilities
  *
- *     m    = max_e L[t,e]
- *     p_e  = exp(L_e - m) / sum_e' exp(L_e' - m)
- *     lse  = m + log sum_e exp(L_e - m)
- *     w_k  = p[id_k] / sum_j p[id_j]
- *
- * probs (T, E) may be NULL.  Returns 0, or -1 if a logit is not finite.
+ * norm_scores and entropy may be NULL.  Returns 0, or -1 if a logit is not
+ * finite.
  */
-int32_t oracle_route(int64_t T, int32_t E, int32_t K, const double *logits, int32_t *ids,
-                     double *weights, double *probs, double *lse)
+int32_t oracle_route(int64_t T, int32_t E, int32_t K, const double *logits, int32_t score_func,
+                     int32_t renormalize, const double *sel_bias, int32_t n_groups,
+                     int32_t topk_groups, double route_scale, int32_t *ids, double *weights,
+                     double *norm_scores, double *lse, double *entropy)
 {
     int32_t bad = 0;
 #pragma omp parallel for schedule(static) reduction(| : bad)
     for (int64_t t = 0; t < T; ++t) {
         const double *L = logits + t * E;
+        double *score = (double *)malloc(sizeof(double) * (size_t)E);
+        double *u = (double *)malloc(sizeof(double) * (size_t)E);
+        unsigned char *eligible = (unsigned char *)malloc((size_t)E);
         double m = L[0];
         for (int32_t e = 0; e < E; ++e) {
             if (!isfinite(L[e]))
@@ -107,32 +122,100 @@ int32_t oracle_route(int64_t T, int32_t E, int32_t K, const double *logits, int3
             s += exp(L[e] - m);
         if (lse)
             lse[t] = m + log(s);
-        if (probs)
+        if (entropy) {
+            double h = 0.0;
+            for (int32_t e = 0; e < E; ++e) {
+                double p = exp(L[e] - m) / s;
+                h -= p * log(p > 1e-9 ? p : 1e-9);
+            }
+            entropy[t] = h;
+        }
+        for (int32_t e = 0; e < E; ++e) {
+            score[e] = score_func == 1 ? 1.0 / (1.0 + exp(-L[e])) : exp(L[e] - m) / s;
+            u[e] = L[e] + (sel_bias ? sel_bias[e] : 0.0);
+            eligible[e] = 1;
+        }
+        if (norm_scores) {
+            double ss = 0.0;
             for (int32_t e = 0; e < E; ++e)
-                probs[t * E + e] = exp(L[e] - m) / s;
-
-        /* K passes, each picking the best expert not yet taken. */
+                ss += score[e];
+            for (int32_t e = 0; e < E; ++e)
+                norm_scores[t * E + e] = score[e] / ss;
+        }
+        if (n_groups > 1) {
+            int32_t gsize = E / n_groups;
+            unsigned char *keep = (unsigned char *)calloc((size_t)n_groups, 1);
+            for (int32_t r = 0; r < topk_groups; ++r) {
+                int32_t best = -1;
+                double bestv = 0.0;
+                for (int32_t g = 0; g < n_groups; ++g) {
+                    if (keep[g])
+                        continue;
+                    double gm = u[g * gsize];
+                    for (int32_t e = g * gsize; e < (g + 1) * gsize; ++e)
+                        if (u[e] > gm)
+                            gm = u[e];
+                    if (best < 0 || gm > bestv) { /* strict: lower group id on ties */
+                        best = g;
+                        bestv = gm;
+                    }
+                }
+                keep[best] = 1;
+            }
+            for (int32_t e = 0; e < E; ++e)
+                eligible[e] = keep[e / gsize];
+            free(keep);
+        }
+        /* K passes, each picking the best eligible expert not yet taken. */
         for (int32_t k = 0; k < K; ++k) {
             int32_t best = -1;
             for (int32_t e = 0; e < E; ++e) {
+                if (!eligible[e])
+                    continue;
                 int32_t taken = 0;
                 for (int32_t j = 0; j < k; ++j)
                     if (ids[t * K + j] == e)
                         taken = 1;
                 if (taken)
                     continue;
-                if (best < 0 || L[e] > L[best])
+                if (best < 0 || u[e] > u[best])
                     best = e; /* strict '>' keeps the lower id on ties */
             }
             ids[t * K + k] = best;
         }
         double sel = 0.0;
         for (int32_t k = 0; k < K; ++k)
-            sel += exp(L[ids[t * K + k]] - m) / s;
-        for (int32_t k = 0; k < K; ++k)
-            weights[t * K + k] = (exp(L[ids[t * K + k]] - m) / s) / sel;
+            sel += score[ids[t * K + k]];
+        for (int32_t k = 0; k < K; ++k) {
+            double w = score[ids[t * K + k]];
+            if (renormalize)
+                w = w / sel;
+            weights[t * K + k] = w * route_scale;
+        }
+        free(score);
+        free(u);
+        free(eligible);
     }
     return bad ? -1 : 0;
+}
+
+/*
+ * DeepSeek-V3 auxiliary-loss-free balancing, [LLMBook] "Exercises" 6
+ * (update_bias): b_e += gamma * sign(mean_e'(counts) - counts_e): overloaded
+ * experts get their selection bias lowered, underloaded ones raised, experts
+ * exactly at the mean keep theirs.
+ */
+void oracle_update_bias(int32_t E, const int64_t *counts, double gamma, double *bias)
+{
+    double mean = 0.0;
+    for (int32_t e = 0; e < E; ++e)
+        mean += (double)counts[e];
+    mean /= (double)E;
+    for (int32_t e = 0; e < E; ++e) {
+        double d = mean - (double)counts[e];
+        double sg = d > 0.0 ? 1.0 : (d < 0.0 ? -1.0 : 0.0);
+        bias[e] += gamma * sg;
+    }
 }
 
 /*
@@ -141,7 +224,7 @@ int32_t oracle_route(int64_t T, int32_t E, int32_t K, const double *logits, int3
  * loss":
  *     counts_e = #{(t,k) : ids[t,k] = e}          (before any capacity drop)
  *     f_e      = counts_e / (T*K)
- *     P_e      = (1/T) sum_t p[t,e]
+ *     P_e      = (1/T) sum_t p[t,e]   (p: the per-token normalised scores)
  *     balance  = E * sum_e f_e * P_e
  *     z        = (1/T) sum_t lse_t^2
  * The raw, unweighted values (the loss coefficients are the caller's).
