@@ -68,8 +68,14 @@ typedef enum moe_status {
 
 typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
-/* Router score function.  Only the softmax router of the sources is built. */
-typedef enum moe_score_func { MOE_SCORE_SOFTMAX = 0 } moe_score_func;
+/*
+ * Router score function: softmax over the experts ("Lab: build a tiny MoE in
+ * PyTorch", "Full implementation") or a per-expert sigmoid (the lab's
+ * extension "sigmoid top-k"; the NeMo Gate's score_func).  Either way the
+ * experts are selected on the logits (plus the selection bias), and the
+ * weights are the scores of the selected experts.
+ */
+typedef enum moe_score_func { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_func;
 
 /* Device status flags (bit set), as read by moe_get_device_status. */
 #define MOE_DEVFLAG_TIMEOUT 0x1
@@ -82,9 +88,15 @@ typedef struct moe_config {
     int32_t E;             /* number of experts, 1..256 */
     int32_t K;             /* experts per token (top-k), 1..min(E, 8) */
     float capacity_factor; /* <= 0: dropless; > 0: C = max(1, ceil(cf * T * K / E)) */
-    int32_t score_func;    /* moe_score_func; MOE_SCORE_SOFTMAX */
-    int32_t renormalize;   /* 1: selected weights renormalised to sum to one (only value) */
+    int32_t score_func;    /* moe_score_func */
+    int32_t renormalize;   /* 1: selected scores renormalised to sum to one (Mixtral);
+                              0: kept as they are (GShard / Switch softmax-then-top-k) */
     int32_t dtype;         /* moe_dtype */
+    int32_t n_groups;      /* 0 or 1: no group limit; else the experts form n_groups
+                              contiguous groups (E divisible by n_groups, <= 32) */
+    int32_t topk_groups;   /* groups a token may use, 1..n_groups, with
+                              topk_groups * E / n_groups >= K (ignored without groups) */
+    float route_scale;     /* multiplies every routing weight; > 0 (1 = none) */
 } moe_config;
 
 /* Returns a static, NUL-terminated description of a status code. */
@@ -130,29 +142,53 @@ MOE_API moe_status moe_forward_workspace_size(const moe_config *cfg, size_t *byt
  * "The Router" (noisy top-k gating adds noise to the logits before top-k).
  *
  *   L[t,e]  = sum_d x[t,d] W_r[d,e] + router_bias[e] + logit_noise[t,e]   (fp32)
- *   p[t,:]  = softmax(L[t,:])
- *   ids[t,:]= the K experts of largest L[t,e], ties to the lower id, in
+ *   s[t,e]  = softmax(L[t,:])_e, or sigmoid(L[t,e]) (score_func)
+ *   u[t,e]  = L[t,e] + selection_bias[e]   (selection only: DeepSeek-V3's
+ *             auxiliary-loss-free balancing, "2.9 Mixture-of-Experts (MoE)
+ *             Architectures", "Exercises" 6)
+ *   groups  with n_groups > 1: a group's score is its largest u; only the
+ *           topk_groups groups of largest score (ties: lower group id) are
+ *           eligible
+ *   ids[t,:]= the K eligible experts of largest u, ties to the lower id, in
  *             descending order
- *   w[t,k]  = p[t,ids[t,k]] / sum_j p[t,ids[t,j]]
+ *   w[t,k]  = route_scale * s[t,ids[t,k]] (/ sum_j s[t,ids[t,j]] when renormalize)
+ *   p[t,e]  = s[t,e] / sum_e' s[t,e']  (the softmax itself, or the normalised
+ *             sigmoid scores)
  *   mean_prob[e] = (1/T) sum_t p[t,e]
  *   losses[0] = z-loss = (1/T) sum_t (logsumexp_e L[t,e])^2
  *   losses[1] = balance = E * sum_e (counts_e / (T*K)) * mean_prob[e],
- *               counts_e = assignments to e before any capacity drop.
+ *               counts_e = assignments to e before any capacity drop
+ *   losses[2] = router entropy = (1/T) sum_t -sum_e q log max(q, 1e-9),
+ *               q = softmax(L[t,:])  ("Full implementation", stats)
  *
- * x (T, D) dtype; w_router (D, E) fp32.  router_bias (E) and logit_noise
- * (T, E) may be NULL.  logits_in (T, E), if not NULL, are taken as the
- * complete routing logits: x, w_router, bias and noise are then not read and
- * may be NULL.  logits_out (T, E) and probs_out (T, E) may be NULL.
+ * x (T, D) dtype; w_router (D, E) fp32.  router_bias (E), selection_bias (E)
+ * and logit_noise (T, E) may be NULL.  logits_in (T, E), if not NULL, are
+ * taken as the complete routing logits L: x, w_router, router_bias and noise
+ * are then not read and may be NULL (selection_bias still applies).
+ * logits_out (T, E) and probs_out (T, E, the p above) may be NULL.
  * topk_ids (T, K) and topk_w (T, K) are required.  mean_prob (E) and
- * losses (2) may be NULL; the statistics are then skipped.
+ * losses (3) may be NULL; the statistics are then skipped.
  * The reductions behind mean_prob and losses run in a fixed order
  * (deterministic run to run).
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router,
-                     const float *router_bias, const float *logit_noise, const float *logits_in,
+                     const float *router_bias, const float *selection_bias,
+                     const float *logit_noise, const float *logits_in,
                      float *logits_out, float *probs_out, int32_t *topk_ids, float *topk_w,
                      float *mean_prob, float *losses, void *workspace, size_t workspace_bytes,
                      void *stream);
+
+/*
+ * DeepSeek-V3 auxiliary-loss-free balancing step, "2.9 Mixture-of-Experts
+ * (MoE) Architectures", "Exercises" 6 (update_bias):
+ *   selection_bias[e] += gamma * sign(mean_e'(counts) - counts[e])
+ * so overloaded experts become less likely to be selected and underloaded
+ * ones more; an expert exactly at the mean keeps its bias.  counts (E, int32,
+ * e.g. from moe_dispatch or moe_forward) and selection_bias (E, fp32) are
+ * device arrays; updated in place on the stream.
+ */
+MOE_API moe_status moe_update_selection_bias(const moe_config *cfg, const int32_t *counts,
+                                             float gamma, float *selection_bias, void *stream);
 
 /*
  * Dispatch: per-expert histogram, capacity drop, exclusive-scan offsets and a
@@ -212,12 +248,13 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
 /*
  * The whole layer: moe_route -> moe_dispatch -> moe_expert_ffn -> moe_combine
  * on one stream, every intermediate in the workspace
- * (moe_forward_workspace_size bytes).  y (T, D) dtype is required; losses (2),
+ * (moe_forward_workspace_size bytes).  y (T, D) dtype is required; losses (3),
  * mean_prob (E), counts (E, before drops), topk_ids (T, K) and topk_w (T, K)
  * are optional copies of the routing results (NULL to skip).
  */
 MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *w_router,
-                       const float *router_bias, const float *logit_noise, const void *w_gate,
+                       const float *router_bias, const float *selection_bias,
+                       const float *logit_noise, const void *w_gate,
                        const void *w_up, const void *w_down, void *y, float *losses,
                        float *mean_prob, int32_t *counts, int32_t *topk_ids, float *topk_w,
                        void *workspace, size_t workspace_bytes, void *stream);

@@ -11,5 +11,6 @@ from ._binding import (  # noqa: F401
     MOE_BF16, MOE_F32, MoeConfig, MoEError, capacity, check_config, forward_kernel_count,
     forward_workspace_size, header_symbols, lib, max_rows, moe_clear_device_status, moe_combine,
     moe_dispatch, moe_dispatch_noalloc, moe_expert_ffn, moe_forward, moe_get_device_status,
-    moe_route, moe_selftest_wait_timeout, moe_trace_attach, status_string, trace_stage_names, workspace_size)
+    moe_route, moe_selftest_wait_timeout, moe_trace_attach, moe_update_selection_bias,
+    status_string, trace_stage_names, workspace_size)
 from .layer import MoELayer  # noqa: F401

@@ -27,6 +27,8 @@ MOE_ERR_WORKSPACE = -8
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_SCORE_SOFTMAX = 0
+MOE_SCORE_SIGMOID = 1
+SCORE_FUNCS = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}
 
 
 class MoEError(RuntimeError):
@@ -46,14 +48,18 @@ class MoeConfig(ctypes.Structure):
         ("score_func", ctypes.c_int32),
         ("renormalize", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
+        ("n_groups", ctypes.c_int32),
+        ("topk_groups", ctypes.c_int32),
+        ("route_scale", ctypes.c_float),
     ]
 
     @classmethod
-    def make(cls, T, D, F, E, K, dtype="bf16", capacity_factor=0.0, score_func=MOE_SCORE_SOFTMAX,
-             renormalize=1):
+    def make(cls, T, D, F, E, K, dtype="bf16", capacity_factor=0.0, score_func="softmax",
+             renormalize=True, n_groups=1, topk_groups=1, route_scale=1.0):
         dt = {"bf16": MOE_BF16, "f32": MOE_F32, MOE_BF16: MOE_BF16, MOE_F32: MOE_F32}[dtype]
-        return cls(int(T), int(D), int(F), int(E), int(K), float(capacity_factor), int(score_func),
-                   int(renormalize), dt)
+        sf = SCORE_FUNCS.get(score_func, score_func)
+        return cls(int(T), int(D), int(F), int(E), int(K), float(capacity_factor), int(sf),
+                   int(bool(renormalize)), dt, int(n_groups), int(topk_groups), float(route_scale))
 
 
 _lib = None
@@ -67,12 +73,13 @@ _SIG = {
     "moe_max_rows": ([_P, _P], ctypes.c_int32),
     "moe_workspace_size": ([_P, _P], ctypes.c_int32),
     "moe_forward_workspace_size": ([_P, _P], ctypes.c_int32),
-    "moe_route": ([_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_route": ([_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch_noalloc": ([_P] * 10, ctypes.c_int32),
     "moe_expert_ffn": ([_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([_P] * 5, ctypes.c_int32),
-    "moe_forward": ([_P] * 15 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_forward": ([_P] * 16 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_update_selection_bias": ([_P, _P, ctypes.c_float, _P, _P], ctypes.c_int32),
     "moe_get_device_status": ([_P, _P, _P], ctypes.c_int32),
     "moe_clear_device_status": ([_P, _P], ctypes.c_int32),
     "moe_forward_kernel_count": ([_P], ctypes.c_int32),
@@ -176,9 +183,10 @@ def forward_workspace_size(cfg: MoeConfig) -> int:
 
 def moe_route(cfg, x, w_router, topk_ids, topk_w, workspace, router_bias=None, logit_noise=None,
               logits_in=None, logits_out=None, probs_out=None, mean_prob=None, losses=None,
-              stream=None):
+              selection_bias=None, stream=None):
     st = lib().moe_route(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
-                         _ptr(logit_noise), _ptr(logits_in), _ptr(logits_out), _ptr(probs_out),
+                         _ptr(selection_bias), _ptr(logit_noise), _ptr(logits_in),
+                         _ptr(logits_out), _ptr(probs_out),
                          _ptr(topk_ids), _ptr(topk_w), _ptr(mean_prob), _ptr(losses),
                          _ptr(workspace), _nbytes(workspace), _stream(stream))
     _check(st, "moe_route")
@@ -217,12 +225,20 @@ def moe_combine(cfg, y_perm, row_of, y, stream=None):
 
 def moe_forward(cfg, x, w_router, w_gate, w_up, w_down, y, workspace, router_bias=None,
                 logit_noise=None, losses=None, mean_prob=None, counts=None, topk_ids=None,
-                topk_w=None, stream=None):
+                topk_w=None, selection_bias=None, stream=None):
     st = lib().moe_forward(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
-                           _ptr(logit_noise), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y),
+                           _ptr(selection_bias), _ptr(logit_noise), _ptr(w_gate), _ptr(w_up),
+                           _ptr(w_down), _ptr(y),
                            _ptr(losses), _ptr(mean_prob), _ptr(counts), _ptr(topk_ids),
                            _ptr(topk_w), _ptr(workspace), _nbytes(workspace), _stream(stream))
     _check(st, "moe_forward")
+
+
+def moe_update_selection_bias(cfg, counts, gamma: float, selection_bias, stream=None):
+    """selection_bias += gamma * sign(mean(counts) - counts), on the device."""
+    _check(lib().moe_update_selection_bias(_cfg(cfg), _ptr(counts), float(gamma),
+                                           _ptr(selection_bias), _stream(stream)),
+           "moe_update_selection_bias")
 
 
 def moe_get_device_status(workspace, stream=None) -> int:

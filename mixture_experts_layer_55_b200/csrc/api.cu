@@ -54,10 +54,12 @@ WsLayout ws_layout(const moe_config& c)
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(float));
     L.r_z = o;
     o += align_up((size_t)rp.nb_topk * sizeof(float));
+    L.r_ent = o;
+    o += align_up((size_t)rp.nb_topk * sizeof(float));
     L.r_cnt = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(int32_t));
     L.r_fin = o;
-    o += align_up((size_t)(2 * c.E + 1) * sizeof(double));
+    o += align_up((size_t)(2 * c.E + 2) * sizeof(double));
     L.d_cnt = o;
     o += align_up((size_t)nch * c.E * sizeof(int32_t));
     L.d_base = o;
@@ -81,7 +83,7 @@ FwdLayout fwd_layout(const moe_config& c, int64_t max_rows)
     F.perm = o;      o += align_up((size_t)max_rows * sizeof(int32_t));
     F.row_of = o;    o += align_up(tk * sizeof(int32_t));
     F.mean_prob = o; o += align_up((size_t)c.E * sizeof(float));
-    F.losses = o;    o += align_up(2 * sizeof(float));
+    F.losses = o;    o += align_up(3 * sizeof(float));
     F.x_perm = o;    o += align_up((size_t)max_rows * c.D * es);
     F.h = o;         o += align_up((size_t)max_rows * c.F * es);
     F.y_perm = o;    o += align_up((size_t)max_rows * c.D * es);
@@ -97,8 +99,16 @@ static moe_status check_config(const moe_config* c)
     if (c->K < 1 || c->K > c->E || c->K > 8) return MOE_ERR_ARG;
     if (c->T * (int64_t)c->K > (int64_t)INT32_MAX) return MOE_ERR_SHAPE;
     if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_ARG;
-    if (c->score_func != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
-    if (c->renormalize != 1) return MOE_ERR_UNSUPPORTED;
+    if (c->score_func != MOE_SCORE_SOFTMAX && c->score_func != MOE_SCORE_SIGMOID)
+        return MOE_ERR_UNSUPPORTED;
+    if (c->renormalize != 0 && c->renormalize != 1) return MOE_ERR_ARG;
+    if (c->n_groups < 0 || c->n_groups > 32) return MOE_ERR_ARG;
+    if (c->n_groups > 1) {
+        if (c->E % c->n_groups != 0) return MOE_ERR_ARG;
+        if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_ARG;
+        if ((int64_t)c->topk_groups * (c->E / c->n_groups) < c->K) return MOE_ERR_ARG;
+    }
+    if (!(c->route_scale > 0.0f) || !isfinite(c->route_scale)) return MOE_ERR_ARG;
     if (c->D % 8 != 0 || c->F % 8 != 0) return MOE_ERR_ALIGN;
     if (!isfinite(c->capacity_factor)) return MOE_ERR_ARG;
     return MOE_OK;
@@ -206,7 +216,8 @@ static moe_status check_ws(const moe_config* cfg, const void* ws, size_t bytes, 
 }
 
 moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router,
-                     const float* router_bias, const float* logit_noise, const float* logits_in,
+                     const float* router_bias, const float* selection_bias,
+                     const float* logit_noise, const float* logits_in,
                      float* logits_out, float* probs_out, int32_t* topk_ids, float* topk_w,
                      float* mean_prob, float* losses, void* workspace, size_t workspace_bytes,
                      void* stream)
@@ -221,7 +232,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router
     if (st != MOE_OK) return st;
     const RouterPlan rp = router_plan(*cfg);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return cuda_status(launch_router(*cfg, rp, x, w_router, router_bias, logit_noise, logits_in,
+    return cuda_status(launch_router(*cfg, rp, x, w_router, router_bias, selection_bias,
+                                     logit_noise, logits_in,
                                      logits_out, probs_out, topk_ids, topk_w, mean_prob, losses,
                                      static_cast<char*>(workspace), L, s));
 }
@@ -283,7 +295,8 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
 }
 
 moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
-                       const float* router_bias, const float* logit_noise, const void* w_gate,
+                       const float* router_bias, const float* selection_bias,
+                       const float* logit_noise, const void* w_gate,
                        const void* w_up, const void* w_down, void* y, float* losses,
                        float* mean_prob, int32_t* counts, int32_t* topk_ids, float* topk_w,
                        void* workspace, size_t workspace_bytes, void* stream)
@@ -315,8 +328,8 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
 
     trace(0, s);
     const RouterPlan rp = router_plan(c);
-    cudaError_t e = launch_router(c, rp, x, w_router, router_bias, logit_noise, nullptr, nullptr,
-                                  nullptr, ids, w, mean_prob, losses, ws, F.ws, s);
+    cudaError_t e = launch_router(c, rp, x, w_router, router_bias, selection_bias, logit_noise,
+                                  nullptr, nullptr, nullptr, ids, w, mean_prob, losses, ws, F.ws, s);
     trace(1, s);
     if (e == cudaSuccess)
         e = launch_dispatch_index(c, capacity_of(c), ids, cnt, kept, offsets, perm, row_of, ws,
@@ -331,6 +344,17 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
     if (e == cudaSuccess) e = launch_combine(c, y_perm, row_of, y, max_rows, s);
     trace(6, s);
     return cuda_status(e);
+}
+
+moe_status moe_update_selection_bias(const moe_config* cfg, const int32_t* counts, float gamma,
+                                     float* selection_bias, void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!counts || !selection_bias) return MOE_ERR_ARG;
+    if (!isfinite(gamma)) return MOE_ERR_ARG;
+    return cuda_status(launch_update_bias(cfg->E, counts, gamma, selection_bias,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_get_device_status(const void* workspace, void* stream, int32_t* flags)

@@ -25,6 +25,27 @@ struct RouterPlan {
 };
 RouterPlan router_plan(const moe_config& c);
 
+// Router options beyond the plain softmax / renormalised top-k.
+struct RouteOpts {
+    const float* sel_bias;  // E or null: added to the logits for selection only
+    int score_func;         // 0 softmax, 1 sigmoid
+    int renorm;             // 1: weights renormalised over the selected experts
+    int n_groups;           // <= 1: no group limit
+    int topk_groups;
+    float route_scale;
+};
+inline RouteOpts route_opts(const moe_config& c, const float* sel_bias)
+{
+    RouteOpts o;
+    o.sel_bias = sel_bias;
+    o.score_func = c.score_func;
+    o.renorm = c.renormalize;
+    o.n_groups = c.n_groups > 1 ? c.n_groups : 1;
+    o.topk_groups = c.n_groups > 1 ? c.topk_groups : 1;
+    o.route_scale = c.route_scale;
+    return o;
+}
+
 // ---------------------------------------------------------- dispatch plan --
 constexpr int kDispatchChunk = 2048;  // assignments per dispatch block
 inline int64_t dispatch_chunks(const moe_config& c)
@@ -39,8 +60,9 @@ struct WsLayout {
                         // router's split weights (3 * D * EP bf16), whichever is larger
     size_t r_mp;        // nb_topk * E fp32
     size_t r_z;         // nb_topk fp32
+    size_t r_ent;       // nb_topk fp32 (entropy partials)
     size_t r_cnt;       // nb_topk * E int32
-    size_t r_fin;       // (2E + 1) fp64: probability sums, z sum, counts
+    size_t r_fin;       // (2E + 2) fp64: probability sums, z sum, counts, entropy sum
     size_t d_cnt;       // chunks * E int32
     size_t d_base;      // chunks * E int32
     size_t total;
@@ -62,19 +84,23 @@ int64_t max_rows_of(const moe_config& c);
 bool router_tc_eligible(const moe_config& c);
 int router_tc_blocks(const moe_config& c);
 size_t router_tc_wsplit_bytes(const moe_config& c);
-cudaError_t launch_router_tc(const moe_config& c, const void* x, const float* w_router,
-                             const float* bias, const float* noise, float* logits_out,
-                             float* probs_out, int32_t* ids, float* w, float* blk_mp, float* blk_z,
-                             int32_t* blk_cnt, int with_stats, void* wsplit_scratch, int* status,
-                             cudaStream_t s);
+cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
+                             const float* w_router, const float* bias, const float* noise,
+                             float* logits_out, float* probs_out, int32_t* ids, float* w,
+                             float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
+                             int with_stats, void* wsplit_scratch, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- launches --
 // Each returns cudaSuccess or the launch error.
 cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void* x,
-                          const float* w_router, const float* bias, const float* noise,
+                          const float* w_router, const float* bias, const float* sel_bias,
+                          const float* noise,
                           const float* logits_in, float* logits_out, float* probs_out,
                           int32_t* ids, float* w, float* mean_prob, float* losses, char* ws,
                           const WsLayout& L, cudaStream_t s);
+
+cudaError_t launch_update_bias(int E, const int32_t* counts, float gamma, float* bias,
+                               cudaStream_t s);
 
 cudaError_t launch_dispatch_index(const moe_config& c, int64_t C, const int32_t* ids,
                                   int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* perm,

@@ -198,17 +198,22 @@ MOE_DEVICE bool ranks_before(float va, int ia, float vb, int ib)
 }
 
 // One warp per token.  Lane l holds experts l, l+32, ... (EPL of them).
+// Scores (softmax or sigmoid), the selection score u = L + selection bias,
+// optional group limit, top-K on (u desc, id asc), weights from the scores of
+// the selected experts (renormalised or not, times route_scale), and per-block
+// statistic partials (normalised scores, counts, lse^2, softmax entropy).
 template <int EPL>
 __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ part, int splits, const float* __restrict__ bias,
-    const float* __restrict__ noise, float* __restrict__ logits_out, float* __restrict__ probs_out,
-    int32_t* __restrict__ ids, float* __restrict__ wout, float* __restrict__ blk_mp,
-    float* __restrict__ blk_z, int32_t* __restrict__ blk_cnt, int64_t T, int E, int K,
-    int with_stats)
+    const float* __restrict__ noise, RouteOpts o, float* __restrict__ logits_out,
+    float* __restrict__ probs_out, int32_t* __restrict__ ids, float* __restrict__ wout,
+    float* __restrict__ blk_mp, float* __restrict__ blk_z, float* __restrict__ blk_ent,
+    int32_t* __restrict__ blk_cnt, int64_t T, int E, int K, int with_stats)
 {
     __shared__ float s_mp[8][256];
     __shared__ int s_cnt[8][256];
-    __shared__ float s_z[8];
+    __shared__ float s_u[8][256];  // a warp's selection scores, for group maxima
+    __shared__ float s_z[8], s_ent[8];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float mp_acc[EPL];
@@ -218,7 +223,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
         mp_acc[j] = 0.f;
         cnt_acc[j] = 0;
     }
-    float z_acc = 0.f;
+    float z_acc = 0.f, ent_acc = 0.f;
+    const int G = o.n_groups, gsz = E / G;
 
     const int64_t tbase = (int64_t)blockIdx.x * kTopkTPB;
     for (int i = 0; i < kTopkTPB / 8; ++i) {  // tokens warp, warp + 8, ...
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
             float v = -INFINITY;
             if (e < E) {
                 v = part[t * E + e];
-                for (int s = 1; s < splits; ++s) v += part[(size_t)s * T * E + t * E + e];
+                for (int sp = 1; sp < splits; ++sp) v += part[(size_t)sp * T * E + t * E + e];
                 if (bias) v += bias[e];
                 if (noise) v += noise[t * E + e];
                 if (logits_out) logits_out[t * E + e] = v;
@@ -242,7 +248,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
 #pragma unroll
         for (int j = 0; j < EPL; ++j) m = fmaxf(m, L[j]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         float ex[EPL];
         float ssum = 0.f;
 #pragma unroll
@@ -251,75 +257,130 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
             ssum += ex[j];
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+        for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
         const float inv = 1.0f / ssum;
-        float p[EPL];
+        // softmax probabilities q, scores sc, normalised scores pn
+        float q[EPL], sc[EPL];
+        float hpart = 0.f, scsum = 0.f;
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
-            p[j] = ex[j] * inv;
-            int e = lane + 32 * j;
+            q[j] = ex[j] * inv;
+            const bool in = lane + 32 * j < E;
+            if (in) hpart -= q[j] * logf(fmaxf(q[j], 1e-9f));
+            sc[j] = !in ? 0.f : (o.score_func == 1 ? 1.0f / (1.0f + expf(-L[j])) : q[j]);
+            scsum += sc[j];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            hpart += __shfl_xor_sync(0xffffffffu, hpart, off);
+            scsum += __shfl_xor_sync(0xffffffffu, scsum, off);
+        }
+        const float scinv = o.score_func == 1 ? 1.0f / scsum : 1.0f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
             if (e < E) {
-                if (probs_out) probs_out[t * E + e] = p[j];
-                mp_acc[j] += p[j];
+                const float pn = o.score_func == 1 ? sc[j] * scinv : q[j];
+                if (probs_out) probs_out[t * E + e] = pn;
+                mp_acc[j] += pn;
             }
         }
         if (lane == 0) {
-            float lse = m + logf(ssum);
+            const float lse = m + logf(ssum);
             z_acc = fmaf(lse, lse, z_acc);
+            ent_acc += hpart;
         }
-        // top-K: K rounds of a warp-wide arg-best over the not-yet-taken experts.
+        // selection scores and the group limit
+        float u[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            u[j] = (e < E) ? L[j] + (o.sel_bias ? o.sel_bias[e] : 0.f) : -INFINITY;
+        }
+        uint32_t elig = 0xffffffffu;  // bit j: expert lane + 32j may be selected
+        if (G > 1) {
+#pragma unroll
+            for (int j = 0; j < EPL; ++j)
+                if (lane + 32 * j < E) s_u[warp][lane + 32 * j] = u[j];
+            __syncwarp();
+            float gm = -INFINITY;  // lane g < G: its group's best selection score
+            if (lane < G)
+                for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) gm = fmaxf(gm, s_u[warp][e]);
+            uint32_t keep = 0;
+            for (int r = 0; r < o.topk_groups; ++r) {
+                float bv = (lane < G && !((keep >> lane) & 1u)) ? gm : -INFINITY;
+                int bi = (lane < G && !((keep >> lane) & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                    if (ranks_before(ov, oi, bv, bi)) {
+                        bv = ov;
+                        bi = oi;
+                    }
+                }
+                keep |= 1u << bi;
+            }
+            elig = 0;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j)
+                if (lane + 32 * j < E && ((keep >> ((lane + 32 * j) / gsz)) & 1u)) elig |= 1u << j;
+            __syncwarp();  // s_u is rewritten by the next token
+        }
+        // top-K: K rounds of a warp-wide arg-best over the eligible, not yet taken
         uint32_t taken = 0;  // bit j: expert lane+32j already selected
-        float sel_p[8];
+        float sel_s[8];
         int sel_id[8];
-        float psum = 0.f;
+        float ssel = 0.f;
         for (int k = 0; k < K; ++k) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
 #pragma unroll
             for (int j = 0; j < EPL; ++j) {
                 int e = lane + 32 * j;
-                if (e < E && !((taken >> j) & 1u) && ranks_before(L[j], e, bv, bi)) {
-                    bv = L[j];
+                if (e < E && ((elig >> j) & 1u) && !((taken >> j) & 1u) &&
+                    ranks_before(u[j], e, bv, bi)) {
+                    bv = u[j];
                     bi = e;
                 }
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            for (int off = 16; off > 0; off >>= 1) {
+                float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                int oi = __shfl_xor_sync(0xffffffffu, bi, off);
                 if (ranks_before(ov, oi, bv, bi)) {
                     bv = ov;
                     bi = oi;
                 }
             }
-            // the owner lane marks it taken and broadcasts its probability
-            float pk = 0.f;
+            // the owner lane marks it taken and broadcasts its score
+            float sk = 0.f;
             if ((bi & 31) == lane) {
                 int j = bi >> 5;
 #pragma unroll
                 for (int jj = 0; jj < EPL; ++jj)
                     if (jj == j) {
                         taken |= 1u << jj;
-                        pk = p[jj];
+                        sk = sc[jj];
                         cnt_acc[jj] += 1;
                     }
             }
-            pk = __shfl_sync(0xffffffffu, pk, bi & 31);
-            sel_p[k] = pk;
+            sk = __shfl_sync(0xffffffffu, sk, bi & 31);
+            sel_s[k] = sk;
             sel_id[k] = bi;
-            psum += pk;
+            ssel += sk;
         }
         if (lane < K) {
-            float pk = 0.f;
+            float sk = 0.f;
             int idk = 0;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 if (k == lane) {
-                    pk = sel_p[k];
+                    sk = sel_s[k];
                     idk = sel_id[k];
                 }
             ids[t * K + lane] = idk;
-            wout[t * K + lane] = pk / psum;
+            wout[t * K + lane] = (o.renorm ? sk / ssel : sk) * o.route_scale;
         }
     }
     if (!with_stats) return;
@@ -332,7 +393,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
             s_cnt[warp][e] = cnt_acc[j];
         }
     }
-    if (lane == 0) s_z[warp] = z_acc;
+    if (lane == 0) {
+        s_z[warp] = z_acc;
+        s_ent[warp] = ent_acc;
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         float a = 0.f;
@@ -345,17 +409,22 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
         blk_cnt[(size_t)blockIdx.x * E + e] = cn;
     }
     if (threadIdx.x == 0) {
-        float a = 0.f;
-        for (int wv = 0; wv < 8; ++wv) a += s_z[wv];
+        float a = 0.f, h = 0.f;
+        for (int wv = 0; wv < 8; ++wv) {
+            a += s_z[wv];
+            h += s_ent[wv];
+        }
         blk_z[blockIdx.x] = a;
+        blk_ent[blockIdx.x] = h;
     }
 }
 
-// Block e < E reduces column e of the per-block partials (mean probability in
-// double, counts in int64); block E reduces the z partials.  Fixed order:
-// strided per-thread sums, then a tree.
+// Block e < E reduces column e of the per-block partials (normalised scores in
+// double, counts in int64); block E reduces the z partials, block E + 1 the
+// entropy partials.  Fixed order: strided per-thread sums, then a tree.
 __global__ void __launch_bounds__(256) router_colsum_kernel(const float* __restrict__ blk_mp,
                                                             const float* __restrict__ blk_z,
+                                                            const float* __restrict__ blk_ent,
                                                             const int32_t* __restrict__ blk_cnt,
                                                             int nb, int E, double* __restrict__ fin)
 {
@@ -368,27 +437,35 @@ __global__ void __launch_bounds__(256) router_colsum_kernel(const float* __restr
         if (col < E) {
             a += (double)blk_mp[(size_t)b * E + col];
             cn += blk_cnt[(size_t)b * E + col];
-        } else {
+        } else if (col == E) {
             a += (double)blk_z[b];
+        } else {
+            a += (double)blk_ent[b];
         }
     }
     s_a[threadIdx.x] = a;
     s_c[threadIdx.x] = cn;
     __syncthreads();
-    for (int o = 128; o > 0; o >>= 1) {
-        if (threadIdx.x < o) {
-            s_a[threadIdx.x] += s_a[threadIdx.x + o];
-            s_c[threadIdx.x] += s_c[threadIdx.x + o];
+    for (int off = 128; off > 0; off >>= 1) {
+        if (threadIdx.x < off) {
+            s_a[threadIdx.x] += s_a[threadIdx.x + off];
+            s_c[threadIdx.x] += s_c[threadIdx.x + off];
         }
         __syncthreads();
     }
     if (threadIdx.x == 0) {
-        fin[col] = s_a[0];                                   // sum of probabilities (or z)
-        if (col < E) fin[E + 1 + col] = (double)s_c[0];      // count (exact in double)
+        if (col < E) {
+            fin[col] = s_a[0];                        // sum of normalised scores
+            fin[E + 1 + col] = (double)s_c[0];        // count (exact in double)
+        } else if (col == E) {
+            fin[E] = s_a[0];                          // sum of lse^2
+        } else {
+            fin[2 * E + 1] = s_a[0];                  // sum of entropies
+        }
     }
 }
 
-// mean_prob[e] = sum_p[e] / T; losses = {z, E * sum_e (count_e / (T*K)) * mean_prob[e]}.
+// mean_prob[e] = sum_p[e] / T; losses = {z, E * sum_e (count_e / (T*K)) * mean_prob[e], entropy}.
 __global__ void __launch_bounds__(256) router_finalize_kernel(const double* __restrict__ fin,
                                                               int64_t T, int E, int K,
                                                               float* __restrict__ mean_prob,
@@ -404,14 +481,40 @@ __global__ void __launch_bounds__(256) router_finalize_kernel(const double* __re
     }
     s_term[e] = term;
     __syncthreads();
-    for (int o = 128; o > 0; o >>= 1) {
-        if (e < o) s_term[e] += s_term[e + o];
+    for (int off = 128; off > 0; off >>= 1) {
+        if (e < off) s_term[e] += s_term[e + off];
         __syncthreads();
     }
     if (e == 0 && losses) {
         losses[0] = (float)(fin[E] / (double)T);
         losses[1] = (float)((double)E * s_term[0]);
+        losses[2] = (float)(fin[2 * E + 1] / (double)T);
     }
+}
+
+// DeepSeek-V3 selection-bias step: b[e] += gamma * sign(mean(counts) - counts[e]).
+__global__ void __launch_bounds__(256) update_bias_kernel(const int32_t* __restrict__ counts, int E,
+                                                          float gamma, float* __restrict__ b)
+{
+    __shared__ long long s_sum;
+    if (threadIdx.x == 0) {
+        long long sum = 0;
+        for (int e = 0; e < E; ++e) sum += counts[e];
+        s_sum = sum;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        // sign(sum/E - c) == sign(sum - c*E): exact in integers
+        const long long d = s_sum - (long long)counts[e] * E;
+        const float sg = d > 0 ? 1.0f : (d < 0 ? -1.0f : 0.0f);
+        b[e] += gamma * sg;
+    }
+}
+
+cudaError_t launch_update_bias(int E, const int32_t* counts, float gamma, float* bias, cudaStream_t s)
+{
+    update_bias_kernel<<<1, 256, 0, s>>>(counts, E, gamma, bias);
+    return cudaGetLastError();
 }
 
 template <typename XT>
@@ -440,72 +543,63 @@ static void launch_logits(const moe_config& c, const RouterPlan& rp, const XT* x
 }
 
 cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void* x,
-                          const float* w_router, const float* bias, const float* noise,
-                          const float* logits_in, float* logits_out, float* probs_out,
-                          int32_t* ids, float* w, float* mean_prob, float* losses, char* ws,
-                          const WsLayout& L, cudaStream_t s)
+                          const float* w_router, const float* bias, const float* sel_bias,
+                          const float* noise, const float* logits_in, float* logits_out,
+                          float* probs_out, int32_t* ids, float* w, float* mean_prob,
+                          float* losses, char* ws, const WsLayout& L, cudaStream_t s)
 {
-    const int with_stats0 = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
-    if (!logits_in && router_tc_eligible(c)) {
-        // bf16 layers with enough tokens: fused tensor-core router
-        float* blk_mp = reinterpret_cast<float*>(ws + L.r_mp);
-        float* blk_z = reinterpret_cast<float*>(ws + L.r_z);
-        int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
-        cudaError_t e = launch_router_tc(c, x, w_router, bias, noise, logits_out, probs_out, ids, w,
-                                         blk_mp, blk_z, blk_cnt, with_stats0, ws + L.r_part,
-                                         reinterpret_cast<int*>(ws + L.status), s);
-        if (e != cudaSuccess) return e;
-        if (with_stats0) {
-            double* fin = reinterpret_cast<double*>(ws + L.r_fin);
-            router_colsum_kernel<<<c.E + 1, 256, 0, s>>>(blk_mp, blk_z, blk_cnt, router_tc_blocks(c),
-                                                          c.E, fin);
-            router_finalize_kernel<<<1, 256, 0, s>>>(fin, c.T, c.E, c.K, mean_prob, losses);
-        }
-        return cudaGetLastError();
-    }
-    const float* part;
-    int splits;
-    if (logits_in) {
-        part = logits_in;
-        splits = 1;
-        bias = nullptr;
-        noise = nullptr;
-    } else {
-        float* p = reinterpret_cast<float*>(ws + L.r_part);
-        if (c.dtype == MOE_BF16)
-            launch_logits(c, rp, static_cast<const __nv_bfloat16*>(x), w_router, p, s);
-        else
-            launch_logits(c, rp, static_cast<const float*>(x), w_router, p, s);
-        if (rp.splits > 1) {
-            const int64_t n = c.T * c.E;
-            int64_t blocks = (n + 255) / 256;
-            if (blocks > 148 * 16) blocks = 148 * 16;
-            router_splitsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rp.splits, n);
-        }
-        part = p;
-        splits = 1;
-    }
+    const RouteOpts o = route_opts(c, sel_bias);
     const int with_stats = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
     float* blk_mp = reinterpret_cast<float*>(ws + L.r_mp);
     float* blk_z = reinterpret_cast<float*>(ws + L.r_z);
+    float* blk_ent = reinterpret_cast<float*>(ws + L.r_ent);
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
-    const int epl = (c.E + 31) / 32;
-    dim3 grid(rp.nb_topk);
-#define MOE_TOPK(N)                                                                              \
-    router_topk_kernel<N><<<grid, 256, 0, s>>>(part, splits, bias, noise, logits_out, probs_out, \
-                                               ids, w, blk_mp, blk_z, blk_cnt, c.T, c.E, c.K,   \
+    double* fin = reinterpret_cast<double*>(ws + L.r_fin);
+    int nb = rp.nb_topk;
+    if (!logits_in && router_tc_eligible(c)) {
+        // bf16 layers with enough tokens: fused tensor-core router
+        cudaError_t e = launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids,
+                                         w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats,
+                                         ws + L.r_part, reinterpret_cast<int*>(ws + L.status), s);
+        if (e != cudaSuccess) return e;
+        nb = router_tc_blocks(c);
+    } else {
+        const float* part;
+        if (logits_in) {
+            part = logits_in;
+            bias = nullptr;
+            noise = nullptr;
+        } else {
+            float* p = reinterpret_cast<float*>(ws + L.r_part);
+            if (c.dtype == MOE_BF16)
+                launch_logits(c, rp, static_cast<const __nv_bfloat16*>(x), w_router, p, s);
+            else
+                launch_logits(c, rp, static_cast<const float*>(x), w_router, p, s);
+            if (rp.splits > 1) {
+                const int64_t n = c.T * c.E;
+                int64_t blocks = (n + 255) / 256;
+                if (blocks > 148 * 16) blocks = 148 * 16;
+                router_splitsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rp.splits, n);
+            }
+            part = p;
+        }
+        const int epl = (c.E + 31) / 32;
+        dim3 grid(rp.nb_topk);
+#define MOE_TOPK(N)                                                                                \
+    router_topk_kernel<N><<<grid, 256, 0, s>>>(part, 1, bias, noise, o, logits_out, probs_out, ids, \
+                                               w, blk_mp, blk_z, blk_ent, blk_cnt, c.T, c.E, c.K,   \
                                                with_stats)
-    switch (epl) {
-        case 1: MOE_TOPK(1); break;
-        case 2: MOE_TOPK(2); break;
-        case 3:
-        case 4: MOE_TOPK(4); break;
-        default: MOE_TOPK(8); break;
-    }
+        switch (epl) {
+            case 1: MOE_TOPK(1); break;
+            case 2: MOE_TOPK(2); break;
+            case 3:
+            case 4: MOE_TOPK(4); break;
+            default: MOE_TOPK(8); break;
+        }
 #undef MOE_TOPK
+    }
     if (with_stats) {
-        double* fin = reinterpret_cast<double*>(ws + L.r_fin);
-        router_colsum_kernel<<<c.E + 1, 256, 0, s>>>(blk_mp, blk_z, blk_cnt, rp.nb_topk, c.E, fin);
+        router_colsum_kernel<<<c.E + 2, 256, 0, s>>>(blk_mp, blk_z, blk_ent, blk_cnt, nb, c.E, fin);
         router_finalize_kernel<<<1, 256, 0, s>>>(fin, c.T, c.E, c.K, mean_prob, losses);
     }
     return cudaGetLastError();

@@ -20,9 +20,11 @@
 //                         tcgen05.mma M=128, N=EP, three per K step into one
 //                         accumulator; warps 2..5 own one token row each:
 //                         logits (+ bias + noise) staged in shared memory,
-//                         max, top-K by (logit desc, id asc) with an unrolled
-//                         insertion network, sum of exponentials, weights,
-//                         probabilities, and fixed-order per-CTA statistics.
+//                         max, softmax sum, entropy, scores (softmax or
+//                         sigmoid), the group limit, top-K by (logit +
+//                         selection bias desc, id asc) with an unrolled
+//                         insertion network, weights, normalised scores, and
+//                         fixed-order per-CTA statistics.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -55,6 +57,7 @@ struct Misc {
 };
 
 struct Args {
+    RouteOpts o;
     const float* bias;        // E or null
     const float* noise;       // T x E or null
     float* logits_out;        // T x E or null
@@ -63,6 +66,7 @@ struct Args {
     float* wout;              // T x K
     float* blk_mp;            // grid x E
     float* blk_z;             // grid
+    float* blk_ent;           // grid
     int32_t* blk_cnt;         // grid x E
     int64_t T;
     int D, E, K;
@@ -190,21 +194,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int64_t t = t0 + r;
         const bool valid = t < a.T;
         const int E = a.E, K = a.K;
+        const RouteOpts& o = a.o;
         // the pipeline buffers are free once the accumulator is complete
-        float* Ls = reinterpret_cast<float*>(stages);  // [BM][EP + 1] logits, then probabilities
+        float* Ls = reinterpret_cast<float*>(stages);  // [BM][EP + 1] logits, then scores
         constexpr int LDS = EP + 1;
         const bool ok = mbar_wait(&m->tfull, 0, a.status, 530, abort_flag);
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+        // pass 1: logits (+ bias + noise) to shared memory and their maximum
         float mx = -INFINITY;
-        float tv[8];
-        int ti[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            tv[k] = -INFINITY;
-            ti[k] = 0x7fffffff;
-        }
-        // pass 1: logits (+ bias + noise) to shared memory, max, top-K insertion
 #pragma unroll 1
         for (int c = 0; c < EP / 32; ++c) {
             uint32_t v[32];
@@ -222,61 +220,107 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 Ls[r * LDS + e] = L;
                 mx = fmaxf(mx, L);
-                // insertion into the list ordered by (value desc, id asc); a
-                // displaced entry carried further down keeps that order too
-                float x = L;
-                int xi = e;
-                if (e < E) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const bool gt = x > tv[k] || (x == tv[k] && xi < ti[k]);
-                        const float nv = gt ? x : tv[k];
-                        const int ni = gt ? xi : ti[k];
-                        x = gt ? tv[k] : x;
-                        xi = gt ? ti[k] : xi;
-                        tv[k] = nv;
-                        ti[k] = ni;
-                    }
-                }
             }
         }
-        // pass 2: sum of exponentials; probabilities back into shared memory
+        // pass 2: softmax sum, entropy, score sum
         float ssum = 0.f;
         for (int e = 0; e < E; ++e) ssum += expf(Ls[r * LDS + e] - mx);
         const float inv = 1.0f / ssum;
+        float ent = 0.f, scsum = 0.f;
         for (int e = 0; e < E; ++e) {
-            const float p = expf(Ls[r * LDS + e] - mx) * inv;
-            Ls[r * LDS + e] = p;
-            if (a.probs_out && valid) a.probs_out[t * E + e] = p;
+            const float L = Ls[r * LDS + e];
+            const float q = expf(L - mx) * inv;
+            ent -= q * logf(fmaxf(q, 1e-9f));
+            scsum += o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : q;
         }
-        // selected weights, renormalised in slot order
-        float psum = 0.f;
-        float pk[8];
+        // group limit: a group's score is its best selection score u = L + b
+        uint32_t keep = 0xffffffffu;
+        const int G = o.n_groups, gsz = E / G;
+        if (G > 1) {
+            float gm[32];
+#pragma unroll
+            for (int g = 0; g < 32; ++g) {
+                gm[g] = -INFINITY;
+                if (g < G)
+                    for (int e = g * gsz; e < (g + 1) * gsz; ++e)
+                        gm[g] = fmaxf(gm[g], Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f));
+            }
+            keep = 0;
+            for (int rr = 0; rr < o.topk_groups; ++rr) {
+                float bv = -INFINITY;
+                int bg = 0;
+#pragma unroll
+                for (int g = 0; g < 32; ++g)
+                    if (g < G && !((keep >> g) & 1u) && gm[g] > bv) {  // strict: lower group id on ties
+                        bv = gm[g];
+                        bg = g;
+                    }
+                keep |= 1u << bg;
+            }
+        }
+        // pass 3: top-K over the eligible experts by (u desc, id asc), an unrolled
+        // insertion network (a displaced entry carried down keeps that order too)
+        float tv[8];
+        int ti[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            pk[k] = (k < K) ? expf(tv[k] - mx) * inv : 0.f;
-            psum += pk[k];
+            tv[k] = -INFINITY;
+            ti[k] = 0x7fffffff;
+        }
+        for (int e = 0; e < E; ++e) {
+            if (G > 1 && !((keep >> (e / gsz)) & 1u)) continue;
+            float x = Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f);
+            int xi = e;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const bool gt = x > tv[k] || (x == tv[k] && xi < ti[k]);
+                const float nv = gt ? x : tv[k];
+                const int ni = gt ? xi : ti[k];
+                x = gt ? tv[k] : x;
+                xi = gt ? ti[k] : xi;
+                tv[k] = nv;
+                ti[k] = ni;
+            }
+        }
+        // weights from the scores of the selected experts
+        float sk[8];
+        float ssel = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            sk[k] = 0.f;
+            if (k < K) {
+                const float L = Ls[r * LDS + ti[k]];
+                sk[k] = o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : expf(L - mx) * inv;
+            }
+            ssel += sk[k];
         }
         if (valid) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 if (k < K) {
                     a.ids[t * K + k] = ti[k];
-                    a.wout[t * K + k] = pk[k] / psum;
+                    a.wout[t * K + k] = (o.renorm ? sk[k] / ssel : sk[k]) * o.route_scale;
                 }
+        }
+        // pass 4: normalised scores into shared memory (and probs_out)
+        const float scinv = 1.0f / scsum;
+        for (int e = 0; e < E; ++e) {
+            const float L = Ls[r * LDS + e];
+            const float pn = (o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : expf(L - mx) * inv) *
+                             (o.score_func == 1 ? scinv : 1.0f);
+            Ls[r * LDS + e] = valid ? pn : 0.f;  // rows past T contribute nothing
+            if (a.probs_out && valid) a.probs_out[t * E + e] = pn;
         }
         if (a.with_stats) {
             // per-CTA statistics in a fixed order: column sums over the rows
             const float lse = mx + logf(ssum);
-            epi_sync();
-            // rows past T contribute nothing
-            if (!valid)
-                for (int e = 0; e < E; ++e) Ls[r * LDS + e] = 0.f;
             int* sid = reinterpret_cast<int*>(Ls + BM * LDS);  // [BM][8]
             float* sz = reinterpret_cast<float*>(sid + BM * 8);
+            float* sh = sz + BM;
 #pragma unroll
             for (int k = 0; k < 8; ++k) sid[r * 8 + k] = (valid && k < K) ? ti[k] : -1;
             sz[r] = valid ? lse * lse : 0.f;
+            sh[r] = valid ? ent : 0.f;
             epi_sync();
             const int tid = threadIdx.x - 64;
             for (int e = tid; e < E; e += 128) {
@@ -291,9 +335,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 a.blk_cnt[(size_t)blockIdx.x * E + e] = cn;
             }
             if (tid == 0) {
-                float zs = 0.f;
-                for (int rr = 0; rr < BM; ++rr) zs += sz[rr];
+                float zs = 0.f, hs = 0.f;
+                for (int rr = 0; rr < BM; ++rr) {
+                    zs += sz[rr];
+                    hs += sh[rr];
+                }
                 a.blk_z[blockIdx.x] = zs;
+                a.blk_ent[blockIdx.x] = hs;
             }
         }
     }
@@ -381,11 +429,11 @@ size_t router_tc_wsplit_bytes(const moe_config& c)
     return (size_t)3 * c.D * ep * sizeof(__nv_bfloat16);
 }
 
-cudaError_t launch_router_tc(const moe_config& c, const void* x, const float* w_router,
-                             const float* bias, const float* noise, float* logits_out,
-                             float* probs_out, int32_t* ids, float* w, float* blk_mp, float* blk_z,
-                             int32_t* blk_cnt, int with_stats, void* wsplit_scratch, int* status,
-                             cudaStream_t s)
+cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
+                             const float* w_router, const float* bias, const float* noise,
+                             float* logits_out, float* probs_out, int32_t* ids, float* w,
+                             float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
+                             int with_stats, void* wsplit_scratch, int* status, cudaStream_t s)
 {
     using namespace rtc;
     const int ep = (c.E + 63) / 64 * 64;
@@ -394,7 +442,7 @@ cudaError_t launch_router_tc(const moe_config& c, const void* x, const float* w_
     int64_t blocks = (n + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     router_wsplit_kernel<<<(unsigned)blocks, 256, 0, s>>>(w_router, wsplit, c.D, c.E, ep);
-    Args a{bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_cnt,
+    Args a{o, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt,
            c.T, c.D, c.E, c.K, with_stats, status};
     return ep == 64 ? launch_t<1>(c, x, wsplit, a, s) : launch_t<2>(c, x, wsplit, a, s);
 }

@@ -19,10 +19,14 @@ class MoELayer:
     """
 
     def __init__(self, T: int, w_router, w_gate, w_up, w_down, K: int, capacity_factor=0.0,
-                 router_bias=None):
+                 router_bias=None, selection_bias=None, **router_options):
+        """router_options: score_func ("softmax" | "sigmoid"), renormalize,
+        n_groups, topk_groups, route_scale (see moe_config in include/moe.h).
+        selection_bias (E) fp32: DeepSeek-V3 bias, for selection only."""
         E, D, F = w_gate.shape
         dtype = "bf16" if w_gate.dtype == torch.bfloat16 else "f32"
-        self.cfg = B.MoeConfig.make(T, D, F, E, K, dtype, capacity_factor)
+        self.cfg = B.MoeConfig.make(T, D, F, E, K, dtype, capacity_factor, **router_options)
+        self.selection_bias = selection_bias
         st = B.check_config(self.cfg)
         if st != B.MOE_OK:
             raise B.MoEError(st, "MoELayer")
@@ -32,18 +36,19 @@ class MoELayer:
         nbytes = B.forward_workspace_size(self.cfg)
         self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         self.torch_dtype = w_gate.dtype
-        self.losses = torch.zeros(2, dtype=torch.float32, device=self.device)
+        self.losses = torch.zeros(3, dtype=torch.float32, device=self.device)  # z, balance, entropy
         self.mean_prob = torch.zeros(E, dtype=torch.float32, device=self.device)
         self.counts = torch.zeros(E, dtype=torch.int32, device=self.device)
 
     def forward(self, x, y=None, logit_noise=None, stats: bool = True, stream=None):
         """y = MoE(x) for x (T, D) on the device; returns y.  With stats the
-        router's z-loss / balance loss, mean probabilities and counts are left in
+        router's z-loss / balance loss / entropy, mean probabilities and counts are left in
         self.losses, self.mean_prob and self.counts."""
         if y is None:
             y = torch.empty_like(x)
         B.moe_forward(self.cfg, x, self.w_router, self.w_gate, self.w_up, self.w_down, y,
                       self.workspace, router_bias=self.router_bias, logit_noise=logit_noise,
+                      selection_bias=self.selection_bias,
                       losses=self.losses if stats else None,
                       mean_prob=self.mean_prob if stats else None,
                       counts=self.counts if stats else None, stream=stream)
@@ -107,3 +112,9 @@ class MoELayer:
             events[1].record(d2h)
         comp.wait_stream(d2h)
         return d2h
+
+    def update_selection_bias(self, gamma: float, stream=None):
+        """One DeepSeek-V3 balancing step from the last forward's counts."""
+        if self.selection_bias is None:
+            raise ValueError("the layer has no selection bias")
+        B.moe_update_selection_bias(self.cfg, self.counts, gamma, self.selection_bias, stream=stream)

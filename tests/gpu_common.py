@@ -50,7 +50,8 @@ class Bufs:
 
     def __init__(self, wl: Workload, device="cuda"):
         self.wl = wl
-        self.cfg = B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K, wl.dtype, wl.capacity_factor)
+        self.cfg = B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K, wl.dtype, wl.capacity_factor,
+                                    **wl.routing())
         T, D, F, E, K = wl.T, wl.D, wl.F, wl.E, wl.K
         dt = wl.torch_dtype
         self.max_rows = B.max_rows(self.cfg)
@@ -62,7 +63,7 @@ class Bufs:
         self.ids = torch.empty(T, K, dtype=i32, device=device)
         self.w = torch.empty(T, K, dtype=f32, device=device)
         self.mean_prob = torch.empty(E, dtype=f32, device=device)
-        self.losses = torch.empty(2, dtype=f32, device=device)
+        self.losses = torch.empty(3, dtype=f32, device=device)
         self.counts = torch.empty(E, dtype=i32, device=device)
         self.kept = torch.empty(E, dtype=i32, device=device)
         self.offsets = torch.empty(E + 1, dtype=i32, device=device)
@@ -78,7 +79,8 @@ class Bufs:
         B.moe_route(c, inp["x"], inp["w_router"], self.ids, self.w, self.ws,
                     router_bias=inp["bias"], logit_noise=inp["noise"], logits_in=logits_in,
                     logits_out=self.logits if logits_in is None else None, probs_out=self.probs,
-                    mean_prob=self.mean_prob, losses=self.losses)
+                    mean_prob=self.mean_prob, losses=self.losses,
+                    selection_bias=inp.get("sel_bias"))
         if logits_in is not None:
             self.logits.copy_(logits_in)
         B.moe_dispatch(c, inp["x"], self.ids, self.counts, self.kept, self.offsets, self.perm,
@@ -109,10 +111,12 @@ def check_logits(wl, inp_cpu, logits_gpu):
     return float((err / np.maximum(mag, 1e-30)).max())
 
 
-def check_routing(wl, b: Bufs):
+def check_routing(wl, b: Bufs, sel_bias=None):
     """Everything the router and the dispatch index pass produce."""
     L = b.logits.cpu().numpy()
-    ids, w, probs, lse = oracle.route(L, wl.K)
+    sb = None if sel_bias is None else sel_bias.detach().cpu().numpy()
+    ids, w, probs, lse, ent = oracle.route(L, wl.K, sel_bias=sb, with_entropy=True,
+                                           **wl.routing())
     counts64, mp, z, bal = oracle.router_stats(ids, probs, lse, wl.E)
     np.testing.assert_array_equal(b.ids.cpu().numpy(), ids)
     np.testing.assert_allclose(b.w.cpu().numpy(), w, rtol=0, atol=1e-5)
@@ -121,6 +125,8 @@ def check_routing(wl, b: Bufs):
     lg = b.losses.cpu().numpy().astype(np.float64)
     assert abs(lg[0] - z) <= 1e-5 * abs(z) + 1e-7, (lg[0], z)
     assert abs(lg[1] - bal) <= 1e-5 * abs(bal) + 1e-7, (lg[1], bal)
+    h = float(ent.mean())
+    assert abs(lg[2] - h) <= 1e-5 * abs(h) + 1e-6, (lg[2], h)
     C = oracle.capacity(wl.T, wl.K, wl.E, wl.capacity_factor)
     assert C == B.capacity(b.cfg)
     d = oracle.dispatch(ids, wl.E, C)

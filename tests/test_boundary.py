@@ -41,9 +41,19 @@ def _cfg(**kw):
     (dict(D=100), B.MOE_ERR_ALIGN),         # 16-byte rows
     (dict(F=12), B.MOE_ERR_ALIGN),
     (dict(T=2**31, K=2), B.MOE_ERR_SHAPE),  # T*K beyond int32
-    (dict(score_func=1), B.MOE_ERR_UNSUPPORTED),
-    (dict(renormalize=0), B.MOE_ERR_UNSUPPORTED),
+    (dict(score_func="sigmoid"), B.MOE_OK),
+    (dict(renormalize=False), B.MOE_OK),
+    (dict(score_func=2), B.MOE_ERR_UNSUPPORTED),
+    (dict(renormalize=2), B.MOE_OK),            # make() maps any truthy value to 1
     (dict(capacity_factor=float("nan")), B.MOE_ERR_ARG),
+    (dict(n_groups=4, topk_groups=2), B.MOE_OK),  # E = 8: groups of 2, 4 eligible >= K
+    (dict(n_groups=3, topk_groups=1), B.MOE_ERR_ARG),   # E not divisible
+    (dict(n_groups=4, topk_groups=0), B.MOE_ERR_ARG),
+    (dict(n_groups=4, topk_groups=5), B.MOE_ERR_ARG),
+    (dict(n_groups=8, topk_groups=1), B.MOE_ERR_ARG),   # 1 eligible expert < K = 2
+    (dict(n_groups=33, topk_groups=1, E=66), B.MOE_ERR_ARG),
+    (dict(route_scale=0.0), B.MOE_ERR_ARG),
+    (dict(route_scale=float("inf")), B.MOE_ERR_ARG),
 ])
 def test_check_config(lib, kw, code):
     assert B.check_config(_cfg(**kw)) == code
@@ -76,8 +86,8 @@ FAKE = 0x10000  # an aligned address the library never dereferences here
 
 def _call_route(lib, cfg, x=FAKE, w=FAKE, ids=FAKE, tw=FAKE, ws=FAKE, nbytes=None):
     nb = B.workspace_size(cfg) if nbytes is None else nbytes
-    return lib.moe_route(ctypes.byref(cfg), x, w, None, None, None, None, None, ids, tw, None,
-                         None, ws, nb, None)
+    return lib.moe_route(ctypes.byref(cfg), x, w, None, None, None, None, None, None, ids, tw,
+                         None, None, ws, nb, None)
 
 
 def test_route_argument_errors(lib):
@@ -111,10 +121,13 @@ def test_dispatch_ffn_combine_forward_argument_errors(lib):
     assert lib.moe_combine(cr, FAKE, None, FAKE, None) == B.MOE_ERR_ARG
     assert lib.moe_combine(cr, FAKE, FAKE, FAKE + 8, None) == B.MOE_ERR_ALIGN
     fb = B.forward_workspace_size(c)
-    assert lib.moe_forward(cr, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                           None, None, FAKE, fb - 1, None) == B.MOE_ERR_WORKSPACE
-    assert lib.moe_forward(cr, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                           None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+    assert lib.moe_forward(cr, FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, None, None,
+                           None, None, None, FAKE, fb - 1, None) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(cr, FAKE, None, None, None, None, FAKE, FAKE, FAKE, FAKE, None, None,
+                           None, None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+    assert lib.moe_update_selection_bias(cr, None, ctypes.c_float(0.01), FAKE, None) == B.MOE_ERR_ARG
+    assert lib.moe_update_selection_bias(cr, FAKE, ctypes.c_float(float("nan")), FAKE,
+                                         None) == B.MOE_ERR_ARG
 
 
 def test_selftest_argument_errors(lib):

@@ -46,6 +46,17 @@ SMALL = [
     _wl("tcr_ragged", T=2500, D=136, F=64, E=8, K=2, seed=16),
     _wl("tcr_e100", T=2100, D=264, F=64, E=100, K=4, bias="zipf", noise=True, seed=17),
     _wl("tcr_e128_k8", T=2048, D=128, F=32, E=128, K=8, seed=18),
+    # router variants, SIMT router (T < 2048) and tensor-core router
+    _wl("sigmoid_simt", T=300, E=16, K=3, score_func="sigmoid", seed=23),
+    _wl("norenorm_scale_simt", T=300, E=8, K=2, renormalize=False, route_scale=2.5, seed=24),
+    _wl("selbias_groups_simt", T=500, D=128, F=64, E=64, K=6, sel_bias=True, n_groups=8,
+        topk_groups=3, seed=25),
+    _wl("e256_groups_sigmoid_simt", T=64, D=256, F=64, E=256, K=8, n_groups=8, topk_groups=4,
+        sel_bias=True, score_func="sigmoid", seed=26),
+    _wl("sigmoid_selbias_tcr", T=2300, D=128, F=32, E=32, K=4, score_func="sigmoid",
+        sel_bias=True, seed=27),
+    _wl("groups_norenorm_tcr", T=2048, D=128, F=32, E=128, K=8, n_groups=8, topk_groups=4,
+        renormalize=False, route_scale=1.5, bias="zipf", seed=28),
 ]
 
 
@@ -60,10 +71,12 @@ def test_small_layers_elementwise(cuda_ok, wl):
     b = Bufs(wl)
     b.run_ops(inp)
     check_logits(wl, inp_cpu, b.logits.cpu().numpy())
-    rt = check_routing(wl, b)
+    rt = check_routing(wl, b, inp_cpu["sel_bias"])
+    sb = None if inp_cpu["sel_bias"] is None else inp_cpu["sel_bias"].double().numpy()
     ref = oracle.forward(inp_cpu["x"], inp_cpu["w_router"], inp_cpu["w_gate"], inp_cpu["w_up"],
                          inp_cpu["w_down"], wl.K, wl.capacity_factor, inp_cpu["bias"],
-                         inp_cpu["noise"], logits=b.logits.cpu().numpy())
+                         inp_cpu["noise"], logits=b.logits.cpu().numpy(), sel_bias=sb,
+                         **wl.routing())
     R = int(ref["offsets"][-1])
     # dispatch gather: exact copies
     assert torch.equal(b.x_perm[:R].cpu().to(torch.float64),
@@ -79,11 +92,11 @@ def test_small_layers_elementwise(cuda_ok, wl):
     # the whole layer in one call gives the same bits as the op-by-op path
     ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
     y2 = torch.empty_like(b.y)
-    losses = torch.empty(2, device="cuda")
+    losses = torch.empty(3, device="cuda")
     counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
     B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y2,
                   ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses,
-                  counts=counts)
+                  counts=counts, selection_bias=inp["sel_bias"])
     torch.cuda.synchronize()
     assert torch.equal(y2, b.y)
     assert torch.equal(losses, b.losses)
@@ -120,6 +133,21 @@ def test_tensor_core_router_ties(cuda_ok):
     assert (rt["ids"] == np.array([4, 7, 11, 15, 1])[None, :]).all()
     np.testing.assert_array_equal(b.logits.cpu().numpy(), np.broadcast_to(
         inp_cpu["bias"].numpy(), (wl.T, wl.E)))
+
+
+def test_update_selection_bias_matches_oracle(cuda_ok):
+    """DeepSeek-V3 balancing step on the device against the oracle's update,
+    with one count exactly at the mean (its bias must not move)."""
+    wl = _wl("upd", T=64, E=8, K=2)
+    cfg = B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K)
+    counts = torch.tensor([40, 3, 16, 0, 16, 25, 12, 16], dtype=torch.int32)  # mean 16
+    bias0 = torch.linspace(-0.5, 0.5, 8, dtype=torch.float32)
+    b = bias0.cuda()
+    B.moe_update_selection_bias(cfg, counts.cuda(), 0.125, b)
+    torch.cuda.synchronize()
+    ref = oracle.update_bias(bias0.double().numpy(), counts.numpy(), 0.125)
+    np.testing.assert_allclose(b.cpu().double().numpy(), ref, rtol=0, atol=1e-7)
+    assert float(b[2]) == float(bias0[2])
 
 
 def test_determinism_bitwise(cuda_ok):
@@ -165,11 +193,11 @@ def test_full_size_layer(cuda_ok, name):
     inp = make_inputs(wl, device="cuda")
     b = Bufs(wl)
     b.run_ops(inp)
-    rt = check_routing(wl, b)
+    rt = check_routing(wl, b, inp["sel_bias"])
     # the benchmark's call: the whole layer through moe_forward
     ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
     y = torch.empty_like(b.y)
-    losses = torch.empty(2, device="cuda")
+    losses = torch.empty(3, device="cuda")
     B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y,
                   ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses)
     torch.cuda.synchronize()

@@ -39,6 +39,19 @@ class Workload:
     noise: bool = False           # logit noise of std 1/E from a second seed
     seed: int = 0
     w_std: float = 0.02
+    # router options (defaults: softmax, renormalised top-k)
+    score_func: str = "softmax"
+    renormalize: bool = True
+    n_groups: int = 1
+    topk_groups: int = 1
+    route_scale: float = 1.0
+    sel_bias: bool = False        # a seeded DeepSeek-V3 selection bias input
+
+    def routing(self) -> dict:
+        """Router options as keyword arguments (oracle.route / MoeConfig.make)."""
+        return dict(score_func=self.score_func, renormalize=self.renormalize,
+                    n_groups=self.n_groups, topk_groups=self.topk_groups,
+                    route_scale=self.route_scale)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -111,7 +124,8 @@ def make_inputs(wl: Workload | str, device="cpu", seed: int | None = None) -> di
     """Generate every input of one layer forward.
 
     Returns a dict with x (T,D), w_router (D,E) fp32, bias (E) fp32 or None,
-    noise (T,E) fp32 or None, w_gate (E,D,F), w_up (E,D,F), w_down (E,F,D).
+    noise (T,E) fp32 or None, w_gate (E,D,F), w_up (E,D,F), w_down (E,F,D),
+    sel_bias (E) fp32 or None (N(0, 0.5^2), generator seed + 2).
     Draw order (one generator, seeded): x, w_router, w_gate, w_up, w_down.
     """
     if isinstance(wl, str):
@@ -130,8 +144,11 @@ def make_inputs(wl: Workload | str, device="cpu", seed: int | None = None) -> di
     if wl.noise:
         g2 = _gen(device, seed + 1)
         noise = _randn((wl.T, wl.E), g2, device, 1.0 / wl.E, torch.float32)
+    sel_bias = None
+    if wl.sel_bias:
+        sel_bias = _randn((wl.E,), _gen(device, seed + 2), device, 0.5, torch.float32)
     return dict(x=x, w_router=w_router, bias=bias, noise=noise,
-                w_gate=w_gate, w_up=w_up, w_down=w_down)
+                w_gate=w_gate, w_up=w_up, w_down=w_down, sel_bias=sel_bias)
 
 
 def make_tokens(wl: Workload | str, device="cpu", seed: int = 1234) -> torch.Tensor:
