@@ -286,13 +286,16 @@ def _expert_slice(w, e):
 
 
 def forward(x, w_router, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
-            bias=None, noise=None, logits=None, **routing) -> dict:
+            bias=None, noise=None, logits=None, shared=None, **routing) -> dict:
     """The whole layer: route -> dispatch -> experts -> combine.
 
     When ``logits`` is given (T, E) the router GEMM is skipped and the layer is
     routed from those logits (parity mode: the CUDA path's fp32 logits).
     ``routing`` passes the router options of ``route`` (score_func,
     renormalize, sel_bias, n_groups, topk_groups, route_scale).
+    ``shared`` = (w_gate_s (D, Fs), w_up_s (D, Fs), w_down_s (Fs, D)) adds a
+    shared SwiGLU expert that every token passes through ("Lab: build a tiny
+    MoE in PyTorch", "Add a shared expert": routed + shared_expert(x)).
     Returns every intermediate: logits, ids, weights, probs, lse, entropy,
     counts, mean_prob, z_loss, balance_loss, capacity, kept, offsets, perm,
     row_of, o (unweighted expert outputs per row), row_weight (w per row), y.
@@ -317,11 +320,15 @@ def forward(x, w_router, w_gate, w_up, w_down, K: int, capacity_factor: float = 
     wflat = w.reshape(-1)
     row_weight = wflat[perm] if R else np.zeros((0,), np.float64)
     y = combine(o, dsp["row_of"], w, T, K) if R else np.zeros((T, D), np.float64)
+    y_shared = None
+    if shared is not None:
+        y_shared = expert_rows(_f64(x), shared[0], shared[1], shared[2])
+        y = y + y_shared
     return dict(logits=L, ids=ids, weights=w, probs=probs, lse=lse, entropy=float(ent.mean()),
                 counts=dsp["counts"],
                 mean_prob=mean_prob, z_loss=z, balance_loss=bal, capacity=C, kept=dsp["kept"],
                 offsets=offsets, perm=perm, row_of=dsp["row_of"], x_perm=x_perm, o=o,
-                row_weight=row_weight, y=y)
+                row_weight=row_weight, y_shared=y_shared, y=y)
 
 
 def slot_outputs(x_rows, slot_ids, slot_kept, get_expert) -> np.ndarray:

@@ -373,3 +373,19 @@ def test_parity_mode_uses_given_logits():
     ids, w, _, _ = oracle.route(L32.astype(np.float64), wl.K)
     assert (a["ids"] == ids).all()
     np.testing.assert_array_equal(a["weights"], w)
+
+
+def test_shared_expert_adds_a_dense_swiglu():
+    """"Add a shared expert": the layer with a shared expert equals the routed
+    layer plus one dense SwiGLU FFN over every token (torch fp64 matmuls)."""
+    wl = _wl(T=30, D=16, F=24, E=4, K=2, dtype="bf16", seed=31)
+    inp = make_inputs(wl)
+    g = torch.Generator().manual_seed(4)
+    Fs = 40
+    sh = tuple((torch.randn(*s, generator=g) * 0.05).to(torch.bfloat16)
+               for s in ((16, Fs), (16, Fs), (Fs, 16)))
+    a = _fwd(inp, wl)
+    b = _fwd(inp, wl, shared=sh)
+    dense = _swiglu_torch(inp["x"].double(), *sh)
+    np.testing.assert_allclose(b["y"] - a["y"], dense.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(b["y_shared"], dense.numpy(), rtol=0, atol=1e-12)
