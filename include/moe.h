@@ -97,6 +97,8 @@ typedef struct moe_config {
     int32_t topk_groups;   /* groups a token may use, 1..n_groups, with
                               topk_groups * E / n_groups >= K (ignored without groups) */
     float route_scale;     /* multiplies every routing weight; > 0 (1 = none) */
+    int32_t F_shared;      /* hidden size of a shared expert that every token passes
+                              through (0: none), multiple of 8 */
 } moe_config;
 
 /* Returns a static, NUL-terminated description of a status code. */
@@ -227,6 +229,8 @@ MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int3
  * tensor cores; fp32 runs in true fp32 (no TF32).
  * h is a caller-provided intermediate of max_rows x F elements.  offsets,
  * perm and topk_w are device arrays as produced by moe_dispatch / moe_route.
+ * perm and topk_w may both be NULL: every row then gets weight 1 (a shared
+ * expert: cfg with E = 1, K = 1, F = F_shared, x_perm = x, offsets = {0, T}).
  */
 MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
                           const int32_t *perm, const float *topk_w, const void *w_gate,
@@ -238,24 +242,31 @@ MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, con
  * "Full implementation" (index_add_ of weighted expert outputs) and "Add a
  * capacity limit" (an all-dropped token returns zero).
  *
- *   y[t, :] = sum over k = 0..K-1 with row_of[t*K+k] >= 0 of y_perm[row_of[t*K+k], :]
- * summed in slot order in fp32 and rounded once to dtype (deterministic; the
- * routing weight was applied by moe_expert_ffn).
+ *   y[t, :] = y_add[t, :] + sum over k = 0..K-1 with row_of[t*K+k] >= 0 of
+ *             y_perm[row_of[t*K+k], :]
+ * summed in fp32 (y_add first, then the slots in order) and rounded once to
+ * dtype (deterministic; the routing weight was applied by moe_expert_ffn).
+ * y_add (T, D) dtype may be NULL; it carries a shared expert's output ("Lab:
+ * build a tiny MoE in PyTorch", "Add a shared expert": routed + shared).
  */
-MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *row_of, void *y,
-                       void *stream);
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *row_of,
+                               const void *y_add, void *y, void *stream);
 
 /*
- * The whole layer: moe_route -> moe_dispatch -> moe_expert_ffn -> moe_combine
- * on one stream, every intermediate in the workspace
- * (moe_forward_workspace_size bytes).  y (T, D) dtype is required; losses (3),
+ * The whole layer: moe_route -> moe_dispatch -> moe_expert_ffn -> (shared
+ * expert) -> moe_combine on one stream, every intermediate in the workspace
+ * (moe_forward_workspace_size bytes).  With cfg->F_shared > 0,
+ * w_gate_shared / w_up_shared (D, F_shared) and w_down_shared (F_shared, D)
+ * are required and the shared SwiGLU expert's output over all tokens is
+ * added in the combine; otherwise they are ignored (may be NULL).  y (T, D) dtype is required; losses (3),
  * mean_prob (E), counts (E, before drops), topk_ids (T, K) and topk_w (T, K)
  * are optional copies of the routing results (NULL to skip).
  */
 MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *w_router,
                        const float *router_bias, const float *selection_bias,
                        const float *logit_noise, const void *w_gate,
-                       const void *w_up, const void *w_down, void *y, float *losses,
+                       const void *w_up, const void *w_down, const void *w_gate_shared,
+                       const void *w_up_shared, const void *w_down_shared, void *y, float *losses,
                        float *mean_prob, int32_t *counts, int32_t *topk_ids, float *topk_w,
                        void *workspace, size_t workspace_bytes, void *stream);
 
@@ -314,8 +325,9 @@ MOE_API moe_status moe_selftest_wait_timeout(void *workspace, size_t workspace_b
  * router 4 (bf16 with E <= 128 and T >= 2048: weight split, fused
  * tensor-core router, two statistic reductions; otherwise logits GEMM, top-k,
  * two statistic reductions, plus a split-sum when the GEMM is split over
- * d_model), dispatch 3, gather 1, expert GEMMs 2, combine 1.  0 for an
- * invalid configuration.
+ * d_model), dispatch 3, gather 1, expert GEMMs 2, shared expert 3 (when
+ * F_shared > 0: its row offsets and two GEMMs), combine 1.  0 for an invalid
+ * configuration.
  */
 MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
 
@@ -324,8 +336,9 @@ MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
  * moe_forward records events[i] (cudaEvent_t values passed as void*) on its
  * stream at each of the first n stage boundaries: 0 before the first kernel,
  * then after the router, the dispatch index pass, the gather, the gate/up
- * GEMM, the down GEMM and the combine (7 boundaries; moe_trace_stage_name
- * names the stage that ends at boundary i).  moe_trace_attach(NULL, 0)
+ * GEMM, the down GEMM, the shared expert (an empty stage without one) and the
+ * combine (8 boundaries; moe_trace_stage_name names the stage that ends at
+ * boundary i).  moe_trace_attach(NULL, 0)
  * detaches.  The table is process-wide and not thread-safe.
  */
 MOE_API moe_status moe_trace_attach(void *const *events, int32_t n_events);

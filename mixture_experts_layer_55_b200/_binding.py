@@ -51,15 +51,17 @@ class MoeConfig(ctypes.Structure):
         ("n_groups", ctypes.c_int32),
         ("topk_groups", ctypes.c_int32),
         ("route_scale", ctypes.c_float),
+        ("F_shared", ctypes.c_int32),
     ]
 
     @classmethod
     def make(cls, T, D, F, E, K, dtype="bf16", capacity_factor=0.0, score_func="softmax",
-             renormalize=True, n_groups=1, topk_groups=1, route_scale=1.0):
+             renormalize=True, n_groups=1, topk_groups=1, route_scale=1.0, F_shared=0):
         dt = {"bf16": MOE_BF16, "f32": MOE_F32, MOE_BF16: MOE_BF16, MOE_F32: MOE_F32}[dtype]
         sf = SCORE_FUNCS.get(score_func, score_func)
         return cls(int(T), int(D), int(F), int(E), int(K), float(capacity_factor), int(sf),
-                   int(bool(renormalize)), dt, int(n_groups), int(topk_groups), float(route_scale))
+                   int(bool(renormalize)), dt, int(n_groups), int(topk_groups), float(route_scale),
+                   int(F_shared))
 
 
 _lib = None
@@ -77,8 +79,8 @@ _SIG = {
     "moe_dispatch": ([_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch_noalloc": ([_P] * 10, ctypes.c_int32),
     "moe_expert_ffn": ([_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
-    "moe_combine": ([_P] * 5, ctypes.c_int32),
-    "moe_forward": ([_P] * 16 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_combine": ([_P] * 6, ctypes.c_int32),
+    "moe_forward": ([_P] * 19 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_update_selection_bias": ([_P, _P, ctypes.c_float, _P, _P], ctypes.c_int32),
     "moe_get_device_status": ([_P, _P, _P], ctypes.c_int32),
     "moe_clear_device_status": ([_P, _P], ctypes.c_int32),
@@ -218,17 +220,20 @@ def moe_expert_ffn(cfg, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h, 
     _check(st, "moe_expert_ffn")
 
 
-def moe_combine(cfg, y_perm, row_of, y, stream=None):
-    st = lib().moe_combine(_cfg(cfg), _ptr(y_perm), _ptr(row_of), _ptr(y), _stream(stream))
+def moe_combine(cfg, y_perm, row_of, y, y_add=None, stream=None):
+    st = lib().moe_combine(_cfg(cfg), _ptr(y_perm), _ptr(row_of), _ptr(y_add), _ptr(y),
+                           _stream(stream))
     _check(st, "moe_combine")
 
 
 def moe_forward(cfg, x, w_router, w_gate, w_up, w_down, y, workspace, router_bias=None,
                 logit_noise=None, losses=None, mean_prob=None, counts=None, topk_ids=None,
-                topk_w=None, selection_bias=None, stream=None):
+                topk_w=None, selection_bias=None, shared=None, stream=None):
+    """shared = (w_gate_s, w_up_s, w_down_s) when cfg.F_shared > 0."""
+    sg, su, sd = shared if shared is not None else (None, None, None)
     st = lib().moe_forward(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
                            _ptr(selection_bias), _ptr(logit_noise), _ptr(w_gate), _ptr(w_up),
-                           _ptr(w_down), _ptr(y),
+                           _ptr(w_down), _ptr(sg), _ptr(su), _ptr(sd), _ptr(y),
                            _ptr(losses), _ptr(mean_prob), _ptr(counts), _ptr(topk_ids),
                            _ptr(topk_w), _ptr(workspace), _nbytes(workspace), _stream(stream))
     _check(st, "moe_forward")

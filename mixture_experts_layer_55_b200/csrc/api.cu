@@ -87,6 +87,12 @@ FwdLayout fwd_layout(const moe_config& c, int64_t max_rows)
     F.x_perm = o;    o += align_up((size_t)max_rows * c.D * es);
     F.h = o;         o += align_up((size_t)max_rows * c.F * es);
     F.y_perm = o;    o += align_up((size_t)max_rows * c.D * es);
+    F.sh_offsets = o; F.sh_h = o; F.sh_y = o;
+    if (c.F_shared > 0) {
+        F.sh_offsets = o; o += align_up(2 * sizeof(int32_t));
+        F.sh_h = o;       o += align_up((size_t)c.T * c.F_shared * es);
+        F.sh_y = o;       o += align_up((size_t)c.T * c.D * es);
+    }
     F.total = o;
     return F;
 }
@@ -109,6 +115,8 @@ static moe_status check_config(const moe_config* c)
         if ((int64_t)c->topk_groups * (c->E / c->n_groups) < c->K) return MOE_ERR_ARG;
     }
     if (!(c->route_scale > 0.0f) || !isfinite(c->route_scale)) return MOE_ERR_ARG;
+    if (c->F_shared < 0) return MOE_ERR_SHAPE;
+    if (c->F_shared % 8 != 0) return MOE_ERR_ALIGN;
     if (c->D % 8 != 0 || c->F % 8 != 0) return MOE_ERR_ALIGN;
     if (!isfinite(c->capacity_factor)) return MOE_ERR_ARG;
     return MOE_OK;
@@ -121,8 +129,9 @@ static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK 
 // ------------------------------------------------------------- tracing --
 static void* g_trace[16];
 static int g_trace_n = 0;
-static const char* kStageNames[7] = {"start", "route", "dispatch_index", "gather",
-                                     "expert_gate_up", "expert_down", "combine"};
+static const char* kStageNames[8] = {"start",          "route",       "dispatch_index",
+                                     "gather",         "expert_gate_up", "expert_down",
+                                     "shared_expert",  "combine"};
 
 static void trace(int boundary, cudaStream_t s)
 {
@@ -131,6 +140,15 @@ static void trace(int boundary, cudaStream_t s)
 }
 
 static void trace_mid_ffn(void*, cudaStream_t s) { trace(4, s); }
+
+// offsets {0, n} of a single expert block covering n rows
+__global__ void set_row_range_kernel(int32_t* off, int32_t n)
+{
+    if (threadIdx.x == 0) {
+        off[0] = 0;
+        off[1] = n;
+    }
+}
 
 cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
@@ -268,8 +286,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
 {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
-    if (!x_perm || !offsets || !perm || !topk_w || !w_gate || !w_up || !w_down || !h || !y_perm)
-        return MOE_ERR_ARG;
+    if (!x_perm || !offsets || !w_gate || !w_up || !w_down || !h || !y_perm) return MOE_ERR_ARG;
+    if ((perm == nullptr) != (topk_w == nullptr)) return MOE_ERR_ARG;
     if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
         !aligned16(h) || !aligned16(y_perm))
         return MOE_ERR_ALIGN;
@@ -283,21 +301,22 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
                                          nullptr));
 }
 
-moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of, void* y,
-                       void* stream)
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of,
+                       const void* y_add, void* y, void* stream)
 {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (!y_perm || !row_of || !y) return MOE_ERR_ARG;
-    if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_ALIGN;
+    if (!aligned16(y_perm) || !aligned16(y) || (y_add && !aligned16(y_add))) return MOE_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return cuda_status(launch_combine(*cfg, y_perm, row_of, y, max_rows_of(*cfg), s));
+    return cuda_status(launch_combine(*cfg, y_perm, row_of, y_add, y, max_rows_of(*cfg), s));
 }
 
 moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
                        const float* router_bias, const float* selection_bias,
                        const float* logit_noise, const void* w_gate,
-                       const void* w_up, const void* w_down, void* y, float* losses,
+                       const void* w_up, const void* w_down, const void* w_gate_shared,
+                       const void* w_up_shared, const void* w_down_shared, void* y, float* losses,
                        float* mean_prob, int32_t* counts, int32_t* topk_ids, float* topk_w,
                        void* workspace, size_t workspace_bytes, void* stream)
 {
@@ -307,6 +326,11 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
     if (!aligned16(x) || !aligned16(y) || !aligned16(w_gate) || !aligned16(w_up) ||
         !aligned16(w_down))
         return MOE_ERR_ALIGN;
+    if (cfg->F_shared > 0) {
+        if (!w_gate_shared || !w_up_shared || !w_down_shared) return MOE_ERR_ARG;
+        if (!aligned16(w_gate_shared) || !aligned16(w_up_shared) || !aligned16(w_down_shared))
+            return MOE_ERR_ALIGN;
+    }
     const moe_config& c = *cfg;
     const int64_t max_rows = max_rows_of(c);
     const FwdLayout F = fwd_layout(c, max_rows);
@@ -341,8 +365,27 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
         e = launch_expert_ffn(c, max_rows, x_perm, offsets, perm, w, w_gate, w_up, w_down, h,
                               y_perm, status, s, trace_mid_ffn, nullptr);
     trace(5, s);
-    if (e == cudaSuccess) e = launch_combine(c, y_perm, row_of, y, max_rows, s);
+    const void* y_add = nullptr;
+    if (e == cudaSuccess && c.F_shared > 0) {
+        // the shared expert: one expert over every token, rows = x, weight 1
+        moe_config cs = c;
+        cs.E = 1;
+        cs.K = 1;
+        cs.F = c.F_shared;
+        cs.capacity_factor = 0.f;
+        cs.n_groups = 1;
+        int32_t* sh_off = reinterpret_cast<int32_t*>(ws + F.sh_offsets);
+        set_row_range_kernel<<<1, 32, 0, s>>>(sh_off, (int32_t)c.T);
+        e = cudaGetLastError();
+        if (e == cudaSuccess)
+            e = launch_expert_ffn(cs, c.T, x, sh_off, nullptr, nullptr, w_gate_shared, w_up_shared,
+                                  w_down_shared, ws + F.sh_h, ws + F.sh_y, status, s, nullptr,
+                                  nullptr);
+        y_add = ws + F.sh_y;
+    }
     trace(6, s);
+    if (e == cudaSuccess) e = launch_combine(c, y_perm, row_of, y_add, y, max_rows, s);
+    trace(7, s);
     return cuda_status(e);
 }
 
@@ -381,8 +424,9 @@ moe_status moe_clear_device_status(void* workspace, void* stream)
 int32_t moe_forward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK) return 0;
-    if (router_tc_eligible(*cfg)) return 11;  // split weights, fused router, colsum, finalize
-    return 11 + (router_plan(*cfg).splits > 1 ? 1 : 0);
+    const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
+    if (router_tc_eligible(*cfg)) return 11 + shared;  // split weights, fused router, 2 reductions
+    return 11 + shared + (router_plan(*cfg).splits > 1 ? 1 : 0);
 }
 
 moe_status moe_trace_attach(void* const* events, int32_t n_events)
@@ -393,11 +437,11 @@ moe_status moe_trace_attach(void* const* events, int32_t n_events)
     return MOE_OK;
 }
 
-int32_t moe_trace_boundary_count(void) { return 7; }
+int32_t moe_trace_boundary_count(void) { return 8; }
 
 const char* moe_trace_stage_name(int32_t boundary)
 {
-    if (boundary < 0 || boundary >= 7) return "";
+    if (boundary < 0 || boundary >= 8) return "";
     return kStageNames[boundary];
 }
 

@@ -3,7 +3,8 @@
 // "Lab: build a tiny MoE in PyTorch", section "Full implementation": every
 // (token, slot) adds its weighted expert output to the token's row
 // (index_add_); section "Add a capacity limit": a dropped assignment adds
-// nothing, so an all-dropped token gets zero.
+// nothing, so an all-dropped token gets zero; section "Add a shared expert":
+// a shared expert's output is added to the routed output.
 //
 // The routing weight is already applied by the down GEMM's epilogue, so the
 // combine is a plain gather-sum: 16-byte vector loads of the token's K rows of
@@ -56,6 +57,7 @@ template <> struct Vec<__nv_bfloat16> {
 template <typename ET, int KS>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ row_of,
+                                                      const uint4* __restrict__ y_add,
                                                       uint4* __restrict__ y, int64_t T, int K,
                                                       int64_t vec_per_row, int64_t max_rows)
 {
@@ -84,6 +86,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
             const int64_t i = base + (int64_t)u * G;
             if (i >= n) break;
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (y_add) Vec<ET>::add(acc, __ldg(y_add + i));  // shared expert output first
 #pragma unroll
             for (int k = 0; k < KS; ++k)
                 if (rows[u][k] >= 0) Vec<ET>::add(acc, vals[u][k]);  // slot order
@@ -94,23 +97,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 
 template <typename ET>
 static void launch_combine_t(const moe_config& c, int64_t blocks, const void* y_perm,
-                             const int32_t* row_of, void* y, int64_t vpr, int64_t max_rows,
-                             cudaStream_t s)
+                             const int32_t* row_of, const void* y_add, void* y, int64_t vpr,
+                             int64_t max_rows, cudaStream_t s)
 {
     const uint4* src = static_cast<const uint4*>(y_perm);
+    const uint4* add = static_cast<const uint4*>(y_add);
     uint4* dst = static_cast<uint4*>(y);
     if (c.K <= 1)
-        combine_kernel<ET, 1><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+        combine_kernel<ET, 1><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+                                                                max_rows);
     else if (c.K == 2)
-        combine_kernel<ET, 2><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+        combine_kernel<ET, 2><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+                                                                max_rows);
     else if (c.K <= 4)
-        combine_kernel<ET, 4><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+        combine_kernel<ET, 4><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+                                                                max_rows);
     else
-        combine_kernel<ET, 8><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, dst, c.T, c.K, vpr, max_rows);
+        combine_kernel<ET, 8><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+                                                                max_rows);
 }
 
 cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
-                           void* y, int64_t max_rows, cudaStream_t s)
+                           const void* y_add, void* y, int64_t max_rows, cudaStream_t s)
 {
     const int64_t row_bytes = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4);
     const int64_t vpr = row_bytes / 16;
@@ -123,9 +131,9 @@ cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (c.dtype == MOE_BF16)
-        launch_combine_t<__nv_bfloat16>(c, blocks, y_perm, row_of, y, vpr, max_rows, s);
+        launch_combine_t<__nv_bfloat16>(c, blocks, y_perm, row_of, y_add, y, vpr, max_rows, s);
     else
-        launch_combine_t<float>(c, blocks, y_perm, row_of, y, vpr, max_rows, s);
+        launch_combine_t<float>(c, blocks, y_perm, row_of, y_add, y, vpr, max_rows, s);
     return cudaGetLastError();
 }
 

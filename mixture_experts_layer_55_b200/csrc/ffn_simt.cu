@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A,
         const int64_t row = row0 + ty + 16 * i;
         if (row >= row_end) continue;
         float wr = 1.f;
-        if (!GATEUP) {
+        if (!GATEUP && perm != nullptr) {  // no perm: unit weights (a shared expert)
             const int32_t pa = perm[row];
             if (pa < 0 || pa >= nk) {
                 raise_flag(status, kFlagBounds, 301);

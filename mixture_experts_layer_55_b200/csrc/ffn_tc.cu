@@ -349,9 +349,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             } else {
                 float w = 0.f;
                 if (valid) {
-                    const int32_t pa = a.perm[row];
-                    if (pa >= 0 && (int64_t)pa < a.nk) w = a.topk_w[pa];
-                    else if (half == 0) raise_flag(a.status, kFlagBounds, 431);
+                    if (a.perm == nullptr) {
+                        w = 1.f;  // unit weights (a shared expert)
+                    } else {
+                        const int32_t pa = a.perm[row];
+                        if (pa >= 0 && (int64_t)pa < a.nk) w = a.topk_w[pa];
+                        else if (half == 0) raise_flag(a.status, kFlagBounds, 431);
+                    }
                 }
 #pragma unroll 1
                 for (int c = 4 * half; c < 4 * half + 4; ++c) {

@@ -73,6 +73,7 @@ struct FwdLayout {
     WsLayout ws;        // scratch at offset 0
     size_t ids, w, counts, kept, offsets, perm, row_of, mean_prob, losses;
     size_t x_perm, h, y_perm;
+    size_t sh_offsets, sh_h, sh_y;  // shared expert (when F_shared > 0)
     size_t total;
 };
 FwdLayout fwd_layout(const moe_config& c, int64_t max_rows);
@@ -110,7 +111,7 @@ cudaError_t launch_gather(const moe_config& c, const void* x, const int32_t* row
                           int64_t max_rows, int* status, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
-                           void* y, int64_t max_rows, cudaStream_t s);
+                           const void* y_add, void* y, int64_t max_rows, cudaStream_t s);
 
 // Expert FFN: gate/up (+SwiGLU) into h, then down (+routing weight) into y_perm.
 // The stage boundary between the two GEMMs is reported through `mid` (may be

@@ -19,13 +19,18 @@ class MoELayer:
     """
 
     def __init__(self, T: int, w_router, w_gate, w_up, w_down, K: int, capacity_factor=0.0,
-                 router_bias=None, selection_bias=None, **router_options):
+                 router_bias=None, selection_bias=None, shared=None, **router_options):
         """router_options: score_func ("softmax" | "sigmoid"), renormalize,
         n_groups, topk_groups, route_scale (see moe_config in include/moe.h).
-        selection_bias (E) fp32: DeepSeek-V3 bias, for selection only."""
+        selection_bias (E) fp32: DeepSeek-V3 bias, for selection only.
+        shared: (w_gate_s (D, Fs), w_up_s (D, Fs), w_down_s (Fs, D)), a shared
+        expert every token passes through."""
         E, D, F = w_gate.shape
         dtype = "bf16" if w_gate.dtype == torch.bfloat16 else "f32"
-        self.cfg = B.MoeConfig.make(T, D, F, E, K, dtype, capacity_factor, **router_options)
+        fs = 0 if shared is None else shared[0].shape[1]
+        self.cfg = B.MoeConfig.make(T, D, F, E, K, dtype, capacity_factor, F_shared=fs,
+                                    **router_options)
+        self.shared = shared
         self.selection_bias = selection_bias
         st = B.check_config(self.cfg)
         if st != B.MOE_OK:
@@ -48,7 +53,7 @@ class MoELayer:
             y = torch.empty_like(x)
         B.moe_forward(self.cfg, x, self.w_router, self.w_gate, self.w_up, self.w_down, y,
                       self.workspace, router_bias=self.router_bias, logit_noise=logit_noise,
-                      selection_bias=self.selection_bias,
+                      selection_bias=self.selection_bias, shared=self.shared,
                       losses=self.losses if stats else None,
                       mean_prob=self.mean_prob if stats else None,
                       counts=self.counts if stats else None, stream=stream)

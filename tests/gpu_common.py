@@ -51,7 +51,7 @@ class Bufs:
     def __init__(self, wl: Workload, device="cuda"):
         self.wl = wl
         self.cfg = B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K, wl.dtype, wl.capacity_factor,
-                                    **wl.routing())
+                                    F_shared=wl.F_shared, **wl.routing())
         T, D, F, E, K = wl.T, wl.D, wl.F, wl.E, wl.K
         dt = wl.torch_dtype
         self.max_rows = B.max_rows(self.cfg)
@@ -73,6 +73,14 @@ class Bufs:
         self.h = torch.empty(R, F, dtype=dt, device=device)
         self.y_perm = torch.empty(R, D, dtype=dt, device=device)
         self.y = torch.empty(T, D, dtype=dt, device=device)
+        self.y_shared = None
+        if wl.F_shared:
+            # the shared expert, run op by op as a one-expert problem over x
+            self.cfg_s = B.MoeConfig.make(T, D, wl.F_shared, 1, 1, wl.dtype)
+            self.ws_s = torch.zeros(B.workspace_size(self.cfg_s), dtype=torch.uint8, device=device)
+            self.offs_s = torch.tensor([0, T], dtype=i32, device=device)
+            self.h_s = torch.empty(T, wl.F_shared, dtype=dt, device=device)
+            self.y_shared = torch.empty(T, D, dtype=dt, device=device)
 
     def run_ops(self, inp, logits_in=None):
         c = self.cfg
@@ -87,7 +95,11 @@ class Bufs:
                        self.row_of, self.x_perm, self.ws)
         B.moe_expert_ffn(c, self.x_perm, self.offsets, self.perm, self.w, inp["w_gate"],
                          inp["w_up"], inp["w_down"], self.h, self.y_perm, self.ws)
-        B.moe_combine(c, self.y_perm, self.row_of, self.y)
+        if self.y_shared is not None:
+            sg, su, sd = inp["shared"]
+            B.moe_expert_ffn(self.cfg_s, inp["x"], self.offs_s, None, None, sg, su, sd, self.h_s,
+                             self.y_shared, self.ws_s)
+        B.moe_combine(c, self.y_perm, self.row_of, self.y, y_add=self.y_shared)
         torch.cuda.synchronize()
         flags = B.moe_get_device_status(self.ws)
         assert flags == 0, f"device status flags {flags:#x}"

@@ -54,6 +54,9 @@ def _cfg(**kw):
     (dict(n_groups=33, topk_groups=1, E=66), B.MOE_ERR_ARG),
     (dict(route_scale=0.0), B.MOE_ERR_ARG),
     (dict(route_scale=float("inf")), B.MOE_ERR_ARG),
+    (dict(F_shared=64), B.MOE_OK),
+    (dict(F_shared=60), B.MOE_ERR_ALIGN),
+    (dict(F_shared=-8), B.MOE_ERR_SHAPE),
 ])
 def test_check_config(lib, kw, code):
     assert B.check_config(_cfg(**kw)) == code
@@ -118,13 +121,25 @@ def test_dispatch_ffn_combine_forward_argument_errors(lib):
                               None) == B.MOE_ERR_ARG
     assert lib.moe_expert_ffn(cr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE,
                               nb, None) == B.MOE_ERR_ALIGN
-    assert lib.moe_combine(cr, FAKE, None, FAKE, None) == B.MOE_ERR_ARG
-    assert lib.moe_combine(cr, FAKE, FAKE, FAKE + 8, None) == B.MOE_ERR_ALIGN
+    assert lib.moe_combine(cr, FAKE, None, None, FAKE, None) == B.MOE_ERR_ARG
+    assert lib.moe_combine(cr, FAKE, FAKE, None, FAKE + 8, None) == B.MOE_ERR_ALIGN
+    assert lib.moe_combine(cr, FAKE, FAKE, FAKE + 4, FAKE, None) == B.MOE_ERR_ALIGN
+    # perm and topk_w: both given, or both NULL (unit weights)
+    assert lib.moe_expert_ffn(cr, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nb,
+                              None) == B.MOE_ERR_ARG
     fb = B.forward_workspace_size(c)
-    assert lib.moe_forward(cr, FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, None, None,
-                           None, None, None, FAKE, fb - 1, None) == B.MOE_ERR_WORKSPACE
-    assert lib.moe_forward(cr, FAKE, None, None, None, None, FAKE, FAKE, FAKE, FAKE, None, None,
-                           None, None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+    assert lib.moe_forward(cr, FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, None, None, None,
+                           FAKE, None, None, None, None, None, FAKE, fb - 1,
+                           None) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(cr, FAKE, None, None, None, None, FAKE, FAKE, FAKE, None, None, None,
+                           FAKE, None, None, None, None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+    # a shared expert needs its three weights
+    cs = _cfg(F_shared=64)
+    fbs = B.forward_workspace_size(cs)
+    assert fbs > fb
+    assert lib.moe_forward(ctypes.byref(cs), FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE,
+                           None, FAKE, FAKE, None, None, None, None, None, FAKE, fbs,
+                           None) == B.MOE_ERR_ARG
     assert lib.moe_update_selection_bias(cr, None, ctypes.c_float(0.01), FAKE, None) == B.MOE_ERR_ARG
     assert lib.moe_update_selection_bias(cr, FAKE, ctypes.c_float(float("nan")), FAKE,
                                          None) == B.MOE_ERR_ARG
@@ -143,13 +158,15 @@ def test_forward_kernel_count(lib):
     assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 11  # tensor-core router
     assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 12  # split SIMT router
     assert B.forward_kernel_count(_cfg(K=0)) == 0
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256)) == 14
 
 
 def test_status_strings_and_trace_table(lib):
     assert B.status_string(0) == "ok"
     assert "workspace" in B.status_string(B.MOE_ERR_WORKSPACE)
     names = B.trace_stage_names()
-    assert names[0] == "start" and names[-1] == "combine" and len(names) == 7
+    assert names[0] == "start" and names[-1] == "combine" and len(names) == 8
+    assert "shared_expert" in names
     assert lib.moe_trace_attach(None, 0) == B.MOE_OK
     assert lib.moe_trace_attach(None, 3) == B.MOE_ERR_ARG
     assert lib.moe_trace_attach(None, 17) == B.MOE_ERR_ARG

@@ -57,11 +57,21 @@ SMALL = [
         sel_bias=True, seed=27),
     _wl("groups_norenorm_tcr", T=2048, D=128, F=32, E=128, K=8, n_groups=8, topk_groups=4,
         renormalize=False, route_scale=1.5, bias="zipf", seed=28),
+    # shared expert (one expert over every token, added in the combine)
+    _wl("shared_bf16_pair", T=700, D=136, F=200, E=4, K=2, F_shared=264, seed=29),
+    _wl("shared_f32", T=300, D=64, F=96, E=8, K=2, F_shared=72, dtype="f32", seed=30),
+    _wl("shared_drops", T=400, D=64, F=96, E=8, K=2, capacity_factor=0.5, F_shared=128, seed=31),
 ]
 
 
 def _to_dev(inp):
-    return {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    def dev(v):
+        if v is None:
+            return None
+        if isinstance(v, tuple):
+            return tuple(t.cuda() for t in v)
+        return v.cuda()
+    return {k: dev(v) for k, v in inp.items()}
 
 
 @pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
@@ -76,7 +86,7 @@ def test_small_layers_elementwise(cuda_ok, wl):
     ref = oracle.forward(inp_cpu["x"], inp_cpu["w_router"], inp_cpu["w_gate"], inp_cpu["w_up"],
                          inp_cpu["w_down"], wl.K, wl.capacity_factor, inp_cpu["bias"],
                          inp_cpu["noise"], logits=b.logits.cpu().numpy(), sel_bias=sb,
-                         **wl.routing())
+                         shared=inp_cpu["shared"], **wl.routing())
     R = int(ref["offsets"][-1])
     # dispatch gather: exact copies
     assert torch.equal(b.x_perm[:R].cpu().to(torch.float64),
@@ -84,11 +94,15 @@ def test_small_layers_elementwise(cuda_ok, wl):
     # expert outputs with the routing weight applied
     assert_close_out(wl, to_np(b.y_perm[:R]), ref["o"] * ref["row_weight"][:, None], "y_perm")
     assert_close_out(wl, to_np(b.y), ref["y"], "y")
-    # dropped-everything tokens are exactly zero
+    # dropped-everything tokens get exactly zero from the routed experts (so
+    # exactly the shared expert's output when there is one)
     kept = ref["row_of"].reshape(wl.T, wl.K) >= 0
     none = np.nonzero(~kept.any(1))[0]
     if none.size:
-        assert (to_np(b.y[none]) == 0).all()
+        if b.y_shared is None:
+            assert (to_np(b.y[none]) == 0).all()
+        else:
+            assert torch.equal(b.y[none], b.y_shared[none])
     # the whole layer in one call gives the same bits as the op-by-op path
     ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
     y2 = torch.empty_like(b.y)
@@ -96,7 +110,7 @@ def test_small_layers_elementwise(cuda_ok, wl):
     counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
     B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y2,
                   ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses,
-                  counts=counts, selection_bias=inp["sel_bias"])
+                  counts=counts, selection_bias=inp["sel_bias"], shared=inp["shared"])
     torch.cuda.synchronize()
     assert torch.equal(y2, b.y)
     assert torch.equal(losses, b.losses)

@@ -46,6 +46,7 @@ class Workload:
     topk_groups: int = 1
     route_scale: float = 1.0
     sel_bias: bool = False        # a seeded DeepSeek-V3 selection bias input
+    F_shared: int = 0             # hidden size of a shared expert (0: none)
 
     def routing(self) -> dict:
         """Router options as keyword arguments (oracle.route / MoeConfig.make)."""
@@ -125,7 +126,8 @@ def make_inputs(wl: Workload | str, device="cpu", seed: int | None = None) -> di
 
     Returns a dict with x (T,D), w_router (D,E) fp32, bias (E) fp32 or None,
     noise (T,E) fp32 or None, w_gate (E,D,F), w_up (E,D,F), w_down (E,F,D),
-    sel_bias (E) fp32 or None (N(0, 0.5^2), generator seed + 2).
+    sel_bias (E) fp32 or None (N(0, 0.5^2), generator seed + 2), shared =
+    (w_gate_s (D,Fs), w_up_s (D,Fs), w_down_s (Fs,D)) or None (generator seed + 3).
     Draw order (one generator, seeded): x, w_router, w_gate, w_up, w_down.
     """
     if isinstance(wl, str):
@@ -147,8 +149,15 @@ def make_inputs(wl: Workload | str, device="cpu", seed: int | None = None) -> di
     sel_bias = None
     if wl.sel_bias:
         sel_bias = _randn((wl.E,), _gen(device, seed + 2), device, 0.5, torch.float32)
+    shared = None
+    if wl.F_shared:
+        g3 = _gen(device, seed + 3)
+        fs = wl.F_shared
+        shared = (_randn((wl.D, fs), g3, device, wl.w_std, dt),
+                  _randn((wl.D, fs), g3, device, wl.w_std, dt),
+                  _randn((fs, wl.D), g3, device, wl.w_std, dt))
     return dict(x=x, w_router=w_router, bias=bias, noise=noise,
-                w_gate=w_gate, w_up=w_up, w_down=w_down, sel_bias=sel_bias)
+                w_gate=w_gate, w_up=w_up, w_down=w_down, sel_bias=sel_bias, shared=shared)
 
 
 def make_tokens(wl: Workload | str, device="cpu", seed: int = 1234) -> torch.Tensor:
