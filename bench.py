@@ -164,6 +164,10 @@ def algorithmic(wl: Workload, counts, kept_rows: int):
         "dispatch_bytes": float(wl.T * wl.D * s + R * wl.D * s),
         "combine_bytes": float(R * wl.D * s + wl.T * wl.D * s),
         "active_weight_bytes": float(sum(1 for c in counts if c > 0) * 3 * wl.D * wl.F * s),
+        # gate/up GEMM: each active expert's two weight matrices, its rows of
+        # x_perm read once, h written once
+        "gateup_bytes": float(sum(1 for c in counts if c > 0) * 2 * wl.D * wl.F * s
+                              + R * wl.D * s + R * wl.F * s),
     }
 
 
@@ -280,12 +284,25 @@ def run_gpu(args):
         key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
         peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
         gu_ms = stage_ms["expert_gate_up"]
-        achieved = alg["gateup_flop"] / (gu_ms / 1e3) / 1e12
-        roofline = {"kernel": "expert_gate_up (grouped GEMM + SwiGLU)", "bound": "tensor",
-                    "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(achieved / peak, 4),
-                    "peak_source": f"{key} of {peak_src}",
-                    "traffic": recorded_traffic(wl.name, "expert_gate_up")}
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        # which roof binds: the kernel's arithmetic intensity against the
+        # ridge point of the two measured peaks
+        intensity = alg["gateup_flop"] / alg["gateup_bytes"]
+        ridge = peak * 1e12 / (hbm_peak * 1e9)
+        if intensity >= ridge:
+            achieved = alg["gateup_flop"] / (gu_ms / 1e3) / 1e12
+            roofline = {"kernel": "expert_gate_up (grouped GEMM + SwiGLU)", "bound": "tensor",
+                        "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                        "frac": round(achieved / peak, 4),
+                        "peak_source": f"{key} of {peak_src}"}
+        else:
+            achieved = alg["gateup_bytes"] / (gu_ms / 1e3) / 1e9
+            roofline = {"kernel": "expert_gate_up (grouped GEMM + SwiGLU)", "bound": "hbm",
+                        "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                        "frac": round(achieved / hbm_peak, 4),
+                        "peak_source": f"hbm_gbs of {peak_src}"}
+        roofline.update(intensity_flop_per_byte=round(intensity, 1), ridge=round(ridge, 1),
+                        traffic=recorded_traffic(wl.name, "expert_gate_up"))
     else:
         # fp32 layer: SIMT FMA pipes; peak from unit counts and the clock:
         # 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock
