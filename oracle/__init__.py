@@ -1,4 +1,4 @@
-"""CPU fp64 oracle of the token-choice top-k MoE layer forward.
+"""CPU fp64 oracle of the token-choice top-k MoE layer: forward and backward.
 
 TEST INFRASTRUCTURE ONLY: this package is the checker the CUDA library is
 compared against.  Only the tests, ``__graft_entry__.smoke()`` and the CPU
@@ -71,6 +71,19 @@ def _load():
             lib.oracle_expert_rows.restype = None
             lib.oracle_combine.argtypes = [i64, i32, i32, P, P, P, P]
             lib.oracle_combine.restype = None
+            lib.oracle_router_backward.argtypes = [i64, i32, i32, P, P, P, P, i32, i32, f64, f64,
+                                                   f64, P]
+            lib.oracle_router_backward.restype = None
+            lib.oracle_router_linear_backward.argtypes = [i64, i32, i32, P, i32, P, P, P, P, P]
+            lib.oracle_router_linear_backward.restype = None
+            lib.oracle_expert_backward_rows.argtypes = [i64, P, P, P, i32, i32, P, i32, P, P, P, P,
+                                                        i32, P, P, P, P, P]
+            lib.oracle_expert_backward_rows.restype = None
+            lib.oracle_expert_backward_cols.argtypes = [i64, P, P, P, i32, i32, i32, P, P, i32, P,
+                                                        P, P, P, i32, P, P, P]
+            lib.oracle_expert_backward_cols.restype = None
+            lib.oracle_expert_wgrad.argtypes = [i64, P, P, i32, i32, P, i32, P, P, P, P, P, P, P]
+            lib.oracle_expert_wgrad.restype = None
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = i32
             _lib = lib
@@ -371,3 +384,180 @@ def token_outputs(x_rows, slot_ids, slot_weights, slot_kept, get_expert, outs=No
             if kp[i, k]:
                 y[i] += ws[i, k] * outs[i, k]
     return y
+
+
+# ----------------------------------------------------------------- backward
+#
+# The gradient of  loss = sum <dY, y> + c_bal * balance + c_z * z  ("Lab: build
+# a tiny MoE in PyTorch", "Smoke test and backward pass"), with the top-k
+# decision as a stop-gradient ("2.9 Mixture-of-Experts (MoE) Architectures",
+# "The Router").  The arithmetic is in moe_oracle.c; these wrappers marshal.
+
+
+def router_backward(logits, ids, dw, counts, c_bal: float = 0.0, c_z: float = 0.0,
+                     score_func: str = "softmax", renormalize: bool = True,
+                     route_scale: float = 1.0) -> np.ndarray:
+    """dL (T, E): gradient of the router logits from the gate-weight
+    gradients dw (T, K), the balance loss (coefficient c_bal, counts fixed) and
+    the z-loss (coefficient c_z)."""
+    lib = _load()
+    L = _f64(logits)
+    ids = _i32(ids)
+    T, E = L.shape
+    K = ids.shape[1]
+    dw = _f64(dw).reshape(T, K)
+    cnt = np.ascontiguousarray(np.asarray(counts, dtype=np.int64))
+    out = np.empty((T, E), np.float64)
+    lib.oracle_router_backward(T, E, K, _ptr(L), _ptr(ids), _ptr(dw), _ptr(cnt),
+                               SCORE_FUNCS[score_func], int(bool(renormalize)), float(route_scale),
+                               float(c_bal), float(c_z), _ptr(out))
+    return out
+
+
+def router_linear_backward(x, w_router, dlogits):
+    """(dW_r (D, E), db (E,), dx_r (T, D)) of L = x W_r + b."""
+    lib = _load()
+    xa, xd = _elem_array(x)
+    w = _f32(w_router)
+    dL = _f64(dlogits)
+    T, D = xa.shape
+    E = w.shape[1]
+    dw = np.empty((D, E), np.float64)
+    db = np.empty((E,), np.float64)
+    dx = np.empty((T, D), np.float64)
+    lib.oracle_router_linear_backward(T, D, E, _ptr(xa), xd, _ptr(w), _ptr(dL), _ptr(dw), _ptr(db),
+                                      _ptr(dx))
+    return dw, db, dx
+
+
+def _weights3(w_gate, w_up, w_down):
+    wg, t1 = _elem_array(w_gate)
+    wu, t2 = _elem_array(w_up)
+    wd, t3 = _elem_array(w_down)
+    if not (t1 == t2 == t3):
+        raise TypeError("expert weights must share one element type")
+    if wg.ndim == 2:  # one expert (a shared expert): (D, F), (D, F), (F, D)
+        wg, wu, wd = wg[None], wu[None], wd[None]
+    return np.ascontiguousarray(wg), np.ascontiguousarray(wu), np.ascontiguousarray(wd), t1
+
+
+def expert_backward_rows(tok, ex, wt, x, dy, w_gate, w_up, w_down, intermediates: bool = False):
+    """Per-row expert backward: dw (n,), dx (n, D) and, with ``intermediates``,
+    h, dg, du (n, F).  Row r is token tok[r] through expert ex[r] with gate
+    weight wt[r]; weights (E, D, F), (E, D, F), (E, F, D) or one expert's 2-D
+    matrices."""
+    lib = _load()
+    xa, xd = _elem_array(x)
+    wg, wu, wd, wdt = _weights3(w_gate, w_up, w_down)
+    dyd = _f64(dy)
+    tok, ex, wt = _i32(tok), _i32(ex), _f64(wt)
+    n = tok.shape[0]
+    D, F = wg.shape[1], wg.shape[2]
+    dw = np.zeros((n,), np.float64)
+    dx = np.zeros((n, D), np.float64)
+    h = np.zeros((n, F), np.float64) if intermediates else None
+    dg = np.zeros((n, F), np.float64) if intermediates else None
+    du = np.zeros((n, F), np.float64) if intermediates else None
+    if n:
+        lib.oracle_expert_backward_rows(n, _ptr(tok), _ptr(ex), _ptr(wt), D, F, _ptr(xa), xd,
+                                        _ptr(dyd), _ptr(wg), _ptr(wu), _ptr(wd), wdt, _ptr(dw),
+                                        _ptr(dx), _ptr(h), _ptr(dg), _ptr(du))
+    if intermediates:
+        return dw, dx, h, dg, du
+    return dw, dx
+
+
+def expert_backward_cols(tok, ex, wt, fcols, x, dy, w_gate, w_up, w_down):
+    """h, dg, du (n, len(fcols)) of the given rows at hidden columns fcols."""
+    lib = _load()
+    xa, xd = _elem_array(x)
+    wg, wu, wd, wdt = _weights3(w_gate, w_up, w_down)
+    dyd = _f64(dy)
+    tok, ex, wt, fc = _i32(tok), _i32(ex), _f64(wt), _i32(fcols)
+    n, nf = tok.shape[0], fc.shape[0]
+    D, F = wg.shape[1], wg.shape[2]
+    h = np.zeros((n, nf), np.float64)
+    dg = np.zeros((n, nf), np.float64)
+    du = np.zeros((n, nf), np.float64)
+    if n:
+        lib.oracle_expert_backward_cols(n, _ptr(tok), _ptr(ex), _ptr(wt), D, F, nf, _ptr(fc),
+                                        _ptr(xa), xd, _ptr(dyd), _ptr(wg), _ptr(wu), _ptr(wd), wdt,
+                                        _ptr(h), _ptr(dg), _ptr(du))
+    return h, dg, du
+
+
+def expert_wgrad(tok, wt, x, dy, h, dg, du):
+    """(dWg (D, F'), dWu (D, F'), dWd (F', D)) of one expert from its rows in
+    row order; F' = h.shape[1] (all hidden columns, or a sampled subset)."""
+    lib = _load()
+    xa, xd = _elem_array(x)
+    dyd = _f64(dy)
+    tok, wt = _i32(tok), _f64(wt)
+    h, dg, du = _f64(h), _f64(dg), _f64(du)
+    n = tok.shape[0]
+    D = xa.shape[1]
+    F = h.shape[1] if h.ndim == 2 else 0
+    dWg = np.zeros((D, F), np.float64)
+    dWu = np.zeros((D, F), np.float64)
+    dWd = np.zeros((F, D), np.float64)
+    lib.oracle_expert_wgrad(n, _ptr(tok), _ptr(wt), D, F, _ptr(xa), xd, _ptr(dyd), _ptr(h),
+                            _ptr(dg), _ptr(du), _ptr(dWg), _ptr(dWu), _ptr(dWd))
+    return dWg, dWu, dWd
+
+
+def backward(x, w_router, w_gate, w_up, w_down, dy, K: int, capacity_factor: float = 0.0,
+             bias=None, noise=None, logits=None, shared=None, c_bal: float = 0.0,
+             c_z: float = 0.0, **routing) -> dict:
+    """Gradients of the whole layer for upstream gradient dy (T, D) of y and
+    loss coefficients c_bal (balance) and c_z (z-loss).
+
+    Runs the oracle forward first (same arguments as ``forward``), then: each
+    kept row's expert backward (dw, dx, h, dg, du); the gate-weight gradient
+    of every slot (0 for a dropped one); the router-logit gradient; the
+    router's linear map; the experts' weight gradients (rows in order); the
+    shared expert.  dx = sum over kept slots (slot order) of the rows' dx,
+    plus the shared expert's, plus the router's.
+    Returns dx, dw_router, db_router, dw_gate, dw_up, dw_down, dlogits,
+    dw_slot, dshared (tuple or None) and fwd (the forward's dict).
+    """
+    fwd = forward(x, w_router, w_gate, w_up, w_down, K, capacity_factor, bias=bias, noise=noise,
+                  logits=logits, shared=shared, **routing)
+    xa, _ = _elem_array(x)
+    T, D = xa.shape
+    wg_all, _, _, _ = _weights3(w_gate, w_up, w_down)
+    E, F = wg_all.shape[0], wg_all.shape[2]
+    dyd = _f64(dy)
+    perm, offsets, row_of = fwd["perm"], fwd["offsets"], fwd["row_of"]
+    R = perm.shape[0]
+    tok = (perm // K).astype(np.int32)
+    ex = np.repeat(np.arange(E, dtype=np.int32), np.diff(offsets))
+    wt = fwd["row_weight"]
+    dw_rows, dx_rows, h, dg, du = expert_backward_rows(tok, ex, wt, x, dyd, w_gate, w_up, w_down,
+                                                       intermediates=True)
+    dw_slot = np.zeros((T * K,), np.float64)
+    dw_slot[perm] = dw_rows
+    counts = np.asarray(fwd["counts"], dtype=np.int64)
+    sf = routing.get("score_func", "softmax")
+    dL = router_backward(fwd["logits"], fwd["ids"], dw_slot.reshape(T, K), counts, c_bal, c_z,
+                         score_func=sf, renormalize=routing.get("renormalize", True),
+                         route_scale=routing.get("route_scale", 1.0))
+    dWr, db, dx_r = router_linear_backward(x, w_router, dL)
+    dx = (combine(dx_rows, row_of, np.ones((T, K)), T, K) if R
+          else np.zeros((T, D), np.float64))
+    dWg = np.zeros((E, D, F), np.float64)
+    dWu = np.zeros((E, D, F), np.float64)
+    dWd = np.zeros((E, F, D), np.float64)
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        dWg[e], dWu[e], dWd[e] = expert_wgrad(tok[a:b], wt[a:b], x, dyd, h[a:b], dg[a:b], du[a:b])
+    dshared = None
+    if shared is not None:
+        ts = np.arange(T, dtype=np.int32)
+        _, dx_s, hs, dgs, dus = expert_backward_rows(ts, np.zeros(T, np.int32), np.ones(T), x, dyd,
+                                                     shared[0], shared[1], shared[2],
+                                                     intermediates=True)
+        dx = dx + dx_s
+        dshared = expert_wgrad(ts, np.ones(T), x, dyd, hs, dgs, dus)
+    dx = dx + dx_r
+    return dict(dx=dx, dw_router=dWr, db_router=db, dw_gate=dWg, dw_up=dWu, dw_down=dWd,
+                dlogits=dL, dw_slot=dw_slot.reshape(T, K), dshared=dshared, fwd=fwd)

@@ -1,6 +1,6 @@
 /*
  * moe_oracle.c -- plain CPU fp64 oracle of the token-choice top-k
- * Mixture-of-Experts layer forward.
+ * Mixture-of-Experts layer: forward, and the backward of its training loss.
  *
  * TEST INFRASTRUCTURE ONLY.  This file is the checker that the CUDA library is
  * compared against.  It shares no code, header, table or helper with the CUDA
@@ -20,6 +20,12 @@
  *              Question", "A Toy MoE Layer From Scratch", "The auxiliary
  *              load-balancing loss", "Capacity Factor, Token Dropping, and the
  *              Worked Numbers".
+ *   Backward:  [TinyMoE] "Smoke test and backward pass" (the training loss is
+ *              main + c_bal * balance + c_z * z, differentiated by autograd) and
+ *              [LLMBook] "The Router" (the top-k index decision is a stop-
+ *              gradient; gradient reaches the router only through the kept gate
+ *              weights and the auxiliary losses; an expert that was not chosen
+ *              gets none from that token).
  *
  * Element types of inputs: 0 = IEEE fp32, 1 = bf16 given as raw 16-bit words.
  * Both convert exactly to double.
@@ -406,6 +412,318 @@ void oracle_combine(int64_t T, int32_t K, int32_t D, const double *o, const int3
             double w = weights[t * K + k];
             for (int32_t j = 0; j < D; ++j)
                 yt[j] += w * o[(int64_t)row * D + j];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ backward
+ *
+ * The gradient of  loss = sum_t <dY_t, y_t> + c_bal * balance + c_z * z,
+ * i.e. the backward of the forward above for an upstream gradient dY of y and
+ * the loss coefficients c_bal, c_z ([TinyMoE] "Smoke test and backward pass":
+ * loss = main + 0.01 * balance + 0.001 * z).  Stop-gradients, as autograd
+ * applies them to the forward: the chosen ids (top-k, the group limit, the
+ * selection bias) and the counts f_e of the balance loss (an integer count)
+ * carry no gradient; the capacity keep mask is a function of the ids only.
+ * Everything else -- the gate weights, the normalised scores of the balance
+ * loss, the logsumexp of the z-loss, the router's linear map and the experts --
+ * is differentiated by the chain rule, written out below step by step.
+ */
+
+/*
+ * Gradient of the router logits for each token, from the gradients of its K
+ * gate weights (dw, T x K; a dropped slot never reached y, so its dw is 0),
+ * and of the two auxiliary losses.  With S the chosen scores' sum and
+ * rs = route_scale:
+ *   gate weights   w_k = rs * score[id_k] / S   (renormalize) or rs * score[id_k]
+ *                  d score[id_j] += rs/S * (dw_j - sum_k dw_k * score[id_k] / S)
+ *                             or += rs * dw_j
+ *   balance        balance = E * sum_e f_e * P_e,  P_e = (1/T) sum_t n[t,e], where
+ *                  n = score / sum_e score (softmax: n = p), f_e = counts_e/(T*K):
+ *                  d n[t,e] = c_bal * E * f_e / T;  for sigmoid scores
+ *                  d score_j += (d n_j - sum_e d n_e * n_e) / sum_e score_e
+ *   scores         softmax: dL_j = p_j * (d p_j - sum_i p_i * d p_i)
+ *                  sigmoid: dL_j = d s_j * s_j * (1 - s_j)
+ *   z-loss         z = (1/T) sum_t lse_t^2:  dL_j += c_z * 2 * lse_t / T * softmax(L)_j
+ * logits (T, E) are the logits the forward routed on.  dlogits (T, E).
+ */
+void oracle_router_backward(int64_t T, int32_t E, int32_t K, const double *logits,
+                            const int32_t *ids, const double *dw, const int64_t *counts,
+                            int32_t score_func, int32_t renormalize, double route_scale,
+                            double c_bal, double c_z, double *dlogits)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double *L = logits + t * E;
+        double *dL = dlogits + t * E;
+        double *p = (double *)malloc(sizeof(double) * (size_t)E);     /* softmax(L) */
+        double *score = (double *)malloc(sizeof(double) * (size_t)E);
+        double *dscore = (double *)malloc(sizeof(double) * (size_t)E);
+        double m = L[0];
+        for (int32_t e = 0; e < E; ++e)
+            if (L[e] > m)
+                m = L[e];
+        double se = 0.0;
+        for (int32_t e = 0; e < E; ++e)
+            se += exp(L[e] - m);
+        const double lse = m + log(se);
+        for (int32_t e = 0; e < E; ++e) {
+            p[e] = exp(L[e] - m) / se;
+            score[e] = score_func == 1 ? 1.0 / (1.0 + exp(-L[e])) : p[e];
+            dscore[e] = 0.0;
+        }
+        /* the gate weights */
+        double S = 0.0, sdw = 0.0;
+        for (int32_t k = 0; k < K; ++k)
+            S += score[ids[t * K + k]];
+        for (int32_t k = 0; k < K; ++k)
+            sdw += dw[t * K + k] * score[ids[t * K + k]] / S;
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t j = ids[t * K + k];
+            if (renormalize)
+                dscore[j] += route_scale / S * (dw[t * K + k] - sdw);
+            else
+                dscore[j] += route_scale * dw[t * K + k];
+        }
+        /* the balance loss, through the normalised scores */
+        double ss = 0.0;
+        for (int32_t e = 0; e < E; ++e)
+            ss += score[e];
+        if (score_func == 1) {
+            double dot = 0.0;
+            for (int32_t e = 0; e < E; ++e)
+                dot += c_bal * (double)E * ((double)counts[e] / (double)(T * K)) / (double)T *
+                       (score[e] / ss);
+            for (int32_t e = 0; e < E; ++e) {
+                double dn = c_bal * (double)E * ((double)counts[e] / (double)(T * K)) / (double)T;
+                dscore[e] += (dn - dot) / ss;
+            }
+        } else {
+            for (int32_t e = 0; e < E; ++e)
+                dscore[e] += c_bal * (double)E * ((double)counts[e] / (double)(T * K)) / (double)T;
+        }
+        /* the scores, from the logits */
+        if (score_func == 1) {
+            for (int32_t e = 0; e < E; ++e)
+                dL[e] = dscore[e] * score[e] * (1.0 - score[e]);
+        } else {
+            double dot = 0.0;
+            for (int32_t e = 0; e < E; ++e)
+                dot += p[e] * dscore[e];
+            for (int32_t e = 0; e < E; ++e)
+                dL[e] = p[e] * (dscore[e] - dot);
+        }
+        /* the z-loss */
+        for (int32_t e = 0; e < E; ++e)
+            dL[e] += c_z * 2.0 * lse / (double)T * p[e];
+        free(p);
+        free(score);
+        free(dscore);
+    }
+}
+
+/*
+ * Gradients of the router's linear map L = x W_r + b (+ noise), from dlogits:
+ *     dW_r[d,e] = sum_t x[t,d] * dL[t,e]      (tokens in order)
+ *     db[e]     = sum_t dL[t,e]
+ *     dx_r[t,d] = sum_e dL[t,e] * W_r[d,e]
+ * The noise is an input, not a parameter.  db and dx_r may be NULL.
+ */
+void oracle_router_linear_backward(int64_t T, int32_t D, int32_t E, const void *x, int32_t x_dtype,
+                                   const float *w_r, const double *dlogits, double *dw_r,
+                                   double *db, double *dx_r)
+{
+#pragma omp parallel for schedule(static)
+    for (int32_t d = 0; d < D; ++d) {
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; ++t)
+                acc += elem(x, x_dtype, t * D + d) * dlogits[t * E + e];
+            dw_r[(int64_t)d * E + e] = acc;
+        }
+    }
+    if (db) {
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; ++t)
+                acc += dlogits[t * E + e];
+            db[e] = acc;
+        }
+    }
+    if (dx_r) {
+#pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t)
+            for (int32_t d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int32_t e = 0; e < E; ++e)
+                    acc += dlogits[t * E + e] * (double)w_r[(int64_t)d * E + e];
+                dx_r[t * D + d] = acc;
+            }
+    }
+}
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+/* d silu / d g = s + g * s * (1 - s), s = 1 / (1 + exp(-g)) */
+static double dsilu(double g)
+{
+    double sg = 1.0 / (1.0 + exp(-g));
+    return sg + g * sg * (1.0 - sg);
+}
+
+/*
+ * Backward of the expert FFN for a list of rows (token tok[r] through expert
+ * ex[r] with gate weight wt[r]).  For one row, with x its token's input and
+ * dYp = wt * dY[tok] (the gradient reaching this expert's output):
+ *     g = x Wg,  u = x Wu,  h = silu(g) * u,  o = h Wd   (the forward, recomputed)
+ *     dw     = <dY[tok], o>                 (gradient of the gate weight)
+ *     dh_f   = sum_j dYp_j Wd[f,j]
+ *     dg_f   = dh_f * u_f * silu'(g_f),   du_f = dh_f * silu(g_f)
+ *     dx_d   = sum_f dg_f Wg[d,f] + du_f Wu[d,f]
+ * Weights are (E, D, F) gate/up and (E, F, D) down, row-major, w_dtype.
+ * dy is (T, D).  Outputs: dw (n), dx (n, D); h, dg, du (n, F) may be NULL.
+ */
+void oracle_expert_backward_rows(int64_t n, const int32_t *tok, const int32_t *ex,
+                                 const double *wt, int32_t D, int32_t F, const void *x,
+                                 int32_t x_dtype, const double *dy, const void *w_gate,
+                                 const void *w_up, const void *w_down, int32_t w_dtype,
+                                 double *dw, double *dx, double *h_out, double *dg_out,
+                                 double *du_out)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+        const int64_t t = tok[r];
+        const int64_t wo = (int64_t)ex[r] * D * F; /* this expert's matrices */
+        double *g = (double *)malloc(sizeof(double) * (size_t)F);
+        double *u = (double *)malloc(sizeof(double) * (size_t)F);
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        double *dh = (double *)malloc(sizeof(double) * (size_t)F);
+        double *xr = (double *)malloc(sizeof(double) * (size_t)D);
+        for (int32_t d = 0; d < D; ++d)
+            xr[d] = elem(x, x_dtype, t * D + d);
+        for (int32_t f = 0; f < F; ++f) {
+            double ga = 0.0, ua = 0.0;
+            for (int32_t d = 0; d < D; ++d) {
+                ga += xr[d] * elem(w_gate, w_dtype, wo + (int64_t)d * F + f);
+                ua += xr[d] * elem(w_up, w_dtype, wo + (int64_t)d * F + f);
+            }
+            g[f] = ga;
+            u[f] = ua;
+            h[f] = silu(ga) * ua;
+        }
+        /* dw = <dY, o> with o = h Wd; dh = dYp Wd^T */
+        double dwr = 0.0;
+        for (int32_t j = 0; j < D; ++j) {
+            double o = 0.0;
+            for (int32_t f = 0; f < F; ++f)
+                o += h[f] * elem(w_down, w_dtype, wo + (int64_t)f * D + j);
+            dwr += dy[t * D + j] * o;
+        }
+        dw[r] = dwr;
+        for (int32_t f = 0; f < F; ++f) {
+            double acc = 0.0;
+            for (int32_t j = 0; j < D; ++j)
+                acc += wt[r] * dy[t * D + j] * elem(w_down, w_dtype, wo + (int64_t)f * D + j);
+            dh[f] = acc;
+        }
+        /* through SwiGLU: reuse g for dg and u for du */
+        for (int32_t f = 0; f < F; ++f) {
+            double dgf = dh[f] * u[f] * dsilu(g[f]);
+            double duf = dh[f] * silu(g[f]);
+            if (h_out)
+                h_out[r * F + f] = h[f];
+            g[f] = dgf;
+            u[f] = duf;
+            if (dg_out)
+                dg_out[r * F + f] = dgf;
+            if (du_out)
+                du_out[r * F + f] = duf;
+        }
+        for (int32_t d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int32_t f = 0; f < F; ++f)
+                acc += g[f] * elem(w_gate, w_dtype, wo + (int64_t)d * F + f) +
+                       u[f] * elem(w_up, w_dtype, wo + (int64_t)d * F + f);
+            dx[r * D + d] = acc;
+        }
+        free(g);
+        free(u);
+        free(h);
+        free(dh);
+        free(xr);
+    }
+}
+
+/*
+ * The same per-row quantities restricted to a list of hidden columns
+ * fcols (nf of them): for each row r and column f = fcols[i]
+ *     g_f = x Wg[:,f],  u_f = x Wu[:,f],  h_f = silu(g_f) u_f,
+ *     dh_f = sum_j wt_r dY[tok_r, j] Wd[f, j],
+ *     dg_f = dh_f u_f silu'(g_f),  du_f = dh_f silu(g_f)
+ * written to h, dg, du (n, nf).  With them, oracle_expert_wgrad (F := nf)
+ * gives the weight gradients' columns fcols of dWg, dWu and rows fcols of dWd
+ * at a cost of n * 3 * D per column.
+ */
+void oracle_expert_backward_cols(int64_t n, const int32_t *tok, const int32_t *ex,
+                                 const double *wt, int32_t D, int32_t F, int32_t nf,
+                                 const int32_t *fcols, const void *x, int32_t x_dtype,
+                                 const double *dy, const void *w_gate, const void *w_up,
+                                 const void *w_down, int32_t w_dtype, double *h, double *dg,
+                                 double *du)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        const int64_t t = tok[r];
+        const int64_t wo = (int64_t)ex[r] * D * F;
+        for (int32_t i = 0; i < nf; ++i) {
+            const int64_t f = fcols[i];
+            double g = 0.0, u = 0.0, dh = 0.0;
+            for (int32_t d = 0; d < D; ++d) {
+                double xd = elem(x, x_dtype, t * D + d);
+                g += xd * elem(w_gate, w_dtype, wo + (int64_t)d * F + f);
+                u += xd * elem(w_up, w_dtype, wo + (int64_t)d * F + f);
+                dh += wt[r] * dy[t * D + d] * elem(w_down, w_dtype, wo + f * D + d);
+            }
+            h[r * nf + i] = silu(g) * u;
+            dg[r * nf + i] = dh * u * dsilu(g);
+            du[r * nf + i] = dh * silu(g);
+        }
+    }
+}
+
+/*
+ * Weight gradients of one expert from its rows (in row order), given each
+ * row's h, dg, du (n, F) from oracle_expert_backward_rows:
+ *     dWg[d,f] = sum_r x[tok_r, d] * dg_r[f]
+ *     dWu[d,f] = sum_r x[tok_r, d] * du_r[f]
+ *     dWd[f,j] = sum_r h_r[f] * wt_r * dY[tok_r, j]
+ * dWg, dWu (D, F) and dWd (F, D), row-major.  n = 0 gives zeros.
+ */
+void oracle_expert_wgrad(int64_t n, const int32_t *tok, const double *wt, int32_t D, int32_t F,
+                         const void *x, int32_t x_dtype, const double *dy, const double *h,
+                         const double *dg, const double *du, double *dWg, double *dWu,
+                         double *dWd)
+{
+#pragma omp parallel for schedule(static)
+    for (int32_t d = 0; d < D; ++d) {
+        for (int32_t f = 0; f < F; ++f) {
+            double ag = 0.0, au = 0.0;
+            for (int64_t r = 0; r < n; ++r) {
+                double xd = elem(x, x_dtype, (int64_t)tok[r] * D + d);
+                ag += xd * dg[r * F + f];
+                au += xd * du[r * F + f];
+            }
+            dWg[(int64_t)d * F + f] = ag;
+            dWu[(int64_t)d * F + f] = au;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int32_t f = 0; f < F; ++f) {
+        for (int32_t j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (int64_t r = 0; r < n; ++r)
+                a += h[r * F + f] * wt[r] * dy[(int64_t)tok[r] * D + j];
+            dWd[(int64_t)f * D + j] = a;
         }
     }
 }
