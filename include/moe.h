@@ -1,6 +1,6 @@
 /*
  * moe.h -- C ABI of libmoe_b200.so: the forward pass of a token-choice top-k
- * Mixture-of-Experts layer on NVIDIA B200 (sm_100a).
+ * Mixture-of-Experts layer on NVIDIA B200 (sm_100a), and its backward.
  *
  * The layer (sources cited by page title and section):
  *   "Lab: build a tiny MoE in PyTorch" (open-llm-engineering), sections
@@ -270,6 +270,89 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        float *mean_prob, int32_t *counts, int32_t *topk_ids, float *topk_w,
                        void *workspace, size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------ training
+ *
+ * The backward of the layer's training loss ("Lab: build a tiny MoE in
+ * PyTorch", "Smoke test and backward pass": loss = main + c_bal * balance +
+ * c_z * z, differentiated by autograd; "2.9 Mixture-of-Experts (MoE)
+ * Architectures", "The Router": the top-k index decision is a stop-gradient,
+ * gradient reaches the router only through the kept gate weights and the
+ * auxiliary losses, and an expert a token did not choose gets nothing from
+ * it).  The stop-gradients, as autograd applies them to the forward: the chosen
+ * ids (with the group limit and the selection bias), the capacity keep mask
+ * and the balance loss's counts f_e.  Logit noise is an input.  bf16 layers
+ * only (MOE_ERR_UNSUPPORTED for MOE_F32).
+ */
+
+/*
+ * Bytes of the state moe_forward_train keeps for moe_backward:
+ * moe_forward_workspace_size plus the routed logits (T, E) fp32, the gate/up
+ * pre-activations (max_rows, 2F) and, with a shared expert, its (T, 2 F_shared).
+ */
+MOE_API moe_status moe_train_state_size(const moe_config *cfg, size_t *bytes);
+
+/*
+ * moe_forward for training: the same arguments and results, with the
+ * workspace replaced by `state` (moe_train_state_size bytes, 256-byte
+ * aligned), which keeps what moe_backward reads: the routing results, the
+ * dispatch layout, x_perm, [g | u] = the gate/up pre-activations rounded to
+ * bf16, h, the unweighted expert outputs and the logits.  The state must not
+ * be written between this call and moe_backward.  y equals moe_forward's up
+ * to rounding order: the routing weight multiplies each expert output in the
+ * combine (fp32) instead of in the down projection's epilogue.
+ */
+MOE_API moe_status moe_forward_train(const moe_config *cfg, const void *x, const float *w_router,
+                                     const float *router_bias, const float *selection_bias,
+                                     const float *logit_noise, const void *w_gate, const void *w_up,
+                                     const void *w_down, const void *w_gate_shared,
+                                     const void *w_up_shared, const void *w_down_shared, void *y,
+                                     float *losses, float *mean_prob, int32_t *counts,
+                                     int32_t *topk_ids, float *topk_w, void *state,
+                                     size_t state_bytes, void *stream);
+
+/* Bytes of device scratch moe_backward needs (its status word first). */
+MOE_API moe_status moe_backward_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/*
+ * Gradients of  loss = sum_{t,d} dy[t,d] * y[t,d] + c_balance * balance + c_z * z
+ * for the forward recorded in `state` by moe_forward_train (pass the same x
+ * and weights).  dy (T, D) bf16 is the upstream gradient of y; c_balance and
+ * c_z are the loss coefficients (the lab's 0.01 and 0.001), host values.
+ *
+ *   gate weights  dw[t,k] = <dy[t], o_k(x_t)> for a kept slot, 0 for a dropped
+ *                 one; through the renormalisation (or not) and route_scale
+ *   router        dL[t] = softmax / sigmoid backward of the gate weights' and
+ *                 the balance loss's score gradients, plus c_z * 2 lse_t / T * p_t
+ *   experts       dH = (w dy) Wd^T, [dg | du] = dH * [u silu'(g) | silu(g)],
+ *                 dx_e = dg Wg^T + du Wu^T; weight gradients summed over each
+ *                 expert's rows
+ *   input         dx = dL W_r^T + sum over kept slots of dx_e (+ shared expert)
+ *
+ * Outputs, all overwritten: dx (T, D) bf16; dw_router (D, E) fp32;
+ * db_router (E) fp32 or NULL; dw_gate, dw_up (E, D, F) fp32; dw_down
+ * (E, F, D) fp32; with a shared expert dw_gate_shared, dw_up_shared
+ * (D, F_shared) and dw_down_shared (F_shared, D) fp32 (ignored otherwise).
+ * Rounding: dy * w, [dg | du] and each expert's dx rows are rounded to bf16
+ * before the next contraction; every sum is fp32.  Deterministic.
+ * workspace: moe_backward_workspace_size bytes, 256-byte aligned; device
+ * faults are reported in its status word (moe_get_device_status(workspace)).
+ */
+MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const float *w_router,
+                                const void *w_gate, const void *w_up, const void *w_down,
+                                const void *w_gate_shared, const void *w_up_shared,
+                                const void *w_down_shared, const void *state, size_t state_bytes,
+                                const void *dy, float c_balance, float c_z, void *dx,
+                                float *dw_router, float *db_router, float *dw_gate, float *dw_up,
+                                float *dw_down, float *dw_gate_shared, float *dw_up_shared,
+                                float *dw_down_shared, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
+ * Number of kernels one moe_backward call launches for this configuration
+ * (0 for an invalid or unsupported one).
+ */
+MOE_API int32_t moe_backward_kernel_count(const moe_config *cfg);
+
 /*
  * moe_dispatch without a workspace, for callers that cannot allocate device
  * memory: code handed only its input and output buffers by a host framework
@@ -344,6 +427,16 @@ MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
 MOE_API moe_status moe_trace_attach(void *const *events, int32_t n_events);
 MOE_API int32_t moe_trace_boundary_count(void);
 MOE_API const char *moe_trace_stage_name(int32_t boundary);
+
+/*
+ * The same for moe_backward (10 boundaries): start, rows (dYp and the
+ * gate-weight gradients), router_bwd, dgrad_h, dgrad_x, wgrad_down,
+ * wgrad_gate_up, shared_expert, router_wgrad, dx.  Separate from the
+ * forward's events.
+ */
+MOE_API moe_status moe_trace_attach_backward(void *const *events, int32_t n_events);
+MOE_API int32_t moe_trace_backward_boundary_count(void);
+MOE_API const char *moe_trace_backward_stage_name(int32_t boundary);
 
 #ifdef __cplusplus
 }

@@ -89,6 +89,15 @@ _SIG = {
     "moe_trace_attach": ([_P, ctypes.c_int32], ctypes.c_int32),
     "moe_trace_boundary_count": ([], ctypes.c_int32),
     "moe_trace_stage_name": ([ctypes.c_int32], ctypes.c_char_p),
+    "moe_train_state_size": ([_P, _P], ctypes.c_int32),
+    "moe_forward_train": ([_P] * 19 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_backward_workspace_size": ([_P, _P], ctypes.c_int32),
+    "moe_backward": ([_P] * 10 + [ctypes.c_size_t, _P, ctypes.c_float, ctypes.c_float]
+                     + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_backward_kernel_count": ([_P], ctypes.c_int32),
+    "moe_trace_attach_backward": ([_P, ctypes.c_int32], ctypes.c_int32),
+    "moe_trace_backward_boundary_count": ([], ctypes.c_int32),
+    "moe_trace_backward_stage_name": ([ctypes.c_int32], ctypes.c_char_p),
 }
 
 
@@ -239,6 +248,53 @@ def moe_forward(cfg, x, w_router, w_gate, w_up, w_down, y, workspace, router_bia
     _check(st, "moe_forward")
 
 
+def train_state_size(cfg: MoeConfig) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().moe_train_state_size(_cfg(cfg), ctypes.byref(v)), "moe_train_state_size")
+    return v.value
+
+
+def backward_workspace_size(cfg: MoeConfig) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().moe_backward_workspace_size(_cfg(cfg), ctypes.byref(v)),
+           "moe_backward_workspace_size")
+    return v.value
+
+
+def moe_forward_train(cfg, x, w_router, w_gate, w_up, w_down, y, state, router_bias=None,
+                      logit_noise=None, losses=None, mean_prob=None, counts=None, topk_ids=None,
+                      topk_w=None, selection_bias=None, shared=None, stream=None):
+    """moe_forward that keeps the backward's activations in ``state``."""
+    sg, su, sd = shared if shared is not None else (None, None, None)
+    st = lib().moe_forward_train(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
+                                 _ptr(selection_bias), _ptr(logit_noise), _ptr(w_gate), _ptr(w_up),
+                                 _ptr(w_down), _ptr(sg), _ptr(su), _ptr(sd), _ptr(y),
+                                 _ptr(losses), _ptr(mean_prob), _ptr(counts), _ptr(topk_ids),
+                                 _ptr(topk_w), _ptr(state), _nbytes(state), _stream(stream))
+    _check(st, "moe_forward_train")
+
+
+def moe_backward(cfg, x, w_router, w_gate, w_up, w_down, state, dy, dx, dw_router, dw_gate, dw_up,
+                 dw_down, workspace, c_balance: float = 0.0, c_z: float = 0.0, db_router=None,
+                 shared=None, dshared=None, stream=None):
+    """shared = (w_gate_s, w_up_s, w_down_s) and dshared = their fp32
+    gradient buffers when cfg.F_shared > 0."""
+    sg, su, sd = shared if shared is not None else (None, None, None)
+    dg, du, dd = dshared if dshared is not None else (None, None, None)
+    st = lib().moe_backward(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up),
+                            _ptr(w_down), _ptr(sg), _ptr(su), _ptr(sd), _ptr(state), _nbytes(state),
+                            _ptr(dy), float(c_balance), float(c_z), _ptr(dx), _ptr(dw_router),
+                            _ptr(db_router), _ptr(dw_gate), _ptr(dw_up), _ptr(dw_down), _ptr(dg),
+                            _ptr(du), _ptr(dd), _ptr(workspace), _nbytes(workspace),
+                            _stream(stream))
+    _check(st, "moe_backward")
+
+
+def backward_kernel_count(cfg: MoeConfig) -> int:
+    """Kernels one moe_backward launches for this configuration."""
+    return int(lib().moe_backward_kernel_count(_cfg(cfg)))
+
+
 def moe_update_selection_bias(cfg, counts, gamma: float, selection_bias, stream=None):
     """selection_bias += gamma * sign(mean(counts) - counts), on the device."""
     _check(lib().moe_update_selection_bias(_cfg(cfg), _ptr(counts), float(gamma),
@@ -287,6 +343,28 @@ def moe_trace_attach(events):
 def trace_stage_names() -> list[str]:
     n = lib().moe_trace_boundary_count()
     return [lib().moe_trace_stage_name(i).decode() for i in range(n)]
+
+
+def _event_handles(events):
+    handles = []
+    for e in events:
+        if not isinstance(e, int) and not e.cuda_event:
+            e.record()
+        handles.append(e if isinstance(e, int) else e.cuda_event)
+    return handles
+
+
+def moe_trace_attach_backward(events):
+    """moe_trace_attach for moe_backward's boundaries."""
+    handles = _event_handles(events)
+    arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
+    _check(lib().moe_trace_attach_backward(arr if handles else None, len(handles)),
+           "moe_trace_attach_backward")
+
+
+def trace_backward_stage_names() -> list[str]:
+    n = lib().moe_trace_backward_boundary_count()
+    return [lib().moe_trace_backward_stage_name(i).decode() for i in range(n)]
 
 
 def _nbytes(t) -> int:

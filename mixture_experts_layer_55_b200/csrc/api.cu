@@ -17,8 +17,8 @@ cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const voi
 cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                const void* w_gate, const void* w_up, const void* w_down, void* h,
-                               void* y_perm, int* status, cudaStream_t s, StageHook mid,
-                               void* mid_ctx);
+                               void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                               StageHook mid, void* mid_ctx);
 
 int64_t capacity_of(const moe_config& c)
 {
@@ -97,6 +97,42 @@ FwdLayout fwd_layout(const moe_config& c, int64_t max_rows)
     return F;
 }
 
+TrainLayout train_layout(const moe_config& c, int64_t max_rows)
+{
+    TrainLayout L;
+    L.f = fwd_layout(c, max_rows);
+    const size_t es = c.dtype == MOE_BF16 ? 2 : 4;
+    size_t o = L.f.total;
+    L.logits = o; o += align_up((size_t)c.T * c.E * sizeof(float));
+    L.gu = o;     o += align_up((size_t)max_rows * 2 * c.F * es);
+    L.sh_gu = o;
+    if (c.F_shared > 0) o += align_up((size_t)c.T * 2 * c.F_shared * es);
+    L.total = o;
+    return L;
+}
+
+BwdLayout bwd_layout(const moe_config& c, int64_t max_rows)
+{
+    BwdLayout B;
+    const size_t es = c.dtype == MOE_BF16 ? 2 : 4;
+    size_t o = 0;
+    B.status = o;  o += align_up(64 * sizeof(int));
+    B.dyp = o;     o += align_up((size_t)max_rows * c.D * es);
+    B.dw_row = o;  o += align_up((size_t)max_rows * sizeof(float));
+    B.dlogits = o; o += align_up((size_t)c.T * c.E * sizeof(float));
+    B.dgu = o;     o += align_up((size_t)max_rows * 2 * c.F * es);
+    B.dxp = o;     o += align_up((size_t)max_rows * c.D * es);
+    B.rw_splits = router_wgrad_splits(c);
+    B.rw_part = o; o += align_up(router_wgrad_part_bytes(c, B.rw_splits));
+    B.sh_dgu = o;  B.sh_dx = o;
+    if (c.F_shared > 0) {
+        B.sh_dgu = o; o += align_up((size_t)c.T * 2 * c.F_shared * es);
+        B.sh_dx = o;  o += align_up((size_t)c.T * c.D * es);
+    }
+    B.total = o;
+    return B;
+}
+
 static moe_status check_config(const moe_config* c)
 {
     if (c == nullptr) return MOE_ERR_ARG;
@@ -141,6 +177,20 @@ static void trace(int boundary, cudaStream_t s)
 
 static void trace_mid_ffn(void*, cudaStream_t s) { trace(4, s); }
 
+static void* g_btrace[16];
+static int g_btrace_n = 0;
+static const char* kBwdStageNames[10] = {"start",      "rows",          "router_bwd",
+                                         "dgrad_h",    "dgrad_x",       "wgrad_down",
+                                         "wgrad_gate_up", "shared_expert", "router_wgrad", "dx"};
+
+static void btrace(int boundary, cudaStream_t s)
+{
+    if (boundary < g_btrace_n && g_btrace[boundary] != nullptr)
+        cudaEventRecord(static_cast<cudaEvent_t>(g_btrace[boundary]), s);
+}
+
+static void btrace_mid_dgrad(void*, cudaStream_t s) { btrace(3, s); }
+
 // offsets {0, n} of a single expert block covering n rows
 __global__ void set_row_range_kernel(int32_t* off, int32_t n)
 {
@@ -153,14 +203,28 @@ __global__ void set_row_range_kernel(int32_t* off, int32_t n)
 cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
                               const void* w_gate, const void* w_up, const void* w_down, void* h,
-                              void* y_perm, int* status, cudaStream_t s, StageHook mid,
-                              void* mid_ctx)
+                              void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                              StageHook mid, void* mid_ctx)
 {
-    if (c.dtype == MOE_F32)
+    if (c.dtype == MOE_F32) {
+        if (gu_keep != nullptr) return cudaErrorNotSupported;
         return launch_ffn_simt_f32(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up,
                                    w_down, h, y_perm, status, s, mid, mid_ctx);
+    }
     return launch_ffn_tc_bf16(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h,
-                              y_perm, status, s, mid, mid_ctx);
+                              y_perm, gu_keep, status, s, mid, mid_ctx);
+}
+
+// the shared expert as a layer of one expert over every token
+static moe_config shared_config(const moe_config& c)
+{
+    moe_config cs = c;
+    cs.E = 1;
+    cs.K = 1;
+    cs.F = c.F_shared;
+    cs.capacity_factor = 0.f;
+    cs.n_groups = 1;
+    return cs;
 }
 
 }  // namespace moe
@@ -297,8 +361,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + L.status);
     return cuda_status(launch_expert_ffn(*cfg, max_rows_of(*cfg), x_perm, offsets, perm, topk_w,
-                                         w_gate, w_up, w_down, h, y_perm, status, s, nullptr,
-                                         nullptr));
+                                         w_gate, w_up, w_down, h, y_perm, nullptr, status, s,
+                                         nullptr, nullptr));
 }
 
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of,
@@ -309,16 +373,85 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
     if (!y_perm || !row_of || !y) return MOE_ERR_ARG;
     if (!aligned16(y_perm) || !aligned16(y) || (y_add && !aligned16(y_add))) return MOE_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return cuda_status(launch_combine(*cfg, y_perm, row_of, y_add, y, max_rows_of(*cfg), s));
+    return cuda_status(launch_combine(*cfg, y_perm, row_of, nullptr, y_add, y, max_rows_of(*cfg), s));
 }
 
-moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
-                       const float* router_bias, const float* selection_bias,
-                       const float* logit_noise, const void* w_gate,
-                       const void* w_up, const void* w_down, const void* w_gate_shared,
-                       const void* w_up_shared, const void* w_down_shared, void* y, float* losses,
-                       float* mean_prob, int32_t* counts, int32_t* topk_ids, float* topk_w,
-                       void* workspace, size_t workspace_bytes, void* stream)
+// The forward's launch sequence; with TL (training) the routed logits and
+// [g | u] are kept, the down projection stores unweighted rows and the combine
+// applies the weights, and the routing results stay in the state (copied to
+// the caller's buffers when asked for).
+static cudaError_t run_forward(const moe_config& c, const void* x, const float* w_router,
+                               const float* router_bias, const float* selection_bias,
+                               const float* logit_noise, const void* w_gate, const void* w_up,
+                               const void* w_down, const void* w_gate_shared,
+                               const void* w_up_shared, const void* w_down_shared, void* y,
+                               float* losses, float* mean_prob, int32_t* counts, int32_t* topk_ids,
+                               float* topk_w, char* ws, const FwdLayout& F, const TrainLayout* TL,
+                               cudaStream_t s)
+{
+    const int64_t max_rows = max_rows_of(c);
+    const bool train = TL != nullptr;
+    int* status = reinterpret_cast<int*>(ws + F.ws.status);
+    int32_t* ids = (topk_ids && !train) ? topk_ids : reinterpret_cast<int32_t*>(ws + F.ids);
+    float* w = (topk_w && !train) ? topk_w : reinterpret_cast<float*>(ws + F.w);
+    int32_t* cnt = (counts && !train) ? counts : reinterpret_cast<int32_t*>(ws + F.counts);
+    int32_t* kept = reinterpret_cast<int32_t*>(ws + F.kept);
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + F.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + F.perm);
+    int32_t* row_of = reinterpret_cast<int32_t*>(ws + F.row_of);
+    void* x_perm = ws + F.x_perm;
+    void* h = ws + F.h;
+    void* y_perm = ws + F.y_perm;
+    float* logits_keep = train ? reinterpret_cast<float*>(ws + TL->logits) : nullptr;
+
+    trace(0, s);
+    const RouterPlan rp = router_plan(c);
+    cudaError_t e = launch_router(c, rp, x, w_router, router_bias, selection_bias, logit_noise,
+                                  nullptr, logits_keep, nullptr, ids, w, mean_prob, losses, ws,
+                                  F.ws, s);
+    trace(1, s);
+    if (e == cudaSuccess)
+        e = launch_dispatch_index(c, capacity_of(c), ids, cnt, kept, offsets, perm, row_of, ws,
+                                  F.ws, s);
+    trace(2, s);
+    if (e == cudaSuccess) e = launch_gather(c, x, row_of, x_perm, max_rows, status, s);
+    trace(3, s);
+    if (e == cudaSuccess)
+        e = launch_expert_ffn(c, max_rows, x_perm, offsets, train ? nullptr : perm,
+                              train ? nullptr : w, w_gate, w_up, w_down, h, y_perm,
+                              train ? ws + TL->gu : nullptr, status, s, trace_mid_ffn, nullptr);
+    trace(5, s);
+    const void* y_add = nullptr;
+    if (e == cudaSuccess && c.F_shared > 0) {
+        // the shared expert: one expert over every token, rows = x, weight 1
+        const moe_config cs = shared_config(c);
+        int32_t* sh_off = reinterpret_cast<int32_t*>(ws + F.sh_offsets);
+        set_row_range_kernel<<<1, 32, 0, s>>>(sh_off, (int32_t)c.T);
+        e = cudaGetLastError();
+        if (e == cudaSuccess)
+            e = launch_expert_ffn(cs, c.T, x, sh_off, nullptr, nullptr, w_gate_shared, w_up_shared,
+                                  w_down_shared, ws + F.sh_h, ws + F.sh_y,
+                                  train ? ws + TL->sh_gu : nullptr, status, s, nullptr, nullptr);
+        y_add = ws + F.sh_y;
+    }
+    trace(6, s);
+    if (e == cudaSuccess) e = launch_combine(c, y_perm, row_of, train ? w : nullptr, y_add, y, max_rows, s);
+    trace(7, s);
+    if (train && e == cudaSuccess) {  // the caller's copies of the routing results
+        const size_t tk = (size_t)c.T * c.K;
+        if (topk_ids) e = cudaMemcpyAsync(topk_ids, ids, tk * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess && topk_w)
+            e = cudaMemcpyAsync(topk_w, w, tk * sizeof(float), cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess && counts)
+            e = cudaMemcpyAsync(counts, cnt, (size_t)c.E * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    }
+    return e;
+}
+
+static moe_status check_forward_args(const moe_config* cfg, const void* x, const float* w_router,
+                                     const void* w_gate, const void* w_up, const void* w_down,
+                                     const void* w_gate_shared, const void* w_up_shared,
+                                     const void* w_down_shared, const void* y)
 {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
@@ -331,61 +464,160 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
         if (!aligned16(w_gate_shared) || !aligned16(w_up_shared) || !aligned16(w_down_shared))
             return MOE_ERR_ALIGN;
     }
-    const moe_config& c = *cfg;
-    const int64_t max_rows = max_rows_of(c);
-    const FwdLayout F = fwd_layout(c, max_rows);
+    return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
+                       const float* router_bias, const float* selection_bias,
+                       const float* logit_noise, const void* w_gate,
+                       const void* w_up, const void* w_down, const void* w_gate_shared,
+                       const void* w_up_shared, const void* w_down_shared, void* y, float* losses,
+                       float* mean_prob, int32_t* counts, int32_t* topk_ids, float* topk_w,
+                       void* workspace, size_t workspace_bytes, void* stream)
+{
+    moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
+                                       w_up_shared, w_down_shared, y);
+    if (st != MOE_OK) return st;
+    const FwdLayout F = fwd_layout(*cfg, max_rows_of(*cfg));
     st = check_ws(cfg, workspace, workspace_bytes, F.total);
     if (st != MOE_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    char* ws = static_cast<char*>(workspace);
-    int* status = reinterpret_cast<int*>(ws + F.ws.status);
-    int32_t* ids = topk_ids ? topk_ids : reinterpret_cast<int32_t*>(ws + F.ids);
-    float* w = topk_w ? topk_w : reinterpret_cast<float*>(ws + F.w);
-    int32_t* cnt = counts ? counts : reinterpret_cast<int32_t*>(ws + F.counts);
-    int32_t* kept = reinterpret_cast<int32_t*>(ws + F.kept);
-    int32_t* offsets = reinterpret_cast<int32_t*>(ws + F.offsets);
-    int32_t* perm = reinterpret_cast<int32_t*>(ws + F.perm);
-    int32_t* row_of = reinterpret_cast<int32_t*>(ws + F.row_of);
-    void* x_perm = ws + F.x_perm;
-    void* h = ws + F.h;
-    void* y_perm = ws + F.y_perm;
+    return cuda_status(run_forward(*cfg, x, w_router, router_bias, selection_bias, logit_noise,
+                                   w_gate, w_up, w_down, w_gate_shared, w_up_shared, w_down_shared,
+                                   y, losses, mean_prob, counts, topk_ids, topk_w,
+                                   static_cast<char*>(workspace), F, nullptr,
+                                   static_cast<cudaStream_t>(stream)));
+}
 
-    trace(0, s);
-    const RouterPlan rp = router_plan(c);
-    cudaError_t e = launch_router(c, rp, x, w_router, router_bias, selection_bias, logit_noise,
-                                  nullptr, nullptr, nullptr, ids, w, mean_prob, losses, ws, F.ws, s);
-    trace(1, s);
-    if (e == cudaSuccess)
-        e = launch_dispatch_index(c, capacity_of(c), ids, cnt, kept, offsets, perm, row_of, ws,
-                                  F.ws, s);
-    trace(2, s);
-    if (e == cudaSuccess) e = launch_gather(c, x, row_of, x_perm, max_rows, status, s);
-    trace(3, s);
-    if (e == cudaSuccess)
-        e = launch_expert_ffn(c, max_rows, x_perm, offsets, perm, w, w_gate, w_up, w_down, h,
-                              y_perm, status, s, trace_mid_ffn, nullptr);
-    trace(5, s);
-    const void* y_add = nullptr;
-    if (e == cudaSuccess && c.F_shared > 0) {
-        // the shared expert: one expert over every token, rows = x, weight 1
-        moe_config cs = c;
-        cs.E = 1;
-        cs.K = 1;
-        cs.F = c.F_shared;
-        cs.capacity_factor = 0.f;
-        cs.n_groups = 1;
-        int32_t* sh_off = reinterpret_cast<int32_t*>(ws + F.sh_offsets);
-        set_row_range_kernel<<<1, 32, 0, s>>>(sh_off, (int32_t)c.T);
-        e = cudaGetLastError();
-        if (e == cudaSuccess)
-            e = launch_expert_ffn(cs, c.T, x, sh_off, nullptr, nullptr, w_gate_shared, w_up_shared,
-                                  w_down_shared, ws + F.sh_h, ws + F.sh_y, status, s, nullptr,
-                                  nullptr);
-        y_add = ws + F.sh_y;
+moe_status moe_train_state_size(const moe_config* cfg, size_t* bytes)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_ARG;
+    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    *bytes = train_layout(*cfg, max_rows_of(*cfg)).total;
+    return MOE_OK;
+}
+
+moe_status moe_forward_train(const moe_config* cfg, const void* x, const float* w_router,
+                             const float* router_bias, const float* selection_bias,
+                             const float* logit_noise, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* w_gate_shared, const void* w_up_shared,
+                             const void* w_down_shared, void* y, float* losses, float* mean_prob,
+                             int32_t* counts, int32_t* topk_ids, float* topk_w, void* state,
+                             size_t state_bytes, void* stream)
+{
+    moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
+                                       w_up_shared, w_down_shared, y);
+    if (st != MOE_OK) return st;
+    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    const TrainLayout TL = train_layout(*cfg, max_rows_of(*cfg));
+    st = check_ws(cfg, state, state_bytes, TL.total);
+    if (st != MOE_OK) return st;
+    return cuda_status(run_forward(*cfg, x, w_router, router_bias, selection_bias, logit_noise,
+                                   w_gate, w_up, w_down, w_gate_shared, w_up_shared, w_down_shared,
+                                   y, losses, mean_prob, counts, topk_ids, topk_w,
+                                   static_cast<char*>(state), TL.f, &TL,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_ARG;
+    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    *bytes = bwd_layout(*cfg, max_rows_of(*cfg)).total;
+    return MOE_OK;
+}
+
+moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_router,
+                        const void* w_gate, const void* w_up, const void* w_down,
+                        const void* w_gate_shared, const void* w_up_shared,
+                        const void* w_down_shared, const void* state, size_t state_bytes,
+                        const void* dy, float c_balance, float c_z, void* dx, float* dw_router,
+                        float* db_router, float* dw_gate, float* dw_up, float* dw_down,
+                        float* dw_gate_shared, float* dw_up_shared, float* dw_down_shared,
+                        void* workspace, size_t workspace_bytes, void* stream)
+{
+    moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
+                                       w_up_shared, w_down_shared, dx);
+    if (st != MOE_OK) return st;
+    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!dy || !dw_router || !dw_gate || !dw_up || !dw_down) return MOE_ERR_ARG;
+    if (!aligned16(dy) || !aligned16(dw_gate) || !aligned16(dw_up) || !aligned16(dw_down))
+        return MOE_ERR_ALIGN;
+    if (cfg->F_shared > 0) {
+        if (!dw_gate_shared || !dw_up_shared || !dw_down_shared) return MOE_ERR_ARG;
+        if (!aligned16(dw_gate_shared) || !aligned16(dw_up_shared) || !aligned16(dw_down_shared))
+            return MOE_ERR_ALIGN;
     }
-    trace(6, s);
-    if (e == cudaSuccess) e = launch_combine(c, y_perm, row_of, y_add, y, max_rows, s);
-    trace(7, s);
+    if (!isfinite(c_balance) || !isfinite(c_z)) return MOE_ERR_ARG;
+    const moe_config& c = *cfg;
+    const int64_t max_rows = max_rows_of(c);
+    const TrainLayout TL = train_layout(c, max_rows);
+    st = check_ws(cfg, state, state_bytes, TL.total);
+    if (st != MOE_OK) return st;
+    const BwdLayout B = bwd_layout(c, max_rows);
+    st = check_ws(cfg, workspace, workspace_bytes, B.total);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const char* sv = static_cast<const char*>(state);
+    char* ws = static_cast<char*>(workspace);
+    const FwdLayout& F = TL.f;
+    int* status = reinterpret_cast<int*>(ws + B.status);
+    const int32_t* ids = reinterpret_cast<const int32_t*>(sv + F.ids);
+    const float* w = reinterpret_cast<const float*>(sv + F.w);
+    const int32_t* cnt = reinterpret_cast<const int32_t*>(sv + F.counts);
+    const int32_t* offsets = reinterpret_cast<const int32_t*>(sv + F.offsets);
+    const int32_t* perm = reinterpret_cast<const int32_t*>(sv + F.perm);
+    const int32_t* row_of = reinterpret_cast<const int32_t*>(sv + F.row_of);
+    const float* logits = reinterpret_cast<const float*>(sv + TL.logits);
+    float* dw_row = reinterpret_cast<float*>(ws + B.dw_row);
+    float* dlogits = reinterpret_cast<float*>(ws + B.dlogits);
+
+    btrace(0, s);
+    cudaError_t e = launch_bwd_rows(c, dy, sv + F.y_perm, offsets, perm, w, ws + B.dyp, dw_row,
+                                    max_rows, status, s);
+    btrace(1, s);
+    if (e == cudaSuccess)
+        e = launch_router_bwd(c, logits, ids, row_of, dw_row, cnt, c_balance, c_z, dlogits,
+                              max_rows, status, s);
+    btrace(2, s);
+    if (e == cudaSuccess)  // dH -> [dg | du], then dXp (boundary 3 between the two)
+        e = launch_dgrad_tc_bf16(c, max_rows, ws + B.dyp, offsets, sv + TL.gu, w_gate, w_up, w_down,
+                                 ws + B.dgu, ws + B.dxp, status, s, btrace_mid_dgrad, nullptr);
+    btrace(4, s);
+    if (e == cudaSuccess)  // dWd = h^T dYp
+        e = launch_wgrad_tc_bf16(c.E, max_rows, offsets, sv + F.h, c.F, ws + B.dyp, c.D, 1, dw_down,
+                                 nullptr, status, s);
+    btrace(5, s);
+    if (e == cudaSuccess)  // [dWg | dWu] = x_perm^T [dg | du]
+        e = launch_wgrad_tc_bf16(c.E, max_rows, offsets, sv + F.x_perm, c.D, ws + B.dgu, c.F, 2,
+                                 dw_gate, dw_up, status, s);
+    btrace(6, s);
+    const void* dx_shared = nullptr;
+    if (e == cudaSuccess && c.F_shared > 0) {
+        const moe_config cs = shared_config(c);
+        const int32_t* sh_off = reinterpret_cast<const int32_t*>(sv + F.sh_offsets);
+        e = launch_dgrad_tc_bf16(cs, c.T, dy, sh_off, sv + TL.sh_gu, w_gate_shared, w_up_shared,
+                                 w_down_shared, ws + B.sh_dgu, ws + B.sh_dx, status, s, nullptr,
+                                 nullptr);
+        if (e == cudaSuccess)
+            e = launch_wgrad_tc_bf16(1, c.T, sh_off, sv + F.sh_h, c.F_shared, dy, c.D, 1,
+                                     dw_down_shared, nullptr, status, s);
+        if (e == cudaSuccess)
+            e = launch_wgrad_tc_bf16(1, c.T, sh_off, x, c.D, ws + B.sh_dgu, c.F_shared, 2,
+                                     dw_gate_shared, dw_up_shared, status, s);
+        dx_shared = ws + B.sh_dx;
+    }
+    btrace(7, s);
+    if (e == cudaSuccess)
+        e = launch_router_wgrad(c, x, dlogits, reinterpret_cast<float*>(ws + B.rw_part), B.rw_splits,
+                                dw_router, db_router, s);
+    btrace(8, s);
+    if (e == cudaSuccess)
+        e = launch_dx_assemble(c, dlogits, w_router, ws + B.dxp, row_of, dx_shared, dx, max_rows, s);
+    btrace(9, s);
     return cuda_status(e);
 }
 
@@ -427,6 +659,30 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
     const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
     if (router_tc_eligible(*cfg)) return 11 + shared;  // split weights, fused router, 2 reductions
     return 11 + shared + (router_plan(*cfg).splits > 1 ? 1 : 0);
+}
+
+int32_t moe_backward_kernel_count(const moe_config* cfg)
+{
+    if (check_config(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;
+    // rows, router, two dgrad GEMMs, two wgrad GEMMs, router weight partials
+    // and their sum, dx; the shared expert adds its two dgrad and two wgrad GEMMs
+    return 9 + (cfg->F_shared > 0 ? 4 : 0);
+}
+
+moe_status moe_trace_attach_backward(void* const* events, int32_t n_events)
+{
+    if (n_events < 0 || n_events > 16 || (n_events > 0 && events == nullptr)) return MOE_ERR_ARG;
+    for (int i = 0; i < 16; ++i) g_btrace[i] = i < n_events ? events[i] : nullptr;
+    g_btrace_n = n_events;
+    return MOE_OK;
+}
+
+int32_t moe_trace_backward_boundary_count(void) { return 10; }
+
+const char* moe_trace_backward_stage_name(int32_t boundary)
+{
+    if (boundary < 0 || boundary >= 10) return "";
+    return kBwdStageNames[boundary];
 }
 
 moe_status moe_trace_attach(void* const* events, int32_t n_events)

@@ -1,0 +1,438 @@
+// bwd.cu -- the memory-bound steps of the layer's backward.
+//
+// "Lab: build a tiny MoE in PyTorch", "Smoke test and backward pass": the
+// training loss main + c_bal * balance + c_z * z is differentiated through
+// the layer; "2.9 Mixture-of-Experts (MoE) Architectures", "The Router": the
+// top-k index decision is a stop-gradient, so the router learns only through
+// the kept gate weights and the auxiliary losses.  With dY the gradient of y:
+//
+//   rows       dYp[r] = bf16(w_r * dY[t_r]),  dw_r = <dY[t_r], o_r>
+//              (o_r = the expert's unweighted output the forward kept)
+//   router     dL[t] from the gate weights' dw (renormalised or not, route
+//              scale), the balance loss through the normalised scores (counts
+//              fixed) and the z-loss through the logsumexp
+//   linear     dW_r = x^T dL,  db = sum_t dL[t]   (split over tokens, then a
+//              fixed-order sum: deterministic)
+//   dx         dx[t] = dL[t] W_r^T + sum over kept slots of dXp[row] (+ the
+//              shared expert's), rounded once
+// No atomics anywhere: every result is bit-reproducible.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------- rows --
+// One warp per row of the expert-major layout; 16-byte vectors of 8 bf16.
+__global__ void __launch_bounds__(256) bwd_rows_kernel(const uint4* __restrict__ dy,
+                                                       const uint4* __restrict__ o,
+                                                       const int32_t* __restrict__ offsets,
+                                                       const int32_t* __restrict__ perm,
+                                                       const float* __restrict__ topk_w,
+                                                       uint4* __restrict__ dyp, float* __restrict__ dw_row,
+                                                       int E, int K, int64_t vpr, int64_t nk,
+                                                       int64_t max_rows, int* status)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    int64_t rows = offsets[E];
+    if (rows > max_rows || rows < 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_flag(status, kFlagBounds, 600);
+        rows = rows < 0 ? 0 : max_rows;
+    }
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int32_t pa = perm[r];
+        if (pa < 0 || (int64_t)pa >= nk) {
+            if (lane == 0) raise_flag(status, kFlagBounds, 601);
+            continue;
+        }
+        const int64_t t = pa / K;
+        const float w = topk_w[pa];
+        const uint4* dyt = dy + t * vpr;
+        const uint4* orow = o + r * vpr;
+        uint4* drow = dyp + r * vpr;
+        float dot = 0.f;
+        for (int64_t v = lane; v < vpr; v += 32) {
+            const uint4 a = __ldg(dyt + v), b = __ldg(orow + v);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+            uint32_t pw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a0 = __uint_as_float(aw[i] << 16), a1 = __uint_as_float(aw[i] & 0xffff0000u);
+                const float b0 = __uint_as_float(bw[i] << 16), b1 = __uint_as_float(bw[i] & 0xffff0000u);
+                dot = fmaf(a0, b0, dot);
+                dot = fmaf(a1, b1, dot);
+                pw[i] = pack_bf16x2(w * a0, w * a1);
+            }
+            drow[v] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        }
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
+        if (lane == 0) dw_row[r] = dot;
+    }
+}
+
+// ----------------------------------------------------------------- router --
+constexpr int kMaxEPerLane = 8;  // E <= 256 = 32 lanes x 8
+
+MOE_DEVICE float warp_sum(float v)
+{
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+    return v;
+}
+
+MOE_DEVICE float warp_max(float v)
+{
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, s));
+    return v;
+}
+
+// One warp per token; lane l holds experts l, l + 32, ...
+__global__ void __launch_bounds__(256) router_bwd_kernel(const float* __restrict__ logits,
+                                                         const int32_t* __restrict__ ids,
+                                                         const int32_t* __restrict__ row_of,
+                                                         const float* __restrict__ dw_row,
+                                                         const int32_t* __restrict__ counts,
+                                                         float* __restrict__ dlogits, int64_t T, int E,
+                                                         int K, int score_func, int renorm,
+                                                         float route_scale, float c_bal, float c_z,
+                                                         int64_t max_rows, int* status)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* L = logits + t * E;
+    float l[kMaxEPerLane];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kMaxEPerLane; ++j) {
+        const int e = lane + 32 * j;
+        l[j] = e < E ? L[e] : -INFINITY;
+        mx = fmaxf(mx, l[j]);
+    }
+    mx = warp_max(mx);
+    float se = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxEPerLane; ++j) se += (lane + 32 * j < E) ? expf(l[j] - mx) : 0.f;
+    se = warp_sum(se);
+    const float lse = mx + logf(se);
+    const bool sig = score_func == 1;
+    // gate weights: every lane evaluates the K chosen scores itself
+    float S = 0.f, sdw = 0.f;
+    int idk[8];
+    float dwk[8], sck[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        idk[k] = -1;
+        dwk[k] = 0.f;
+        sck[k] = 0.f;
+        if (k < K) {
+            int id = ids[t * K + k];
+            if (id < 0 || id >= E) {
+                if (lane == 0) raise_flag(status, kFlagBounds, 610);
+                continue;
+            }
+            idk[k] = id;
+            const float li = L[id];
+            sck[k] = sig ? 1.f / (1.f + expf(-li)) : expf(li - mx) / se;
+            const int32_t r = row_of[t * K + k];
+            dwk[k] = (r >= 0 && r < max_rows) ? dw_row[r] : 0.f;  // a dropped slot: 0
+            S += sck[k];
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sdw += dwk[k] * sck[k] / S;
+    float p[kMaxEPerLane], sc[kMaxEPerLane], ds[kMaxEPerLane];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxEPerLane; ++j) {
+        const int e = lane + 32 * j;
+        const bool in = e < E;
+        p[j] = in ? expf(l[j] - mx) / se : 0.f;
+        sc[j] = in ? (sig ? 1.f / (1.f + expf(-l[j])) : p[j]) : 0.f;
+        ss += sc[j];
+        float d = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (idk[k] == e) d += renorm ? route_scale / S * (dwk[k] - sdw) : route_scale * dwk[k];
+        ds[j] = d;
+    }
+    // the balance loss: d n[e] = c_bal * E * f_e / T, f_e = counts_e / (T K)
+    const float bal_scale = c_bal * (float)E / ((float)T * (float)K) / (float)T;
+    if (sig) {
+        ss = warp_sum(ss);
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxEPerLane; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) dot += bal_scale * (float)counts[e] * (sc[j] / ss);
+        }
+        dot = warp_sum(dot);
+#pragma unroll
+        for (int j = 0; j < kMaxEPerLane; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) ds[j] += (bal_scale * (float)counts[e] - dot) / ss;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kMaxEPerLane; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) ds[j] += bal_scale * (float)counts[e];
+        }
+    }
+    // the scores from the logits, then the z-loss
+    float dot2 = 0.f;
+    if (!sig) {
+#pragma unroll
+        for (int j = 0; j < kMaxEPerLane; ++j) dot2 += p[j] * ds[j];
+        dot2 = warp_sum(dot2);
+    }
+    const float zc = c_z * 2.f * lse / (float)T;
+#pragma unroll
+    for (int j = 0; j < kMaxEPerLane; ++j) {
+        const int e = lane + 32 * j;
+        if (e >= E) continue;
+        const float g = sig ? ds[j] * sc[j] * (1.f - sc[j]) : p[j] * (ds[j] - dot2);
+        dlogits[t * E + e] = g + zc * p[j];
+    }
+}
+
+// ---------------------------------------------------- router weight grads --
+// part[s][d][e] = sum over the tokens of split s of x[t,d] * dL[t,e]; row d = D
+// of part takes x = 1 (the bias gradient).  Block: 64 d x ET experts, a token
+// chunk of the split staged through shared memory 64 tokens at a time.
+template <typename XT, int ET>
+__global__ void __launch_bounds__(256) router_wgrad_partial_kernel(const XT* __restrict__ x,
+                                                                   const float* __restrict__ dL,
+                                                                   float* __restrict__ part, int64_t T,
+                                                                   int D, int E, int64_t t_per_split)
+{
+    constexpr int EPT = ET / 4;  // experts per thread
+    __shared__ float sdl[64][ET];
+    const int dl = threadIdx.x & 63, eg = threadIdx.x >> 6;
+    const int d = blockIdx.x * 64 + dl;
+    const int e0 = blockIdx.y * ET;
+    const int64_t t0 = (int64_t)blockIdx.z * t_per_split;
+    const int64_t t1 = t0 + t_per_split < T ? t0 + t_per_split : T;
+    float acc[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) acc[j] = 0.f;
+    for (int64_t tc = t0; tc < t1; tc += 64) {
+        for (int i = threadIdx.x; i < 64 * ET; i += 256) {
+            const int tt = i / ET, ee = i - tt * ET;
+            const int64_t t = tc + tt;
+            sdl[tt][ee] = (t < t1 && e0 + ee < E) ? dL[t * E + e0 + ee] : 0.f;
+        }
+        __syncthreads();
+        const int n = (int)(t1 - tc < 64 ? t1 - tc : 64);
+        if (d <= D) {
+#pragma unroll 4
+            for (int i = 0; i < n; ++i) {
+                const float xv = d < D ? to_f32(x[(tc + i) * D + d]) : 1.f;
+#pragma unroll
+                for (int j = 0; j < EPT; ++j) acc[j] = fmaf(xv, sdl[i][eg * EPT + j], acc[j]);
+            }
+        }
+        __syncthreads();
+    }
+    if (d <= D) {
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            const int e = e0 + eg * EPT + j;
+            if (e < E) part[((int64_t)blockIdx.z * (D + 1) + d) * E + e] = acc[j];
+        }
+    }
+}
+
+// dW[d][e] = sum over splits in order; row D goes to db (may be null).
+__global__ void router_wgrad_reduce_kernel(const float* __restrict__ part, int splits, int D, int E,
+                                           float* __restrict__ dw, float* __restrict__ db)
+{
+    const int64_t n = (int64_t)(D + 1) * E;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float s = 0.f;
+        for (int k = 0; k < splits; ++k) s += part[(int64_t)k * n + i];
+        if (i < (int64_t)D * E) dw[i] = s;
+        else if (db) db[i - (int64_t)D * E] = s;
+    }
+}
+
+// --------------------------------------------------------------------- dx --
+// Block: 16 tokens x 256 d; warp w owns tokens 2w, 2w+1, lane l the columns
+// l, l + 32, ..., l + 224 of the tile (so the shared-memory reads of W_r are
+// conflict-free).  The router term dL W_r^T is accumulated through shared
+// memory in chunks of 32 experts, then the token's kept rows of dXp (slot
+// order) and the shared expert's row are added, and the sum is rounded once.
+constexpr int kDxTok = 16;
+constexpr int kDxCols = 256;
+
+template <typename ET>
+__global__ void __launch_bounds__(256) dx_assemble_kernel(const float* __restrict__ dL,
+                                                          const float* __restrict__ w_r,
+                                                          const ET* __restrict__ dxp,
+                                                          const int32_t* __restrict__ row_of,
+                                                          const ET* __restrict__ dx_shared,
+                                                          ET* __restrict__ dx, int64_t T, int D, int E,
+                                                          int K, int64_t max_rows)
+{
+    __shared__ float swr[kDxCols][33];
+    __shared__ float sdl[kDxTok][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t tb = (int64_t)blockIdx.x * kDxTok;
+    const int d0 = blockIdx.y * kDxCols;
+    float acc[2][8];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        for (int i = threadIdx.x; i < kDxCols * 32; i += 256) {
+            const int dd = i >> 5, ee = i & 31;
+            swr[dd][ee] = (d0 + dd < D && e0 + ee < E) ? w_r[(int64_t)(d0 + dd) * E + e0 + ee] : 0.f;
+        }
+        for (int i = threadIdx.x; i < kDxTok * 32; i += 256) {
+            const int tt = i >> 5, ee = i & 31;
+            sdl[tt][ee] = (tb + tt < T && e0 + ee < E) ? dL[(tb + tt) * E + e0 + ee] : 0.f;
+        }
+        __syncthreads();
+        const int ne = E - e0 < 32 ? E - e0 : 32;
+        for (int ee = 0; ee < ne; ++ee) {
+            const float g0 = sdl[2 * warp][ee], g1 = sdl[2 * warp + 1][ee];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float wv = swr[lane + 32 * j][ee];
+                acc[0][j] = fmaf(g0, wv, acc[0][j]);
+                acc[1][j] = fmaf(g1, wv, acc[1][j]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int64_t t = tb + 2 * warp + i;
+        if (t >= T) break;
+        for (int k = 0; k < K; ++k) {
+            const int32_t r = row_of[t * K + k];
+            if (r < 0 || r >= max_rows) continue;
+            const ET* src = dxp + (int64_t)r * D + d0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (d0 + lane + 32 * j < D) acc[i][j] += to_f32(src[lane + 32 * j]);
+        }
+        if (dx_shared) {
+            const ET* src = dx_shared + t * D + d0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (d0 + lane + 32 * j < D) acc[i][j] += to_f32(src[lane + 32 * j]);
+        }
+        ET* dst = dx + t * D + d0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (d0 + lane + 32 * j < D) dst[lane + 32 * j] = from_f32<ET>(acc[i][j]);
+    }
+}
+
+// ------------------------------------------------------------------ host --
+static int sm_count()
+{
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+cudaError_t launch_bwd_rows(const moe_config& c, const void* dy, const void* o, const int32_t* offsets,
+                            const int32_t* perm, const float* topk_w, void* dyp, float* dw_row,
+                            int64_t max_rows, int* status, cudaStream_t s)
+{
+    const int64_t vpr = (int64_t)c.D * 2 / 16;  // bf16 rows
+    int64_t blocks = (max_rows + 7) / 8;
+    const int64_t cap = (int64_t)sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    bwd_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+        static_cast<const uint4*>(dy), static_cast<const uint4*>(o), offsets, perm, topk_w,
+        static_cast<uint4*>(dyp), dw_row, c.E, c.K, vpr, c.T * c.K, max_rows, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_bwd(const moe_config& c, const float* logits, const int32_t* ids,
+                              const int32_t* row_of, const float* dw_row, const int32_t* counts,
+                              float c_bal, float c_z, float* dlogits, int64_t max_rows, int* status,
+                              cudaStream_t s)
+{
+    const int64_t blocks = (c.T + 7) / 8;
+    router_bwd_kernel<<<(unsigned)blocks, 256, 0, s>>>(logits, ids, row_of, dw_row, counts, dlogits,
+                                                        c.T, c.E, c.K, c.score_func, c.renormalize,
+                                                        c.route_scale, c_bal, c_z, max_rows, status);
+    return cudaGetLastError();
+}
+
+int router_wgrad_splits(const moe_config& c)
+{
+    // enough blocks to fill the GPU a few times; each split at least 256 tokens
+    const int64_t dblocks = (c.D + 1 + 63) / 64;
+    const int64_t eblocks = c.E <= 8 ? 1 : (c.E + 31) / 32;
+    int64_t want = (int64_t)sm_count() * 4 / (dblocks * eblocks);
+    int64_t most = (c.T + 255) / 256;
+    int64_t sp = want < most ? want : most;
+    if (sp < 1) sp = 1;
+    if (sp > 64) sp = 64;
+    return (int)sp;
+}
+
+size_t router_wgrad_part_bytes(const moe_config& c, int splits)
+{
+    return (size_t)splits * (size_t)(c.D + 1) * c.E * sizeof(float);
+}
+
+cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float* dL, float* part,
+                                int splits, float* dw, float* db, cudaStream_t s)
+{
+    const int64_t tps = (c.T + splits - 1) / splits;
+    const dim3 grid((unsigned)((c.D + 1 + 63) / 64), 1, (unsigned)splits);
+    if (c.E <= 8) {
+        if (c.dtype == MOE_BF16)
+            router_wgrad_partial_kernel<__nv_bfloat16, 8><<<grid, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(x), dL, part, c.T, c.D, c.E, tps);
+        else
+            router_wgrad_partial_kernel<float, 8><<<grid, 256, 0, s>>>(static_cast<const float*>(x), dL,
+                                                                       part, c.T, c.D, c.E, tps);
+    } else {
+        const dim3 g2(grid.x, (unsigned)((c.E + 31) / 32), grid.z);
+        if (c.dtype == MOE_BF16)
+            router_wgrad_partial_kernel<__nv_bfloat16, 32><<<g2, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(x), dL, part, c.T, c.D, c.E, tps);
+        else
+            router_wgrad_partial_kernel<float, 32><<<g2, 256, 0, s>>>(static_cast<const float*>(x), dL,
+                                                                      part, c.T, c.D, c.E, tps);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t n = (int64_t)(c.D + 1) * c.E;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    router_wgrad_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(part, splits, c.D, c.E, dw, db);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float* w_r, const void* dxp,
+                               const int32_t* row_of, const void* dx_shared, void* dx,
+                               int64_t max_rows, cudaStream_t s)
+{
+    const dim3 grid((unsigned)((c.T + kDxTok - 1) / kDxTok), (unsigned)((c.D + kDxCols - 1) / kDxCols));
+    if (c.dtype == MOE_BF16)
+        dx_assemble_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            dL, w_r, static_cast<const __nv_bfloat16*>(dxp), row_of,
+            static_cast<const __nv_bfloat16*>(dx_shared), static_cast<__nv_bfloat16*>(dx), c.T, c.D,
+            c.E, c.K, max_rows);
+    else
+        dx_assemble_kernel<float><<<grid, 256, 0, s>>>(dL, w_r, static_cast<const float*>(dxp), row_of,
+                                                       static_cast<const float*>(dx_shared),
+                                                       static_cast<float*>(dx), c.T, c.D, c.E, c.K,
+                                                       max_rows);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

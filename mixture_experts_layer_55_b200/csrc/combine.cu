@@ -6,9 +6,11 @@
 // nothing, so an all-dropped token gets zero; section "Add a shared expert":
 // a shared expert's output is added to the routed output.
 //
-// The routing weight is already applied by the down GEMM's epilogue, so the
+// The routing weight is normally applied by the down GEMM's epilogue, so the
 // combine is a plain gather-sum: 16-byte vector loads of the token's K rows of
-// y_perm, summed in slot order in fp32 and rounded once.
+// y_perm, summed in slot order in fp32 and rounded once.  The training forward
+// keeps the expert outputs unweighted (the backward needs them), and then the
+// combine multiplies each row by its slot's weight as it adds it.
 // No atomics: the result is deterministic.
 #include "common.cuh"
 #include "internal.h"
@@ -24,6 +26,13 @@ template <> struct Vec<float> {
         a[1] += __uint_as_float(v.y);
         a[2] += __uint_as_float(v.z);
         a[3] += __uint_as_float(v.w);
+    }
+    MOE_DEVICE static void add_scaled(float (&a)[8], const uint4& v, float w)
+    {
+        a[0] = fmaf(w, __uint_as_float(v.x), a[0]);
+        a[1] = fmaf(w, __uint_as_float(v.y), a[1]);
+        a[2] = fmaf(w, __uint_as_float(v.z), a[2]);
+        a[3] = fmaf(w, __uint_as_float(v.w), a[3]);
     }
     MOE_DEVICE static uint4 pack(const float (&a)[8])
     {
@@ -42,6 +51,15 @@ template <> struct Vec<__nv_bfloat16> {
             a[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
         }
     }
+    MOE_DEVICE static void add_scaled(float (&a)[8], const uint4& v, float w)
+    {
+        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[2 * i] = fmaf(w, __uint_as_float(x[i] << 16), a[2 * i]);
+            a[2 * i + 1] = fmaf(w, __uint_as_float(x[i] & 0xffff0000u), a[2 * i + 1]);
+        }
+    }
     MOE_DEVICE static uint4 pack(const float (&a)[8])
     {
         return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
@@ -57,6 +75,7 @@ template <> struct Vec<__nv_bfloat16> {
 template <typename ET, int KS>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ row_of,
+                                                      const float* __restrict__ slot_w,
                                                       const uint4* __restrict__ y_add,
                                                       uint4* __restrict__ y, int64_t T, int K,
                                                       int64_t vec_per_row, int64_t max_rows)
@@ -87,9 +106,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
             if (i >= n) break;
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (y_add) Vec<ET>::add(acc, __ldg(y_add + i));  // shared expert output first
+            const int64_t t = i / vec_per_row;
 #pragma unroll
             for (int k = 0; k < KS; ++k)
-                if (rows[u][k] >= 0) Vec<ET>::add(acc, vals[u][k]);  // slot order
+                if (rows[u][k] >= 0) {  // slot order
+                    if (slot_w) Vec<ET>::add_scaled(acc, vals[u][k], __ldg(slot_w + t * K + k));
+                    else Vec<ET>::add(acc, vals[u][k]);
+                }
             y[i] = Vec<ET>::pack(acc);
         }
     }
@@ -97,28 +120,29 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 
 template <typename ET>
 static void launch_combine_t(const moe_config& c, int64_t blocks, const void* y_perm,
-                             const int32_t* row_of, const void* y_add, void* y, int64_t vpr,
-                             int64_t max_rows, cudaStream_t s)
+                             const int32_t* row_of, const float* slot_w, const void* y_add, void* y,
+                             int64_t vpr, int64_t max_rows, cudaStream_t s)
 {
     const uint4* src = static_cast<const uint4*>(y_perm);
     const uint4* add = static_cast<const uint4*>(y_add);
     uint4* dst = static_cast<uint4*>(y);
     if (c.K <= 1)
-        combine_kernel<ET, 1><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+        combine_kernel<ET, 1><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
                                                                 max_rows);
     else if (c.K == 2)
-        combine_kernel<ET, 2><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+        combine_kernel<ET, 2><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
                                                                 max_rows);
     else if (c.K <= 4)
-        combine_kernel<ET, 4><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+        combine_kernel<ET, 4><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
                                                                 max_rows);
     else
-        combine_kernel<ET, 8><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, add, dst, c.T, c.K, vpr,
+        combine_kernel<ET, 8><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
                                                                 max_rows);
 }
 
 cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
-                           const void* y_add, void* y, int64_t max_rows, cudaStream_t s)
+                           const float* slot_w, const void* y_add, void* y, int64_t max_rows,
+                           cudaStream_t s)
 {
     const int64_t row_bytes = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4);
     const int64_t vpr = row_bytes / 16;
@@ -131,9 +155,9 @@ cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (c.dtype == MOE_BF16)
-        launch_combine_t<__nv_bfloat16>(c, blocks, y_perm, row_of, y_add, y, vpr, max_rows, s);
+        launch_combine_t<__nv_bfloat16>(c, blocks, y_perm, row_of, slot_w, y_add, y, vpr, max_rows, s);
     else
-        launch_combine_t<float>(c, blocks, y_perm, row_of, y_add, y, vpr, max_rows, s);
+        launch_combine_t<float>(c, blocks, y_perm, row_of, slot_w, y_add, y, vpr, max_rows, s);
     return cudaGetLastError();
 }
 

@@ -12,6 +12,14 @@
 //   down:     Y = h[block] . Wd_e                       (K = F)
 //             y_perm = bf16(topk_w[perm[row]] * Y)      (epilogue)
 //
+// and the two data-gradient contractions of the backward ("Lab: build a tiny
+// MoE in PyTorch", "Smoke test and backward pass"), on the same tiles:
+//
+//   dgrad-h:  dH = dYp[block] . Wd_e^T                  (K = D; Wd_e read K-major)
+//             [dg | du] = bf16(dH * u * silu'(g) | dH * silu(g))
+//                         (epilogue; g, u = the forward's saved pre-activations)
+//   dgrad-x:  dXp = [dg | du][block] . [Wg_e | Wu_e]^T  (K = 2F; both read K-major)
+//
 // Persistent kernel, one CTA per SM, either alone (M = 128 rows per tile,
 // cta_group::1) or as a CTA pair on two SMs (M = 256, cta_group::2: each CTA
 // holds its 128 rows of A and half of B's columns, the leader issues the MMAs
@@ -53,12 +61,17 @@ constexpr int MAX_E = 256;
 // Tile geometry.  Single CTA: M = 128 rows, all N columns of the tile's B in
 // this CTA (gate/up: 128 gate + 128 up; down: 256).  CTA pair: M = 256 rows,
 // 128 per CTA, and each CTA holds half of every B tile's columns.
-template <bool GATEUP, bool PAIR> struct Geo {
+// Contraction modes (the template argument; the forward's values are 0 and 1).
+enum : int { kDown = 0, kGateUp = 1, kDgradH = 2, kDgradX = 3 };
+
+template <int MODE, bool PAIR> struct Geo {
+    static constexpr bool GATEUP = MODE == kGateUp;
+    static constexpr bool B_KMAJOR = MODE == kDgradH || MODE == kDgradX;  // B = a weight, transposed
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BM = 128 * CTAS;                  // rows per tile
     static constexpr int BN = GATEUP ? 128 : 256;          // output columns per tile
-    static constexpr int B_BOXES = (GATEUP ? 2 * 128 : 256) / 64 / CTAS;  // B boxes per CTA per stage
-    static constexpr int B_BYTES = B_BOXES * BOX_BYTES;
+    static constexpr int B_BOXES = 256 / 64 / CTAS;        // 64-wide B boxes per CTA per stage
+    static constexpr int B_BYTES = B_BOXES * BOX_BYTES;    // (K-major B: one box of 256/CTAS rows)
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB single, 32 KB pair
     static constexpr int STAGES = PAIR ? 6 : 4;
     static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;  // one per epilogue warp
@@ -77,10 +90,10 @@ struct Misc {
     int pref[MAX_E + 1];  // first tile index of each expert; pref[E] = total tiles
 };
 
-template <bool GATEUP, bool PAIR>
+template <int MODE, bool PAIR>
 constexpr size_t smem_bytes()
 {
-    return 1024 /*alignment slack*/ + (size_t)Geo<GATEUP, PAIR>::STAGES * Geo<GATEUP, PAIR>::STAGE_BYTES +
+    return 1024 /*alignment slack*/ + (size_t)Geo<MODE, PAIR>::STAGES * Geo<MODE, PAIR>::STAGE_BYTES +
            sizeof(Misc);
 }
 
@@ -88,13 +101,16 @@ struct Args {
     const int32_t* offsets;
     const int32_t* perm;
     const float* topk_w;
-    __nv_bfloat16* out;  // h (gate/up) or y_perm (down), row-major (max_rows, N)
+    __nv_bfloat16* out;  // h (gate/up), y_perm (down), [dg | du] (dgrad-h), dXp (dgrad-x)
     int E;
-    int Kdim;            // D for gate/up, F for down
-    int N;               // F for gate/up, D for down
+    int Kdim;            // D for gate/up and dgrad-h, F for down and for each half of dgrad-x
+    int N;               // F for gate/up and dgrad-h, D for down and dgrad-x
     int n_tiles;         // ceil(N / BN)
+    int64_t ldo;         // row stride of out in elements (N; 2N for dgrad-h)
     int64_t max_rows;
     int64_t nk;          // T * K (range of perm values)
+    __nv_bfloat16* gu_out;       // gate/up: keep [g | u] here, row stride 2N (null: do not)
+    const __nv_bfloat16* gu_in;  // dgrad-h: the kept [g | u], row stride 2N
     int* status;
 };
 
@@ -116,12 +132,22 @@ MOE_DEVICE void decode_tile(const Misc* m, int E, int bm, int bn, int t, int& e,
     n0 = n * bn;
 }
 
-template <bool GATEUP, bool PAIR>
+// silu(g) and its derivative s + g s (1 - s), s = sigmoid(g), in fp32 for the
+// backward's epilogue (the exponent is clamped where s underflows anyway).
+MOE_DEVICE void silu_and_grad(float g, float& silu, float& dsilu)
+{
+    const float s = __fdividef(1.0f, 1.0f + __expf(fminf(-g, 80.0f)));
+    silu = g * s;
+    dsilu = fmaf(g * s, 1.0f - s, s);
+}
+
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                   const __grid_constant__ CUtensorMap tmB1, const Args a)
 {
-    using G = Geo<GATEUP, PAIR>;
+    using G = Geo<MODE, PAIR>;
+    constexpr bool GATEUP = G::GATEUP;
     constexpr int BM = G::BM, BN = G::BN, STAGES = G::STAGES, STAGE_BYTES = G::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -148,7 +174,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB0);
-        if (GATEUP) prefetch_tmap(&tmB1);
+        if (GATEUP || MODE == kDgradX) prefetch_tmap(&tmB1);
     }
     if (warp == 1) {
         if (PAIR) {
@@ -187,7 +213,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
     const int total = m->pref[E];
-    const int num_kb = (a.Kdim + BK - 1) / BK;
+    const int kh = (a.Kdim + BK - 1) / BK;                  // K blocks (per half for dgrad-x)
+    const int num_kb = MODE == kDgradX ? 2 * kh : kh;
     volatile int* abort_flag = &m->abort_flag;
 
     if (warp == 0 && lane == 0) {
@@ -209,7 +236,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
                 uint8_t* sB = sA + A_BYTES;
                 const int k0 = kb * BK;
-                if (PAIR) {
+                if (MODE == kDgradX) {
+                    // K = [dg | du]: half 0 against Wg, half 1 against Wu (each K-major)
+                    const int hf = kb >= kh ? 1 : 0;
+                    const int kk0 = (kb - hf * kh) * BK;
+                    const CUtensorMap* mb = hf ? &tmB1 : &tmB0;
+                    if (PAIR) {
+                        if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
+                        const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
+                        tma_load_3d_pair(sA, &tmA, kk0, hf, a_row, fb);
+                        tma_load_3d_pair(sB, mb, kk0, n0 + 128 * (int)rank, e, fb);
+                    } else {
+                        uint64_t* fb = &m->full[stage];
+                        mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                        tma_load_3d(sA, &tmA, kk0, hf, a_row, fb);
+                        tma_load_3d(sB, mb, kk0, n0, e, fb);
+                    }
+                } else if (MODE == kDgradH) {
+                    // B = Wd_e read K-major: rows n (= f) of 64 K (= d) elements
+                    if (PAIR) {
+                        if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
+                        const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
+                        tma_load_2d_pair(sA, &tmA, k0, a_row, fb);
+                        tma_load_3d_pair(sB, &tmB0, k0, n0 + 128 * (int)rank, e, fb);
+                    } else {
+                        uint64_t* fb = &m->full[stage];
+                        mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                        tma_load_2d(sA, &tmA, k0, a_row, fb);
+                        tma_load_3d(sB, &tmB0, k0, n0, e, fb);
+                    }
+                } else if (PAIR) {
                     // both CTAs' bytes are counted on the leader's full barrier
                     if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
                     const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
@@ -249,7 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 411, nullptr);
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ------------------------------------------------ MMA issuer (leader only)
-        constexpr uint32_t idesc = umma_idesc_bf16(BM, 256, 0, 1);
+        constexpr uint32_t idesc = umma_idesc_bf16(BM, 256, 0, G::B_KMAJOR ? 0 : 1);
         // B: N-major; 64-column blocks 8 KB apart (LBO), 8-row K groups 1024 B apart (SBO)
         int stage = 0;
         uint32_t phase = 0;
@@ -274,8 +330,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     // A: K-major, 8-row groups 1024 B apart; +32 B per 16-element K step
                     const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
                     // one N = 256 MMA: the 64-column boxes of B (for gate/up,
-                    // gate and up interleaved) are 8 KB apart
-                    const uint64_t bdesc = umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
+                    // gate and up interleaved) are 8 KB apart; a K-major B (the
+                    // dgrad modes) is laid out like A
+                    const uint64_t bdesc = G::B_KMAJOR ? umma_desc_sw128(sB + kk * 32, 16, 1024)
+                                                       : umma_desc_sw128(sB + kk * 2048, BOX_BYTES, 1024);
                     if (PAIR) umma_f16_ss_pair(d0, adesc, bdesc, idesc, accum);
                     else umma_f16_ss(d0, adesc, bdesc, idesc, accum);
                 }
@@ -314,12 +372,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = unit; t < total; t += units) {
             int e, m_row0, row_end, n0;
             decode_tile(m, E, BM, BN, t, e, m_row0, row_end, n0);
-            if (!mbar_wait(&m->tfull[acc], acc_phase, a.status, 430, abort_flag)) break;
+            // tcgen05.ld is warp-collective: the vote keeps the warp converged
+            if (!__all_sync(0xffffffffu, mbar_wait(&m->tfull[acc], acc_phase, a.status, 430, abort_flag)))
+                break;
             tc_fence_after();
             const int64_t row = (int64_t)m_row0 + r_in_tile;
             const bool valid = row < row_end;
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-            __nv_bfloat16* orow = a.out + row * (int64_t)a.N;
+            __nv_bfloat16* orow = a.out + row * a.ldo;
             if (GATEUP) {
 #pragma unroll 1
                 for (int c = 2 * half; c < 2 * half + 2; ++c) {
@@ -344,6 +404,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             if (col + 8 * q < a.N)
                                 *reinterpret_cast<uint4*>(orow + col + 8 * q) =
                                     make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                        if (a.gu_out != nullptr) {  // keep the pre-activations for the backward
+                            __nv_bfloat16* grow = a.gu_out + row * 2 * (int64_t)a.N + col;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                p[j] = pack_bf16x2(__uint_as_float(g[2 * j]), __uint_as_float(g[2 * j + 1]));
+                                g[j] = pack_bf16x2(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                if (col + 8 * q < a.N) {
+                                    *reinterpret_cast<uint4*>(grow + 8 * q) =
+                                        make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                                    *reinterpret_cast<uint4*>(grow + a.N + 8 * q) =
+                                        make_uint4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                                }
+                        }
+                    }
+                }
+            } else if (MODE == kDgradH) {
+#pragma unroll 1
+                for (int c = 4 * half; c < 4 * half + 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    tmem_ld_wait();
+                    const int col = n0 + c * 32;
+                    if (valid && col < a.N) {
+                        const __nv_bfloat16* grow = a.gu_in + row * 2 * (int64_t)a.N + col;
+                        uint32_t dg[16], du[16];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 gq = make_uint4(0, 0, 0, 0), uq = make_uint4(0, 0, 0, 0);
+                            if (col + 8 * q < a.N) {
+                                gq = *reinterpret_cast<const uint4*>(grow + 8 * q);
+                                uq = *reinterpret_cast<const uint4*>(grow + a.N + 8 * q);
+                            }
+                            const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+                            const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float o[2][2];
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const float gg = __uint_as_float(hh ? (gw[i] & 0xffff0000u) : (gw[i] << 16));
+                                    const float uu = __uint_as_float(hh ? (uw[i] & 0xffff0000u) : (uw[i] << 16));
+                                    const float dh = __uint_as_float(v[8 * q + 2 * i + hh]);
+                                    float sl, dsl;
+                                    silu_and_grad(gg, sl, dsl);
+                                    o[0][hh] = dh * uu * dsl;  // dg
+                                    o[1][hh] = dh * sl;        // du
+                                }
+                                dg[4 * q + i] = pack_bf16x2(o[0][0], o[0][1]);
+                                du[4 * q + i] = pack_bf16x2(o[1][0], o[1][1]);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (col + 8 * q < a.N) {
+                                *reinterpret_cast<uint4*>(orow + col + 8 * q) =
+                                    make_uint4(dg[4 * q], dg[4 * q + 1], dg[4 * q + 2], dg[4 * q + 3]);
+                                *reinterpret_cast<uint4*>(orow + a.N + col + 8 * q) =
+                                    make_uint4(du[4 * q], du[4 * q + 1], du[4 * q + 2], du[4 * q + 3]);
+                            }
                     }
                 }
             } else {
@@ -448,12 +570,43 @@ static bool map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over (E, rows, cols) row-major weights read K-major (the
+// weight transposed): box = 64 cols (K) x box_rows rows (N) x 1.
+static bool map_3d_kmajor(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E,
+                          uint32_t box_rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cols, rows, E};
+    cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map viewing a (rows, 2 * half) row-major matrix as (rows, 2, half):
+// box = 64 cols x 1 half x box_rows rows, so each half pads to 64 on its own.
+static bool map_halves(CUtensorMap* m, const void* base, uint64_t half, uint64_t rows, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {half, 2, rows};
+    cuuint64_t strides[2] = {half * 2, half * 4};
+    cuuint32_t box[3] = {64, 1, box_rows};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Per device: dynamic shared memory opted in, and the number of CTAs (or CTA
 // pairs) that can be resident at once, which sizes the persistent grid.
-template <bool GATEUP, bool PAIR>
+template <int MODE, bool PAIR>
 static cudaError_t prepare(int* resident_units)
 {
-    static int cached[32];  // 0 = not yet queried on that device
+    static int cached[32];  // 0 = not yet queried on that device (per MODE, PAIR instance)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -461,13 +614,13 @@ static cudaError_t prepare(int* resident_units)
         *resident_units = cached[dev];
         return cudaSuccess;
     }
-    constexpr size_t smem = smem_bytes<GATEUP, PAIR>();
-    e = cudaFuncSetAttribute(ffn_tc_kernel<GATEUP, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    constexpr size_t smem = smem_bytes<MODE, PAIR>();
+    e = cudaFuncSetAttribute(ffn_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     int units = 0;
     if (PAIR) {
-        e = cudaFuncSetAttribute(ffn_tc_kernel<GATEUP, PAIR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+        e = cudaFuncSetAttribute(ffn_tc_kernel<MODE, PAIR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -479,7 +632,7 @@ static cudaError_t prepare(int* resident_units)
         cfg.dynamicSmemBytes = smem;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaOccupancyMaxActiveClusters(&units, ffn_tc_kernel<GATEUP, PAIR>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&units, ffn_tc_kernel<MODE, PAIR>, &cfg);
         if (e != cudaSuccess) return e;
     } else {
         int sms = 0;
@@ -493,18 +646,18 @@ static cudaError_t prepare(int* resident_units)
     return cudaSuccess;
 }
 
-template <bool GATEUP, bool PAIR>
+template <int MODE, bool PAIR>
 static cudaError_t launch_one(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
                               const Args& a, int64_t tiles_bound, cudaStream_t s)
 {
     int units = 0;
-    cudaError_t e = prepare<GATEUP, PAIR>(&units);
+    cudaError_t e = prepare<MODE, PAIR>(&units);
     if (e != cudaSuccess) return e;
     int64_t n = tiles_bound < units ? tiles_bound : units;
     if (n < 1) n = 1;
-    constexpr size_t smem = smem_bytes<GATEUP, PAIR>();
+    constexpr size_t smem = smem_bytes<MODE, PAIR>();
     if (!PAIR) {
-        ffn_tc_kernel<GATEUP, false><<<(unsigned)n, NUM_THREADS, smem, s>>>(mA, mB0, mB1, a);
+        ffn_tc_kernel<MODE, false><<<(unsigned)n, NUM_THREADS, smem, s>>>(mA, mB0, mB1, a);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
@@ -519,7 +672,7 @@ static cudaError_t launch_one(const CUtensorMap& mA, const CUtensorMap& mB0, con
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<GATEUP, true>, mA, mB0, mB1, a);
+    return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<MODE, true>, mA, mB0, mB1, a);
 }
 
 }  // namespace tc
@@ -532,8 +685,8 @@ static bool use_pairs(const moe_config& c, int64_t max_rows) { return max_rows >
 cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                const void* w_gate, const void* w_up, const void* w_down, void* h,
-                               void* y_perm, int* status, cudaStream_t s, StageHook mid,
-                               void* mid_ctx)
+                               void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                               StageHook mid, void* mid_ctx)
 {
     using namespace tc;
     CUtensorMap mA, mG, mU, mH, mD;
@@ -548,15 +701,48 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
 
     Args a1{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(h), c.E, c.D, c.F,
-            (c.F + 127) / 128, max_rows, c.T * c.K, status};
-    cudaError_t err = pair ? launch_one<true, true>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s)
-                           : launch_one<true, false>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s);
+            (c.F + 127) / 128, c.F, max_rows, c.T * c.K,
+            static_cast<__nv_bfloat16*>(gu_keep), nullptr, status};
+    cudaError_t err = pair ? launch_one<kGateUp, true>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<kGateUp, false>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     Args a2{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(y_perm), c.E, c.F, c.D,
-            (c.D + 255) / 256, max_rows, c.T * c.K, status};
-    return pair ? launch_one<false, true>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s)
-                : launch_one<false, false>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s);
+            (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status};
+    return pair ? launch_one<kDown, true>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s)
+                : launch_one<kDown, false>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s);
+}
+
+cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const void* dyp,
+                                 const int32_t* offsets, const void* gu, const void* w_gate,
+                                 const void* w_up, const void* w_down, void* dgu, void* dxp,
+                                 int* status, cudaStream_t s, StageHook mid, void* mid_ctx)
+{
+    using namespace tc;
+    const bool pair = use_pairs(c, max_rows);
+    const uint32_t brows = pair ? 128 : 256;  // K-major B rows per CTA
+    CUtensorMap mA, mWd, mDGU, mG, mU;
+    if (!map_2d(&mA, dyp, (uint64_t)c.D, (uint64_t)max_rows, 128) ||
+        !map_3d_kmajor(&mWd, w_down, (uint64_t)c.D, (uint64_t)c.F, (uint64_t)c.E, brows) ||
+        !map_halves(&mDGU, dgu, (uint64_t)c.F, (uint64_t)max_rows, 128) ||
+        !map_3d_kmajor(&mG, w_gate, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows) ||
+        !map_3d_kmajor(&mU, w_up, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows))
+        return cudaErrorInvalidValue;
+    const int64_t bm = pair ? 256 : 128;
+    const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
+    // dH = dYp . Wd^T (K = D), epilogue through SwiGLU into [dg | du]
+    Args a1{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dgu), c.E, c.D, c.F,
+            (c.F + 255) / 256, 2 * (int64_t)c.F, max_rows, c.T * c.K, nullptr,
+            static_cast<const __nv_bfloat16*>(gu), status};
+    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mWd, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<kDgradH, false>(mA, mWd, mWd, a1, mtiles_bound * a1.n_tiles, s);
+    if (err != cudaSuccess) return err;
+    if (mid) mid(mid_ctx, s);
+    // dXp = [dg | du] . [Wg | Wu]^T (K = 2F), unit weights
+    Args a2{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dxp), c.E, c.F, c.D,
+            (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status};
+    return pair ? launch_one<kDgradX, true>(mDGU, mG, mU, a2, mtiles_bound * a2.n_tiles, s)
+                : launch_one<kDgradX, false>(mDGU, mG, mU, a2, mtiles_bound * a2.n_tiles, s);
 }
 
 }  // namespace moe

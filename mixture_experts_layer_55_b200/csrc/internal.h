@@ -78,6 +78,33 @@ struct FwdLayout {
 };
 FwdLayout fwd_layout(const moe_config& c, int64_t max_rows);
 
+// The training forward's state: the forward layout (its y_perm holds the
+// unweighted expert outputs) plus what only the backward reads.
+struct TrainLayout {
+    FwdLayout f;
+    size_t logits;      // (T, E) fp32: the logits the layer was routed on
+    size_t gu;          // (max_rows, 2F) dtype: [g | u] pre-activations
+    size_t sh_gu;       // (T, 2 F_shared) dtype
+    size_t total;
+};
+TrainLayout train_layout(const moe_config& c, int64_t max_rows);
+
+// The backward's scratch.
+struct BwdLayout {
+    size_t status;      // int32[64]
+    size_t dyp;         // (max_rows, D): w_r * dY[t_r]
+    size_t dw_row;      // (max_rows) fp32: gate-weight gradient of each row
+    size_t dlogits;     // (T, E) fp32
+    size_t dgu;         // (max_rows, 2F): [dg | du]
+    size_t dxp;         // (max_rows, D)
+    size_t rw_part;     // router weight-gradient partials
+    size_t sh_dgu;      // (T, 2 F_shared)
+    size_t sh_dx;       // (T, D)
+    int rw_splits;
+    size_t total;
+};
+BwdLayout bwd_layout(const moe_config& c, int64_t max_rows);
+
 int64_t capacity_of(const moe_config& c);
 int64_t max_rows_of(const moe_config& c);
 
@@ -110,17 +137,45 @@ cudaError_t launch_dispatch_index(const moe_config& c, int64_t C, const int32_t*
 cudaError_t launch_gather(const moe_config& c, const void* x, const int32_t* row_of, void* x_perm,
                           int64_t max_rows, int* status, cudaStream_t s);
 
+// slot_w (T, K) or null: when given, each slot's row is multiplied by its weight.
 cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
-                           const void* y_add, void* y, int64_t max_rows, cudaStream_t s);
+                           const float* slot_w, const void* y_add, void* y, int64_t max_rows,
+                           cudaStream_t s);
 
 // Expert FFN: gate/up (+SwiGLU) into h, then down (+routing weight) into y_perm.
 // The stage boundary between the two GEMMs is reported through `mid` (may be
 // null): it is called after the gate/up launch.
 typedef void (*StageHook)(void* ctx, cudaStream_t s);
+// gu_keep (max_rows, 2F) or null: where the gate/up GEMM keeps [g | u] (bf16 only).
 cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
                               const void* w_gate, const void* w_up, const void* w_down, void* h,
-                              void* y_perm, int* status, cudaStream_t s, StageHook mid,
-                              void* mid_ctx);
+                              void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                              StageHook mid, void* mid_ctx);
+
+// ---------------------------------------------------------------- backward --
+// dH = dYp . Wd^T through SwiGLU into dgu = [dg | du], then dXp = dgu . [Wg | Wu]^T.
+cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const void* dyp,
+                                 const int32_t* offsets, const void* gu, const void* w_gate,
+                                 const void* w_up, const void* w_down, void* dgu, void* dxp,
+                                 int* status, cudaStream_t s, StageHook mid, void* mid_ctx);
+// out0 / out1 (E, M, Nh) fp32 = A[block]^T . B[block] per expert block.
+cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets, const void* A,
+                                 int M, const void* B, int Nh, int halves, float* out0, float* out1,
+                                 int* status, cudaStream_t s);
+cudaError_t launch_bwd_rows(const moe_config& c, const void* dy, const void* o, const int32_t* offsets,
+                            const int32_t* perm, const float* topk_w, void* dyp, float* dw_row,
+                            int64_t max_rows, int* status, cudaStream_t s);
+cudaError_t launch_router_bwd(const moe_config& c, const float* logits, const int32_t* ids,
+                              const int32_t* row_of, const float* dw_row, const int32_t* counts,
+                              float c_bal, float c_z, float* dlogits, int64_t max_rows, int* status,
+                              cudaStream_t s);
+int router_wgrad_splits(const moe_config& c);
+size_t router_wgrad_part_bytes(const moe_config& c, int splits);
+cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float* dL, float* part,
+                                int splits, float* dw, float* db, cudaStream_t s);
+cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float* w_r, const void* dxp,
+                               const int32_t* row_of, const void* dx_shared, void* dx,
+                               int64_t max_rows, cudaStream_t s);
 
 }  // namespace moe

@@ -1,0 +1,383 @@
+// wgrad_tc.cu -- weight gradients of the grouped expert GEMMs on the
+// 5th-generation tensor cores (tcgen05 MMA, fp32 accumulators in tensor
+// memory, operands staged by TMA).
+//
+// "Lab: build a tiny MoE in PyTorch", "Smoke test and backward pass": the
+// experts' weights receive gradient from the rows routed to them.  Each
+// expert's rows are one contiguous block of the expert-major layout, so every
+// weight gradient is one GEMM per expert contracting over that block:
+//
+//   dWd_e          = h[block]^T      . dYp[block]        (M = F, N = D)
+//   [dWg_e | dWu_e] = x_perm[block]^T . [dg | du][block]  (M = D, N = 2F, split at F)
+//
+// Both operands are row blocks of row-major (rows, M) and (rows, N) matrices,
+// so both are read MN-major (128-byte swizzle, 64-column boxes); K is the
+// expert's row count, ragged.  A K block that runs past the expert's last row
+// reads the next expert's rows: the MMA warp zeroes those rows of the stage in
+// shared memory before issuing (an expert with no rows writes zeros).  The
+// result is stored in fp32 (the precision weight gradients are accumulated in).
+//
+// Persistent kernel, one CTA per SM, tiles M = 128 x N = 256, 4-stage ring of
+// 48 KB, double-buffered 2 x 256-column accumulators.  10 warps: warp 0 TMA,
+// warp 1 MMA (all lanes wait and zero; one issues), warps 2..9 epilogue.
+// Every wait is bounded (device status flag).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace wg {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                  // K rows per stage
+constexpr int UK = 16;                  // K per tcgen05.mma (bf16)
+constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64-column x 64-row box
+constexpr int A_BOXES = BM / 64;
+constexpr int B_BOXES = BN / 64;
+constexpr int A_BYTES = A_BOXES * BOX_BYTES;
+constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;  // 48 KB
+constexpr int STAGES = 4;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;
+constexpr int MAX_E = 256;
+
+struct Misc {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int row0[MAX_E];
+    int rowend[MAX_E];
+};
+
+constexpr size_t smem_bytes() { return 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Misc); }
+
+struct Args {
+    const int32_t* offsets;  // (E + 1) row offsets of the experts' blocks
+    float* out0;             // (E, M, Nh) fp32: product columns [0, Nh)
+    float* out1;             // (E, M, Nh) fp32: columns [Nh, 2 Nh) when halves = 2
+    int E;
+    int M;                   // output rows (A's columns)
+    int Nh;                  // output columns per half
+    int halves;              // 1, or 2 when B holds two Nh-column halves
+    int mt;                  // ceil(M / BM)
+    int nth;                 // ceil(Nh / BN)
+    int64_t max_rows;
+    int* status;
+};
+
+MOE_DEVICE void decode(const Args& a, int t, int& e, int& m0, int& hf, int& n0)
+{
+    const int per_e = a.mt * a.nth * a.halves;
+    e = t / per_e;
+    const int r = t - e * per_e;
+    const int j = r / a.mt;  // n tile over both halves
+    m0 = (r - j * a.mt) * BM;
+    hf = j / a.nth;
+    n0 = (j - hf * a.nth) * BN;
+}
+
+MOE_DEVICE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&m->tfull[b], 1);
+            mbar_init(&m->tempty[b], EPI_WARPS);
+        }
+        mbar_init(&m->drain, 1);
+        m->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&m->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    for (int e = threadIdx.x; e < E; e += NUM_THREADS) {
+        m->row0[e] = a.offsets[e];
+        m->rowend[e] = a.offsets[e + 1];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // validate the blocks: a malformed one is treated as empty
+        int prev = 0;
+        for (int e = 0; e < E; ++e) {
+            int r0 = m->row0[e], r1 = m->rowend[e];
+            if (r0 < prev || r1 < r0 || (int64_t)r1 > a.max_rows) {
+                raise_flag(a.status, kFlagBounds, 500);
+                r0 = r1 = prev;
+            }
+            m->row0[e] = r0;
+            m->rowend[e] = r1;
+            prev = r1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = m->tmem_base;
+    const int total = E * a.mt * a.nth * a.halves;
+    volatile int* abort_flag = &m->abort_flag;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int last_phase[STAGES];
+        for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int e, m0, hf, n0;
+            decode(a, t, e, m0, hf, n0);
+            const int r0 = m->row0[e], r1 = m->rowend[e];
+            const int bcol = hf * a.Nh + n0;
+            for (int k = r0; k < r1; k += BK) {
+                if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
+                uint8_t* sB = sA + A_BYTES;
+                uint64_t* fb = &m->full[stage];
+                mbar_arrive_expect_tx(fb, STAGE_BYTES);
+#pragma unroll
+                for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, &tmA, m0 + 64 * j, k, fb);
+#pragma unroll
+                for (int j = 0; j < B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
+                last_phase[stage] = (int)phase;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        for (int s = 0; s < STAGES; ++s)
+            if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
+    } else if (warp == 1) {
+        // ------------------------------------------- MMA issuer (whole warp)
+        // A and B MN-major: 64-column boxes 8 KB apart (LBO), 8-row K groups
+        // 1024 B apart (SBO), +2048 B per 16-row K step
+        constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, 1, 1);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int e, m0, hf, n0;
+            decode(a, t, e, m0, hf, n0);
+            const int r0 = m->row0[e], r1 = m->rowend[e];
+            // every lane waits (each wait is bounded); the vote keeps the warp converged
+            if (!__all_sync(0xffffffffu, mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 520, abort_flag)))
+                break;
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + (uint32_t)(acc * ACC_COLS);
+            for (int k = r0; k < r1; k += BK) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&m->full[stage], phase, a.status, 521, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
+                const int valid = r1 - k;
+                if (valid < BK) {
+                    // rows valid..63 of this block belong to the next expert (or
+                    // lie past the end): zero them in every box of the stage
+                    const int n16 = (BK - valid) * 8;  // 16-byte words per box
+#pragma unroll 1
+                    for (int b = 0; b < A_BOXES + B_BOXES; ++b) {
+                        uint4* p = reinterpret_cast<uint4*>(sA + b * BOX_BYTES + valid * 128);
+                        for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t a32 = smem_u32(sA);
+                    const uint32_t b32 = a32 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk) {
+                        const uint32_t accum = (k != r0 || kk != 0) ? 1u : 0u;
+                        const uint64_t adesc = umma_desc_sw128(a32 + kk * 2048, BOX_BYTES, 1024);
+                        const uint64_t bdesc = umma_desc_sw128(b32 + kk * 2048, BOX_BYTES, 1024);
+                        umma_f16_ss(d0, adesc, bdesc, idesc, accum);
+                    }
+                    umma_commit(&m->empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&m->tfull[acc]);  // with no rows: arrives at once
+            __syncwarp();
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) {
+            umma_commit(&m->drain);
+            mbar_wait(&m->drain, 0, a.status, 522, nullptr);
+        }
+        __syncwarp();
+    } else if (warp >= 2) {
+        // -------------------------------------------------------- epilogue
+        // warp w: tensor-memory lanes 32*(w%4) .. +31 (output rows), half of
+        // the 256 columns (warps 2..5 the first, 6..9 the second)
+        const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            int e, m0, hf, n0;
+            decode(a, t, e, m0, hf, n0);
+            const bool empty_block = m->rowend[e] == m->row0[e];
+            // tcgen05.ld is warp-collective: the vote keeps the warp converged
+            if (!__all_sync(0xffffffffu, mbar_wait(&m->tfull[acc], acc_phase, a.status, 530, abort_flag)))
+                break;
+            tc_fence_after();
+            const int row = m0 + quad * 32 + lane;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            float* orow = (hf ? a.out1 : a.out0) + ((int64_t)e * a.M + row) * (int64_t)a.Nh;
+#pragma unroll 1
+            for (int c = 4 * half; c < 4 * half + 4; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, v);
+                tmem_ld_wait();
+                const int col = n0 + c * 32;
+                if (row < a.M) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        if (col + 4 * q < a.Nh) {
+                            const uint4 w = empty_block ? make_uint4(0, 0, 0, 0)
+                                                        : make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                                                     v[4 * q + 3]);
+                            *reinterpret_cast<uint4*>(orow + col + 4 * q) = w;
+                        }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&m->tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------- host --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encoder()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 map over a row-major (rows, cols) matrix; box = 64 cols x 64 rows.
+static bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static cudaError_t prepare(int* ctas)
+{
+    static int cached[32];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 32 && cached[dev] > 0) {
+        *ctas = cached[dev];
+        return cudaSuccess;
+    }
+    e = cudaFuncSetAttribute(wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_bytes());
+    if (e != cudaSuccess) return e;
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (sms < 1) return cudaErrorInvalidConfiguration;
+    if (dev < 32) cached[dev] = sms;
+    *ctas = sms;
+    return cudaSuccess;
+}
+
+}  // namespace wg
+
+// out0/out1 (E, M, Nh) fp32 = for each expert, A[block]^T . B[block] with A
+// (max_rows, M) and B (max_rows, halves * Nh) bf16 row-major.
+cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets, const void* A,
+                                 int M, const void* B, int Nh, int halves, float* out0, float* out1,
+                                 int* status, cudaStream_t s)
+{
+    using namespace wg;
+    if (E < 1 || E > MAX_E || M < 1 || Nh < 1 || (halves != 1 && halves != 2)) return cudaErrorInvalidValue;
+    CUtensorMap mA, mB;
+    if (!map_rows(&mA, A, (uint64_t)M, (uint64_t)max_rows) ||
+        !map_rows(&mB, B, (uint64_t)Nh * halves, (uint64_t)max_rows))
+        return cudaErrorInvalidValue;
+    int ctas = 0;
+    cudaError_t e = prepare(&ctas);
+    if (e != cudaSuccess) return e;
+    Args a{offsets, out0, halves == 2 ? out1 : out0, E, M, Nh, halves, (M + BM - 1) / BM,
+           (Nh + BN - 1) / BN, max_rows, status};
+    const int64_t total = (int64_t)E * a.mt * a.nth * a.halves;
+    const int grid = (int)(total < ctas ? total : ctas);
+    wgrad_tc_kernel<<<grid, NUM_THREADS, smem_bytes(), s>>>(mA, mB, a);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -118,6 +118,53 @@ class MoELayer:
         comp.wait_stream(d2h)
         return d2h
 
+    # ----------------------------------------------------------- training
+    def forward_train(self, x, y=None, logit_noise=None, stream=None):
+        """forward() that keeps the activations moe_backward reads (bf16
+        layers); the state buffer is allocated on first use."""
+        if getattr(self, "state", None) is None:
+            self.state = torch.zeros(B.train_state_size(self.cfg), dtype=torch.uint8,
+                                     device=self.device)
+        if y is None:
+            y = torch.empty_like(x)
+        B.moe_forward_train(self.cfg, x, self.w_router, self.w_gate, self.w_up, self.w_down, y,
+                            self.state, router_bias=self.router_bias, logit_noise=logit_noise,
+                            selection_bias=self.selection_bias, shared=self.shared,
+                            losses=self.losses, mean_prob=self.mean_prob, counts=self.counts,
+                            stream=stream)
+        self._train_x = x
+        return y
+
+    def backward(self, dy, c_balance: float = 0.0, c_z: float = 0.0, grads=None, stream=None):
+        """Gradients of sum(dy * y) + c_balance * balance + c_z * z for the
+        last forward_train.  Returns a dict of dx (layer dtype) and fp32
+        dw_router, db_router (when the layer has a router bias), dw_gate,
+        dw_up, dw_down (and dshared); ``grads`` may pass that dict back to
+        reuse its buffers."""
+        x = getattr(self, "_train_x", None)
+        if x is None:
+            raise RuntimeError("backward() needs a forward_train() first")
+        if getattr(self, "bwd_workspace", None) is None:
+            self.bwd_workspace = torch.zeros(B.backward_workspace_size(self.cfg),
+                                             dtype=torch.uint8, device=self.device)
+        if grads is None:
+            f32 = dict(dtype=torch.float32, device=self.device)
+            grads = dict(dx=torch.empty_like(x),
+                         dw_router=torch.empty(self.w_router.shape, **f32),
+                         dw_gate=torch.empty(self.w_gate.shape, **f32),
+                         dw_up=torch.empty(self.w_up.shape, **f32),
+                         dw_down=torch.empty(self.w_down.shape, **f32))
+            if self.router_bias is not None:
+                grads["db_router"] = torch.empty(self.router_bias.shape, **f32)
+            if self.shared is not None:
+                grads["dshared"] = tuple(torch.empty(w.shape, **f32) for w in self.shared)
+        B.moe_backward(self.cfg, x, self.w_router, self.w_gate, self.w_up, self.w_down, self.state,
+                       dy, grads["dx"], grads["dw_router"], grads["dw_gate"], grads["dw_up"],
+                       grads["dw_down"], self.bwd_workspace, c_balance=c_balance, c_z=c_z,
+                       db_router=grads.get("db_router"), shared=self.shared,
+                       dshared=grads.get("dshared"), stream=stream)
+        return grads
+
     def update_selection_bias(self, gamma: float, stream=None):
         """One DeepSeek-V3 balancing step from the last forward's counts."""
         if self.selection_bias is None:

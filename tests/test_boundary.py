@@ -170,3 +170,51 @@ def test_status_strings_and_trace_table(lib):
     assert lib.moe_trace_attach(None, 0) == B.MOE_OK
     assert lib.moe_trace_attach(None, 3) == B.MOE_ERR_ARG
     assert lib.moe_trace_attach(None, 17) == B.MOE_ERR_ARG
+
+
+def test_backward_sizes_counts_and_trace(lib):
+    c = _cfg(T=1200, D=256, F=384, E=4, K=2)
+    assert B.train_state_size(c) > B.forward_workspace_size(c)
+    assert B.backward_workspace_size(c) > 0
+    assert B.backward_kernel_count(c) == 9
+    assert B.backward_kernel_count(_cfg(T=600, F=320, F_shared=192, capacity_factor=1.0)) == 13
+    assert B.backward_kernel_count(_cfg(dtype="f32")) == 0  # bf16 layers only
+    with pytest.raises(B.MoEError):
+        B.train_state_size(_cfg(dtype="f32"))
+    names = B.trace_backward_stage_names()
+    assert names[0] == "start" and names[-1] == "dx" and len(names) == 10
+    assert lib.moe_trace_attach_backward(None, 0) == B.MOE_OK
+    assert lib.moe_trace_attach_backward(None, 2) == B.MOE_ERR_ARG
+
+
+def test_training_argument_errors(lib):
+    c = _cfg()
+    cr = ctypes.byref(c)
+    sb = B.train_state_size(c)
+    bb = B.backward_workspace_size(c)
+    fwd = lambda state, nbytes, x=FAKE: lib.moe_forward_train(  # noqa: E731
+        cr, x, FAKE, None, None, None, FAKE, FAKE, FAKE, None, None, None, FAKE, None, None, None,
+        None, None, state, nbytes, None)
+    assert fwd(FAKE, sb - 1) == B.MOE_ERR_WORKSPACE
+    assert fwd(None, sb) == B.MOE_ERR_WORKSPACE
+    assert fwd(FAKE + 16, sb) == B.MOE_ERR_ALIGN
+    assert fwd(FAKE, sb, x=None) == B.MOE_ERR_ARG
+    cf = _cfg(dtype="f32")
+    assert lib.moe_forward_train(ctypes.byref(cf), FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE,
+                                 None, None, None, FAKE, None, None, None, None, None, FAKE, 1 << 30,
+                                 None) == B.MOE_ERR_UNSUPPORTED
+
+    def bwd(dy=FAKE, state_bytes=sb, ws_bytes=bb, c_bal=0.0, dw_gate=FAKE, shared=None, cfg=c):
+        return lib.moe_backward(ctypes.byref(cfg), FAKE, FAKE, FAKE, FAKE, FAKE, shared, shared,
+                                shared, FAKE, state_bytes, dy, ctypes.c_float(c_bal),
+                                ctypes.c_float(0.0), FAKE, FAKE, None, dw_gate, FAKE, FAKE, shared,
+                                shared, shared, FAKE, ws_bytes, None)
+    assert bwd(dy=None) == B.MOE_ERR_ARG
+    assert bwd(dw_gate=None) == B.MOE_ERR_ARG
+    assert bwd(dy=FAKE + 2) == B.MOE_ERR_ALIGN
+    assert bwd(state_bytes=sb - 1) == B.MOE_ERR_WORKSPACE
+    assert bwd(ws_bytes=bb - 1) == B.MOE_ERR_WORKSPACE
+    assert bwd(c_bal=float("inf")) == B.MOE_ERR_ARG
+    cs = _cfg(F_shared=64)
+    assert bwd(cfg=cs, state_bytes=B.train_state_size(cs),
+               ws_bytes=B.backward_workspace_size(cs)) == B.MOE_ERR_ARG  # shared grads missing

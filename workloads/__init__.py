@@ -166,3 +166,12 @@ def make_tokens(wl: Workload | str, device="cpu", seed: int = 1234) -> torch.Ten
         wl = WORKLOADS[wl]
     g = _gen(device, seed)
     return _randn((wl.T, wl.D), g, device, 1.0, wl.torch_dtype)
+
+
+def make_output_grad(wl: Workload | str, device="cpu", seed: int = 4321) -> torch.Tensor:
+    """A seeded upstream gradient dY (T, D) ~ N(0, 1) in the layer dtype, for
+    the backward of the layer."""
+    if isinstance(wl, str):
+        wl = WORKLOADS[wl]
+    g = _gen(device, seed)
+    return _randn((wl.T, wl.D), g, device, 1.0, wl.torch_dtype)
