@@ -7,6 +7,11 @@ the Mixtral-shaped dropless layer (T=8192, D=4096, F=14336, E=8, K=2, bf16).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle on the host cores
+    python bench.py --pass train ...       # a training step: forward + backward
+
+With --pass train one step is moe_forward_train + moe_backward (the gradient
+of sum <dY, y> + 0.01 balance + 0.001 z) over one batch, and the line reports
+training-step tokens/s with the backward kernels' stage times.
 
 N > 1 runs under torchrun: one independent replica per GPU (the layer is
 per-token, so ranks share nothing on the data path); value = all ranks'
@@ -30,10 +35,13 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, Workload, make_inputs, make_tokens  # noqa: E402
+from workloads import (WORKLOADS, Workload, make_inputs, make_output_grad,  # noqa: E402
+                       make_tokens)
 
 METRIC = "routed tokens/s per MoE layer fwd on 1 B200; % bf16 tensor peak / % HBM BW"
 UNIT = "tokens/s"
+METRIC_TRAIN = "routed tokens/s per MoE layer training step (fwd + bwd) on 1 B200"
+C_BAL, C_Z = 0.01, 0.001  # the lab's loss coefficients
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -369,6 +377,159 @@ def run_gpu(args):
     _finish(world)
 
 
+def run_gpu_train(args):
+    """A training step per iteration: moe_forward_train + moe_backward."""
+    import mixture_experts_layer_55_b200 as M
+
+    rank, world, local_rank = rank_info()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    init_dist(world, "nccl")
+    wl = workload_of(args)
+    if wl.dtype != "bf16":
+        raise SystemExit("--pass train needs a bf16 workload")
+    inp = make_inputs(wl, device=dev)
+    layer = M.MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
+                       wl.capacity_factor, router_bias=inp["bias"])
+    noise = inp["noise"]
+    nbuf = 3
+    xs = [make_tokens(wl, device=dev, seed=rank_token_seed(rank) * 16 + i) for i in range(nbuf)]
+    dys = [make_output_grad(wl, device=dev, seed=rank_token_seed(rank) * 16 + 8 + i)
+           for i in range(nbuf)]
+    y = torch.empty_like(xs[0])
+    stream = torch.cuda.current_stream(dev)
+    grads = None
+
+    def step(i):
+        nonlocal grads
+        layer.forward_train(xs[i % nbuf], y, logit_noise=noise)
+        grads = layer.backward(dys[i % nbuf], C_BAL, C_Z, grads=grads)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    nf = M._binding.lib().moe_trace_boundary_count()
+    nbk = M._binding.lib().moe_trace_backward_boundary_count()
+    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(nf)] for _ in range(args.steps)]
+    evb = [[torch.cuda.Event(enable_timing=True) for _ in range(nbk)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(args.steps):
+        M.moe_trace_attach(evf[i])
+        M._binding.moe_trace_attach_backward(evb[i])
+        step(i)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    M.moe_trace_attach([])
+    M._binding.moe_trace_attach_backward([])
+    clk = clocks.stop()
+    ms_total, ms_step, value = aggregate(start.elapsed_time(stop), world, wl.T, args.steps, dev)
+
+    def stage_times(evs, names, prefix):
+        out = {}
+        for j in range(1, len(names)):
+            d = [evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(args.steps)]
+            out[prefix + names[j]] = sum(d) / len(d)
+        return out
+    stage_ms = stage_times(evf, M.trace_stage_names(), "fwd.")
+    stage_ms.update(stage_times(evb, M._binding.trace_backward_stage_names(), "bwd."))
+
+    counts = layer.counts.cpu().tolist()
+    kept_rows = int(min(sum(min(c, M.capacity(layer.cfg)) for c in counts), M.max_rows(layer.cfg)))
+    R = kept_rows
+    flop = {"fwd.expert_gate_up": 4.0 * R * wl.D * wl.F, "fwd.expert_down": 2.0 * R * wl.F * wl.D,
+            "bwd.dgrad_h": 2.0 * R * wl.D * wl.F, "bwd.dgrad_x": 4.0 * R * wl.F * wl.D,
+            "bwd.wgrad_down": 2.0 * R * wl.F * wl.D, "bwd.wgrad_gate_up": 4.0 * R * wl.D * wl.F}
+
+    # ---------------- end to end: x and dY in from pinned memory, dx and losses out ----------
+    x_h = [t.cpu().pin_memory() for t in xs]
+    dy_h = [t.cpu().pin_memory() for t in dys]
+    dx_h = torch.empty_like(x_h[0]).pin_memory()
+    loss_h = torch.empty(3, dtype=torch.float32).pin_memory()
+    xd, dyd = torch.empty_like(xs[0]), torch.empty_like(dys[0])
+
+    def e2e_step(i):
+        nonlocal grads
+        xd.copy_(x_h[i % nbuf], non_blocking=True)
+        dyd.copy_(dy_h[i % nbuf], non_blocking=True)
+        layer.forward_train(xd, y, logit_noise=noise)
+        grads = layer.backward(dyd, C_BAL, C_Z, grads=grads)
+        dx_h.copy_(grads["dx"], non_blocking=True)
+        loss_h.copy_(layer.losses, non_blocking=True)
+    for i in range(max(2, args.warmup)):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    io = wl.T * wl.D * wl.elem_bytes
+
+    for ws in (layer.state, layer.bwd_workspace):
+        flags = M.moe_get_device_status(ws)
+        if flags:
+            raise RuntimeError(f"device status flags {flags:#x} after the benchmark")
+    if rank != 0:
+        _finish(world)
+        return
+
+    peaks, peak_src = load_peaks()
+    key = "bf16_tflops_sustained" if ms_total > 1000.0 else "bf16_tflops"
+    peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
+    gemms = [k for k in flop if k.startswith("bwd.")]
+    top = max(gemms, key=lambda k: stage_ms[k])
+    achieved = flop[top] / (stage_ms[top] / 1e3) / 1e12
+    roofline = {"kernel": top, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{key} of {peak_src}", "traffic": None}
+    stages = {}
+    for name, ms in stage_ms.items():
+        ent = {"ms": round(ms, 4)}
+        if name in flop:
+            ent["TFLOPs"] = round(flop[name] / (ms / 1e3) / 1e12, 1)
+        stages[name] = ent
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_train(wl, args.cpu_seconds)
+    line = {
+        "metric": METRIC_TRAIN, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) tokens and output gradients, N(0,0.02^2) weights)",
+        "config": {"workload": wl.name, "pass": "train", "T": wl.T, "D": wl.D, "F": wl.F,
+                   "E": wl.E, "K": wl.K, "capacity_factor": wl.capacity_factor,
+                   "loss": f"sum(dY*y) + {C_BAL} balance + {C_Z} z",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (expert weights and fp32 weight gradients)"},
+        "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": 2 * io,
+                "d2h_bytes_per_step": io + 12,
+                "how": "per step: x and dY in from pinned host memory, moe_forward_train, "
+                       "moe_backward, dx and the losses out, one stream"},
+        "gpu_launches": (M.forward_kernel_count(layer.cfg)
+                         + M._binding.backward_kernel_count(layer.cfg)) * args.steps,
+        "roofline": roofline,
+        "stages": stages,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if args.warmup < 3:
+        line["note"] = "fewer than 3 warm-up steps: not a valid measurement"
+    print(json.dumps(line), flush=True)
+    _finish(world)
+
+
 def _finish(world):
     if world > 1:
         import torch.distributed as dist
@@ -416,6 +577,52 @@ def cpu_baseline(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
             "sample": (f"router + routing + dispatch layout on all {wl.T} tokens "
                        f"({t_route:.2f} s), expert FFN + combine on {n} sampled tokens "
                        f"({t_ffn:.2f} s); value extrapolated per token")}
+
+
+def cpu_baseline_train(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
+    """The oracle's training step on a bounded sample: forward routing and the
+    router's backward for all T tokens, then each sampled token's kept rows
+    through the expert backward and their share of the weight gradients."""
+    import numpy as np
+
+    import oracle
+    cpu_inp = _cpu_inputs_for_sample(wl)
+    dy = make_output_grad(wl, device="cpu")
+    t0 = time.perf_counter()
+    L = oracle.router_logits(cpu_inp["x"], cpu_inp["w_router"], cpu_inp["bias"], cpu_inp["noise"])
+    ids, w, probs, lse = oracle.route(L, wl.K)
+    C = oracle.capacity(wl.T, wl.K, wl.E, wl.capacity_factor)
+    d = oracle.dispatch(ids, wl.E, C)
+    dL = oracle.router_backward(L, ids, np.zeros((wl.T, wl.K)), d["counts"], C_BAL, C_Z)
+    oracle.router_linear_backward(cpu_inp["x"], cpu_inp["w_router"], dL)
+    t_route = time.perf_counter() - t0
+    kept = d["row_of"].reshape(wl.T, wl.K) >= 0
+    get = cpu_inp["get_expert"]
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(wl.T)
+    n, t_rows, batch = 0, 0.0, 1
+    budget = max(1.0, seconds - t_route)
+    while t_rows < budget and n < wl.T:
+        toks = sorted(order[n:n + batch].tolist())
+        t1 = time.perf_counter()
+        for e in sorted({int(ids[t, k]) for t in toks for k in range(wl.K) if kept[t, k]}):
+            rows = [(t, k) for t in toks for k in range(wl.K) if kept[t, k] and ids[t, k] == e]
+            tok = np.array([t for t, _ in rows], np.int32)
+            wt = np.array([w[t, k] for t, k in rows])
+            wg, wu, wd = get(e)
+            _, _, h, dg, du = oracle.expert_backward_rows(tok, np.zeros(len(rows), np.int32), wt,
+                                                          cpu_inp["x"], dy, wg, wu, wd,
+                                                          intermediates=True)
+            oracle.expert_wgrad(tok, wt, cpu_inp["x"], dy, h, dg, du)
+        t_rows += time.perf_counter() - t1
+        n += len(toks)
+        batch = min(batch * 2, 32)
+    per_token = t_route / wl.T + t_rows / n
+    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"routing, dispatch layout and the router's backward on all {wl.T} tokens "
+                       f"({t_route:.2f} s); expert backward and weight-gradient rows of {n} "
+                       f"sampled tokens ({t_rows:.2f} s); value extrapolated per token")}
 
 
 def _cpu_inputs_for_sample(wl: Workload):
@@ -469,18 +676,21 @@ def run_reference(args):
         return
     wl = workload_of(args)
     per_step = max(2.0, args.cpu_seconds / 2)
+    train = getattr(args, "pass_", "forward") == "train"
+    base = cpu_baseline_train if train else cpu_baseline
     if args.warmup > 0:
-        cpu_baseline(wl, min(per_step, 4.0) / 2)
+        base(wl, min(per_step, 4.0) / 2)
     vals = []
     t0 = time.perf_counter()
     for i in range(args.steps):
-        vals.append(cpu_baseline(wl, per_step, seed=i))
+        vals.append(base(wl, per_step, seed=i))
         if time.perf_counter() - t0 > 240:
             break
     value = statistics.median(v["value"] for v in vals)
     ms_step = 1e3 * wl.T / value
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "impl": "reference", "metric": METRIC_TRAIN if train else METRIC,
+        "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": len(vals), "warmup": args.warmup,
         "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -505,9 +715,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--override", action="append", default=[],
                     help="KEY=VALUE change of the workload shape (profiling cases only)")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "train"], default="forward",
+                    help="forward (default) or a training step (forward + backward)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.pass_ == "train":
+        run_gpu_train(args)
     else:
         run_gpu(args)
 

@@ -124,6 +124,7 @@ BwdLayout bwd_layout(const moe_config& c, int64_t max_rows)
     B.dxp = o;     o += align_up((size_t)max_rows * c.D * es);
     B.rw_splits = router_wgrad_splits(c);
     B.rw_part = o; o += align_up(router_wgrad_part_bytes(c, B.rw_splits));
+    B.db_scratch = o; o += align_up((size_t)c.E * sizeof(float));
     B.sh_dgu = o;  B.sh_dx = o;
     if (c.F_shared > 0) {
         B.sh_dgu = o; o += align_up((size_t)c.T * 2 * c.F_shared * es);
@@ -613,7 +614,8 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
     btrace(7, s);
     if (e == cudaSuccess)
         e = launch_router_wgrad(c, x, dlogits, reinterpret_cast<float*>(ws + B.rw_part), B.rw_splits,
-                                dw_router, db_router, s);
+                                dw_router,
+                                db_router ? db_router : reinterpret_cast<float*>(ws + B.db_scratch), s);
     btrace(8, s);
     if (e == cudaSuccess)
         e = launch_dx_assemble(c, dlogits, w_router, ws + B.dxp, row_of, dx_shared, dx, max_rows, s);
@@ -664,9 +666,10 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
 int32_t moe_backward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;
-    // rows, router, two dgrad GEMMs, two wgrad GEMMs, router weight partials
-    // and their sum, dx; the shared expert adds its two dgrad and two wgrad GEMMs
-    return 9 + (cfg->F_shared > 0 ? 4 : 0);
+    // rows, router, two dgrad GEMMs, two wgrad GEMMs, router weight partials,
+    // their sum, the bias gradient, dx; the shared expert adds its two dgrad
+    // and two wgrad GEMMs
+    return 10 + (cfg->F_shared > 0 ? 4 : 0);
 }
 
 moe_status moe_trace_attach_backward(void* const* events, int32_t n_events)

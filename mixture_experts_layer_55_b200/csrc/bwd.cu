@@ -11,8 +11,8 @@
 //   router     dL[t] from the gate weights' dw (renormalised or not, route
 //              scale), the balance loss through the normalised scores (counts
 //              fixed) and the z-loss through the logsumexp
-//   linear     dW_r = x^T dL,  db = sum_t dL[t]   (split over tokens, then a
-//              fixed-order sum: deterministic)
+//   linear     dW_r = x^T dL (split over tokens, then a fixed-order sum of the
+//              splits), db = sum_t dL[t] (a fixed-order tree): deterministic
 //   dx         dx[t] = dL[t] W_r^T + sum over kept slots of dXp[row] (+ the
 //              shared expert's), rounded once
 // No atomics anywhere: every result is bit-reproducible.
@@ -199,137 +199,171 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const float* __restrict
 }
 
 // ---------------------------------------------------- router weight grads --
-// part[s][d][e] = sum over the tokens of split s of x[t,d] * dL[t,e]; row d = D
-// of part takes x = 1 (the bias gradient).  Block: 64 d x ET experts, a token
-// chunk of the split staged through shared memory 64 tokens at a time.
-template <typename XT, int ET>
-__global__ void __launch_bounds__(256) router_wgrad_partial_kernel(const XT* __restrict__ x,
-                                                                   const float* __restrict__ dL,
-                                                                   float* __restrict__ part, int64_t T,
-                                                                   int D, int E, int64_t t_per_split)
+// 8 consecutive d of x as fp32 (one 16-byte load for bf16, two for fp32).
+MOE_DEVICE void load8(const __nv_bfloat16* p, float (&v)[8])
 {
-    constexpr int EPT = ET / 4;  // experts per thread
-    __shared__ float sdl[64][ET];
-    const int dl = threadIdx.x & 63, eg = threadIdx.x >> 6;
-    const int d = blockIdx.x * 64 + dl;
-    const int e0 = blockIdx.y * ET;
-    const int64_t t0 = (int64_t)blockIdx.z * t_per_split;
-    const int64_t t1 = t0 + t_per_split < T ? t0 + t_per_split : T;
-    float acc[EPT];
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) acc[j] = 0.f;
-    for (int64_t tc = t0; tc < t1; tc += 64) {
-        for (int i = threadIdx.x; i < 64 * ET; i += 256) {
-            const int tt = i / ET, ee = i - tt * ET;
-            const int64_t t = tc + tt;
-            sdl[tt][ee] = (t < t1 && e0 + ee < E) ? dL[t * E + e0 + ee] : 0.f;
-        }
-        __syncthreads();
-        const int n = (int)(t1 - tc < 64 ? t1 - tc : 64);
-        if (d <= D) {
-#pragma unroll 4
-            for (int i = 0; i < n; ++i) {
-                const float xv = d < D ? to_f32(x[(tc + i) * D + d]) : 1.f;
-#pragma unroll
-                for (int j = 0; j < EPT; ++j) acc[j] = fmaf(xv, sdl[i][eg * EPT + j], acc[j]);
-            }
-        }
-        __syncthreads();
-    }
-    if (d <= D) {
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) {
-            const int e = e0 + eg * EPT + j;
-            if (e < E) part[((int64_t)blockIdx.z * (D + 1) + d) * E + e] = acc[j];
-        }
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     }
 }
-
-// dW[d][e] = sum over splits in order; row D goes to db (may be null).
-__global__ void router_wgrad_reduce_kernel(const float* __restrict__ part, int splits, int D, int E,
-                                           float* __restrict__ dw, float* __restrict__ db)
+MOE_DEVICE void load8(const float* p, float (&v)[8])
 {
-    const int64_t n = (int64_t)(D + 1) * E;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+MOE_DEVICE void store8(__nv_bfloat16* p, const float (&v)[8])
+{
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+MOE_DEVICE void store8(float* p, const float (&v)[8])
+{
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+constexpr int kRwThreads = 128;  // x 8 d = 1024 d per block
+constexpr int kRwE = 8;          // experts per block
+
+// part[z][d][e] = sum over the tokens of split z of x[t,d] * dL[t,e]: each
+// thread owns 8 consecutive d and the block's 8 experts (64 accumulators).
+template <typename XT>
+__global__ void __launch_bounds__(kRwThreads) router_wgrad_partial_kernel(const XT* __restrict__ x,
+                                                                          const float* __restrict__ dL,
+                                                                          float* __restrict__ part,
+                                                                          int64_t T, int D, int E,
+                                                                          int64_t t_per_split)
+{
+    const int d0 = (blockIdx.x * kRwThreads + threadIdx.x) * 8;
+    const int e0 = blockIdx.y * kRwE;
+    const int64_t t0 = (int64_t)blockIdx.z * t_per_split;
+    const int64_t t1 = t0 + t_per_split < T ? t0 + t_per_split : T;
+    if (d0 >= D) return;
+    float acc[8][kRwE];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < kRwE; ++j) acc[i][j] = 0.f;
+    const int ne = E - e0 < kRwE ? E - e0 : kRwE;
+#pragma unroll 2
+    for (int64_t t = t0; t < t1; ++t) {
+        float xv[8], g[kRwE];
+        load8(x + t * D + d0, xv);
+#pragma unroll
+        for (int j = 0; j < kRwE; ++j) g[j] = j < ne ? __ldg(dL + t * E + e0 + j) : 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < kRwE; ++j) acc[i][j] = fmaf(xv[i], g[j], acc[i][j]);
+    }
+    float* out = part + ((int64_t)blockIdx.z * D + d0) * E + e0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < kRwE; ++j)
+            if (j < ne) out[(int64_t)i * E + j] = acc[i][j];
+}
+
+// dW[d][e] = sum over splits in order.
+__global__ void router_wgrad_reduce_kernel(const float* __restrict__ part, int splits, int D, int E,
+                                           float* __restrict__ dw)
+{
+    const int64_t n = (int64_t)D * E;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         float s = 0.f;
         for (int k = 0; k < splits; ++k) s += part[(int64_t)k * n + i];
-        if (i < (int64_t)D * E) dw[i] = s;
-        else if (db) db[i - (int64_t)D * E] = s;
+        dw[i] = s;
     }
 }
 
-// --------------------------------------------------------------------- dx --
-// Block: 16 tokens x 256 d; warp w owns tokens 2w, 2w+1, lane l the columns
-// l, l + 32, ..., l + 224 of the tile (so the shared-memory reads of W_r are
-// conflict-free).  The router term dL W_r^T is accumulated through shared
-// memory in chunks of 32 experts, then the token's kept rows of dXp (slot
-// order) and the shared expert's row are added, and the sum is rounded once.
-constexpr int kDxTok = 16;
-constexpr int kDxCols = 256;
-
-template <typename ET>
-__global__ void __launch_bounds__(256) dx_assemble_kernel(const float* __restrict__ dL,
-                                                          const float* __restrict__ w_r,
-                                                          const ET* __restrict__ dxp,
-                                                          const int32_t* __restrict__ row_of,
-                                                          const ET* __restrict__ dx_shared,
-                                                          ET* __restrict__ dx, int64_t T, int D, int E,
-                                                          int K, int64_t max_rows)
+// db[e] = sum_t dL[t,e]: one block per expert, a fixed-order tree.
+__global__ void __launch_bounds__(256) router_bias_grad_kernel(const float* __restrict__ dL, int64_t T,
+                                                               int E, float* __restrict__ db)
 {
-    __shared__ float swr[kDxCols][33];
-    __shared__ float sdl[kDxTok][32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t tb = (int64_t)blockIdx.x * kDxTok;
-    const int d0 = blockIdx.y * kDxCols;
-    float acc[2][8];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-        for (int i = threadIdx.x; i < kDxCols * 32; i += 256) {
-            const int dd = i >> 5, ee = i & 31;
-            swr[dd][ee] = (d0 + dd < D && e0 + ee < E) ? w_r[(int64_t)(d0 + dd) * E + e0 + ee] : 0.f;
-        }
-        for (int i = threadIdx.x; i < kDxTok * 32; i += 256) {
-            const int tt = i >> 5, ee = i & 31;
-            sdl[tt][ee] = (tb + tt < T && e0 + ee < E) ? dL[(tb + tt) * E + e0 + ee] : 0.f;
-        }
-        __syncthreads();
-        const int ne = E - e0 < 32 ? E - e0 : 32;
-        for (int ee = 0; ee < ne; ++ee) {
-            const float g0 = sdl[2 * warp][ee], g1 = sdl[2 * warp + 1][ee];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float wv = swr[lane + 32 * j][ee];
-                acc[0][j] = fmaf(g0, wv, acc[0][j]);
-                acc[1][j] = fmaf(g1, wv, acc[1][j]);
-            }
-        }
+    __shared__ float red[256];
+    const int e = blockIdx.x;
+    float s = 0.f;
+    for (int64_t t = threadIdx.x; t < T; t += 256) s += dL[t * E + e];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
         __syncthreads();
     }
+    if (threadIdx.x == 0) db[e] = red[0];
+}
+
+// --------------------------------------------------------------------- dx --
+// Block: kDxTok tokens x 1024 d; each thread owns 8 consecutive d of every
+// token of the block.  The router term dL W_r^T runs over the experts 8 at a
+// time (this thread's 8 x 8 block of W_r in registers), then the token's kept
+// rows of dXp (slot order) and the shared expert's row are added as 16-byte
+// vectors, and the sum is rounded once.
+constexpr int kDxTok = 8;
+constexpr int kDxThreads = 128;
+
+template <typename ET>
+__global__ void __launch_bounds__(kDxThreads) dx_assemble_kernel(const float* __restrict__ dL,
+                                                                 const float* __restrict__ w_r,
+                                                                 const ET* __restrict__ dxp,
+                                                                 const int32_t* __restrict__ row_of,
+                                                                 const ET* __restrict__ dx_shared,
+                                                                 ET* __restrict__ dx, int64_t T, int D,
+                                                                 int E, int K, int64_t max_rows)
+{
+    const int d0 = (blockIdx.x * kDxThreads + threadIdx.x) * 8;
+    const int64_t tb = (int64_t)blockIdx.y * kDxTok;
+    if (d0 >= D) return;
+    float acc[kDxTok][8];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int64_t t = tb + 2 * warp + i;
-        if (t >= T) break;
-        for (int k = 0; k < K; ++k) {
-            const int32_t r = row_of[t * K + k];
-            if (r < 0 || r >= max_rows) continue;
-            const ET* src = dxp + (int64_t)r * D + d0;
+    for (int i = 0; i < kDxTok; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (d0 + lane + 32 * j < D) acc[i][j] += to_f32(src[lane + 32 * j]);
-        }
-        if (dx_shared) {
-            const ET* src = dx_shared + t * D + d0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (d0 + lane + 32 * j < D) acc[i][j] += to_f32(src[lane + 32 * j]);
-        }
-        ET* dst = dx + t * D + d0;
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += 8) {
+        float w[8][8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            if (d0 + lane + 32 * j < D) dst[lane + 32 * j] = from_f32<ET>(acc[i][j]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                w[j][k] = e0 + k < E ? __ldg(w_r + (int64_t)(d0 + j) * E + e0 + k) : 0.f;
+#pragma unroll
+        for (int i = 0; i < kDxTok; ++i) {
+            const int64_t t = tb + i;
+            if (t >= T) break;
+            float g[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) g[k] = e0 + k < E ? __ldg(dL + t * E + e0 + k) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[i][j] = fmaf(g[k], w[j][k], acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kDxTok; ++i) {
+        const int64_t t = tb + i;
+        if (t >= T) break;
+        for (int k = 0; k < K; ++k) {
+            const int32_t r = __ldg(row_of + t * K + k);
+            if (r < 0 || r >= max_rows) continue;
+            float v[8];
+            load8(dxp + (int64_t)r * D + d0, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+        }
+        if (dx_shared) {
+            float v[8];
+            load8(dx_shared + t * D + d0, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+        }
+        store8(dx + t * D + d0, acc[i]);
     }
 }
 
@@ -371,49 +405,43 @@ cudaError_t launch_router_bwd(const moe_config& c, const float* logits, const in
 
 int router_wgrad_splits(const moe_config& c)
 {
-    // enough blocks to fill the GPU a few times; each split at least 256 tokens
-    const int64_t dblocks = (c.D + 1 + 63) / 64;
-    const int64_t eblocks = c.E <= 8 ? 1 : (c.E + 31) / 32;
+    // about four waves of blocks; each split at least 32 tokens
+    const int64_t dblocks = (c.D + kRwThreads * 8 - 1) / (kRwThreads * 8);
+    const int64_t eblocks = (c.E + kRwE - 1) / kRwE;
     int64_t want = (int64_t)sm_count() * 4 / (dblocks * eblocks);
-    int64_t most = (c.T + 255) / 256;
+    int64_t most = (c.T + 31) / 32;
     int64_t sp = want < most ? want : most;
     if (sp < 1) sp = 1;
-    if (sp > 64) sp = 64;
+    if (sp > 256) sp = 256;
     return (int)sp;
 }
 
 size_t router_wgrad_part_bytes(const moe_config& c, int splits)
 {
-    return (size_t)splits * (size_t)(c.D + 1) * c.E * sizeof(float);
+    return (size_t)splits * (size_t)c.D * c.E * sizeof(float);
 }
 
 cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float* dL, float* part,
                                 int splits, float* dw, float* db, cudaStream_t s)
 {
     const int64_t tps = (c.T + splits - 1) / splits;
-    const dim3 grid((unsigned)((c.D + 1 + 63) / 64), 1, (unsigned)splits);
-    if (c.E <= 8) {
-        if (c.dtype == MOE_BF16)
-            router_wgrad_partial_kernel<__nv_bfloat16, 8><<<grid, 256, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(x), dL, part, c.T, c.D, c.E, tps);
-        else
-            router_wgrad_partial_kernel<float, 8><<<grid, 256, 0, s>>>(static_cast<const float*>(x), dL,
+    const dim3 grid((unsigned)((c.D + kRwThreads * 8 - 1) / (kRwThreads * 8)),
+                    (unsigned)((c.E + kRwE - 1) / kRwE), (unsigned)splits);
+    if (c.dtype == MOE_BF16)
+        router_wgrad_partial_kernel<__nv_bfloat16><<<grid, kRwThreads, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(x), dL, part, c.T, c.D, c.E, tps);
+    else
+        router_wgrad_partial_kernel<float><<<grid, kRwThreads, 0, s>>>(static_cast<const float*>(x), dL,
                                                                        part, c.T, c.D, c.E, tps);
-    } else {
-        const dim3 g2(grid.x, (unsigned)((c.E + 31) / 32), grid.z);
-        if (c.dtype == MOE_BF16)
-            router_wgrad_partial_kernel<__nv_bfloat16, 32><<<g2, 256, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(x), dL, part, c.T, c.D, c.E, tps);
-        else
-            router_wgrad_partial_kernel<float, 32><<<g2, 256, 0, s>>>(static_cast<const float*>(x), dL,
-                                                                      part, c.T, c.D, c.E, tps);
-    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t n = (int64_t)(c.D + 1) * c.E;
+    const int64_t n = (int64_t)c.D * c.E;
     int64_t blocks = (n + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    router_wgrad_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(part, splits, c.D, c.E, dw, db);
+    router_wgrad_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(part, splits, c.D, c.E, dw);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || db == nullptr) return e;
+    router_bias_grad_kernel<<<(unsigned)c.E, 256, 0, s>>>(dL, c.T, c.E, db);
     return cudaGetLastError();
 }
 
@@ -421,17 +449,18 @@ cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float
                                const int32_t* row_of, const void* dx_shared, void* dx,
                                int64_t max_rows, cudaStream_t s)
 {
-    const dim3 grid((unsigned)((c.T + kDxTok - 1) / kDxTok), (unsigned)((c.D + kDxCols - 1) / kDxCols));
+    const dim3 grid((unsigned)((c.D + kDxThreads * 8 - 1) / (kDxThreads * 8)),
+                    (unsigned)((c.T + kDxTok - 1) / kDxTok));
     if (c.dtype == MOE_BF16)
-        dx_assemble_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        dx_assemble_kernel<__nv_bfloat16><<<grid, kDxThreads, 0, s>>>(
             dL, w_r, static_cast<const __nv_bfloat16*>(dxp), row_of,
             static_cast<const __nv_bfloat16*>(dx_shared), static_cast<__nv_bfloat16*>(dx), c.T, c.D,
             c.E, c.K, max_rows);
     else
-        dx_assemble_kernel<float><<<grid, 256, 0, s>>>(dL, w_r, static_cast<const float*>(dxp), row_of,
-                                                       static_cast<const float*>(dx_shared),
-                                                       static_cast<float*>(dx), c.T, c.D, c.E, c.K,
-                                                       max_rows);
+        dx_assemble_kernel<float><<<grid, kDxThreads, 0, s>>>(dL, w_r, static_cast<const float*>(dxp), row_of,
+                                                              static_cast<const float*>(dx_shared),
+                                                              static_cast<float*>(dx), c.T, c.D, c.E, c.K,
+                                                              max_rows);
     return cudaGetLastError();
 }
 

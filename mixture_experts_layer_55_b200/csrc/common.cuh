@@ -192,6 +192,21 @@ MOE_DEVICE void tma_load_3d(void* smem_dst, const void* tmap, int32_t c0, int32_
         : "memory");
 }
 
+// shared -> global tiled store (bulk async group; commit, then wait with
+// bulk_wait_read before the shared source is rewritten).  Out-of-range parts
+// of the box are not written.
+MOE_DEVICE void tma_store_3d(const void* tmap, const void* smem_src, int32_t c0, int32_t c1, int32_t c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     tmap),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy accesses (TMA stores, tcgen05.mma operand reads).
+MOE_DEVICE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 MOE_DEVICE void prefetch_tmap(const void* tmap)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

@@ -98,6 +98,7 @@ struct BwdLayout {
     size_t dgu;         // (max_rows, 2F): [dg | du]
     size_t dxp;         // (max_rows, D)
     size_t rw_part;     // router weight-gradient partials
+    size_t db_scratch;  // (E) fp32: the bias gradient when the caller wants none
     size_t sh_dgu;      // (T, 2 F_shared)
     size_t sh_dx;       // (T, D)
     int rw_splits;

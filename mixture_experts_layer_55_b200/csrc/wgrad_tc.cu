@@ -19,8 +19,11 @@
 //
 // Persistent kernel, one CTA per SM, tiles M = 128 x N = 256, 4-stage ring of
 // 48 KB, double-buffered 2 x 256-column accumulators.  10 warps: warp 0 TMA,
-// warp 1 MMA (all lanes wait and zero; one issues), warps 2..9 epilogue.
-// Every wait is bounded (device status flag).
+// warp 1 MMA (all lanes wait and zero; one issues), warps 2..9 epilogue.  The
+// epilogue stages each warp's 32 x 32 fp32 piece in shared memory (128-byte
+// swizzle, conflict-free) and writes it with a TMA tensor store over an
+// (E, M, N) map, so the stores are whole lines and the map clips the tile's
+// edges per expert.  Every wait is bounded (device status flag).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -39,6 +42,7 @@ constexpr int B_BOXES = BN / 64;
 constexpr int A_BYTES = A_BOXES * BOX_BYTES;
 constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;  // 48 KB
 constexpr int STAGES = 4;
+constexpr int OUT_BYTES = 32 * 32 * 4;  // one epilogue warp's staged 32 x 32 fp32 piece
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 320;
@@ -53,11 +57,14 @@ struct Misc {
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
-    int row0[MAX_E];
-    int rowend[MAX_E];
+    int off[MAX_E + 1];  // validated row offsets: expert e owns rows off[e] .. off[e+1]-1
 };
 
-constexpr size_t smem_bytes() { return 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Misc); }
+constexpr size_t smem_bytes()
+{
+    return 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)EPI_WARPS * OUT_BYTES + sizeof(Misc);
+}
+static_assert(smem_bytes() <= 232448, "shared memory per block");
 
 struct Args {
     const int32_t* offsets;  // (E + 1) row offsets of the experts' blocks
@@ -84,17 +91,17 @@ MOE_DEVICE void decode(const Args& a, int t, int& e, int& m0, int& hf, int& n0)
     n0 = (j - hf * a.nth) * BN;
 }
 
-MOE_DEVICE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                     const Args a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* stages = smem;
-    Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint8_t* outbuf = smem + (size_t)STAGES * STAGE_BYTES;  // EPI_WARPS x OUT_BYTES, 1 KB aligned
+    Misc* m = reinterpret_cast<Misc*>(outbuf + (size_t)EPI_WARPS * OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = a.E;
 
@@ -112,28 +119,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        prefetch_tmap(&tmO0);
+        if (a.halves == 2) prefetch_tmap(&tmO1);
     }
     if (warp == 1) {
         tmem_alloc(&m->tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
-    for (int e = threadIdx.x; e < E; e += NUM_THREADS) {
-        m->row0[e] = a.offsets[e];
-        m->rowend[e] = a.offsets[e + 1];
-    }
+    for (int e = threadIdx.x; e <= E; e += NUM_THREADS) m->off[e] = a.offsets[e];
     __syncthreads();
-    if (threadIdx.x == 0) {  // validate the blocks: a malformed one is treated as empty
+    if (threadIdx.x == 0) {  // validate: offsets non-decreasing from 0, within max_rows
         int prev = 0;
-        for (int e = 0; e < E; ++e) {
-            int r0 = m->row0[e], r1 = m->rowend[e];
-            if (r0 < prev || r1 < r0 || (int64_t)r1 > a.max_rows) {
-                raise_flag(a.status, kFlagBounds, 500);
-                r0 = r1 = prev;
+        bool bad = false;
+        for (int e = 0; e <= E; ++e) {
+            int r = m->off[e];
+            if (r < prev || (int64_t)r > a.max_rows || (e == 0 && r != 0)) {
+                bad = true;
+                r = prev;  // a malformed block becomes empty
             }
-            m->row0[e] = r0;
-            m->rowend[e] = r1;
-            prev = r1;
+            m->off[e] = r;
+            prev = r;
         }
+        if (bad) raise_flag(a.status, kFlagBounds, 500);
     }
     tc_fence_before();
     __syncthreads();
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             int e, m0, hf, n0;
             decode(a, t, e, m0, hf, n0);
-            const int r0 = m->row0[e], r1 = m->rowend[e];
+            const int r0 = m->off[e], r1 = m->off[e + 1];
             const int bcol = hf * a.Nh + n0;
             for (int k = r0; k < r1; k += BK) {
                 if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) {
@@ -189,7 +196,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             int e, m0, hf, n0;
             decode(a, t, e, m0, hf, n0);
-            const int r0 = m->row0[e], r1 = m->rowend[e];
+            const int r0 = m->off[e], r1 = m->off[e + 1];
             // every lane waits (each wait is bounded); the vote keeps the warp converged
             if (!__all_sync(0xffffffffu, mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 520, abort_flag)))
                 break;
@@ -252,34 +259,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // the 256 columns (warps 2..5 the first, 6..9 the second)
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
+        uint8_t* buf = outbuf + (size_t)(warp - 2) * OUT_BYTES;
+        const int swz = lane & 7;  // the 128-byte swizzle of this lane's staged row
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             int e, m0, hf, n0;
             decode(a, t, e, m0, hf, n0);
-            const bool empty_block = m->rowend[e] == m->row0[e];
+            const bool empty_block = m->off[e + 1] == m->off[e];
             // tcgen05.ld is warp-collective: the vote keeps the warp converged
             if (!__all_sync(0xffffffffu, mbar_wait(&m->tfull[acc], acc_phase, a.status, 530, abort_flag)))
                 break;
             tc_fence_after();
-            const int row = m0 + quad * 32 + lane;
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-            float* orow = (hf ? a.out1 : a.out0) + ((int64_t)e * a.M + row) * (int64_t)a.Nh;
+            const CUtensorMap* tmo = hf ? &tmO1 : &tmO0;
 #pragma unroll 1
             for (int c = 4 * half; c < 4 * half + 4; ++c) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, v);
                 tmem_ld_wait();
-                const int col = n0 + c * 32;
-                if (row < a.M) {
+                if (lane == 0) bulk_wait_read<0>();  // the previous store has read the buffer
+                __syncwarp();
+                uint4* row = reinterpret_cast<uint4*>(buf + lane * 128);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        if (col + 4 * q < a.Nh) {
-                            const uint4 w = empty_block ? make_uint4(0, 0, 0, 0)
-                                                        : make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
-                                                                     v[4 * q + 3]);
-                            *reinterpret_cast<uint4*>(orow + col + 4 * q) = w;
-                        }
+                for (int q = 0; q < 8; ++q)
+                    row[q ^ swz] = empty_block ? make_uint4(0, 0, 0, 0)
+                                               : make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {  // rows >= M and columns >= Nh fall outside the map: not written
+                    tma_store_3d(tmo, buf, n0 + c * 32, m0 + quad * 32, e);
+                    bulk_commit();
                 }
             }
             tc_fence_before();
@@ -290,6 +300,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc_phase ^= 1u;
             }
         }
+        if (lane == 0) bulk_wait_all<0>();  // every store of this warp has completed
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -333,6 +345,21 @@ static bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map over (E, M, Nh) row-major outputs; box = 32 cols x 32 rows x 1,
+// 128-byte swizzle (the epilogue stages its pieces in that layout).
+static bool map_out(CUtensorMap* m, const float* base, uint64_t Nh, uint64_t M, uint64_t E)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {Nh, M, E};
+    cuuint64_t strides[2] = {Nh * 4, Nh * M * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static cudaError_t prepare(int* ctas)
 {
     static int cached[32];
@@ -365,9 +392,11 @@ cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets
 {
     using namespace wg;
     if (E < 1 || E > MAX_E || M < 1 || Nh < 1 || (halves != 1 && halves != 2)) return cudaErrorInvalidValue;
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mO0, mO1;
     if (!map_rows(&mA, A, (uint64_t)M, (uint64_t)max_rows) ||
-        !map_rows(&mB, B, (uint64_t)Nh * halves, (uint64_t)max_rows))
+        !map_rows(&mB, B, (uint64_t)Nh * halves, (uint64_t)max_rows) ||
+        !map_out(&mO0, out0, (uint64_t)Nh, (uint64_t)M, (uint64_t)E) ||
+        !map_out(&mO1, halves == 2 ? out1 : out0, (uint64_t)Nh, (uint64_t)M, (uint64_t)E))
         return cudaErrorInvalidValue;
     int ctas = 0;
     cudaError_t e = prepare(&ctas);
@@ -376,7 +405,7 @@ cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets
            (Nh + BN - 1) / BN, max_rows, status};
     const int64_t total = (int64_t)E * a.mt * a.nth * a.halves;
     const int grid = (int)(total < ctas ? total : ctas);
-    wgrad_tc_kernel<<<grid, NUM_THREADS, smem_bytes(), s>>>(mA, mB, a);
+    wgrad_tc_kernel<<<grid, NUM_THREADS, smem_bytes(), s>>>(mA, mB, mO0, mO1, a);
     return cudaGetLastError();
 }
 

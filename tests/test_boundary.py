@@ -176,8 +176,8 @@ def test_backward_sizes_counts_and_trace(lib):
     c = _cfg(T=1200, D=256, F=384, E=4, K=2)
     assert B.train_state_size(c) > B.forward_workspace_size(c)
     assert B.backward_workspace_size(c) > 0
-    assert B.backward_kernel_count(c) == 9
-    assert B.backward_kernel_count(_cfg(T=600, F=320, F_shared=192, capacity_factor=1.0)) == 13
+    assert B.backward_kernel_count(c) == 10
+    assert B.backward_kernel_count(_cfg(T=600, F=320, F_shared=192, capacity_factor=1.0)) == 14
     assert B.backward_kernel_count(_cfg(dtype="f32")) == 0  # bf16 layers only
     with pytest.raises(B.MoEError):
         B.train_state_size(_cfg(dtype="f32"))
