@@ -487,17 +487,37 @@ def run_gpu_train(args):
     peaks, peak_src = load_peaks()
     key = "bf16_tflops_sustained" if ms_total > 1000.0 else "bf16_tflops"
     peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
-    gemms = [k for k in flop if k.startswith("bwd.")]
-    top = max(gemms, key=lambda k: stage_ms[k])
-    achieved = flop[top] / (stage_ms[top] / 1e3) / 1e12
-    roofline = {"kernel": top, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{key} of {peak_src}", "traffic": None}
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # algorithmic bytes of the backward GEMMs (bf16 operands, fp32 weight gradients)
+    s2, Ea = wl.elem_bytes, sum(1 for c in counts if c > 0)
+    D, F, E = wl.D, wl.F, wl.E
+    nbytes = {"bwd.dgrad_h": R * D * s2 + Ea * F * D * s2 + 2 * (R * 2 * F * s2),
+              "bwd.dgrad_x": R * 2 * F * s2 + Ea * 2 * D * F * s2 + R * D * s2,
+              "bwd.wgrad_down": R * F * s2 + R * D * s2 + E * F * D * 4,
+              "bwd.wgrad_gate_up": R * D * s2 + R * 2 * F * s2 + E * 2 * D * F * 4}
+    top = max(nbytes, key=lambda k: stage_ms[k])
+    t_top = stage_ms[top] / 1e3
+    intensity = flop[top] / nbytes[top]
+    ridge = peak * 1e12 / (hbm_peak * 1e9)
+    if intensity >= ridge:
+        achieved = flop[top] / t_top / 1e12
+        roofline = {"kernel": top, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_source": f"{key} of {peak_src}"}
+    else:
+        achieved = nbytes[top] / t_top / 1e9
+        roofline = {"kernel": top, "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                    "peak_source": f"hbm_gbs of {peak_src}"}
+    roofline.update(intensity_flop_per_byte=round(intensity, 1), ridge=round(ridge, 1),
+                    traffic=None)
     stages = {}
     for name, ms in stage_ms.items():
         ent = {"ms": round(ms, 4)}
         if name in flop:
             ent["TFLOPs"] = round(flop[name] / (ms / 1e3) / 1e12, 1)
+        if name in nbytes:
+            ent["GBs"] = round(nbytes[name] / (ms / 1e3) / 1e9, 1)
         stages[name] = ent
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -300,12 +300,14 @@ __global__ void __launch_bounds__(256) router_bias_grad_kernel(const float* __re
 }
 
 // --------------------------------------------------------------------- dx --
-// Block: kDxTok tokens x 1024 d; each thread owns 8 consecutive d of every
-// token of the block.  The router term dL W_r^T runs over the experts 8 at a
-// time (this thread's 8 x 8 block of W_r in registers), then the token's kept
-// rows of dXp (slot order) and the shared expert's row are added as 16-byte
-// vectors, and the sum is rounded once.
-constexpr int kDxTok = 8;
+// Block: kDxTok tokens (in groups of kDxGroup) x 1024 d; each thread owns 8
+// consecutive d.  The router term dL W_r^T runs over the experts 8 at a time:
+// the block's 1024 x 8 slice of W_r is staged transposed in shared memory
+// (coalesced global reads, conflict-free 16-byte shared reads), once per block
+// when E <= 8.  Then each token's kept rows of dXp (slot order) and the shared
+// expert's row are added as 16-byte vectors and the sum is rounded once.
+constexpr int kDxTok = 32;
+constexpr int kDxGroup = 8;
 constexpr int kDxThreads = 128;
 
 template <typename ET>
@@ -317,53 +319,76 @@ __global__ void __launch_bounds__(kDxThreads) dx_assemble_kernel(const float* __
                                                                  ET* __restrict__ dx, int64_t T, int D,
                                                                  int E, int K, int64_t max_rows)
 {
-    const int d0 = (blockIdx.x * kDxThreads + threadIdx.x) * 8;
-    const int64_t tb = (int64_t)blockIdx.y * kDxTok;
-    if (d0 >= D) return;
-    float acc[kDxTok][8];
+    __shared__ __align__(16) float swt[8][kDxThreads * 8];  // W_r^T chunk: 8 experts x 1024 d
+    __shared__ float sdl[kDxGroup][8];
+    const int dblk = blockIdx.x * kDxThreads * 8;
+    const int d0 = dblk + threadIdx.x * 8;
+    const bool active = d0 < D;
+    for (int g0 = 0; g0 < kDxTok; g0 += kDxGroup) {
+        const int64_t tb = (int64_t)blockIdx.y * kDxTok + g0;
+        if (tb >= T) break;  // uniform across the block
+        float acc[kDxGroup][8];
 #pragma unroll
-    for (int i = 0; i < kDxTok; ++i)
+        for (int i = 0; i < kDxGroup; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    for (int e0 = 0; e0 < E; e0 += 8) {
-        float w[8][8];
+            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+        for (int e0 = 0; e0 < E; e0 += 8) {
+            __syncthreads();  // the previous chunk's shared reads are done
+            if (E > 8 || g0 == 0) {
+#pragma unroll 1
+                for (int r = 0; r < 8; ++r) {
+                    const int il = threadIdx.x + kDxThreads * r;
+                    const int d = dblk + il;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+                    for (int k = 0; k < 8; ++k)
+                        swt[k][il] = (d < D && e0 + k < E) ? __ldg(w_r + (int64_t)d * E + e0 + k) : 0.f;
+                }
+            }
+            if (threadIdx.x < kDxGroup * 8) {
+                const int tt = threadIdx.x >> 3, k = threadIdx.x & 7;
+                sdl[tt][k] = (tb + tt < T && e0 + k < E) ? __ldg(dL + (tb + tt) * E + e0 + k) : 0.f;
+            }
+            __syncthreads();
+            if (active) {
+                float w[8][8];  // w[j][k] = W_r[d0 + j][e0 + k]
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                w[j][k] = e0 + k < E ? __ldg(w_r + (int64_t)(d0 + j) * E + e0 + k) : 0.f;
+                for (int k = 0; k < 8; ++k) {
+                    const float4 lo = *reinterpret_cast<const float4*>(&swt[k][threadIdx.x * 8]);
+                    const float4 hi = *reinterpret_cast<const float4*>(&swt[k][threadIdx.x * 8 + 4]);
+                    w[0][k] = lo.x; w[1][k] = lo.y; w[2][k] = lo.z; w[3][k] = lo.w;
+                    w[4][k] = hi.x; w[5][k] = hi.y; w[6][k] = hi.z; w[7][k] = hi.w;
+                }
 #pragma unroll
-        for (int i = 0; i < kDxTok; ++i) {
+                for (int i = 0; i < kDxGroup; ++i)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float gk = sdl[i][k];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(gk, w[j][k], acc[i][j]);
+                    }
+            }
+        }
+        if (!active) continue;
+#pragma unroll
+        for (int i = 0; i < kDxGroup; ++i) {
             const int64_t t = tb + i;
             if (t >= T) break;
-            float g[8];
+            for (int k = 0; k < K; ++k) {
+                const int32_t r = __ldg(row_of + t * K + k);
+                if (r < 0 || r >= max_rows) continue;
+                float v[8];
+                load8(dxp + (int64_t)r * D + d0, v);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) g[k] = e0 + k < E ? __ldg(dL + t * E + e0 + k) : 0.f;
+                for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+            }
+            if (dx_shared) {
+                float v[8];
+                load8(dx_shared + t * D + d0, v);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) acc[i][j] = fmaf(g[k], w[j][k], acc[i][j]);
+                for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+            }
+            store8(dx + t * D + d0, acc[i]);
         }
-    }
-#pragma unroll
-    for (int i = 0; i < kDxTok; ++i) {
-        const int64_t t = tb + i;
-        if (t >= T) break;
-        for (int k = 0; k < K; ++k) {
-            const int32_t r = __ldg(row_of + t * K + k);
-            if (r < 0 || r >= max_rows) continue;
-            float v[8];
-            load8(dxp + (int64_t)r * D + d0, v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
-        }
-        if (dx_shared) {
-            float v[8];
-            load8(dx_shared + t * D + d0, v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
-        }
-        store8(dx + t * D + d0, acc[i]);
     }
 }
 

@@ -32,16 +32,10 @@
 namespace moe {
 namespace wg {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BN = 256;                 // output columns per tile
 constexpr int BK = 64;                  // K rows per stage
 constexpr int UK = 16;                  // K per tcgen05.mma (bf16)
 constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64-column x 64-row box
-constexpr int A_BOXES = BM / 64;
-constexpr int B_BOXES = BN / 64;
-constexpr int A_BYTES = A_BOXES * BOX_BYTES;
-constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;  // 48 KB
-constexpr int STAGES = 4;
 constexpr int OUT_BYTES = 32 * 32 * 4;  // one epilogue warp's staged 32 x 32 fp32 piece
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
@@ -49,9 +43,23 @@ constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;
 constexpr int MAX_E = 256;
 
+// Single CTA: M = 128 output rows, all 256 columns in this CTA (2 A + 4 B
+// boxes per stage, 4 stages).  CTA pair: M = 256, each CTA its 128 rows of A
+// and 128 of the columns of B (2 + 2 boxes, 6 stages); the leader issues.
+template <bool PAIR> struct Geo {
+    static constexpr int CTAS = PAIR ? 2 : 1;
+    static constexpr int BM = 128 * CTAS;
+    static constexpr int A_BOXES = 2;
+    static constexpr int B_BOXES = 4 / CTAS;
+    static constexpr int A_BYTES = A_BOXES * BOX_BYTES;
+    static constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;  // 48 KB single, 32 KB pair
+    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;
+};
+
 struct Misc {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[6];
+    uint64_t empty[6];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -60,16 +68,15 @@ struct Misc {
     int off[MAX_E + 1];  // validated row offsets: expert e owns rows off[e] .. off[e+1]-1
 };
 
-constexpr size_t smem_bytes()
+template <bool PAIR> constexpr size_t smem_bytes()
 {
-    return 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)EPI_WARPS * OUT_BYTES + sizeof(Misc);
+    return 1024 + (size_t)Geo<PAIR>::STAGES * Geo<PAIR>::STAGE_BYTES + (size_t)EPI_WARPS * OUT_BYTES +
+           sizeof(Misc);
 }
-static_assert(smem_bytes() <= 232448, "shared memory per block");
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory per block");
 
 struct Args {
     const int32_t* offsets;  // (E + 1) row offsets of the experts' blocks
-    float* out0;             // (E, M, Nh) fp32: product columns [0, Nh)
-    float* out1;             // (E, M, Nh) fp32: columns [Nh, 2 Nh) when halves = 2
     int E;
     int M;                   // output rows (A's columns)
     int Nh;                  // output columns per half
@@ -80,22 +87,32 @@ struct Args {
     int* status;
 };
 
-MOE_DEVICE void decode(const Args& a, int t, int& e, int& m0, int& hf, int& n0)
+MOE_DEVICE void decode(const Args& a, int bm, int t, int& e, int& m0, int& hf, int& n0)
 {
     const int per_e = a.mt * a.nth * a.halves;
     e = t / per_e;
     const int r = t - e * per_e;
     const int j = r / a.mt;  // n tile over both halves
-    m0 = (r - j * a.mt) * BM;
+    m0 = (r - j * a.mt) * bm;
     hf = j / a.nth;
     n0 = (j - hf * a.nth) * BN;
 }
 
+MOE_DEVICE void fence_proxy_async_cluster() { asm volatile("fence.proxy.async.shared::cluster;" ::: "memory"); }
+
+MOE_DEVICE void st_cluster_zero16(uint32_t cluster_addr)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(cluster_addr), "r"(0) : "memory");
+}
+
+template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                     const Args a)
 {
+    using G = Geo<PAIR>;
+    constexpr int BM = G::BM, STAGES = G::STAGES, STAGE_BYTES = G::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -104,6 +121,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     Misc* m = reinterpret_cast<Misc*>(outbuf + (size_t)EPI_WARPS * OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = a.E;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader (issues the MMAs)
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -112,7 +132,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&m->tfull[b], 1);
-            mbar_init(&m->tempty[b], EPI_WARPS);
+            mbar_init(&m->tempty[b], G::EPI_ARRIVALS);
         }
         mbar_init(&m->drain, 1);
         m->abort_flag = 0;
@@ -123,8 +143,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (a.halves == 2) prefetch_tmap(&tmO1);
     }
     if (warp == 1) {
-        tmem_alloc(&m->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&m->tmem_base, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&m->tmem_base, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     for (int e = threadIdx.x; e <= E; e += NUM_THREADS) m->off[e] = a.offsets[e];
     __syncthreads();
@@ -143,37 +168,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (bad) raise_flag(a.status, kFlagBounds, 500);
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote signal
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
     const int total = E * a.mt * a.nth * a.halves;
     volatile int* abort_flag = &m->abort_flag;
 
     if (warp == 0 && lane == 0) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (each CTA)
         int stage = 0;
         uint32_t phase = 0;
         int last_phase[STAGES];
         for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = unit; t < total && ok; t += units) {
             int e, m0, hf, n0;
-            decode(a, t, e, m0, hf, n0);
+            decode(a, BM, t, e, m0, hf, n0);
             const int r0 = m->off[e], r1 = m->off[e + 1];
-            const int bcol = hf * a.Nh + n0;
+            const int acol = m0 + 128 * (int)rank;                      // this CTA's A columns
+            const int bcol = hf * a.Nh + n0 + (PAIR ? 128 * (int)rank : 0);  // and B columns
             for (int k = r0; k < r1; k += BK) {
                 if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) {
                     ok = false;
                     break;
                 }
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
-                uint8_t* sB = sA + A_BYTES;
-                uint64_t* fb = &m->full[stage];
-                mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                uint8_t* sB = sA + G::A_BYTES;
+                if (PAIR) {
+                    // both CTAs' bytes are counted on the leader's full barrier
+                    if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
 #pragma unroll
-                for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, &tmA, m0 + 64 * j, k, fb);
+                    for (int j = 0; j < G::A_BOXES; ++j)
+                        tma_load_2d_pair(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, fb);
 #pragma unroll
-                for (int j = 0; j < B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
+                    for (int j = 0; j < G::B_BOXES; ++j)
+                        tma_load_2d_pair(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
+                } else {
+                    uint64_t* fb = &m->full[stage];
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+#pragma unroll
+                    for (int j = 0; j < G::A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, fb);
+#pragma unroll
+                    for (int j = 0; j < G::B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
+                }
                 last_phase[stage] = (int)phase;
                 if (++stage == STAGES) {
                     stage = 0;
@@ -181,10 +220,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
         }
-        for (int s = 0; s < STAGES; ++s)
-            if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
-    } else if (warp == 1) {
-        // ------------------------------------------- MMA issuer (whole warp)
+        // never leave the CTA with a copy in flight (the leader sees every completion)
+        if (!PAIR || rank == 0)
+            for (int s = 0; s < STAGES; ++s)
+                if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
+    } else if (warp == 1 && rank == 0) {
+        // -------------------------------- MMA issuer (leader; whole warp)
         // A and B MN-major: 64-column boxes 8 KB apart (LBO), 8-row K groups
         // 1024 B apart (SBO), +2048 B per 16-row K step
         constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, 1, 1);
@@ -193,9 +234,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = unit; t < total && ok; t += units) {
             int e, m0, hf, n0;
-            decode(a, t, e, m0, hf, n0);
+            decode(a, BM, t, e, m0, hf, n0);
             const int r0 = m->off[e], r1 = m->off[e + 1];
             // every lane waits (each wait is bounded); the vote keeps the warp converged
             if (!__all_sync(0xffffffffu, mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 520, abort_flag)))
@@ -210,29 +251,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
                 const int valid = r1 - k;
                 if (valid < BK) {
-                    // rows valid..63 of this block belong to the next expert (or
-                    // lie past the end): zero them in every box of the stage
+                    // rows valid..63 of this block belong to the next expert or lie
+                    // past the written rows: zero them in every box of the stage, in
+                    // both CTAs of a pair (the peer's through its shared::cluster
+                    // address; every copy of the stage has landed: the full barrier
+                    // counts both CTAs' bytes)
                     const int n16 = (BK - valid) * 8;  // 16-byte words per box
+                    const uint32_t base = smem_u32(sA) + (uint32_t)(valid * 128);
 #pragma unroll 1
-                    for (int b = 0; b < A_BOXES + B_BOXES; ++b) {
-                        uint4* p = reinterpret_cast<uint4*>(sA + b * BOX_BYTES + valid * 128);
-                        for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0, 0, 0, 0);
+                    for (uint32_t cta = 0; cta < (uint32_t)G::CTAS; ++cta) {
+                        const uint32_t cbase = PAIR ? mapa_shared(base, cta) : base;
+#pragma unroll 1
+                        for (int b = 0; b < G::A_BOXES + G::B_BOXES; ++b)
+                            for (int i = lane; i < n16; i += 32)
+                                st_cluster_zero16(cbase + (uint32_t)(b * BOX_BYTES + i * 16));
                     }
-                    fence_proxy_async_smem();
+                    fence_proxy_async_cluster();
                 }
                 __syncwarp();
                 if (lane == 0) {
                     tc_fence_after();
                     const uint32_t a32 = smem_u32(sA);
-                    const uint32_t b32 = a32 + A_BYTES;
+                    const uint32_t b32 = a32 + G::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
                         const uint32_t accum = (k != r0 || kk != 0) ? 1u : 0u;
                         const uint64_t adesc = umma_desc_sw128(a32 + kk * 2048, BOX_BYTES, 1024);
                         const uint64_t bdesc = umma_desc_sw128(b32 + kk * 2048, BOX_BYTES, 1024);
-                        umma_f16_ss(d0, adesc, bdesc, idesc, accum);
+                        if (PAIR) umma_f16_ss_pair(d0, adesc, bdesc, idesc, accum);
+                        else umma_f16_ss(d0, adesc, bdesc, idesc, accum);
                     }
-                    umma_commit(&m->empty[stage]);
+                    // frees the stage (in both CTAs) once these MMAs complete
+                    if (PAIR) umma_commit_pair_mc(&m->empty[stage], 0x3);
+                    else umma_commit(&m->empty[stage]);
                 }
                 __syncwarp();
                 if (++stage == STAGES) {
@@ -241,7 +292,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
             if (!ok) break;
-            if (lane == 0) umma_commit(&m->tfull[acc]);  // with no rows: arrives at once
+            if (lane == 0) {  // with no rows: arrives at once
+                if (PAIR) umma_commit_pair_mc(&m->tfull[acc], 0x3);
+                else umma_commit(&m->tfull[acc]);
+            }
             __syncwarp();
             if (++acc == 2) {
                 acc = 0;
@@ -249,23 +303,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
         }
         if (lane == 0) {
-            umma_commit(&m->drain);
+            if (PAIR) umma_commit_pair_mc(&m->drain, 0x1);
+            else umma_commit(&m->drain);
             mbar_wait(&m->drain, 0, a.status, 522, nullptr);
         }
         __syncwarp();
     } else if (warp >= 2) {
         // -------------------------------------------------------- epilogue
-        // warp w: tensor-memory lanes 32*(w%4) .. +31 (output rows), half of
-        // the 256 columns (warps 2..5 the first, 6..9 the second)
+        // warp w: tensor-memory lanes 32*(w%4) .. +31 (this CTA's output rows),
+        // half of the 256 columns (warps 2..5 the first, 6..9 the second)
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
         uint8_t* buf = outbuf + (size_t)(warp - 2) * OUT_BYTES;
         const int swz = lane & 7;  // the 128-byte swizzle of this lane's staged row
+        const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m->tempty[0]), 0);
+        const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m->tempty[1]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        for (int t = unit; t < total; t += units) {
             int e, m0, hf, n0;
-            decode(a, t, e, m0, hf, n0);
+            decode(a, BM, t, e, m0, hf, n0);
             const bool empty_block = m->off[e + 1] == m->off[e];
             // tcgen05.ld is warp-collective: the vote keeps the warp converged
             if (!__all_sync(0xffffffffu, mbar_wait(&m->tfull[acc], acc_phase, a.status, 530, abort_flag)))
@@ -273,6 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
             const CUtensorMap* tmo = hf ? &tmO1 : &tmO0;
+            const int orow = m0 + 128 * (int)rank + quad * 32;
 #pragma unroll 1
             for (int c = 4 * half; c < 4 * half + 4; ++c) {
                 uint32_t v[32];
@@ -288,13 +346,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {  // rows >= M and columns >= Nh fall outside the map: not written
-                    tma_store_3d(tmo, buf, n0 + c * 32, m0 + quad * 32, e);
+                    tma_store_3d(tmo, buf, n0 + c * 32, orow, e);
                     bulk_commit();
                 }
             }
+            // this warp is done reading the accumulator: one arrival, on the leader
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&m->tempty[acc]);
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+                else mbar_arrive(&m->tempty[acc]);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -304,10 +366,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync();  // no CTA leaves while its peer may still signal it
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
@@ -360,32 +424,81 @@ static bool map_out(CUtensorMap* m, const float* base, uint64_t Nh, uint64_t M, 
                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static cudaError_t prepare(int* ctas)
+// Per device and mode: dynamic shared memory opted in, and how many CTAs (or
+// CTA pairs) can be resident at once, which sizes the persistent grid.
+template <bool PAIR> static cudaError_t prepare(int* units_out)
 {
     static int cached[32];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 32 && cached[dev] > 0) {
-        *ctas = cached[dev];
+        *units_out = cached[dev];
         return cudaSuccess;
     }
-    e = cudaFuncSetAttribute(wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_bytes());
+    constexpr size_t smem = smem_bytes<PAIR>();
+    e = cudaFuncSetAttribute(wgrad_tc_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int sms = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    if (sms < 1) return cudaErrorInvalidConfiguration;
-    if (dev < 32) cached[dev] = sms;
-    *ctas = sms;
+    int units = 0;
+    if (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaOccupancyMaxActiveClusters(&units, wgrad_tc_kernel<true>, &cfg);
+        if (e != cudaSuccess) return e;
+    } else {
+        e = cudaDeviceGetAttribute(&units, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    if (units < 1) return cudaErrorInvalidConfiguration;
+    if (dev < 32) cached[dev] = units;
+    *units_out = units;
     return cudaSuccess;
+}
+
+template <bool PAIR>
+static cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mO0,
+                               const CUtensorMap& mO1, Args a, cudaStream_t s)
+{
+    int units = 0;
+    cudaError_t e = prepare<PAIR>(&units);
+    if (e != cudaSuccess) return e;
+    a.mt = (a.M + Geo<PAIR>::BM - 1) / Geo<PAIR>::BM;
+    const int64_t total = (int64_t)a.E * a.mt * a.nth * a.halves;
+    const int n = (int)(total < units ? total : units);
+    constexpr size_t smem = smem_bytes<PAIR>();
+    if (!PAIR) {
+        wgrad_tc_kernel<false><<<n, NUM_THREADS, smem, s>>>(mA, mB, mO0, mO1, a);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * n), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, wgrad_tc_kernel<true>, mA, mB, mO0, mO1, a);
 }
 
 }  // namespace wg
 
 // out0/out1 (E, M, Nh) fp32 = for each expert, A[block]^T . B[block] with A
-// (max_rows, M) and B (max_rows, halves * Nh) bf16 row-major.
+// (max_rows, M) and B (max_rows, halves * Nh) bf16 row-major.  CTA pairs
+// (256-row output tiles) when M >= 256, single CTAs otherwise.
 cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets, const void* A,
                                  int M, const void* B, int Nh, int halves, float* out0, float* out1,
                                  int* status, cudaStream_t s)
@@ -398,15 +511,8 @@ cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets
         !map_out(&mO0, out0, (uint64_t)Nh, (uint64_t)M, (uint64_t)E) ||
         !map_out(&mO1, halves == 2 ? out1 : out0, (uint64_t)Nh, (uint64_t)M, (uint64_t)E))
         return cudaErrorInvalidValue;
-    int ctas = 0;
-    cudaError_t e = prepare(&ctas);
-    if (e != cudaSuccess) return e;
-    Args a{offsets, out0, halves == 2 ? out1 : out0, E, M, Nh, halves, (M + BM - 1) / BM,
-           (Nh + BN - 1) / BN, max_rows, status};
-    const int64_t total = (int64_t)E * a.mt * a.nth * a.halves;
-    const int grid = (int)(total < ctas ? total : ctas);
-    wgrad_tc_kernel<<<grid, NUM_THREADS, smem_bytes(), s>>>(mA, mB, mO0, mO1, a);
-    return cudaGetLastError();
+    Args a{offsets, E, M, Nh, halves, 0, (Nh + BN - 1) / BN, max_rows, status};
+    return M >= 256 ? launch_mode<true>(mA, mB, mO0, mO1, a, s) : launch_mode<false>(mA, mB, mO0, mO1, a, s);
 }
 
 }  // namespace moe
