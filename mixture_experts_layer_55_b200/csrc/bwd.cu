@@ -228,46 +228,81 @@ MOE_DEVICE void store8(float* p, const float (&v)[8])
     reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-constexpr int kRwThreads = 128;  // x 8 d = 1024 d per block
-constexpr int kRwE = 8;          // experts per block
+constexpr int kRwCols = 256;  // d per block
+constexpr int kRwE = 32;      // experts per block
+constexpr int kRwTok = 32;    // tokens staged per step
 
-// part[z][d][e] = sum over the tokens of split z of x[t,d] * dL[t,e]: each
-// thread owns 8 consecutive d and the block's 8 experts (64 accumulators).
+// part[z][d][e] = sum over the tokens of split z of x[t,d] * dL[t,e].  Block:
+// 256 d x 32 experts, 256 threads; thread (ty = warp, tx = lane) owns
+// d = 8 tx .. 8 tx + 7 and experts 4 ty .. 4 ty + 3.  Tokens are staged 32 at
+// a time (x with 16-byte loads; dL reads in the loop are warp broadcasts).
 template <typename XT>
-__global__ void __launch_bounds__(kRwThreads) router_wgrad_partial_kernel(const XT* __restrict__ x,
-                                                                          const float* __restrict__ dL,
-                                                                          float* __restrict__ part,
-                                                                          int64_t T, int D, int E,
-                                                                          int64_t t_per_split)
+__global__ void __launch_bounds__(256) router_wgrad_partial_kernel(const XT* __restrict__ x,
+                                                                   const float* __restrict__ dL,
+                                                                   float* __restrict__ part, int64_t T,
+                                                                   int D, int E, int64_t t_per_split)
 {
-    const int d0 = (blockIdx.x * kRwThreads + threadIdx.x) * 8;
+    __shared__ __align__(16) XT sx[kRwTok][kRwCols];
+    __shared__ float sdl[kRwTok][kRwE];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int dblk = blockIdx.x * kRwCols;
     const int e0 = blockIdx.y * kRwE;
     const int64_t t0 = (int64_t)blockIdx.z * t_per_split;
     const int64_t t1 = t0 + t_per_split < T ? t0 + t_per_split : T;
-    if (d0 >= D) return;
-    float acc[8][kRwE];
+    constexpr int VEC = 16 / sizeof(XT);  // elements per 16-byte load
+    float acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < kRwE; ++j) acc[i][j] = 0.f;
-    const int ne = E - e0 < kRwE ? E - e0 : kRwE;
-#pragma unroll 2
-    for (int64_t t = t0; t < t1; ++t) {
-        float xv[8], g[kRwE];
-        load8(x + t * D + d0, xv);
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int64_t tc = t0; tc < t1; tc += kRwTok) {
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < kRwTok * kRwCols / VEC; idx += 256) {
+            const int tt = idx / (kRwCols / VEC), v = idx - tt * (kRwCols / VEC);
+            const int d = dblk + v * VEC;
+            uint4 q = make_uint4(0, 0, 0, 0);
+            if (tc + tt < t1 && d < D) q = __ldg(reinterpret_cast<const uint4*>(x + (tc + tt) * D + d));
+            *reinterpret_cast<uint4*>(&sx[tt][v * VEC]) = q;
+        }
+        for (int idx = threadIdx.x; idx < kRwTok * kRwE; idx += 256) {
+            const int tt = idx / kRwE, el = idx - tt * kRwE;
+            sdl[tt][el] = (tc + tt < t1 && e0 + el < E) ? __ldg(dL + (tc + tt) * E + e0 + el) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int tt = 0; tt < kRwTok; ++tt) {
+            float xv[8];
+            if constexpr (sizeof(XT) == 2) {
+                const uint4 q = *reinterpret_cast<const uint4*>(&sx[tt][tx * 8]);
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int j = 0; j < kRwE; ++j) g[j] = j < ne ? __ldg(dL + t * E + e0 + j) : 0.f;
+                for (int i = 0; i < 4; ++i) {
+                    xv[2 * i] = __uint_as_float(w[i] << 16);
+                    xv[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+                }
+            } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 8; ++i) xv[i] = to_f32(sx[tt][tx * 8 + i]);
+            }
+            float g[4];
 #pragma unroll
-            for (int j = 0; j < kRwE; ++j) acc[i][j] = fmaf(xv[i], g[j], acc[i][j]);
+            for (int j = 0; j < 4; ++j) g[j] = sdl[tt][ty * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xv[i], g[j], acc[i][j]);
+        }
     }
-    float* out = part + ((int64_t)blockIdx.z * D + d0) * E + e0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 8; ++i) {
+        const int d = dblk + tx * 8 + i;
+        if (d >= D) break;
 #pragma unroll
-        for (int j = 0; j < kRwE; ++j)
-            if (j < ne) out[(int64_t)i * E + j] = acc[i][j];
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + ty * 4 + j;
+            if (e < E) part[((int64_t)blockIdx.z * D + d) * E + e] = acc[i][j];
+        }
+    }
 }
 
 // dW[d][e] = sum over splits in order.
@@ -300,95 +335,83 @@ __global__ void __launch_bounds__(256) router_bias_grad_kernel(const float* __re
 }
 
 // --------------------------------------------------------------------- dx --
-// Block: kDxTok tokens (in groups of kDxGroup) x 1024 d; each thread owns 8
-// consecutive d.  The router term dL W_r^T runs over the experts 8 at a time:
-// the block's 1024 x 8 slice of W_r is staged transposed in shared memory
-// (coalesced global reads, conflict-free 16-byte shared reads), once per block
-// when E <= 8.  Then each token's kept rows of dXp (slot order) and the shared
-// expert's row are added as 16-byte vectors and the sum is rounded once.
-constexpr int kDxTok = 32;
-constexpr int kDxGroup = 8;
-constexpr int kDxThreads = 128;
+// Block: 64 tokens x 256 d, 256 threads; thread (ty = warp, tx = lane) owns
+// tokens 8 ty .. 8 ty + 7 and d = 8 tx .. 8 tx + 7 of the tile.  The router
+// term dL W_r^T is a small product over the experts, 32 at a time: the
+// chunk's W_r^T (32 x 256, fp32) and dL (64 x 32) are staged in shared memory
+// (lanes walk d when writing W_r^T, so the stores are conflict-free; the
+// 16-byte reads of a W_r^T row are too, and dL reads are warp broadcasts).
+// Then each token's kept rows of dXp (slot order) and the shared expert's row
+// are added as 16-byte vectors, and the sum is rounded once.
+constexpr int kDxTok = 64;
+constexpr int kDxCols = 256;
+constexpr int kDxE = 32;
 
 template <typename ET>
-__global__ void __launch_bounds__(kDxThreads) dx_assemble_kernel(const float* __restrict__ dL,
-                                                                 const float* __restrict__ w_r,
-                                                                 const ET* __restrict__ dxp,
-                                                                 const int32_t* __restrict__ row_of,
-                                                                 const ET* __restrict__ dx_shared,
-                                                                 ET* __restrict__ dx, int64_t T, int D,
-                                                                 int E, int K, int64_t max_rows)
+__global__ void __launch_bounds__(256) dx_assemble_kernel(const float* __restrict__ dL,
+                                                          const float* __restrict__ w_r,
+                                                          const ET* __restrict__ dxp,
+                                                          const int32_t* __restrict__ row_of,
+                                                          const ET* __restrict__ dx_shared,
+                                                          ET* __restrict__ dx, int64_t T, int D, int E,
+                                                          int K, int64_t max_rows)
 {
-    __shared__ __align__(16) float swt[8][kDxThreads * 8];  // W_r^T chunk: 8 experts x 1024 d
-    __shared__ float sdl[kDxGroup][8];
-    const int dblk = blockIdx.x * kDxThreads * 8;
-    const int d0 = dblk + threadIdx.x * 8;
-    const bool active = d0 < D;
-    for (int g0 = 0; g0 < kDxTok; g0 += kDxGroup) {
-        const int64_t tb = (int64_t)blockIdx.y * kDxTok + g0;
-        if (tb >= T) break;  // uniform across the block
-        float acc[kDxGroup][8];
+    __shared__ __align__(16) float swt[kDxE][kDxCols];
+    __shared__ float sdl[kDxTok][kDxE + 1];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int dblk = blockIdx.x * kDxCols;
+    const int64_t tb = (int64_t)blockIdx.y * kDxTok;
+    const int d0 = dblk + tx * 8;
+    float acc[8][8];
 #pragma unroll
-        for (int i = 0; i < kDxGroup; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-        for (int e0 = 0; e0 < E; e0 += 8) {
-            __syncthreads();  // the previous chunk's shared reads are done
-            if (E > 8 || g0 == 0) {
-#pragma unroll 1
-                for (int r = 0; r < 8; ++r) {
-                    const int il = threadIdx.x + kDxThreads * r;
-                    const int d = dblk + il;
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += kDxE) {
+        __syncthreads();  // the previous chunk's shared reads are done
+        for (int idx = threadIdx.x; idx < kDxE * kDxCols; idx += 256) {
+            const int el = idx / kDxCols, dl = idx - el * kDxCols;
+            const int d = dblk + dl;
+            swt[el][dl] = (d < D && e0 + el < E) ? __ldg(w_r + (int64_t)d * E + e0 + el) : 0.f;
+        }
+        for (int idx = threadIdx.x; idx < kDxTok * kDxE; idx += 256) {
+            const int tt = idx / kDxE, el = idx - tt * kDxE;
+            sdl[tt][el] = (tb + tt < T && e0 + el < E) ? __ldg(dL + (tb + tt) * E + e0 + el) : 0.f;
+        }
+        __syncthreads();
+        const int ne = E - e0 < kDxE ? E - e0 : kDxE;
+        for (int e = 0; e < ne; ++e) {
+            const float4 lo = *reinterpret_cast<const float4*>(&swt[e][tx * 8]);
+            const float4 hi = *reinterpret_cast<const float4*>(&swt[e][tx * 8 + 4]);
+            const float w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        swt[k][il] = (d < D && e0 + k < E) ? __ldg(w_r + (int64_t)d * E + e0 + k) : 0.f;
-                }
-            }
-            if (threadIdx.x < kDxGroup * 8) {
-                const int tt = threadIdx.x >> 3, k = threadIdx.x & 7;
-                sdl[tt][k] = (tb + tt < T && e0 + k < E) ? __ldg(dL + (tb + tt) * E + e0 + k) : 0.f;
-            }
-            __syncthreads();
-            if (active) {
-                float w[8][8];  // w[j][k] = W_r[d0 + j][e0 + k]
+            for (int i = 0; i < 8; ++i) {
+                const float g = sdl[ty * 8 + i][e];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float4 lo = *reinterpret_cast<const float4*>(&swt[k][threadIdx.x * 8]);
-                    const float4 hi = *reinterpret_cast<const float4*>(&swt[k][threadIdx.x * 8 + 4]);
-                    w[0][k] = lo.x; w[1][k] = lo.y; w[2][k] = lo.z; w[3][k] = lo.w;
-                    w[4][k] = hi.x; w[5][k] = hi.y; w[6][k] = hi.z; w[7][k] = hi.w;
-                }
-#pragma unroll
-                for (int i = 0; i < kDxGroup; ++i)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float gk = sdl[i][k];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(gk, w[j][k], acc[i][j]);
-                    }
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(g, w[j], acc[i][j]);
             }
         }
-        if (!active) continue;
+    }
+    if (d0 >= D) return;
 #pragma unroll
-        for (int i = 0; i < kDxGroup; ++i) {
-            const int64_t t = tb + i;
-            if (t >= T) break;
-            for (int k = 0; k < K; ++k) {
-                const int32_t r = __ldg(row_of + t * K + k);
-                if (r < 0 || r >= max_rows) continue;
-                float v[8];
-                load8(dxp + (int64_t)r * D + d0, v);
+    for (int i = 0; i < 8; ++i) {
+        const int64_t t = tb + ty * 8 + i;
+        if (t >= T) break;
+        for (int k = 0; k < K; ++k) {
+            const int32_t r = __ldg(row_of + t * K + k);
+            if (r < 0 || r >= max_rows) continue;
+            float v[8];
+            load8(dxp + (int64_t)r * D + d0, v);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
-            }
-            if (dx_shared) {
-                float v[8];
-                load8(dx_shared + t * D + d0, v);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
-            }
-            store8(dx + t * D + d0, acc[i]);
+            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
         }
+        if (dx_shared) {
+            float v[8];
+            load8(dx_shared + t * D + d0, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+        }
+        store8(dx + t * D + d0, acc[i]);
     }
 }
 
@@ -430,11 +453,11 @@ cudaError_t launch_router_bwd(const moe_config& c, const float* logits, const in
 
 int router_wgrad_splits(const moe_config& c)
 {
-    // about four waves of blocks; each split at least 32 tokens
-    const int64_t dblocks = (c.D + kRwThreads * 8 - 1) / (kRwThreads * 8);
+    // about four waves of blocks; each split at least 64 tokens
+    const int64_t dblocks = (c.D + kRwCols - 1) / kRwCols;
     const int64_t eblocks = (c.E + kRwE - 1) / kRwE;
     int64_t want = (int64_t)sm_count() * 4 / (dblocks * eblocks);
-    int64_t most = (c.T + 31) / 32;
+    int64_t most = (c.T + 63) / 64;
     int64_t sp = want < most ? want : most;
     if (sp < 1) sp = 1;
     if (sp > 256) sp = 256;
@@ -450,14 +473,14 @@ cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float*
                                 int splits, float* dw, float* db, cudaStream_t s)
 {
     const int64_t tps = (c.T + splits - 1) / splits;
-    const dim3 grid((unsigned)((c.D + kRwThreads * 8 - 1) / (kRwThreads * 8)),
-                    (unsigned)((c.E + kRwE - 1) / kRwE), (unsigned)splits);
+    const dim3 grid((unsigned)((c.D + kRwCols - 1) / kRwCols), (unsigned)((c.E + kRwE - 1) / kRwE),
+                    (unsigned)splits);
     if (c.dtype == MOE_BF16)
-        router_wgrad_partial_kernel<__nv_bfloat16><<<grid, kRwThreads, 0, s>>>(
+        router_wgrad_partial_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(x), dL, part, c.T, c.D, c.E, tps);
     else
-        router_wgrad_partial_kernel<float><<<grid, kRwThreads, 0, s>>>(static_cast<const float*>(x), dL,
-                                                                       part, c.T, c.D, c.E, tps);
+        router_wgrad_partial_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), dL, part,
+                                                                c.T, c.D, c.E, tps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t n = (int64_t)c.D * c.E;
@@ -474,15 +497,14 @@ cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float
                                const int32_t* row_of, const void* dx_shared, void* dx,
                                int64_t max_rows, cudaStream_t s)
 {
-    const dim3 grid((unsigned)((c.D + kDxThreads * 8 - 1) / (kDxThreads * 8)),
-                    (unsigned)((c.T + kDxTok - 1) / kDxTok));
+    const dim3 grid((unsigned)((c.D + kDxCols - 1) / kDxCols), (unsigned)((c.T + kDxTok - 1) / kDxTok));
     if (c.dtype == MOE_BF16)
-        dx_assemble_kernel<__nv_bfloat16><<<grid, kDxThreads, 0, s>>>(
+        dx_assemble_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
             dL, w_r, static_cast<const __nv_bfloat16*>(dxp), row_of,
             static_cast<const __nv_bfloat16*>(dx_shared), static_cast<__nv_bfloat16*>(dx), c.T, c.D,
             c.E, c.K, max_rows);
     else
-        dx_assemble_kernel<float><<<grid, kDxThreads, 0, s>>>(dL, w_r, static_cast<const float*>(dxp), row_of,
+        dx_assemble_kernel<float><<<grid, 256, 0, s>>>(dL, w_r, static_cast<const float*>(dxp), row_of,
                                                               static_cast<const float*>(dx_shared),
                                                               static_cast<float*>(dx), c.T, c.D, c.E, c.K,
                                                               max_rows);
