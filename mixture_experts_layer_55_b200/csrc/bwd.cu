@@ -347,7 +347,7 @@ constexpr int kDxTok = 64;
 constexpr int kDxCols = 256;
 constexpr int kDxE = 32;
 
-template <typename ET>
+template <typename ET, int KS>
 __global__ void __launch_bounds__(256) dx_assemble_kernel(const float* __restrict__ dL,
                                                           const float* __restrict__ w_r,
                                                           const ET* __restrict__ dxp,
@@ -397,14 +397,25 @@ __global__ void __launch_bounds__(256) dx_assemble_kernel(const float* __restric
     for (int i = 0; i < 8; ++i) {
         const int64_t t = tb + ty * 8 + i;
         if (t >= T) break;
-        for (int k = 0; k < K; ++k) {
-            const int32_t r = __ldg(row_of + t * K + k);
-            if (r < 0 || r >= max_rows) continue;
-            float v[8];
-            load8(dxp + (int64_t)r * D + d0, v);
+        // the token's KS >= K slot rows: indices first, then all loads in flight together
+        int32_t rows[KS];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+        for (int k = 0; k < KS; ++k) {
+            const int32_t r = k < K ? __ldg(row_of + t * K + k) : -1;
+            rows[k] = (r >= 0 && r < max_rows) ? r : -1;
         }
+        float v[KS][8];
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            if (rows[k] >= 0) load8(dxp + (int64_t)rows[k] * D + d0, v[k]);
+            else
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[k][j] = 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < KS; ++k)  // slot order
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] += v[k][j];
         if (dx_shared) {
             float v[8];
             load8(dx_shared + t * D + d0, v);
@@ -493,21 +504,36 @@ cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float*
     return cudaGetLastError();
 }
 
+template <typename ET, int KS>
+static void dx_launch(const moe_config& c, dim3 grid, const float* dL, const float* w_r, const void* dxp,
+                      const int32_t* row_of, const void* dx_shared, void* dx, int64_t max_rows,
+                      cudaStream_t s)
+{
+    dx_assemble_kernel<ET, KS><<<grid, 256, 0, s>>>(dL, w_r, static_cast<const ET*>(dxp), row_of,
+                                                    static_cast<const ET*>(dx_shared), static_cast<ET*>(dx),
+                                                    c.T, c.D, c.E, c.K, max_rows);
+}
+
+template <typename ET>
+static void dx_launch_k(const moe_config& c, dim3 grid, const float* dL, const float* w_r, const void* dxp,
+                        const int32_t* row_of, const void* dx_shared, void* dx, int64_t max_rows,
+                        cudaStream_t s)
+{
+    if (c.K <= 1) dx_launch<ET, 1>(c, grid, dL, w_r, dxp, row_of, dx_shared, dx, max_rows, s);
+    else if (c.K == 2) dx_launch<ET, 2>(c, grid, dL, w_r, dxp, row_of, dx_shared, dx, max_rows, s);
+    else if (c.K <= 4) dx_launch<ET, 4>(c, grid, dL, w_r, dxp, row_of, dx_shared, dx, max_rows, s);
+    else dx_launch<ET, 8>(c, grid, dL, w_r, dxp, row_of, dx_shared, dx, max_rows, s);
+}
+
 cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float* w_r, const void* dxp,
                                const int32_t* row_of, const void* dx_shared, void* dx,
                                int64_t max_rows, cudaStream_t s)
 {
     const dim3 grid((unsigned)((c.D + kDxCols - 1) / kDxCols), (unsigned)((c.T + kDxTok - 1) / kDxTok));
     if (c.dtype == MOE_BF16)
-        dx_assemble_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            dL, w_r, static_cast<const __nv_bfloat16*>(dxp), row_of,
-            static_cast<const __nv_bfloat16*>(dx_shared), static_cast<__nv_bfloat16*>(dx), c.T, c.D,
-            c.E, c.K, max_rows);
+        dx_launch_k<__nv_bfloat16>(c, grid, dL, w_r, dxp, row_of, dx_shared, dx, max_rows, s);
     else
-        dx_assemble_kernel<float><<<grid, 256, 0, s>>>(dL, w_r, static_cast<const float*>(dxp), row_of,
-                                                              static_cast<const float*>(dx_shared),
-                                                              static_cast<float*>(dx), c.T, c.D, c.E, c.K,
-                                                              max_rows);
+        dx_launch_k<float>(c, grid, dL, w_r, dxp, row_of, dx_shared, dx, max_rows, s);
     return cudaGetLastError();
 }
 

@@ -20,10 +20,11 @@
 // Persistent kernel, one CTA per SM, tiles M = 128 x N = 256, 4-stage ring of
 // 48 KB, double-buffered 2 x 256-column accumulators.  10 warps: warp 0 TMA,
 // warp 1 MMA (all lanes wait and zero; one issues), warps 2..9 epilogue.  The
-// epilogue stages each warp's 32 x 32 fp32 piece in shared memory (128-byte
-// swizzle, conflict-free) and writes it with a TMA tensor store over an
-// (E, M, N) map, so the stores are whole lines and the map clips the tile's
-// edges per expert.  Every wait is bounded (device status flag).
+// epilogue stages each warp's 32 x 32 fp32 pieces in shared memory (128-byte
+// swizzle, conflict-free; two buffers per warp, so a store's read of one
+// overlaps the filling of the other) and writes them with TMA tensor stores
+// over an (E, M, N) map, so the stores are whole lines and the map clips the
+// tile's edges per expert.  Every wait is bounded (device status flag).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -36,7 +37,8 @@ constexpr int BN = 256;                 // output columns per tile
 constexpr int BK = 64;                  // K rows per stage
 constexpr int UK = 16;                  // K per tcgen05.mma (bf16)
 constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64-column x 64-row box
-constexpr int OUT_BYTES = 32 * 32 * 4;  // one epilogue warp's staged 32 x 32 fp32 piece
+constexpr int OUT_BYTES = 32 * 32 * 4;  // one staged 32 x 32 fp32 piece
+constexpr int OUT_BUFS = 2;             // staged pieces per epilogue warp (double-buffered)
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 320;
@@ -44,8 +46,8 @@ constexpr int EPI_WARPS = 8;
 constexpr int MAX_E = 256;
 
 // Single CTA: M = 128 output rows, all 256 columns in this CTA (2 A + 4 B
-// boxes per stage, 4 stages).  CTA pair: M = 256, each CTA its 128 rows of A
-// and 128 of the columns of B (2 + 2 boxes, 6 stages); the leader issues.
+// boxes per stage, 3 stages).  CTA pair: M = 256, each CTA its 128 rows of A
+// and 128 of the columns of B (2 + 2 boxes, 5 stages); the leader issues.
 template <bool PAIR> struct Geo {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BM = 128 * CTAS;
@@ -53,7 +55,7 @@ template <bool PAIR> struct Geo {
     static constexpr int B_BOXES = 4 / CTAS;
     static constexpr int A_BYTES = A_BOXES * BOX_BYTES;
     static constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;  // 48 KB single, 32 KB pair
-    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int STAGES = PAIR ? 5 : 3;
     static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;
 };
 
@@ -70,8 +72,8 @@ struct Misc {
 
 template <bool PAIR> constexpr size_t smem_bytes()
 {
-    return 1024 + (size_t)Geo<PAIR>::STAGES * Geo<PAIR>::STAGE_BYTES + (size_t)EPI_WARPS * OUT_BYTES +
-           sizeof(Misc);
+    return 1024 + (size_t)Geo<PAIR>::STAGES * Geo<PAIR>::STAGE_BYTES +
+           (size_t)EPI_WARPS * OUT_BUFS * OUT_BYTES + sizeof(Misc);
 }
 static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory per block");
 
@@ -117,8 +119,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* stages = smem;
-    uint8_t* outbuf = smem + (size_t)STAGES * STAGE_BYTES;  // EPI_WARPS x OUT_BYTES, 1 KB aligned
-    Misc* m = reinterpret_cast<Misc*>(outbuf + (size_t)EPI_WARPS * OUT_BYTES);
+    uint8_t* outbuf = smem + (size_t)STAGES * STAGE_BYTES;  // EPI_WARPS x OUT_BUFS pieces, 1 KB aligned
+    Misc* m = reinterpret_cast<Misc*>(outbuf + (size_t)EPI_WARPS * OUT_BUFS * OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = a.E;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader (issues the MMAs)
@@ -314,7 +316,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // half of the 256 columns (warps 2..5 the first, 6..9 the second)
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
-        uint8_t* buf = outbuf + (size_t)(warp - 2) * OUT_BYTES;
+        uint8_t* bufs = outbuf + (size_t)(warp - 2) * OUT_BUFS * OUT_BYTES;
+        int nb = 0;  // the staging buffer to fill next
         const int swz = lane & 7;  // the 128-byte swizzle of this lane's staged row
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m->tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m->tempty[1]), 0);
@@ -336,7 +339,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, v);
                 tmem_ld_wait();
-                if (lane == 0) bulk_wait_read<0>();  // the previous store has read the buffer
+                uint8_t* buf = bufs + nb * OUT_BYTES;
+                nb ^= 1;
+                if (lane == 0) bulk_wait_read<1>();  // the store before last has read this buffer
                 __syncwarp();
                 uint4* row = reinterpret_cast<uint4*>(buf + lane * 128);
 #pragma unroll
