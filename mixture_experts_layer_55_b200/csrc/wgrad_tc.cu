@@ -21,10 +21,10 @@
 // 48 KB, double-buffered 2 x 256-column accumulators.  10 warps: warp 0 TMA,
 // warp 1 MMA (all lanes wait and zero; one issues), warps 2..9 epilogue.  The
 // epilogue stages each warp's 32 x 32 fp32 pieces in shared memory (128-byte
-// swizzle, conflict-free; two buffers per warp, so a store's read of one
-// overlaps the filling of the other) and writes them with TMA tensor stores
-// over an (E, M, N) map, so the stores are whole lines and the map clips the
-// tile's edges per expert.  Every wait is bounded (device status flag).
+// swizzle, conflict-free) and writes them with TMA tensor stores over an
+// (E, M, N) map, so the stores are whole lines and the map clips the tile's
+// edges per expert.  (Measured: six operand stages with one staging buffer per
+// warp beat five stages with two.)  Every wait is bounded (device status flag).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -38,16 +38,17 @@ constexpr int BK = 64;                  // K rows per stage
 constexpr int UK = 16;                  // K per tcgen05.mma (bf16)
 constexpr int BOX_BYTES = 64 * 64 * 2;  // one 64-column x 64-row box
 constexpr int OUT_BYTES = 32 * 32 * 4;  // one staged 32 x 32 fp32 piece
-constexpr int OUT_BUFS = 2;             // staged pieces per epilogue warp (double-buffered)
+constexpr int OUT_BUFS = 1;             // staged pieces per epilogue warp
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 352;  // warp 0 TMA, 1 MMA, 2..9 epilogue, 10 tail fixer
 constexpr int EPI_WARPS = 8;
+constexpr int FIX_WARP = 2 + EPI_WARPS;
 constexpr int MAX_E = 256;
 
 // Single CTA: M = 128 output rows, all 256 columns in this CTA (2 A + 4 B
-// boxes per stage, 3 stages).  CTA pair: M = 256, each CTA its 128 rows of A
-// and 128 of the columns of B (2 + 2 boxes, 5 stages); the leader issues.
+// boxes per stage, 4 stages).  CTA pair: M = 256, each CTA its 128 rows of A
+// and 128 of the columns of B (2 + 2 boxes, 6 stages); the leader issues.
 template <bool PAIR> struct Geo {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BM = 128 * CTAS;
@@ -55,13 +56,15 @@ template <bool PAIR> struct Geo {
     static constexpr int B_BOXES = 4 / CTAS;
     static constexpr int A_BYTES = A_BOXES * BOX_BYTES;
     static constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;  // 48 KB single, 32 KB pair
-    static constexpr int STAGES = PAIR ? 5 : 3;
+    static constexpr int STAGES = PAIR ? 6 : 4;
     static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;
 };
 
 struct Misc {
     uint64_t full[6];
     uint64_t empty[6];
+    uint64_t pfull[6];  // a partial block's copies have landed (leader; the fixer waits)
+    uint64_t fixed[6];  // a partial block's tail rows are zeroed (leader; the MMA warp waits)
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -131,6 +134,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&m->full[s], 1);
             mbar_init(&m->empty[s], 1);
+            mbar_init(&m->pfull[s], 1);
+            mbar_init(&m->fixed[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&m->tfull[b], 1);
@@ -179,28 +184,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer (each CTA)
+        // A block whose last 16-row step is partial completes on pfull[] (the
+        // fixer zeroes its tail before the MMA warp sees it), every other block
+        // on full[]; each barrier's phases are tracked per stage.
         int stage = 0;
-        uint32_t phase = 0;
-        int last_phase[STAGES];
-        for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+        uint32_t phase = 0;                 // of empty[]: every block passes through it
+        uint32_t fullph = 0, pfullph = 0;   // per-stage parity of the next full[] / pfull[] phase
+        int last_bar[STAGES];               // per stage: -1 unused, 0 full, 1 pfull
+        uint32_t last_par[STAGES];
+        for (int s = 0; s < STAGES; ++s) last_bar[s] = -1;
         bool ok = true;
         for (int t = unit; t < total && ok; t += units) {
             int e, m0, hf, n0;
             decode(a, BM, t, e, m0, hf, n0);
             const int r0 = m->off[e], r1 = m->off[e + 1];
-            const int acol = m0 + 128 * (int)rank;                      // this CTA's A columns
+            const int acol = m0 + 128 * (int)rank;                           // this CTA's A columns
             const int bcol = hf * a.Nh + n0 + (PAIR ? 128 * (int)rank : 0);  // and B columns
             for (int k = r0; k < r1; k += BK) {
                 if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) {
                     ok = false;
                     break;
                 }
+                const int valid = r1 - k < BK ? r1 - k : BK;
+                const bool partial = (valid % UK) != 0;
+                uint64_t* bar = partial ? &m->pfull[stage] : &m->full[stage];
+                last_bar[stage] = partial ? 1 : 0;
+                last_par[stage] = ((partial ? pfullph : fullph) >> stage) & 1u;
+                if (partial) pfullph ^= 1u << stage;
+                else fullph ^= 1u << stage;
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
                 uint8_t* sB = sA + G::A_BYTES;
                 if (PAIR) {
-                    // both CTAs' bytes are counted on the leader's full barrier
-                    if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
-                    const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
+                    // both CTAs' bytes are counted on the leader's barrier
+                    if (rank == 0) mbar_arrive_expect_tx(bar, 2 * STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(smem_u32(bar), 0);
 #pragma unroll
                     for (int j = 0; j < G::A_BOXES; ++j)
                         tma_load_2d_pair(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, fb);
@@ -208,14 +225,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int j = 0; j < G::B_BOXES; ++j)
                         tma_load_2d_pair(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
                 } else {
-                    uint64_t* fb = &m->full[stage];
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    mbar_arrive_expect_tx(bar, STAGE_BYTES);
 #pragma unroll
-                    for (int j = 0; j < G::A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, fb);
+                    for (int j = 0; j < G::A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, bar);
 #pragma unroll
-                    for (int j = 0; j < G::B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
+                    for (int j = 0; j < G::B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, bar);
                 }
-                last_phase[stage] = (int)phase;
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -225,16 +240,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // never leave the CTA with a copy in flight (the leader sees every completion)
         if (!PAIR || rank == 0)
             for (int s = 0; s < STAGES; ++s)
-                if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
+                if (last_bar[s] >= 0)
+                    mbar_wait(last_bar[s] ? &m->pfull[s] : &m->full[s], last_par[s], a.status, 511, nullptr);
     } else if (warp == 1 && rank == 0) {
         // -------------------------------- MMA issuer (leader; whole warp)
         // A and B MN-major: 64-column boxes 8 KB apart (LBO), 8-row K groups
         // 1024 B apart (SBO), +2048 B per 16-row K step
         constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, 1, 1);
         int stage = 0;
-        uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
+        uint32_t fph = 0;     // per-stage parity of the next fixed[] phase
+        uint32_t fullph = 0;  // and of the next full[] phase
         bool ok = true;
         for (int t = unit; t < total && ok; t += units) {
             int e, m0, hf, n0;
@@ -246,37 +263,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * ACC_COLS);
             for (int k = r0; k < r1; k += BK) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&m->full[stage], phase, a.status, 521, abort_flag))) {
+                // rows of this block that belong to the expert; steps past the
+                // expert's last row are not issued, and a partial step's tail rows
+                // (the next expert's, or rows past the written ones) are zeroed by
+                // the fixer warp first: then this warp waits on fixed[] instead
+                const int valid = r1 - k < BK ? r1 - k : BK;
+                const int nsteps = (valid + UK - 1) / UK, rem = valid % UK;
+                bool got;
+                if (rem != 0) {
+                    got = mbar_wait(&m->fixed[stage], (fph >> stage) & 1u, a.status, 523, abort_flag);
+                    fph ^= 1u << stage;
+                } else {
+                    got = mbar_wait(&m->full[stage], (fullph >> stage) & 1u, a.status, 521, abort_flag);
+                    fullph ^= 1u << stage;
+                }
+                if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
                 }
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
-                const int valid = r1 - k;
-                if (valid < BK) {
-                    // rows valid..63 of this block belong to the next expert or lie
-                    // past the written rows: zero them in every box of the stage, in
-                    // both CTAs of a pair (the peer's through its shared::cluster
-                    // address; every copy of the stage has landed: the full barrier
-                    // counts both CTAs' bytes)
-                    const int n16 = (BK - valid) * 8;  // 16-byte words per box
-                    const uint32_t base = smem_u32(sA) + (uint32_t)(valid * 128);
-#pragma unroll 1
-                    for (uint32_t cta = 0; cta < (uint32_t)G::CTAS; ++cta) {
-                        const uint32_t cbase = PAIR ? mapa_shared(base, cta) : base;
-#pragma unroll 1
-                        for (int b = 0; b < G::A_BOXES + G::B_BOXES; ++b)
-                            for (int i = lane; i < n16; i += 32)
-                                st_cluster_zero16(cbase + (uint32_t)(b * BOX_BYTES + i * 16));
-                    }
-                    fence_proxy_async_cluster();
-                }
+                const uint32_t a32 = smem_u32(sA);
+                const uint32_t b32 = a32 + G::A_BYTES;
                 __syncwarp();
                 if (lane == 0) {
                     tc_fence_after();
-                    const uint32_t a32 = smem_u32(sA);
-                    const uint32_t b32 = a32 + G::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
+                        if (kk >= nsteps) break;
                         const uint32_t accum = (k != r0 || kk != 0) ? 1u : 0u;
                         const uint64_t adesc = umma_desc_sw128(a32 + kk * 2048, BOX_BYTES, 1024);
                         const uint64_t bdesc = umma_desc_sw128(b32 + kk * 2048, BOX_BYTES, 1024);
@@ -288,10 +301,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     else umma_commit(&m->empty[stage]);
                 }
                 __syncwarp();
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                if (++stage == STAGES) stage = 0;
             }
             if (!ok) break;
             if (lane == 0) {  // with no rows: arrives at once
@@ -310,7 +320,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_wait(&m->drain, 0, a.status, 522, nullptr);
         }
         __syncwarp();
-    } else if (warp >= 2) {
+    } else if (warp == FIX_WARP && rank == 0) {
+        // ------------------------------------ tail fixer (leader; whole warp)
+        // Walks the MMA warp's schedule; for each partial block, once every copy
+        // of the stage has landed (pfull[] counts both CTAs' bytes), it
+        // zeroes the partial step's tail rows in every box of the stage, in both
+        // CTAs of a pair (the peer's through its shared::cluster address), makes
+        // the writes visible to the tensor cores, and signals fixed[].  It runs
+        // ahead of the MMA warp, so the zeroing is off the MMA issue path.
+        int stage = 0;
+        uint32_t pfullph = 0;  // per-stage parity of the next pfull[] phase
+        bool ok = true;
+        for (int t = unit; t < total && ok; t += units) {
+            int e, m0, hf, n0;
+            decode(a, BM, t, e, m0, hf, n0);
+            const int r0 = m->off[e], r1 = m->off[e + 1];
+            for (int k = r0; k < r1; k += BK) {
+                const int valid = r1 - k < BK ? r1 - k : BK;
+                const int nsteps = (valid + UK - 1) / UK, rem = valid % UK;
+                if (rem != 0) {
+                    // only partial blocks advance pfull[stage], and the next one
+                    // cannot land before the MMA warp has used this one (which
+                    // waits for fixed[]): each wait is on the very next phase
+                    const bool got = mbar_wait(&m->pfull[stage], (pfullph >> stage) & 1u, a.status, 540,
+                                               abort_flag);
+                    pfullph ^= 1u << stage;
+                    if (!__all_sync(0xffffffffu, got)) {
+                        ok = false;
+                        break;
+                    }
+                    const int n16 = (UK - rem) * 8;  // 16-byte words per box
+                    const uint32_t base = smem_u32(stages + (size_t)stage * STAGE_BYTES) +
+                                          (uint32_t)(((nsteps - 1) * UK + rem) * 128);
+#pragma unroll 1
+                    for (uint32_t cta = 0; cta < (uint32_t)G::CTAS; ++cta) {
+                        const uint32_t cbase = PAIR ? mapa_shared(base, cta) : base;
+#pragma unroll 1
+                        for (int bx = 0; bx < G::A_BOXES + G::B_BOXES; ++bx)
+                            for (int i = lane; i < n16; i += 32)
+                                st_cluster_zero16(cbase + (uint32_t)(bx * BOX_BYTES + i * 16));
+                    }
+                    fence_proxy_async_cluster();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&m->fixed[stage]);
+                }
+                if (++stage == STAGES) stage = 0;
+            }
+        }
+    } else if (warp >= 2 && warp < 2 + EPI_WARPS) {
         // -------------------------------------------------------- epilogue
         // warp w: tensor-memory lanes 32*(w%4) .. +31 (this CTA's output rows),
         // half of the 256 columns (warps 2..5 the first, 6..9 the second)
@@ -340,8 +397,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tmem_ld_32x32b_x32(taddr + c * 32, v);
                 tmem_ld_wait();
                 uint8_t* buf = bufs + nb * OUT_BYTES;
-                nb ^= 1;
-                if (lane == 0) bulk_wait_read<1>();  // the store before last has read this buffer
+                nb = (nb + 1) % OUT_BUFS;
+                if (lane == 0) bulk_wait_read<OUT_BUFS - 1>();  // this buffer's last store has read it
                 __syncwarp();
                 uint4* row = reinterpret_cast<uint4*>(buf + lane * 128);
 #pragma unroll
