@@ -194,7 +194,11 @@ def kernel_source_hash(files=GEMM_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, kernel: str):
+# and those of the backward's weight-gradient GEMM (the training step's roofline kernel)
+WGRAD_SOURCES = ("wgrad_tc.cu", "common.cuh")
+
+
+def recorded_traffic(workload: str, kernel: str, files=GEMM_SOURCES):
     """DRAM bytes per launch from a committed ncu summary, if the kernels have
     not changed since it was taken (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -203,7 +207,7 @@ def recorded_traffic(workload: str, kernel: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(files):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -510,7 +514,8 @@ def run_gpu_train(args):
                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                     "peak_source": f"hbm_gbs of {peak_src}"}
     roofline.update(intensity_flop_per_byte=round(intensity, 1), ridge=round(ridge, 1),
-                    traffic=None)
+                    traffic=recorded_traffic(wl.name, top, WGRAD_SOURCES)
+                    if top.startswith("bwd.wgrad") else None)
     stages = {}
     for name, ms in stage_ms.items():
         ent = {"ms": round(ms, 4)}
