@@ -555,6 +555,103 @@ def run_gpu_train(args):
     _finish(world)
 
 
+def run_gpu_ep(args):
+    """Expert parallelism: rank r of N holds experts r*E/N .. (r+1)*E/N - 1 and
+    its own T tokens; a step is one ExpertParallelMoE forward on every rank
+    (route, owner-sorted dispatch, NCCL all-to-all, grouped local experts,
+    reverse all-to-all, weighted combine)."""
+    import mixture_experts_layer_55_b200 as M
+    from mixture_experts_layer_55_b200.ep import ExpertParallelMoE
+
+    rank, world, local_rank = rank_info()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29531")
+        os.environ.setdefault("RANK", str(rank))
+        os.environ.setdefault("WORLD_SIZE", str(world))
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    wl = workload_of(args)
+    if wl.E % world:
+        raise SystemExit(f"E = {wl.E} experts do not divide among {world} ranks")
+    EL = wl.E // world
+    inp = make_inputs(wl, device=dev)
+    sl = slice(rank * EL, (rank + 1) * EL)
+    layer = ExpertParallelMoE(wl.T, inp["w_router"], inp["w_gate"][sl].contiguous(),
+                              inp["w_up"][sl].contiguous(), inp["w_down"][sl].contiguous(), wl.E,
+                              wl.K, wl.capacity_factor, router_bias=inp["bias"])
+    del inp["w_gate"], inp["w_up"], inp["w_down"]
+    nbuf = 3
+    xs = [make_tokens(wl, device=dev, seed=rank_token_seed(rank) * 16 + i) for i in range(nbuf)]
+    stream = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        layer.forward(xs[i % nbuf], logit_noise=inp["noise"])
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        y = layer.forward(xs[i % nbuf], logit_noise=inp["noise"])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    ms_total, ms_step, value = aggregate(start.elapsed_time(stop), world, wl.T, args.steps, dev)
+    # end to end: x in from pinned memory, y out, every step
+    x_h = [t.cpu().pin_memory() for t in xs]
+    y_h = torch.empty_like(x_h[0]).pin_memory()
+    xd = torch.empty_like(xs[0])
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        xd.copy_(x_h[i % nbuf], non_blocking=True)
+        y = layer.forward(xd, logit_noise=inp["noise"])
+        y_h.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    flags = layer.ops.status()
+    if flags:
+        raise RuntimeError(f"device status flags {flags:#x} after the benchmark")
+    if rank == 0:
+        io = wl.T * wl.D * wl.elem_bytes
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(wl, args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) random-init weights)",
+            "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
+                       "capacity_factor": wl.capacity_factor,
+                       "parallelism": f"expert parallel x{world} ({EL} experts per rank, "
+                                      "NCCL all-to-all)",
+                       "l2": "inputs larger than L2"},
+            "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
+                    "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io, "d2h_bytes_per_step": io,
+                    "how": "per step: x in from pinned host memory, ExpertParallelMoE.forward, y out"},
+            "gpu_launches": None,
+            "roofline": None,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        if args.warmup < 3:
+            line["note"] = "fewer than 3 warm-up steps: not a valid measurement"
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+
+
 def _finish(world):
     if world > 1:
         import torch.distributed as dist
@@ -742,9 +839,13 @@ def main(argv=None):
                     help="KEY=VALUE change of the workload shape (profiling cases only)")
     ap.add_argument("--pass", dest="pass_", choices=["forward", "train"], default="forward",
                     help="forward (default) or a training step (forward + backward)")
+    ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
+                    help="replicas (default): every GPU holds all experts; ep: experts sharded")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.parallel == "ep":
+        run_gpu_ep(args)
     elif args.pass_ == "train":
         run_gpu_train(args)
     else:

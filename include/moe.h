@@ -353,6 +353,52 @@ MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const floa
  */
 MOE_API int32_t moe_backward_kernel_count(const moe_config *cfg);
 
+/* ------------------------------------------------------- expert parallelism
+ *
+ * "Lab: build a tiny MoE in PyTorch", "From local loop to expert
+ * parallelism": sort by owner -> exchange counts -> all-to-all dispatch ->
+ * grouped local experts -> reverse all-to-all -> scatter-add, with the same
+ * mathematical output as the local layer.  Rank r of W owns the contiguous
+ * experts r*EL .. r*EL + EL - 1 (EL = E / W).  moe_dispatch's expert-major rows
+ * are already sorted by owner; the exchanges themselves are collectives of the
+ * caller's communication library.  These entry points are the layer's own
+ * steps around them.
+ */
+
+/* Bytes of device scratch moe_ep_layout needs (status word first). */
+MOE_API moe_status moe_ep_workspace_size(int32_t world, int32_t experts_per_rank, size_t *bytes);
+
+/*
+ * Receive layout of one rank's experts.  recv_counts (world, EL) int32: rows
+ * that arrive from source rank s for local expert e, in the order they arrive
+ * (source-major: all of source 0's rows, its expert 0 first, then source 1's).
+ * Writes offsets (EL + 1) int32, the expert-major row offsets of the local
+ * experts (expert e's rows are its segments from sources 0..W-1 in order);
+ * dst_of (rows) int32, the expert-major row of each arrived row; src_of
+ * (rows) int32, the inverse.  rows = sum of recv_counts <= max_rows; world *
+ * EL <= 256.  All device pointers; workspace = moe_ep_workspace_size bytes.
+ */
+MOE_API moe_status moe_ep_layout(int32_t world, int32_t experts_per_rank, const int32_t *recv_counts,
+                                 int64_t max_rows, int32_t *offsets, int32_t *dst_of, int32_t *src_of,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * out[i, :] = in[idx[i], :] for i < n: rows of row_bytes (a multiple of 16)
+ * bytes; in has in_rows rows; an idx outside [0, in_rows) sets the bounds flag
+ * of `workspace`'s status word and leaves that row unwritten.  Device pointers.
+ */
+MOE_API moe_status moe_permute_rows(const void *in, int64_t in_rows, const int32_t *idx, int64_t n,
+                                    int64_t row_bytes, void *out, void *workspace, void *stream);
+
+/*
+ * moe_combine with the routing weight applied here: y[t] = y_add[t] + sum over
+ * kept slots of topk_w[t, k] * y_perm[row_of[t, k]], fp32, rounded once.  For
+ * unweighted expert outputs (the rows that come back from the experts' owners).
+ */
+MOE_API moe_status moe_combine_weighted(const moe_config *cfg, const void *y_perm,
+                                        const int32_t *row_of, const float *topk_w,
+                                        const void *y_add, void *y, void *stream);
+
 /*
  * moe_dispatch without a workspace, for callers that cannot allocate device
  * memory: code handed only its input and output buffers by a host framework

@@ -98,6 +98,12 @@ _SIG = {
     "moe_trace_attach_backward": ([_P, ctypes.c_int32], ctypes.c_int32),
     "moe_trace_backward_boundary_count": ([], ctypes.c_int32),
     "moe_trace_backward_stage_name": ([ctypes.c_int32], ctypes.c_char_p),
+    "moe_ep_workspace_size": ([ctypes.c_int32, ctypes.c_int32, _P], ctypes.c_int32),
+    "moe_ep_layout": ([ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int64, _P, _P, _P, _P,
+                       ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_permute_rows": ([_P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P],
+                         ctypes.c_int32),
+    "moe_combine_weighted": ([_P] * 7, ctypes.c_int32),
 }
 
 
@@ -373,3 +379,31 @@ def _nbytes(t) -> int:
     if isinstance(t, int):
         raise ValueError("pass the workspace as a tensor so its size is known")
     return t.numel() * t.element_size()
+
+
+# ------------------------------------------------------- expert parallelism
+
+def ep_workspace_size(world: int, experts_per_rank: int) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().moe_ep_workspace_size(int(world), int(experts_per_rank), ctypes.byref(v)),
+           "moe_ep_workspace_size")
+    return v.value
+
+
+def moe_ep_layout(world: int, experts_per_rank: int, recv_counts, max_rows: int, offsets, dst_of,
+                  src_of, workspace, stream=None):
+    _check(lib().moe_ep_layout(int(world), int(experts_per_rank), _ptr(recv_counts), int(max_rows),
+                               _ptr(offsets), _ptr(dst_of), _ptr(src_of), _ptr(workspace),
+                               _nbytes(workspace), _stream(stream)), "moe_ep_layout")
+
+
+def moe_permute_rows(inp, idx, n: int, out, workspace, stream=None):
+    """out[:n] = inp[idx[:n]] (rows), on the device."""
+    row_bytes = inp.stride(0) * inp.element_size()
+    _check(lib().moe_permute_rows(_ptr(inp), int(inp.shape[0]), _ptr(idx), int(n), int(row_bytes),
+                                  _ptr(out), _ptr(workspace), _stream(stream)), "moe_permute_rows")
+
+
+def moe_combine_weighted(cfg, y_perm, row_of, topk_w, y, y_add=None, stream=None):
+    _check(lib().moe_combine_weighted(_cfg(cfg), _ptr(y_perm), _ptr(row_of), _ptr(topk_w),
+                                      _ptr(y_add), _ptr(y), _stream(stream)), "moe_combine_weighted")

@@ -663,6 +663,56 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
     return 11 + shared + (router_plan(*cfg).splits > 1 ? 1 : 0);
 }
 
+moe_status moe_ep_workspace_size(int32_t world, int32_t experts_per_rank, size_t* bytes)
+{
+    if (bytes == nullptr || world < 1 || experts_per_rank < 1 || world * experts_per_rank > 256)
+        return MOE_ERR_ARG;
+    *bytes = align_up(64 * sizeof(int)) + align_up((size_t)(2 * world * experts_per_rank + 1) * sizeof(int32_t));
+    return MOE_OK;
+}
+
+moe_status moe_ep_layout(int32_t world, int32_t experts_per_rank, const int32_t* recv_counts,
+                         int64_t max_rows, int32_t* offsets, int32_t* dst_of, int32_t* src_of,
+                         void* workspace, size_t workspace_bytes, void* stream)
+{
+    size_t need = 0;
+    moe_status st = moe_ep_workspace_size(world, experts_per_rank, &need);
+    if (st != MOE_OK) return st;
+    if (!recv_counts || !offsets || !dst_of || !src_of) return MOE_ERR_ARG;
+    if (max_rows < 1 || max_rows > (int64_t)INT32_MAX) return MOE_ERR_SHAPE;
+    st = check_ws(nullptr, workspace, workspace_bytes, need);
+    if (st != MOE_OK) return st;
+    char* ws = static_cast<char*>(workspace);
+    int32_t* seg = reinterpret_cast<int32_t*>(ws + align_up(64 * sizeof(int)));
+    const int n = world * experts_per_rank;
+    return cuda_status(launch_ep_layout(recv_counts, world, experts_per_rank, max_rows, offsets, seg + n,
+                                        seg, dst_of, src_of, reinterpret_cast<int*>(ws),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute_rows(const void* in, int64_t in_rows, const int32_t* idx, int64_t n,
+                            int64_t row_bytes, void* out, void* workspace, void* stream)
+{
+    if (n < 0 || in_rows < 0 || row_bytes < 16) return MOE_ERR_SHAPE;
+    if (row_bytes % 16 != 0) return MOE_ERR_ALIGN;
+    if (n > 0 && (!in || !idx || !out)) return MOE_ERR_ARG;
+    if (n > 0 && (!aligned16(in) || !aligned16(out))) return MOE_ERR_ALIGN;
+    if (workspace == nullptr) return MOE_ERR_WORKSPACE;
+    return cuda_status(launch_permute_rows(in, idx, out, n, row_bytes, in_rows,
+                                           static_cast<int*>(workspace), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_combine_weighted(const moe_config* cfg, const void* y_perm, const int32_t* row_of,
+                                const float* topk_w, const void* y_add, void* y, void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!y_perm || !row_of || !topk_w || !y) return MOE_ERR_ARG;
+    if (!aligned16(y_perm) || !aligned16(y) || (y_add && !aligned16(y_add))) return MOE_ERR_ALIGN;
+    return cuda_status(launch_combine(*cfg, y_perm, row_of, topk_w, y_add, y, max_rows_of(*cfg),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 int32_t moe_backward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;

@@ -175,6 +175,11 @@ int router_wgrad_splits(const moe_config& c);
 size_t router_wgrad_part_bytes(const moe_config& c, int splits);
 cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float* dL, float* part,
                                 int splits, float* dw, float* db, cudaStream_t s);
+cudaError_t launch_ep_layout(const int32_t* recv, int W, int EL, int64_t max_rows, int32_t* offsets,
+                             int32_t* seg_src, int32_t* seg_dst, int32_t* dst_of, int32_t* src_of,
+                             int* status, cudaStream_t s);
+cudaError_t launch_permute_rows(const void* in, const int32_t* idx, void* out, int64_t n, int64_t row_bytes,
+                                int64_t in_rows, int* status, cudaStream_t s);
 cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float* w_r, const void* dxp,
                                const int32_t* row_of, const void* dx_shared, void* dx,
                                int64_t max_rows, cudaStream_t s);
