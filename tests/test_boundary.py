@@ -218,3 +218,26 @@ def test_training_argument_errors(lib):
     cs = _cfg(F_shared=64)
     assert bwd(cfg=cs, state_bytes=B.train_state_size(cs),
                ws_bytes=B.backward_workspace_size(cs)) == B.MOE_ERR_ARG  # shared grads missing
+
+
+def test_expert_parallel_argument_errors(lib):
+    v = ctypes.c_size_t()
+    assert lib.moe_ep_workspace_size(2, 4, ctypes.byref(v)) == B.MOE_OK and v.value > 0
+    assert lib.moe_ep_workspace_size(0, 4, ctypes.byref(v)) == B.MOE_ERR_ARG
+    assert lib.moe_ep_workspace_size(16, 32, ctypes.byref(v)) == B.MOE_ERR_ARG  # 512 segments > 256
+    need = B.ep_workspace_size(2, 4)
+    ok = lambda **kw: lib.moe_ep_layout(  # noqa: E731
+        kw.get("W", 2), kw.get("EL", 4), kw.get("recv", FAKE), kw.get("max_rows", 100), FAKE, FAKE,
+        kw.get("src_of", FAKE), kw.get("ws", FAKE), kw.get("nb", need), None)
+    assert ok(recv=None) == B.MOE_ERR_ARG
+    assert ok(src_of=None) == B.MOE_ERR_ARG
+    assert ok(max_rows=0) == B.MOE_ERR_SHAPE
+    assert ok(nb=need - 1) == B.MOE_ERR_WORKSPACE
+    assert ok(ws=FAKE + 16) == B.MOE_ERR_ALIGN
+    assert lib.moe_permute_rows(FAKE, 10, FAKE, 5, 24, FAKE, FAKE, None) == B.MOE_ERR_ALIGN
+    assert lib.moe_permute_rows(FAKE, 10, FAKE, -1, 32, FAKE, FAKE, None) == B.MOE_ERR_SHAPE
+    assert lib.moe_permute_rows(FAKE, 10, None, 5, 32, FAKE, FAKE, None) == B.MOE_ERR_ARG
+    assert lib.moe_permute_rows(FAKE, 10, FAKE, 5, 32, FAKE, None, None) == B.MOE_ERR_WORKSPACE
+    c = _cfg()
+    assert lib.moe_combine_weighted(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, None) == B.MOE_ERR_ARG
+    assert lib.moe_combine_weighted(ctypes.byref(c), FAKE, FAKE, FAKE, None, FAKE + 8, None) == B.MOE_ERR_ALIGN
