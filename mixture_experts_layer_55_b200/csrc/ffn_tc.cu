@@ -73,7 +73,10 @@ template <int MODE, bool PAIR> struct Geo {
     static constexpr int B_BOXES = 256 / 64 / CTAS;        // 64-wide B boxes per CTA per stage
     static constexpr int B_BYTES = B_BOXES * BOX_BYTES;    // (K-major B: one box of 256/CTAS rows)
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB single, 32 KB pair
-    static constexpr int STAGES = PAIR ? 6 : 4;
+    // dgrad-h stages its [dg | du] pieces for TMA stores (4 KB per epilogue
+    // warp), which costs it one operand stage
+    static constexpr int OUT_BYTES = MODE == kDgradH ? 4096 : 0;
+    static constexpr int STAGES = MODE == kDgradH ? (PAIR ? 5 : 3) : (PAIR ? 6 : 4);
     static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;  // one per epilogue warp
 };
 
@@ -94,7 +97,7 @@ template <int MODE, bool PAIR>
 constexpr size_t smem_bytes()
 {
     return 1024 /*alignment slack*/ + (size_t)Geo<MODE, PAIR>::STAGES * Geo<MODE, PAIR>::STAGE_BYTES +
-           sizeof(Misc);
+           (size_t)EPI_WARPS * Geo<MODE, PAIR>::OUT_BYTES + sizeof(Misc);
 }
 
 struct Args {
@@ -153,7 +156,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* stages = smem;
-    Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint8_t* outbuf = smem + (size_t)STAGES * STAGE_BYTES;  // dgrad-h: EPI_WARPS x 4 KB, 1 KB aligned
+    Misc* m = reinterpret_cast<Misc*>(outbuf + (size_t)EPI_WARPS * G::OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = a.E;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader (issues the MMAs)
@@ -174,7 +178,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB0);
-        if (GATEUP || MODE == kDgradX) prefetch_tmap(&tmB1);
+        if (GATEUP || MODE == kDgradX || MODE == kDgradH) prefetch_tmap(&tmB1);
     }
     if (warp == 1) {
         if (PAIR) {
@@ -367,6 +371,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r_in_tile = (int)rank * 128 + quad * 32 + lane;
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m->tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m->tempty[1]), 0);
+        uint8_t* obuf = outbuf + (size_t)(warp - 2) * G::OUT_BYTES;  // dgrad-h: [dg 2 KB | du 2 KB]
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = unit; t < total; t += units) {
@@ -423,12 +428,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             } else if (MODE == kDgradH) {
+                // the warp's 32 rows all belong to the expert: stage and TMA-store them
+                const int64_t warp_row0 = (int64_t)m_row0 + (int)rank * 128 + quad * 32;
+                const bool warp_full = warp_row0 + 32 <= row_end;
 #pragma unroll 1
                 for (int c = 4 * half; c < 4 * half + 4; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
                     tmem_ld_wait();
                     const int col = n0 + c * 32;
+                    if (warp_full && col < a.N) {
+                        if (lane == 0) bulk_wait_read<0>();  // the last stores have read the buffer
+                        __syncwarp();
+                    }
                     if (valid && col < a.N) {
                         const __nv_bfloat16* grow = a.gu_in + row * 2 * (int64_t)a.N + col;
                         uint32_t dg[16], du[16];
@@ -458,14 +470,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                 du[4 * q + i] = pack_bf16x2(o[1][0], o[1][1]);
                             }
                         }
+                        if (!warp_full) {  // rows past the expert's end: per-lane stores of the valid rows
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (col + 8 * q < a.N) {
-                                *reinterpret_cast<uint4*>(orow + col + 8 * q) =
-                                    make_uint4(dg[4 * q], dg[4 * q + 1], dg[4 * q + 2], dg[4 * q + 3]);
-                                *reinterpret_cast<uint4*>(orow + a.N + col + 8 * q) =
-                                    make_uint4(du[4 * q], du[4 * q + 1], du[4 * q + 2], du[4 * q + 3]);
+                            for (int q = 0; q < 4; ++q)
+                                if (col + 8 * q < a.N) {
+                                    *reinterpret_cast<uint4*>(orow + col + 8 * q) =
+                                        make_uint4(dg[4 * q], dg[4 * q + 1], dg[4 * q + 2], dg[4 * q + 3]);
+                                    *reinterpret_cast<uint4*>(orow + a.N + col + 8 * q) =
+                                        make_uint4(du[4 * q], du[4 * q + 1], du[4 * q + 2], du[4 * q + 3]);
+                                }
+                        } else {
+                            // the piece through shared memory (64-byte swizzle: 16-byte chunk q of
+                            // row r at chunk q ^ ((r >> 1) & 3)) and two TMA stores
+                            uint4* gdst = reinterpret_cast<uint4*>(obuf + lane * 64);
+                            uint4* udst = reinterpret_cast<uint4*>(obuf + 2048 + lane * 64);
+                            const int sw = (lane >> 1) & 3;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                gdst[q ^ sw] = make_uint4(dg[4 * q], dg[4 * q + 1], dg[4 * q + 2], dg[4 * q + 3]);
+                                udst[q ^ sw] = make_uint4(du[4 * q], du[4 * q + 1], du[4 * q + 2], du[4 * q + 3]);
                             }
+                        }
+                    }
+                    if (warp_full && col < a.N) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {  // columns >= F fall outside the map: not written
+                            tma_store_3d(&tmB1, obuf, col, 0, warp_row0);
+                            tma_store_3d(&tmB1, obuf + 2048, col, 1, warp_row0);
+                            bulk_commit();
+                        }
                     }
                 }
             } else {
@@ -510,6 +544,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc = 0;
                 acc_phase ^= 1u;
             }
+        }
+        if (MODE == kDgradH) {
+            if (lane == 0) bulk_wait_all<0>();  // every store of this warp has completed
+            __syncwarp();
         }
     }
     tc_fence_before();
@@ -599,6 +637,21 @@ static bool map_halves(CUtensorMap* m, const void* base, uint64_t half, uint64_t
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over (rows, 2 * half) viewed as (rows, 2, half) for 32 x 32
+// stores from shared memory laid out with the 64-byte swizzle.
+static bool map_halves_store(CUtensorMap* m, const void* base, uint64_t half, uint64_t rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {half, 2, rows};
+    cuuint64_t strides[2] = {half * 2, half * 4};
+    cuuint32_t box[3] = {32, 1, 32};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Per device: dynamic shared memory opted in, and the number of CTAs (or CTA
@@ -728,14 +781,16 @@ cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const vo
         !map_3d_kmajor(&mG, w_gate, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows) ||
         !map_3d_kmajor(&mU, w_up, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows))
         return cudaErrorInvalidValue;
+    CUtensorMap mOut;  // [dg | du] viewed as (rows, 2, F): 32 x 32 pieces for the epilogue's stores
+    if (!map_halves_store(&mOut, dgu, (uint64_t)c.F, (uint64_t)max_rows)) return cudaErrorInvalidValue;
     const int64_t bm = pair ? 256 : 128;
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
     // dH = dYp . Wd^T (K = D), epilogue through SwiGLU into [dg | du]
     Args a1{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dgu), c.E, c.D, c.F,
             (c.F + 255) / 256, 2 * (int64_t)c.F, max_rows, c.T * c.K, nullptr,
             static_cast<const __nv_bfloat16*>(gu), status};
-    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mWd, a1, mtiles_bound * a1.n_tiles, s)
-                           : launch_one<kDgradH, false>(mA, mWd, mWd, a1, mtiles_bound * a1.n_tiles, s);
+    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mOut, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<kDgradH, false>(mA, mWd, mOut, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     // dXp = [dg | du] . [Wg | Wu]^T (K = 2F), unit weights
