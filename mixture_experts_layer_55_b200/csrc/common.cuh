@@ -203,6 +203,13 @@ MOE_DEVICE void tma_store_3d(const void* tmap, const void* smem_src, int32_t c0,
                  : "memory");
 }
 
+MOE_DEVICE void tma_store_2d(const void* tmap, const void* smem_src, int32_t c0, int32_t c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tmap),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy accesses (TMA stores, tcgen05.mma operand reads).
 MOE_DEVICE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

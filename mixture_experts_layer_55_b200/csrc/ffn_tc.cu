@@ -73,9 +73,10 @@ template <int MODE, bool PAIR> struct Geo {
     static constexpr int B_BOXES = 256 / 64 / CTAS;        // 64-wide B boxes per CTA per stage
     static constexpr int B_BYTES = B_BOXES * BOX_BYTES;    // (K-major B: one box of 256/CTAS rows)
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB single, 32 KB pair
-    // dgrad-h stages its [dg | du] pieces for TMA stores (4 KB per epilogue
-    // warp), which costs it one operand stage
-    static constexpr int OUT_BYTES = MODE == kDgradH ? 4096 : 0;
+    // the epilogue stages its 32 x 32 bf16 pieces for TMA stores: 2 KB per
+    // epilogue warp; dgrad-h writes two at a time (4 KB), which costs it one
+    // operand stage
+    static constexpr int OUT_BYTES = MODE == kDgradH ? 4096 : 2048;
     static constexpr int STAGES = MODE == kDgradH ? (PAIR ? 5 : 3) : (PAIR ? 6 : 4);
     static constexpr int EPI_ARRIVALS = EPI_WARPS * CTAS;  // one per epilogue warp
 };
@@ -144,10 +145,35 @@ MOE_DEVICE void silu_and_grad(float g, float& silu, float& dsilu)
     dsilu = fmaf(g * s, 1.0f - s, s);
 }
 
+// One 32 x 32 bf16 piece of the output, held one row per lane (16 packed
+// words), written through the warp's staging buffer (64-byte swizzle: the
+// 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3), conflict-free) by a
+// TMA tensor store.  The map clips columns past its extent; the caller only
+// takes this path when all 32 rows are the expert's.
+template <int DIMS>
+MOE_DEVICE void store_piece(uint8_t* buf, int lane, const uint32_t (&p)[16], const CUtensorMap* map, int c0,
+                            int c1, int c2)
+{
+    if (lane == 0) bulk_wait_read<0>();  // the buffer's last store has read it
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64);
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q ^ sw] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        if (DIMS == 2) tma_store_2d(map, buf, c0, c1);
+        else tma_store_3d(map, buf, c0, c1, c2);
+        bulk_commit();
+    }
+}
+
 template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                  const __grid_constant__ CUtensorMap tmB1, const Args a)
+                  const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmO0,
+                  const __grid_constant__ CUtensorMap tmO1, const Args a)
 {
     using G = Geo<MODE, PAIR>;
     constexpr bool GATEUP = G::GATEUP;
@@ -156,7 +182,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* stages = smem;
-    uint8_t* outbuf = smem + (size_t)STAGES * STAGE_BYTES;  // dgrad-h: EPI_WARPS x 4 KB, 1 KB aligned
+    uint8_t* outbuf = smem + (size_t)STAGES * STAGE_BYTES;  // EPI_WARPS x OUT_BYTES, 1 KB aligned
     Misc* m = reinterpret_cast<Misc*>(outbuf + (size_t)EPI_WARPS * G::OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = a.E;
@@ -178,7 +204,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB0);
-        if (GATEUP || MODE == kDgradX || MODE == kDgradH) prefetch_tmap(&tmB1);
+        if (GATEUP || MODE == kDgradX) prefetch_tmap(&tmB1);
+        prefetch_tmap(&tmO0);
+        if ((GATEUP && a.gu_out != nullptr) || MODE == kDgradH) prefetch_tmap(&tmO1);
     }
     if (warp == 1) {
         if (PAIR) {
@@ -371,7 +399,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r_in_tile = (int)rank * 128 + quad * 32 + lane;
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m->tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m->tempty[1]), 0);
-        uint8_t* obuf = outbuf + (size_t)(warp - 2) * G::OUT_BYTES;  // dgrad-h: [dg 2 KB | du 2 KB]
+        uint8_t* obuf = outbuf + (size_t)(warp - 2) * G::OUT_BYTES;  // staging (dgrad-h: [dg | du])
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = unit; t < total; t += units) {
@@ -385,6 +413,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const bool valid = row < row_end;
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
             __nv_bfloat16* orow = a.out + row * a.ldo;
+            // the warp's 32 rows all belong to the expert: its pieces go through
+            // shared memory and TMA stores; otherwise each lane stores its valid row
+            const int64_t warp_row0 = (int64_t)m_row0 + (int)rank * 128 + quad * 32;
+            const bool warp_full = warp_row0 + 32 <= row_end;
             if (GATEUP) {
 #pragma unroll 1
                 for (int c = 2 * half; c < 2 * half + 2; ++c) {
@@ -404,33 +436,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             p[j] = pack_bf16x2(h0, h1);
                         }
                         const int col = n0 + c * 32;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (col + 8 * q < a.N)
-                                *reinterpret_cast<uint4*>(orow + col + 8 * q) =
-                                    make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
-                        if (a.gu_out != nullptr) {  // keep the pre-activations for the backward
-                            __nv_bfloat16* grow = a.gu_out + row * 2 * (int64_t)a.N + col;
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                p[j] = pack_bf16x2(__uint_as_float(g[2 * j]), __uint_as_float(g[2 * j + 1]));
-                                g[j] = pack_bf16x2(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
-                            }
+                        if (warp_full) {
+                            if (col < a.N) store_piece<2>(obuf, lane, p, &tmO0, col, (int)warp_row0, 0);
+                        } else {
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
-                                if (col + 8 * q < a.N) {
-                                    *reinterpret_cast<uint4*>(grow + 8 * q) =
+                                if (col + 8 * q < a.N)
+                                    *reinterpret_cast<uint4*>(orow + col + 8 * q) =
                                         make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
-                                    *reinterpret_cast<uint4*>(grow + a.N + 8 * q) =
-                                        make_uint4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                        }
+                        if (a.gu_out != nullptr) {  // keep the pre-activations for the backward
+                            __nv_bfloat16* grow = a.gu_out + row * 2 * (int64_t)a.N + col;
+#pragma unroll 1
+                            for (int which = 0; which < 2; ++which) {  // g, then u
+                                const uint32_t* src = which ? u : g;
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    p[j] = pack_bf16x2(__uint_as_float(src[2 * j]), __uint_as_float(src[2 * j + 1]));
+                                if (warp_full) {
+                                    if (col < a.N) store_piece<3>(obuf, lane, p, &tmO1, col, which, (int)warp_row0);
+                                } else {
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q)
+                                        if (col + 8 * q < a.N)
+                                            *reinterpret_cast<uint4*>(grow + which * a.N + 8 * q) =
+                                                make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
                                 }
+                            }
                         }
                     }
                 }
             } else if (MODE == kDgradH) {
-                // the warp's 32 rows all belong to the expert: stage and TMA-store them
-                const int64_t warp_row0 = (int64_t)m_row0 + (int)rank * 128 + quad * 32;
-                const bool warp_full = warp_row0 + 32 <= row_end;
 #pragma unroll 1
                 for (int c = 4 * half; c < 4 * half + 4; ++c) {
                     uint32_t v[32];
@@ -496,8 +532,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {  // columns >= F fall outside the map: not written
-                            tma_store_3d(&tmB1, obuf, col, 0, warp_row0);
-                            tma_store_3d(&tmB1, obuf + 2048, col, 1, warp_row0);
+                            tma_store_3d(&tmO0, obuf, col, 0, warp_row0);
+                            tma_store_3d(&tmO0, obuf + 2048, col, 1, warp_row0);
                             bulk_commit();
                         }
                     }
@@ -524,11 +560,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int j = 0; j < 16; ++j)
                             p[j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
                         const int col = n0 + c * 32;
+                        if (warp_full) {
+                            if (col < a.N) store_piece<2>(obuf, lane, p, &tmO0, col, (int)warp_row0, 0);
+                        } else {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (col + 8 * q < a.N)
-                                *reinterpret_cast<uint4*>(orow + col + 8 * q) =
-                                    make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                            for (int q = 0; q < 4; ++q)
+                                if (col + 8 * q < a.N)
+                                    *reinterpret_cast<uint4*>(orow + col + 8 * q) =
+                                        make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                        }
                     }
                 }
             }
@@ -545,10 +585,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc_phase ^= 1u;
             }
         }
-        if (MODE == kDgradH) {
-            if (lane == 0) bulk_wait_all<0>();  // every store of this warp has completed
-            __syncwarp();
-        }
+        if (lane == 0) bulk_wait_all<0>();  // every store of this warp has completed
+        __syncwarp();
     }
     tc_fence_before();
     if (PAIR) cluster_sync();  // no CTA leaves while its peer may still signal it
@@ -639,6 +677,21 @@ static bool map_halves(CUtensorMap* m, const void* base, uint64_t half, uint64_t
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over a row-major (rows, cols) output for 32 x 32 stores from
+// shared memory laid out with the 64-byte swizzle.
+static bool map_store_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D bf16 map over (rows, 2 * half) viewed as (rows, 2, half) for 32 x 32
 // stores from shared memory laid out with the 64-byte swizzle.
 static bool map_halves_store(CUtensorMap* m, const void* base, uint64_t half, uint64_t rows)
@@ -701,6 +754,7 @@ static cudaError_t prepare(int* resident_units)
 
 template <int MODE, bool PAIR>
 static cudaError_t launch_one(const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
+                              const CUtensorMap& mO0, const CUtensorMap& mO1,
                               const Args& a, int64_t tiles_bound, cudaStream_t s)
 {
     int units = 0;
@@ -710,7 +764,7 @@ static cudaError_t launch_one(const CUtensorMap& mA, const CUtensorMap& mB0, con
     if (n < 1) n = 1;
     constexpr size_t smem = smem_bytes<MODE, PAIR>();
     if (!PAIR) {
-        ffn_tc_kernel<MODE, false><<<(unsigned)n, NUM_THREADS, smem, s>>>(mA, mB0, mB1, a);
+        ffn_tc_kernel<MODE, false><<<(unsigned)n, NUM_THREADS, smem, s>>>(mA, mB0, mB1, mO0, mO1, a);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
@@ -725,7 +779,7 @@ static cudaError_t launch_one(const CUtensorMap& mA, const CUtensorMap& mB0, con
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<MODE, true>, mA, mB0, mB1, a);
+    return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<MODE, true>, mA, mB0, mB1, mO0, mO1, a);
 }
 
 }  // namespace tc
@@ -749,6 +803,12 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
         !map_2d(&mH, h, (uint64_t)c.F, (uint64_t)max_rows, 128) ||
         !map_3d(&mD, w_down, (uint64_t)c.D, (uint64_t)c.F, (uint64_t)c.E))
         return cudaErrorInvalidValue;
+    // the epilogues' stores: h (rows, F), [g | u] (rows, 2, F), y_perm (rows, D)
+    CUtensorMap mHo, mGUo, mYo;
+    if (!map_store_2d(&mHo, h, (uint64_t)c.F, (uint64_t)max_rows) ||
+        !map_halves_store(&mGUo, gu_keep ? gu_keep : h, (uint64_t)c.F, (uint64_t)max_rows) ||
+        !map_store_2d(&mYo, y_perm, (uint64_t)c.D, (uint64_t)max_rows))
+        return cudaErrorInvalidValue;
     const bool pair = use_pairs(c, max_rows);
     const int64_t bm = pair ? 256 : 128;
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
@@ -756,14 +816,14 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
     Args a1{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(h), c.E, c.D, c.F,
             (c.F + 127) / 128, c.F, max_rows, c.T * c.K,
             static_cast<__nv_bfloat16*>(gu_keep), nullptr, status};
-    cudaError_t err = pair ? launch_one<kGateUp, true>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s)
-                           : launch_one<kGateUp, false>(mA, mG, mU, a1, mtiles_bound * a1.n_tiles, s);
+    cudaError_t err = pair ? launch_one<kGateUp, true>(mA, mG, mU, mHo, mGUo, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<kGateUp, false>(mA, mG, mU, mHo, mGUo, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     Args a2{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(y_perm), c.E, c.F, c.D,
             (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status};
-    return pair ? launch_one<kDown, true>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s)
-                : launch_one<kDown, false>(mH, mD, mD, a2, mtiles_bound * a2.n_tiles, s);
+    return pair ? launch_one<kDown, true>(mH, mD, mD, mYo, mYo, a2, mtiles_bound * a2.n_tiles, s)
+                : launch_one<kDown, false>(mH, mD, mD, mYo, mYo, a2, mtiles_bound * a2.n_tiles, s);
 }
 
 cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const void* dyp,
@@ -781,23 +841,26 @@ cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const vo
         !map_3d_kmajor(&mG, w_gate, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows) ||
         !map_3d_kmajor(&mU, w_up, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows))
         return cudaErrorInvalidValue;
-    CUtensorMap mOut;  // [dg | du] viewed as (rows, 2, F): 32 x 32 pieces for the epilogue's stores
-    if (!map_halves_store(&mOut, dgu, (uint64_t)c.F, (uint64_t)max_rows)) return cudaErrorInvalidValue;
+    // the epilogues' stores: [dg | du] viewed as (rows, 2, F), dXp (rows, D)
+    CUtensorMap mOut, mXo;
+    if (!map_halves_store(&mOut, dgu, (uint64_t)c.F, (uint64_t)max_rows) ||
+        !map_store_2d(&mXo, dxp, (uint64_t)c.D, (uint64_t)max_rows))
+        return cudaErrorInvalidValue;
     const int64_t bm = pair ? 256 : 128;
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
     // dH = dYp . Wd^T (K = D), epilogue through SwiGLU into [dg | du]
     Args a1{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dgu), c.E, c.D, c.F,
             (c.F + 255) / 256, 2 * (int64_t)c.F, max_rows, c.T * c.K, nullptr,
             static_cast<const __nv_bfloat16*>(gu), status};
-    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mOut, a1, mtiles_bound * a1.n_tiles, s)
-                           : launch_one<kDgradH, false>(mA, mWd, mOut, a1, mtiles_bound * a1.n_tiles, s);
+    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mWd, mOut, mOut, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<kDgradH, false>(mA, mWd, mWd, mOut, mOut, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     // dXp = [dg | du] . [Wg | Wu]^T (K = 2F), unit weights
     Args a2{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dxp), c.E, c.F, c.D,
             (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status};
-    return pair ? launch_one<kDgradX, true>(mDGU, mG, mU, a2, mtiles_bound * a2.n_tiles, s)
-                : launch_one<kDgradX, false>(mDGU, mG, mU, a2, mtiles_bound * a2.n_tiles, s);
+    return pair ? launch_one<kDgradX, true>(mDGU, mG, mU, mXo, mXo, a2, mtiles_bound * a2.n_tiles, s)
+                : launch_one<kDgradX, false>(mDGU, mG, mU, mXo, mXo, a2, mtiles_bound * a2.n_tiles, s);
 }
 
 }  // namespace moe
