@@ -2,7 +2,8 @@
 
 A convenience over the C ABI for callers that work in PyTorch: it allocates
 the device workspace once (through torch), keeps the weights resident, and
-calls ``moe_forward``.  It adds no arithmetic of its own.
+calls ``moe_forward`` (inference), or ``moe_forward_train`` and
+``moe_backward`` (training).  It adds no arithmetic of its own.
 """
 from __future__ import annotations
 
@@ -12,7 +13,8 @@ from . import _binding as B
 
 
 class MoELayer:
-    """Token-choice top-k MoE layer forward on one CUDA device.
+    """Token-choice top-k MoE layer (forward, and the backward of bf16 layers)
+    on one CUDA device.
 
     weights: w_router (D, E) fp32; w_gate, w_up (E, D, F); w_down (E, F, D) in
     the layer dtype (bf16 or fp32); optional router_bias (E) fp32.
