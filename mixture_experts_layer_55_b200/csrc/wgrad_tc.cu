@@ -18,8 +18,8 @@
 // result is stored in fp32 (the precision weight gradients are accumulated in).
 //
 // Persistent kernel, one CTA per SM, tiles M = 128 x N = 256, 4-stage ring of
-// 48 KB, double-buffered 2 x 256-column accumulators.  10 warps: warp 0 TMA,
-// warp 1 MMA (all lanes wait and zero; one issues), warps 2..9 epilogue.  The
+// 48 KB, double-buffered 2 x 256-column accumulators.  11 warps: warp 0 TMA,
+// warp 1 MMA (one thread), warps 2..9 epilogue, warp 10 the tail fixer.  The
 // epilogue stages each warp's 32 x 32 fp32 pieces in shared memory (128-byte
 // swizzle, conflict-free) and writes them with TMA tensor stores over an
 // (E, M, N) map, so the stores are whole lines and the map clips the tile's
@@ -242,8 +242,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int s = 0; s < STAGES; ++s)
                 if (last_bar[s] >= 0)
                     mbar_wait(last_bar[s] ? &m->pfull[s] : &m->full[s], last_par[s], a.status, 511, nullptr);
-    } else if (warp == 1 && rank == 0) {
-        // -------------------------------- MMA issuer (leader; whole warp)
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ---------------------------------------- MMA issuer (leader; one thread)
         // A and B MN-major: 64-column boxes 8 KB apart (LBO), 8-row K groups
         // 1024 B apart (SBO), +2048 B per 16-row K step
         constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, 1, 1);
@@ -257,16 +257,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int e, m0, hf, n0;
             decode(a, BM, t, e, m0, hf, n0);
             const int r0 = m->off[e], r1 = m->off[e + 1];
-            // every lane waits (each wait is bounded); the vote keeps the warp converged
-            if (!__all_sync(0xffffffffu, mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 520, abort_flag)))
-                break;
+            if (!mbar_wait(&m->tempty[acc], acc_phase ^ 1u, a.status, 520, abort_flag)) break;
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * ACC_COLS);
             for (int k = r0; k < r1; k += BK) {
                 // rows of this block that belong to the expert; steps past the
                 // expert's last row are not issued, and a partial step's tail rows
                 // (the next expert's, or rows past the written ones) are zeroed by
-                // the fixer warp first: then this warp waits on fixed[] instead
+                // the fixer warp first: then this thread waits on fixed[] instead
                 const int valid = r1 - k < BK ? r1 - k : BK;
                 const int nsteps = (valid + UK - 1) / UK, rem = valid % UK;
                 bool got;
@@ -277,49 +275,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     got = mbar_wait(&m->full[stage], (fullph >> stage) & 1u, a.status, 521, abort_flag);
                     fullph ^= 1u << stage;
                 }
-                if (!__all_sync(0xffffffffu, got)) {
+                if (!got) {
                     ok = false;
                     break;
                 }
-                uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
-                const uint32_t a32 = smem_u32(sA);
+                tc_fence_after();
+                const uint32_t a32 = smem_u32(stages + (size_t)stage * STAGE_BYTES);
                 const uint32_t b32 = a32 + G::A_BYTES;
-                __syncwarp();
-                if (lane == 0) {
-                    tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < BK / UK; ++kk) {
-                        if (kk >= nsteps) break;
-                        const uint32_t accum = (k != r0 || kk != 0) ? 1u : 0u;
-                        const uint64_t adesc = umma_desc_sw128(a32 + kk * 2048, BOX_BYTES, 1024);
-                        const uint64_t bdesc = umma_desc_sw128(b32 + kk * 2048, BOX_BYTES, 1024);
-                        if (PAIR) umma_f16_ss_pair(d0, adesc, bdesc, idesc, accum);
-                        else umma_f16_ss(d0, adesc, bdesc, idesc, accum);
-                    }
-                    // frees the stage (in both CTAs) once these MMAs complete
-                    if (PAIR) umma_commit_pair_mc(&m->empty[stage], 0x3);
-                    else umma_commit(&m->empty[stage]);
+                for (int kk = 0; kk < BK / UK; ++kk) {
+                    if (kk >= nsteps) break;
+                    const uint32_t accum = (k != r0 || kk != 0) ? 1u : 0u;
+                    const uint64_t adesc = umma_desc_sw128(a32 + kk * 2048, BOX_BYTES, 1024);
+                    const uint64_t bdesc = umma_desc_sw128(b32 + kk * 2048, BOX_BYTES, 1024);
+                    if (PAIR) umma_f16_ss_pair(d0, adesc, bdesc, idesc, accum);
+                    else umma_f16_ss(d0, adesc, bdesc, idesc, accum);
                 }
-                __syncwarp();
+                // frees the stage (in both CTAs) once these MMAs complete
+                if (PAIR) umma_commit_pair_mc(&m->empty[stage], 0x3);
+                else umma_commit(&m->empty[stage]);
                 if (++stage == STAGES) stage = 0;
             }
             if (!ok) break;
-            if (lane == 0) {  // with no rows: arrives at once
-                if (PAIR) umma_commit_pair_mc(&m->tfull[acc], 0x3);
-                else umma_commit(&m->tfull[acc]);
-            }
-            __syncwarp();
+            // accumulator ready for the epilogue (of both CTAs); with no rows: at once
+            if (PAIR) umma_commit_pair_mc(&m->tfull[acc], 0x3);
+            else umma_commit(&m->tfull[acc]);
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
         }
-        if (lane == 0) {
-            if (PAIR) umma_commit_pair_mc(&m->drain, 0x1);
-            else umma_commit(&m->drain);
-            mbar_wait(&m->drain, 0, a.status, 522, nullptr);
-        }
-        __syncwarp();
+        // wait for every MMA issued here before the allocation is released
+        if (PAIR) umma_commit_pair_mc(&m->drain, 0x1);
+        else umma_commit(&m->drain);
+        mbar_wait(&m->drain, 0, a.status, 522, nullptr);
     } else if (warp == FIX_WARP && rank == 0) {
         // ------------------------------------ tail fixer (leader; whole warp)
         // Walks the MMA warp's schedule; for each partial block, once every copy
