@@ -118,9 +118,25 @@ MOE_DEVICE bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that may suspend the thread until the phase completes or about
+// `hint_ns` pass, so a waiting role does not take issue slots from the others.
+MOE_DEVICE bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false (and raises the timeout
 // flag) if the phase did not complete within limit_ns (kWaitLimitNs by
-// default), or if *abort was set by another role of the same CTA.
+// default), or if *abort was set by another role of the same CTA.  Each poll
+// may sleep up to 0.1 ms (woken early when the phase completes).
 MOE_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where,
                           volatile int* abort_flag, uint64_t limit_ns = kWaitLimitNs)
 {
@@ -128,7 +144,7 @@ MOE_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where
     uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
         if (((++spins) & 255u) == 0u) {
             if (abort_flag != nullptr && *abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
