@@ -88,17 +88,29 @@ struct Args {
     int halves;              // 1, or 2 when B holds two Nh-column halves
     int mt;                  // ceil(M / BM)
     int nth;                 // ceil(Nh / BN)
+    int n_fast;              // tile order within an expert: n tiles fastest (else m)
     int64_t max_rows;
     int* status;
 };
 
+// Tiles of one expert are consecutive; within the expert the fast index is
+// the one whose operand block is the smaller, so that the concurrently running
+// tiles keep that whole block in L2 and read the other block's slabs once.
 MOE_DEVICE void decode(const Args& a, int bm, int t, int& e, int& m0, int& hf, int& n0)
 {
-    const int per_e = a.mt * a.nth * a.halves;
+    const int nn = a.nth * a.halves;  // n tiles over both halves
+    const int per_e = a.mt * nn;
     e = t / per_e;
     const int r = t - e * per_e;
-    const int j = r / a.mt;  // n tile over both halves
-    m0 = (r - j * a.mt) * bm;
+    int i, j;
+    if (a.n_fast) {
+        i = r / nn;
+        j = r - i * nn;
+    } else {
+        j = r / a.mt;
+        i = r - j * a.mt;
+    }
+    m0 = i * bm;
     hf = j / a.nth;
     n0 = (j - hf * a.nth) * BN;
 }
@@ -562,7 +574,10 @@ cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets
         !map_out(&mO0, out0, (uint64_t)Nh, (uint64_t)M, (uint64_t)E) ||
         !map_out(&mO1, halves == 2 ? out1 : out0, (uint64_t)Nh, (uint64_t)M, (uint64_t)E))
         return cudaErrorInvalidValue;
-    Args a{offsets, E, M, Nh, halves, 0, (Nh + BN - 1) / BN, max_rows, status};
+    // the A block of an expert (M columns) larger than its B block (halves * Nh):
+    // walk the n tiles fastest (e.g. the down projection's gradient, M = F)
+    const int n_fast = (int64_t)M > (int64_t)Nh * halves ? 1 : 0;
+    Args a{offsets, E, M, Nh, halves, 0, (Nh + BN - 1) / BN, n_fast, max_rows, status};
     return M >= 256 ? launch_mode<true>(mA, mB, mO0, mO1, a, s) : launch_mode<false>(mA, mB, mO0, mO1, a, s);
 }
 
