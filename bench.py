@@ -559,7 +559,9 @@ def run_gpu_ep(args):
     """Expert parallelism: rank r of N holds experts r*E/N .. (r+1)*E/N - 1 and
     its own T tokens; a step is one ExpertParallelMoE forward on every rank
     (route, owner-sorted dispatch, NCCL all-to-all, grouped local experts,
-    reverse all-to-all, weighted combine)."""
+    reverse all-to-all, weighted combine; or, with --exchange peer, the
+    dispatch kernel storing rows into the owners' peer-mapped buffers, the
+    experts in place and the combine kernel loading from the owners)."""
     import mixture_experts_layer_55_b200 as M
     from mixture_experts_layer_55_b200.ep import ExpertParallelMoE
 
@@ -582,7 +584,8 @@ def run_gpu_ep(args):
     sl = slice(rank * EL, (rank + 1) * EL)
     layer = ExpertParallelMoE(wl.T, inp["w_router"], inp["w_gate"][sl].contiguous(),
                               inp["w_up"][sl].contiguous(), inp["w_down"][sl].contiguous(), wl.E,
-                              wl.K, wl.capacity_factor, router_bias=inp["bias"])
+                              wl.K, wl.capacity_factor, router_bias=inp["bias"],
+                              exchange=args.exchange)
     del inp["w_gate"], inp["w_up"], inp["w_down"]
     nbuf = 3
     xs = [make_tokens(wl, device=dev, seed=rank_token_seed(rank) * 16 + i) for i in range(nbuf)]
@@ -620,6 +623,7 @@ def run_gpu_ep(args):
     torch.cuda.synchronize(dev)
     dist.barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    per_step = count_library_launches(lambda: layer.forward(xs[0], logit_noise=inp["noise"]), dev)
     flags = layer.ops.status()
     if flags:
         raise RuntimeError(f"device status flags {flags:#x} after the benchmark")
@@ -636,12 +640,13 @@ def run_gpu_ep(args):
             "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
                        "capacity_factor": wl.capacity_factor,
                        "parallelism": f"expert parallel x{world} ({EL} experts per rank, "
-                                      "NCCL all-to-all)",
+                                      + ("NCCL all-to-all)" if args.exchange == "all_to_all" else
+                                         "peer-memory dispatch and combine kernels)"),
                        "l2": "inputs larger than L2"},
             "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io, "d2h_bytes_per_step": io,
                     "how": "per step: x in from pinned host memory, ExpertParallelMoE.forward, y out"},
-            "gpu_launches": None,
+            "gpu_launches": None if per_step is None else per_step * args.steps,
             "roofline": None,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -649,7 +654,23 @@ def run_gpu_ep(args):
         if args.warmup < 3:
             line["note"] = "fewer than 3 warm-up steps: not a valid measurement"
         print(json.dumps(line), flush=True)
+    layer.close()
     dist.destroy_process_group()
+
+
+def count_library_launches(step, dev):
+    """Kernels of this library (namespace moe::) that one call of `step`
+    launches, counted by the CUDA profiler on an extra, untimed call; None if
+    the profiler is unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step()
+            torch.cuda.synchronize(dev)
+        return sum(1 for ev in prof.events()
+                   if ev.device_type == torch.autograd.DeviceType.CUDA and "moe::" in ev.name)
+    except Exception:  # pragma: no cover - profiler missing on this machine
+        return None
 
 
 def _finish(world):
@@ -841,6 +862,9 @@ def main(argv=None):
                     help="forward (default) or a training step (forward + backward)")
     ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
                     help="replicas (default): every GPU holds all experts; ep: experts sharded")
+    ap.add_argument("--exchange", choices=["all_to_all", "peer"], default="all_to_all",
+                    help="with --parallel ep: NCCL all-to-all, or the library's kernels over "
+                         "peer-mapped buffers")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         run_reference(args)

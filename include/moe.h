@@ -399,6 +399,93 @@ MOE_API moe_status moe_combine_weighted(const moe_config *cfg, const void *y_per
                                         const int32_t *row_of, const float *topk_w,
                                         const void *y_add, void *y, void *stream);
 
+/* ------------------------------------------ expert parallelism over peer memory
+ *
+ * The same layer with the two exchanges done by this library's kernels
+ * instead of all-to-all collectives: every rank's receive buffers are mapped
+ * into every rank's address space (CUDA IPC; NVLink between the GPUs of one
+ * node), the dispatch kernel stores each kept token row straight into its
+ * owner's receive buffer at its expert-major row, the owner runs moe_expert_ffn
+ * on that buffer, and the combine kernel loads each kept slot's result from
+ * its owner's output buffer.  The caller's communication library supplies an
+ * all-gather of the kept counts (world x E int32, each rank's moe_dispatch
+ * `kept`) before moe_ep_peer_dispatch, and two stream-ordered barriers: after
+ * moe_ep_peer_dispatch on every rank (all rows have arrived) and after every
+ * owner's moe_expert_ffn (all results are ready).  No host synchronisation.
+ *
+ * Receive layout.  Rank o's buffer holds its experts e = o*EL .. o*EL+EL-1
+ * (EL = E / world) in order; expert e's block holds the kept rows of sources
+ * 0 .. world-1 in order, each source's rows in its own expert-major order.
+ * The slot (t, k) of source `rank`, routed to expert e and kept at local row
+ * r = row_of[t, k], lands at
+ *   sum_{o*EL <= e' < e} sum_s kept_all[s][e'] + sum_{s < rank} kept_all[s][e]
+ *     + (r - offsets[e])
+ * of its owner's buffer -- the expert-major order of the all-to-all path's
+ * moe_ep_layout.
+ */
+
+/* Bytes of one peer-exchange handle (a cudaIpcMemHandle_t). */
+#define MOE_IPC_HANDLE_BYTES 64
+
+/*
+ * Setup-time entry points for the peer-mapped buffers (not for the per-step
+ * path: they allocate, and opening a mapping synchronises).  moe_ipc_alloc:
+ * `bytes` of device memory on the current device (*ptr) and its exchange
+ * handle (MOE_IPC_HANDLE_BYTES host bytes, written to `handle`), to be sent
+ * to the other ranks.  moe_ipc_open: map another process's buffer from its
+ * handle into this process (*ptr; a handle of this process's own buffer is
+ * refused by CUDA: use the pointer itself).  moe_ipc_close unmaps, moe_ipc_free
+ * frees the owner's buffer (after every peer has closed it).  MOE_ERR_CUDA on
+ * any CUDA error; *ptr is NULL then.
+ */
+MOE_API moe_status moe_ipc_alloc(size_t bytes, void **ptr, void *handle);
+MOE_API moe_status moe_ipc_open(const void *handle, void **ptr);
+MOE_API moe_status moe_ipc_close(void *ptr);
+MOE_API moe_status moe_ipc_free(void *ptr);
+
+/*
+ * Dispatch of this rank's tokens into the owners' receive buffers.
+ *   cfg            this rank's layer: T tokens, all E experts (E % world == 0)
+ *   rank, world    this rank and the number of ranks (1 <= world <= 64)
+ *   kept_all       (world, E) int32, device: every rank's kept counts
+ *   x              (T, D) activations, device, 16-byte aligned
+ *   topk_ids, row_of, offsets
+ *                  this rank's moe_route ids (T, K) and moe_dispatch row_of
+ *                  (T, K) and offsets (E + 1), device (moe_dispatch may be
+ *                  called with x = x_perm = NULL: no local gather is needed)
+ *   recv_bufs      device array of `world` device pointers: rank o's receive
+ *                  buffer (its own pointer at index `rank`, peers' from
+ *                  moe_ipc_open), each recv_rows rows of D elements
+ *   local_offsets  out, device (EL + 1) int32: this rank's receive layout,
+ *                  the offsets moe_expert_ffn takes (cfg.T = recv_rows, E = EL,
+ *                  K = 1)
+ *   remote_row     out, device (T, K) int32: the slot's row in its owner's
+ *                  buffer, -1 for a dropped slot (moe_ep_peer_combine's map)
+ *   workspace      moe_ep_workspace_size(world, EL) bytes
+ * A count, id, row or destination out of range raises the bounds flag of
+ * the workspace's status word (moe_get_device_status) and skips the slot.
+ */
+MOE_API moe_status moe_ep_peer_dispatch(const moe_config *cfg, int32_t rank, int32_t world,
+                                        const int32_t *kept_all, const void *x,
+                                        const int32_t *topk_ids, const int32_t *row_of,
+                                        const int32_t *offsets, void *const *recv_bufs,
+                                        int64_t recv_rows, int32_t *local_offsets,
+                                        int32_t *remote_row, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/*
+ * Weighted combine from the owners' output buffers: y[t] = y_add[t] + sum over
+ * kept slots, in slot order, of topk_w[t, k] * y_bufs[owner][remote_row[t, k]],
+ * fp32 sums rounded once to cfg.dtype.  y_bufs: device array of `world`
+ * device pointers to the owners' moe_expert_ffn outputs (unweighted:
+ * perm = topk_w = NULL there), recv_rows rows each.  y_add (T, D) or NULL.
+ */
+MOE_API moe_status moe_ep_peer_combine(const moe_config *cfg, int32_t world, const int32_t *topk_ids,
+                                       const int32_t *remote_row, const float *topk_w,
+                                       const void *const *y_bufs, int64_t recv_rows,
+                                       const void *y_add, void *y, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
 /*
  * moe_dispatch without a workspace, for callers that cannot allocate device
  * memory: code handed only its input and output buffers by a host framework

@@ -104,6 +104,14 @@ _SIG = {
     "moe_permute_rows": ([_P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P],
                          ctypes.c_int32),
     "moe_combine_weighted": ([_P] * 7, ctypes.c_int32),
+    "moe_ipc_alloc": ([ctypes.c_size_t, _P, _P], ctypes.c_int32),
+    "moe_ipc_open": ([_P, _P], ctypes.c_int32),
+    "moe_ipc_close": ([_P], ctypes.c_int32),
+    "moe_ipc_free": ([_P], ctypes.c_int32),
+    "moe_ep_peer_dispatch": ([_P, ctypes.c_int32, ctypes.c_int32] + [_P] * 6
+                             + [ctypes.c_int64, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_ep_peer_combine": ([_P, ctypes.c_int32] + [_P] * 4 + [ctypes.c_int64, _P, _P, _P,
+                                                               ctypes.c_size_t, _P], ctypes.c_int32),
 }
 
 
@@ -407,3 +415,73 @@ def moe_permute_rows(inp, idx, n: int, out, workspace, stream=None):
 def moe_combine_weighted(cfg, y_perm, row_of, topk_w, y, y_add=None, stream=None):
     _check(lib().moe_combine_weighted(_cfg(cfg), _ptr(y_perm), _ptr(row_of), _ptr(topk_w),
                                       _ptr(y_add), _ptr(y), _stream(stream)), "moe_combine_weighted")
+
+
+# ------------------------------------------ expert parallelism over peer memory
+
+IPC_HANDLE_BYTES = 64
+
+
+def ipc_alloc(nbytes: int):
+    """(device address, handle bytes) of a new peer-mappable buffer."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().moe_ipc_alloc(int(nbytes), ctypes.byref(ptr), handle), "moe_ipc_alloc")
+    return ptr.value, handle.raw
+
+
+def ipc_open(handle: bytes) -> int:
+    """Device address of another process's buffer, from its handle."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has 64 bytes")
+    ptr = ctypes.c_void_p()
+    buf = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+    _check(lib().moe_ipc_open(buf, ctypes.byref(ptr)), "moe_ipc_open")
+    return ptr.value
+
+
+def ipc_close(ptr: int):
+    _check(lib().moe_ipc_close(ptr), "moe_ipc_close")
+
+
+def ipc_free(ptr: int):
+    _check(lib().moe_ipc_free(ptr), "moe_ipc_free")
+
+
+class DeviceBuffer:
+    """A raw device buffer seen as a tensor (no copy), through the CUDA array
+    interface; keeps nothing alive but the address."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(int(v) for v in shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+def as_tensor(ptr: int, shape, dtype):
+    """Tensor view of `shape` elements of `dtype` at device address ptr."""
+    import torch
+    typestr = {torch.bfloat16: "<V2", torch.float32: "<f4", torch.int32: "<i4",
+               torch.uint8: "|u1"}[dtype]
+    if dtype == torch.bfloat16:  # the array interface has no bf16: view int16 as bf16
+        t = torch.as_tensor(DeviceBuffer(ptr, shape, "<i2"), device="cuda")
+        return t.view(torch.bfloat16)
+    return torch.as_tensor(DeviceBuffer(ptr, shape, typestr), device="cuda")
+
+
+def moe_ep_peer_dispatch(cfg, rank: int, world: int, kept_all, x, topk_ids, row_of, offsets,
+                         recv_bufs, recv_rows: int, local_offsets, remote_row, workspace, stream=None):
+    """recv_bufs: int64 device tensor of `world` receive-buffer addresses."""
+    _check(lib().moe_ep_peer_dispatch(_cfg(cfg), int(rank), int(world), _ptr(kept_all), _ptr(x),
+                                      _ptr(topk_ids), _ptr(row_of), _ptr(offsets), _ptr(recv_bufs),
+                                      int(recv_rows), _ptr(local_offsets), _ptr(remote_row),
+                                      _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "moe_ep_peer_dispatch")
+
+
+def moe_ep_peer_combine(cfg, world: int, topk_ids, remote_row, topk_w, y_bufs, recv_rows: int, y,
+                        workspace, y_add=None, stream=None):
+    """y_bufs: int64 device tensor of `world` expert-output buffer addresses."""
+    _check(lib().moe_ep_peer_combine(_cfg(cfg), int(world), _ptr(topk_ids), _ptr(remote_row),
+                                     _ptr(topk_w), _ptr(y_bufs), int(recv_rows), _ptr(y_add), _ptr(y),
+                                     _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "moe_ep_peer_combine")

@@ -713,6 +713,94 @@ moe_status moe_combine_weighted(const moe_config* cfg, const void* y_perm, const
                                       static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_ipc_alloc(size_t bytes, void** ptr, void* handle)
+{
+    static_assert(sizeof(cudaIpcMemHandle_t) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+    if (ptr == nullptr || handle == nullptr || bytes == 0) return MOE_ERR_ARG;
+    *ptr = nullptr;
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    e = cudaIpcGetMemHandle(&h, p);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return MOE_ERR_CUDA;
+    }
+    memcpy(handle, &h, sizeof h);
+    *ptr = p;
+    return MOE_OK;
+}
+
+moe_status moe_ipc_free(void* ptr)
+{
+    if (ptr == nullptr) return MOE_OK;
+    return cuda_status(cudaFree(ptr));
+}
+
+moe_status moe_ipc_open(const void* handle, void** ptr)
+{
+    if (ptr == nullptr || handle == nullptr) return MOE_ERR_ARG;
+    *ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof h);
+    void* p = nullptr;
+    cudaError_t e = cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    *ptr = p;
+    return MOE_OK;
+}
+
+moe_status moe_ipc_close(void* ptr)
+{
+    if (ptr == nullptr) return MOE_OK;
+    return cuda_status(cudaIpcCloseMemHandle(ptr));
+}
+
+static moe_status check_peer_args(const moe_config* cfg, int32_t world, int64_t recv_rows, const void* ws,
+                                  size_t ws_bytes)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (world < 1 || world > 64 || cfg->E % world != 0) return MOE_ERR_ARG;
+    if (recv_rows < 1 || recv_rows > (int64_t)INT32_MAX) return MOE_ERR_SHAPE;
+    size_t need = 0;
+    st = moe_ep_workspace_size(world, cfg->E / world, &need);
+    if (st != MOE_OK) return st;
+    return check_ws(nullptr, ws, ws_bytes, need);
+}
+
+moe_status moe_ep_peer_dispatch(const moe_config* cfg, int32_t rank, int32_t world, const int32_t* kept_all,
+                                const void* x, const int32_t* topk_ids, const int32_t* row_of,
+                                const int32_t* offsets, void* const* recv_bufs, int64_t recv_rows,
+                                int32_t* local_offsets, int32_t* remote_row, void* workspace,
+                                size_t workspace_bytes, void* stream)
+{
+    moe_status st = check_peer_args(cfg, world, recv_rows, workspace, workspace_bytes);
+    if (st != MOE_OK) return st;
+    if (rank < 0 || rank >= world) return MOE_ERR_ARG;
+    if (!kept_all || !x || !topk_ids || !row_of || !offsets || !recv_bufs || !local_offsets || !remote_row)
+        return MOE_ERR_ARG;
+    if (!aligned16(x)) return MOE_ERR_ALIGN;
+    return cuda_status(launch_peer_dispatch(*cfg, rank, world, kept_all, x, topk_ids, row_of, offsets,
+                                            recv_bufs, recv_rows, max_rows_of(*cfg), local_offsets,
+                                            remote_row, static_cast<int*>(workspace),
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_peer_combine(const moe_config* cfg, int32_t world, const int32_t* topk_ids,
+                               const int32_t* remote_row, const float* topk_w, const void* const* y_bufs,
+                               int64_t recv_rows, const void* y_add, void* y, void* workspace,
+                               size_t workspace_bytes, void* stream)
+{
+    moe_status st = check_peer_args(cfg, world, recv_rows, workspace, workspace_bytes);
+    if (st != MOE_OK) return st;
+    if (!topk_ids || !remote_row || !topk_w || !y_bufs || !y) return MOE_ERR_ARG;
+    if (!aligned16(y) || (y_add && !aligned16(y_add))) return MOE_ERR_ALIGN;
+    return cuda_status(launch_peer_combine(*cfg, world, y_bufs, topk_ids, remote_row, topk_w, recv_rows, y_add,
+                                           y, static_cast<int*>(workspace), static_cast<cudaStream_t>(stream)));
+}
+
 int32_t moe_backward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;

@@ -16,6 +16,7 @@
 // layout from the exchanged counts and move rows between the two orders.
 #include "common.cuh"
 #include "internal.h"
+#include "vec.cuh"
 
 namespace moe {
 
@@ -148,6 +149,264 @@ cudaError_t launch_permute_rows(const void* in, const int32_t* idx, void* out, i
     if (blocks > cap) blocks = cap;
     permute_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(in), idx,
                                                          static_cast<uint4*>(out), n, vpr, in_rows, status);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------ exchange over peer memory --
+//
+// The same exchange done by the layer's own kernels, with every rank's
+// receive buffers mapped into every other rank's address space (CUDA IPC over
+// NVLink).  The dispatch kernel reads each token row once and stores it
+// straight into the owner's receive buffer at its expert-major row; the owner
+// runs its grouped experts there; the combine kernel loads each kept slot's
+// result from the owner's output buffer and adds it, weighted, at home.  That
+// replaces the host read of the sizes, both all-to-alls and both
+// permutations.  The only collectives left are an all-gather of the kept
+// counts (world x E int32) before the dispatch and two stream-ordered
+// barriers of the caller's communication library: after the dispatch (every
+// row has arrived) and after the experts (every result is ready).
+//
+// Row of slot (t, k) in its owner's receive buffer.  Expert e (owner
+// o = e / EL, local index e - o*EL) holds, in order, the rows of sources
+// 0 .. world-1; source `rank`'s rows of e follow the other sources' before it:
+//   seg_base[e] = sum_{o*EL <= e' < e} sum_s kept_all[s][e']
+//               + sum_{s < rank} kept_all[s][e]
+//   remote_row(t, k) = seg_base[e] + (row_of[t, k] - offsets[e])
+// where row_of[t, k] - offsets[e] is the slot's rank among this source's kept
+// rows of e (the local expert-major dispatch).
+constexpr int kPeerMaxWorld = 64;
+constexpr int kPeerMaxE = 256;
+
+// seg_base (and own_base: the first part alone) of every expert, computed by
+// the whole block from the gathered counts; negative counts raise the bounds
+// flag and count as 0.
+MOE_DEVICE void peer_segment_bases(const int32_t* __restrict__ kept_all, int W, int E, int EL, int rank,
+                                   int32_t* tot, int32_t* own_base, int32_t* seg_base, int* status)
+{
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t sum = 0, before = 0;
+        for (int s = 0; s < W; ++s) {
+            int32_t c = kept_all[(int64_t)s * E + e];
+            if (c < 0) {
+                raise_flag(status, kFlagBounds, 720);
+                c = 0;
+            }
+            sum += c;
+            if (s < rank) before += c;
+        }
+        tot[e] = sum;
+        seg_base[e] = before;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int first = (e / EL) * EL;
+        int32_t acc = 0;
+        for (int j = first; j < e; ++j) acc += tot[j];
+        own_base[e] = acc;
+        seg_base[e] += acc;
+    }
+    __syncthreads();
+}
+
+// Slot (t, k) -> (owner, remote row), or owner -1 for a dropped slot; an
+// out-of-range id, row or remote row raises the bounds flag and drops it.
+MOE_DEVICE int peer_slot(const int32_t* __restrict__ ids, const int32_t* __restrict__ row_of,
+                         const int32_t* offs, const int32_t* seg_base, int64_t slot, int E, int EL,
+                         int64_t recv_rows, int64_t max_rows, int32_t* remote, int* status, int where)
+{
+    const int32_t r = row_of[slot];
+    if (r < 0) return -1;
+    const int32_t e = ids[slot];
+    if (e < 0 || e >= E || r >= max_rows || r < offs[e] || r >= offs[e + 1]) {
+        raise_flag(status, kFlagBounds, where);
+        return -1;
+    }
+    const int64_t d = (int64_t)seg_base[e] + (r - offs[e]);
+    if (d < 0 || d >= recv_rows) {
+        raise_flag(status, kFlagBounds, where + 1);
+        return -1;
+    }
+    *remote = (int32_t)d;
+    return e / EL;
+}
+
+// Each thread moves VPT 16-byte vectors of token rows: vector i of the
+// flattened (T x vpr) input is loaded once and stored to each kept slot's
+// row in its owner's receive buffer.  Block 0 also writes this rank's local
+// offsets; every block writes remote_row for its share of the slots (the
+// combine's map back).  Every thread ends with a system-scope fence, so its
+// peer stores are visible before the barrier that follows the kernel.
+template <int KS>
+__global__ void __launch_bounds__(256) peer_dispatch_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ ids, const int32_t* __restrict__ row_of,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ kept_all,
+    uint4* const* __restrict__ recv_bufs, int64_t T, int K, int E, int EL, int W, int rank, int64_t vpr,
+    int64_t recv_rows, int64_t max_rows, int32_t* __restrict__ local_offsets,
+    int32_t* __restrict__ remote_row, int* status)
+{
+    constexpr int VPT = 8 / KS;
+    __shared__ int32_t tot[kPeerMaxE], own[kPeerMaxE], seg[kPeerMaxE], offs[kPeerMaxE + 1];
+    __shared__ uint4* bufs[kPeerMaxWorld];
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) offs[i] = offsets[i];
+    for (int i = threadIdx.x; i < W; i += blockDim.x) bufs[i] = recv_bufs[i];
+    peer_segment_bases(kept_all, W, E, EL, rank, tot, own, seg, status);
+    if (blockIdx.x == 0)
+        for (int j = threadIdx.x; j <= EL; j += blockDim.x) {
+            const int e = rank * EL + (j < EL ? j : EL - 1);
+            local_offsets[j] = j < EL ? own[e] : own[e] + tot[e];
+        }
+    const int64_t G = (int64_t)gridDim.x * blockDim.x;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t sl = tid; sl < T * K; sl += G) {
+        int32_t d = -1;
+        if (peer_slot(ids, row_of, offs, seg, sl, E, EL, recv_rows, max_rows, &d, status, 730) < 0) d = -1;
+        remote_row[sl] = d;
+    }
+    const int64_t n = T * vpr;
+    for (int64_t base = tid; base < n; base += G * VPT) {
+        uint4 vals[VPT];
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) {
+            const int64_t i = base + (int64_t)u * G;
+            vals[u] = i < n ? __ldg(x + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) {
+            const int64_t i = base + (int64_t)u * G;
+            if (i >= n) break;
+            const int64_t t = i / vpr, v = i - t * vpr;
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                if (k >= K) break;
+                int32_t d = 0;
+                const int o = peer_slot(ids, row_of, offs, seg, t * K + k, E, EL, recv_rows, max_rows, &d,
+                                        status, 732);
+                if (o >= 0) bufs[o][(int64_t)d * vpr + v] = vals[u];
+            }
+        }
+    }
+    __threadfence_system();
+}
+
+// y[t] = y_add[t] + sum over kept slots, in slot order, of topk_w[t, k] *
+// (owner's y_loc)[remote_row[t, k]]: fp32 sums, rounded once.  The owners'
+// rows are read with plain (coherent) loads: they were written by another
+// GPU's kernel before the barrier that precedes this one.
+template <typename ET, int KS>
+__global__ void __launch_bounds__(256) peer_combine_kernel(
+    const uint4* const* __restrict__ y_bufs, const int32_t* __restrict__ ids,
+    const int32_t* __restrict__ remote_row, const float* __restrict__ topk_w,
+    const uint4* __restrict__ y_add, uint4* __restrict__ y, int64_t T, int K, int E, int EL, int W,
+    int64_t vpr, int64_t recv_rows, int* status)
+{
+    constexpr int VPT = 8 / KS;
+    __shared__ const uint4* bufs[kPeerMaxWorld];
+    for (int i = threadIdx.x; i < W; i += blockDim.x) bufs[i] = y_bufs[i];
+    __syncthreads();
+    const int64_t n = T * vpr;
+    const int64_t G = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n; base += G * VPT) {
+        uint4 vals[VPT][KS];
+        int32_t own[VPT][KS];
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) {
+            const int64_t i = base + (int64_t)u * G;
+            const int64_t t = i < n ? i / vpr : 0, v = i - t * vpr;
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                own[u][k] = -1;
+                vals[u][k] = make_uint4(0, 0, 0, 0);
+                if (i >= n || k >= K) continue;
+                const int32_t d = __ldg(remote_row + t * K + k);
+                if (d < 0) continue;
+                const int32_t e = __ldg(ids + t * K + k);
+                if (e < 0 || e >= E || d >= recv_rows) {
+                    if (v == 0) raise_flag(status, kFlagBounds, 740);
+                    continue;
+                }
+                own[u][k] = e / EL;
+                vals[u][k] = bufs[own[u][k]][(int64_t)d * vpr + v];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) {
+            const int64_t i = base + (int64_t)u * G;
+            if (i >= n) break;
+            const int64_t t = i / vpr;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (y_add) Vec<ET>::add(acc, __ldg(y_add + i));
+#pragma unroll
+            for (int k = 0; k < KS; ++k)
+                if (own[u][k] >= 0) Vec<ET>::add_scaled(acc, vals[u][k], __ldg(topk_w + t * K + k));
+            y[i] = Vec<ET>::pack(acc);
+        }
+    }
+}
+
+static int64_t peer_blocks(int64_t n_vec, int vpt)
+{
+    int64_t blocks = (n_vec + 256LL * vpt - 1) / (256LL * vpt);
+    const int64_t cap = (int64_t)sm_count_ep() * 8;
+    if (blocks > cap) blocks = cap;
+    return blocks < 1 ? 1 : blocks;
+}
+
+cudaError_t launch_peer_dispatch(const moe_config& c, int rank, int W, const int32_t* kept_all, const void* x,
+                                 const int32_t* ids, const int32_t* row_of, const int32_t* offsets,
+                                 void* const* recv_bufs, int64_t recv_rows, int64_t max_rows,
+                                 int32_t* local_offsets, int32_t* remote_row, int* status, cudaStream_t s)
+{
+    const int64_t vpr = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
+    const int EL = c.E / W;
+    const int vpt = c.K <= 1 ? 8 : c.K == 2 ? 4 : c.K <= 4 ? 2 : 1;
+    const unsigned blocks = (unsigned)peer_blocks(c.T * vpr, vpt);
+    const uint4* xv = static_cast<const uint4*>(x);
+    uint4* const* rb = reinterpret_cast<uint4* const*>(recv_bufs);
+#define MOE_PEER_DISPATCH(KS)                                                                          \
+    peer_dispatch_kernel<KS><<<blocks, 256, 0, s>>>(xv, ids, row_of, offsets, kept_all, rb, c.T, c.K, c.E, \
+                                                    EL, W, rank, vpr, recv_rows, max_rows, local_offsets, \
+                                                    remote_row, status)
+    if (c.K <= 1) MOE_PEER_DISPATCH(1);
+    else if (c.K == 2) MOE_PEER_DISPATCH(2);
+    else if (c.K <= 4) MOE_PEER_DISPATCH(4);
+    else MOE_PEER_DISPATCH(8);
+#undef MOE_PEER_DISPATCH
+    return cudaGetLastError();
+}
+
+template <typename ET>
+static void launch_peer_combine_t(const moe_config& c, int W, unsigned blocks, const uint4* const* yb,
+                                  const int32_t* ids, const int32_t* remote_row, const float* topk_w,
+                                  const uint4* add, uint4* y, int64_t vpr, int64_t recv_rows, int* status,
+                                  cudaStream_t s)
+{
+    const int EL = c.E / W;
+#define MOE_PEER_COMBINE(KS)                                                                            \
+    peer_combine_kernel<ET, KS><<<blocks, 256, 0, s>>>(yb, ids, remote_row, topk_w, add, y, c.T, c.K, c.E, \
+                                                       EL, W, vpr, recv_rows, status)
+    if (c.K <= 1) MOE_PEER_COMBINE(1);
+    else if (c.K == 2) MOE_PEER_COMBINE(2);
+    else if (c.K <= 4) MOE_PEER_COMBINE(4);
+    else MOE_PEER_COMBINE(8);
+#undef MOE_PEER_COMBINE
+}
+
+cudaError_t launch_peer_combine(const moe_config& c, int W, const void* const* y_bufs, const int32_t* ids,
+                                const int32_t* remote_row, const float* topk_w, int64_t recv_rows,
+                                const void* y_add, void* y, int* status, cudaStream_t s)
+{
+    const int64_t vpr = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
+    const int vpt = c.K <= 1 ? 8 : c.K == 2 ? 4 : c.K <= 4 ? 2 : 1;
+    const unsigned blocks = (unsigned)peer_blocks(c.T * vpr, vpt);
+    const uint4* const* yb = reinterpret_cast<const uint4* const*>(y_bufs);
+    const uint4* add = static_cast<const uint4*>(y_add);
+    uint4* out = static_cast<uint4*>(y);
+    if (c.dtype == MOE_BF16)
+        launch_peer_combine_t<__nv_bfloat16>(c, W, blocks, yb, ids, remote_row, topk_w, add, out, vpr,
+                                             recv_rows, status, s);
+    else
+        launch_peer_combine_t<float>(c, W, blocks, yb, ids, remote_row, topk_w, add, out, vpr, recv_rows,
+                                     status, s);
     return cudaGetLastError();
 }
 

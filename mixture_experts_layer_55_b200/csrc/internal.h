@@ -178,6 +178,13 @@ cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float*
 cudaError_t launch_ep_layout(const int32_t* recv, int W, int EL, int64_t max_rows, int32_t* offsets,
                              int32_t* seg_src, int32_t* seg_dst, int32_t* dst_of, int32_t* src_of,
                              int* status, cudaStream_t s);
+cudaError_t launch_peer_dispatch(const moe_config& c, int rank, int W, const int32_t* kept_all, const void* x,
+                                 const int32_t* ids, const int32_t* row_of, const int32_t* offsets,
+                                 void* const* recv_bufs, int64_t recv_rows, int64_t max_rows,
+                                 int32_t* local_offsets, int32_t* remote_row, int* status, cudaStream_t s);
+cudaError_t launch_peer_combine(const moe_config& c, int W, const void* const* y_bufs, const int32_t* ids,
+                                const int32_t* remote_row, const float* topk_w, int64_t recv_rows,
+                                const void* y_add, void* y, int* status, cudaStream_t s);
 cudaError_t launch_permute_rows(const void* in, const int32_t* idx, void* out, int64_t n, int64_t row_bytes,
                                 int64_t in_rows, int* status, cudaStream_t s);
 cudaError_t launch_dx_assemble(const moe_config& c, const float* dL, const float* w_r, const void* dxp,

@@ -12,14 +12,26 @@ result sent back).  Rank r of W holds the contiguous experts r*EL .. r*EL+EL-1
 (EL = E / W) and its own batch of tokens; each rank's output equals the local
 layer's on that batch (routing, capacity and combine are the batch's own).
 
-The exchanges are collectives of ``torch.distributed`` (NCCL over NVLink on
-GPUs; all-to-all with per-rank sizes, which needs the counts on the host, one
-device-to-host read per forward).  Every other step is a kernel of the CUDA
-library, through its C ABI: routing and the owner-sorted (expert-major)
-dispatch, the receive layout and the row permutations, the grouped experts,
-the weighted combine.  ``ops`` can replace those steps (the CPU tests of the
-exchange logic pass the oracle's); the default is the CUDA library, and it
-fails loudly when that is not built.
+Two exchanges are built:
+
+- ``exchange="all_to_all"``: the exchanges are collectives of
+  ``torch.distributed`` (NCCL over NVLink on GPUs; all-to-all with per-rank
+  sizes, which needs the counts on the host, one device-to-host read per
+  forward).  Every other step is a kernel of the CUDA library, through its C
+  ABI: routing and the owner-sorted (expert-major) dispatch, the receive
+  layout and the row permutations, the grouped experts, the weighted combine.
+  ``ops`` can replace those steps (the CPU tests of the exchange logic pass
+  the oracle's).
+- ``exchange="peer"``: every rank's receive and expert-output buffers are
+  mapped into every rank (CUDA IPC), and the library's kernels move the rows
+  themselves: the dispatch kernel stores each kept token row straight into its
+  owner's buffer at its expert-major row, the owner's grouped experts run in
+  place, and the combine kernel loads each slot's result from its owner and
+  adds it, weighted, at home.  The communication library only all-gathers the
+  kept counts (world x E int32) and provides two stream-ordered barriers (a
+  one-element all-reduce): no host read, no all-to-all, no permutation.
+
+The default ops are the CUDA library, which fails loudly when it is not built.
 """
 from __future__ import annotations
 
@@ -98,6 +110,80 @@ class CudaOps:
             flags |= B.moe_get_device_status(ws)
         return flags
 
+    # ---- peer exchange: routing and the dispatch index only (no local gather),
+    # rows stored into the owners' buffers, experts in place, combine from the owners
+
+    def route_index(self, x, w_router, router_bias, selection_bias, logit_noise):
+        B.moe_route(self.cfg, x, w_router, self.ids, self.w, self.ws, router_bias=router_bias,
+                    logit_noise=logit_noise, selection_bias=selection_bias)
+        B.moe_dispatch(self.cfg, None, self.ids, self.counts, self.kept, self.offsets, self.perm,
+                       self.row_of, None, self.ws)
+        return self.kept
+
+    def peer_dispatch(self, x, kept_all, rank, W, peer):
+        if not hasattr(self, "remote_row"):
+            self.remote_row = torch.empty_like(self.row_of)
+        B.moe_ep_peer_dispatch(self.cfg, rank, W, kept_all, x, self.ids, self.row_of, self.offsets,
+                               peer.recv_ptrs, peer.rows, self.offsets_local, self.remote_row,
+                               self.ws_ep)
+
+    def peer_experts(self, peer, w_gate, w_up, w_down):
+        if not hasattr(self, "h_local"):
+            self.h_local = torch.empty((self.max_recv, w_gate.shape[2]), dtype=w_gate.dtype,
+                                       device=self.device)
+        B.moe_expert_ffn(self.cfg_local, peer.recv_x, self.offsets_local, None, None, w_gate, w_up,
+                         w_down, self.h_local, peer.y_loc, self.ws_local)
+
+    def peer_combine(self, x, W, peer):
+        y = torch.empty_like(x)
+        B.moe_ep_peer_combine(self.cfg, W, self.ids, self.remote_row, self.w, peer.out_ptrs,
+                              peer.rows, y, self.ws_ep)
+        return y
+
+
+class PeerBuffers:
+    """Every rank's receive buffer and expert-output buffer (rows x D elements
+    each), mapped into this process: this rank's own from moe_ipc_alloc, the
+    others' opened from the handles all ranks exchange at construction.
+    recv_ptrs / out_ptrs: int64 device tensors of the W addresses, indexed by
+    rank.  close() unmaps and frees them (collective: every rank calls it)."""
+
+    def __init__(self, rows: int, D: int, elem_bytes: int, group, device):
+        self.group = group
+        self.rows = int(rows)
+        W, rank = dist.get_world_size(group), dist.get_rank(group)
+        nbytes = self.rows * D * elem_bytes
+        self.recv_x, hx = B.ipc_alloc(nbytes)
+        self.y_loc, hy = B.ipc_alloc(nbytes)
+        handles = [None] * W
+        dist.all_gather_object(handles, (hx, hy), group=group)
+        self._opened = []
+        xs, ys = [], []
+        for r, (px_h, py_h) in enumerate(handles):
+            if r == rank:
+                xs.append(self.recv_x)
+                ys.append(self.y_loc)
+            else:
+                px, py = B.ipc_open(px_h), B.ipc_open(py_h)
+                self._opened += [px, py]
+                xs.append(px)
+                ys.append(py)
+        self.recv_ptrs = torch.tensor(xs, dtype=torch.int64, device=device)
+        self.out_ptrs = torch.tensor(ys, dtype=torch.int64, device=device)
+
+    def close(self):
+        if self.recv_x is None:
+            return
+        torch.cuda.synchronize()
+        dist.barrier(group=self.group)  # nobody reads a peer's buffer any more
+        for p in self._opened:
+            B.ipc_close(p)
+        self._opened = []
+        dist.barrier(group=self.group)  # every mapping of this rank's buffers is gone
+        B.ipc_free(self.recv_x)
+        B.ipc_free(self.y_loc)
+        self.recv_x = self.y_loc = None
+
 
 class ExpertParallelMoE:
     """One rank's share of an expert-parallel MoE layer.
@@ -110,7 +196,12 @@ class ExpertParallelMoE:
 
     def __init__(self, T: int, w_router, w_gate_local, w_up_local, w_down_local, E: int, K: int,
                  capacity_factor: float = 0.0, router_bias=None, selection_bias=None, group=None,
-                 ops=None, **router_options):
+                 ops=None, exchange: str = "all_to_all", **router_options):
+        if exchange not in ("all_to_all", "peer"):
+            raise ValueError("exchange is 'all_to_all' or 'peer'")
+        if exchange == "peer" and ops is not None:
+            raise ValueError("the peer exchange runs on the CUDA library's kernels only")
+        self.exchange = exchange
         self.group = group
         self.W = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -128,8 +219,37 @@ class ExpertParallelMoE:
             ops = CudaOps(T, self.D, self.F, E, K, self.EL, self.W, dtype, capacity_factor,
                           router_options, w_gate_local.device)
         self.ops = ops
+        self.peer = None
+        if exchange == "peer":
+            dev = w_gate_local.device
+            self.kept_all = torch.empty(self.W * E, dtype=torch.int32, device=dev)
+            self._sync = torch.zeros(1, dtype=torch.int32, device=dev)
+            self.peer = PeerBuffers(ops.max_recv, self.D, w_gate_local.element_size(), group, dev)
+
+    def close(self):
+        """Release the peer buffers (collective for the peer exchange)."""
+        if self.peer is not None:
+            self.peer.close()
+            self.peer = None
+
+    def _barrier(self):
+        # stream-ordered: the next kernel on this stream starts after every
+        # rank's kernels before its own all-reduce have finished
+        dist.all_reduce(self._sync, group=self.group)
+
+    def _forward_peer(self, x, logit_noise):
+        ops = self.ops
+        kept = ops.route_index(x, self.w_router, self.router_bias, self.selection_bias, logit_noise)
+        dist.all_gather_into_tensor(self.kept_all, kept, group=self.group)
+        ops.peer_dispatch(x, self.kept_all, self.rank, self.W, self.peer)
+        self._barrier()  # every rank's rows are in their owners' buffers
+        ops.peer_experts(self.peer, self.w_gate, self.w_up, self.w_down)
+        self._barrier()  # every owner's results are ready
+        return ops.peer_combine(x, self.W, self.peer)
 
     def forward(self, x, logit_noise=None):
+        if self.exchange == "peer":
+            return self._forward_peer(x, logit_noise)
         W, EL = self.W, self.EL
         ops = self.ops
         # route this rank's tokens and sort their rows by expert (so by owner)

@@ -241,3 +241,42 @@ def test_expert_parallel_argument_errors(lib):
     c = _cfg()
     assert lib.moe_combine_weighted(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, None) == B.MOE_ERR_ARG
     assert lib.moe_combine_weighted(ctypes.byref(c), FAKE, FAKE, FAKE, None, FAKE + 8, None) == B.MOE_ERR_ALIGN
+
+
+def test_peer_exchange_argument_errors(lib):
+    """Host-side checks of the peer-memory exchange, all before any launch."""
+    c = _cfg()  # E = 8
+    need = B.ep_workspace_size(2, c.E // 2)
+    disp = lambda **kw: lib.moe_ep_peer_dispatch(  # noqa: E731
+        ctypes.byref(kw.get("cfg", c)), kw.get("rank", 0), kw.get("W", 2), kw.get("kept_all", FAKE),
+        kw.get("x", FAKE), FAKE, FAKE, FAKE, kw.get("bufs", FAKE), kw.get("rows", 64), FAKE,
+        kw.get("remote", FAKE), kw.get("ws", FAKE), kw.get("nb", need), None)
+    assert disp(W=3) == B.MOE_ERR_ARG            # 8 experts do not divide among 3 ranks
+    assert disp(W=0) == B.MOE_ERR_ARG
+    assert disp(W=128) == B.MOE_ERR_ARG          # more ranks than the kernels' table
+    assert disp(rank=2) == B.MOE_ERR_ARG
+    assert disp(rank=-1) == B.MOE_ERR_ARG
+    assert disp(kept_all=None) == B.MOE_ERR_ARG
+    assert disp(bufs=None) == B.MOE_ERR_ARG
+    assert disp(remote=None) == B.MOE_ERR_ARG
+    assert disp(rows=0) == B.MOE_ERR_SHAPE
+    assert disp(nb=need - 1) == B.MOE_ERR_WORKSPACE
+    assert disp(x=FAKE + 8) == B.MOE_ERR_ALIGN
+    comb = lambda **kw: lib.moe_ep_peer_combine(  # noqa: E731
+        ctypes.byref(c), kw.get("W", 2), FAKE, FAKE, kw.get("w", FAKE), kw.get("bufs", FAKE),
+        kw.get("rows", 64), kw.get("add", None), kw.get("y", FAKE), FAKE, need, None)
+    assert comb(W=3) == B.MOE_ERR_ARG
+    assert comb(w=None) == B.MOE_ERR_ARG
+    assert comb(bufs=None) == B.MOE_ERR_ARG
+    assert comb(y=FAKE + 8) == B.MOE_ERR_ALIGN
+    assert comb(add=FAKE + 4) == B.MOE_ERR_ALIGN
+    assert comb(rows=-5) == B.MOE_ERR_SHAPE
+    # the IPC entry points refuse null arguments without touching CUDA
+    p = ctypes.c_void_p()
+    h = ctypes.create_string_buffer(B.IPC_HANDLE_BYTES)
+    assert lib.moe_ipc_alloc(0, ctypes.byref(p), h) == B.MOE_ERR_ARG
+    assert lib.moe_ipc_alloc(64, None, h) == B.MOE_ERR_ARG
+    assert lib.moe_ipc_open(None, ctypes.byref(p)) == B.MOE_ERR_ARG
+    assert lib.moe_ipc_open(h, None) == B.MOE_ERR_ARG
+    assert lib.moe_ipc_close(None) == B.MOE_OK
+    assert lib.moe_ipc_free(None) == B.MOE_OK

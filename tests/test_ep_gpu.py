@@ -21,7 +21,7 @@ import torch.distributed as dist
 import oracle
 from mixture_experts_layer_55_b200 import _binding as B
 from mixture_experts_layer_55_b200.ep import ExpertParallelMoE
-from workloads import Workload, make_inputs
+from workloads import Workload, make_inputs, make_tokens
 
 from tests.test_ep_cpu import receive_layout
 from tests.gpu_common import to_np
@@ -107,3 +107,203 @@ def test_expert_parallel_one_rank(wl):
         assert np.abs(got - to_np(yt)).max() <= 1e-2 * m * 0.1 + 1e-4
     finally:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------ exchange over peer memory --
+
+def _expected_remote_rows(kept_all, ids, row_of, offsets, rank, W, EL):
+    """Where each slot of source `rank` lands in its owner's buffer, from the
+    all-to-all path's definition: the rows for owner o leave in expert-major
+    order, arrive after the rows of sources < rank, and the owner's receive
+    layout moves arrival position p to expert-major row dst_of[p]."""
+    E = W * EL
+    K = ids.shape[1]
+    out = np.full(ids.shape[0] * K, -1, np.int64)
+    layouts = [receive_layout(kept_all[:, o * EL:(o + 1) * EL], W, EL) for o in range(W)]
+    for t in range(ids.shape[0]):
+        for k in range(K):
+            r = row_of[t * K + k]
+            if r < 0:
+                continue
+            o = ids[t, k] // EL
+            recv_o = kept_all[:, o * EL:(o + 1) * EL]
+            arrival = int(recv_o[:rank].sum()) + (r - offsets[o * EL])
+            out[t * K + k] = layouts[o][1][arrival]
+    return out, [lay[0] for lay in layouts]
+
+
+def _emulated_peer_layer(wl, W, bias=None, token_seed=77):
+    """W ranks of the peer-exchange layer emulated on one GPU: each rank has its
+    own tokens; every rank's receive and output buffers live on this device,
+    so the kernels' stores into and loads from "peer" buffers are ordinary
+    device accesses.  The ranks' kernels run one after another in stream
+    order; none waits on another."""
+    dev = "cuda"
+    inp = make_inputs(wl)
+    if bias is not None:
+        inp["bias"] = bias
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    E, K, T, D, F = wl.E, wl.K, wl.T, wl.D, wl.F
+    EL = E // W
+    cfg = B.MoeConfig.make(T, D, F, E, K, wl.dtype, wl.capacity_factor)
+    max_recv = W * T * K
+    cfg_local = B.MoeConfig.make(max_recv, D, F, EL, 1, wl.dtype, 0.0)
+    i32 = dict(dtype=torch.int32, device=dev)
+    ranks = []
+    for r in range(W):
+        x = make_tokens(wl, device="cpu", seed=token_seed * 16 + r)
+        st = dict(x_cpu=x, x=x.to(dev), ids=torch.empty(T, K, **i32),
+                  w=torch.empty(T, K, dtype=torch.float32, device=dev),
+                  counts=torch.empty(E, **i32), kept=torch.empty(E, **i32),
+                  offsets=torch.empty(E + 1, **i32), perm=torch.empty(B.max_rows(cfg), **i32),
+                  row_of=torch.empty(T * K, **i32), L=torch.empty(T, E, device=dev),
+                  ws=torch.zeros(B.workspace_size(cfg), dtype=torch.uint8, device=dev),
+                  ws_ep=torch.zeros(B.ep_workspace_size(W, EL), dtype=torch.uint8, device=dev),
+                  local_offsets=torch.full((EL + 1,), -7, **i32),
+                  remote_row=torch.full((T * K,), -7, **i32))
+        B.moe_route(cfg, st["x"], g["w_router"], st["ids"], st["w"], st["ws"], router_bias=g["bias"],
+                    logits_out=st["L"])
+        B.moe_dispatch(cfg, None, st["ids"], st["counts"], st["kept"], st["offsets"], st["perm"],
+                       st["row_of"], None, st["ws"])
+        ranks.append(st)
+    kept_all = torch.stack([st["kept"] for st in ranks]).reshape(-1).contiguous()
+    recv = [torch.zeros(max_recv, D, dtype=wl.torch_dtype, device=dev) for _ in range(W)]
+    outs = [torch.zeros(max_recv, D, dtype=wl.torch_dtype, device=dev) for _ in range(W)]
+    recv_ptrs = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device=dev)
+    out_ptrs = torch.tensor([t.data_ptr() for t in outs], dtype=torch.int64, device=dev)
+    for r, st in enumerate(ranks):
+        B.moe_ep_peer_dispatch(cfg, r, W, kept_all, st["x"], st["ids"], st["row_of"], st["offsets"],
+                               recv_ptrs, max_recv, st["local_offsets"], st["remote_row"], st["ws_ep"])
+    ws_local = torch.zeros(B.workspace_size(cfg_local), dtype=torch.uint8, device=dev)
+    h = torch.empty(max_recv, F, dtype=wl.torch_dtype, device=dev)
+    for o, st in enumerate(ranks):
+        sl = slice(o * EL, (o + 1) * EL)
+        B.moe_expert_ffn(cfg_local, recv[o], st["local_offsets"], None, None, g["w_gate"][sl],
+                         g["w_up"][sl], g["w_down"][sl], h, outs[o], ws_local)
+    for st in ranks:
+        st["y"] = torch.empty_like(st["x"])
+        B.moe_ep_peer_combine(cfg, W, st["ids"], st["remote_row"], st["w"], out_ptrs, max_recv, st["y"],
+                              st["ws_ep"])
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert B.moe_get_device_status(st["ws"]) == 0
+        assert B.moe_get_device_status(st["ws_ep"]) == 0
+    assert B.moe_get_device_status(ws_local) == 0
+    return cfg, inp, g, ranks, kept_all.view(W, E).cpu().numpy()
+
+
+PEER_CASES = {
+    "w2": (2, Workload("peer_w2", T=320, D=256, F=384, E=8, K=2), None),
+    "w4_drops": (4, Workload("peer_w4_drops", T=256, D=256, F=256, E=8, K=2, capacity_factor=0.5,
+                             bias="zipf"), None),
+    "w8_one_expert_per_rank": (8, Workload("peer_w8", T=192, D=256, F=256, E=8, K=1), None),
+    "w4_k4": (4, Workload("peer_w4_k4", T=160, D=256, F=256, E=16, K=4), None),
+    "w2_k6": (2, Workload("peer_w2_k6", T=136, D=256, F=256, E=16, K=6), None),
+    # every token prefers the last rank's experts: the other owners receive little or nothing
+    "w4_skewed": (4, Workload("peer_w4_skew", T=192, D=256, F=256, E=8, K=2), "last_rank"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PEER_CASES))
+def test_peer_exchange_emulated_ranks(name):
+    W, wl, skew = PEER_CASES[name]
+    bias = None
+    if skew == "last_rank":
+        bias = torch.zeros(wl.E)
+        bias[-(wl.E // W):] = 8.0
+    cfg, inp, g, ranks, kept_all = _emulated_peer_layer(wl, W, bias=bias)
+    EL = wl.E // W
+    for r, st in enumerate(ranks):
+        ids = st["ids"].cpu().numpy()
+        row_of = st["row_of"].cpu().numpy()
+        offsets = st["offsets"].cpu().numpy()
+        exp_rows, exp_offsets = _expected_remote_rows(kept_all, ids, row_of, offsets, r, W, EL)
+        np.testing.assert_array_equal(st["remote_row"].cpu().numpy(), exp_rows)
+        np.testing.assert_array_equal(st["local_offsets"].cpu().numpy(), exp_offsets[r])
+        # the output against the oracle's local layer on this rank's tokens
+        ref = oracle.forward(st["x_cpu"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                             wl.K, wl.capacity_factor, bias=inp["bias"], logits=st["L"].cpu().numpy())
+        assert np.array_equal(ids, ref["ids"])
+        assert np.array_equal(row_of, ref["row_of"])
+        got = to_np(st["y"])
+        m = float(np.abs(ref["y"]).max())
+        assert np.abs(got - ref["y"]).max() <= 1e-2 * m + 1e-3
+        # and against the local training forward (the same weighted combine)
+        state = torch.zeros(B.train_state_size(cfg), dtype=torch.uint8, device="cuda")
+        yt = torch.empty_like(st["x"])
+        B.moe_forward_train(cfg, st["x"], g["w_router"], g["w_gate"], g["w_up"], g["w_down"], yt, state,
+                            router_bias=g["bias"])
+        torch.cuda.synchronize()
+        assert np.abs(got - to_np(yt)).max() <= 1e-3 * m + 1e-4
+    if name == "w4_drops":
+        assert any((st["row_of"] < 0).any().item() for st in ranks), "case must drop assignments"
+    if name == "w4_skewed":
+        assert kept_all[:, : wl.E - EL].sum() == 0, "every row must go to the last rank"
+
+
+@pytest.mark.parametrize("wl", [
+    Workload("peer_w1", T=640, D=256, F=384, E=8, K=2),
+    Workload("peer_w1_drops", T=512, D=256, F=256, E=8, K=2, capacity_factor=0.5, bias="zipf"),
+], ids=lambda w: w.name)
+def test_peer_exchange_one_rank(wl):
+    """The layer object with exchange='peer' at world size 1 over NCCL: the
+    same output as the all-to-all exchange, twice in a row (the barriers and
+    buffer reuse between steps), then the buffers released."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        inp = make_inputs(wl)
+        g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        args = (wl.T, g["w_router"], g["w_gate"], g["w_up"], g["w_down"], wl.E, wl.K, wl.capacity_factor)
+        peer = ExpertParallelMoE(*args, router_bias=g["bias"], exchange="peer")
+        a2a = ExpertParallelMoE(*args, router_bias=g["bias"])
+        for seed in (3, 4):
+            x = make_tokens(wl, device="cuda", seed=seed)
+            y_peer = peer.forward(x)
+            y_a2a = a2a.forward(x)
+            torch.cuda.synchronize()
+            assert peer.ops.status() == 0 and a2a.ops.status() == 0
+            m = float(y_a2a.float().abs().max())
+            assert float((y_peer.float() - y_a2a.float()).abs().max()) <= 1e-3 * m + 1e-4
+        peer.close()
+    finally:
+        dist.destroy_process_group()
+
+
+def _ipc_child(handle, n, q):
+    try:
+        torch.cuda.set_device(0)
+        from mixture_experts_layer_55_b200 import _binding as Bc
+        ptr = Bc.ipc_open(handle)
+        v = Bc.as_tensor(ptr, (n,), torch.int32)
+        seen = bool(torch.equal(v.cpu(), torch.arange(n, dtype=torch.int32)))
+        v.copy_(torch.arange(n, dtype=torch.int32, device="cuda") * 3)
+        torch.cuda.synchronize()
+        Bc.ipc_close(ptr)
+        q.put((seen, None))
+    except Exception as exc:  # pragma: no cover - reported by the parent
+        q.put((False, repr(exc)))
+
+
+def test_ipc_buffer_between_processes():
+    """A buffer from moe_ipc_alloc, opened by another process from its handle
+    (same GPU, one after the other: nothing waits on the other process)."""
+    import torch.multiprocessing as mp
+    n = 4096
+    ptr, handle = B.ipc_alloc(n * 4)
+    try:
+        t = B.as_tensor(ptr, (n,), torch.int32)
+        t.copy_(torch.arange(n, dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        ctx = mp.get_context("spawn")
+        q = ctx.Queue()
+        p = ctx.Process(target=_ipc_child, args=(handle, n, q))
+        p.start()
+        seen, exc = q.get(timeout=240)
+        p.join(timeout=60)
+        assert exc is None, exc
+        assert seen, "the other process read different values"
+        assert torch.equal(t.cpu(), torch.arange(n, dtype=torch.int32) * 3)
+    finally:
+        B.ipc_free(ptr)
