@@ -390,8 +390,6 @@ def run_gpu_train(args):
     dev = torch.device("cuda", local_rank)
     init_dist(world, "nccl")
     wl = workload_of(args)
-    if wl.dtype != "bf16":
-        raise SystemExit("--pass train needs a bf16 workload")
     inp = make_inputs(wl, device=dev)
     layer = M.MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
                        wl.capacity_factor, router_bias=inp["bias"])
@@ -502,8 +500,17 @@ def run_gpu_train(args):
     top = max(nbytes, key=lambda k: stage_ms[k])
     t_top = stage_ms[top] / 1e3
     intensity = flop[top] / nbytes[top]
+    if wl.dtype == "f32":
+        # fp32 layer: SIMT FMA pipes (148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock)
+        peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        key = "fp32 FMA"
     ridge = peak * 1e12 / (hbm_peak * 1e9)
-    if intensity >= ridge:
+    if wl.dtype == "f32":
+        achieved = flop[top] / t_top / 1e12
+        roofline = {"kernel": top, "bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 1),
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_source": "148 SMs x 128 FMA x 2 x max clock"}
+    elif intensity >= ridge:
         achieved = flop[top] / t_top / 1e12
         roofline = {"kernel": top, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),

@@ -281,7 +281,8 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
  * it).  The stop-gradients, as autograd applies them to the forward: the chosen
  * ids (with the group limit and the selection bias), the capacity keep mask
  * and the balance loss's counts f_e.  Logit noise is an input.  bf16 layers
- * only (MOE_ERR_UNSUPPORTED for MOE_F32).
+ * run the backward's GEMMs on the tensor cores; fp32 layers in true fp32 on
+ * the SIMT pipes (no TF32).
  */
 
 /*
@@ -295,8 +296,8 @@ MOE_API moe_status moe_train_state_size(const moe_config *cfg, size_t *bytes);
  * moe_forward for training: the same arguments and results, with the
  * workspace replaced by `state` (moe_train_state_size bytes, 256-byte
  * aligned), which keeps what moe_backward reads: the routing results, the
- * dispatch layout, x_perm, [g | u] = the gate/up pre-activations rounded to
- * bf16, h, the unweighted expert outputs and the logits.  The state must not
+ * dispatch layout, x_perm, [g | u] = the gate/up pre-activations in the
+ * layer dtype, h, the unweighted expert outputs and the logits.  The state must not
  * be written between this call and moe_backward.  y equals moe_forward's up
  * to rounding order: the routing weight multiplies each expert output in the
  * combine (fp32) instead of in the down projection's epilogue.
@@ -316,7 +317,7 @@ MOE_API moe_status moe_backward_workspace_size(const moe_config *cfg, size_t *by
 /*
  * Gradients of  loss = sum_{t,d} dy[t,d] * y[t,d] + c_balance * balance + c_z * z
  * for the forward recorded in `state` by moe_forward_train (pass the same x
- * and weights).  dy (T, D) bf16 is the upstream gradient of y; c_balance and
+ * and weights).  dy (T, D) in the layer dtype is the upstream gradient of y; c_balance and
  * c_z are the loss coefficients (the lab's 0.01 and 0.001), host values.
  *
  *   gate weights  dw[t,k] = <dy[t], o_k(x_t)> for a kept slot, 0 for a dropped
@@ -328,12 +329,13 @@ MOE_API moe_status moe_backward_workspace_size(const moe_config *cfg, size_t *by
  *                 expert's rows
  *   input         dx = dL W_r^T + sum over kept slots of dx_e (+ shared expert)
  *
- * Outputs, all overwritten: dx (T, D) bf16; dw_router (D, E) fp32;
+ * Outputs, all overwritten: dx (T, D) in the layer dtype; dw_router (D, E) fp32;
  * db_router (E) fp32 or NULL; dw_gate, dw_up (E, D, F) fp32; dw_down
  * (E, F, D) fp32; with a shared expert dw_gate_shared, dw_up_shared
  * (D, F_shared) and dw_down_shared (F_shared, D) fp32 (ignored otherwise).
- * Rounding: dy * w, [dg | du] and each expert's dx rows are rounded to bf16
- * before the next contraction; every sum is fp32.  Deterministic.
+ * Rounding (bf16 layers): dy * w, [dg | du] and each expert's dx rows are
+ * rounded to bf16 before the next contraction; every sum is fp32 (fp32 layers
+ * keep every value in fp32).  Deterministic.
  * workspace: moe_backward_workspace_size bytes, 256-byte aligned; device
  * faults are reported in its status word (moe_get_device_status(workspace)).
  */

@@ -12,7 +12,7 @@ namespace moe {
 cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const void* x_perm,
                                 const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                 const void* w_gate, const void* w_up, const void* w_down, void* h,
-                                void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                                void* y_perm, void* gu_keep, int* status, cudaStream_t s, StageHook mid,
                                 void* mid_ctx);
 cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
@@ -207,13 +207,32 @@ cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void*
                               void* y_perm, void* gu_keep, int* status, cudaStream_t s,
                               StageHook mid, void* mid_ctx)
 {
-    if (c.dtype == MOE_F32) {
-        if (gu_keep != nullptr) return cudaErrorNotSupported;
+    if (c.dtype == MOE_F32)
         return launch_ffn_simt_f32(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up,
-                                   w_down, h, y_perm, status, s, mid, mid_ctx);
-    }
+                                   w_down, h, y_perm, gu_keep, status, s, mid, mid_ctx);
     return launch_ffn_tc_bf16(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h,
                               y_perm, gu_keep, status, s, mid, mid_ctx);
+}
+
+// the backward's GEMMs in the layer's dtype: tensor cores for bf16, fp32 SIMT for fp32
+static cudaError_t launch_dgrad(const moe_config& c, int64_t max_rows, const void* dyp, const int32_t* offsets,
+                                const void* gu, const void* w_gate, const void* w_up, const void* w_down,
+                                void* dgu, void* dxp, int* status, cudaStream_t s, StageHook mid, void* mid_ctx)
+{
+    if (c.dtype == MOE_F32)
+        return launch_dgrad_simt_f32(c, max_rows, dyp, offsets, gu, w_gate, w_up, w_down, dgu, dxp, status, s,
+                                     mid, mid_ctx);
+    return launch_dgrad_tc_bf16(c, max_rows, dyp, offsets, gu, w_gate, w_up, w_down, dgu, dxp, status, s, mid,
+                                mid_ctx);
+}
+
+static cudaError_t launch_wgrad(int32_t dt, int E, int64_t max_rows, const int32_t* offsets, const void* a,
+                                int M, const void* b, int N, int halves, float* out0, float* out1, int* status,
+                                cudaStream_t s)
+{
+    if (dt == MOE_F32)
+        return launch_wgrad_simt_f32(E, max_rows, offsets, a, M, b, N, halves, out0, out1, status, s);
+    return launch_wgrad_tc_bf16(E, max_rows, offsets, a, M, b, N, halves, out0, out1, status, s);
 }
 
 // the shared expert as a layer of one expert over every token
@@ -494,8 +513,7 @@ moe_status moe_train_state_size(const moe_config* cfg, size_t* bytes)
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (bytes == nullptr) return MOE_ERR_ARG;
-    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    *bytes = train_layout(*cfg, max_rows_of(*cfg)).total;
+        *bytes = train_layout(*cfg, max_rows_of(*cfg)).total;
     return MOE_OK;
 }
 
@@ -510,8 +528,7 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const float* 
     moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
                                        w_up_shared, w_down_shared, y);
     if (st != MOE_OK) return st;
-    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    const TrainLayout TL = train_layout(*cfg, max_rows_of(*cfg));
+        const TrainLayout TL = train_layout(*cfg, max_rows_of(*cfg));
     st = check_ws(cfg, state, state_bytes, TL.total);
     if (st != MOE_OK) return st;
     return cuda_status(run_forward(*cfg, x, w_router, router_bias, selection_bias, logit_noise,
@@ -526,8 +543,7 @@ moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes)
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (bytes == nullptr) return MOE_ERR_ARG;
-    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    *bytes = bwd_layout(*cfg, max_rows_of(*cfg)).total;
+        *bytes = bwd_layout(*cfg, max_rows_of(*cfg)).total;
     return MOE_OK;
 }
 
@@ -543,8 +559,7 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
     moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
                                        w_up_shared, w_down_shared, dx);
     if (st != MOE_OK) return st;
-    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    if (!dy || !dw_router || !dw_gate || !dw_up || !dw_down) return MOE_ERR_ARG;
+        if (!dy || !dw_router || !dw_gate || !dw_up || !dw_down) return MOE_ERR_ARG;
     if (!aligned16(dy) || !aligned16(dw_gate) || !aligned16(dw_up) || !aligned16(dw_down))
         return MOE_ERR_ALIGN;
     if (cfg->F_shared > 0) {
@@ -585,29 +600,29 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
                               max_rows, status, s);
     btrace(2, s);
     if (e == cudaSuccess)  // dH -> [dg | du], then dXp (boundary 3 between the two)
-        e = launch_dgrad_tc_bf16(c, max_rows, ws + B.dyp, offsets, sv + TL.gu, w_gate, w_up, w_down,
+        e = launch_dgrad(c, max_rows, ws + B.dyp, offsets, sv + TL.gu, w_gate, w_up, w_down,
                                  ws + B.dgu, ws + B.dxp, status, s, btrace_mid_dgrad, nullptr);
     btrace(4, s);
     if (e == cudaSuccess)  // dWd = h^T dYp
-        e = launch_wgrad_tc_bf16(c.E, max_rows, offsets, sv + F.h, c.F, ws + B.dyp, c.D, 1, dw_down,
+        e = launch_wgrad(c.dtype, c.E, max_rows, offsets, sv + F.h, c.F, ws + B.dyp, c.D, 1, dw_down,
                                  nullptr, status, s);
     btrace(5, s);
     if (e == cudaSuccess)  // [dWg | dWu] = x_perm^T [dg | du]
-        e = launch_wgrad_tc_bf16(c.E, max_rows, offsets, sv + F.x_perm, c.D, ws + B.dgu, c.F, 2,
+        e = launch_wgrad(c.dtype, c.E, max_rows, offsets, sv + F.x_perm, c.D, ws + B.dgu, c.F, 2,
                                  dw_gate, dw_up, status, s);
     btrace(6, s);
     const void* dx_shared = nullptr;
     if (e == cudaSuccess && c.F_shared > 0) {
         const moe_config cs = shared_config(c);
         const int32_t* sh_off = reinterpret_cast<const int32_t*>(sv + F.sh_offsets);
-        e = launch_dgrad_tc_bf16(cs, c.T, dy, sh_off, sv + TL.sh_gu, w_gate_shared, w_up_shared,
+        e = launch_dgrad(cs, c.T, dy, sh_off, sv + TL.sh_gu, w_gate_shared, w_up_shared,
                                  w_down_shared, ws + B.sh_dgu, ws + B.sh_dx, status, s, nullptr,
                                  nullptr);
         if (e == cudaSuccess)
-            e = launch_wgrad_tc_bf16(1, c.T, sh_off, sv + F.sh_h, c.F_shared, dy, c.D, 1,
+            e = launch_wgrad(c.dtype, 1, c.T, sh_off, sv + F.sh_h, c.F_shared, dy, c.D, 1,
                                      dw_down_shared, nullptr, status, s);
         if (e == cudaSuccess)
-            e = launch_wgrad_tc_bf16(1, c.T, sh_off, x, c.D, ws + B.sh_dgu, c.F_shared, 2,
+            e = launch_wgrad(c.dtype, 1, c.T, sh_off, x, c.D, ws + B.sh_dgu, c.F_shared, 2,
                                      dw_gate_shared, dw_up_shared, status, s);
         dx_shared = ws + B.sh_dx;
     }
@@ -803,7 +818,7 @@ moe_status moe_ep_peer_combine(const moe_config* cfg, int32_t world, const int32
 
 int32_t moe_backward_kernel_count(const moe_config* cfg)
 {
-    if (check_config(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;
+    if (check_config(cfg) != MOE_OK) return 0;
     // rows, router, two dgrad GEMMs, two wgrad GEMMs, router weight partials,
     // their sum, the bias gradient, dx; the shared expert adds its two dgrad
     // and two wgrad GEMMs

@@ -6,7 +6,7 @@
 // top-k index decision is a stop-gradient, so the router learns only through
 // the kept gate weights and the auxiliary losses.  With dY the gradient of y:
 //
-//   rows       dYp[r] = bf16(w_r * dY[t_r]),  dw_r = <dY[t_r], o_r>
+//   rows       dYp[r] = w_r * dY[t_r] (in the layer dtype),  dw_r = <dY[t_r], o_r>
 //              (o_r = the expert's unweighted output the forward kept)
 //   router     dL[t] from the gate weights' dw (renormalised or not, route
 //              scale), the balance loss through the normalised scores (counts
@@ -22,7 +22,9 @@
 namespace moe {
 
 // ------------------------------------------------------------------- rows --
-// One warp per row of the expert-major layout; 16-byte vectors of 8 bf16.
+// One warp per row of the expert-major layout; 16-byte vectors (8 bf16 or 4
+// fp32 elements).
+template <typename ET>
 __global__ void __launch_bounds__(256) bwd_rows_kernel(const uint4* __restrict__ dy,
                                                        const uint4* __restrict__ o,
                                                        const int32_t* __restrict__ offsets,
@@ -55,13 +57,22 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const uint4* __restrict__
             const uint4 a = __ldg(dyt + v), b = __ldg(orow + v);
             const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
             uint32_t pw[4];
+            if constexpr (sizeof(ET) == 2) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float a0 = __uint_as_float(aw[i] << 16), a1 = __uint_as_float(aw[i] & 0xffff0000u);
-                const float b0 = __uint_as_float(bw[i] << 16), b1 = __uint_as_float(bw[i] & 0xffff0000u);
-                dot = fmaf(a0, b0, dot);
-                dot = fmaf(a1, b1, dot);
-                pw[i] = pack_bf16x2(w * a0, w * a1);
+                for (int i = 0; i < 4; ++i) {
+                    const float a0 = __uint_as_float(aw[i] << 16), a1 = __uint_as_float(aw[i] & 0xffff0000u);
+                    const float b0 = __uint_as_float(bw[i] << 16), b1 = __uint_as_float(bw[i] & 0xffff0000u);
+                    dot = fmaf(a0, b0, dot);
+                    dot = fmaf(a1, b1, dot);
+                    pw[i] = pack_bf16x2(w * a0, w * a1);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float a0 = __uint_as_float(aw[i]), b0 = __uint_as_float(bw[i]);
+                    dot = fmaf(a0, b0, dot);
+                    pw[i] = __float_as_uint(w * a0);
+                }
             }
             drow[v] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
@@ -439,14 +450,21 @@ cudaError_t launch_bwd_rows(const moe_config& c, const void* dy, const void* o, 
                             const int32_t* perm, const float* topk_w, void* dyp, float* dw_row,
                             int64_t max_rows, int* status, cudaStream_t s)
 {
-    const int64_t vpr = (int64_t)c.D * 2 / 16;  // bf16 rows
+    const int64_t vpr = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
     int64_t blocks = (max_rows + 7) / 8;
     const int64_t cap = (int64_t)sm_count() * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    bwd_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(
-        static_cast<const uint4*>(dy), static_cast<const uint4*>(o), offsets, perm, topk_w,
-        static_cast<uint4*>(dyp), dw_row, c.E, c.K, vpr, c.T * c.K, max_rows, status);
+    const uint4* dyv = static_cast<const uint4*>(dy);
+    const uint4* ov = static_cast<const uint4*>(o);
+    if (c.dtype == MOE_BF16)
+        bwd_rows_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            dyv, ov, offsets, perm, topk_w, static_cast<uint4*>(dyp), dw_row, c.E, c.K, vpr, c.T * c.K,
+            max_rows, status);
+    else
+        bwd_rows_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(
+            dyv, ov, offsets, perm, topk_w, static_cast<uint4*>(dyp), dw_row, c.E, c.K, vpr, c.T * c.K,
+            max_rows, status);
     return cudaGetLastError();
 }
 

@@ -5,6 +5,7 @@
 // (SwiGLUExpert: down(silu(gate x) * up x); each expert output scaled by its
 // combine weight).  Two launches over each expert's contiguous row block:
 //   gate/up: h = silu(x_perm Wg_e) * (x_perm Wu_e)         (rows x F)
+//            (the training forward also keeps [g | u], rows x 2F)
 //   down:    y_perm = topk_w[perm[row]] * (h Wd_e)         (rows x D)
 // Tiles are 64 rows x 64 columns; the m-tile -> (expert, first row) map is
 // derived on the device from the offsets (no host synchronisation).
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A,
                                                        const int32_t* __restrict__ perm,
                                                        const float* __restrict__ topk_w, int E,
                                                        int Kd, int N, int64_t max_rows, int64_t nk,
-                                                       int* status)
+                                                       T* __restrict__ gu_keep, int* status)
 {
     __shared__ int s_off[257];
     __shared__ int s_pref[257];
@@ -130,6 +131,10 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A,
             if (col >= N) continue;
             float v = GATEUP ? silu_f32(acc0[i][j]) * acc1[i][j] : wr * acc0[i][j];
             out[row * N + col] = from_f32<T>(v);
+            if (GATEUP && gu_keep != nullptr) {  // [g | u] for the backward
+                gu_keep[row * 2 * N + col] = from_f32<T>(acc0[i][j]);
+                gu_keep[row * 2 * N + N + col] = from_f32<T>(acc1[i][j]);
+            }
         }
     }
 }
@@ -144,7 +149,7 @@ template <typename T>
 static cudaError_t launch_simt(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                const void* w_gate, const void* w_up, const void* w_down, void* h,
-                               void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                               void* y_perm, void* gu_keep, int* status, cudaStream_t s, StageHook mid,
                                void* mid_ctx)
 {
     const int64_t mtiles = simt_mtiles_bound(max_rows, c.E);
@@ -152,23 +157,24 @@ static cudaError_t launch_simt(const moe_config& c, int64_t max_rows, const void
     dim3 g1((c.F + kSBN - 1) / kSBN, (unsigned)mtiles);
     ffn_simt_kernel<T, true><<<g1, 256, 0, s>>>(
         static_cast<const T*>(x_perm), static_cast<const T*>(w_gate), static_cast<const T*>(w_up),
-        static_cast<T*>(h), offsets, perm, topk_w, c.E, c.D, c.F, max_rows, nk, status);
+        static_cast<T*>(h), offsets, perm, topk_w, c.E, c.D, c.F, max_rows, nk, static_cast<T*>(gu_keep),
+        status);
     if (mid) mid(mid_ctx, s);
     dim3 g2((c.D + kSBN - 1) / kSBN, (unsigned)mtiles);
     ffn_simt_kernel<T, false><<<g2, 256, 0, s>>>(
         static_cast<const T*>(h), static_cast<const T*>(w_down), nullptr, static_cast<T*>(y_perm),
-        offsets, perm, topk_w, c.E, c.F, c.D, max_rows, nk, status);
+        offsets, perm, topk_w, c.E, c.F, c.D, max_rows, nk, nullptr, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const void* x_perm,
                                 const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                 const void* w_gate, const void* w_up, const void* w_down, void* h,
-                                void* y_perm, int* status, cudaStream_t s, StageHook mid,
+                                void* y_perm, void* gu_keep, int* status, cudaStream_t s, StageHook mid,
                                 void* mid_ctx)
 {
     return launch_simt<float>(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h,
-                              y_perm, status, s, mid, mid_ctx);
+                              y_perm, gu_keep, status, s, mid, mid_ctx);
 }
 
 }  // namespace moe

@@ -178,6 +178,12 @@ cudaError_t launch_router_wgrad(const moe_config& c, const void* x, const float*
 cudaError_t launch_ep_layout(const int32_t* recv, int W, int EL, int64_t max_rows, int32_t* offsets,
                              int32_t* seg_src, int32_t* seg_dst, int32_t* dst_of, int32_t* src_of,
                              int* status, cudaStream_t s);
+cudaError_t launch_dgrad_simt_f32(const moe_config& c, int64_t max_rows, const void* dyp, const int32_t* offsets,
+                                  const void* gu, const void* w_gate, const void* w_up, const void* w_down,
+                                  void* dgu, void* dxp, int* status, cudaStream_t s, StageHook mid, void* mid_ctx);
+cudaError_t launch_wgrad_simt_f32(int E, int64_t max_rows, const int32_t* offsets, const void* a, int M,
+                                  const void* b, int N, int halves, float* out0, float* out1, int* status,
+                                  cudaStream_t s);
 cudaError_t launch_peer_dispatch(const moe_config& c, int rank, int W, const int32_t* kept_all, const void* x,
                                  const int32_t* ids, const int32_t* row_of, const int32_t* offsets,
                                  void* const* recv_bufs, int64_t recv_rows, int64_t max_rows,

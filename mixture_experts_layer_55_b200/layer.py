@@ -13,7 +13,7 @@ from . import _binding as B
 
 
 class MoELayer:
-    """Token-choice top-k MoE layer (forward, and the backward of bf16 layers)
+    """Token-choice top-k MoE layer (forward and backward)
     on one CUDA device.
 
     weights: w_router (D, E) fp32; w_gate, w_up (E, D, F); w_down (E, F, D) in
@@ -122,8 +122,8 @@ class MoELayer:
 
     # ----------------------------------------------------------- training
     def forward_train(self, x, y=None, logit_noise=None, stream=None):
-        """forward() that keeps the activations moe_backward reads (bf16
-        layers); the state buffer is allocated on first use."""
+        """forward() that keeps the activations moe_backward reads; the state
+        buffer is allocated on first use."""
         if getattr(self, "state", None) is None:
             self.state = torch.zeros(B.train_state_size(self.cfg), dtype=torch.uint8,
                                      device=self.device)

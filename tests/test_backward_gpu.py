@@ -8,7 +8,8 @@ the CUDA path's own fp32 logits (as the forward's parity tests do), so the
 discrete decisions agree and every gradient is compared element by element.
 
 Tolerance, per gradient tensor G (bf16 path): |gpu - oracle| <= 2e-2 * max|oracle|
-per element and ||gpu - oracle|| <= 1e-2 * ||oracle|| as a whole.  The CUDA path
+per element and ||gpu - oracle|| <= 1e-2 * ||oracle|| as a whole; fp32 layers:
+1e-4 * max|oracle| per element and 1e-5 normwise.  The CUDA path
 rounds five intermediates to bf16 on the way to dx (the expert output o for
 dw, w * dY, the saved [g | u], [dg | du], each expert's dx row), each within
 2^-9 relative; every sum is fp32.
@@ -84,19 +85,26 @@ def run_train(wl: Workload, inp, dy, c_bal=C_BAL, c_z=C_Z):
                 dw_up=dwu, dw_down=dwd, dshared=dsh)
 
 
-def assert_grad(got, ref, what):
+def assert_grad(got, ref, what, elem=2e-2, norm=1e-2):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     m = float(np.abs(ref).max()) if ref.size else 0.0
     err = np.abs(got - ref)
-    bad = err > 2e-2 * m
-    assert not bad.any(), (f"{what}: {int(bad.sum())} of {ref.size} beyond 2e-2*max|ref| "
+    bad = err > elem * m
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {ref.size} beyond {elem:g}*max|ref| "
                            f"(max err {err.max():.3e}, max|ref| {m:.3e})")
     nr = float(np.linalg.norm(ref))
     if nr > 0:
         rel = float(np.linalg.norm(got - ref)) / nr
-        assert rel <= 1e-2, f"{what}: normwise error {rel:.3e}"
+        assert rel <= norm, f"{what}: normwise error {rel:.3e}"
+
+
+def grad_tolerances(wl):
+    """(per element of max|ref|, normwise): the bf16 bar above; for fp32 layers
+    every value stays fp32, so only fp32 sums of at most a few thousand terms
+    separate the path from the fp64 oracle (relative error a few 1e-6)."""
+    return (1e-4, 1e-5) if wl.dtype == "f32" else (2e-2, 1e-2)
 
 
 def compare_all(wl, inp, dy, got, c_bal=C_BAL, c_z=C_Z):
@@ -107,17 +115,19 @@ def compare_all(wl, inp, dy, got, c_bal=C_BAL, c_z=C_Z):
                           sel_bias=sb, **wl.routing())
     fwd_y = ref["fwd"]["y"]
     m = float(np.abs(fwd_y).max())
-    assert np.abs(to_np(got["y"]) - fwd_y).max() <= 1e-2 * m + 1e-3, "training forward y"
-    assert_grad(to_np(got["dx"]), ref["dx"], "dx")
-    assert_grad(to_np(got["dw_router"]), ref["dw_router"], "dw_router")
+    ytol = 1e-4 * m if wl.dtype == "f32" else 1e-2 * m + 1e-3
+    assert np.abs(to_np(got["y"]) - fwd_y).max() <= ytol, "training forward y"
+    el, nm = grad_tolerances(wl)
+    assert_grad(to_np(got["dx"]), ref["dx"], "dx", el, nm)
+    assert_grad(to_np(got["dw_router"]), ref["dw_router"], "dw_router", el, nm)
     if got["db_router"] is not None:
-        assert_grad(to_np(got["db_router"]), ref["db_router"], "db_router")
+        assert_grad(to_np(got["db_router"]), ref["db_router"], "db_router", el, nm)
     for k in ("dw_gate", "dw_up", "dw_down"):
-        assert_grad(to_np(got[k]), ref[k], k)
+        assert_grad(to_np(got[k]), ref[k], k, el, nm)
     if got["dshared"] is not None:
         for name, a, b in zip(("dw_gate_s", "dw_up_s", "dw_down_s"), got["dshared"],
                               ref["dshared"]):
-            assert_grad(to_np(a), b, name)
+            assert_grad(to_np(a), b, name, el, nm)
     return ref
 
 
@@ -136,6 +146,12 @@ SMALL = {
     "many_experts_top1": Workload("many_experts_top1", T=256, D=128, F=128, E=64, K=1),
     "single_expert": Workload("single_expert", T=100, D=128, F=192, E=1, K=1),
     "one_token": Workload("one_token", T=1, D=128, F=128, E=8, K=2),
+    # fp32 layers (SIMT GEMMs): the fp32 reference layer's shape, and drops with a shared expert
+    "f32_layer": Workload("f32_layer", T=512, D=256, F=512, E=8, K=2, dtype="f32"),
+    "f32_drops_shared": Workload("f32_drops_shared", T=300, D=128, F=192, E=8, K=2, dtype="f32",
+                                 capacity_factor=0.5, F_shared=64, bias="zipf"),
+    "f32_sigmoid": Workload("f32_sigmoid", T=200, D=96, F=160, E=16, K=3, dtype="f32",
+                            score_func="sigmoid", renormalize=False),
 }
 
 

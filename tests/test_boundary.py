@@ -178,9 +178,10 @@ def test_backward_sizes_counts_and_trace(lib):
     assert B.backward_workspace_size(c) > 0
     assert B.backward_kernel_count(c) == 10
     assert B.backward_kernel_count(_cfg(T=600, F=320, F_shared=192, capacity_factor=1.0)) == 14
-    assert B.backward_kernel_count(_cfg(dtype="f32")) == 0  # bf16 layers only
-    with pytest.raises(B.MoEError):
-        B.train_state_size(_cfg(dtype="f32"))
+    cf = _cfg(dtype="f32")  # fp32 layers: the same launches, SIMT GEMMs
+    assert B.backward_kernel_count(cf) == 10
+    assert B.train_state_size(cf) > B.train_state_size(_cfg())  # 4-byte activations
+    assert B.backward_workspace_size(cf) > B.backward_workspace_size(_cfg())
     names = B.trace_backward_stage_names()
     assert names[0] == "start" and names[-1] == "dx" and len(names) == 10
     assert lib.moe_trace_attach_backward(None, 0) == B.MOE_OK
@@ -199,10 +200,10 @@ def test_training_argument_errors(lib):
     assert fwd(None, sb) == B.MOE_ERR_WORKSPACE
     assert fwd(FAKE + 16, sb) == B.MOE_ERR_ALIGN
     assert fwd(FAKE, sb, x=None) == B.MOE_ERR_ARG
-    cf = _cfg(dtype="f32")
+    cf = _cfg(dtype="f32")  # fp32 layers are checked the same way (the state is larger)
     assert lib.moe_forward_train(ctypes.byref(cf), FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE,
-                                 None, None, None, FAKE, None, None, None, None, None, FAKE, 1 << 30,
-                                 None) == B.MOE_ERR_UNSUPPORTED
+                                 None, None, None, FAKE, None, None, None, None, None, FAKE,
+                                 B.train_state_size(cf) - 1, None) == B.MOE_ERR_WORKSPACE
 
     def bwd(dy=FAKE, state_bytes=sb, ws_bytes=bb, c_bal=0.0, dw_gate=FAKE, shared=None, cfg=c):
         return lib.moe_backward(ctypes.byref(cfg), FAKE, FAKE, FAKE, FAKE, FAKE, shared, shared,
