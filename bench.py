@@ -605,15 +605,27 @@ def run_gpu_ep(args):
     time.sleep(0.3)
     dist.barrier()
     torch.cuda.synchronize(dev)
+    names = layer.stage_names()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+           for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
+        layer.trace_events = evs[i]
         y = layer.forward(xs[i % nbuf], logit_noise=inp["noise"])
     stop.record(stream)
     torch.cuda.synchronize(dev)
     dist.barrier()
+    layer.trace_events = None
     clk = clocks.stop()
     ms_total, ms_step, value = aggregate(start.elapsed_time(stop), world, wl.T, args.steps, dev)
+    stage_ms = {}
+    for j, name in enumerate(names):
+        d = [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]
+        stage_ms[name] = sum(d) / len(d)
+    # rows this rank's experts ran on (the same every step: the batches share a shape, not
+    # their routing, so read the last step's)
+    local_rows = int(layer.ops.offsets_local[EL].item())
     # end to end: x in from pinned memory, y out, every step
     x_h = [t.cpu().pin_memory() for t in xs]
     y_h = torch.empty_like(x_h[0]).pin_memory()
@@ -639,6 +651,19 @@ def run_gpu_ep(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(wl, args.cpu_seconds)
+        # the local experts' two grouped GEMMs (the step's dominant work), rank 0's last step
+        peaks, peak_src = load_peaks()
+        key = "bf16_tflops_sustained" if ms_total > 1000.0 else "bf16_tflops"
+        peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
+        bound, src = "tensor", f"{key} of {peak_src}"
+        if wl.dtype == "f32":  # SIMT FMA pipes
+            peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+            bound, src = "alu", "148 SMs x 128 FMA x 2 x max clock"
+        achieved = 6.0 * local_rows * wl.D * wl.F / (stage_ms["experts"] / 1e3) / 1e12
+        roof = {"kernel": "experts (grouped gate/up + SwiGLU and down GEMMs of this rank's experts)",
+                "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": src,
+                "rows": local_rows, "traffic": None}
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -654,7 +679,8 @@ def run_gpu_ep(args):
                     "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io, "d2h_bytes_per_step": io,
                     "how": "per step: x in from pinned host memory, ExpertParallelMoE.forward, y out"},
             "gpu_launches": None if per_step is None else per_step * args.steps,
-            "roofline": None,
+            "roofline": roof,
+            "stages": {k: {"ms": round(v, 4)} for k, v in stage_ms.items()},
             "clocks": clk,
             "cpu_baseline": cpu,
         }

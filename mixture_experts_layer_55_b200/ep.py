@@ -219,6 +219,9 @@ class ExpertParallelMoE:
             ops = CudaOps(T, self.D, self.F, E, K, self.EL, self.W, dtype, capacity_factor,
                           router_options, w_gate_local.device)
         self.ops = ops
+        # optional CUDA events recorded on the current stream at the step
+        # boundaries of forward() (stage_names() + 1 of them), for stage timing
+        self.trace_events = None
         self.peer = None
         if exchange == "peer":
             dev = w_gate_local.device
@@ -232,6 +235,18 @@ class ExpertParallelMoE:
             self.peer.close()
             self.peer = None
 
+    PEER_STAGES = ("route", "counts_allgather", "dispatch", "barrier_rows", "experts",
+                   "barrier_results", "combine")
+    A2A_STAGES = ("route_dispatch", "counts_exchange", "rows_all_to_all", "to_expert_major",
+                  "experts", "results_all_to_all", "combine")
+
+    def stage_names(self):
+        return self.PEER_STAGES if self.exchange == "peer" else self.A2A_STAGES
+
+    def _mark(self, i):
+        if self.trace_events is not None:
+            self.trace_events[i].record()
+
     def _barrier(self):
         # stream-ordered: the next kernel on this stream starts after every
         # rank's kernels before its own all-reduce have finished
@@ -239,22 +254,33 @@ class ExpertParallelMoE:
 
     def _forward_peer(self, x, logit_noise):
         ops = self.ops
+        self._mark(0)
         kept = ops.route_index(x, self.w_router, self.router_bias, self.selection_bias, logit_noise)
+        self._mark(1)
         dist.all_gather_into_tensor(self.kept_all, kept, group=self.group)
+        self._mark(2)
         ops.peer_dispatch(x, self.kept_all, self.rank, self.W, self.peer)
+        self._mark(3)
         self._barrier()  # every rank's rows are in their owners' buffers
+        self._mark(4)
         ops.peer_experts(self.peer, self.w_gate, self.w_up, self.w_down)
+        self._mark(5)
         self._barrier()  # every owner's results are ready
-        return ops.peer_combine(x, self.W, self.peer)
+        self._mark(6)
+        y = ops.peer_combine(x, self.W, self.peer)
+        self._mark(7)
+        return y
 
     def forward(self, x, logit_noise=None):
         if self.exchange == "peer":
             return self._forward_peer(x, logit_noise)
         W, EL = self.W, self.EL
         ops = self.ops
+        self._mark(0)
         # route this rank's tokens and sort their rows by expert (so by owner)
         kept, offsets, x_perm = ops.route_dispatch(x, self.w_router, self.router_bias,
                                                    self.selection_bias, logit_noise)
+        self._mark(1)
         # exchange the per-expert row counts: recv[s, e] = rows source s sends for my expert e
         send_counts = kept.reshape(W, EL).contiguous()
         recv_counts = torch.empty_like(send_counts)
@@ -264,18 +290,25 @@ class ExpertParallelMoE:
         send_rows = (owner_bounds[1:] - owner_bounds[:-1]).cpu().tolist()
         recv_rows = recv_counts.sum(1).cpu().tolist()
         n_send, n_recv = sum(send_rows), sum(recv_rows)
+        self._mark(2)
         # rows to their owners
         x_recv = torch.empty((max(n_recv, 1), self.D), dtype=x.dtype, device=x.device)
         dist.all_to_all_single(x_recv[:n_recv], x_perm[:n_send].contiguous(), recv_rows, send_rows,
                                group=self.group)
+        self._mark(3)
         # arrived source-major; the grouped experts want expert-major
         offsets_local, dst_of, src_of = ops.layout(recv_counts, W, EL)
         x_loc = ops.to_expert_major(x_recv, src_of, n_recv)
+        self._mark(4)
         y_loc = ops.experts(x_loc, offsets_local, self.w_gate, self.w_up, self.w_down)
+        self._mark(5)
         # results back in arrival order, then to the tokens' home ranks
         y_back = ops.to_arrival_order(y_loc, dst_of, n_recv)
         y_perm = torch.empty((max(n_send, 1), self.D), dtype=x.dtype, device=x.device)
         dist.all_to_all_single(y_perm[:n_send], y_back[:n_recv].contiguous(), send_rows, recv_rows,
                                group=self.group)
+        self._mark(6)
         # weighted scatter-add at home
-        return ops.combine(y_perm, x)
+        y = ops.combine(y_perm, x)
+        self._mark(7)
+        return y
