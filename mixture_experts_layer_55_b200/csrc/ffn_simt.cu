@@ -7,116 +7,70 @@
 //   gate/up: h = silu(x_perm Wg_e) * (x_perm Wu_e)         (rows x F)
 //            (the training forward also keeps [g | u], rows x 2F)
 //   down:    y_perm = topk_w[perm[row]] * (h Wd_e)         (rows x D)
-// Tiles are 64 rows x 64 columns; the m-tile -> (expert, first row) map is
-// derived on the device from the offsets (no host synchronisation).
+// Tiles are 32 rows x 64 columns (gate/up: 32 h columns, their gate and up
+// columns side by side), on the double-buffered main loop of simt_gemm.cuh;
+// the m-tile -> (expert, first row) map is derived on the device from the
+// offsets (no host synchronisation).
 #include "common.cuh"
 #include "internal.h"
+#include "simt_gemm.cuh"
 
 namespace moe {
 
-constexpr int kSBM = 64, kSBN = 64, kSBK = 16;
+constexpr int kBM = 32, kBN = 64, kBK = 16;
 
-// s_pref[e] = number of kSBM-row tiles of experts < e; s_pref[E] = total.
-MOE_DEVICE void simt_tile_prefix(const int32_t* offsets, int E, int64_t max_rows, int* s_off,
-                                 int* s_pref, int* status)
+// One BM-row tile of an expert's rows: gate/up (GATEUP: the tile's B columns
+// are kBN/2 gate columns then the same kBN/2 up columns, so each thread holds
+// g and u of the same h column) or down (kBN output columns, scaled by the
+// row's routing weight).  grid (ceil(N / columns per tile), m-tile bound).
+template <bool GATEUP>
+__global__ void __launch_bounds__(simt::kThreads) ffn_simt_kernel(
+    const float* __restrict__ A, const float* __restrict__ B0, const float* __restrict__ B1,
+    float* __restrict__ out, const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
+    const float* __restrict__ topk_w, int E, int Kd, int N, int64_t max_rows, int64_t nk,
+    float* __restrict__ gu_keep, int* status)
 {
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        int prev = 0;
-        for (int e = 0; e < E; ++e) {
-            int a = s_off[e], b = s_off[e + 1];
-            if (a < prev || b < a || b > max_rows) {  // malformed offsets: treat as empty
-                raise_flag(status, kFlagBounds, 300);
-                b = a = prev;
-            }
-            prev = b;
-            s_pref[e] = run;
-            run += (b - a + kSBM - 1) / kSBM;
-        }
-        s_pref[E] = run;
-    }
-    __syncthreads();
-}
-
-template <typename T, bool GATEUP>
-__global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A,
-                                                       const T* __restrict__ B0,
-                                                       const T* __restrict__ B1, T* __restrict__ out,
-                                                       const int32_t* __restrict__ offsets,
-                                                       const int32_t* __restrict__ perm,
-                                                       const float* __restrict__ topk_w, int E,
-                                                       int Kd, int N, int64_t max_rows, int64_t nk,
-                                                       T* __restrict__ gu_keep, int* status)
-{
+    constexpr int NC = GATEUP ? kBN / 2 : kBN;  // output columns per tile
+    constexpr int TM = kBM / 16, TN = kBN / 16;
     __shared__ int s_off[257];
     __shared__ int s_pref[257];
-    __shared__ float As[kSBK][kSBM + 4];
-    __shared__ float Bs0[kSBK][kSBN];
-    __shared__ float Bs1[GATEUP ? kSBK : 1][kSBN];
+    __shared__ simt::Smem<kBM, kBN, kBK> sm;
+    simt::row_tile_prefix<kBM>(offsets, E, max_rows, s_off, s_pref, status, 300);
+    int e;
+    int64_t row0, row_end;
+    if (!simt::row_tile(s_off, s_pref, E, kBM, blockIdx.y, e, row0, row_end)) return;
+    const int n0 = blockIdx.x * NC;
 
-    simt_tile_prefix(offsets, E, max_rows, s_off, s_pref, status);
-    const int mt = blockIdx.y;
-    if (mt >= s_pref[E]) return;
-    int e = 0;
-    while (e + 1 < E && s_pref[e + 1] <= mt) ++e;  // experts with no tiles are skipped
-    const int64_t row0 = (int64_t)s_off[e] + (int64_t)(mt - s_pref[e]) * kSBM;
-    const int64_t row_end = s_off[e + 1];
-    const int n0 = blockIdx.x * kSBN;
-
-    const T* Bg = B0 + (size_t)e * Kd * N;
-    const T* Bu = GATEUP ? B1 + (size_t)e * Kd * N : nullptr;
-
-    const int tid = threadIdx.x;
-    const int tx = tid % 16, ty = tid / 16;  // 4x4 outputs: rows ty+16i, cols tx+16j
-    float acc0[4][4], acc1[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc0[i][j] = acc1[i][j] = 0.f;
-
-    for (int k0 = 0; k0 < Kd; k0 += kSBK) {
-        for (int idx = tid; idx < kSBM * kSBK; idx += 256) {
-            int r = idx / kSBK, kk = idx % kSBK;
-            int64_t row = row0 + r;
-            int k = k0 + kk;
-            As[kk][r] = (row < row_end && k < Kd) ? to_f32(A[row * Kd + k]) : 0.f;
+    struct LA {
+        const float* p;
+        int64_t r0, rend;
+        int lda;
+        MOE_DEVICE float ld(int m, int64_t k) const
+        {
+            const int64_t row = r0 + m;
+            return row < rend ? p[row * lda + k] : 0.f;
         }
-        for (int idx = tid; idx < kSBK * kSBN; idx += 256) {
-            int kk = idx / kSBN, cc = idx % kSBN;
-            int k = k0 + kk, col = n0 + cc;
-            bool ok = k < Kd && col < N;
-            Bs0[kk][cc] = ok ? to_f32(Bg[(size_t)k * N + col]) : 0.f;
-            if (GATEUP) Bs1[kk][cc] = ok ? to_f32(Bu[(size_t)k * N + col]) : 0.f;
+    } la{A, row0, row_end, Kd};
+    struct LB {
+        const float *g, *u;
+        int n0, N;
+        MOE_DEVICE float ld(int64_t k, int n) const
+        {
+            const bool up = GATEUP && n >= kBN / 2;
+            const int col = n0 + (up ? n - kBN / 2 : n);
+            return col < N ? (up ? u : g)[k * N + col] : 0.f;
         }
-        __syncthreads();
+    } lb{B0 + (size_t)e * Kd * N, GATEUP ? B1 + (size_t)e * Kd * N : nullptr, n0, N};
+
+    float acc[TM][TN];
+    simt::mainloop<kBM, kBN, kBK, true, false>(acc, la, lb, 0, Kd, sm);
+
 #pragma unroll
-        for (int kk = 0; kk < kSBK; ++kk) {
-            float a[4], b0[4], b1[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                b0[j] = Bs0[kk][tx + 16 * j];
-                if (GATEUP) b1[j] = Bs1[kk][tx + 16 * j];
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc0[i][j] = fmaf(a[i], b0[j], acc0[i][j]);
-                    if (GATEUP) acc1[i][j] = fmaf(a[i], b1[j], acc1[i][j]);
-                }
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t row = row0 + ty + 16 * i;
+    for (int i = 0; i < TM; ++i) {
+        const int64_t row = row0 + threadIdx.x / 16 + 16 * i;
         if (row >= row_end) continue;
         float wr = 1.f;
-        if (!GATEUP && perm != nullptr) {  // no perm: unit weights (a shared expert)
+        if (!GATEUP && perm != nullptr) {  // no perm: unit weights (a shared expert, training)
             const int32_t pa = perm[row];
             if (pa < 0 || pa >= nk) {
                 raise_flag(status, kFlagBounds, 301);
@@ -126,43 +80,42 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A,
             }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int col = n0 + tx + 16 * j;
+        for (int j = 0; j < (GATEUP ? TN / 2 : TN); ++j) {
+            const int col = n0 + threadIdx.x % 16 + 16 * j;
             if (col >= N) continue;
-            float v = GATEUP ? silu_f32(acc0[i][j]) * acc1[i][j] : wr * acc0[i][j];
-            out[row * N + col] = from_f32<T>(v);
-            if (GATEUP && gu_keep != nullptr) {  // [g | u] for the backward
-                gu_keep[row * 2 * N + col] = from_f32<T>(acc0[i][j]);
-                gu_keep[row * 2 * N + N + col] = from_f32<T>(acc1[i][j]);
+            if (GATEUP) {
+                const float g = acc[i][j], u = acc[i][j + TN / 2];
+                out[row * N + col] = silu_f32(g) * u;
+                if (gu_keep != nullptr) {  // [g | u] for the backward
+                    gu_keep[row * 2 * N + col] = g;
+                    gu_keep[row * 2 * N + N + col] = u;
+                }
+            } else {
+                out[row * N + col] = wr * acc[i][j];
             }
         }
     }
 }
 
-// Upper bound of the m-tiles: sum_e ceil(kept_e / BM) <= max_rows / BM + E.
-static inline int64_t simt_mtiles_bound(int64_t max_rows, int E)
-{
-    return (max_rows + kSBM - 1) / kSBM + E;
-}
-
-template <typename T>
 static cudaError_t launch_simt(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                const void* w_gate, const void* w_up, const void* w_down, void* h,
                                void* y_perm, void* gu_keep, int* status, cudaStream_t s, StageHook mid,
                                void* mid_ctx)
 {
-    const int64_t mtiles = simt_mtiles_bound(max_rows, c.E);
+    const int64_t mtiles = simt::mtiles_bound(max_rows, c.E, kBM);
     const int64_t nk = c.T * c.K;
-    dim3 g1((c.F + kSBN - 1) / kSBN, (unsigned)mtiles);
-    ffn_simt_kernel<T, true><<<g1, 256, 0, s>>>(
-        static_cast<const T*>(x_perm), static_cast<const T*>(w_gate), static_cast<const T*>(w_up),
-        static_cast<T*>(h), offsets, perm, topk_w, c.E, c.D, c.F, max_rows, nk, static_cast<T*>(gu_keep),
-        status);
+    dim3 g1((c.F + kBN / 2 - 1) / (kBN / 2), (unsigned)mtiles);
+    ffn_simt_kernel<true><<<g1, simt::kThreads, 0, s>>>(
+        static_cast<const float*>(x_perm), static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
+        static_cast<float*>(h), offsets, perm, topk_w, c.E, c.D, c.F, max_rows, nk,
+        static_cast<float*>(gu_keep), status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     if (mid) mid(mid_ctx, s);
-    dim3 g2((c.D + kSBN - 1) / kSBN, (unsigned)mtiles);
-    ffn_simt_kernel<T, false><<<g2, 256, 0, s>>>(
-        static_cast<const T*>(h), static_cast<const T*>(w_down), nullptr, static_cast<T*>(y_perm),
+    dim3 g2((c.D + kBN - 1) / kBN, (unsigned)mtiles);
+    ffn_simt_kernel<false><<<g2, simt::kThreads, 0, s>>>(
+        static_cast<const float*>(h), static_cast<const float*>(w_down), nullptr, static_cast<float*>(y_perm),
         offsets, perm, topk_w, c.E, c.F, c.D, max_rows, nk, nullptr, status);
     return cudaGetLastError();
 }
@@ -173,8 +126,8 @@ cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const voi
                                 void* y_perm, void* gu_keep, int* status, cudaStream_t s, StageHook mid,
                                 void* mid_ctx)
 {
-    return launch_simt<float>(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h,
-                              y_perm, gu_keep, status, s, mid, mid_ctx);
+    return launch_simt(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h, y_perm, gu_keep,
+                       status, s, mid, mid_ctx);
 }
 
 }  // namespace moe
