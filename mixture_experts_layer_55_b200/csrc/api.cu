@@ -47,8 +47,11 @@ WsLayout ws_layout(const moe_config& c)
     o += align_up(64 * sizeof(int));
     L.r_part = o;
     size_t part_bytes = (size_t)rp.splits * (size_t)c.T * c.E * sizeof(float);
-    if (router_tc_eligible(c) && router_tc_wsplit_bytes(c) > part_bytes)
-        part_bytes = router_tc_wsplit_bytes(c);
+    if (router_tc_eligible(c)) {  // split weights, then the split-K partial logits
+        const size_t tc = align_up(router_tc_wsplit_bytes(c)) +
+                          (size_t)router_tc_splits(c) * (size_t)c.T * c.E * sizeof(float);
+        if (tc > part_bytes) part_bytes = tc;
+    }
     o += align_up(part_bytes);
     L.r_mp = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(float));
@@ -674,7 +677,8 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK) return 0;
     const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
-    if (router_tc_eligible(*cfg)) return 11 + shared;  // split weights, fused router, 2 reductions
+    if (router_tc_eligible(*cfg))  // split weights, router (+ top-k after split-K), 2 reductions
+        return 11 + shared + (router_tc_splits(*cfg) > 1 ? 1 : 0);
     return 11 + shared + (router_plan(*cfg).splits > 1 ? 1 : 0);
 }
 

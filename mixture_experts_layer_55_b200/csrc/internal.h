@@ -112,12 +112,16 @@ int64_t max_rows_of(const moe_config& c);
 // Tensor-core router (router_tc.cu): bf16 layers with E <= 128 and T >= 2048.
 bool router_tc_eligible(const moe_config& c);
 int router_tc_blocks(const moe_config& c);
+// splits of d_model (1: the fused router; > 1: partial logits for the top-k kernel)
+int router_tc_splits(const moe_config& c);
 size_t router_tc_wsplit_bytes(const moe_config& c);
+// part_out: (splits, T, E) fp32 partial logits, used when router_tc_splits > 1
 cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
                              const float* w_router, const float* bias, const float* noise,
                              float* logits_out, float* probs_out, int32_t* ids, float* w,
                              float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
-                             int with_stats, void* wsplit_scratch, int* status, cudaStream_t s);
+                             int with_stats, void* wsplit_scratch, void* part_out, int* status,
+                             cudaStream_t s);
 
 // ---------------------------------------------------------------- launches --
 // Each returns cudaSuccess or the launch error.

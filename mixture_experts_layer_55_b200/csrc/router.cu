@@ -542,6 +542,30 @@ static void launch_logits(const moe_config& c, const RouterPlan& rp, const XT* x
     }
 }
 
+// softmax / sigmoid, top-k, weights and statistic partials from `splits`
+// partial logit buffers (T x E each), summed in split order
+static cudaError_t launch_topk(const moe_config& c, const RouteOpts& o, const float* part, int splits,
+                               const float* bias, const float* noise, float* logits_out, float* probs_out,
+                               int32_t* ids, float* w, float* blk_mp, float* blk_z, float* blk_ent,
+                               int32_t* blk_cnt, int with_stats, const RouterPlan& rp, cudaStream_t s)
+{
+    const int epl = (c.E + 31) / 32;
+    dim3 grid(rp.nb_topk);
+#define MOE_TOPK(N)                                                                                     \
+    router_topk_kernel<N><<<grid, 256, 0, s>>>(part, splits, bias, noise, o, logits_out, probs_out, ids, \
+                                               w, blk_mp, blk_z, blk_ent, blk_cnt, c.T, c.E, c.K,       \
+                                               with_stats)
+    switch (epl) {
+        case 1: MOE_TOPK(1); break;
+        case 2: MOE_TOPK(2); break;
+        case 3:
+        case 4: MOE_TOPK(4); break;
+        default: MOE_TOPK(8); break;
+    }
+#undef MOE_TOPK
+    return cudaGetLastError();
+}
+
 cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void* x,
                           const float* w_router, const float* bias, const float* sel_bias,
                           const float* noise, const float* logits_in, float* logits_out,
@@ -556,13 +580,22 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
     double* fin = reinterpret_cast<double*>(ws + L.r_fin);
     int nb = rp.nb_topk;
+    int tc_splits = 0;  // > 1: the tensor-core router wrote split partial logits
     if (!logits_in && router_tc_eligible(c)) {
-        // bf16 layers with enough tokens: fused tensor-core router
+        // bf16 layers with enough tokens: tensor-core router (fused, or split over d_model)
+        tc_splits = router_tc_splits(c);
+        char* part_tc = ws + L.r_part + align_up(router_tc_wsplit_bytes(c));
         cudaError_t e = launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids,
                                          w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats,
-                                         ws + L.r_part, reinterpret_cast<int*>(ws + L.status), s);
+                                         ws + L.r_part, part_tc, reinterpret_cast<int*>(ws + L.status), s);
         if (e != cudaSuccess) return e;
         nb = router_tc_blocks(c);
+        if (tc_splits > 1) {
+            nb = rp.nb_topk;
+            e = launch_topk(c, o, reinterpret_cast<const float*>(part_tc), tc_splits, bias, noise, logits_out,
+                            probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats, rp, s);
+            if (e != cudaSuccess) return e;
+        }
     } else {
         const float* part;
         if (logits_in) {
@@ -583,20 +616,9 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
             }
             part = p;
         }
-        const int epl = (c.E + 31) / 32;
-        dim3 grid(rp.nb_topk);
-#define MOE_TOPK(N)                                                                                \
-    router_topk_kernel<N><<<grid, 256, 0, s>>>(part, 1, bias, noise, o, logits_out, probs_out, ids, \
-                                               w, blk_mp, blk_z, blk_ent, blk_cnt, c.T, c.E, c.K,   \
-                                               with_stats)
-        switch (epl) {
-            case 1: MOE_TOPK(1); break;
-            case 2: MOE_TOPK(2); break;
-            case 3:
-            case 4: MOE_TOPK(4); break;
-            default: MOE_TOPK(8); break;
-        }
-#undef MOE_TOPK
+        cudaError_t e = launch_topk(c, o, part, 1, bias, noise, logits_out, probs_out, ids, w, blk_mp,
+                                    blk_z, blk_ent, blk_cnt, with_stats, rp, s);
+        if (e != cudaSuccess) return e;
     }
     if (with_stats) {
         router_colsum_kernel<<<c.E + 2, 256, 0, s>>>(blk_mp, blk_z, blk_ent, blk_cnt, nb, c.E, fin);

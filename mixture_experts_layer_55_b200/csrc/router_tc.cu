@@ -15,7 +15,11 @@
 //
 //   router_wsplit_kernel  W_r (D, E) fp32 -> (3, D, EP) bf16, EP = E rounded
 //                         up to 64 (zero columns), N-major for TMA.
-//   router_tc_kernel      one CTA per 128 tokens: warp 0 TMA (x tile 128 x 64,
+//   router_tc_kernel      one CTA per 128 tokens (and per split of d_model when
+//                         the token tiles leave most SMs idle: the splits write
+//                         fp32 partial logits, which the top-k kernel of the
+//                         SIMT router sums in split order and routes; the fused
+//                         epilogue below runs otherwise): warp 0 TMA (x tile 128 x 64,
 //                         three 64 x EP weight tiles per stage), warp 1
 //                         tcgen05.mma M=128, N=EP, three per K step into one
 //                         accumulator; warps 2..5 own one token row each:
@@ -72,6 +76,8 @@ struct Args {
     int D, E, K;
     int with_stats;
     int* status;
+    float* part;              // split mode: (splits, T, E) fp32 partial logits, else null
+    int split_kb;             // split mode: K blocks per split (blockIdx.y = split)
 };
 
 __global__ void __launch_bounds__(256) router_wsplit_kernel(const float* __restrict__ w,
@@ -111,6 +117,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
     const int num_kb = (a.D + BK - 1) / BK;
+    // this CTA's K blocks: all of them, or its split's share (never empty)
+    const int kb_begin = a.part ? (int)blockIdx.y * a.split_kb : 0;
+    const int kb_end = a.part ? min(num_kb, kb_begin + a.split_kb) : num_kb;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -139,7 +148,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t phase = 0;
         int last_phase[STAGES];
         for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
             if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
             uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
             uint8_t* sB = sA + A_BYTES;
@@ -165,7 +174,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         constexpr uint32_t idesc = umma_idesc_bf16(BM, EP, 0, 1);
         int stage = 0;
         uint32_t phase = 0;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
             if (!mbar_wait(&m->full[stage], phase, a.status, 520, abort_flag)) break;
             tc_fence_after();
             const uint32_t sA = smem_u32(stages + (size_t)stage * STAGE_BYTES);
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int p = 0; p < 3; ++p) {
                     const uint64_t bdesc =
                         umma_desc_sw128(sB + p * EPB * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
-                    umma_f16_ss(tmem_base, adesc, bdesc, idesc, (kb | kk | p) != 0 ? 1u : 0u);
+                    umma_f16_ss(tmem_base, adesc, bdesc, idesc, (kb != kb_begin || kk || p) ? 1u : 0u);
                 }
             }
             umma_commit(&m->empty[stage]);
@@ -201,6 +210,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool ok = mbar_wait(&m->tfull, 0, a.status, 530, abort_flag);
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+        if (a.part != nullptr) {
+            // split mode: this split's partial logits of the row, summed (in split
+            // order) with bias and noise by the top-k kernel
+            float* prow = a.part + ((size_t)blockIdx.y * a.T + t) * E;
+#pragma unroll 1
+            for (int c = 0; c < EP / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, v);
+                tmem_ld_wait();
+                if (valid)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c * 32 + j < E) prow[c * 32 + j] = ok ? __uint_as_float(v[j]) : 0.f;
+            }
+        } else {
         // pass 1: logits (+ bias + noise) to shared memory and their maximum
         float mx = -INFINITY;
 #pragma unroll 1
@@ -344,6 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 a.blk_ent[blockIdx.x] = hs;
             }
         }
+        }  // fused epilogue
     }
     tc_fence_before();
     __syncthreads();
@@ -409,7 +434,9 @@ static cudaError_t launch_t(const moe_config& c, const void* x, const __nv_bfloa
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    const unsigned grid = (unsigned)((c.T + BM - 1) / BM);
+    const int nkb = (c.D + BK - 1) / BK;
+    const unsigned splits = a.part ? (unsigned)((nkb + a.split_kb - 1) / a.split_kb) : 1u;
+    const dim3 grid((unsigned)((c.T + BM - 1) / BM), splits);
     router_tc_kernel<EPB><<<grid, NUM_THREADS, G::SMEM, s>>>(mX, mW, a);
     return cudaGetLastError();
 }
@@ -423,6 +450,21 @@ bool router_tc_eligible(const moe_config& c)
 
 int router_tc_blocks(const moe_config& c) { return (int)((c.T + rtc::BM - 1) / rtc::BM); }
 
+int router_tc_splits(const moe_config& c)
+{
+    // Split the contraction over d_model when the token tiles alone leave most
+    // SMs idle (a large d_model with few tokens): up to 4 splits of at least
+    // 8 K blocks each, so that tiles x splits stays within one wave.
+    const int tiles = router_tc_blocks(c);
+    const int nkb = (c.D + rtc::BK - 1) / rtc::BK;
+    int sp = 148 / (tiles > 0 ? tiles : 1);
+    if (sp > 4) sp = 4;
+    if (sp > nkb / 8) sp = nkb / 8;
+    if (sp < 2) return 1;
+    const int per = (nkb + sp - 1) / sp;  // K blocks per split; every split non-empty
+    return (nkb + per - 1) / per;
+}
+
 size_t router_tc_wsplit_bytes(const moe_config& c)
 {
     const int ep = (c.E + 63) / 64 * 64;
@@ -433,7 +475,8 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
                              const float* w_router, const float* bias, const float* noise,
                              float* logits_out, float* probs_out, int32_t* ids, float* w,
                              float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
-                             int with_stats, void* wsplit_scratch, int* status, cudaStream_t s)
+                             int with_stats, void* wsplit_scratch, void* part_out, int* status,
+                             cudaStream_t s)
 {
     using namespace rtc;
     const int ep = (c.E + 63) / 64 * 64;
@@ -442,8 +485,11 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
     int64_t blocks = (n + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     router_wsplit_kernel<<<(unsigned)blocks, 256, 0, s>>>(w_router, wsplit, c.D, c.E, ep);
+    const int splits = router_tc_splits(c);
+    const int nkb = (c.D + BK - 1) / BK;
     Args a{o, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt,
-           c.T, c.D, c.E, c.K, with_stats, status};
+           c.T, c.D, c.E, c.K, with_stats, status,
+           splits > 1 ? static_cast<float*>(part_out) : nullptr, (nkb + splits - 1) / splits};
     return ep == 64 ? launch_t<1>(c, x, wsplit, a, s) : launch_t<2>(c, x, wsplit, a, s);
 }
 

@@ -46,6 +46,11 @@ SMALL = [
     _wl("tcr_ragged", T=2500, D=136, F=64, E=8, K=2, seed=16),
     _wl("tcr_e100", T=2100, D=264, F=64, E=100, K=4, bias="zipf", noise=True, seed=17),
     _wl("tcr_e128_k8", T=2048, D=128, F=32, E=128, K=8, seed=18),
+    # tensor-core router split over d_model (few token tiles, long d_model): 2 splits with a
+    # ragged last one, and 4 splits under the group limit, selection bias and sigmoid scores
+    _wl("tcr_split2", T=2200, D=1088, F=64, E=8, K=2, bias="zipf", noise=True, seed=40),
+    _wl("tcr_split4_groups", T=2048, D=2048, F=32, E=64, K=6, n_groups=8, topk_groups=3,
+        sel_bias=True, score_func="sigmoid", seed=41),
     # router variants, SIMT router (T < 2048) and tensor-core router
     _wl("sigmoid_simt", T=300, E=16, K=3, score_func="sigmoid", seed=23),
     _wl("norenorm_scale_simt", T=300, E=8, K=2, renormalize=False, route_scale=2.5, seed=24),
