@@ -230,21 +230,24 @@ MOE_DEVICE int peer_slot(const int32_t* __restrict__ ids, const int32_t* __restr
     return e / EL;
 }
 
-// Each thread moves VPT 16-byte vectors of token rows: vector i of the
-// flattened (T x vpr) input is loaded once and stored to each kept slot's
-// row in its owner's receive buffer.  Block 0 also writes this rank's local
-// offsets; every block writes remote_row for its share of the slots (the
-// combine's map back).  Every thread ends with a system-scope fence, so its
-// peer stores are visible before the barrier that follows the kernel.
+// One warp per token (grid-stride over tokens).  Lanes k < K place slot k
+// (its owner and row in the owner's buffer; remote_row, the combine's map
+// back) and the warp broadcasts them; then the lanes move the token row's
+// 16-byte vectors, kUnroll loads in flight per lane, each stored to every
+// kept slot's destination.  Block 0 also writes this rank's local offsets.
+// Every thread ends with a system-scope fence, so its peer stores are
+// visible before the barrier that follows the kernel.
+constexpr int kPeerUnroll = 4;
+constexpr int kPeerWarps = 8;
+
 template <int KS>
-__global__ void __launch_bounds__(256) peer_dispatch_kernel(
+__global__ void __launch_bounds__(kPeerWarps * 32) peer_dispatch_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ ids, const int32_t* __restrict__ row_of,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ kept_all,
     uint4* const* __restrict__ recv_bufs, int64_t T, int K, int E, int EL, int W, int rank, int64_t vpr,
     int64_t recv_rows, int64_t max_rows, int32_t* __restrict__ local_offsets,
     int32_t* __restrict__ remote_row, int* status)
 {
-    constexpr int VPT = 8 / KS;
     __shared__ int32_t tot[kPeerMaxE], own[kPeerMaxE], seg[kPeerMaxE], offs[kPeerMaxE + 1];
     __shared__ uint4* bufs[kPeerMaxWorld];
     for (int i = threadIdx.x; i <= E; i += blockDim.x) offs[i] = offsets[i];
@@ -255,33 +258,38 @@ __global__ void __launch_bounds__(256) peer_dispatch_kernel(
             const int e = rank * EL + (j < EL ? j : EL - 1);
             local_offsets[j] = j < EL ? own[e] : own[e] + tot[e];
         }
-    const int64_t G = (int64_t)gridDim.x * blockDim.x;
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (int64_t sl = tid; sl < T * K; sl += G) {
-        int32_t d = -1;
-        if (peer_slot(ids, row_of, offs, seg, sl, E, EL, recv_rows, max_rows, &d, status, 730) < 0) d = -1;
-        remote_row[sl] = d;
-    }
-    const int64_t n = T * vpr;
-    for (int64_t base = tid; base < n; base += G * VPT) {
-        uint4 vals[VPT];
-#pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int64_t i = base + (int64_t)u * G;
-            vals[u] = i < n ? __ldg(x + i) : make_uint4(0, 0, 0, 0);
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * kPeerWarps;
+    for (int64_t t = (int64_t)blockIdx.x * kPeerWarps + (threadIdx.x >> 5); t < T; t += nw) {
+        int o = -1;
+        int32_t d = 0;
+        if (lane < K) {
+            o = peer_slot(ids, row_of, offs, seg, t * K + lane, E, EL, recv_rows, max_rows, &d, status, 730);
+            remote_row[t * K + lane] = o >= 0 ? d : -1;
         }
+        uint4* dst[KS];
 #pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int64_t i = base + (int64_t)u * G;
-            if (i >= n) break;
-            const int64_t t = i / vpr, v = i - t * vpr;
+        for (int k = 0; k < KS; ++k) {
+            const int ok = __shfl_sync(0xffffffffu, o, k);
+            const int32_t dk = __shfl_sync(0xffffffffu, d, k);
+            dst[k] = ok >= 0 ? bufs[ok] + (int64_t)dk * vpr : nullptr;
+        }
+        const uint4* xr = x + t * vpr;
+        for (int64_t v0 = lane; v0 < vpr; v0 += 32 * kPeerUnroll) {
+            uint4 val[kPeerUnroll];
+#pragma unroll
+            for (int u = 0; u < kPeerUnroll; ++u) {
+                const int64_t v = v0 + 32 * u;
+                val[u] = v < vpr ? __ldg(xr + v) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
             for (int k = 0; k < KS; ++k) {
-                if (k >= K) break;
-                int32_t d = 0;
-                const int o = peer_slot(ids, row_of, offs, seg, t * K + k, E, EL, recv_rows, max_rows, &d,
-                                        status, 732);
-                if (o >= 0) bufs[o][(int64_t)d * vpr + v] = vals[u];
+                if (dst[k] == nullptr) continue;
+#pragma unroll
+                for (int u = 0; u < kPeerUnroll; ++u) {
+                    const int64_t v = v0 + 32 * u;
+                    if (v < vpr) dst[k][v] = val[u];
+                }
             }
         }
     }
@@ -289,66 +297,83 @@ __global__ void __launch_bounds__(256) peer_dispatch_kernel(
 }
 
 // y[t] = y_add[t] + sum over kept slots, in slot order, of topk_w[t, k] *
-// (owner's y_loc)[remote_row[t, k]]: fp32 sums, rounded once.  The owners'
-// rows are read with plain (coherent) loads: they were written by another
-// GPU's kernel before the barrier that precedes this one.
+// (owner's y_loc)[remote_row[t, k]]: fp32 sums, rounded once.  One warp per
+// token: lanes k < K read slot k's owner, row and weight, the warp broadcasts
+// them, and each lane sums kPeerUnroll vectors of the row at a time (K x
+// kPeerUnroll loads in flight).  The owners' rows are read with plain
+// (coherent) loads: another GPU's kernel wrote them before the barrier that
+// precedes this one.
 template <typename ET, int KS>
-__global__ void __launch_bounds__(256) peer_combine_kernel(
+__global__ void __launch_bounds__(kPeerWarps * 32) peer_combine_kernel(
     const uint4* const* __restrict__ y_bufs, const int32_t* __restrict__ ids,
     const int32_t* __restrict__ remote_row, const float* __restrict__ topk_w,
     const uint4* __restrict__ y_add, uint4* __restrict__ y, int64_t T, int K, int E, int EL, int W,
     int64_t vpr, int64_t recv_rows, int* status)
 {
-    constexpr int VPT = 8 / KS;
     __shared__ const uint4* bufs[kPeerMaxWorld];
     for (int i = threadIdx.x; i < W; i += blockDim.x) bufs[i] = y_bufs[i];
     __syncthreads();
-    const int64_t n = T * vpr;
-    const int64_t G = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n; base += G * VPT) {
-        uint4 vals[VPT][KS];
-        int32_t own[VPT][KS];
-#pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int64_t i = base + (int64_t)u * G;
-            const int64_t t = i < n ? i / vpr : 0, v = i - t * vpr;
-#pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                own[u][k] = -1;
-                vals[u][k] = make_uint4(0, 0, 0, 0);
-                if (i >= n || k >= K) continue;
-                const int32_t d = __ldg(remote_row + t * K + k);
-                if (d < 0) continue;
-                const int32_t e = __ldg(ids + t * K + k);
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * kPeerWarps;
+    for (int64_t t = (int64_t)blockIdx.x * kPeerWarps + (threadIdx.x >> 5); t < T; t += nw) {
+        const uint4* src = nullptr;
+        float wk = 0.f;
+        if (lane < K) {
+            const int32_t d = __ldg(remote_row + t * K + lane);
+            const int32_t e = __ldg(ids + t * K + lane);
+            if (d >= 0) {
                 if (e < 0 || e >= E || d >= recv_rows) {
-                    if (v == 0) raise_flag(status, kFlagBounds, 740);
-                    continue;
+                    raise_flag(status, kFlagBounds, 740);
+                } else {
+                    src = bufs[e / EL] + (int64_t)d * vpr;
+                    wk = __ldg(topk_w + t * K + lane);
                 }
-                own[u][k] = e / EL;
-                vals[u][k] = bufs[own[u][k]][(int64_t)d * vpr + v];
             }
         }
+        const uint4* srck[KS];
+        float wks[KS];
 #pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int64_t i = base + (int64_t)u * G;
-            if (i >= n) break;
-            const int64_t t = i / vpr;
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (y_add) Vec<ET>::add(acc, __ldg(y_add + i));
+        for (int k = 0; k < KS; ++k) {
+            srck[k] = reinterpret_cast<const uint4*>(
+                __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), k));
+            wks[k] = __shfl_sync(0xffffffffu, wk, k);
+        }
+        for (int64_t v0 = lane; v0 < vpr; v0 += 32 * kPeerUnroll) {
+            float acc[kPeerUnroll][8];
 #pragma unroll
-            for (int k = 0; k < KS; ++k)
-                if (own[u][k] >= 0) Vec<ET>::add_scaled(acc, vals[u][k], __ldg(topk_w + t * K + k));
-            y[i] = Vec<ET>::pack(acc);
+            for (int u = 0; u < kPeerUnroll; ++u) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+                const int64_t v = v0 + 32 * u;
+                if (y_add && v < vpr) Vec<ET>::add(acc[u], __ldg(y_add + t * vpr + v));
+            }
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                if (srck[k] == nullptr) continue;
+                uint4 val[kPeerUnroll];
+#pragma unroll
+                for (int u = 0; u < kPeerUnroll; ++u) {
+                    const int64_t v = v0 + 32 * u;
+                    val[u] = v < vpr ? srck[k][v] : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < kPeerUnroll; ++u) Vec<ET>::add_scaled(acc[u], val[u], wks[k]);
+            }
+#pragma unroll
+            for (int u = 0; u < kPeerUnroll; ++u) {
+                const int64_t v = v0 + 32 * u;
+                if (v < vpr) y[t * vpr + v] = Vec<ET>::pack(acc[u]);
+            }
         }
     }
 }
 
-static int64_t peer_blocks(int64_t n_vec, int vpt)
+static unsigned peer_blocks(int64_t T)
 {
-    int64_t blocks = (n_vec + 256LL * vpt - 1) / (256LL * vpt);
-    const int64_t cap = (int64_t)sm_count_ep() * 8;
+    int64_t blocks = (T + kPeerWarps - 1) / kPeerWarps;
+    const int64_t cap = (int64_t)sm_count_ep() * 16;
     if (blocks > cap) blocks = cap;
-    return blocks < 1 ? 1 : blocks;
+    return (unsigned)(blocks < 1 ? 1 : blocks);
 }
 
 cudaError_t launch_peer_dispatch(const moe_config& c, int rank, int W, const int32_t* kept_all, const void* x,
@@ -358,14 +383,14 @@ cudaError_t launch_peer_dispatch(const moe_config& c, int rank, int W, const int
 {
     const int64_t vpr = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
     const int EL = c.E / W;
-    const int vpt = c.K <= 1 ? 8 : c.K == 2 ? 4 : c.K <= 4 ? 2 : 1;
-    const unsigned blocks = (unsigned)peer_blocks(c.T * vpr, vpt);
+    const unsigned blocks = peer_blocks(c.T);
     const uint4* xv = static_cast<const uint4*>(x);
     uint4* const* rb = reinterpret_cast<uint4* const*>(recv_bufs);
 #define MOE_PEER_DISPATCH(KS)                                                                          \
-    peer_dispatch_kernel<KS><<<blocks, 256, 0, s>>>(xv, ids, row_of, offsets, kept_all, rb, c.T, c.K, c.E, \
-                                                    EL, W, rank, vpr, recv_rows, max_rows, local_offsets, \
-                                                    remote_row, status)
+    peer_dispatch_kernel<KS><<<blocks, kPeerWarps * 32, 0, s>>>(xv, ids, row_of, offsets, kept_all, rb, \
+                                                                c.T, c.K, c.E, EL, W, rank, vpr,       \
+                                                                recv_rows, max_rows, local_offsets,    \
+                                                                remote_row, status)
     if (c.K <= 1) MOE_PEER_DISPATCH(1);
     else if (c.K == 2) MOE_PEER_DISPATCH(2);
     else if (c.K <= 4) MOE_PEER_DISPATCH(4);
@@ -381,9 +406,10 @@ static void launch_peer_combine_t(const moe_config& c, int W, unsigned blocks, c
                                   cudaStream_t s)
 {
     const int EL = c.E / W;
-#define MOE_PEER_COMBINE(KS)                                                                            \
-    peer_combine_kernel<ET, KS><<<blocks, 256, 0, s>>>(yb, ids, remote_row, topk_w, add, y, c.T, c.K, c.E, \
-                                                       EL, W, vpr, recv_rows, status)
+#define MOE_PEER_COMBINE(KS)                                                                      \
+    peer_combine_kernel<ET, KS><<<blocks, kPeerWarps * 32, 0, s>>>(yb, ids, remote_row, topk_w, add, y, \
+                                                                   c.T, c.K, c.E, EL, W, vpr,         \
+                                                                   recv_rows, status)
     if (c.K <= 1) MOE_PEER_COMBINE(1);
     else if (c.K == 2) MOE_PEER_COMBINE(2);
     else if (c.K <= 4) MOE_PEER_COMBINE(4);
@@ -396,8 +422,7 @@ cudaError_t launch_peer_combine(const moe_config& c, int W, const void* const* y
                                 const void* y_add, void* y, int* status, cudaStream_t s)
 {
     const int64_t vpr = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4) / 16;
-    const int vpt = c.K <= 1 ? 8 : c.K == 2 ? 4 : c.K <= 4 ? 2 : 1;
-    const unsigned blocks = (unsigned)peer_blocks(c.T * vpr, vpt);
+    const unsigned blocks = peer_blocks(c.T);
     const uint4* const* yb = reinterpret_cast<const uint4* const*>(y_bufs);
     const uint4* add = static_cast<const uint4*>(y_add);
     uint4* out = static_cast<uint4*>(y);
