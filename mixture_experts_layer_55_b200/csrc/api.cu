@@ -677,8 +677,8 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK) return 0;
     const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
-    if (router_tc_eligible(*cfg))  // split weights, router (+ top-k after split-K), 2 reductions
-        return 11 + shared + (router_tc_splits(*cfg) > 1 ? 1 : 0);
+    if (router_tc_eligible(*cfg))  // split weights, router (+ top-k from its logits), 2 reductions
+        return 11 + shared + (router_tc_partial(*cfg) ? 1 : 0);
     return 11 + shared + (router_plan(*cfg).splits > 1 ? 1 : 0);
 }
 

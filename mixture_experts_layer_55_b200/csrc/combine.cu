@@ -8,7 +8,7 @@
 //
 // The routing weight is normally applied by the down GEMM's epilogue, so the
 // combine is a plain gather-sum: 16-byte vector loads of the token's K rows of
-// y_perm, summed in slot order in fp32 and rounded once.  The training forward
+// y_perm (a warp per token), summed in slot order in fp32 and rounded once.  The training forward
 // keeps the expert outputs unweighted (the backward needs them), and then the
 // combine multiplies each row by its slot's weight as it adds it.
 // No atomics: the result is deterministic.
@@ -18,53 +18,69 @@
 
 namespace moe {
 
-// Each thread produces VPT 16-byte vectors of the output, with KS >= K slots
-// per token and VPT * KS = 8, so that about 8 loads are in flight per thread
-// whatever K is: vectors i, i + G, ... of the flattened (T x vec_per_row)
-// output, G = total threads.  row_of is shared by a row's threads through L1.
-// Consecutive threads cover consecutive vectors of a row (coalesced).
+// One warp per token (grid-stride over tokens): lanes k < K read slot k's row
+// (and weight), the warp broadcasts them, and each lane sums kCombineUnroll
+// 16-byte vectors of the token's output at a time (K x kCombineUnroll loads
+// in flight), in slot order, in fp32, rounded once.  An out-of-range row is
+// never read (the slot counts as dropped).
+constexpr int kCombineUnroll = 4;
+constexpr int kCombineWarps = 8;
+
 template <typename ET, int KS>
-__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
-                                                      const int32_t* __restrict__ row_of,
-                                                      const float* __restrict__ slot_w,
-                                                      const uint4* __restrict__ y_add,
-                                                      uint4* __restrict__ y, int64_t T, int K,
-                                                      int64_t vec_per_row, int64_t max_rows)
+__global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const uint4* __restrict__ y_perm,
+                                                                     const int32_t* __restrict__ row_of,
+                                                                     const float* __restrict__ slot_w,
+                                                                     const uint4* __restrict__ y_add,
+                                                                     uint4* __restrict__ y, int64_t T, int K,
+                                                                     int64_t vpr, int64_t max_rows)
 {
-    constexpr int VPT = 8 / KS;
-    const int64_t n = T * vec_per_row;
-    const int64_t G = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n; base += G * VPT) {
-        uint4 vals[VPT][KS];
-        int32_t rows[VPT][KS];
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * kCombineWarps;
+    for (int64_t t = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5); t < T; t += nw) {
+        int32_t r = -1;
+        float wk = 1.f;
+        if (lane < K) {
+            r = __ldg(row_of + t * K + lane);
+            if (r >= max_rows) r = -1;  // never read outside y_perm
+            if (slot_w && r >= 0) wk = __ldg(slot_w + t * K + lane);
+        }
+        int32_t rows[KS];
+        float ws[KS];
 #pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int64_t i = base + (int64_t)u * G;
-            const int64_t t = i < n ? i / vec_per_row : 0, v = i - t * vec_per_row;
+        for (int k = 0; k < KS; ++k) {
+            rows[k] = __shfl_sync(0xffffffffu, r, k);
+            ws[k] = __shfl_sync(0xffffffffu, wk, k);
+        }
+        for (int64_t v0 = lane; v0 < vpr; v0 += 32 * kCombineUnroll) {
+            float acc[kCombineUnroll][8];
 #pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                int32_t r = (i < n && k < K) ? __ldg(row_of + t * K + k) : -1;
-                rows[u][k] = (r >= 0 && r < max_rows) ? r : -1;  // never read outside y_perm
+            for (int u = 0; u < kCombineUnroll; ++u) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+                const int64_t v = v0 + 32 * u;
+                if (y_add && v < vpr) Vec<ET>::add(acc[u], __ldg(y_add + t * vpr + v));  // shared expert first
             }
 #pragma unroll
-            for (int k = 0; k < KS; ++k)
-                vals[u][k] = rows[u][k] >= 0 ? __ldg(y_perm + (int64_t)rows[u][k] * vec_per_row + v)
-                                             : make_uint4(0, 0, 0, 0);
-        }
+            for (int k = 0; k < KS; ++k) {
+                if (rows[k] < 0) continue;  // slot order; dropped or absent slots add nothing
+                const uint4* src = y_perm + (int64_t)rows[k] * vpr;
+                uint4 val[kCombineUnroll];
 #pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int64_t i = base + (int64_t)u * G;
-            if (i >= n) break;
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (y_add) Vec<ET>::add(acc, __ldg(y_add + i));  // shared expert output first
-            const int64_t t = i / vec_per_row;
-#pragma unroll
-            for (int k = 0; k < KS; ++k)
-                if (rows[u][k] >= 0) {  // slot order
-                    if (slot_w) Vec<ET>::add_scaled(acc, vals[u][k], __ldg(slot_w + t * K + k));
-                    else Vec<ET>::add(acc, vals[u][k]);
+                for (int u = 0; u < kCombineUnroll; ++u) {
+                    const int64_t v = v0 + 32 * u;
+                    val[u] = v < vpr ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
                 }
-            y[i] = Vec<ET>::pack(acc);
+#pragma unroll
+                for (int u = 0; u < kCombineUnroll; ++u) {
+                    if (slot_w) Vec<ET>::add_scaled(acc[u], val[u], ws[k]);
+                    else Vec<ET>::add(acc[u], val[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kCombineUnroll; ++u) {
+                const int64_t v = v0 + 32 * u;
+                if (v < vpr) y[t * vpr + v] = Vec<ET>::pack(acc[u]);
+            }
         }
     }
 }
@@ -77,18 +93,15 @@ static void launch_combine_t(const moe_config& c, int64_t blocks, const void* y_
     const uint4* src = static_cast<const uint4*>(y_perm);
     const uint4* add = static_cast<const uint4*>(y_add);
     uint4* dst = static_cast<uint4*>(y);
+    const unsigned g = (unsigned)blocks, nt = kCombineWarps * 32;
     if (c.K <= 1)
-        combine_kernel<ET, 1><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
-                                                                max_rows);
+        combine_kernel<ET, 1><<<g, nt, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr, max_rows);
     else if (c.K == 2)
-        combine_kernel<ET, 2><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
-                                                                max_rows);
+        combine_kernel<ET, 2><<<g, nt, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr, max_rows);
     else if (c.K <= 4)
-        combine_kernel<ET, 4><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
-                                                                max_rows);
+        combine_kernel<ET, 4><<<g, nt, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr, max_rows);
     else
-        combine_kernel<ET, 8><<<(unsigned)blocks, 256, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr,
-                                                                max_rows);
+        combine_kernel<ET, 8><<<g, nt, 0, s>>>(src, row_of, slot_w, add, dst, c.T, c.K, vpr, max_rows);
 }
 
 cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_t* row_of,
@@ -100,8 +113,7 @@ cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int vpt = c.K <= 1 ? 8 : c.K == 2 ? 4 : c.K <= 4 ? 2 : 1;
-    int64_t blocks = (c.T * vpr + 256LL * vpt - 1) / (256LL * vpt);
+    int64_t blocks = (c.T + kCombineWarps - 1) / kCombineWarps;
     const int64_t cap = (int64_t)sms * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

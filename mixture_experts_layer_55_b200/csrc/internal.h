@@ -114,6 +114,8 @@ bool router_tc_eligible(const moe_config& c);
 int router_tc_blocks(const moe_config& c);
 // splits of d_model (1: the fused router; > 1: partial logits for the top-k kernel)
 int router_tc_splits(const moe_config& c);
+// true: the tensor-core router writes (partial) logits and the top-k kernel routes
+bool router_tc_partial(const moe_config& c);
 size_t router_tc_wsplit_bytes(const moe_config& c);
 // part_out: (splits, T, E) fp32 partial logits, used when router_tc_splits > 1
 cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,

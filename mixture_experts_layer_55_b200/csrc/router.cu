@@ -580,17 +580,16 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
     double* fin = reinterpret_cast<double*>(ws + L.r_fin);
     int nb = rp.nb_topk;
-    int tc_splits = 0;  // > 1: the tensor-core router wrote split partial logits
     if (!logits_in && router_tc_eligible(c)) {
-        // bf16 layers with enough tokens: tensor-core router (fused, or split over d_model)
-        tc_splits = router_tc_splits(c);
+        // bf16 layers with enough tokens: tensor-core router (fused, or logits for the top-k kernel)
+        const int tc_splits = router_tc_splits(c);
         char* part_tc = ws + L.r_part + align_up(router_tc_wsplit_bytes(c));
         cudaError_t e = launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids,
                                          w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats,
                                          ws + L.r_part, part_tc, reinterpret_cast<int*>(ws + L.status), s);
         if (e != cudaSuccess) return e;
         nb = router_tc_blocks(c);
-        if (tc_splits > 1) {
+        if (router_tc_partial(c)) {
             nb = rp.nb_topk;
             e = launch_topk(c, o, reinterpret_cast<const float*>(part_tc), tc_splits, bias, noise, logits_out,
                             probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats, rp, s);

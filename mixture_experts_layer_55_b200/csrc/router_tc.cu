@@ -16,10 +16,11 @@
 //   router_wsplit_kernel  W_r (D, E) fp32 -> (3, D, EP) bf16, EP = E rounded
 //                         up to 64 (zero columns), N-major for TMA.
 //   router_tc_kernel      one CTA per 128 tokens (and per split of d_model when
-//                         the token tiles leave most SMs idle: the splits write
-//                         fp32 partial logits, which the top-k kernel of the
-//                         SIMT router sums in split order and routes; the fused
-//                         epilogue below runs otherwise): warp 0 TMA (x tile 128 x 64,
+//                         the token tiles leave most SMs idle).  With splits,
+//                         or more than 16 experts, it writes fp32 (partial)
+//                         logits, which the top-k kernel of the SIMT router sums
+//                         in split order and routes; otherwise the fused
+//                         epilogue below routes: warp 0 TMA (x tile 128 x 64,
 //                         three 64 x EP weight tiles per stage), warp 1
 //                         tcgen05.mma M=128, N=EP, three per K step into one
 //                         accumulator; warps 2..5 own one token row each:
@@ -465,6 +466,15 @@ int router_tc_splits(const moe_config& c)
     return (nkb + per - 1) / per;
 }
 
+bool router_tc_partial(const moe_config& c)
+{
+    // the fused epilogue gives each token to one thread, which walks all E
+    // experts several times; above 16 experts the SIMT top-k kernel (a warp
+    // per token, the experts spread over its lanes) routes faster from the
+    // logits the tensor cores wrote
+    return router_tc_splits(c) > 1 || c.E > 16;
+}
+
 size_t router_tc_wsplit_bytes(const moe_config& c)
 {
     const int ep = (c.E + 63) / 64 * 64;
@@ -489,7 +499,7 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
     const int nkb = (c.D + BK - 1) / BK;
     Args a{o, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt,
            c.T, c.D, c.E, c.K, with_stats, status,
-           splits > 1 ? static_cast<float*>(part_out) : nullptr, (nkb + splits - 1) / splits};
+           router_tc_partial(c) ? static_cast<float*>(part_out) : nullptr, (nkb + splits - 1) / splits};
     return ep == 64 ? launch_t<1>(c, x, wsplit, a, s) : launch_t<2>(c, x, wsplit, a, s);
 }
 
