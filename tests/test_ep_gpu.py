@@ -21,7 +21,7 @@ import torch.distributed as dist
 import oracle
 from mixture_experts_layer_55_b200 import _binding as B
 from mixture_experts_layer_55_b200.ep import ExpertParallelMoE
-from workloads import Workload, make_inputs, make_tokens
+from workloads import WORKLOADS, Workload, make_inputs, make_tokens
 
 from tests.test_ep_cpu import receive_layout
 from tests.gpu_common import to_np
@@ -132,14 +132,15 @@ def _expected_remote_rows(kept_all, ids, row_of, offsets, rank, W, EL):
     return out, [lay[0] for lay in layouts]
 
 
-def _emulated_peer_layer(wl, W, bias=None, token_seed=77):
+def _emulated_peer_layer(wl, W, bias=None, token_seed=77, device_inputs=False):
     """W ranks of the peer-exchange layer emulated on one GPU: each rank has its
     own tokens; every rank's receive and output buffers live on this device,
     so the kernels' stores into and loads from "peer" buffers are ordinary
     device accesses.  The ranks' kernels run one after another in stream
-    order; none waits on another."""
+    order; none waits on another.  device_inputs: draw the inputs on the GPU
+    (full sizes; no host copies are kept)."""
     dev = "cuda"
-    inp = make_inputs(wl)
+    inp = make_inputs(wl, device=dev if device_inputs else "cpu")
     if bias is not None:
         inp["bias"] = bias
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
@@ -151,8 +152,8 @@ def _emulated_peer_layer(wl, W, bias=None, token_seed=77):
     i32 = dict(dtype=torch.int32, device=dev)
     ranks = []
     for r in range(W):
-        x = make_tokens(wl, device="cpu", seed=token_seed * 16 + r)
-        st = dict(x_cpu=x, x=x.to(dev), ids=torch.empty(T, K, **i32),
+        x = make_tokens(wl, device=dev if device_inputs else "cpu", seed=token_seed * 16 + r)
+        st = dict(x_cpu=None if device_inputs else x, x=x.to(dev), ids=torch.empty(T, K, **i32),
                   w=torch.empty(T, K, dtype=torch.float32, device=dev),
                   counts=torch.empty(E, **i32), kept=torch.empty(E, **i32),
                   offsets=torch.empty(E + 1, **i32), perm=torch.empty(B.max_rows(cfg), **i32),
@@ -239,6 +240,46 @@ def test_peer_exchange_emulated_ranks(name):
         assert any((st["row_of"] < 0).any().item() for st in ranks), "case must drop assignments"
     if name == "w4_skewed":
         assert kept_all[:, : wl.E - EL].sum() == 0, "every row must go to the last rank"
+
+
+def test_peer_exchange_full_size():
+    """The Mixtral-shaped layer (T = 8192 tokens per rank, D = 4096, F = 14336,
+    E = 8, K = 2) as two emulated ranks of four experts each: the receive
+    layout against its definition, every output element against the local
+    training forward of the same tokens (which weights the expert outputs in
+    the combine the same way), and sampled tokens against the oracle (dropless
+    routing makes each token's output depend on that token alone)."""
+    wl = WORKLOADS["mixtral_8x"]
+    W = 2
+    cfg, inp, g, ranks, kept_all = _emulated_peer_layer(wl, W, device_inputs=True)
+    EL = wl.E // W
+    wg, wu, wd = (g[k].cpu() for k in ("w_gate", "w_up", "w_down"))
+    for r, st in enumerate(ranks):
+        ids = st["ids"].cpu().numpy()
+        row_of = st["row_of"].cpu().numpy()
+        offsets = st["offsets"].cpu().numpy()
+        exp_rows, exp_offsets = _expected_remote_rows(kept_all, ids, row_of, offsets, r, W, EL)
+        np.testing.assert_array_equal(st["remote_row"].cpu().numpy(), exp_rows)
+        np.testing.assert_array_equal(st["local_offsets"].cpu().numpy(), exp_offsets[r])
+        state = torch.zeros(B.train_state_size(cfg), dtype=torch.uint8, device="cuda")
+        yt = torch.empty_like(st["x"])
+        B.moe_forward_train(cfg, st["x"], g["w_router"], g["w_gate"], g["w_up"], g["w_down"], yt, state,
+                            router_bias=g["bias"])
+        torch.cuda.synchronize()
+        assert B.moe_get_device_status(state) == 0
+        got = to_np(st["y"])
+        m = float(np.abs(got).max())
+        assert np.abs(got - to_np(yt)).max() <= 1e-3 * m + 1e-4
+        del state
+        rng = np.random.default_rng(100 + r)
+        tok = np.sort(rng.choice(wl.T, 3, replace=False))
+        L = st["L"][torch.from_numpy(tok).cuda()].cpu().numpy()
+        ref = oracle.forward(st["x"][torch.from_numpy(tok).cuda()].cpu(), g["w_router"].cpu(), wg, wu, wd,
+                             wl.K, 0.0, logits=L)
+        assert np.array_equal(ids[tok], ref["ids"])
+        mref = float(np.abs(ref["y"]).max())
+        assert np.abs(got[tok] - ref["y"]).max() <= 1e-2 * mref + 1e-3
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("wl", [
