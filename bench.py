@@ -235,6 +235,11 @@ def run_gpu(args):
     for i in range(args.warmup):
         layer.forward(xs[i % nbuf], y, logit_noise=noise)
     torch.cuda.synchronize(dev)
+    # --graph: one CUDA graph of the whole forward per input buffer, replayed
+    graphs = [layer.capture(xs[i], y, logit_noise=noise) for i in range(nbuf)] if args.graph else []
+    for i in range(args.warmup if graphs else 0):
+        graphs[i % nbuf].replay()
+    torch.cuda.synchronize(dev)
     nb = M._binding.lib().moe_trace_boundary_count()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -245,14 +250,24 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     start.record(stream)
     for i in range(args.steps):
-        M.moe_trace_attach(evs[i])
-        layer.forward(xs[i % nbuf], y, logit_noise=noise)
+        if graphs:
+            graphs[i % nbuf].replay()
+        else:
+            M.moe_trace_attach(evs[i])
+            layer.forward(xs[i % nbuf], y, logit_noise=noise)
     stop.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     M.moe_trace_attach([])
     clk = clocks.stop()
     ms_total, ms_step, value = aggregate(start.elapsed_time(stop), world, wl.T, args.steps, dev)
+    if graphs:  # stage times from eager steps (events are not recorded inside the graphs)
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            M.moe_trace_attach(evs[i])
+            layer.forward(xs[i % nbuf], y, logit_noise=noise)
+        torch.cuda.synchronize(dev)
+        M.moe_trace_attach([])
 
     names = M.trace_stage_names()
     stage_ms = {}
@@ -356,6 +371,7 @@ def run_gpu(args):
         "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
                    "capacity_factor": wl.capacity_factor, "router_bias": wl.bias,
                    "logit_noise": wl.noise, "parallelism": f"replicas x{world}",
+                   "launch": "cuda_graph" if graphs else "stream",
                    "l2": "inputs larger than L2 (expert weights "
                          f"{3 * wl.E * wl.D * wl.F * wl.elem_bytes / 1e9:.2f} GB read per step)"},
         "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
@@ -895,6 +911,8 @@ def main(argv=None):
                     help="forward (default) or a training step (forward + backward)")
     ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
                     help="replicas (default): every GPU holds all experts; ep: experts sharded")
+    ap.add_argument("--graph", action="store_true",
+                    help="forward: time replays of a CUDA graph of the whole layer")
     ap.add_argument("--exchange", choices=["all_to_all", "peer"], default="all_to_all",
                     help="with --parallel ep: NCCL all-to-all, or the library's kernels over "
                          "peer-mapped buffers")

@@ -61,6 +61,24 @@ class MoELayer:
                       counts=self.counts if stats else None, stream=stream)
         return y
 
+    def capture(self, x, y, logit_noise=None, stats: bool = True):
+        """One forward over the buffers x -> y captured as a CUDA graph; returns
+        the torch.cuda.CUDAGraph (graph.replay() runs the layer again on
+        whatever x then holds).  The forward takes no host decision between
+        its launches and never synchronises, so all of them form one graph;
+        the first call runs outside the capture (one-time kernel attributes).
+        Trace events must not be attached while capturing."""
+        dev = self.device
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            self.forward(x, y, logit_noise=logit_noise, stats=stats)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(x, y, logit_noise=logit_noise, stats=stats)
+        return graph
+
     def forward_host(self, x_host, y_host, x_dev=None, y_dev=None, logit_noise=None,
                      stream=None):
         """End to end from host memory: copy x_host (pinned) in, run the layer,

@@ -269,3 +269,26 @@ def test_host_stream_matches_device_forward(cuda_ok):
         y = layer.forward(x.cuda())
         torch.cuda.synchronize()
         assert torch.equal(y.cpu(), yh)
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "ragged_bf16"])
+def test_cuda_graph_replay_matches_eager(cuda_ok, name):
+    """MoELayer.capture: the whole forward as one CUDA graph; replays on new
+    contents of the captured input give the eager forward's output bit for bit."""
+    from mixture_experts_layer_55_b200 import MoELayer
+    from workloads import make_tokens
+    wl = WORKLOADS[name] if name in WORKLOADS else next(w for w in SMALL if w.name == name)
+    inp = _to_dev(make_inputs(wl))
+    layer = MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
+                     wl.capacity_factor, router_bias=inp["bias"])
+    x = inp["x"].clone()
+    y = torch.empty_like(x)
+    graph = layer.capture(x, y)
+    for seed in (11, 12):
+        xn = make_tokens(wl, device="cuda", seed=seed)
+        x.copy_(xn)
+        graph.replay()
+        y_eager = layer.forward(xn)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_eager)
+    assert B.moe_get_device_status(layer.workspace) == 0
