@@ -65,6 +65,8 @@ class CudaOps:
         self.offsets_local = torch.empty(EL + 1, **i32)
         self.dst_of = torch.empty(self.max_recv, **i32)
         self.src_of = torch.empty(self.max_recv, **i32)
+        self.remote_row = None  # peer exchange: row of each slot in its owner's buffer
+        self.h_local = None     # peer exchange: the local experts' hidden activations
 
     def route_dispatch(self, x, w_router, router_bias, selection_bias, logit_noise):
         x_perm = torch.empty((self.max_rows, x.shape[1]), dtype=x.dtype, device=x.device)
@@ -121,14 +123,14 @@ class CudaOps:
         return self.kept
 
     def peer_dispatch(self, x, kept_all, rank, W, peer):
-        if not hasattr(self, "remote_row"):
+        if self.remote_row is None:
             self.remote_row = torch.empty_like(self.row_of)
         B.moe_ep_peer_dispatch(self.cfg, rank, W, kept_all, x, self.ids, self.row_of, self.offsets,
                                peer.recv_ptrs, peer.rows, self.offsets_local, self.remote_row,
                                self.ws_ep)
 
     def peer_experts(self, peer, w_gate, w_up, w_down):
-        if not hasattr(self, "h_local"):
+        if self.h_local is None:
             self.h_local = torch.empty((self.max_recv, w_gate.shape[2]), dtype=w_gate.dtype,
                                        device=self.device)
         B.moe_expert_ffn(self.cfg_local, peer.recv_x, self.offsets_local, None, None, w_gate, w_up,
