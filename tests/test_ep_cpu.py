@@ -159,3 +159,47 @@ def test_receive_layout_definition():
     assert offsets.tolist() == [0, 4, 6]
     assert dst_of.tolist() == [0, 4, 5, 1, 2, 3]
     assert src_of.tolist() == [0, 3, 4, 5, 1, 2]
+
+
+def _peer_rows(kept_all, ids, row_of, offsets, rank, W, EL):
+    """The peer exchange's placement as include/moe.h states it: slot (t, k) of
+    source `rank`, routed to expert e of owner o = e // EL and kept at local row
+    r, lands at  sum_{o*EL <= e' < e} sum_s kept[s][e'] + sum_{s < rank}
+    kept[s][e] + (r - offsets[e])  of o's buffer."""
+    out = np.full(row_of.shape, -1, np.int64)
+    for i, r in enumerate(row_of):
+        if r < 0:
+            continue
+        e = int(ids.reshape(-1)[i])
+        o = e // EL
+        out[i] = kept_all[:, o * EL:e].sum() + kept_all[:rank, e].sum() + (r - offsets[e])
+    return out
+
+
+@pytest.mark.parametrize("W,EL,seed", [(2, 4, 0), (4, 2, 1), (8, 1, 2), (3, 5, 3)])
+def test_peer_placement_formula_equals_all_to_all_layout(W, EL, seed):
+    """The closed-form placement of the peer exchange agrees with the all-to-all
+    path's layout: rows leave each source expert-major, arrive source-major,
+    and the owner's receive layout moves them to expert-major order."""
+    rng = np.random.default_rng(seed)
+    E, T, K = W * EL, 50, min(2, W * EL)
+    kept_all = np.zeros((W, E), np.int64)
+    for rank in range(W):
+        ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)])
+        d = oracle.dispatch(ids.astype(np.int32), E, oracle.capacity(T, K, E, 0.6))
+        kept_all[rank] = d["kept"]
+    # each source's own layout again, to place its slots
+    rng = np.random.default_rng(seed)
+    for rank in range(W):
+        ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)])
+        d = oracle.dispatch(ids.astype(np.int32), E, oracle.capacity(T, K, E, 0.6))
+        got = _peer_rows(kept_all, ids, d["row_of"], d["offsets"], rank, W, EL)
+        for i, r in enumerate(d["row_of"]):
+            if r < 0:
+                assert got[i] == -1
+                continue
+            o = int(ids.reshape(-1)[i]) // EL
+            recv_o = kept_all[:, o * EL:(o + 1) * EL]
+            arrival = int(recv_o[:rank].sum()) + (r - d["offsets"][o * EL])
+            _, dst_of, _ = receive_layout(recv_o, W, EL)
+            assert got[i] == dst_of[arrival]
