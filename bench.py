@@ -764,11 +764,37 @@ def cpu_baseline(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
         n += len(toks)
         batch = min(batch * 2, 64)
     per_token = t_route / wl.T + t_ffn / n
-    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": oracle.num_threads(),
+    cores = oracle.num_threads()
+    # the same on one thread: routing on the first tokens, the expert FFN on a few sampled ones
+    oracle.set_num_threads(1)
+    try:
+        n1 = min(wl.T, 1024)
+        t0 = time.perf_counter()
+        L1 = oracle.router_logits(cpu_inp["x"][:n1], cpu_inp["w_router"], cpu_inp["bias"],
+                                  None if cpu_inp["noise"] is None else cpu_inp["noise"][:n1])
+        ids1, _, probs1, lse1 = oracle.route(L1, wl.K)
+        oracle.router_stats(ids1, probs1, lse1, wl.E)
+        oracle.dispatch(ids1, wl.E, oracle.capacity(n1, wl.K, wl.E, wl.capacity_factor))
+        t_route1 = time.perf_counter() - t0
+        m, t_ffn1, budget1 = 0, 0.0, max(0.5, seconds / 5)
+        while t_ffn1 < budget1 and m < wl.T:
+            tok = [int(order[m])]
+            t1 = time.perf_counter()
+            oracle.token_outputs(cpu_inp["x"][tok], ids[tok], w[tok], kept[tok], get)
+            t_ffn1 += time.perf_counter() - t1
+            m += 1
+    finally:
+        oracle.set_num_threads(cores)
+    per_token1 = t_route1 / n1 + t_ffn1 / m
+    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": (f"router + routing + dispatch layout on all {wl.T} tokens "
                        f"({t_route:.2f} s), expert FFN + combine on {n} sampled tokens "
-                       f"({t_ffn:.2f} s); value extrapolated per token")}
+                       f"({t_ffn:.2f} s); value extrapolated per token"),
+            "single_thread": {"value": round(1.0 / per_token1, 3), "unit": UNIT, "cores": 1,
+                              "sample": (f"routing on {n1} tokens ({t_route1:.2f} s), expert FFN + "
+                                         f"combine on {m} sampled tokens ({t_ffn1:.2f} s); "
+                                         "value extrapolated per token")}}
 
 
 def cpu_baseline_train(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:

@@ -86,6 +86,8 @@ def _load():
             lib.oracle_expert_wgrad.restype = None
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = i32
+            lib.oracle_set_num_threads.argtypes = [i32]
+            lib.oracle_set_num_threads.restype = None
             _lib = lib
     return _lib
 
@@ -155,6 +157,12 @@ def _ptr(a):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops from now on (results do not
+    depend on it)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def router_logits(x, w_router, bias=None, noise=None) -> np.ndarray:

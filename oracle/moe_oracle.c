@@ -738,3 +738,15 @@ int32_t oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads for the following parallel loops (no effect without OpenMP).  The
+   results do not depend on it: every parallel loop owns disjoint outputs. */
+void oracle_set_num_threads(int32_t n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n < 1 ? 1 : (int)n);
+#else
+    (void)n;
+#endif
+}
