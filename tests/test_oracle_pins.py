@@ -389,3 +389,23 @@ def test_shared_expert_adds_a_dense_swiglu():
     dense = _swiglu_torch(inp["x"].double(), *sh)
     np.testing.assert_allclose(b["y"] - a["y"], dense.numpy(), rtol=0, atol=1e-12)
     np.testing.assert_allclose(b["y_shared"], dense.numpy(), rtol=0, atol=1e-12)
+
+
+def test_results_do_not_depend_on_thread_count():
+    """Every parallel loop of the oracle owns disjoint outputs: one thread and
+    several give the same bits."""
+    from workloads import Workload, make_inputs
+    wl = Workload("threads", T=96, D=64, F=48, E=8, K=2, capacity_factor=0.75, bias="zipf", seed=3)
+    inp = make_inputs(wl)
+    n = oracle.num_threads()
+    try:
+        oracle.set_num_threads(1)
+        a = oracle.forward(inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
+                           wl.capacity_factor, bias=inp["bias"])
+        oracle.set_num_threads(4)
+        b = oracle.forward(inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
+                           wl.capacity_factor, bias=inp["bias"])
+    finally:
+        oracle.set_num_threads(n)
+    for k in ("logits", "ids", "weights", "row_of", "o", "y", "z_loss", "balance_loss"):
+        assert np.array_equal(a[k], b[k]), k
