@@ -460,11 +460,9 @@ class DeviceBuffer:
 def as_tensor(ptr: int, shape, dtype):
     """Tensor view of `shape` elements of `dtype` at device address ptr."""
     import torch
-    typestr = {torch.bfloat16: "<V2", torch.float32: "<f4", torch.int32: "<i4",
-               torch.uint8: "|u1"}[dtype]
     if dtype == torch.bfloat16:  # the array interface has no bf16: view int16 as bf16
-        t = torch.as_tensor(DeviceBuffer(ptr, shape, "<i2"), device="cuda")
-        return t.view(torch.bfloat16)
+        return torch.as_tensor(DeviceBuffer(ptr, shape, "<i2"), device="cuda").view(torch.bfloat16)
+    typestr = {torch.float32: "<f4", torch.int32: "<i4", torch.uint8: "|u1"}[dtype]
     return torch.as_tensor(DeviceBuffer(ptr, shape, typestr), device="cuda")
 
 
