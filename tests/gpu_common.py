@@ -18,7 +18,7 @@ import torch
 
 import oracle
 from mixture_experts_layer_55_b200 import _binding as B
-from workloads import Workload, make_inputs
+from workloads import Workload
 
 U32 = 2.0 ** -24
 
