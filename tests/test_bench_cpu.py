@@ -1,0 +1,48 @@
+"""bench.py's host-side bookkeeping on the CPU: the DRAM traffic recorded under
+profiles/ is reported only while the measured kernels' sources are unchanged,
+and the whole-job aggregate is the slowest rank's time over all ranks' tokens."""
+import json
+
+import bench
+
+
+def test_recorded_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    h = bench.kernel_source_hash()
+    assert len(h) == 16 and h == bench.kernel_source_hash()  # deterministic
+    assert bench.kernel_source_hash(bench.WGRAD_SOURCES) != h  # other kernels, other hash
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"wl": {"expert_gate_up": {"dram_bytes_per_launch": 123, "source_hash": h},
+                  "expert_down": {"dram_bytes_per_launch": 456, "source_hash": "0" * 16}}}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the sources are read from the package, the record from the patched root: link them
+    real = bench.kernel_source_hash
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files=bench.GEMM_SOURCES: h)
+    assert bench.recorded_traffic("wl", "expert_gate_up") == 123
+    assert bench.recorded_traffic("wl", "expert_down") is None       # stale record
+    assert bench.recorded_traffic("wl", "missing") is None
+    assert bench.recorded_traffic("other", "expert_gate_up") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", real)
+
+
+def test_committed_traffic_record_is_consistent():
+    """The committed record is self-consistent, and the bench reports it only
+    while the forward GEMMs' sources hash to what it was taken on (after a
+    kernel change and before a new capture, traffic is null)."""
+    with open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    e = rec["mixtral_8x"]["expert_gate_up"]
+    assert e["dram_bytes_per_launch"] == e["read"] + e["write"]
+    assert e["dram_bytes_per_launch"] >= e["algorithmic_bytes"] * 0.5
+    got = bench.recorded_traffic("mixtral_8x", "expert_gate_up")
+    if e["source_hash"] == bench.kernel_source_hash():
+        assert got == e["dram_bytes_per_launch"]
+    else:
+        assert got is None
+
+
+def test_aggregate_single_rank():
+    ms_total, ms_step, value = bench.aggregate(100.0, 1, 8192, 20, "cpu")
+    assert ms_total == 100.0 and ms_step == 5.0
+    assert abs(value - 8192 / 5e-3) < 1e-6
