@@ -253,12 +253,15 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
                                const void *y_add, void *y, void *stream);
 
 /*
- * The whole layer: moe_route -> moe_dispatch -> moe_expert_ffn -> (shared
- * expert) -> moe_combine on one stream, every intermediate in the workspace
+ * The whole layer ("Lab: build a tiny MoE in PyTorch", "Full implementation";
+ * "2.9 Mixture-of-Experts (MoE) Architectures", "A Toy MoE Layer From
+ * Scratch"): moe_route -> moe_dispatch -> moe_expert_ffn -> (shared expert)
+ * -> moe_combine on one stream, every intermediate in the workspace
  * (moe_forward_workspace_size bytes).  With cfg->F_shared > 0,
  * w_gate_shared / w_up_shared (D, F_shared) and w_down_shared (F_shared, D)
  * are required and the shared SwiGLU expert's output over all tokens is
- * added in the combine; otherwise they are ignored (may be NULL).  y (T, D) dtype is required; losses (3),
+ * added in the combine; otherwise they are ignored (may be NULL).  y (T, D)
+ * dtype is required; losses (3),
  * mean_prob (E), counts (E, before drops), topk_ids (T, K) and topk_w (T, K)
  * are optional copies of the routing results (NULL to skip).
  */
@@ -293,7 +296,8 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
 MOE_API moe_status moe_train_state_size(const moe_config *cfg, size_t *bytes);
 
 /*
- * moe_forward for training: the same arguments and results, with the
+ * moe_forward for training ("Lab: build a tiny MoE in PyTorch", "Smoke test
+ * and backward pass"): the same arguments and results, with the
  * workspace replaced by `state` (moe_train_state_size bytes, 256-byte
  * aligned), which keeps what moe_backward reads: the routing results, the
  * dispatch layout, x_perm, [g | u] = the gate/up pre-activations in the
@@ -393,7 +397,8 @@ MOE_API moe_status moe_permute_rows(const void *in, int64_t in_rows, const int32
                                     int64_t row_bytes, void *out, void *workspace, void *stream);
 
 /*
- * moe_combine with the routing weight applied here: y[t] = y_add[t] + sum over
+ * moe_combine with the routing weight applied here (the combine's weighted
+ * index_add_ of "Full implementation"): y[t] = y_add[t] + sum over
  * kept slots of topk_w[t, k] * y_perm[row_of[t, k]], fp32, rounded once.  For
  * unweighted expert outputs (the rows that come back from the experts' owners).
  */
@@ -446,7 +451,9 @@ MOE_API moe_status moe_ipc_close(void *ptr);
 MOE_API moe_status moe_ipc_free(void *ptr);
 
 /*
- * Dispatch of this rank's tokens into the owners' receive buffers.
+ * Dispatch of this rank's tokens into the owners' receive buffers (the
+ * all-to-all dispatch of "From local loop to expert parallelism", done by
+ * stores into the owners' memory).
  *   cfg            this rank's layer: T tokens, all E experts (E % world == 0)
  *   rank, world    this rank and the number of ranks (1 <= world <= 64)
  *   kept_all       (world, E) int32, device: every rank's kept counts
@@ -476,7 +483,9 @@ MOE_API moe_status moe_ep_peer_dispatch(const moe_config *cfg, int32_t rank, int
                                         size_t workspace_bytes, void *stream);
 
 /*
- * Weighted combine from the owners' output buffers: y[t] = y_add[t] + sum over
+ * Weighted combine from the owners' output buffers (the reverse all-to-all and
+ * scatter-add of "From local loop to expert parallelism", done by loads from
+ * the owners' memory): y[t] = y_add[t] + sum over
  * kept slots, in slot order, of topk_w[t, k] * y_bufs[owner][remote_row[t, k]],
  * fp32 sums rounded once to cfg.dtype.  y_bufs: device array of `world`
  * device pointers to the owners' moe_expert_ffn outputs (unweighted:
