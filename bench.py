@@ -176,6 +176,9 @@ def algorithmic(wl: Workload, counts, kept_rows: int):
         # x_perm read once, h written once
         "gateup_bytes": float(sum(1 for c in counts if c > 0) * 2 * wl.D * wl.F * s
                               + R * wl.D * s + R * wl.F * s),
+        # router: x read once, fp32 router weight, routed ids and weights written
+        "route_bytes": float(wl.T * wl.D * s + wl.D * wl.E * 4 + wl.T * wl.K * 8),
+        "shared_flop": 6.0 * wl.T * wl.D * wl.F_shared,
     }
 
 
@@ -212,108 +215,31 @@ def recorded_traffic(workload: str, kernel: str, files=GEMM_SOURCES):
     return e.get("dram_bytes_per_launch")
 
 
-def run_gpu(args):
-    import mixture_experts_layer_55_b200 as M
+# the other layer shapes measured after the headline one, in the same process
+# (each freed before the next); the Mixtral shape again with a shared expert of
+# its own hidden size measures the shared-expert stage
+EXTRA_CONFIGS = ("fine_skewed", "stmoe_capacity", "decode_e256", "tiny_fp32",
+                 "mixtral_8x+shared")
+# latency-bound shapes: timed as replays of one CUDA graph of the whole layer
+GRAPH_CONFIGS = ("tiny_fp32", "decode_e256")
+L2_BYTES = 126 * 1024 * 1024
 
-    rank, world, local_rank = rank_info()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    init_dist(world, "nccl")
-    wl = workload_of(args)
 
-    inp = make_inputs(wl, device=dev)
-    layer = M.MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
-                       wl.capacity_factor, router_bias=inp["bias"])
-    noise = inp["noise"]
-    # a few batches of tokens, rotated between steps
-    nbuf = 3
-    xs = [make_tokens(wl, device=dev, seed=rank_token_seed(rank) * 16 + i) for i in range(nbuf)]
-    y = torch.empty_like(xs[0])
-    stream = torch.cuda.current_stream(dev)
+def config_workload(name: str) -> Workload:
+    if name == "mixtral_8x+shared":
+        return WORKLOADS["mixtral_8x"].with_(name=name, F_shared=WORKLOADS["mixtral_8x"].F)
+    return WORKLOADS[name]
 
-    # ---------------- device-resident timing (value) ----------------
-    for i in range(args.warmup):
-        layer.forward(xs[i % nbuf], y, logit_noise=noise)
-    torch.cuda.synchronize(dev)
-    # --graph: one CUDA graph of the whole forward per input buffer, replayed
-    graphs = [layer.capture(xs[i], y, logit_noise=noise) for i in range(nbuf)] if args.graph else []
-    for i in range(args.warmup if graphs else 0):
-        graphs[i % nbuf].replay()
-    torch.cuda.synchronize(dev)
-    nb = M._binding.lib().moe_trace_boundary_count()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    time.sleep(0.3)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    start.record(stream)
-    for i in range(args.steps):
-        if graphs:
-            graphs[i % nbuf].replay()
-        else:
-            M.moe_trace_attach(evs[i])
-            layer.forward(xs[i % nbuf], y, logit_noise=noise)
-    stop.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    M.moe_trace_attach([])
-    clk = clocks.stop()
-    ms_total, ms_step, value = aggregate(start.elapsed_time(stop), world, wl.T, args.steps, dev)
-    if graphs:  # stage times from eager steps (events are not recorded inside the graphs)
-        torch.cuda.synchronize(dev)
-        for i in range(args.steps):
-            M.moe_trace_attach(evs[i])
-            layer.forward(xs[i % nbuf], y, logit_noise=noise)
-        torch.cuda.synchronize(dev)
-        M.moe_trace_attach([])
 
-    names = M.trace_stage_names()
-    stage_ms = {}
-    for j in range(1, nb):
-        d = [evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(args.steps)]
-        stage_ms[names[j]] = sum(d) / len(d)
-
-    counts = layer.counts.cpu().tolist()
-    kept_rows = int(min(sum(min(c, M.capacity(layer.cfg)) for c in counts), M.max_rows(layer.cfg)))
-    alg = algorithmic(wl, counts, kept_rows)
-
-    # ---------------- end to end from pinned host memory (e2e) ----------------
-    # every step copies its batch in from pinned host memory and its result out;
-    # copies of neighbouring steps overlap the forward (MoELayer.forward_host_stream)
-    x_hosts = [xs[i % nbuf].cpu().pin_memory() for i in range(nbuf)]
-    y_hosts = [torch.empty_like(x_hosts[0]).pin_memory() for _ in range(nbuf)]
-    seq_in = [x_hosts[i % nbuf] for i in range(args.steps)]
-    seq_out = [y_hosts[i % nbuf] for i in range(args.steps)]
-    layer.forward_host_stream(seq_in[:max(2, args.warmup)], seq_out[:max(2, args.warmup)],
-                              logit_noise=noise)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    layer.forward_host_stream(seq_in, seq_out, logit_noise=noise, events=(e0, e1))
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-    io_bytes = wl.T * wl.D * wl.elem_bytes
-
-    flags = M.moe_get_device_status(layer.workspace)
-    if flags:
-        raise RuntimeError(f"device status flags {flags:#x} after the benchmark")
-
-    if rank != 0:
-        _finish(world)
-        return
-
+def forward_roofline(wl: Workload, alg: dict, stage_ms: dict, ms_total: float):
+    """Roofline of the dominant kernel, the gate/up GEMM, against the roof its
+    arithmetic intensity selects (the ridge of the two measured peaks)."""
     peaks, peak_src = load_peaks()
-    long_region = ms_total > 1000.0
+    gu_ms = stage_ms["expert_gate_up"]
     if wl.dtype == "bf16":
-        key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        key = "bf16_tflops_sustained" if ms_total > 1000.0 else "bf16_tflops"
         peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
-        gu_ms = stage_ms["expert_gate_up"]
         hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        # which roof binds: the kernel's arithmetic intensity against the
-        # ridge point of the two measured peaks
         intensity = alg["gateup_flop"] / alg["gateup_bytes"]
         ridge = peak * 1e12 / (hbm_peak * 1e9)
         if intensity >= ridge:
@@ -330,17 +256,20 @@ def run_gpu(args):
                         "peak_source": f"hbm_gbs of {peak_src}"}
         roofline.update(intensity_flop_per_byte=round(intensity, 1), ridge=round(ridge, 1),
                         traffic=recorded_traffic(wl.name, "expert_gate_up"))
-    else:
-        # fp32 layer: SIMT FMA pipes; peak from unit counts and the clock:
-        # 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock
-        sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
-        peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
-        gu_ms = stage_ms["expert_gate_up"]
-        achieved = alg["gateup_flop"] / (gu_ms / 1e3) / 1e12
-        roofline = {"kernel": "expert_gate_up (fp32 SIMT)", "bound": "alu",
-                    "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
-                    "frac": round(achieved / peak, 4), "peak_source": "148 SMs x 128 FMA x 2 x max clock",
-                    "traffic": recorded_traffic(wl.name, "expert_gate_up")}
+        return roofline
+    # fp32 layer: SIMT FMA pipes; peak from unit counts and the clock:
+    # 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock
+    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    achieved = alg["gateup_flop"] / (gu_ms / 1e3) / 1e12
+    return {"kernel": "expert_gate_up (fp32 SIMT)", "bound": "alu",
+            "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_source": "148 SMs x 128 FMA x 2 x max clock",
+            "traffic": recorded_traffic(wl.name, "expert_gate_up")}
+
+
+def stage_table(wl: Workload, alg: dict, stage_ms: dict) -> dict:
+    peaks, _ = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     stages = {}
     for name, ms in stage_ms.items():
@@ -351,48 +280,230 @@ def run_gpu(args):
         elif name == "combine":
             gbs = alg["combine_bytes"] / (ms / 1e3) / 1e9
             ent.update(GBs=round(gbs, 1), hbm_frac=round(gbs / hbm, 4))
+        elif name == "route":
+            gbs = alg["route_bytes"] / (ms / 1e3) / 1e9
+            ent.update(GBs=round(gbs, 1), hbm_frac=round(gbs / hbm, 4))
         elif name == "expert_gate_up":
             ent.update(TFLOPs=round(alg["gateup_flop"] / (ms / 1e3) / 1e12, 1))
         elif name == "expert_down":
             ent.update(TFLOPs=round(alg["down_flop"] / (ms / 1e3) / 1e12, 1))
+        elif name == "shared_expert" and alg["shared_flop"]:
+            ent.update(TFLOPs=round(alg["shared_flop"] / (ms / 1e3) / 1e12, 1))
         stages[name] = ent
+    return stages
+
+
+class _Flusher:
+    """Writes a buffer larger than L2 between timed steps (for layers whose
+    inputs fit in L2)."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def measure_forward(M, wl: Workload, args, rank: int, world: int, dev, *, headline: bool,
+                    graph: bool, cpu_seconds: float) -> dict:
+    """Time one layer shape.  Returns the fields of its JSON record (rank 0's
+    view; device times are the max over ranks)."""
+    inp = make_inputs(wl, device=dev)
+    layer = M.MoELayer(wl.T, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], wl.K,
+                       wl.capacity_factor, router_bias=inp["bias"], shared=inp["shared"])
+    noise = inp["noise"]
+    nbuf = 3  # a few batches of tokens, rotated between steps
+    xs = [make_tokens(wl, device=dev, seed=rank_token_seed(rank) * 16 + i) for i in range(nbuf)]
+    y = torch.empty_like(xs[0])
+    stream = torch.cuda.current_stream(dev)
+    weight_bytes = 3 * wl.E * wl.D * wl.F * wl.elem_bytes + 3 * wl.D * wl.F_shared * wl.elem_bytes
+    # inputs smaller than L2: flush it before every step and time the steps one by one
+    flush = None if weight_bytes > L2_BYTES else _Flusher(dev)
+    nb = M._binding.lib().moe_trace_boundary_count()
+
+    for i in range(args.warmup):
+        layer.forward(xs[i % nbuf], y, logit_noise=noise)
+    torch.cuda.synchronize(dev)
+    # steps: at least args.steps, and enough for >= 100 ms of timed work
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
+    layer.forward(xs[0], y, logit_noise=noise)
+    w1.record(stream)
+    torch.cuda.synchronize(dev)
+    est = max(w0.elapsed_time(w1), 1e-3)
+    steps = args.steps if headline else max(args.steps, min(2000, int(100.0 / est) + 1))
+    steps = int(max_over_ranks(float(steps), world, dev))
+
+    def timed(run_step, per_step_events=None):
+        """Device time of `steps` steps (ms, this rank), with the clock record."""
+        clocks = ClockSampler(dev.index if dev.index is not None else 0)
+        clocks.start()
+        time.sleep(0.3)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        if flush is None:
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for i in range(steps):
+                if per_step_events is not None:
+                    M.moe_trace_attach(per_step_events[i])
+                run_step(i)
+            t1.record(stream)
+            torch.cuda.synchronize(dev)
+            total = t0.elapsed_time(t1)
+        else:
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(steps)]
+            for i in range(steps):
+                flush()
+                if per_step_events is not None:
+                    M.moe_trace_attach(per_step_events[i])
+                pairs[i][0].record(stream)
+                run_step(i)
+                pairs[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            total = sum(a.elapsed_time(b) for a, b in pairs)
+        barrier(world)
+        M.moe_trace_attach([])
+        return total, clocks.stop()
+
+    # eager: stream launches, with per-stage events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(steps)]
+    eager_total, eager_clk = timed(lambda i: layer.forward(xs[i % nbuf], y, logit_noise=noise),
+                                   evs)
+    names = M.trace_stage_names()
+    stage_ms = {}
+    for j in range(1, nb):
+        d = [evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(steps)]
+        stage_ms[names[j]] = sum(d) / len(d)
+    launch = "stream"
+    total, clk = eager_total, eager_clk
+    eager_ms_step = max_over_ranks(eager_total, world, dev) / steps
+    if graph:
+        # one CUDA graph of the whole forward per input buffer, replayed
+        graphs = [layer.capture(xs[i], y, logit_noise=noise) for i in range(nbuf)]
+        for i in range(args.warmup):
+            graphs[i % nbuf].replay()
+        torch.cuda.synchronize(dev)
+        total, clk = timed(lambda i: graphs[i % nbuf].replay())
+        launch = "cuda_graph"
+        del graphs
+    ms_total, ms_step, value = aggregate(total, world, wl.T, steps, dev)
+
+    counts = layer.counts.cpu().tolist()
+    kept_rows = int(min(sum(min(c, M.capacity(layer.cfg)) for c in counts), M.max_rows(layer.cfg)))
+    alg = algorithmic(wl, counts, kept_rows)
+    rec = {"value": round(value, 1), "unit": UNIT, "ms_per_step": round(ms_step, 4),
+           "steps": steps, "launch": launch}
+    if graph:
+        rec["stream_ms_per_step"] = round(eager_ms_step, 4)
+
+    if headline:
+        # end to end from pinned host memory: every step copies its batch in and
+        # its result out; copies of neighbouring steps overlap the forward
+        # (MoELayer.forward_host_stream)
+        x_hosts = [xs[i % nbuf].cpu().pin_memory() for i in range(nbuf)]
+        y_hosts = [torch.empty_like(x_hosts[0]).pin_memory() for _ in range(nbuf)]
+        seq_in = [x_hosts[i % nbuf] for i in range(steps)]
+        seq_out = [y_hosts[i % nbuf] for i in range(steps)]
+        layer.forward_host_stream(seq_in[:max(2, args.warmup)], seq_out[:max(2, args.warmup)],
+                                  logit_noise=noise)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        layer.forward_host_stream(seq_in, seq_out, logit_noise=noise, events=(e0, e1))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+        io_bytes = wl.T * wl.D * wl.elem_bytes
+        rec["e2e"] = {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
+                      "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io_bytes,
+                      "d2h_bytes_per_step": io_bytes,
+                      "how": "MoELayer.forward_host_stream: per step, x in from pinned host "
+                             "memory, moe_forward, y out; copies overlap neighbouring steps' "
+                             "forwards"}
+
+    flags = M.moe_get_device_status(layer.workspace)
+    if flags:
+        raise RuntimeError(f"device status flags {flags:#x} after the benchmark ({wl.name})")
+
     ffn_ms = stage_ms["expert_gate_up"] + stage_ms["expert_down"]
-    weights_gbs = alg["active_weight_bytes"] / (ffn_ms / 1e3) / 1e9
-
-    cpu = None
-    if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, args.cpu_seconds)
-
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
-        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) random-init weights)",
+    rec.update({
         "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
                    "capacity_factor": wl.capacity_factor, "router_bias": wl.bias,
-                   "logit_noise": wl.noise, "parallelism": f"replicas x{world}",
-                   "launch": "cuda_graph" if graphs else "stream",
-                   "l2": "inputs larger than L2 (expert weights "
-                         f"{3 * wl.E * wl.D * wl.F * wl.elem_bytes / 1e9:.2f} GB read per step)"},
-        "e2e": {"value": round(world * wl.T / (e2e_ms / 1e3), 1), "unit": UNIT,
-                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": io_bytes,
-                "d2h_bytes_per_step": io_bytes,
-                "how": "MoELayer.forward_host_stream: per step, x in from pinned host memory, "
-                       "moe_forward, y out; copies overlap neighbouring steps' forwards"},
-        "gpu_launches": M.forward_kernel_count(layer.cfg) * args.steps,
-        "roofline": roofline,
-        "stages": stages,
+                   "logit_noise": wl.noise, "F_shared": wl.F_shared,
+                   "parallelism": f"replicas x{world}", "launch": launch,
+                   "l2": ("inputs larger than L2 (expert weights "
+                          f"{weight_bytes / 1e9:.2f} GB read per step)") if flush is None else
+                         ("inputs fit in L2: a 252 MB buffer is written before every step and "
+                          "the steps are timed one by one")},
+        "dtype": wl.dtype,
+        "gpu_launches": M.forward_kernel_count(layer.cfg) * steps,
+        "roofline": forward_roofline(wl, alg, stage_ms, ms_total),
+        "stages": stage_table(wl, alg, stage_ms),
         "layer": {"assignments_per_s": round(world * wl.T * wl.K / (ms_step / 1e3), 1),
                   "kept_rows": kept_rows, "max_over_mean_load": round(
                       max(counts) / (sum(counts) / len(counts)), 3),
-                  "expert_weights_GBs": round(weights_gbs, 1),
-                  "expert_tflops": round((alg["gateup_flop"] + alg["down_flop"]) / (ffn_ms / 1e3) / 1e12, 1)},
+                  "expert_weights_GBs": round(alg["active_weight_bytes"] / (ffn_ms / 1e3) / 1e9, 1),
+                  "expert_tflops": round((alg["gateup_flop"] + alg["down_flop"])
+                                         / (ffn_ms / 1e3) / 1e12, 1)},
         "clocks": clk,
-        "cpu_baseline": cpu,
+    })
+    if wl.capacity_factor > 0:
+        losses = layer.losses.cpu().tolist()
+        rec["layer"].update(capacity=M.capacity(layer.cfg), z_loss=round(losses[0], 6),
+                            balance_loss=round(losses[1], 6))
+    del layer, inp, xs, y
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and cpu_seconds > 0:
+        rec["cpu_baseline"] = cpu_baseline(wl, cpu_seconds)
+    else:
+        rec["cpu_baseline"] = None
+    return rec
+
+
+def run_gpu(args):
+    import mixture_experts_layer_55_b200 as M
+
+    rank, world, local_rank = rank_info()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    init_dist(world, "nccl")
+    wl = workload_of(args)
+    cpu_s = 0.0 if args.no_cpu_baseline else args.cpu_seconds
+    head = measure_forward(M, wl, args, rank, world, dev, headline=True, graph=args.graph,
+                           cpu_seconds=cpu_s)
+    extras = {}
+    if args.configs == "all" and not args.override and args.workload == "mixtral_8x":
+        for name in EXTRA_CONFIGS:
+            cw = config_workload(name)
+            extras[name] = measure_forward(M, cw, args, rank, world, dev, headline=False,
+                                           graph=name in GRAPH_CONFIGS,
+                                           cpu_seconds=0.0 if (args.no_cpu_baseline or
+                                                               cw.F_shared) else 4.0)
+    if rank != 0:
+        _finish(world)
+        return
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": head["steps"], "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) random-init weights)",
+        "config": head["config"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "roofline": head["roofline"],
+        "stages": head["stages"],
+        "layer": head["layer"],
+        "clocks": head["clocks"],
+        "cpu_baseline": head["cpu_baseline"],
     }
+    if extras:
+        line["configs"] = {k: {kk: vv for kk, vv in v.items()
+                               if kk not in ("unit",)} for k, v in extras.items()}
     if args.warmup < 3:
         line["note"] = "fewer than 3 warm-up steps: not a valid measurement"
-
     print(json.dumps(line), flush=True)
     _finish(world)
 
@@ -730,20 +841,68 @@ def _finish(world):
 
 # ------------------------------------------------------------ CPU oracle --
 
-def cpu_baseline(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
+def _run_experts(jobs, work, cores: int):
+    """Run work(e) for every (e, n_rows) in jobs on all `cores` host threads and
+    time it: an expert with at least `cores` rows runs alone, its rows spread
+    over the threads by the oracle's own OpenMP loop; experts with fewer rows
+    run `cores` at a time, concurrently, one OpenMP thread each (the oracle's
+    results do not depend on its thread count).  Returns ({e: result}, s)."""
+    import concurrent.futures as cf
+
+    import oracle
+    out, secs = {}, 0.0
+    big = [e for e, n in jobs if n >= cores or cores == 1]
+    small = [e for e, n in jobs if not (n >= cores or cores == 1)]
+    for e in big:
+        t0 = time.perf_counter()
+        out[e] = work(e)
+        secs += time.perf_counter() - t0
+    if small:
+        with cf.ThreadPoolExecutor(cores, initializer=oracle.set_num_threads,
+                                   initargs=(1,)) as ex:
+            t0 = time.perf_counter()
+            for e, r in zip(small, ex.map(work, small)):
+                out[e] = r
+            secs += time.perf_counter() - t0
+    return out, secs
+
+
+def _sample_tokens(wl: Workload, ids, kept, order, rows_target: float):
+    """Tokens of the CPU sample, in random order until about rows_target kept
+    rows, limited to the experts whose weights fit a 1.5 G-element host budget
+    (generating expert weights on the host is not timed, but it takes wall
+    time).  Returns the sorted tokens and the experts they need."""
+    e_cap = max(1, int(1.5e9 // (3 * wl.D * wl.F)))
+    toks, experts, rows = [], set(), 0
+    for t in order:
+        te = {int(ids[t, k]) for k in range(wl.K) if kept[t, k]}
+        if toks and len(experts | te) > e_cap:
+            continue
+        toks.append(int(t))
+        experts |= te
+        rows += len(te)
+        if rows >= rows_target:
+            break
+    return sorted(toks), sorted(experts)
+
+
+def cpu_baseline(wl: Workload, seconds: float = 15.0, seed: int = 0, cpu_inp=None) -> dict:
     """Time the oracle as it stands on a bounded sample of the workload.
 
     Router logits + routing + dispatch layout for all T tokens, then the expert
-    FFN and combine for a sample of tokens (grown until the time budget is
-    used).  value = tokens/s extrapolated from the per-token costs.
+    FFN and combine for a sample of tokens sized to the time budget (a first
+    call calibrates the per-row cost).  Every expert's sampled rows go to the
+    oracle in one call, using all host cores (_run_experts); the expert weights
+    are generated before the timed calls.  value = tokens/s extrapolated from
+    the per-token costs.
     """
     import numpy as np
 
     import oracle
-    torch.manual_seed(seed)
-    cpu_inp = _cpu_inputs_for_sample(wl)
+    cpu_inp = cpu_inp or _cpu_inputs_for_sample(wl)
+    x = cpu_inp["x"]
     t0 = time.perf_counter()
-    L = oracle.router_logits(cpu_inp["x"], cpu_inp["w_router"], cpu_inp["bias"], cpu_inp["noise"])
+    L = oracle.router_logits(x, cpu_inp["w_router"], cpu_inp["bias"], cpu_inp["noise"])
     ids, w, probs, lse = oracle.route(L, wl.K)
     oracle.router_stats(ids, probs, lse, wl.E)
     C = oracle.capacity(wl.T, wl.K, wl.E, wl.capacity_factor)
@@ -751,60 +910,87 @@ def cpu_baseline(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
     t_route = time.perf_counter() - t0
     kept = d["row_of"].reshape(wl.T, wl.K) >= 0
     get = cpu_inp["get_expert"]
-    n, t_ffn = 0, 0.0
-    budget = max(1.0, seconds - t_route)
+    cores = oracle.num_threads()
     rng = np.random.default_rng(seed)
     order = rng.permutation(wl.T)
-    batch = 1
-    while t_ffn < budget and n < wl.T:
-        toks = sorted(order[n:n + batch].tolist())
-        t1 = time.perf_counter()
-        oracle.token_outputs(cpu_inp["x"][toks], ids[toks], w[toks], kept[toks], get)
-        t_ffn += time.perf_counter() - t1
-        n += len(toks)
-        batch = min(batch * 2, 64)
+    # calibration: `cores` rows of one expert on all threads
+    e0 = int(ids[order[0], 0])
+    w0 = get(e0)
+    xcal = x[torch.from_numpy(order[:min(cores, wl.T)].copy())]
+    t1 = time.perf_counter()
+    oracle.expert_rows(xcal.double().numpy(), *w0)
+    sec_row = (time.perf_counter() - t1) / xcal.shape[0]
+    budget = max(1.0, seconds - t_route)
+    toks, experts = _sample_tokens(wl, ids, kept, order, 0.8 * budget / max(sec_row, 1e-9))
+    xs = x[torch.tensor(toks)].double().numpy()
+    weights = {e: get(e) for e in experts}  # generated before the timed calls
+    jobs = []
+    rows_of = {}
+    for e in experts:
+        sel = [(i, k) for i, t in enumerate(toks) for k in range(wl.K)
+               if kept[t, k] and int(ids[t, k]) == e]
+        rows_of[e] = sel
+        jobs.append((e, len(sel)))
+    res, t_ffn = _run_experts(
+        jobs, lambda e: oracle.expert_rows(xs[[i for i, _ in rows_of[e]]], *weights[e]), cores)
+    n_rows = sum(n for _, n in jobs)
+    outs = np.zeros((len(toks), wl.K, wl.D))
+    for e, sel in rows_of.items():
+        for j, (i, k) in enumerate(sel):
+            outs[i, k] = res[e][j]
+    t1 = time.perf_counter()
+    oracle.token_outputs(xs, ids[toks], w[toks], kept[toks], None, outs=outs)
+    t_ffn += time.perf_counter() - t1
+    n = len(toks)
     per_token = t_route / wl.T + t_ffn / n
-    cores = oracle.num_threads()
-    # the same on one thread: routing on the first tokens, the expert FFN on a few sampled ones
+    # the same on one thread: routing on the first tokens, the expert FFN on a
+    # part of the same sample
     oracle.set_num_threads(1)
     try:
         n1 = min(wl.T, 1024)
         t0 = time.perf_counter()
-        L1 = oracle.router_logits(cpu_inp["x"][:n1], cpu_inp["w_router"], cpu_inp["bias"],
+        L1 = oracle.router_logits(x[:n1], cpu_inp["w_router"], cpu_inp["bias"],
                                   None if cpu_inp["noise"] is None else cpu_inp["noise"][:n1])
         ids1, _, probs1, lse1 = oracle.route(L1, wl.K)
         oracle.router_stats(ids1, probs1, lse1, wl.E)
         oracle.dispatch(ids1, wl.E, oracle.capacity(n1, wl.K, wl.E, wl.capacity_factor))
         t_route1 = time.perf_counter() - t0
-        m, t_ffn1, budget1 = 0, 0.0, max(0.5, seconds / 5)
-        while t_ffn1 < budget1 and m < wl.T:
-            tok = [int(order[m])]
-            t1 = time.perf_counter()
-            oracle.token_outputs(cpu_inp["x"][tok], ids[tok], w[tok], kept[tok], get)
-            t_ffn1 += time.perf_counter() - t1
-            m += 1
+        budget1 = max(0.5, seconds / 5)
+        rows1, t_ffn1 = 0, 0.0
+        for e in experts:
+            for (i, _) in rows_of[e]:
+                if t_ffn1 >= budget1:
+                    break
+                t1 = time.perf_counter()
+                oracle.expert_rows(xs[[i]], *weights[e])
+                t_ffn1 += time.perf_counter() - t1
+                rows1 += 1
     finally:
         oracle.set_num_threads(cores)
-    per_token1 = t_route1 / n1 + t_ffn1 / m
+    per_token1 = t_route1 / n1 + (t_ffn1 / max(rows1, 1)) * (n_rows / n)
     return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": (f"router + routing + dispatch layout on all {wl.T} tokens "
-                       f"({t_route:.2f} s), expert FFN + combine on {n} sampled tokens "
-                       f"({t_ffn:.2f} s); value extrapolated per token"),
+                       f"({t_route:.2f} s); expert FFN + combine on {n} sampled tokens = "
+                       f"{n_rows} expert rows over {len(experts)} experts ({t_ffn:.2f} s on "
+                       f"{cores} threads: each expert's rows in one oracle call, experts with "
+                       f"fewer rows than threads run concurrently); value extrapolated per token"),
             "single_thread": {"value": round(1.0 / per_token1, 3), "unit": UNIT, "cores": 1,
-                              "sample": (f"routing on {n1} tokens ({t_route1:.2f} s), expert FFN + "
-                                         f"combine on {m} sampled tokens ({t_ffn1:.2f} s); "
-                                         "value extrapolated per token")}}
+                              "sample": (f"routing on {n1} tokens ({t_route1:.2f} s), "
+                                         f"{rows1} expert rows ({t_ffn1:.2f} s); value "
+                                         "extrapolated per token")}}
 
 
-def cpu_baseline_train(wl: Workload, seconds: float = 15.0, seed: int = 0) -> dict:
+def cpu_baseline_train(wl: Workload, seconds: float = 15.0, seed: int = 0, cpu_inp=None) -> dict:
     """The oracle's training step on a bounded sample: forward routing and the
-    router's backward for all T tokens, then each sampled token's kept rows
-    through the expert backward and their share of the weight gradients."""
+    router's backward for all T tokens, then the kept rows of sampled tokens
+    through the expert backward and their share of the weight gradients (each
+    expert's rows in one call, on all host cores; weights generated before
+    the timed calls)."""
     import numpy as np
 
     import oracle
-    cpu_inp = _cpu_inputs_for_sample(wl)
+    cpu_inp = cpu_inp or _cpu_inputs_for_sample(wl)
     dy = make_output_grad(wl, device="cpu")
     t0 = time.perf_counter()
     L = oracle.router_logits(cpu_inp["x"], cpu_inp["w_router"], cpu_inp["bias"], cpu_inp["noise"])
@@ -816,31 +1002,43 @@ def cpu_baseline_train(wl: Workload, seconds: float = 15.0, seed: int = 0) -> di
     t_route = time.perf_counter() - t0
     kept = d["row_of"].reshape(wl.T, wl.K) >= 0
     get = cpu_inp["get_expert"]
+    cores = oracle.num_threads()
     rng = np.random.default_rng(seed)
     order = rng.permutation(wl.T)
-    n, t_rows, batch = 0, 0.0, 1
     budget = max(1.0, seconds - t_route)
-    while t_rows < budget and n < wl.T:
-        toks = sorted(order[n:n + batch].tolist())
-        t1 = time.perf_counter()
-        for e in sorted({int(ids[t, k]) for t in toks for k in range(wl.K) if kept[t, k]}):
-            rows = [(t, k) for t in toks for k in range(wl.K) if kept[t, k] and ids[t, k] == e]
-            tok = np.array([t for t, _ in rows], np.int32)
-            wt = np.array([w[t, k] for t, k in rows])
-            wg, wu, wd = get(e)
-            _, _, h, dg, du = oracle.expert_backward_rows(tok, np.zeros(len(rows), np.int32), wt,
-                                                          cpu_inp["x"], dy, wg, wu, wd,
-                                                          intermediates=True)
-            oracle.expert_wgrad(tok, wt, cpu_inp["x"], dy, h, dg, du)
-        t_rows += time.perf_counter() - t1
-        n += len(toks)
-        batch = min(batch * 2, 32)
+
+    def rows(e, toks):
+        sel = [(t, k) for t in toks for k in range(wl.K) if kept[t, k] and ids[t, k] == e]
+        return (np.array([t for t, _ in sel], np.int32), np.array([w[t, k] for t, k in sel]))
+
+    def work(e, toks, wts):
+        tok, wt = rows(e, toks)
+        wg, wu, wd = wts[e]
+        _, _, h, dg, du = oracle.expert_backward_rows(tok, np.zeros(len(tok), np.int32), wt,
+                                                      cpu_inp["x"], dy, wg, wu, wd,
+                                                      intermediates=True)
+        oracle.expert_wgrad(tok, wt, cpu_inp["x"], dy, h, dg, du)
+        return len(tok)
+
+    # calibration: the first token's kept rows on all threads
+    cal = [int(order[0])]
+    cal_e = sorted({int(ids[cal[0], k]) for k in range(wl.K) if kept[cal[0], k]})
+    wts = {e: get(e) for e in cal_e}
+    _, t_cal = _run_experts([(e, 1) for e in cal_e], lambda e: work(e, cal, wts), cores)
+    sec_row = t_cal / max(1, len(cal_e))
+    toks, experts = _sample_tokens(wl, ids, kept, order, 0.8 * budget * cores / max(sec_row, 1e-9))
+    wts = {e: get(e) for e in experts}
+    jobs = [(e, len(rows(e, toks)[0])) for e in experts]
+    _, t_rows = _run_experts(jobs, lambda e: work(e, toks, wts), cores)
+    n = len(toks)
     per_token = t_route / wl.T + t_rows / n
-    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": oracle.num_threads(),
+    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": (f"routing, dispatch layout and the router's backward on all {wl.T} tokens "
                        f"({t_route:.2f} s); expert backward and weight-gradient rows of {n} "
-                       f"sampled tokens ({t_rows:.2f} s); value extrapolated per token")}
+                       f"sampled tokens = {sum(j for _, j in jobs)} rows over {len(experts)} "
+                       f"experts ({t_rows:.2f} s on {cores} threads); value extrapolated per "
+                       "token")}
 
 
 def _cpu_inputs_for_sample(wl: Workload):
@@ -864,7 +1062,6 @@ def _cpu_inputs_for_sample(wl: Workload):
 
     def get(e):
         if e not in cache:
-            cache.clear()
             ge = torch.Generator().manual_seed(10_000 + e)
             mk = (lambda *s: (torch.randn(*s, generator=ge) * wl.w_std).to(wl.torch_dtype))
             cache[e] = (mk(wl.D, wl.F), mk(wl.D, wl.F), mk(wl.F, wl.D))
@@ -888,20 +1085,24 @@ def workload_of(args) -> Workload:
 
 
 def run_reference(args):
-    """The oracle on the host cores, timed per step on a bounded sample."""
+    """The oracle on the host cores, timed per step on a bounded sample.  Each
+    step's value is extrapolated per token from its sample (routing on every
+    token, the expert FFN on sampled tokens); ms_per_step = T / value is that
+    extrapolation, not a timed step of the whole layer."""
     rank, world, _ = rank_info()
     if rank != 0:
         return
     wl = workload_of(args)
-    per_step = max(2.0, args.cpu_seconds / 2)
+    per_step = max(2.0, args.cpu_seconds / 4)
     train = getattr(args, "pass_", "forward") == "train"
     base = cpu_baseline_train if train else cpu_baseline
+    cpu_inp = _cpu_inputs_for_sample(wl)  # shared by every step (weights drawn once)
     if args.warmup > 0:
-        base(wl, min(per_step, 4.0) / 2)
+        base(wl, 2.0, cpu_inp=cpu_inp)
     vals = []
     t0 = time.perf_counter()
     for i in range(args.steps):
-        vals.append(base(wl, per_step, seed=i))
+        vals.append(base(wl, per_step, seed=i, cpu_inp=cpu_inp))
         if time.perf_counter() - t0 > 240:
             break
     value = statistics.median(v["value"] for v in vals)
@@ -910,7 +1111,11 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC_TRAIN if train else METRIC,
         "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": len(vals), "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(ms_step, 3), "extrapolated": True,
+        "extrapolation": ("ms_per_step = T / value, the per-token cost of each step's bounded "
+                          "sample times T; no step ran the whole layer (the steps together "
+                          f"took {time.perf_counter() - t0:.1f} s)"),
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,
                    "capacity_factor": wl.capacity_factor, "parallelism": "host cores (oracle)"},
@@ -939,6 +1144,9 @@ def main(argv=None):
                     help="replicas (default): every GPU holds all experts; ep: experts sharded")
     ap.add_argument("--graph", action="store_true",
                     help="forward: time replays of a CUDA graph of the whole layer")
+    ap.add_argument("--configs", choices=["all", "none"], default="all",
+                    help="forward at the default shape: also measure the other layer shapes "
+                         "(one record each under the line's 'configs' key)")
     ap.add_argument("--exchange", choices=["all_to_all", "peer"], default="all_to_all",
                     help="with --parallel ep: NCCL all-to-all, or the library's kernels over "
                          "peer-mapped buffers")

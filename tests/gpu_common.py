@@ -179,10 +179,55 @@ def sample_tokens(wl, rt, n_random=16, seed=0):
     return sorted(toks)
 
 
+def stratified_rows(rt, block=128, seed=0):
+    """Expert-major rows that reach every tile of the grouped GEMMs.
+
+    For each expert with kept rows [a, b): its first and last row, and one row
+    at a seeded random position inside every `block`-row block of [a, b).  A
+    128-row block is one single-CTA tile, or one CTA's half of a 256-row
+    CTA-pair tile, so every m-tile (and both CTAs of a pair) is compared; the
+    random position varies the tensor-memory lane and epilogue warp.  Each
+    compared row spans all output columns, so every n-tile of the down GEMM
+    is reached through it.  Returns (rows, number of blocks, number of
+    (expert, 256-row tile) pairs).
+    """
+    rng = np.random.default_rng(seed)
+    offs = np.asarray(rt["offsets"])
+    rows, blocks, tiles256 = set(), 0, 0
+    for e in range(len(offs) - 1):
+        a, b = int(offs[e]), int(offs[e + 1])
+        if b <= a:
+            continue
+        rows.update((a, b - 1))
+        for s in range(a, b, block):
+            rows.add(int(rng.integers(s, min(s + block, b))))
+            blocks += 1
+        tiles256 += (b - a + 255) // 256
+    return sorted(rows), blocks, tiles256
+
+
+def full_size_tokens(wl, rt, seed=0, drop_cap=256):
+    """Tokens whose outputs a full-size test compares: the owners of the
+    stratified rows, the first/last/random/hottest/coldest-expert sample, and
+    the tokens with a dropped slot (up to drop_cap, spread over the batch).
+    Returns (tokens, stratified rows, blocks, (expert, 256-row tile) pairs)."""
+    rows, blocks, tiles = stratified_rows(rt, seed=seed)
+    perm = np.asarray(rt["perm"])
+    toks = {int(perm[r]) // wl.K for r in rows}
+    toks.update(sample_tokens(wl, rt, 12, seed))
+    dropped = np.nonzero((np.asarray(rt["row_of"]).reshape(wl.T, wl.K) < 0).any(1))[0]
+    if dropped.size > drop_cap:
+        dropped = dropped[np.linspace(0, dropped.size - 1, drop_cap).round().astype(np.int64)]
+    toks.update(int(t) for t in dropped)
+    return sorted(toks), rows, blocks, tiles
+
+
 def check_tokens(wl, inp, rt, tokens, y_gpu, y_perm=None, x_perm=None):
     """Sampled tokens: the direct per-token computation against y, and (when
     given) each kept slot's y_perm row against w * expert(x) and its x_perm
-    row against the token row (an exact copy)."""
+    row against the token row (an exact copy).  The oracle evaluates each
+    expert's sampled rows in one call.  Returns (max error, tolerance, the
+    y_perm rows compared)."""
     T, K = wl.T, wl.K
     row_of = rt["row_of"].reshape(T, K)
     kept = row_of >= 0
@@ -191,20 +236,20 @@ def check_tokens(wl, inp, rt, tokens, y_gpu, y_perm=None, x_perm=None):
     ref = oracle.token_outputs(x_rows, rt["ids"][tokens], rt["w"][tokens], kept[tokens], None,
                                outs=outs)
     err, tol = assert_close_out(wl, to_np(y_gpu[tokens]), ref, "y (sampled tokens)")
-    if y_perm is not None:
-        rows, refs = [], []
-        for i, t in enumerate(tokens):
-            for k in range(K):
-                r = int(row_of[t, k])
-                if r >= 0:
-                    rows.append(r)
-                    refs.append(rt["w"][t, k] * outs[i, k])
-        if rows:
-            assert_close_out(wl, to_np(y_perm[rows]), np.stack(refs), "y_perm (sampled rows)")
-    if x_perm is not None:
-        for t in tokens:
-            for k in range(K):
-                r = int(row_of[t, k])
-                if r >= 0:
-                    assert torch.equal(x_perm[r].cpu(), inp["x"][t].cpu()), f"x_perm[{r}] != x[{t}]"
-    return err, tol
+    rows, refs, src = [], [], []
+    for i, t in enumerate(tokens):
+        for k in range(K):
+            r = int(row_of[t, k])
+            if r >= 0:
+                rows.append(r)
+                refs.append(rt["w"][t, k] * outs[i, k])
+                src.append(t)
+    if y_perm is not None and rows:
+        assert_close_out(wl, to_np(y_perm[rows]), np.stack(refs), "y_perm (sampled rows)")
+    if x_perm is not None and rows:
+        ri = torch.tensor(rows, dtype=torch.int64, device=x_perm.device)
+        ti = torch.tensor(src, dtype=torch.int64, device=inp["x"].device)
+        same = (x_perm.index_select(0, ri) == inp["x"].index_select(0, ti)).all(1).cpu()
+        bad = [rows[j] for j in np.nonzero(~same.numpy())[0][:5]]
+        assert not bad, f"x_perm rows {bad} are not exact copies of their token rows"
+    return err, tol, rows

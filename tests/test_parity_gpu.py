@@ -1,10 +1,13 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle.
 
 Small cases compare every output element by element; they span several
-tiles and ragged tails.  The five full-size layer shapes compare the routing
-and dispatch results in full and the layer output on a token sample (tokens
-of the hottest and coldest experts and tokens with dropped slots included),
-through moe_forward, the call the benchmark times.
+tiles and ragged tails, and two of them put three or more tiles through every
+CTA pair.  The five full-size layer shapes (and the ST-MoE shape at capacity
+factor 1.0, which drops) compare the routing and dispatch results in full,
+and, through moe_forward, the call the benchmark times: every token of the
+two small-T layers, and elsewhere a stratified sample that reaches every
+(expert, 128-row block) of the grouped GEMMs plus the tokens with dropped
+slots, compared on y, y_perm and x_perm.
 """
 import numpy as np
 import pytest
@@ -13,7 +16,7 @@ import torch
 import oracle
 from mixture_experts_layer_55_b200 import _binding as B
 from tests.gpu_common import (Bufs, assert_close_out, check_logits, check_routing, check_tokens,
-                              sample_tokens, to_np)
+                              full_size_tokens, to_np)
 from workloads import WORKLOADS, Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -41,11 +44,20 @@ SMALL = [
     _wl("pair_ragged", T=1200, D=200, F=392, E=4, K=2, seed=13),
     _wl("pair_skewed", T=1500, D=128, F=136, E=8, K=2, bias="zipf", seed=14),
     _wl("pair_drops", T=2000, D=64, F=256, E=8, K=2, capacity_factor=0.75, noise=True, seed=15),
+    # three or more tiles through every CTA pair (74 pairs on 148 SMs), so each
+    # tensor-memory accumulator buffer is reused and the operand ring wraps many
+    # times: 256 gate/up tiles (4 m-tiles x 8 n-tiles x 8 experts), then 256
+    # down tiles with the long d_model
+    _wl("pair_reuse_gateup", T=4096, D=256, F=1024, E=8, K=2, seed=42),
+    _wl("pair_reuse_down", T=4096, D=2048, F=256, E=8, K=2, seed=43),
     # tensor-core router (bf16, E <= 128, T >= 2048): ragged 128-token tail, E not
     # a multiple of 64, bias and noise, K = 8
     _wl("tcr_ragged", T=2500, D=136, F=64, E=8, K=2, seed=16),
     _wl("tcr_e100", T=2100, D=264, F=64, E=100, K=4, bias="zipf", noise=True, seed=17),
     _wl("tcr_e128_k8", T=2048, D=128, F=32, E=128, K=8, seed=18),
+    # more token tiles than SMs: two router CTAs per SM (shallower rings)
+    _wl("tcr_two_per_sm", T=19200, D=136, F=32, E=24, K=3, noise=True, seed=44),
+    _wl("tcr_two_per_sm_e64", T=19000, D=64, F=32, E=64, K=6, bias="zipf", seed=45),
     # tensor-core router split over d_model (few token tiles, long d_model): 2 splits with a
     # ragged last one, and 4 splits under the group limit, selection bias and sigmoid scores
     _wl("tcr_split2", T=2200, D=1088, F=64, E=8, K=2, bias="zipf", noise=True, seed=40),
@@ -202,12 +214,22 @@ def test_out_of_range_ids_raise_bounds_flag(cuda_ok):
 
 # ------------------------------------------------------------- full sizes --
 
-FULL = ["tiny_fp32", "mixtral_8x", "fine_skewed", "stmoe_capacity", "decode_e256"]
+FULL = ["tiny_fp32", "mixtral_8x", "fine_skewed", "stmoe_capacity", "decode_e256",
+        "stmoe_capacity_cf1"]
+
+
+def _full_workload(name):
+    if name == "stmoe_capacity_cf1":
+        # the ST-MoE shape at capacity factor 1.0: C = 2048 against a hottest
+        # expert of about 2290 assignments, so the token-order drop rule runs
+        # on a 32768-token layer with hundreds of tiles per GEMM
+        return WORKLOADS["stmoe_capacity"].with_(name=name, capacity_factor=1.0)
+    return WORKLOADS[name]
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_layer(cuda_ok, name):
-    wl = WORKLOADS[name]
+def test_full_size_layer(cuda_ok, capsys, name):
+    wl = _full_workload(name)
     torch.manual_seed(0)
     inp = make_inputs(wl, device="cuda")
     b = Bufs(wl)
@@ -222,15 +244,30 @@ def test_full_size_layer(cuda_ok, name):
     torch.cuda.synchronize()
     assert B.moe_get_device_status(ws) == 0
     assert torch.equal(y, b.y), "moe_forward differs from the op-by-op path"
+    n_drop = int((rt["row_of"] < 0).sum())
     if wl.T <= 512:
-        tokens = list(range(wl.T)) if wl.name == "tiny_fp32" else sample_tokens(wl, rt, 6)
+        # the tiny fp32 layer and the decode layer: every token
+        tokens, rows, blocks, tiles = list(range(wl.T)), None, None, None
     else:
-        tokens = sample_tokens(wl, rt, 12)
-    if wl.name == "decode_e256":
-        tokens = tokens[:6]
-    check_tokens(wl, inp, rt, tokens, y, y_perm=b.y_perm, x_perm=b.x_perm)
+        # every (expert, 128-row block) of the grouped GEMMs, each expert's first
+        # and last row, and the tokens with dropped slots
+        tokens, rows, blocks, tiles = full_size_tokens(wl, rt)
+    err, tol, compared = check_tokens(wl, inp, rt, tokens, y, y_perm=b.y_perm, x_perm=b.x_perm)
+    R = int(rt["offsets"][-1])
+    if rows is not None:
+        assert set(rows) <= set(compared), "a stratified row was not compared"
+    else:
+        assert sorted(compared) == list(range(R)), "every kept row should be compared"
     if wl.capacity_factor > 0:
-        assert rt["C"] == 2560
+        assert rt["C"] == int(np.ceil(wl.capacity_factor * wl.T * wl.K / wl.E))
+    if name == "stmoe_capacity_cf1":
+        assert rt["C"] == 2048 and n_drop > 0, "capacity factor 1.0 should drop assignments"
+    with capsys.disabled():
+        cov = (f"all {R} kept rows" if rows is None else
+               f"{len(compared)} of {R} kept rows; every one of the {blocks} (expert, 128-row) "
+               f"blocks = {tiles} (expert, 256-row tile) pairs")
+        print(f"\n[full-size parity] {name}: {len(tokens)} tokens, {cov}; "
+              f"{n_drop} dropped slots; max err {err:.3e} (tol {tol:.3e})")
     del inp
     torch.cuda.empty_cache()
 
