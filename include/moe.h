@@ -171,7 +171,9 @@ MOE_API moe_status moe_forward_workspace_size(const moe_config *cfg, size_t *byt
  * topk_ids (T, K) and topk_w (T, K) are required.  mean_prob (E) and
  * losses (3) may be NULL; the statistics are then skipped.
  * The reductions behind mean_prob and losses run in a fixed order
- * (deterministic run to run).
+ * (deterministic run to run), finished on the device by the router kernel's
+ * block that completes last (workspace status word 16 counts the blocks and
+ * is left at zero).
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router,
                      const float *router_bias, const float *selection_bias,
@@ -511,8 +513,10 @@ MOE_API moe_status moe_ep_peer_combine(const moe_config *cfg, int32_t world, con
  * library holds until the process exits.  A problem whose scratch would not
  * fit (2 * ceil(T*K / 2048) * E int32 words plus 256 bytes) is rejected with
  * MOE_ERR_WORKSPACE before anything is enqueued.  Allocates nothing.
- *   - The first call on a device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (a table read; nothing is cached, so the address stays right after a
+ *     cudaDeviceReset).  The first call on a device may load the library's
+ *     device code there: make that first call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; each call clears what must start at zero.  Calls whose work
  *     overlaps on the GPU (other streams, other threads) race on the array:
@@ -549,12 +553,11 @@ MOE_API moe_status moe_selftest_wait_timeout(void *workspace, size_t workspace_b
 
 /*
  * Number of kernels one moe_forward call launches for this configuration:
- * router 4 (bf16 with E <= 128 and T >= 2048: weight split, fused
- * tensor-core router, two statistic reductions; otherwise logits GEMM, top-k,
- * two statistic reductions, plus a split-sum when the GEMM is split over
- * d_model), dispatch 3, gather 1, expert GEMMs 2, shared expert 3 (when
- * F_shared > 0: its row offsets and two GEMMs), combine 1.  0 for an invalid
- * configuration.
+ * router 1 (bf16 with E <= 128 and T >= 2048: the tensor-core router, which
+ * also routes and finishes the statistics) or 2 (logits GEMM and top-k, plus
+ * a split-sum when the GEMM is split over d_model), dispatch 3, gather 1,
+ * expert GEMMs 2, shared expert 3 (when F_shared > 0: its row offsets and two
+ * GEMMs), combine 1.  0 for an invalid configuration.
  */
 MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
 

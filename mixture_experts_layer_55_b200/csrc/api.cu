@@ -46,12 +46,9 @@ WsLayout ws_layout(const moe_config& c)
     L.status = o;
     o += align_up(64 * sizeof(int));
     L.r_part = o;
-    size_t part_bytes = (size_t)rp.splits * (size_t)c.T * c.E * sizeof(float);
-    if (router_tc_eligible(c)) {  // split weights, then the split-K partial logits
-        const size_t tc = align_up(router_tc_wsplit_bytes(c)) +
-                          (size_t)router_tc_splits(c) * (size_t)c.T * c.E * sizeof(float);
-        if (tc > part_bytes) part_bytes = tc;
-    }
+    // the SIMT router's (partial) logits per d_model split (also the fallback of the
+    // tensor-core router for an unaligned W_r)
+    const size_t part_bytes = (size_t)rp.splits * (size_t)c.T * c.E * sizeof(float);
     o += align_up(part_bytes);
     L.r_mp = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(float));
@@ -61,8 +58,6 @@ WsLayout ws_layout(const moe_config& c)
     o += align_up((size_t)rp.nb_topk * sizeof(float));
     L.r_cnt = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(int32_t));
-    L.r_fin = o;
-    o += align_up((size_t)(2 * c.E + 2) * sizeof(double));
     L.d_cnt = o;
     o += align_up((size_t)nch * c.E * sizeof(int32_t));
     L.d_base = o;
@@ -164,7 +159,6 @@ static moe_status check_config(const moe_config* c)
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // ------------------------------------------------------------- tracing --
 static void* g_trace[16];
@@ -677,9 +671,10 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK) return 0;
     const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
-    if (router_tc_eligible(*cfg))  // split weights, router (+ top-k from its logits), 2 reductions
-        return 11 + shared + (router_tc_partial(*cfg) ? 1 : 0);
-    return 11 + shared + (router_plan(*cfg).splits > 1 ? 1 : 0);
+    // dispatch 3, gather 1, expert GEMMs 2, combine 1; router: the tensor-core
+    // kernel alone, or the logits GEMM (+ its split sum) and the top-k kernel
+    if (router_tc_eligible(*cfg)) return 1 + 7 + shared;
+    return 2 + (router_plan(*cfg).splits > 1 ? 1 : 0) + 7 + shared;
 }
 
 moe_status moe_ep_workspace_size(int32_t world, int32_t experts_per_rank, size_t* bytes)

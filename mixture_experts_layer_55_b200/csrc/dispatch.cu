@@ -21,6 +21,9 @@
 //                             into shared memory and stored to each of its
 //                             kept rows of x_perm.
 // Every result is fully determined by the ids (no atomics decide an order).
+// Steps 1-3 normally run as one cooperative kernel (dispatch_index_kernel).
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -156,6 +159,176 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(
     }
 }
 
+// ------------------------------------------------- one-kernel index pass --
+// The three steps above in one cooperative launch (every block resident), for
+// the usual sizes: block b ranks chunk b within itself (as the rank kernel
+// does) and publishes the chunk's per-expert counts; after one grid barrier
+// each block reads all chunks' counts (a few thousand integers from L2) and
+// derives its own rank bases and the offsets, so the scan needs no block of
+// its own and no second barrier.  Same arithmetic, same results.
+
+// Words of the workspace status region used by the grid barrier: arrivals,
+// and a generation that the last block to arrive advances.  Both start at
+// zero with the workspace, and the count is back at zero after every barrier.
+constexpr int kGridBarCount = 17;
+constexpr int kGridBarGen = 18;
+
+// Grid-wide barrier of a cooperative launch.  Bounded: after kWaitLimitNs a
+// waiting block raises the timeout flag and goes on (its results are then
+// flagged as invalid).
+MOE_DEVICE void grid_barrier(int* status, int where)
+{
+    __threadfence();  // this thread's global writes before the arrival
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile int* gen = status + kGridBarGen;
+        const int my_gen = *gen;
+        __threadfence();
+        const int nb = (int)(gridDim.x * gridDim.y * gridDim.z);
+        if (atomicAdd(status + kGridBarCount, 1) == nb - 1) {
+            atomicExch(status + kGridBarCount, 0);
+            __threadfence();
+            atomicAdd(status + kGridBarGen, 1);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t spins = 0;
+            while (*gen == my_gen) {
+                __nanosleep(64);
+                if (((++spins) & 1023u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+                    raise_flag(status, kFlagTimeout, where);
+                    break;
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) dispatch_index_kernel(
+    const int32_t* __restrict__ ids, int64_t n, int E, int64_t C, int32_t* blk_cnt,
+    int32_t* __restrict__ counts, int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm, int32_t* __restrict__ row_of, int64_t max_rows, int* status)
+{
+    __shared__ int32_t s_wcnt[8][256];  // per-warp counts, then warp prefixes
+    __shared__ int32_t s_base[256];     // this chunk's rank base per expert
+    __shared__ int32_t s_scan[256];     // kept, then its inclusive scan
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nch = (int)gridDim.x;
+    for (int i = threadIdx.x; i < 8 * 256; i += 256) (&s_wcnt[0][0])[i] = 0;
+    __syncthreads();
+
+    // phase 1: ranks within the chunk, and the chunk's counts
+    const int64_t base = (int64_t)blockIdx.x * kChunk + (int64_t)warp * 256;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    int32_t my_e[kPerThread];
+    int32_t my_local[kPerThread];
+#pragma unroll
+    for (int sgm = 0; sgm < kPerThread; ++sgm) {
+        const int64_t a = base + sgm * 32 + lane;
+        int e = -1;
+        if (a < n) {
+            e = ids[a];
+            if (e < 0 || e >= E) {
+                raise_flag(status, kFlagBounds, 100);
+                e = -1;
+            }
+        }
+        unsigned same = __match_any_sync(0xffffffffu, e);
+        int before = 0;
+        if (e >= 0) before = s_wcnt[warp][e];
+        __syncwarp();
+        const int leader = __ffs(same) - 1;
+        if (e >= 0 && lane == leader) s_wcnt[warp][e] = before + __popc(same);
+        __syncwarp();
+        my_e[sgm] = e;
+        my_local[sgm] = before + __popc(same & lt_mask);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += 256) {
+        int32_t run = 0;
+        for (int w = 0; w < 8; ++w) {
+            const int32_t v = s_wcnt[w][e];
+            s_wcnt[w][e] = run;
+            run += v;
+        }
+        blk_cnt[(size_t)blockIdx.x * E + e] = run;
+    }
+    grid_barrier(status, 102);
+
+    // phase 2: this chunk's bases, every expert's count, kept and offset
+    {
+        const int e = threadIdx.x;
+        int32_t kp = 0;
+        if (e < E) {
+            int64_t run = 0, mine = 0;
+            for (int b = 0; b < nch; ++b) {
+                if (b == (int)blockIdx.x) mine = run;
+                run += __ldcg(blk_cnt + (size_t)b * E + e);
+            }
+            s_base[e] = (int32_t)mine;
+            kp = (int32_t)(run < C ? run : C);
+            if (blockIdx.x == 0) {
+                counts[e] = (int32_t)run;
+                kept[e] = kp;
+            }
+        }
+        s_scan[e] = kp;
+        __syncthreads();
+        for (int o = 1; o < 256; o <<= 1) {  // inclusive Hillis-Steele scan
+            const int32_t v = e >= o ? s_scan[e - o] : 0;
+            __syncthreads();
+            s_scan[e] += v;
+            __syncthreads();
+        }
+        if (blockIdx.x == 0) {
+            if (e < E) offsets[e + 1] = s_scan[e];
+            if (e == 0) offsets[0] = 0;
+        }
+    }
+    __syncthreads();
+
+    // phase 3: keep iff rank < C; row = offset + rank
+#pragma unroll
+    for (int sgm = 0; sgm < kPerThread; ++sgm) {
+        const int64_t a = base + sgm * 32 + lane;
+        if (a >= n) continue;
+        const int e = my_e[sgm];
+        int32_t row = -1;
+        if (e >= 0) {
+            const int64_t rank = (int64_t)s_base[e] + s_wcnt[warp][e] + my_local[sgm];
+            if (rank < C) {
+                const int64_t r = (int64_t)(e > 0 ? s_scan[e - 1] : 0) + rank;
+                if (r >= 0 && r < max_rows) {
+                    row = (int32_t)r;
+                    perm[r] = (int32_t)a;
+                } else {
+                    raise_flag(status, kFlagBounds, 101);
+                }
+            }
+        }
+        row_of[a] = row;
+    }
+}
+
+// Blocks of dispatch_index_kernel that can be resident at once (per device).
+static int resident_index_blocks()
+{
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int v = cached[dev].load(std::memory_order_acquire);
+    if (v > 0) return v;
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_index_kernel, 256, 0) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    v = per_sm * sms;
+    cached[dev].store(v, std::memory_order_release);
+    return v;
+}
+
 cudaError_t launch_dispatch_index(const moe_config& c, int64_t C, const int32_t* ids,
                                   int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* perm,
                                   int32_t* row_of, char* ws, const WsLayout& L, cudaStream_t s)
@@ -166,6 +339,15 @@ cudaError_t launch_dispatch_index(const moe_config& c, int64_t C, const int32_t*
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.d_cnt);
     int32_t* blk_base = reinterpret_cast<int32_t*>(ws + L.d_base);
     const int64_t max_rows = max_rows_of(c);
+    if (nch <= resident_index_blocks()) {
+        // one cooperative launch: all chunks' blocks resident at once
+        int E = c.E;
+        void* args[] = {(void*)&ids, (void*)&n, (void*)&E, (void*)&C, (void*)&blk_cnt,
+                        (void*)&counts, (void*)&kept, (void*)&offsets, (void*)&perm,
+                        (void*)&row_of, (void*)&max_rows, (void*)&status};
+        return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(dispatch_index_kernel),
+                                           dim3((unsigned)nch), dim3(256), args, 0, s);
+    }
     dispatch_count_kernel<<<(unsigned)nch, 256, 0, s>>>(ids, n, c.E, blk_cnt, status);
     dispatch_scan_kernel<<<1, 256, 0, s>>>(blk_cnt, blk_base, nch, c.E, C, counts, kept, offsets);
     dispatch_rank_kernel<<<(unsigned)nch, 256, 0, s>>>(ids, n, c.E, C, blk_base, offsets, perm,
@@ -263,13 +445,9 @@ cudaError_t launch_gather(const moe_config& c, const void* x, const int32_t* row
 {
     const int64_t row_bytes = (int64_t)c.D * (c.dtype == MOE_BF16 ? 2 : 4);
     const size_t smem = (size_t)kGatherWarps * kGatherBufs * kGatherPiece;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static PerDeviceFlag smem_set;
+    cudaError_t ae = opt_in_smem(smem_set, reinterpret_cast<const void*>(gather_kernel), smem);
+    if (ae != cudaSuccess) return ae;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

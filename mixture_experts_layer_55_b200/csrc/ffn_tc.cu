@@ -712,12 +712,12 @@ static bool map_halves_store(CUtensorMap* m, const void* base, uint64_t half, ui
 template <int MODE, bool PAIR>
 static cudaError_t prepare(int* resident_units)
 {
-    static int cached[32];  // 0 = not yet queried on that device (per MODE, PAIR instance)
+    static std::atomic<int> cached[32];  // 0 = not yet queried on that device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 32 && cached[dev] > 0) {
-        *resident_units = cached[dev];
+    if (dev >= 0 && dev < 32 && cached[dev].load(std::memory_order_acquire) > 0) {
+        *resident_units = cached[dev].load(std::memory_order_acquire);
         return cudaSuccess;
     }
     constexpr size_t smem = smem_bytes<MODE, PAIR>();
@@ -747,7 +747,7 @@ static cudaError_t prepare(int* resident_units)
         units = sms;  // one CTA per SM (shared memory allows no second)
     }
     if (units < 1) return cudaErrorInvalidConfiguration;
-    if (dev < 32) cached[dev] = units;
+    if (dev >= 0 && dev < 32) cached[dev].store(units, std::memory_order_release);
     *resident_units = units;
     return cudaSuccess;
 }

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "moe.h"
 
 namespace moe {
@@ -13,6 +15,27 @@ namespace moe {
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// A kernel attribute is per device: remember, per device, that a kernel's
+// dynamic shared memory has been opted in (one bit per device for ordinals
+// below 64; above that the attribute is set on every call).  Safe to use from
+// several host threads: setting the attribute twice is harmless.
+struct PerDeviceFlag {
+    std::atomic<uint64_t> mask{0};
+};
+inline cudaError_t opt_in_smem(PerDeviceFlag& flag, const void* kernel, size_t smem)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+    if (bit && (flag.mask.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && bit) flag.mask.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 // ------------------------------------------------------------ router plan --
 struct RouterPlan {
@@ -56,13 +79,11 @@ inline int64_t dispatch_chunks(const moe_config& c)
 // ------------------------------------------------------ workspace layout --
 struct WsLayout {
     size_t status;      // int32[64]
-    size_t r_part;      // splits * T * E fp32 partial logits, or the tensor-core
-                        // router's split weights (3 * D * EP bf16), whichever is larger
+    size_t r_part;      // splits * T * E fp32 partial logits of the SIMT router
     size_t r_mp;        // nb_topk * E fp32
     size_t r_z;         // nb_topk fp32
     size_t r_ent;       // nb_topk fp32 (entropy partials)
     size_t r_cnt;       // nb_topk * E int32
-    size_t r_fin;       // (2E + 2) fp64: probability sums, z sum, counts, entropy sum
     size_t d_cnt;       // chunks * E int32
     size_t d_base;      // chunks * E int32
     size_t total;
@@ -110,20 +131,17 @@ int64_t capacity_of(const moe_config& c);
 int64_t max_rows_of(const moe_config& c);
 
 // Tensor-core router (router_tc.cu): bf16 layers with E <= 128 and T >= 2048.
+// One kernel: logits, routing, and (when mean_prob or losses is given) the
+// statistics, finished by the CTA that completes last.
 bool router_tc_eligible(const moe_config& c);
 int router_tc_blocks(const moe_config& c);
-// splits of d_model (1: the fused router; > 1: partial logits for the top-k kernel)
+// CTAs per token tile (a cluster splitting d_model; 1: no split)
 int router_tc_splits(const moe_config& c);
-// true: the tensor-core router writes (partial) logits and the top-k kernel routes
-bool router_tc_partial(const moe_config& c);
-size_t router_tc_wsplit_bytes(const moe_config& c);
-// part_out: (splits, T, E) fp32 partial logits, used when router_tc_splits > 1
 cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
                              const float* w_router, const float* bias, const float* noise,
                              float* logits_out, float* probs_out, int32_t* ids, float* w,
                              float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
-                             int with_stats, void* wsplit_scratch, void* part_out, int* status,
-                             cudaStream_t s);
+                             float* mean_prob, float* losses, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- launches --
 // Each returns cudaSuccess or the launch error.

@@ -10,10 +10,12 @@
 // The scratch (device status word, per-chunk expert counts and rank bases)
 // lives in g_noalloc_scratch, kNoallocScratchBytes = 256 KiB, which every GPU
 // that loads the library holds until the process exits.  In host code the
-// array's name is only a host-side stand-in, so its device address is taken
-// with cudaGetSymbolAddress once per device, on that device's first call.
-#include <mutex>
-
+// array's name is only a host-side stand-in, so every call looks up its device
+// address on the current device with cudaGetSymbolAddress.  The lookup is a
+// table read once the library's device code is loaded on that device (the
+// first call there loads it); it is repeated on every call rather than cached
+// so that a cudaDeviceReset, after which the array may sit at a new address,
+// leaves no stale pointer behind.
 #include "internal.h"
 
 namespace moe {
@@ -21,26 +23,13 @@ namespace moe {
 constexpr size_t kNoallocScratchBytes = 256 * 1024;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-static void* g_noalloc_ptr[kMaxDevices];
-static std::mutex g_noalloc_mutex;
-
-// Device address of the static scratch on the current device (set-up on the
-// first call made with that device current).
+// Device address of the static scratch on the current device.
 static cudaError_t noalloc_scratch(char** out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = static_cast<char*>(g_noalloc_ptr[dev]);
+    *out = static_cast<char*>(p);
     return cudaSuccess;
 }
 
@@ -73,10 +62,11 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
     const WsLayout L = noalloc_layout(*cfg);
     if (L.total > kNoallocScratchBytes) return MOE_ERR_WORKSPACE;  // beyond the static array
     char* scratch = nullptr;
-    if (noalloc_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_status(e);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the status word collects flags with atomic OR: it must start at zero
-    cudaError_t e = cudaMemsetAsync(scratch + L.status, 0, 64 * sizeof(int), s);
+    e = cudaMemsetAsync(scratch + L.status, 0, 64 * sizeof(int), s);
     if (e == cudaSuccess) {
         int64_t C = 0;
         moe_capacity(cfg, &C);
@@ -89,5 +79,5 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
         e = launch_gather(*cfg, x, row_of, x_perm, rows, reinterpret_cast<int*>(scratch + L.status),
                           s);
     }
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return cuda_status(e);
 }

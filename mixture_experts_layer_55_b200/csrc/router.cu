@@ -12,11 +12,15 @@
 //   router_splitsum_kernel sums the d-split partials in split order.
 //   router_topk_kernel    one warp per token: adds bias and noise, softmax, top-k by
 //                         (logit desc, id asc) with warp shuffles, weights,
-//                         and per-block statistic partials.
-//   router_colsum_kernel  per-expert fixed-order reduction of the block partials.
-//   router_finalize_kernel mean probabilities, z-loss and balance loss.
+//                         and per-block statistic partials, which the block
+//                         that finishes last reduces in a fixed order into
+//                         the mean probabilities, z-loss and balance loss
+//                         (router_stats.cuh).
+// bf16 layers with E <= 128 and T >= 2048 route on the tensor cores instead
+// (router_tc.cu).
 #include "common.cuh"
 #include "internal.h"
+#include "router_stats.cuh"
 
 namespace moe {
 
@@ -208,7 +212,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ noise, RouteOpts o, float* __restrict__ logits_out,
     float* __restrict__ probs_out, int32_t* __restrict__ ids, float* __restrict__ wout,
     float* __restrict__ blk_mp, float* __restrict__ blk_z, float* __restrict__ blk_ent,
-    int32_t* __restrict__ blk_cnt, int64_t T, int E, int K, int with_stats)
+    int32_t* __restrict__ blk_cnt, int64_t T, int E, int K, int with_stats,
+    float* __restrict__ mean_prob, float* __restrict__ losses, int* __restrict__ counter)
 {
     __shared__ float s_mp[8][256];
     __shared__ int s_cnt[8][256];
@@ -417,79 +422,19 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
         blk_z[blockIdx.x] = a;
         blk_ent[blockIdx.x] = h;
     }
-}
-
-// Block e < E reduces column e of the per-block partials (normalised scores in
-// double, counts in int64); block E reduces the z partials, block E + 1 the
-// entropy partials.  Fixed order: strided per-thread sums, then a tree.
-__global__ void __launch_bounds__(256) router_colsum_kernel(const float* __restrict__ blk_mp,
-                                                            const float* __restrict__ blk_z,
-                                                            const float* __restrict__ blk_ent,
-                                                            const int32_t* __restrict__ blk_cnt,
-                                                            int nb, int E, double* __restrict__ fin)
-{
-    __shared__ double s_a[256];
-    __shared__ long long s_c[256];
-    const int col = blockIdx.x;
-    double a = 0.0;
-    long long cn = 0;
-    for (int b = threadIdx.x; b < nb; b += 256) {
-        if (col < E) {
-            a += (double)blk_mp[(size_t)b * E + col];
-            cn += blk_cnt[(size_t)b * E + col];
-        } else if (col == E) {
-            a += (double)blk_z[b];
-        } else {
-            a += (double)blk_ent[b];
-        }
-    }
-    s_a[threadIdx.x] = a;
-    s_c[threadIdx.x] = cn;
+    // the block that finishes last reduces every block's partials
+    __threadfence();
     __syncthreads();
-    for (int off = 128; off > 0; off >>= 1) {
-        if (threadIdx.x < off) {
-            s_a[threadIdx.x] += s_a[threadIdx.x + off];
-            s_c[threadIdx.x] += s_c[threadIdx.x + off];
-        }
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        if (col < E) {
-            fin[col] = s_a[0];                        // sum of normalised scores
-            fin[E + 1 + col] = (double)s_c[0];        // count (exact in double)
-        } else if (col == E) {
-            fin[E] = s_a[0];                          // sum of lse^2
-        } else {
-            fin[2 * E + 1] = s_a[0];                  // sum of entropies
-        }
-    }
-}
-
-// mean_prob[e] = sum_p[e] / T; losses = {z, E * sum_e (count_e / (T*K)) * mean_prob[e], entropy}.
-__global__ void __launch_bounds__(256) router_finalize_kernel(const double* __restrict__ fin,
-                                                              int64_t T, int E, int K,
-                                                              float* __restrict__ mean_prob,
-                                                              float* __restrict__ losses)
-{
-    __shared__ double s_term[256];
-    const int e = threadIdx.x;
-    double term = 0.0;
-    if (e < E) {
-        const double mp = fin[e] / (double)T;
-        if (mean_prob) mean_prob[e] = (float)mp;
-        term = (fin[E + 1 + e] / ((double)T * (double)K)) * mp;
-    }
-    s_term[e] = term;
+    __shared__ int s_last;
+    if (threadIdx.x == 0) s_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
     __syncthreads();
-    for (int off = 128; off > 0; off >>= 1) {
-        if (e < off) s_term[e] += s_term[e + off];
-        __syncthreads();
-    }
-    if (e == 0 && losses) {
-        losses[0] = (float)(fin[E] / (double)T);
-        losses[1] = (float)((double)E * s_term[0]);
-        losses[2] = (float)(fin[2 * E + 1] / (double)T);
-    }
+    if (!s_last) return;
+    __threadfence();
+    __shared__ double s_d[kStatD];
+    __shared__ long long s_c[kStatC];
+    finish_router_stats(blk_mp, blk_z, blk_ent, blk_cnt, (int)gridDim.x, T, E, K, mean_prob, losses,
+                        s_d, s_c, (int)blockDim.x, (int)threadIdx.x, [] { __syncthreads(); });
+    if (threadIdx.x == 0) *counter = 0;
 }
 
 // DeepSeek-V3 selection-bias step: b[e] += gamma * sign(mean(counts) - counts[e]).
@@ -547,14 +492,15 @@ static void launch_logits(const moe_config& c, const RouterPlan& rp, const XT* x
 static cudaError_t launch_topk(const moe_config& c, const RouteOpts& o, const float* part, int splits,
                                const float* bias, const float* noise, float* logits_out, float* probs_out,
                                int32_t* ids, float* w, float* blk_mp, float* blk_z, float* blk_ent,
-                               int32_t* blk_cnt, int with_stats, const RouterPlan& rp, cudaStream_t s)
+                               int32_t* blk_cnt, int with_stats, float* mean_prob, float* losses,
+                               int* counter, const RouterPlan& rp, cudaStream_t s)
 {
     const int epl = (c.E + 31) / 32;
     dim3 grid(rp.nb_topk);
 #define MOE_TOPK(N)                                                                                     \
     router_topk_kernel<N><<<grid, 256, 0, s>>>(part, splits, bias, noise, o, logits_out, probs_out, ids, \
                                                w, blk_mp, blk_z, blk_ent, blk_cnt, c.T, c.E, c.K,       \
-                                               with_stats)
+                                               with_stats, mean_prob, losses, counter)
     switch (epl) {
         case 1: MOE_TOPK(1); break;
         case 2: MOE_TOPK(2); break;
@@ -578,52 +524,33 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
     float* blk_z = reinterpret_cast<float*>(ws + L.r_z);
     float* blk_ent = reinterpret_cast<float*>(ws + L.r_ent);
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
-    double* fin = reinterpret_cast<double*>(ws + L.r_fin);
-    int nb = rp.nb_topk;
-    if (!logits_in && router_tc_eligible(c)) {
-        // bf16 layers with enough tokens: tensor-core router (fused, or logits for the top-k kernel)
-        const int tc_splits = router_tc_splits(c);
-        char* part_tc = ws + L.r_part + align_up(router_tc_wsplit_bytes(c));
-        cudaError_t e = launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids,
-                                         w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats,
-                                         ws + L.r_part, part_tc, reinterpret_cast<int*>(ws + L.status), s);
-        if (e != cudaSuccess) return e;
-        nb = router_tc_blocks(c);
-        if (router_tc_partial(c)) {
-            nb = rp.nb_topk;
-            e = launch_topk(c, o, reinterpret_cast<const float*>(part_tc), tc_splits, bias, noise, logits_out,
-                            probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt, with_stats, rp, s);
-            if (e != cudaSuccess) return e;
-        }
+    int* status = reinterpret_cast<int*>(ws + L.status);
+    // bf16 layers with enough tokens: one tensor-core kernel (its bulk copies of W_r
+    // need a 16-byte aligned W_r; an unaligned one takes the SIMT router)
+    if (!logits_in && router_tc_eligible(c) && (reinterpret_cast<uintptr_t>(w_router) & 15u) == 0)
+        return launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids, w, blk_mp,
+                                blk_z, blk_ent, blk_cnt, mean_prob, losses, status, s);
+    const float* part;
+    if (logits_in) {
+        part = logits_in;
+        bias = nullptr;
+        noise = nullptr;
     } else {
-        const float* part;
-        if (logits_in) {
-            part = logits_in;
-            bias = nullptr;
-            noise = nullptr;
-        } else {
-            float* p = reinterpret_cast<float*>(ws + L.r_part);
-            if (c.dtype == MOE_BF16)
-                launch_logits(c, rp, static_cast<const __nv_bfloat16*>(x), w_router, p, s);
-            else
-                launch_logits(c, rp, static_cast<const float*>(x), w_router, p, s);
-            if (rp.splits > 1) {
-                const int64_t n = c.T * c.E;
-                int64_t blocks = (n + 255) / 256;
-                if (blocks > 148 * 16) blocks = 148 * 16;
-                router_splitsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rp.splits, n);
-            }
-            part = p;
+        float* p = reinterpret_cast<float*>(ws + L.r_part);
+        if (c.dtype == MOE_BF16)
+            launch_logits(c, rp, static_cast<const __nv_bfloat16*>(x), w_router, p, s);
+        else
+            launch_logits(c, rp, static_cast<const float*>(x), w_router, p, s);
+        if (rp.splits > 1) {
+            const int64_t n = c.T * c.E;
+            int64_t blocks = (n + 255) / 256;
+            if (blocks > 148 * 16) blocks = 148 * 16;
+            router_splitsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rp.splits, n);
         }
-        cudaError_t e = launch_topk(c, o, part, 1, bias, noise, logits_out, probs_out, ids, w, blk_mp,
-                                    blk_z, blk_ent, blk_cnt, with_stats, rp, s);
-        if (e != cudaSuccess) return e;
+        part = p;
     }
-    if (with_stats) {
-        router_colsum_kernel<<<c.E + 2, 256, 0, s>>>(blk_mp, blk_z, blk_ent, blk_cnt, nb, c.E, fin);
-        router_finalize_kernel<<<1, 256, 0, s>>>(fin, c.T, c.E, c.K, mean_prob, losses);
-    }
-    return cudaGetLastError();
+    return launch_topk(c, o, part, 1, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_ent,
+                       blk_cnt, with_stats, mean_prob, losses, status + kRouterCounterWord, rp, s);
 }
 
 }  // namespace moe

@@ -1,0 +1,92 @@
+// router_stats.cuh -- the last step of the router statistics, run by the
+// block of a router kernel that finishes last.
+//
+// "Lab: build a tiny MoE in PyTorch", section "Full implementation": the
+// balance loss E * sum_e f_e P_e with f_e = count_e / (T K) and P_e the mean
+// router probability of expert e, and the z-loss mean_t logsumexp_t^2; its
+// stats also report the mean router entropy.  Each block of a router kernel
+// leaves per-block partials (probability sums per expert, counts per expert,
+// sums of lse^2 and of the entropy); the block that increments the counter
+// last adds them up in a fixed order (so results are bitwise reproducible,
+// whichever block is last), writes mean_prob and losses, and resets the
+// counter to zero for the next launch.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Word of the workspace status region that counts finished router blocks.
+constexpr int kRouterCounterWord = 16;
+
+// Shared scratch of finish_router_stats: kStatD doubles, kStatC long longs.
+constexpr int kStatD = 768;
+constexpr int kStatC = 512;
+
+// Called by all `nthreads` threads (tid = 0 .. nthreads-1) of the last block,
+// after a block-wide barrier; `sync` is that block's barrier.  E <= 256.
+template <typename Sync>
+MOE_DEVICE void finish_router_stats(const float* blk_mp, const float* blk_z, const float* blk_ent,
+                                    const int32_t* blk_cnt, int nb, int64_t T, int E, int K,
+                                    float* mean_prob, float* losses, double* sd, long long* sc,
+                                    int nthreads, int tid, Sync sync)
+{
+    const int ncol = E + 2;  // E probability sums (and counts), the z sum, the entropy sum
+    int cc = nthreads / ncol;
+    if (cc < 1) cc = 1;
+    // chunk sums over a fixed range of blocks each
+    for (int j = tid; j < ncol * cc; j += nthreads) {
+        const int col = j % ncol, ch = j / ncol;
+        const int b0 = (int)((int64_t)nb * ch / cc), b1 = (int)((int64_t)nb * (ch + 1) / cc);
+        double a = 0.0;
+        long long c = 0;
+        for (int b = b0; b < b1; ++b) {
+            if (col < E) {
+                a += (double)__ldcg(blk_mp + (size_t)b * E + col);
+                c += __ldcg(blk_cnt + (size_t)b * E + col);
+            } else if (col == E) {
+                a += (double)__ldcg(blk_z + b);
+            } else {
+                a += (double)__ldcg(blk_ent + b);
+            }
+        }
+        sd[j] = a;
+        sc[j] = c;
+    }
+    sync();
+    // each column: its chunks in order
+    for (int col = tid; col < ncol; col += nthreads) {
+        double a = 0.0;
+        long long c = 0;
+        for (int ch = 0; ch < cc; ++ch) {
+            a += sd[ch * ncol + col];
+            c += sc[ch * ncol + col];
+        }
+        sd[col] = a;
+        sc[col] = c;
+    }
+    sync();
+    // mean probabilities, and the balance-loss terms summed by a fixed tree
+    double* term = sd + 512;
+    for (int e = tid; e < 256; e += nthreads) {
+        double v = 0.0;
+        if (e < E) {
+            const double mp = sd[e] / (double)T;
+            if (mean_prob) mean_prob[e] = (float)mp;
+            v = ((double)sc[e] / ((double)T * (double)K)) * mp;
+        }
+        term[e] = v;
+    }
+    sync();
+    for (int off = 128; off > 0; off >>= 1) {
+        for (int e = tid; e < off; e += nthreads) term[e] += term[e + off];
+        sync();
+    }
+    if (tid == 0 && losses) {
+        losses[0] = (float)(sd[E] / (double)T);
+        losses[1] = (float)((double)E * term[0]);
+        losses[2] = (float)(sd[E + 1] / (double)T);
+    }
+}
+
+}  // namespace moe

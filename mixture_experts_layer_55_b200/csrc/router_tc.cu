@@ -1,5 +1,6 @@
 // router_tc.cu -- router for bf16 layers on the tensor cores: the logits GEMM,
-// softmax, top-k and renormalised weights fused in one kernel.
+// softmax (or sigmoid scores), top-k, the routing weights and the router
+// statistics, all in one kernel.
 //
 // "Lab: build a tiny MoE in PyTorch", section "Full implementation": fp32
 // router logits, softmax over the experts, top-k, weights divided by the sum
@@ -9,129 +10,178 @@
 // fp32 logits on bf16 tensor cores: x is bf16 already, and each fp32 router
 // weight is split exactly into three bf16 terms w = hi + mid + lo (hi =
 // bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid): 3 x 8 significand
-// bits cover fp32's 24).  Every product x*part is exact in fp32, and the
-// three MMAs accumulate in fp32 in tensor memory, so the logits carry fp32
-// accumulation error only (no bf16 rounding of the weights).
+// bits cover fp32's 24).  Every product x*term is exact in fp32, and the
+// three MMAs of a K step accumulate in fp32 in tensor memory, so the logits
+// carry fp32 accumulation error only (no bf16 rounding of the weights).
 //
-//   router_wsplit_kernel  W_r (D, E) fp32 -> (3, D, EP) bf16, EP = E rounded
-//                         up to 64 (zero columns), N-major for TMA.
-//   router_tc_kernel      one CTA per 128 tokens (and per split of d_model when
-//                         the token tiles leave most SMs idle).  With splits,
-//                         or more than 16 experts, it writes fp32 (partial)
-//                         logits, which the top-k kernel of the SIMT router sums
-//                         in split order and routes; otherwise the fused
-//                         epilogue below routes: warp 0 TMA (x tile 128 x 64,
-//                         three 64 x EP weight tiles per stage), warp 1
-//                         tcgen05.mma M=128, N=EP, three per K step into one
-//                         accumulator; warps 2..5 own one token row each:
-//                         logits (+ bias + noise) staged in shared memory,
-//                         max, softmax sum, entropy, scores (softmax or
-//                         sigmoid), the group limit, top-K by (logit +
-//                         selection bias desc, id asc) with an unrolled
-//                         insertion network, weights, normalised scores, and
-//                         fixed-order per-CTA statistics.
+// One CTA per 128 tokens (M = 128) and per split of d_model; N = EPN, the
+// expert count rounded up to 16, 32, 64 or 128.  Warps:
+//   warp 0      TMA: the x tile (128 tokens x 64 of d_model, 128-byte
+//               swizzle) and a bulk copy of the 64 x E fp32 slice of W_r of
+//               each stage of a deep ring (up to 10 stages)
+//   warp 1      tcgen05.mma, three per K step of 16 (one per weight term)
+//   warps 2..5  first the weight split: each stage's fp32 slice is split in
+//               shared memory into its three bf16 terms, written K-major
+//               (expert rows of 64 d_model values, 128-byte swizzle) next
+//               to the x tile, so no weight kernel runs before this one and
+//               the weight tiles are E rows wide, not a padded 64; then the
+//               epilogue, one token row per
+//               thread: logits (+ bias + noise), max, softmax sum and
+//               entropy, scores, the group limit, top-K by (logit +
+//               selection bias desc, id asc) with an unrolled insertion
+//               network, weights, normalised scores, and the per-CTA
+//               statistics (counts by shared-memory atomics; column sums
+//               in a fixed order).
+// When the token tiles alone leave most SMs idle, d_model is split over a
+// cluster of CTAs along grid y: each non-leader CTA sends its partial logits
+// to the leader's shared memory (distributed shared memory), and the leader
+// adds them in split order and runs the epilogue.  With more token tiles
+// than SMs, two CTAs share an SM (shallower rings).  The CTA whose
+// statistics land last finishes them for the whole grid
+// (router_stats.cuh).  Every wait is bounded.
 #include <cuda.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "router_stats.cuh"
 
 namespace moe {
 namespace rtc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int A_BYTES = BM * BK * 2;       // 16 KB
-constexpr int BOX_BYTES = 64 * 64 * 2;     // 8 KB
-constexpr int NUM_THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB x tile per stage
+constexpr int NUM_THREADS = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 weights + epilogue
+constexpr int MAX_STAGES = 10;
+constexpr int MAX_SPLITS = 4;
+constexpr int CONVERTER_WARPS = 4;
 
-template <int EPB> struct Geo {            // EPB = EP / 64 (1 or 2)
-    static constexpr int EP = 64 * EPB;
-    static constexpr int B_BYTES = 3 * EPB * BOX_BYTES;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 40 KB or 64 KB
-    static constexpr int STAGES = EPB == 1 ? 4 : 3;
-    static constexpr int TMEM_COLS = EP;                   // 64 or 128 (powers of two)
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+template <int EPN> struct Geo {
+    static constexpr int TERM_BYTES = EPN * 128;  // EPN expert rows x 64 d_model (bf16)
+    static constexpr int W_OFF = A_BYTES + 3 * TERM_BYTES;  // the stage's fp32 W_r slice
+    static constexpr int TMEM_COLS = EPN < 32 ? 32 : EPN;
+    static constexpr int LDS = EPN + 1;  // epilogue row stride in floats (odd: conflict-free)
 };
 
+// Bytes of one ring stage: x tile, three weight terms, the fp32 slice (64 x E).
+inline size_t stage_bytes_of(int epn, int E)
+{
+    return align_up((size_t)A_BYTES + (size_t)3 * epn * 128 + (size_t)64 * E * 4, 1024);
+}
+
 struct Misc {
-    uint64_t full[4];
-    uint64_t empty[4];
+    uint64_t lfull[MAX_STAGES];  // the stage's x tile and fp32 weights have landed
+    uint64_t full[MAX_STAGES];   // and its weight terms are written: the MMAs may read it
+    uint64_t empty[MAX_STAGES];
     uint64_t tfull;
     uint32_t tmem_base;
     int abort_flag;
+    int last;         // this CTA finishes the statistics of the grid
+    int cnt[128];     // this CTA's expert counts
+    float psum[128];  // chunk sums of the normalised scores
+    float wz[4];      // per lane-quadrant sums of lse^2
+    float wh[4];      // and of the entropy
 };
 
 struct Args {
     RouteOpts o;
+    const float* w;           // W_r (D, E) fp32
     const float* bias;        // E or null
     const float* noise;       // T x E or null
     float* logits_out;        // T x E or null
     float* probs_out;         // T x E or null
     int32_t* ids;             // T x K
     float* wout;              // T x K
-    float* blk_mp;            // grid x E
-    float* blk_z;             // grid
-    float* blk_ent;           // grid
-    int32_t* blk_cnt;         // grid x E
+    float* blk_mp;            // tiles x E
+    float* blk_z;             // tiles
+    float* blk_ent;           // tiles
+    int32_t* blk_cnt;         // tiles x E
+    float* mean_prob;         // E or null
+    float* losses;            // 3 or null
+    int* counter;             // finished-CTA counter (zero between launches)
     int64_t T;
     int D, E, K;
     int with_stats;
     int* status;
-    float* part;              // split mode: (splits, T, E) fp32 partial logits, else null
-    int split_kb;             // split mode: K blocks per split (blockIdx.y = split)
+    int stages;               // ring depth
+    int stage_bytes;          // bytes per ring stage
+    int splits;               // CTAs per token tile (cluster size along y)
+    int split_kb;             // K blocks per split
+    uint32_t misc_off;        // byte offsets in the aligned shared memory
+    uint32_t recv_off;        // (splits - 1) x BM x EPN fp32 partial logits (leader)
 };
-
-__global__ void __launch_bounds__(256) router_wsplit_kernel(const float* __restrict__ w,
-                                                            __nv_bfloat16* __restrict__ out, int D,
-                                                            int E, int EP)
-{
-    const int64_t n = (int64_t)D * EP;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int d = (int)(i / EP), e = (int)(i % EP);
-        const float v = e < E ? w[(int64_t)d * E + e] : 0.f;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const float r1 = v - __bfloat162float(hi);
-        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-        const float r2 = r1 - __bfloat162float(mid);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-        out[i] = hi;
-        out[n + i] = mid;
-        out[2 * n + i] = lo;
-    }
-}
 
 MOE_DEVICE void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int EPB>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     const Args a)
+MOE_DEVICE void st_cluster_f32(uint32_t cluster_addr, float v)
 {
-    using G = Geo<EPB>;
-    constexpr int EP = G::EP, STAGES = G::STAGES, STAGE_BYTES = G::STAGE_BYTES;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+
+// The three bf16 terms of two fp32 weights, packed in pairs.
+MOE_DEVICE void split3(float a, float b, uint32_t& hi, uint32_t& mid, uint32_t& lo)
+{
+    const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
+    const float ra = a - __bfloat162float(ha), rb = b - __bfloat162float(hb);
+    const __nv_bfloat16 ma = __float2bfloat16_rn(ra), mb = __float2bfloat16_rn(rb);
+    const __nv_bfloat16 la = __float2bfloat16_rn(ra - __bfloat162float(ma));
+    const __nv_bfloat16 lb = __float2bfloat16_rn(rb - __bfloat162float(mb));
+    hi = (uint32_t)__bfloat16_as_ushort(ha) | ((uint32_t)__bfloat16_as_ushort(hb) << 16);
+    mid = (uint32_t)__bfloat16_as_ushort(ma) | ((uint32_t)__bfloat16_as_ushort(mb) << 16);
+    lo = (uint32_t)__bfloat16_as_ushort(la) | ((uint32_t)__bfloat16_as_ushort(lb) << 16);
+}
+
+template <int EPN, int KM, int MINB>
+__global__ void __launch_bounds__(NUM_THREADS, MINB)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const Args a)
+{
+    using G = Geo<EPN>;
+    constexpr int TERM = G::TERM_BYTES, LDS = G::LDS;
+    const int STAGE_BYTES = a.stage_bytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* stages = smem;
-    Misc* m = reinterpret_cast<Misc*>(smem + (size_t)STAGES * STAGE_BYTES);
+    Misc* m = reinterpret_cast<Misc*>(smem + a.misc_off);
+    float* recv = reinterpret_cast<float*>(smem + a.recv_off);
+    const int S = a.stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
+    const int split = (int)blockIdx.y;  // the CTA's rank in its cluster when splits > 1
     const int num_kb = (a.D + BK - 1) / BK;
-    // this CTA's K blocks: all of them, or its split's share (never empty)
-    const int kb_begin = a.part ? (int)blockIdx.y * a.split_kb : 0;
-    const int kb_end = a.part ? min(num_kb, kb_begin + a.split_kb) : num_kb;
+    const int kb_begin = split * a.split_kb;                // never empty (host guarantee)
+    const int kb_end = min(num_kb, kb_begin + a.split_kb);
+    const int E = a.E;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&m->full[s], 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&m->lfull[s], 1);               // the producer, with the bytes
+            mbar_init(&m->full[s], CONVERTER_WARPS);  // the weight warps
             mbar_init(&m->empty[s], 1);
         }
         mbar_init(&m->tfull, 1);
         m->abort_flag = 0;
+        m->last = 0;
         fence_mbar_init();
         prefetch_tmap(&tmX);
-        prefetch_tmap(&tmW);
+    }
+    if (warp >= 2) {
+        // weight tiles: rows E .. EPN-1 (if any) stay zero in every stage
+        const int tid = threadIdx.x - 64;
+        m->cnt[tid] = 0;
+        const int pad = EPN - E;
+        if (pad > 0) {
+            const int per_stage = 3 * pad * 8;  // 16-byte chunks
+            for (int i = tid; i < S * per_stage; i += 128) {
+                const int s = i / per_stage;
+                int r = i % per_stage;
+                const int p = r / (pad * 8);
+                r %= pad * 8;
+                uint8_t* dst = stages + (size_t)s * STAGE_BYTES + A_BYTES + p * TERM +
+                               (E + r / 8) * 128 + (r % 8) * 16;
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(&m->tmem_base, G::TMEM_COLS);
@@ -143,120 +193,171 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem_base = m->tmem_base;
     volatile int* abort_flag = &m->abort_flag;
 
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------ TMA producer
-        int stage = 0;
-        uint32_t phase = 0;
-        int last_phase[STAGES];
-        for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
-        for (int kb = kb_begin; kb < kb_end; ++kb) {
-            if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
-            uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
-            uint8_t* sB = sA + A_BYTES;
-            uint64_t* fb = &m->full[stage];
-            mbar_arrive_expect_tx(fb, STAGE_BYTES);
-            const int k0 = kb * BK;
-            tma_load_2d(sA, &tmX, k0, (int32_t)t0, fb);
-#pragma unroll
-            for (int p = 0; p < 3; ++p)
-#pragma unroll
-                for (int j = 0; j < EPB; ++j)
-                    tma_load_3d(sB + (p * EPB + j) * BOX_BYTES, &tmW, 64 * j, k0, p, fb);
-            last_phase[stage] = (int)phase;
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
-            }
-        }
-        for (int s = 0; s < STAGES; ++s)
-            if (last_phase[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = umma_idesc_bf16(BM, EP, 0, 1);
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int kb = kb_begin; kb < kb_end; ++kb) {
-            if (!mbar_wait(&m->full[stage], phase, a.status, 520, abort_flag)) break;
-            tc_fence_after();
-            const uint32_t sA = smem_u32(stages + (size_t)stage * STAGE_BYTES);
-            const uint32_t sB = sA + A_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-                const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
-#pragma unroll
-                for (int p = 0; p < 3; ++p) {
-                    const uint64_t bdesc =
-                        umma_desc_sw128(sB + p * EPB * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
-                    umma_f16_ss(tmem_base, adesc, bdesc, idesc, (kb != kb_begin || kk || p) ? 1u : 0u);
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ producer: x tile + fp32 weights
+            int stage = 0;
+            uint32_t phase = 0;
+            int last_phase[MAX_STAGES];
+            for (int s = 0; s < MAX_STAGES; ++s) last_phase[s] = -1;
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
+                if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
+                uint8_t* st = stages + (size_t)stage * STAGE_BYTES;
+                uint64_t* fb = &m->lfull[stage];
+                const int d0 = kb * BK;
+                const int rows = min(BK, a.D - d0);  // a multiple of 8 (D % 8 == 0)
+                const uint32_t wbytes = (uint32_t)rows * (uint32_t)E * 4u;
+                mbar_arrive_expect_tx(fb, A_BYTES + wbytes);
+                tma_load_2d(st, &tmX, d0, (int32_t)t0, fb);
+                bulk_load_g2s(st + G::W_OFF, a.w + (size_t)d0 * E, wbytes, fb);
+                last_phase[stage] = (int)phase;
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            umma_commit(&m->empty[stage]);
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
+            // every copy issued has landed before the ring is reused or the CTA exits
+            for (int s = 0; s < S; ++s)
+                if (last_phase[s] >= 0)
+                    mbar_wait(&m->lfull[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, EPN, 0, 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
+                if (!mbar_wait(&m->full[stage], phase, a.status, 520, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t sA = smem_u32(stages + (size_t)stage * STAGE_BYTES);
+                const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        const uint64_t bdesc = umma_desc_sw128(sB + p * TERM + kk * 32, 16, 1024);
+                        umma_f16_ss(tmem_base, adesc, bdesc, idesc,
+                                    (kb != kb_begin || kk || p) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&m->empty[stage]);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            umma_commit(&m->tfull);  // also the drain: every MMA done once it fires
+        }
+    } else {
+        // ------------------------------------------------ weight split (warps 2..5)
+        const int tid = threadIdx.x - 64;
+        {
+            int stage = 0;
+            uint32_t phase = 0;
+            const int pairs = E * 8;  // (expert, 8-wide chunk of d_model)
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
+                if (!mbar_wait(&m->lfull[stage], phase, a.status, 540, abort_flag)) break;
+                uint8_t* sB = stages + (size_t)stage * STAGE_BYTES + A_BYTES;
+                const float* wsm = reinterpret_cast<const float*>(sB - A_BYTES + G::W_OFF);
+                const int d0 = kb * BK;
+                for (int i = tid; i < pairs; i += 128) {
+                    const int e = i % E, c = i / E;
+                    const bool in = d0 + c * 8 < a.D;  // D % 8 == 0: a chunk is all in or all out
+                    float v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] = in ? wsm[(c * 8 + j) * E + e] : 0.f;
+                    uint32_t h[4], md[4], l[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) split3(v[2 * j], v[2 * j + 1], h[j], md[j], l[j]);
+                    const int off = e * 128 + ((c ^ (e & 7)) << 4);
+                    *reinterpret_cast<uint4*>(sB + off) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4*>(sB + TERM + off) = make_uint4(md[0], md[1], md[2], md[3]);
+                    *reinterpret_cast<uint4*>(sB + 2 * TERM + off) = make_uint4(l[0], l[1], l[2], l[3]);
+                }
+                fence_proxy_async_smem();  // visible to the tensor cores
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&m->full[stage]);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
-        umma_commit(&m->tfull);  // also the drain: every MMA done once it fires
-    } else if (warp >= 2) {
-        // ------------------------------------------------ epilogue: one token row per thread
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;  // row in tile = tensor-memory lane
-        const int64_t t = t0 + r;
-        const bool valid = t < a.T;
-        const int E = a.E, K = a.K;
-        const RouteOpts& o = a.o;
-        // the pipeline buffers are free once the accumulator is complete
-        float* Ls = reinterpret_cast<float*>(stages);  // [BM][EP + 1] logits, then scores
-        constexpr int LDS = EP + 1;
+        // ------------------------------------------------ accumulators out of tensor memory
+        const int quad = warp & 3;        // the lane quadrant this warp may read
+        const int r = quad * 32 + lane;   // token row in the tile
+        float* Ls = reinterpret_cast<float*>(stages);  // [BM][LDS]
         const bool ok = mbar_wait(&m->tfull, 0, a.status, 530, abort_flag);
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
-        if (a.part != nullptr) {
-            // split mode: this split's partial logits of the row, summed (in split
-            // order) with bias and noise by the top-k kernel
-            float* prow = a.part + ((size_t)blockIdx.y * a.T + t) * E;
+        uint32_t remote = 0;
+        if (split > 0)  // this row's slot in the leader's receive buffer
+            remote = mapa_shared(smem_u32(recv + ((size_t)(split - 1) * BM + r) * EPN), 0);
 #pragma unroll 1
-            for (int c = 0; c < EP / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(taddr + c * 32, v);
-                tmem_ld_wait();
-                if (valid)
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c * 32 + j < E) prow[c * 32 + j] = ok ? __uint_as_float(v[j]) : 0.f;
-            }
-        } else {
-        // pass 1: logits (+ bias + noise) to shared memory and their maximum
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < EP / 32; ++c) {
+        for (int c = 0; c < (EPN + 31) / 32; ++c) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr + c * 32, v);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int e = c * 32 + j;
-                float L = -INFINITY;
-                if (e < E && ok) {
-                    L = __uint_as_float(v[j]);
-                    if (a.bias) L += a.bias[e];
-                    if (a.noise && valid) L += a.noise[t * E + e];
-                    if (a.logits_out && valid) a.logits_out[t * E + e] = L;
+                if (e < EPN) {
+                    const float x = ok ? __uint_as_float(v[j]) : 0.f;
+                    if (split > 0)
+                        st_cluster_f32(remote + e * 4, x);
+                    else
+                        Ls[r * LDS + e] = x;
                 }
-                Ls[r * LDS + e] = L;
-                mx = fmaxf(mx, L);
             }
         }
-        // pass 2: softmax sum, entropy, score sum
+    }
+    __syncwarp();
+    if (a.splits > 1) cluster_sync();  // the other splits' partials are in the leader's buffer
+
+    if (warp >= 2 && split == 0) {
+        // ------------------------------------------------ epilogue: one token row per thread
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int tid = threadIdx.x - 64;
+        const int64_t t = t0 + r;
+        const bool valid = t < a.T;
+        const int K = a.K;
+        const RouteOpts& o = a.o;
+        float* Ls = reinterpret_cast<float*>(stages);  // logits, then normalised scores
+        float* Xs = Ls + BM * LDS;                     // exp(L - max), then scores
+        // pass 1: logits (own K range + the other splits in order, + bias + noise)
+        float mx = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            float L = Ls[r * LDS + e];
+            for (int sp = 1; sp < a.splits; ++sp) L += recv[((size_t)(sp - 1) * BM + r) * EPN + e];
+            if (a.bias) L += a.bias[e];
+            if (a.noise && valid) L += a.noise[t * E + e];
+            if (a.logits_out && valid) a.logits_out[t * E + e] = L;
+            Ls[r * LDS + e] = L;
+            mx = fmaxf(mx, L);
+        }
+        // pass 2: softmax sum
         float ssum = 0.f;
-        for (int e = 0; e < E; ++e) ssum += expf(Ls[r * LDS + e] - mx);
+        for (int e = 0; e < E; ++e) {
+            const float x = expf(Ls[r * LDS + e] - mx);
+            Xs[r * LDS + e] = x;
+            ssum += x;
+        }
         const float inv = 1.0f / ssum;
+        const float lss = logf(ssum);
+        // pass 3: entropy -sum q log(max(q, 1e-9)) with log q = (L - max) - log(sum),
+        // scores (softmax q or sigmoid) into Xs, their sum
+        const float log_floor = logf(1e-9f);
         float ent = 0.f, scsum = 0.f;
         for (int e = 0; e < E; ++e) {
             const float L = Ls[r * LDS + e];
-            const float q = expf(L - mx) * inv;
-            ent -= q * logf(fmaxf(q, 1e-9f));
-            scsum += o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : q;
+            const float q = Xs[r * LDS + e] * inv;
+            ent -= q * (q >= 1e-9f ? (L - mx) - lss : log_floor);
+            const float sc = o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : q;
+            Xs[r * LDS + e] = sc;
+            scsum += sc;
         }
         // group limit: a group's score is its best selection score u = L + b
         uint32_t keep = 0xffffffffu;
@@ -283,96 +384,106 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 keep |= 1u << bg;
             }
         }
-        // pass 3: top-K over the eligible experts by (u desc, id asc), an unrolled
-        // insertion network (a displaced entry carried down keeps that order too)
-        float tv[8];
-        int ti[8];
+        // pass 4: top-K over the eligible experts by (u desc, id asc), an unrolled
+        // insertion network of KM >= K slots (a displaced entry carried down
+        // keeps that order too)
+        float tv[KM];
+        int ti[KM];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < KM; ++k) {
             tv[k] = -INFINITY;
             ti[k] = 0x7fffffff;
         }
         for (int e = 0; e < E; ++e) {
             if (G > 1 && !((keep >> (e / gsz)) & 1u)) continue;
-            float x = Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f);
+            float xv = Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f);
             int xi = e;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const bool gt = x > tv[k] || (x == tv[k] && xi < ti[k]);
-                const float nv = gt ? x : tv[k];
+            for (int k = 0; k < KM; ++k) {
+                const bool gt = xv > tv[k] || (xv == tv[k] && xi < ti[k]);
+                const float nv = gt ? xv : tv[k];
                 const int ni = gt ? xi : ti[k];
-                x = gt ? tv[k] : x;
+                xv = gt ? tv[k] : xv;
                 xi = gt ? ti[k] : xi;
                 tv[k] = nv;
                 ti[k] = ni;
             }
         }
         // weights from the scores of the selected experts
-        float sk[8];
+        float sk[KM];
         float ssel = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            sk[k] = 0.f;
-            if (k < K) {
-                const float L = Ls[r * LDS + ti[k]];
-                sk[k] = o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : expf(L - mx) * inv;
-            }
+        for (int k = 0; k < KM; ++k) {
+            sk[k] = k < K ? Xs[r * LDS + ti[k]] : 0.f;
             ssel += sk[k];
         }
         if (valid) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < KM; ++k)
                 if (k < K) {
                     a.ids[t * K + k] = ti[k];
                     a.wout[t * K + k] = (o.renorm ? sk[k] / ssel : sk[k]) * o.route_scale;
+                    if (a.with_stats) atomicAdd(&m->cnt[ti[k]], 1);  // integer: order-free
                 }
         }
-        // pass 4: normalised scores into shared memory (and probs_out)
-        const float scinv = 1.0f / scsum;
+        // pass 5: normalised scores into Ls (and probs_out); rows past T give nothing
+        const float scinv = o.score_func == 1 ? 1.0f / scsum : 1.0f;
         for (int e = 0; e < E; ++e) {
-            const float L = Ls[r * LDS + e];
-            const float pn = (o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : expf(L - mx) * inv) *
-                             (o.score_func == 1 ? scinv : 1.0f);
-            Ls[r * LDS + e] = valid ? pn : 0.f;  // rows past T contribute nothing
+            const float pn = Xs[r * LDS + e] * scinv;
+            Ls[r * LDS + e] = valid ? pn : 0.f;
             if (a.probs_out && valid) a.probs_out[t * E + e] = pn;
         }
         if (a.with_stats) {
-            // per-CTA statistics in a fixed order: column sums over the rows
-            const float lse = mx + logf(ssum);
-            int* sid = reinterpret_cast<int*>(Ls + BM * LDS);  // [BM][8]
-            float* sz = reinterpret_cast<float*>(sid + BM * 8);
-            float* sh = sz + BM;
+            // per-CTA statistics, each in a fixed order
+            const float lse = mx + lss;
+            float z = valid ? lse * lse : 0.f, h = valid ? ent : 0.f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) sid[r * 8 + k] = (valid && k < K) ? ti[k] : -1;
-            sz[r] = valid ? lse * lse : 0.f;
-            sh[r] = valid ? ent : 0.f;
+            for (int off = 16; off > 0; off >>= 1) {
+                z += __shfl_xor_sync(0xffffffffu, z, off);
+                h += __shfl_xor_sync(0xffffffffu, h, off);
+            }
+            if (lane == 0) {
+                m->wz[quad] = z;
+                m->wh[quad] = h;
+            }
             epi_sync();
-            const int tid = threadIdx.x - 64;
-            for (int e = tid; e < E; e += 128) {
+            constexpr int CH = 128 / EPN;  // row chunks per column (EPN x CH = 128 threads)
+            constexpr int RC = BM / CH;
+            {
+                const int col = tid % EPN, ch = tid / EPN;
                 float sp = 0.f;
-                int cn = 0;
-                for (int rr = 0; rr < BM; ++rr) {
-                    sp += Ls[rr * LDS + e];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) cn += sid[rr * 8 + k] == e;
-                }
-                a.blk_mp[(size_t)blockIdx.x * E + e] = sp;
-                a.blk_cnt[(size_t)blockIdx.x * E + e] = cn;
+                if (col < E)
+                    for (int rr = ch * RC; rr < (ch + 1) * RC; ++rr) sp += Ls[rr * LDS + col];
+                m->psum[ch * EPN + col] = sp;
+            }
+            epi_sync();
+            if (tid < E) {
+                float sp = 0.f;
+                for (int ch = 0; ch < CH; ++ch) sp += m->psum[ch * EPN + tid];
+                a.blk_mp[(size_t)blockIdx.x * E + tid] = sp;
+                a.blk_cnt[(size_t)blockIdx.x * E + tid] = m->cnt[tid];
             }
             if (tid == 0) {
-                float zs = 0.f, hs = 0.f;
-                for (int rr = 0; rr < BM; ++rr) {
-                    zs += sz[rr];
-                    hs += sh[rr];
-                }
-                a.blk_z[blockIdx.x] = zs;
-                a.blk_ent[blockIdx.x] = hs;
+                a.blk_z[blockIdx.x] = ((m->wz[0] + m->wz[1]) + m->wz[2]) + m->wz[3];
+                a.blk_ent[blockIdx.x] = ((m->wh[0] + m->wh[1]) + m->wh[2]) + m->wh[3];
             }
+            __threadfence();
+            epi_sync();
+            if (tid == 0) m->last = atomicAdd(a.counter, 1) == (int)gridDim.x - 1;
         }
-        }  // fused epilogue
     }
     tc_fence_before();
     __syncthreads();
+    if (split == 0 && a.with_stats && m->last) {
+        // the last CTA: the statistics of the whole grid (all 192 threads)
+        __threadfence();
+        double* sd = reinterpret_cast<double*>(stages);
+        long long* sc = reinterpret_cast<long long*>(sd + kStatD);
+        finish_router_stats(a.blk_mp, a.blk_z, a.blk_ent, a.blk_cnt, (int)gridDim.x, a.T, E, a.K,
+                            a.mean_prob, a.losses, sd, sc, NUM_THREADS, (int)threadIdx.x,
+                            [] { __syncthreads(); });
+        if (threadIdx.x == 0) *a.counter = 0;
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, G::TMEM_COLS);
@@ -398,48 +509,87 @@ static EncodeTiledFn encoder()
     return fn;
 }
 
-template <int EPB>
-static cudaError_t launch_t(const moe_config& c, const void* x, const __nv_bfloat16* wsplit,
-                            const Args& a, cudaStream_t s)
+// Ring depth and shared-memory layout for `ctas_per_sm` CTAs on each SM.
+struct Plan {
+    int epn, splits, split_kb, ctas_per_sm, stages, stage_bytes;
+    uint32_t misc_off, recv_off;
+    size_t smem;  // dynamic shared memory, with 1 KB of alignment slack
+};
+
+static int epn_of(int E) { return E <= 16 ? 16 : E <= 32 ? 32 : E <= 64 ? 64 : 128; }
+
+static Plan make_plan(const moe_config& c)
 {
-    using G = Geo<EPB>;
-    static int done_mask = 0;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 31 || !((done_mask >> dev) & 1)) {
-        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EPB>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev < 31) done_mask |= 1 << dev;
-    }
-    EncodeTiledFn enc = encoder();
-    if (!enc) return cudaErrorInvalidValue;
-    CUtensorMap mX, mW;
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)c.D, (cuuint64_t)c.T};
-        cuuint64_t strides[1] = {(cuuint64_t)c.D * 2};
-        cuuint32_t box[2] = {64, BM};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        cuuint64_t dims[3] = {(cuuint64_t)G::EP, (cuuint64_t)c.D, 3};
-        cuuint64_t strides[2] = {(cuuint64_t)G::EP * 2, (cuuint64_t)G::EP * c.D * 2};
-        cuuint32_t box[3] = {64, 64, 1};
-        cuuint32_t es[3] = {1, 1, 1};
-        if (enc(&mW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(wsplit), dims,
-                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    Plan p{};
+    p.epn = epn_of(c.E);
+    const int tiles = router_tc_blocks(c);
     const int nkb = (c.D + BK - 1) / BK;
-    const unsigned splits = a.part ? (unsigned)((nkb + a.split_kb - 1) / a.split_kb) : 1u;
-    const dim3 grid((unsigned)((c.T + BM - 1) / BM), splits);
-    router_tc_kernel<EPB><<<grid, NUM_THREADS, G::SMEM, s>>>(mX, mW, a);
-    return cudaGetLastError();
+    p.splits = router_tc_splits(c);
+    p.split_kb = (nkb + p.splits - 1) / p.splits;
+    p.ctas_per_sm = (tiles * p.splits > 148 && p.epn <= 64) ? 2 : 1;
+    const size_t stage_bytes = stage_bytes_of(p.epn, c.E);
+    const size_t recv = (size_t)(p.splits - 1) * BM * p.epn * sizeof(float);
+    const size_t misc = align_up(sizeof(Misc), 1024);
+    // two CTAs per SM only while two stages of each still fit in half the SM
+    if (p.ctas_per_sm == 2 && 1024 + misc + 2 * stage_bytes > 112 * 1024) p.ctas_per_sm = 1;
+    const size_t budget = p.ctas_per_sm == 2 ? 112 * 1024 : 226 * 1024;
+    const size_t fixed = 1024 + misc + align_up(recv, 1024);
+    int st = (int)((budget - fixed) / stage_bytes);
+    if (st > MAX_STAGES) st = MAX_STAGES;
+    if (st < 2) st = 2;
+    // the epilogue scratch (and the statistics' last step) live in the ring
+    const size_t epi = (size_t)2 * BM * (p.epn + 1) * sizeof(float);
+    const size_t fin = (size_t)kStatD * sizeof(double) + (size_t)kStatC * sizeof(long long);
+    while ((size_t)st * stage_bytes < epi || (size_t)st * stage_bytes < fin) ++st;
+    p.stages = st;
+    p.stage_bytes = (int)stage_bytes;
+    p.misc_off = (uint32_t)((size_t)st * stage_bytes);
+    p.recv_off = p.misc_off + (uint32_t)misc;
+    p.smem = (size_t)p.recv_off + align_up(recv, 1024) + 1024;
+    return p;
+}
+
+template <int EPN, int KM, int MINB>
+static cudaError_t launch_t(const moe_config& c, const CUtensorMap& mX, const Args& a, const Plan& p,
+                            cudaStream_t s)
+{
+    auto kern = router_tc_kernel<EPN, KM, MINB>;
+    static PerDeviceFlag smem_set;
+    // the largest ring this instance is launched with (one attribute per device)
+    cudaError_t ae = opt_in_smem(smem_set, reinterpret_cast<const void*>(kern),
+                                 MINB == 2 ? 113 * 1024 : 227 * 1024);
+    if (ae != cudaSuccess) return ae;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)router_tc_blocks(c), (unsigned)p.splits, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)p.splits;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.splits > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, mX, a);
+}
+
+template <int EPN>
+static cudaError_t launch_k(const moe_config& c, const CUtensorMap& mX, const Args& a, const Plan& p,
+                            cudaStream_t s)
+{
+    const int km = c.K <= 2 ? 2 : c.K <= 4 ? 4 : 8;
+    if (p.ctas_per_sm == 2) {
+        if constexpr (EPN <= 64) {
+            return km == 2 ? launch_t<EPN, 2, 2>(c, mX, a, p, s)
+                 : km == 4 ? launch_t<EPN, 4, 2>(c, mX, a, p, s)
+                           : launch_t<EPN, 8, 2>(c, mX, a, p, s);
+        }
+        return cudaErrorInvalidValue;
+    }
+    return km == 2 ? launch_t<EPN, 2, 1>(c, mX, a, p, s)
+         : km == 4 ? launch_t<EPN, 4, 1>(c, mX, a, p, s)
+                   : launch_t<EPN, 8, 1>(c, mX, a, p, s);
 }
 
 }  // namespace rtc
@@ -459,48 +609,68 @@ int router_tc_splits(const moe_config& c)
     const int tiles = router_tc_blocks(c);
     const int nkb = (c.D + rtc::BK - 1) / rtc::BK;
     int sp = 148 / (tiles > 0 ? tiles : 1);
-    if (sp > 4) sp = 4;
+    if (sp > rtc::MAX_SPLITS) sp = rtc::MAX_SPLITS;
     if (sp > nkb / 8) sp = nkb / 8;
     if (sp < 2) return 1;
     const int per = (nkb + sp - 1) / sp;  // K blocks per split; every split non-empty
     return (nkb + per - 1) / per;
 }
 
-bool router_tc_partial(const moe_config& c)
-{
-    // the fused epilogue gives each token to one thread, which walks all E
-    // experts several times; above 16 experts the SIMT top-k kernel (a warp
-    // per token, the experts spread over its lanes) routes faster from the
-    // logits the tensor cores wrote
-    return router_tc_splits(c) > 1 || c.E > 16;
-}
-
-size_t router_tc_wsplit_bytes(const moe_config& c)
-{
-    const int ep = (c.E + 63) / 64 * 64;
-    return (size_t)3 * c.D * ep * sizeof(__nv_bfloat16);
-}
-
 cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
                              const float* w_router, const float* bias, const float* noise,
                              float* logits_out, float* probs_out, int32_t* ids, float* w,
                              float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
-                             int with_stats, void* wsplit_scratch, void* part_out, int* status,
-                             cudaStream_t s)
+                             float* mean_prob, float* losses, int* status, cudaStream_t s)
 {
     using namespace rtc;
-    const int ep = (c.E + 63) / 64 * 64;
-    __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(wsplit_scratch);
-    const int64_t n = (int64_t)c.D * ep;
-    int64_t blocks = (n + 255) / 256;
-    if (blocks > 148 * 8) blocks = 148 * 8;
-    router_wsplit_kernel<<<(unsigned)blocks, 256, 0, s>>>(w_router, wsplit, c.D, c.E, ep);
-    const int splits = router_tc_splits(c);
-    const int nkb = (c.D + BK - 1) / BK;
-    Args a{o, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_ent, blk_cnt,
-           c.T, c.D, c.E, c.K, with_stats, status,
-           router_tc_partial(c) ? static_cast<float*>(part_out) : nullptr, (nkb + splits - 1) / splits};
-    return ep == 64 ? launch_t<1>(c, x, wsplit, a, s) : launch_t<2>(c, x, wsplit, a, s);
+    const Plan p = make_plan(c);
+    EncodeTiledFn enc = encoder();
+    if (!enc) return cudaErrorInvalidValue;
+    CUtensorMap mX;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)c.D, (cuuint64_t)c.T};
+        cuuint64_t strides[1] = {(cuuint64_t)c.D * 2};
+        cuuint32_t box[2] = {64, BM};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    Args a{};
+    a.o = o;
+    a.w = w_router;
+    a.bias = bias;
+    a.noise = noise;
+    a.logits_out = logits_out;
+    a.probs_out = probs_out;
+    a.ids = ids;
+    a.wout = w;
+    a.blk_mp = blk_mp;
+    a.blk_z = blk_z;
+    a.blk_ent = blk_ent;
+    a.blk_cnt = blk_cnt;
+    a.mean_prob = mean_prob;
+    a.losses = losses;
+    a.counter = status + kRouterCounterWord;
+    a.T = c.T;
+    a.D = c.D;
+    a.E = c.E;
+    a.K = c.K;
+    a.with_stats = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
+    a.status = status;
+    a.stages = p.stages;
+    a.stage_bytes = p.stage_bytes;
+    a.splits = p.splits;
+    a.split_kb = p.split_kb;
+    a.misc_off = p.misc_off;
+    a.recv_off = p.recv_off;
+    switch (p.epn) {
+        case 16: return launch_k<16>(c, mX, a, p, s);
+        case 32: return launch_k<32>(c, mX, a, p, s);
+        case 64: return launch_k<64>(c, mX, a, p, s);
+        default: return launch_k<128>(c, mX, a, p, s);
+    }
 }
 
 }  // namespace moe

@@ -491,12 +491,12 @@ static bool map_out(CUtensorMap* m, const float* base, uint64_t Nh, uint64_t M, 
 // CTA pairs) can be resident at once, which sizes the persistent grid.
 template <bool PAIR> static cudaError_t prepare(int* units_out)
 {
-    static int cached[32];
+    static std::atomic<int> cached[32];  // 0 = not yet queried on that device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 32 && cached[dev] > 0) {
-        *units_out = cached[dev];
+    if (dev >= 0 && dev < 32 && cached[dev].load(std::memory_order_acquire) > 0) {
+        *units_out = cached[dev].load(std::memory_order_acquire);
         return cudaSuccess;
     }
     constexpr size_t smem = smem_bytes<PAIR>();
@@ -522,7 +522,7 @@ template <bool PAIR> static cudaError_t prepare(int* units_out)
         if (e != cudaSuccess) return e;
     }
     if (units < 1) return cudaErrorInvalidConfiguration;
-    if (dev < 32) cached[dev] = units;
+    if (dev >= 0 && dev < 32) cached[dev].store(units, std::memory_order_release);
     *units_out = units;
     return cudaSuccess;
 }
