@@ -554,8 +554,10 @@ MOE_API moe_status moe_selftest_wait_timeout(void *workspace, size_t workspace_b
 /*
  * Number of kernels one moe_forward call launches for this configuration:
  * router 1 (bf16 with E <= 128 and T >= 2048: the tensor-core router, which
- * also routes and finishes the statistics) or 2 (logits GEMM and top-k, plus
- * a split-sum when the GEMM is split over d_model), dispatch 3, gather 1,
+ * also routes and finishes the statistics) or 2 (the SIMT logits GEMM and the
+ * top-k kernel, plus a split-sum when that GEMM is split over d_model; also
+ * the path of a router weight that is not 16-byte aligned), dispatch 1 (3 when the
+ * chunks of 2048 assignments outnumber the resident blocks), gather 1,
  * expert GEMMs 2, shared expert 3 (when F_shared > 0: its row offsets and two
  * GEMMs), combine 1.  0 for an invalid configuration.
  */

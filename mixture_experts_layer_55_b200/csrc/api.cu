@@ -671,10 +671,12 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
 {
     if (check_config(cfg) != MOE_OK) return 0;
     const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
-    // dispatch 3, gather 1, expert GEMMs 2, combine 1; router: the tensor-core
-    // kernel alone, or the logits GEMM (+ its split sum) and the top-k kernel
-    if (router_tc_eligible(*cfg)) return 1 + 7 + shared;
-    return 2 + (router_plan(*cfg).splits > 1 ? 1 : 0) + 7 + shared;
+    // dispatch 1 (one cooperative kernel; 3 for more chunks than resident blocks),
+    // gather 1, expert GEMMs 2, combine 1; router: the tensor-core kernel alone,
+    // or logits (tensor-core, or SIMT + its split sum) and the top-k kernel
+    const int rest = 5 + (dispatch_index_fused(*cfg) ? 0 : 2) + shared;
+    if (router_tc_eligible(*cfg)) return 1 + rest;
+    return 2 + (router_plan(*cfg).splits > 1 ? 1 : 0) + rest;
 }
 
 moe_status moe_ep_workspace_size(int32_t world, int32_t experts_per_rank, size_t* bytes)

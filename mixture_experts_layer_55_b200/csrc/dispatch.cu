@@ -339,7 +339,7 @@ cudaError_t launch_dispatch_index(const moe_config& c, int64_t C, const int32_t*
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.d_cnt);
     int32_t* blk_base = reinterpret_cast<int32_t*>(ws + L.d_base);
     const int64_t max_rows = max_rows_of(c);
-    if (nch <= resident_index_blocks()) {
+    if (dispatch_index_fused(c) && nch <= resident_index_blocks()) {
         // one cooperative launch: all chunks' blocks resident at once
         int E = c.E;
         void* args[] = {(void*)&ids, (void*)&n, (void*)&E, (void*)&C, (void*)&blk_cnt,

@@ -75,6 +75,10 @@ inline int64_t dispatch_chunks(const moe_config& c)
 {
     return (c.T * c.K + kDispatchChunk - 1) / kDispatchChunk;
 }
+// The index pass runs as one cooperative kernel (a block per chunk, all
+// resident) up to one chunk per SM of a B200 (T*K <= 303104); beyond, or on a
+// GPU where that many blocks cannot be resident, as three kernels.
+inline bool dispatch_index_fused(const moe_config& c) { return dispatch_chunks(c) <= 148; }
 
 // ------------------------------------------------------ workspace layout --
 struct WsLayout {

@@ -525,12 +525,12 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
     float* blk_ent = reinterpret_cast<float*>(ws + L.r_ent);
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
     int* status = reinterpret_cast<int*>(ws + L.status);
-    // bf16 layers with enough tokens: one tensor-core kernel (its bulk copies of W_r
+    const float* part;
+    // bf16 layers with enough tokens: the tensor-core router (its bulk copies of W_r
     // need a 16-byte aligned W_r; an unaligned one takes the SIMT router)
     if (!logits_in && router_tc_eligible(c) && (reinterpret_cast<uintptr_t>(w_router) & 15u) == 0)
         return launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids, w, blk_mp,
                                 blk_z, blk_ent, blk_cnt, mean_prob, losses, status, s);
-    const float* part;
     if (logits_in) {
         part = logits_in;
         bias = nullptr;

@@ -34,20 +34,29 @@ MOE_DEVICE void finish_router_stats(const float* blk_mp, const float* blk_z, con
     const int ncol = E + 2;  // E probability sums (and counts), the z sum, the entropy sum
     int cc = nthreads / ncol;
     if (cc < 1) cc = 1;
-    // chunk sums over a fixed range of blocks each
+    // chunk sums over a fixed range of blocks each: the loads of 16 blocks are
+    // issued together, then added in block order
     for (int j = tid; j < ncol * cc; j += nthreads) {
         const int col = j % ncol, ch = j / ncol;
         const int b0 = (int)((int64_t)nb * ch / cc), b1 = (int)((int64_t)nb * (ch + 1) / cc);
+        const float* src = col < E ? blk_mp + col : (col == E ? blk_z : blk_ent);
+        const size_t stride = col < E ? (size_t)E : 1;
+        const int32_t* csrc = col < E ? blk_cnt + col : nullptr;
         double a = 0.0;
         long long c = 0;
-        for (int b = b0; b < b1; ++b) {
-            if (col < E) {
-                a += (double)__ldcg(blk_mp + (size_t)b * E + col);
-                c += __ldcg(blk_cnt + (size_t)b * E + col);
-            } else if (col == E) {
-                a += (double)__ldcg(blk_z + b);
-            } else {
-                a += (double)__ldcg(blk_ent + b);
+        for (int b = b0; b < b1; b += 16) {
+            float v[16];
+            int32_t n[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const bool in = b + u < b1;
+                v[u] = in ? __ldcg(src + (size_t)(b + u) * stride) : 0.f;
+                n[u] = (in && csrc) ? __ldcg(csrc + (size_t)(b + u) * stride) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                a += (double)v[u];
+                c += n[u];
             }
         }
         sd[j] = a;

@@ -16,20 +16,22 @@
 //
 // One CTA per 128 tokens (M = 128) and per split of d_model; N = EPN, the
 // expert count rounded up to 16, 32, 64 or 128.  Warps:
-//   warp 0      TMA: the x tile (128 tokens x 64 of d_model, 128-byte
-//               swizzle) and a bulk copy of the 64 x E fp32 slice of W_r of
-//               each stage of a deep ring (up to 10 stages)
+//   warp 0      TMA: the x tiles (128 tokens x 64 of d_model, 128-byte
+//               swizzle) into a deep ring (up to 10 stages of 16 KB)
 //   warp 1      tcgen05.mma, three per K step of 16 (one per weight term)
-//   warps 2..5  first the weight split: each stage's fp32 slice is split in
-//               shared memory into its three bf16 terms, written K-major
-//               (expert rows of 64 d_model values, 128-byte swizzle) next
-//               to the x tile, so no weight kernel runs before this one and
-//               the weight tiles are E rows wide, not a padded 64; then the
-//               epilogue, one token row per
-//               thread: logits (+ bias + noise), max, softmax sum and
-//               entropy, scores, the group limit, top-K by (logit +
-//               selection bias desc, id asc) with an unrolled insertion
-//               network, weights, normalised scores, and the per-CTA
+//   warps 2..5  first the weight split: the 64 x E fp32 slice of W_r of each
+//               K block arrives by bulk copy in a shallow ring of its own,
+//               is split in shared memory into its three bf16 terms and
+//               written K-major (expert rows of 64 d_model values, 128-byte
+//               swizzle) into a shallow ring of weight tiles, so no weight
+//               kernel runs before this one, the weight tiles are E rows
+//               wide, not a padded 64, and the x ring keeps its depth; then
+//               the epilogue, one token row per
+//               thread: logits (+ bias + noise), max and top-K by (logit +
+//               selection bias desc, id asc, an unrolled insertion network)
+//               in one pass over the experts, softmax sum and entropy
+//               (closed form) and scores in a second, the group limit when
+//               set, weights, normalised scores in a third, and the per-CTA
 //               statistics (counts by shared-memory atomics; column sums
 //               in a fixed order).
 // When the token tiles alone leave most SMs idle, d_model is split over a
@@ -58,21 +60,20 @@ constexpr int CONVERTER_WARPS = 4;
 
 template <int EPN> struct Geo {
     static constexpr int TERM_BYTES = EPN * 128;  // EPN expert rows x 64 d_model (bf16)
-    static constexpr int W_OFF = A_BYTES + 3 * TERM_BYTES;  // the stage's fp32 W_r slice
+    static constexpr int B_BYTES = 3 * TERM_BYTES;
     static constexpr int TMEM_COLS = EPN < 32 ? 32 : EPN;
     static constexpr int LDS = EPN + 1;  // epilogue row stride in floats (odd: conflict-free)
 };
 
-// Bytes of one ring stage: x tile, three weight terms, the fp32 slice (64 x E).
-inline size_t stage_bytes_of(int epn, int E)
-{
-    return align_up((size_t)A_BYTES + (size_t)3 * epn * 128 + (size_t)64 * E * 4, 1024);
-}
+constexpr int WDEPTH = 2;  // slots of the weight rings (fp32 slices and their bf16 terms)
 
 struct Misc {
-    uint64_t lfull[MAX_STAGES];  // the stage's x tile and fp32 weights have landed
-    uint64_t full[MAX_STAGES];   // and its weight terms are written: the MMAs may read it
-    uint64_t empty[MAX_STAGES];
+    uint64_t xfull[MAX_STAGES];   // x tile landed
+    uint64_t xempty[MAX_STAGES];  // its MMAs are done
+    uint64_t wl[WDEPTH];          // fp32 weight slice landed
+    uint64_t bfull[WDEPTH];       // its bf16 terms are written
+    uint64_t bempty[WDEPTH];      // their MMAs are done
+    uint64_t wfree[WDEPTH];       // every weight warp is done reading the fp32 slice
     uint64_t tfull;
     uint32_t tmem_base;
     int abort_flag;
@@ -103,8 +104,10 @@ struct Args {
     int D, E, K;
     int with_stats;
     int* status;
-    int stages;               // ring depth
-    int stage_bytes;          // bytes per ring stage
+    int stages;               // depth of the x ring (16 KB stages)
+    uint32_t b_off;           // the bf16 weight-term ring (WDEPTH x 3 x EPN x 128 bytes)
+    uint32_t w_off;           // the fp32 weight-slice ring (WDEPTH x w_slot bytes)
+    uint32_t w_slot;          // bytes per fp32 slice slot (64 x E x 4, rounded up)
     int splits;               // CTAs per token tile (cluster size along y)
     int split_kb;             // K blocks per split
     uint32_t misc_off;        // byte offsets in the aligned shared memory
@@ -118,17 +121,21 @@ MOE_DEVICE void st_cluster_f32(uint32_t cluster_addr, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
 }
 
-// The three bf16 terms of two fp32 weights, packed in pairs.
+// The three bf16 terms of two fp32 weights, packed in pairs (a in the low
+// half): hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid), each pair
+// rounded by one paired conversion.
+MOE_DEVICE uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 MOE_DEVICE void split3(float a, float b, uint32_t& hi, uint32_t& mid, uint32_t& lo)
 {
-    const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
-    const float ra = a - __bfloat162float(ha), rb = b - __bfloat162float(hb);
-    const __nv_bfloat16 ma = __float2bfloat16_rn(ra), mb = __float2bfloat16_rn(rb);
-    const __nv_bfloat16 la = __float2bfloat16_rn(ra - __bfloat162float(ma));
-    const __nv_bfloat16 lb = __float2bfloat16_rn(rb - __bfloat162float(mb));
-    hi = (uint32_t)__bfloat16_as_ushort(ha) | ((uint32_t)__bfloat16_as_ushort(hb) << 16);
-    mid = (uint32_t)__bfloat16_as_ushort(ma) | ((uint32_t)__bfloat16_as_ushort(mb) << 16);
-    lo = (uint32_t)__bfloat16_as_ushort(la) | ((uint32_t)__bfloat16_as_ushort(lb) << 16);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const float ra = a - hf.x, rb = b - hf.y;
+    const __nv_bfloat162 m = __floats2bfloat162_rn(ra, rb);
+    const float2 mf = __bfloat1622float2(m);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(ra - mf.x, rb - mf.y);
+    hi = bf16x2_bits(h);
+    mid = bf16x2_bits(m);
+    lo = bf16x2_bits(l);
 }
 
 template <int EPN, int KM, int MINB>
@@ -137,11 +144,12 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
 {
     using G = Geo<EPN>;
     constexpr int TERM = G::TERM_BYTES, LDS = G::LDS;
-    const int STAGE_BYTES = a.stage_bytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* stages = smem;
+    uint8_t* xring = smem;              // S x 16 KB; the whole ring area is the epilogue's scratch
+    uint8_t* bring = smem + a.b_off;    // WDEPTH x B_BYTES
+    uint8_t* wring = smem + a.w_off;    // WDEPTH x w_slot
     Misc* m = reinterpret_cast<Misc*>(smem + a.misc_off);
     float* recv = reinterpret_cast<float*>(smem + a.recv_off);
     const int S = a.stages;
@@ -151,13 +159,19 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     const int num_kb = (a.D + BK - 1) / BK;
     const int kb_begin = split * a.split_kb;                // never empty (host guarantee)
     const int kb_end = min(num_kb, kb_begin + a.split_kb);
+    const int nkb = kb_end - kb_begin;
     const int E = a.E;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&m->lfull[s], 1);               // the producer, with the bytes
-            mbar_init(&m->full[s], CONVERTER_WARPS);  // the weight warps
-            mbar_init(&m->empty[s], 1);
+            mbar_init(&m->xfull[s], 1);
+            mbar_init(&m->xempty[s], 1);
+        }
+        for (int j = 0; j < WDEPTH; ++j) {
+            mbar_init(&m->wl[j], 1);
+            mbar_init(&m->bfull[j], CONVERTER_WARPS);
+            mbar_init(&m->bempty[j], 1);
+            mbar_init(&m->wfree[j], CONVERTER_WARPS);
         }
         mbar_init(&m->tfull, 1);
         m->abort_flag = 0;
@@ -166,19 +180,18 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         prefetch_tmap(&tmX);
     }
     if (warp >= 2) {
-        // weight tiles: rows E .. EPN-1 (if any) stay zero in every stage
+        // weight terms: rows E .. EPN-1 (if any) stay zero in every slot
         const int tid = threadIdx.x - 64;
         m->cnt[tid] = 0;
         const int pad = EPN - E;
         if (pad > 0) {
-            const int per_stage = 3 * pad * 8;  // 16-byte chunks
-            for (int i = tid; i < S * per_stage; i += 128) {
-                const int s = i / per_stage;
-                int r = i % per_stage;
+            const int per_slot = 3 * pad * 8;  // 16-byte chunks
+            for (int i = tid; i < WDEPTH * per_slot; i += 128) {
+                const int j = i / per_slot;
+                int r = i % per_slot;
                 const int p = r / (pad * 8);
                 r %= pad * 8;
-                uint8_t* dst = stages + (size_t)s * STAGE_BYTES + A_BYTES + p * TERM +
-                               (E + r / 8) * 128 + (r % 8) * 16;
+                uint8_t* dst = bring + (size_t)j * G::B_BYTES + p * TERM + (E + r / 8) * 128 + (r % 8) * 16;
                 *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
@@ -192,24 +205,26 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
     volatile int* abort_flag = &m->abort_flag;
+    // the fp32 weight slice of K block kb into slot j (issued by one converter thread)
+    auto load_w = [&](int kb, int j) {
+        const int d0 = kb * BK;
+        const int rows = min(BK, a.D - d0);  // a multiple of 8 (D % 8 == 0)
+        const uint32_t bytes = (uint32_t)rows * (uint32_t)E * 4u;
+        mbar_arrive_expect_tx(&m->wl[j], bytes);
+        bulk_load_g2s(wring + (size_t)j * a.w_slot, a.w + (size_t)d0 * E, bytes, &m->wl[j]);
+    };
 
     if (warp == 0) {
         if (lane == 0) {
-            // ------------------------------------------------ producer: x tile + fp32 weights
+            // ------------------------------------------------ x tiles, S stages ahead
             int stage = 0;
             uint32_t phase = 0;
             int last_phase[MAX_STAGES];
             for (int s = 0; s < MAX_STAGES; ++s) last_phase[s] = -1;
             for (int kb = kb_begin; kb < kb_end; ++kb) {
-                if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
-                uint8_t* st = stages + (size_t)stage * STAGE_BYTES;
-                uint64_t* fb = &m->lfull[stage];
-                const int d0 = kb * BK;
-                const int rows = min(BK, a.D - d0);  // a multiple of 8 (D % 8 == 0)
-                const uint32_t wbytes = (uint32_t)rows * (uint32_t)E * 4u;
-                mbar_arrive_expect_tx(fb, A_BYTES + wbytes);
-                tma_load_2d(st, &tmX, d0, (int32_t)t0, fb);
-                bulk_load_g2s(st + G::W_OFF, a.w + (size_t)d0 * E, wbytes, fb);
+                if (!mbar_wait(&m->xempty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
+                mbar_arrive_expect_tx(&m->xfull[stage], A_BYTES);
+                tma_load_2d(xring + (size_t)stage * A_BYTES, &tmX, kb * BK, (int32_t)t0, &m->xfull[stage]);
                 last_phase[stage] = (int)phase;
                 if (++stage == S) {
                     stage = 0;
@@ -219,34 +234,30 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             // every copy issued has landed before the ring is reused or the CTA exits
             for (int s = 0; s < S; ++s)
                 if (last_phase[s] >= 0)
-                    mbar_wait(&m->lfull[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
+                    mbar_wait(&m->xfull[s], (uint32_t)last_phase[s], a.status, 511, nullptr);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = umma_idesc_bf16(BM, EPN, 0, 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
-                if (!mbar_wait(&m->full[stage], phase, a.status, 520, abort_flag)) break;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % S, j = i % WDEPTH;
+                if (!mbar_wait(&m->xfull[s], (uint32_t)((i / S) & 1), a.status, 520, abort_flag)) break;
+                if (!mbar_wait(&m->bfull[j], (uint32_t)((i / WDEPTH) & 1), a.status, 521, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t sA = smem_u32(stages + (size_t)stage * STAGE_BYTES);
-                const uint32_t sB = sA + A_BYTES;
+                const uint32_t sA = smem_u32(xring + (size_t)s * A_BYTES);
+                const uint32_t sB = smem_u32(bring + (size_t)j * G::B_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
 #pragma unroll
                     for (int p = 0; p < 3; ++p) {
                         const uint64_t bdesc = umma_desc_sw128(sB + p * TERM + kk * 32, 16, 1024);
-                        umma_f16_ss(tmem_base, adesc, bdesc, idesc,
-                                    (kb != kb_begin || kk || p) ? 1u : 0u);
+                        umma_f16_ss(tmem_base, adesc, bdesc, idesc, (i || kk || p) ? 1u : 0u);
                     }
                 }
-                umma_commit(&m->empty[stage]);
-                if (++stage == S) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                umma_commit(&m->xempty[s]);
+                umma_commit(&m->bempty[j]);
             }
             umma_commit(&m->tfull);  // also the drain: every MMA done once it fires
         }
@@ -254,23 +265,28 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         // ------------------------------------------------ weight split (warps 2..5)
         const int tid = threadIdx.x - 64;
         {
-            int stage = 0;
-            uint32_t phase = 0;
+            int issued = 0;  // fp32 slices issued (slot = index % WDEPTH)
+            if (tid == 0)
+                for (; issued < WDEPTH && issued < nkb; ++issued) load_w(kb_begin + issued, issued);
             const int pairs = E * 8;  // (expert, 8-wide chunk of d_model)
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
-                if (!mbar_wait(&m->lfull[stage], phase, a.status, 540, abort_flag)) break;
-                uint8_t* sB = stages + (size_t)stage * STAGE_BYTES + A_BYTES;
-                const float* wsm = reinterpret_cast<const float*>(sB - A_BYTES + G::W_OFF);
-                const int d0 = kb * BK;
-                for (int i = tid; i < pairs; i += 128) {
-                    const int e = i % E, c = i / E;
+            int i = 0;
+            for (; i < nkb; ++i) {
+                const int j = i % WDEPTH;
+                const uint32_t ph = (uint32_t)((i / WDEPTH) & 1);
+                if (!mbar_wait(&m->wl[j], ph, a.status, 540, abort_flag)) break;
+                if (!mbar_wait(&m->bempty[j], ph ^ 1u, a.status, 541, abort_flag)) break;
+                uint8_t* sB = bring + (size_t)j * G::B_BYTES;
+                const float* wsm = reinterpret_cast<const float*>(wring + (size_t)j * a.w_slot);
+                const int d0 = (kb_begin + i) * BK;
+                for (int q = tid; q < pairs; q += 128) {
+                    const int e = q % E, c = q / E;
                     const bool in = d0 + c * 8 < a.D;  // D % 8 == 0: a chunk is all in or all out
                     float v[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) v[j] = in ? wsm[(c * 8 + j) * E + e] : 0.f;
+                    for (int jj = 0; jj < 8; ++jj) v[jj] = in ? wsm[(c * 8 + jj) * E + e] : 0.f;
                     uint32_t h[4], md[4], l[4];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) split3(v[2 * j], v[2 * j + 1], h[j], md[j], l[j]);
+                    for (int jj = 0; jj < 4; ++jj) split3(v[2 * jj], v[2 * jj + 1], h[jj], md[jj], l[jj]);
                     const int off = e * 128 + ((c ^ (e & 7)) << 4);
                     *reinterpret_cast<uint4*>(sB + off) = make_uint4(h[0], h[1], h[2], h[3]);
                     *reinterpret_cast<uint4*>(sB + TERM + off) = make_uint4(md[0], md[1], md[2], md[3]);
@@ -278,17 +294,26 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 }
                 fence_proxy_async_smem();  // visible to the tensor cores
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&m->full[stage]);
-                if (++stage == S) {
-                    stage = 0;
-                    phase ^= 1u;
+                if (lane == 0) {
+                    mbar_arrive(&m->bfull[j]);
+                    mbar_arrive(&m->wfree[j]);
+                }
+                // refill fp32 slot j once every weight warp is done with it
+                if (tid == 0 && issued < nkb) {
+                    if (!mbar_wait(&m->wfree[j], ph, a.status, 543, abort_flag)) break;
+                    load_w(kb_begin + issued, issued % WDEPTH);
+                    ++issued;
                 }
             }
+            // after an early exit, the slices still in flight land before the CTA goes on
+            if (tid == 0)
+                for (int k = i; k < issued; ++k)
+                    mbar_wait(&m->wl[k % WDEPTH], (uint32_t)((k / WDEPTH) & 1), a.status, 542, nullptr);
         }
         // ------------------------------------------------ accumulators out of tensor memory
         const int quad = warp & 3;        // the lane quadrant this warp may read
         const int r = quad * 32 + lane;   // token row in the tile
-        float* Ls = reinterpret_cast<float*>(stages);  // [BM][LDS]
+        float* Ls = reinterpret_cast<float*>(xring);  // [BM][LDS]
         const bool ok = mbar_wait(&m->tfull, 0, a.status, 530, abort_flag);
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -325,9 +350,32 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         const bool valid = t < a.T;
         const int K = a.K;
         const RouteOpts& o = a.o;
-        float* Ls = reinterpret_cast<float*>(stages);  // logits, then normalised scores
-        float* Xs = Ls + BM * LDS;                     // exp(L - max), then scores
-        // pass 1: logits (own K range + the other splits in order, + bias + noise)
+        float* Ls = reinterpret_cast<float*>(xring);  // logits, then normalised scores
+        float* Xs = Ls + BM * LDS;                     // scores: exp(L - max), or sigmoid(L)
+        const int G = o.n_groups, gsz = E / G;
+        // top-K by (u desc, id asc), u = L + selection bias: an unrolled insertion
+        // network of KM >= K slots (a displaced entry carried down keeps that order)
+        float tv[KM];
+        int ti[KM];
+#pragma unroll
+        for (int k = 0; k < KM; ++k) {
+            tv[k] = -INFINITY;
+            ti[k] = 0x7fffffff;
+        }
+        auto insert = [&](float xv, int xi) {
+#pragma unroll
+            for (int k = 0; k < KM; ++k) {
+                const bool gt = xv > tv[k] || (xv == tv[k] && xi < ti[k]);
+                const float nv = gt ? xv : tv[k];
+                const int ni = gt ? xi : ti[k];
+                xv = gt ? tv[k] : xv;
+                xi = gt ? ti[k] : xi;
+                tv[k] = nv;
+                ti[k] = ni;
+            }
+        };
+        // pass 1: logits (own K range + the other splits in order, + bias + noise),
+        // their maximum, and (without a group limit) the top-K
         float mx = -INFINITY;
         for (int e = 0; e < E; ++e) {
             float L = Ls[r * LDS + e];
@@ -337,32 +385,31 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             if (a.logits_out && valid) a.logits_out[t * E + e] = L;
             Ls[r * LDS + e] = L;
             mx = fmaxf(mx, L);
+            if (G == 1) insert(L + (o.sel_bias ? o.sel_bias[e] : 0.f), e);
         }
-        // pass 2: softmax sum
-        float ssum = 0.f;
+        // pass 2: softmax sum, sum of exp(L - max) (L - max) for the entropy, and
+        // the scores (sigmoid scores and their sum with score_func sigmoid)
+        float ssum = 0.f, s1 = 0.f, scsum = 0.f;
         for (int e = 0; e < E; ++e) {
-            const float x = expf(Ls[r * LDS + e] - mx);
-            Xs[r * LDS + e] = x;
+            const float L = Ls[r * LDS + e];
+            const float x = expf(L - mx);
             ssum += x;
+            s1 = fmaf(x, L - mx, s1);
+            float sc = x;
+            if (o.score_func == 1) {
+                sc = 1.0f / (1.0f + expf(-L));
+                scsum += sc;
+            }
+            Xs[r * LDS + e] = sc;
         }
         const float inv = 1.0f / ssum;
         const float lss = logf(ssum);
-        // pass 3: entropy -sum q log(max(q, 1e-9)) with log q = (L - max) - log(sum),
-        // scores (softmax q or sigmoid) into Xs, their sum
-        const float log_floor = logf(1e-9f);
-        float ent = 0.f, scsum = 0.f;
-        for (int e = 0; e < E; ++e) {
-            const float L = Ls[r * LDS + e];
-            const float q = Xs[r * LDS + e] * inv;
-            ent -= q * (q >= 1e-9f ? (L - mx) - lss : log_floor);
-            const float sc = o.score_func == 1 ? 1.0f / (1.0f + expf(-L)) : q;
-            Xs[r * LDS + e] = sc;
-            scsum += sc;
-        }
-        // group limit: a group's score is its best selection score u = L + b
-        uint32_t keep = 0xffffffffu;
-        const int G = o.n_groups, gsz = E / G;
+        // entropy -sum q log q = log(sum) - sum q (L - max), q = exp(L - max) / sum
+        const float ent = lss - s1 * inv;
+        // softmax scores are Xs * inv, sigmoid scores Xs itself
+        const float sc_mul = o.score_func == 1 ? 1.0f : inv;
         if (G > 1) {
+            // group limit: a group's score is its best selection score u = L + b
             float gm[32];
 #pragma unroll
             for (int g = 0; g < 32; ++g) {
@@ -371,7 +418,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                     for (int e = g * gsz; e < (g + 1) * gsz; ++e)
                         gm[g] = fmaxf(gm[g], Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f));
             }
-            keep = 0;
+            uint32_t keep = 0;
             for (int rr = 0; rr < o.topk_groups; ++rr) {
                 float bv = -INFINITY;
                 int bg = 0;
@@ -383,38 +430,15 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                     }
                 keep |= 1u << bg;
             }
-        }
-        // pass 4: top-K over the eligible experts by (u desc, id asc), an unrolled
-        // insertion network of KM >= K slots (a displaced entry carried down
-        // keeps that order too)
-        float tv[KM];
-        int ti[KM];
-#pragma unroll
-        for (int k = 0; k < KM; ++k) {
-            tv[k] = -INFINITY;
-            ti[k] = 0x7fffffff;
-        }
-        for (int e = 0; e < E; ++e) {
-            if (G > 1 && !((keep >> (e / gsz)) & 1u)) continue;
-            float xv = Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f);
-            int xi = e;
-#pragma unroll
-            for (int k = 0; k < KM; ++k) {
-                const bool gt = xv > tv[k] || (xv == tv[k] && xi < ti[k]);
-                const float nv = gt ? xv : tv[k];
-                const int ni = gt ? xi : ti[k];
-                xv = gt ? tv[k] : xv;
-                xi = gt ? ti[k] : xi;
-                tv[k] = nv;
-                ti[k] = ni;
-            }
+            for (int e = 0; e < E; ++e)
+                if ((keep >> (e / gsz)) & 1u) insert(Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f), e);
         }
         // weights from the scores of the selected experts
         float sk[KM];
         float ssel = 0.f;
 #pragma unroll
         for (int k = 0; k < KM; ++k) {
-            sk[k] = k < K ? Xs[r * LDS + ti[k]] : 0.f;
+            sk[k] = k < K ? Xs[r * LDS + ti[k]] * sc_mul : 0.f;
             ssel += sk[k];
         }
         if (valid) {
@@ -426,8 +450,8 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                     if (a.with_stats) atomicAdd(&m->cnt[ti[k]], 1);  // integer: order-free
                 }
         }
-        // pass 5: normalised scores into Ls (and probs_out); rows past T give nothing
-        const float scinv = o.score_func == 1 ? 1.0f / scsum : 1.0f;
+        // pass 3: normalised scores into Ls (and probs_out); rows past T give nothing
+        const float scinv = o.score_func == 1 ? 1.0f / scsum : inv;
         for (int e = 0; e < E; ++e) {
             const float pn = Xs[r * LDS + e] * scinv;
             Ls[r * LDS + e] = valid ? pn : 0.f;
@@ -477,7 +501,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     if (split == 0 && a.with_stats && m->last) {
         // the last CTA: the statistics of the whole grid (all 192 threads)
         __threadfence();
-        double* sd = reinterpret_cast<double*>(stages);
+        double* sd = reinterpret_cast<double*>(xring);
         long long* sc = reinterpret_cast<long long*>(sd + kStatD);
         finish_router_stats(a.blk_mp, a.blk_z, a.blk_ent, a.blk_cnt, (int)gridDim.x, a.T, E, a.K,
                             a.mean_prob, a.losses, sd, sc, NUM_THREADS, (int)threadIdx.x,
@@ -509,10 +533,13 @@ static EncodeTiledFn encoder()
     return fn;
 }
 
-// Ring depth and shared-memory layout for `ctas_per_sm` CTAs on each SM.
+// Ring depth and shared-memory layout for `ctas_per_sm` CTAs on each SM:
+// [x ring: stages x 16 KB][weight terms: WDEPTH x 3 x EPN x 128][fp32 slices:
+// WDEPTH x w_slot][Misc][split partials]; the rings together are the
+// epilogue's scratch.
 struct Plan {
-    int epn, splits, split_kb, ctas_per_sm, stages, stage_bytes;
-    uint32_t misc_off, recv_off;
+    int epn, splits, split_kb, ctas_per_sm, stages;
+    uint32_t b_off, w_off, w_slot, misc_off, recv_off;
     size_t smem;  // dynamic shared memory, with 1 KB of alignment slack
 };
 
@@ -526,24 +553,28 @@ static Plan make_plan(const moe_config& c)
     const int nkb = (c.D + BK - 1) / BK;
     p.splits = router_tc_splits(c);
     p.split_kb = (nkb + p.splits - 1) / p.splits;
-    p.ctas_per_sm = (tiles * p.splits > 148 && p.epn <= 64) ? 2 : 1;
-    const size_t stage_bytes = stage_bytes_of(p.epn, c.E);
+    const size_t b_bytes = (size_t)3 * p.epn * 128;
+    p.w_slot = (uint32_t)align_up((size_t)64 * c.E * 4, 1024);
     const size_t recv = (size_t)(p.splits - 1) * BM * p.epn * sizeof(float);
     const size_t misc = align_up(sizeof(Misc), 1024);
-    // two CTAs per SM only while two stages of each still fit in half the SM
-    if (p.ctas_per_sm == 2 && 1024 + misc + 2 * stage_bytes > 112 * 1024) p.ctas_per_sm = 1;
-    const size_t budget = p.ctas_per_sm == 2 ? 112 * 1024 : 226 * 1024;
-    const size_t fixed = 1024 + misc + align_up(recv, 1024);
-    int st = (int)((budget - fixed) / stage_bytes);
-    if (st > MAX_STAGES) st = MAX_STAGES;
-    if (st < 2) st = 2;
-    // the epilogue scratch (and the statistics' last step) live in the ring
+    const size_t fixed = 1024 + WDEPTH * (b_bytes + p.w_slot) + misc + align_up(recv, 1024);
+    // the epilogue scratch (and the statistics' last step) live in the rings
     const size_t epi = (size_t)2 * BM * (p.epn + 1) * sizeof(float);
     const size_t fin = (size_t)kStatD * sizeof(double) + (size_t)kStatC * sizeof(long long);
-    while ((size_t)st * stage_bytes < epi || (size_t)st * stage_bytes < fin) ++st;
-    p.stages = st;
-    p.stage_bytes = (int)stage_bytes;
-    p.misc_off = (uint32_t)((size_t)st * stage_bytes);
+    auto stages_for = [&](size_t budget) {
+        if (budget <= fixed) return 0;
+        int st = (int)((budget - fixed) / A_BYTES);
+        if (st > MAX_STAGES) st = MAX_STAGES;
+        const size_t rings = (size_t)st * A_BYTES + WDEPTH * (b_bytes + p.w_slot);
+        return (rings >= epi && rings >= fin) ? st : 0;
+    };
+    // two CTAs per SM when the tiles outnumber the SMs and each still gets 3 x stages
+    p.ctas_per_sm = 1;
+    if (tiles * p.splits > 148 && p.epn <= 64 && stages_for(112 * 1024) >= 3) p.ctas_per_sm = 2;
+    p.stages = stages_for(p.ctas_per_sm == 2 ? 112 * 1024 : 226 * 1024);
+    p.b_off = (uint32_t)((size_t)p.stages * A_BYTES);
+    p.w_off = p.b_off + (uint32_t)(WDEPTH * b_bytes);
+    p.misc_off = p.w_off + (uint32_t)(WDEPTH * p.w_slot);
     p.recv_off = p.misc_off + (uint32_t)misc;
     p.smem = (size_t)p.recv_off + align_up(recv, 1024) + 1024;
     return p;
@@ -578,17 +609,19 @@ template <int EPN>
 static cudaError_t launch_k(const moe_config& c, const CUtensorMap& mX, const Args& a, const Plan& p,
                             cudaStream_t s)
 {
-    const int km = c.K <= 2 ? 2 : c.K <= 4 ? 4 : 8;
+    const int km = c.K <= 2 ? 2 : c.K <= 4 ? 4 : c.K <= 6 ? 6 : 8;
     if (p.ctas_per_sm == 2) {
         if constexpr (EPN <= 64) {
             return km == 2 ? launch_t<EPN, 2, 2>(c, mX, a, p, s)
                  : km == 4 ? launch_t<EPN, 4, 2>(c, mX, a, p, s)
+                 : km == 6 ? launch_t<EPN, 6, 2>(c, mX, a, p, s)
                            : launch_t<EPN, 8, 2>(c, mX, a, p, s);
         }
         return cudaErrorInvalidValue;
     }
     return km == 2 ? launch_t<EPN, 2, 1>(c, mX, a, p, s)
          : km == 4 ? launch_t<EPN, 4, 1>(c, mX, a, p, s)
+         : km == 6 ? launch_t<EPN, 6, 1>(c, mX, a, p, s)
                    : launch_t<EPN, 8, 1>(c, mX, a, p, s);
 }
 
@@ -660,7 +693,9 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
     a.with_stats = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
     a.status = status;
     a.stages = p.stages;
-    a.stage_bytes = p.stage_bytes;
+    a.b_off = p.b_off;
+    a.w_off = p.w_off;
+    a.w_slot = p.w_slot;
     a.splits = p.splits;
     a.split_kb = p.split_kb;
     a.misc_off = p.misc_off;

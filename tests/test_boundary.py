@@ -154,16 +154,19 @@ def test_selftest_argument_errors(lib):
 
 
 def test_forward_kernel_count(lib):
-    # SIMT router: logits GEMM + top-k (the top-k kernel finishes the statistics)
-    assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 9
+    # dispatch 1 (one cooperative kernel), gather 1, expert GEMMs 2, combine 1, and the
+    # router: SIMT logits GEMM + top-k (the top-k kernel finishes the statistics)
+    assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 7
     # tensor-core router: one kernel for routing and statistics, with or without the
     # d_model split (64 tiles of 128 tokens: a cluster of 2 CTAs per tile)
-    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=16, K=2)) == 8
-    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=64, K=6)) == 8
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 8
-    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 10  # split SIMT router
+    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=16, K=2)) == 6
+    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=64, K=6)) == 6
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 6
+    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 8  # split SIMT router
     assert B.forward_kernel_count(_cfg(K=0)) == 0
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256)) == 11
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256)) == 9
+    # more chunks of 2048 assignments than SMs: the three-kernel index pass
+    assert B.forward_kernel_count(_cfg(T=160000, D=256, F=256, E=8, K=2)) == 8
 
 
 def test_status_strings_and_trace_table(lib):

@@ -181,6 +181,40 @@ def test_update_selection_bias_matches_oracle(cuda_ok):
     assert float(b[2]) == float(bias0[2])
 
 
+def test_unaligned_router_weight_takes_the_simt_router(cuda_ok):
+    """A router weight that is not 16-byte aligned cannot be bulk-copied by the
+    tensor-core router; the SIMT router routes instead, with the same results
+    against the oracle."""
+    wl = _wl("unaligned_wr", T=2304, D=128, F=32, E=12, K=3, bias="zipf", seed=47)
+    inp_cpu = make_inputs(wl, device="cpu")
+    inp = _to_dev(inp_cpu)
+    buf = torch.empty(wl.D * wl.E + 1, device="cuda")
+    w_un = buf[1:].view(wl.D, wl.E)
+    w_un.copy_(inp["w_router"])
+    assert w_un.data_ptr() % 16 != 0
+    inp["w_router"] = w_un
+    b = Bufs(wl)
+    b.run_ops(inp)
+    check_logits(wl, inp_cpu, b.logits.cpu().numpy())
+    check_routing(wl, b)
+
+
+def test_dispatch_index_three_kernel_path(cuda_ok):
+    """More chunks of 2048 assignments than SMs (T*K = 320000): the index pass
+    runs as three kernels instead of one cooperative launch; routing, counts,
+    kept, offsets, perm and row_of are bit-exact against the oracle, with drops."""
+    wl = _wl("many_chunks", T=160000, D=64, F=32, E=8, K=2, capacity_factor=1.0, noise=True,
+             seed=46)
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    b = Bufs(wl)
+    b.run_ops(inp)
+    rt = check_routing(wl, b)
+    assert int((rt["row_of"] < 0).sum()) > 0
+    R = int(rt["offsets"][-1])
+    src = torch.from_numpy(rt["perm"][:R] // wl.K).long().cuda()
+    assert torch.equal(b.x_perm[:R], inp["x"].index_select(0, src))
+
+
 def test_determinism_bitwise(cuda_ok):
     wl = _wl("det", T=1000, D=128, F=128, E=16, K=4, bias="zipf", seed=12)
     inp = _to_dev(make_inputs(wl, device="cpu"))
