@@ -46,3 +46,37 @@ def test_aggregate_single_rank():
     ms_total, ms_step, value = bench.aggregate(100.0, 1, 8192, 20, "cpu")
     assert ms_total == 100.0 and ms_step == 5.0
     assert abs(value - 8192 / 5e-3) < 1e-6
+
+
+def test_cpu_baseline_batches_each_expert_on_all_threads():
+    """The oracle baseline on the tiny fp32 layer: every sampled row goes to the
+    oracle once, all host threads are used, the value is positive, and the
+    single-thread figure is the slower one."""
+    import oracle
+    from workloads import WORKLOADS
+    r = bench.cpu_baseline(WORKLOADS["tiny_fp32"], seconds=1.0)
+    assert r["kind"] == "oracle" and r["cores"] == oracle.num_threads()
+    assert r["value"] > 0 and r["single_thread"]["value"] > 0
+    if r["cores"] > 1:
+        assert r["value"] > r["single_thread"]["value"]
+    assert "1024 expert rows over 8 experts" in r["sample"]
+
+
+def test_sample_tokens_respects_the_expert_budget():
+    """The CPU sample stops adding tokens that need experts beyond the host
+    weight budget (1.5 G elements), and otherwise follows the random order."""
+    import numpy as np
+    from workloads import WORKLOADS
+    wl = WORKLOADS["decode_e256"]  # 3 * 7168 * 2048 elements per expert: 34 experts fit
+    rng = np.random.default_rng(0)
+    ids = np.stack([rng.permutation(wl.E)[:wl.K] for _ in range(wl.T)])
+    kept = np.ones_like(ids, dtype=bool)
+    toks, experts = bench._sample_tokens(wl, ids, kept, np.arange(wl.T), rows_target=1e9)
+    assert len(experts) <= 34 and len(toks) >= 1
+    assert set(experts) == {int(e) for t in toks for e in ids[t]}
+
+
+def test_extra_config_workloads():
+    w = bench.config_workload("mixtral_8x+shared")
+    assert w.F_shared == w.F == 14336 and w.T == 8192
+    assert bench.config_workload("fine_skewed").E == 64
