@@ -35,13 +35,15 @@ MOE_DEVICE void finish_router_stats(const float* blk_mp, const float* blk_z, con
     int cc = nthreads / ncol;
     if (cc < 1) cc = 1;
     // chunk sums over a fixed range of blocks each: the loads of 16 blocks are
-    // issued together, then added in block order
+    // issued together (unconditionally, at clamped indices, so that none waits
+    // for another), then the ones in range are added in block order
     for (int j = tid; j < ncol * cc; j += nthreads) {
         const int col = j % ncol, ch = j / ncol;
         const int b0 = (int)((int64_t)nb * ch / cc), b1 = (int)((int64_t)nb * (ch + 1) / cc);
         const float* src = col < E ? blk_mp + col : (col == E ? blk_z : blk_ent);
         const size_t stride = col < E ? (size_t)E : 1;
-        const int32_t* csrc = col < E ? blk_cnt + col : nullptr;
+        const int32_t* csrc = blk_cnt + (col < E ? col : 0);
+        const size_t cstride = (size_t)E;
         double a = 0.0;
         long long c = 0;
         for (int b = b0; b < b1; b += 16) {
@@ -49,15 +51,16 @@ MOE_DEVICE void finish_router_stats(const float* blk_mp, const float* blk_z, con
             int32_t n[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                const bool in = b + u < b1;
-                v[u] = in ? __ldcg(src + (size_t)(b + u) * stride) : 0.f;
-                n[u] = (in && csrc) ? __ldcg(csrc + (size_t)(b + u) * stride) : 0;
+                const int bb = min(b + u, b1 - 1);
+                v[u] = __ldcg(src + (size_t)bb * stride);
+                n[u] = __ldcg(csrc + (size_t)bb * cstride);
             }
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                a += (double)v[u];
-                c += n[u];
-            }
+            for (int u = 0; u < 16; ++u)
+                if (b + u < b1) {
+                    a += (double)v[u];
+                    c += col < E ? n[u] : 0;
+                }
         }
         sd[j] = a;
         sc[j] = c;

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     const int kb_begin = split * a.split_kb;                // never empty (host guarantee)
     const int kb_end = min(num_kb, kb_begin + a.split_kb);
     const int nkb = kb_end - kb_begin;
+    auto kb_at = [&](int i) { return kb_begin + i; };
     const int E = a.E;
 
     if (threadIdx.x == 0) {
@@ -221,10 +222,11 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             uint32_t phase = 0;
             int last_phase[MAX_STAGES];
             for (int s = 0; s < MAX_STAGES; ++s) last_phase[s] = -1;
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
+            for (int i = 0; i < nkb; ++i) {
                 if (!mbar_wait(&m->xempty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
                 mbar_arrive_expect_tx(&m->xfull[stage], A_BYTES);
-                tma_load_2d(xring + (size_t)stage * A_BYTES, &tmX, kb * BK, (int32_t)t0, &m->xfull[stage]);
+                tma_load_2d(xring + (size_t)stage * A_BYTES, &tmX, kb_at(i) * BK, (int32_t)t0,
+                            &m->xfull[stage]);
                 last_phase[stage] = (int)phase;
                 if (++stage == S) {
                     stage = 0;
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         {
             int issued = 0;  // fp32 slices issued (slot = index % WDEPTH)
             if (tid == 0)
-                for (; issued < WDEPTH && issued < nkb; ++issued) load_w(kb_begin + issued, issued);
+                for (; issued < WDEPTH && issued < nkb; ++issued) load_w(kb_at(issued), issued);
             const int pairs = E * 8;  // (expert, 8-wide chunk of d_model)
             int i = 0;
             for (; i < nkb; ++i) {
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 if (!mbar_wait(&m->bempty[j], ph ^ 1u, a.status, 541, abort_flag)) break;
                 uint8_t* sB = bring + (size_t)j * G::B_BYTES;
                 const float* wsm = reinterpret_cast<const float*>(wring + (size_t)j * a.w_slot);
-                const int d0 = (kb_begin + i) * BK;
+                const int d0 = kb_at(i) * BK;
                 for (int q = tid; q < pairs; q += 128) {
                     const int e = q % E, c = q / E;
                     const bool in = d0 + c * 8 < a.D;  // D % 8 == 0: a chunk is all in or all out
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 // refill fp32 slot j once every weight warp is done with it
                 if (tid == 0 && issued < nkb) {
                     if (!mbar_wait(&m->wfree[j], ph, a.status, 543, abort_flag)) break;
-                    load_w(kb_begin + issued, issued % WDEPTH);
+                    load_w(kb_at(issued), issued % WDEPTH);
                     ++issued;
                 }
             }
@@ -377,6 +379,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         // pass 1: logits (own K range + the other splits in order, + bias + noise),
         // their maximum, and (without a group limit) the top-K
         float mx = -INFINITY;
+#pragma unroll 4
         for (int e = 0; e < E; ++e) {
             float L = Ls[r * LDS + e];
             for (int sp = 1; sp < a.splits; ++sp) L += recv[((size_t)(sp - 1) * BM + r) * EPN + e];
@@ -390,14 +393,15 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         // pass 2: softmax sum, sum of exp(L - max) (L - max) for the entropy, and
         // the scores (sigmoid scores and their sum with score_func sigmoid)
         float ssum = 0.f, s1 = 0.f, scsum = 0.f;
+#pragma unroll 4
         for (int e = 0; e < E; ++e) {
             const float L = Ls[r * LDS + e];
-            const float x = expf(L - mx);
+            const float x = __expf(L - mx);
             ssum += x;
             s1 = fmaf(x, L - mx, s1);
             float sc = x;
             if (o.score_func == 1) {
-                sc = 1.0f / (1.0f + expf(-L));
+                sc = 1.0f / (1.0f + __expf(-L));
                 scsum += sc;
             }
             Xs[r * LDS + e] = sc;
@@ -452,6 +456,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         }
         // pass 3: normalised scores into Ls (and probs_out); rows past T give nothing
         const float scinv = o.score_func == 1 ? 1.0f / scsum : inv;
+#pragma unroll 4
         for (int e = 0; e < E; ++e) {
             const float pn = Xs[r * LDS + e] * scinv;
             Ls[r * LDS + e] = valid ? pn : 0.f;
