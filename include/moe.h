@@ -555,7 +555,8 @@ MOE_API moe_status moe_selftest_wait_timeout(void *workspace, size_t workspace_b
  * Number of kernels one moe_forward call launches for this configuration:
  * router 1 (bf16 with E <= 128 and T >= 2048: the tensor-core router, which
  * also routes and finishes the statistics) or 2 (the SIMT logits GEMM and the
- * top-k kernel, plus a split-sum when that GEMM is split over d_model; also
+ * top-k kernel, plus a split-sum when that GEMM is split over d_model in more
+ * than 4 parts; also
  * the path of a router weight that is not 16-byte aligned), dispatch 1 (3 when the
  * chunks of 2048 assignments outnumber the resident blocks), gather 1,
  * expert GEMMs 2, shared expert 3 (when F_shared > 0: its row offsets and two

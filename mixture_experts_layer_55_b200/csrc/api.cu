@@ -676,7 +676,7 @@ int32_t moe_forward_kernel_count(const moe_config* cfg)
     // or logits (tensor-core, or SIMT + its split sum) and the top-k kernel
     const int rest = 5 + (dispatch_index_fused(*cfg) ? 0 : 2) + shared;
     if (router_tc_eligible(*cfg)) return 1 + rest;
-    return 2 + (router_plan(*cfg).splits > 1 ? 1 : 0) + rest;
+    return 2 + (router_plan(*cfg).splits > kTopkMaxSplits ? 1 : 0) + rest;
 }
 
 moe_status moe_ep_workspace_size(int32_t world, int32_t experts_per_rank, size_t* bytes)

@@ -7,9 +7,8 @@
 //   gate/up: h = silu(x_perm Wg_e) * (x_perm Wu_e)         (rows x F)
 //            (the training forward also keeps [g | u], rows x 2F)
 //   down:    y_perm = topk_w[perm[row]] * (h Wd_e)         (rows x D)
-// Tiles are 32 rows x 64 columns for gate/up (32 h columns, their gate and up
-// columns side by side) and 32 x 32 for down (twice the blocks of a narrow
-// d_model), K steps of 32, on the double-buffered main loop of simt_gemm.cuh;
+// Tiles are 32 rows x 64 columns (gate/up: 32 h columns, their gate and up
+// columns side by side), on the double-buffered main loop of simt_gemm.cuh;
 // the m-tile -> (expert, first row) map is derived on the device from the
 // offsets (no host synchronisation).
 #include "common.cuh"
@@ -18,14 +17,13 @@
 
 namespace moe {
 
-constexpr int kBM = 32, kBK = 32;
-constexpr int kBNGateUp = 64, kBNDown = 32;
+constexpr int kBM = 32, kBN = 64, kBK = 16;
 
 // One BM-row tile of an expert's rows: gate/up (GATEUP: the tile's B columns
 // are kBN/2 gate columns then the same kBN/2 up columns, so each thread holds
 // g and u of the same h column) or down (kBN output columns, scaled by the
 // row's routing weight).  grid (ceil(N / columns per tile), m-tile bound).
-template <bool GATEUP, int kBN>
+template <bool GATEUP>
 __global__ void __launch_bounds__(simt::kThreads) ffn_simt_kernel(
     const float* __restrict__ A, const float* __restrict__ B0, const float* __restrict__ B1,
     float* __restrict__ out, const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
@@ -107,16 +105,16 @@ static cudaError_t launch_simt(const moe_config& c, int64_t max_rows, const void
 {
     const int64_t mtiles = simt::mtiles_bound(max_rows, c.E, kBM);
     const int64_t nk = c.T * c.K;
-    dim3 g1((c.F + kBNGateUp / 2 - 1) / (kBNGateUp / 2), (unsigned)mtiles);
-    ffn_simt_kernel<true, kBNGateUp><<<g1, simt::kThreads, 0, s>>>(
+    dim3 g1((c.F + kBN / 2 - 1) / (kBN / 2), (unsigned)mtiles);
+    ffn_simt_kernel<true><<<g1, simt::kThreads, 0, s>>>(
         static_cast<const float*>(x_perm), static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
         static_cast<float*>(h), offsets, perm, topk_w, c.E, c.D, c.F, max_rows, nk,
         static_cast<float*>(gu_keep), status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (mid) mid(mid_ctx, s);
-    dim3 g2((c.D + kBNDown - 1) / kBNDown, (unsigned)mtiles);
-    ffn_simt_kernel<false, kBNDown><<<g2, simt::kThreads, 0, s>>>(
+    dim3 g2((c.D + kBN - 1) / kBN, (unsigned)mtiles);
+    ffn_simt_kernel<false><<<g2, simt::kThreads, 0, s>>>(
         static_cast<const float*>(h), static_cast<const float*>(w_down), nullptr, static_cast<float*>(y_perm),
         offsets, perm, topk_w, c.E, c.F, c.D, max_rows, nk, nullptr, status);
     return cudaGetLastError();

@@ -47,6 +47,8 @@ struct RouterPlan {
     int nb_topk;     // blocks of the softmax/top-k kernel (64 tokens each)
 };
 RouterPlan router_plan(const moe_config& c);
+// up to this many d_model splits the top-k kernel adds the partial logits itself
+constexpr int kTopkMaxSplits = 4;
 
 // Router options beyond the plain softmax / renormalised top-k.
 struct RouteOpts {

@@ -9,7 +9,8 @@
 // Kernels:
 //   router_logits_kernel  tiled SIMT fp32 GEMM (T x D) * (D x E), optionally
 //                         split over d_model; partial sums go to scratch.
-//   router_splitsum_kernel sums the d-split partials in split order.
+//   router_splitsum_kernel sums the d-split partials in split order (more than
+//                         kTopkMaxSplits splits; fewer, the top-k kernel adds them).
 //   router_topk_kernel    one warp per token: adds bias and noise, softmax, top-k by
 //                         (logit desc, id asc) with warp shuffles, weights,
 //                         and per-block statistic partials, which the block
@@ -40,7 +41,12 @@ RouterPlan router_plan(const moe_config& c)
     p.grid_e = (c.E + p.be - 1) / p.be;
     int64_t base = (int64_t)p.grid_t * p.grid_e;
     int want = (int)((6 * 148 + base - 1) / base);  // enough blocks to hide load latency
-    int max_splits = c.D / 256 > 1 ? c.D / 256 : 1;
+    // at least 256 of d_model per split, or down to 64 for up to 4 splits (a short
+    // d_model with few tokens)
+    int max_splits = c.D / 256;
+    const int short_splits = c.D / 64 < 4 ? c.D / 64 : 4;
+    if (max_splits < short_splits) max_splits = short_splits;
+    if (max_splits < 1) max_splits = 1;
     if (want > max_splits) want = max_splits;
     if (want < 1) want = 1;
     int dps = (c.D + want - 1) / want;
@@ -526,6 +532,7 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
     int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + L.r_cnt);
     int* status = reinterpret_cast<int*>(ws + L.status);
     const float* part;
+    int splits = 1;
     // bf16 layers with enough tokens: the tensor-core router (its bulk copies of W_r
     // need a 16-byte aligned W_r; an unaligned one takes the SIMT router)
     if (!logits_in && router_tc_eligible(c) && (reinterpret_cast<uintptr_t>(w_router) & 15u) == 0)
@@ -541,16 +548,18 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
             launch_logits(c, rp, static_cast<const __nv_bfloat16*>(x), w_router, p, s);
         else
             launch_logits(c, rp, static_cast<const float*>(x), w_router, p, s);
-        if (rp.splits > 1) {
+        if (rp.splits > kTopkMaxSplits) {
             const int64_t n = c.T * c.E;
             int64_t blocks = (n + 255) / 256;
             if (blocks > 148 * 16) blocks = 148 * 16;
             router_splitsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rp.splits, n);
+        } else {
+            splits = rp.splits;  // few splits: the top-k kernel adds them in order
         }
         part = p;
     }
-    return launch_topk(c, o, part, 1, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z, blk_ent,
-                       blk_cnt, with_stats, mean_prob, losses, status + kRouterCounterWord, rp, s);
+    return launch_topk(c, o, part, splits, bias, noise, logits_out, probs_out, ids, w, blk_mp, blk_z,
+                       blk_ent, blk_cnt, with_stats, mean_prob, losses, status + kRouterCounterWord, rp, s);
 }
 
 }  // namespace moe
