@@ -1112,9 +1112,10 @@ def run_reference(args):
         "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": len(vals), "warmup": args.warmup,
         "ms_per_step": round(ms_step, 3), "extrapolated": True,
-        "extrapolation": ("ms_per_step = T / value, the per-token cost of each step's bounded "
-                          "sample times T; no step ran the whole layer (the steps together "
-                          f"took {time.perf_counter() - t0:.1f} s)"),
+        "extrapolation": ("ms_per_step = T / value: each step times the routing and dispatch "
+                          "of all T tokens and the expert FFN of a bounded token sample (every "
+                          "token only for small layers), and value is the per-token cost "
+                          f"extrapolated (the steps together took {time.perf_counter() - t0:.1f} s)"),
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "F": wl.F, "E": wl.E, "K": wl.K,

@@ -44,7 +44,8 @@ struct RouterPlan {
     int grid_e;      // expert blocks
     int splits;      // d_model splits of the logits GEMM
     int d_per_split; // multiple of 32
-    int nb_topk;     // blocks of the softmax/top-k kernel (64 tokens each)
+    int tpb_topk;    // tokens per block of the softmax/top-k kernel (8 or 16)
+    int nb_topk;     // its blocks
 };
 RouterPlan router_plan(const moe_config& c);
 // up to this many d_model splits the top-k kernel adds the partial logits itself

@@ -26,7 +26,9 @@
 namespace moe {
 
 constexpr int kLogitsBD = 32;  // d_model per shared-memory step
-constexpr int kTopkTPB = 16;   // tokens per top-k block (8 warps x 2)
+// tokens per top-k block: 8 warps x 2, or x 1 when the tokens are too few to
+// give every SM several blocks of two (decode-sized batches)
+inline int topk_tokens_per_block(int64_t T) { return T <= 148 * 16 * 2 ? 8 : 16; }
 
 // Tokens per logits block for an expert tile of be columns (see the kernel's
 // thread layout): 128 for be = 8, else 64.
@@ -53,7 +55,8 @@ RouterPlan router_plan(const moe_config& c)
     dps = (dps + kLogitsBD - 1) / kLogitsBD * kLogitsBD;
     p.d_per_split = dps;
     p.splits = (c.D + dps - 1) / dps;
-    p.nb_topk = (int)((c.T + kTopkTPB - 1) / kTopkTPB);
+    p.tpb_topk = topk_tokens_per_block(c.T);
+    p.nb_topk = (int)((c.T + p.tpb_topk - 1) / p.tpb_topk);
     return p;
 }
 
@@ -219,7 +222,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     float* __restrict__ probs_out, int32_t* __restrict__ ids, float* __restrict__ wout,
     float* __restrict__ blk_mp, float* __restrict__ blk_z, float* __restrict__ blk_ent,
     int32_t* __restrict__ blk_cnt, int64_t T, int E, int K, int with_stats,
-    float* __restrict__ mean_prob, float* __restrict__ losses, int* __restrict__ counter)
+    float* __restrict__ mean_prob, float* __restrict__ losses, int* __restrict__ counter, int tpb)
 {
     __shared__ float s_mp[8][256];
     __shared__ int s_cnt[8][256];
@@ -237,8 +240,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     float z_acc = 0.f, ent_acc = 0.f;
     const int G = o.n_groups, gsz = E / G;
 
-    const int64_t tbase = (int64_t)blockIdx.x * kTopkTPB;
-    for (int i = 0; i < kTopkTPB / 8; ++i) {  // tokens warp, warp + 8, ...
+    const int64_t tbase = (int64_t)blockIdx.x * tpb;
+    for (int i = 0; i < tpb / 8; ++i) {  // tokens warp, warp + 8, ...
         const int64_t t = tbase + warp + 8 * i;
         if (t >= T) break;
         float L[EPL];
@@ -506,7 +509,7 @@ static cudaError_t launch_topk(const moe_config& c, const RouteOpts& o, const fl
 #define MOE_TOPK(N)                                                                                     \
     router_topk_kernel<N><<<grid, 256, 0, s>>>(part, splits, bias, noise, o, logits_out, probs_out, ids, \
                                                w, blk_mp, blk_z, blk_ent, blk_cnt, c.T, c.E, c.K,       \
-                                               with_stats, mean_prob, losses, counter)
+                                               with_stats, mean_prob, losses, counter, rp.tpb_topk)
     switch (epl) {
         case 1: MOE_TOPK(1); break;
         case 2: MOE_TOPK(2); break;

@@ -146,6 +146,10 @@ SMALL = {
     "many_experts_top1": Workload("many_experts_top1", T=256, D=128, F=128, E=64, K=1),
     "single_expert": Workload("single_expert", T=100, D=128, F=192, E=1, K=1),
     "one_token": Workload("one_token", T=1, D=128, F=128, E=8, K=2),
+    # few tokens and a long d_model: the combine splits each row over several warps
+    # (weighted slots here, the training forward's combine), with a shared expert
+    "split_combine_shared": Workload("split_combine_shared", T=64, D=2048, F=64, E=8, K=3,
+                                     F_shared=64),
     # fp32 layers (SIMT GEMMs): the fp32 reference layer's shape, and drops with a shared expert
     "f32_layer": Workload("f32_layer", T=512, D=256, F=512, E=8, K=2, dtype="f32"),
     "f32_drops_shared": Workload("f32_drops_shared", T=300, D=128, F=192, E=8, K=2, dtype="f32",

@@ -78,6 +78,10 @@ SMALL = [
     _wl("shared_bf16_pair", T=700, D=136, F=200, E=4, K=2, F_shared=264, seed=29),
     _wl("shared_f32", T=300, D=64, F=96, E=8, K=2, F_shared=72, dtype="f32", seed=30),
     _wl("shared_drops", T=400, D=64, F=96, E=8, K=2, capacity_factor=0.5, F_shared=128, seed=31),
+    # few tokens, long d_model: the combine splits each row over several warps; a shared
+    # expert's rows are added first and a capacity drop leaves a slot out
+    _wl("split_combine", T=96, D=2048, F=64, E=8, K=3, F_shared=64, capacity_factor=0.6, seed=48),
+    _wl("split_combine_f32", T=40, D=1024, F=32, E=4, K=2, dtype="f32", seed=49),
 ]
 
 
