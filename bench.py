@@ -438,7 +438,7 @@ def measure_forward(M, wl: Workload, args, rank: int, world: int, dev, *, headli
                          ("inputs fit in L2: a 252 MB buffer is written before every step and "
                           "the steps are timed one by one")},
         "dtype": wl.dtype,
-        "gpu_launches": M.forward_kernel_count(layer.cfg) * steps,
+        "gpu_launches": M.forward_kernel_count(layer.cfg, layer.router_terms is not None) * steps,
         "roofline": forward_roofline(wl, alg, stage_ms, ms_total),
         "stages": stage_table(wl, alg, stage_ms),
         "layer": {"assignments_per_s": round(world * wl.T * wl.K / (ms_step / 1e3), 1),

@@ -138,6 +138,28 @@ MOE_API moe_status moe_workspace_size(const moe_config *cfg, size_t *bytes);
 MOE_API moe_status moe_forward_workspace_size(const moe_config *cfg, size_t *bytes);
 
 /*
+ * The router weight prepared for the tensor-core router of bf16 layers
+ * ("Lab: build a tiny MoE in PyTorch", "Full implementation": the router
+ * logits are fp32).  Each fp32 weight W_r[d, e] is split exactly into three
+ * bf16 terms, hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)
+ * (round to nearest even), so that x * hi + x * mid + x * lo, accumulated in
+ * fp32 on the tensor cores, is the fp32 product.  Layout: bf16
+ * terms[p][e][d] for p = 0 (hi), 1 (mid), 2 (lo), e < E16 and d < D, where
+ * E16 is E rounded up to 16, 32, 64 or 128; the rows e >= E are zero.
+ *
+ * moe_router_terms_size: 3 * E16 * D * 2 bytes for bf16 layers with E <= 128
+ * (the layers whose router can run on the tensor cores), 0 for the others.
+ * moe_router_prepare writes the terms of w_router (D, E) fp32 into
+ * w_router_terms (16-byte aligned, moe_router_terms_size bytes) on the
+ * stream; MOE_ERR_UNSUPPORTED where the size is 0.  The terms depend on the
+ * weight only: prepare them once per weight value (again after every update
+ * of W_r) and pass them to moe_route / moe_forward, which then skip the split.
+ */
+MOE_API moe_status moe_router_terms_size(const moe_config *cfg, size_t *bytes);
+MOE_API moe_status moe_router_prepare(const moe_config *cfg, const float *w_router,
+                                      void *w_router_terms, void *stream);
+
+/*
  * Router: "Lab: build a tiny MoE in PyTorch", section "Full implementation"
  * (fp32 router logits, softmax, top-k, renormalised weights, balance loss and
  * router z-loss) and "2.9 Mixture-of-Experts (MoE) Architectures", section
@@ -163,7 +185,11 @@ MOE_API moe_status moe_forward_workspace_size(const moe_config *cfg, size_t *byt
  *   losses[2] = router entropy = (1/T) sum_t -sum_e q log max(q, 1e-9),
  *               q = softmax(L[t,:])  ("Full implementation", stats)
  *
- * x (T, D) dtype; w_router (D, E) fp32.  router_bias (E), selection_bias (E)
+ * x (T, D) dtype; w_router (D, E) fp32.  w_router_terms may be NULL or the
+ * terms moe_router_prepare wrote for this w_router (same D and E): the
+ * tensor-core router (bf16 layers, E <= 128, T >= 2048) then reads them
+ * instead of splitting w_router itself, one kernel fewer; the other routers
+ * ignore them.  router_bias (E), selection_bias (E)
  * and logit_noise (T, E) may be NULL.  logits_in (T, E), if not NULL, are
  * taken as the complete routing logits L: x, w_router, router_bias and noise
  * are then not read and may be NULL (selection_bias still applies).
@@ -176,7 +202,7 @@ MOE_API moe_status moe_forward_workspace_size(const moe_config *cfg, size_t *byt
  * is left at zero).
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router,
-                     const float *router_bias, const float *selection_bias,
+                     const void *w_router_terms, const float *router_bias, const float *selection_bias,
                      const float *logit_noise, const float *logits_in,
                      float *logits_out, float *probs_out, int32_t *topk_ids, float *topk_w,
                      float *mean_prob, float *losses, void *workspace, size_t workspace_bytes,
@@ -259,7 +285,8 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
  * "2.9 Mixture-of-Experts (MoE) Architectures", "A Toy MoE Layer From
  * Scratch"): moe_route -> moe_dispatch -> moe_expert_ffn -> (shared expert)
  * -> moe_combine on one stream, every intermediate in the workspace
- * (moe_forward_workspace_size bytes).  With cfg->F_shared > 0,
+ * (moe_forward_workspace_size bytes).  w_router_terms as for moe_route
+ * (NULL: the router splits w_router itself).  With cfg->F_shared > 0,
  * w_gate_shared / w_up_shared (D, F_shared) and w_down_shared (F_shared, D)
  * are required and the shared SwiGLU expert's output over all tokens is
  * added in the combine; otherwise they are ignored (may be NULL).  y (T, D)
@@ -268,7 +295,7 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
  * are optional copies of the routing results (NULL to skip).
  */
 MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *w_router,
-                       const float *router_bias, const float *selection_bias,
+                       const void *w_router_terms, const float *router_bias, const float *selection_bias,
                        const float *logit_noise, const void *w_gate,
                        const void *w_up, const void *w_down, const void *w_gate_shared,
                        const void *w_up_shared, const void *w_down_shared, void *y, float *losses,
@@ -554,15 +581,15 @@ MOE_API moe_status moe_selftest_wait_timeout(void *workspace, size_t workspace_b
 /*
  * Number of kernels one moe_forward call launches for this configuration:
  * router 1 (bf16 with E <= 128 and T >= 2048: the tensor-core router, which
- * also routes and finishes the statistics) or 2 (the SIMT logits GEMM and the
- * top-k kernel, plus a split-sum when that GEMM is split over d_model in more
- * than 4 parts; also
- * the path of a router weight that is not 16-byte aligned), dispatch 1 (3 when the
- * chunks of 2048 assignments outnumber the resident blocks), gather 1,
- * expert GEMMs 2, shared expert 3 (when F_shared > 0: its row offsets and two
- * GEMMs), combine 1.  0 for an invalid configuration.
+ * also routes and finishes the statistics; 2 when router_terms_given is 0,
+ * the first splitting w_router into the workspace) or 2 (the SIMT logits GEMM
+ * and the top-k kernel, plus a split-sum when that GEMM is split over d_model
+ * in more than 4 parts), dispatch 1 (3 when the chunks of 2048 assignments
+ * outnumber the resident blocks), gather 1, expert GEMMs 2, shared expert 3
+ * (when F_shared > 0: its row offsets and two GEMMs), combine 1.  0 for an
+ * invalid configuration.
  */
-MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg);
+MOE_API int32_t moe_forward_kernel_count(const moe_config *cfg, int32_t router_terms_given);
 
 /*
  * Kernel-boundary tracing for timing.  After moe_trace_attach(events, n),

@@ -75,16 +75,18 @@ _SIG = {
     "moe_max_rows": ([_P, _P], ctypes.c_int32),
     "moe_workspace_size": ([_P, _P], ctypes.c_int32),
     "moe_forward_workspace_size": ([_P, _P], ctypes.c_int32),
-    "moe_route": ([_P] * 14 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_router_terms_size": ([_P, _P], ctypes.c_int32),
+    "moe_router_prepare": ([_P] * 4, ctypes.c_int32),
+    "moe_route": ([_P] * 15 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch_noalloc": ([_P] * 10, ctypes.c_int32),
     "moe_expert_ffn": ([_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([_P] * 6, ctypes.c_int32),
-    "moe_forward": ([_P] * 19 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_forward": ([_P] * 20 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_update_selection_bias": ([_P, _P, ctypes.c_float, _P, _P], ctypes.c_int32),
     "moe_get_device_status": ([_P, _P, _P], ctypes.c_int32),
     "moe_clear_device_status": ([_P, _P], ctypes.c_int32),
-    "moe_forward_kernel_count": ([_P], ctypes.c_int32),
+    "moe_forward_kernel_count": ([_P, ctypes.c_int32], ctypes.c_int32),
     "moe_selftest_wait_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
     "moe_trace_attach": ([_P, ctypes.c_int32], ctypes.c_int32),
     "moe_trace_boundary_count": ([], ctypes.c_int32),
@@ -206,10 +208,24 @@ def forward_workspace_size(cfg: MoeConfig) -> int:
     return v.value
 
 
+def router_terms_size(cfg: MoeConfig) -> int:
+    """Bytes of the prepared router weight (0: this layer's router takes none)."""
+    v = ctypes.c_size_t()
+    _check(lib().moe_router_terms_size(_cfg(cfg), ctypes.byref(v)), "moe_router_terms_size")
+    return int(v.value)
+
+
+def moe_router_prepare(cfg, w_router, w_router_terms, stream=None):
+    """Split w_router into the three bf16 terms the tensor-core router reads."""
+    _check(lib().moe_router_prepare(_cfg(cfg), _ptr(w_router), _ptr(w_router_terms),
+                                    _stream(stream)), "moe_router_prepare")
+
+
 def moe_route(cfg, x, w_router, topk_ids, topk_w, workspace, router_bias=None, logit_noise=None,
               logits_in=None, logits_out=None, probs_out=None, mean_prob=None, losses=None,
-              selection_bias=None, stream=None):
-    st = lib().moe_route(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
+              selection_bias=None, w_router_terms=None, stream=None):
+    st = lib().moe_route(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(w_router_terms),
+                         _ptr(router_bias),
                          _ptr(selection_bias), _ptr(logit_noise), _ptr(logits_in),
                          _ptr(logits_out), _ptr(probs_out),
                          _ptr(topk_ids), _ptr(topk_w), _ptr(mean_prob), _ptr(losses),
@@ -251,10 +267,11 @@ def moe_combine(cfg, y_perm, row_of, y, y_add=None, stream=None):
 
 def moe_forward(cfg, x, w_router, w_gate, w_up, w_down, y, workspace, router_bias=None,
                 logit_noise=None, losses=None, mean_prob=None, counts=None, topk_ids=None,
-                topk_w=None, selection_bias=None, shared=None, stream=None):
+                topk_w=None, selection_bias=None, shared=None, w_router_terms=None, stream=None):
     """shared = (w_gate_s, w_up_s, w_down_s) when cfg.F_shared > 0."""
     sg, su, sd = shared if shared is not None else (None, None, None)
-    st = lib().moe_forward(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
+    st = lib().moe_forward(_cfg(cfg), _ptr(x), _ptr(w_router), _ptr(w_router_terms),
+                           _ptr(router_bias),
                            _ptr(selection_bias), _ptr(logit_noise), _ptr(w_gate), _ptr(w_up),
                            _ptr(w_down), _ptr(sg), _ptr(su), _ptr(sd), _ptr(y),
                            _ptr(losses), _ptr(mean_prob), _ptr(counts), _ptr(topk_ids),
@@ -335,9 +352,9 @@ def moe_selftest_wait_timeout(workspace, limit_ns: int, stream=None):
                                            _stream(stream)), "moe_selftest_wait_timeout")
 
 
-def forward_kernel_count(cfg: MoeConfig) -> int:
+def forward_kernel_count(cfg: MoeConfig, router_terms_given: bool = False) -> int:
     """Kernels one moe_forward launches for this configuration."""
-    return int(lib().moe_forward_kernel_count(_cfg(cfg)))
+    return int(lib().moe_forward_kernel_count(_cfg(cfg), int(bool(router_terms_given))))
 
 
 def moe_trace_attach(events):

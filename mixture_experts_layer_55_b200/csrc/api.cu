@@ -46,10 +46,11 @@ WsLayout ws_layout(const moe_config& c)
     L.status = o;
     o += align_up(64 * sizeof(int));
     L.r_part = o;
-    // the SIMT router's (partial) logits per d_model split (also the fallback of the
-    // tensor-core router for an unaligned W_r)
+    // the SIMT router's (partial) logits per d_model split
     const size_t part_bytes = (size_t)rp.splits * (size_t)c.T * c.E * sizeof(float);
     o += align_up(part_bytes);
+    L.r_terms = o;
+    o += align_up(router_tc_eligible(c) ? router_terms_bytes(c) : 0);
     L.r_mp = o;
     o += align_up((size_t)rp.nb_topk * c.E * sizeof(float));
     L.r_z = o;
@@ -315,8 +316,8 @@ static moe_status check_ws(const moe_config* cfg, const void* ws, size_t bytes, 
 }
 
 moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router,
-                     const float* router_bias, const float* selection_bias,
-                     const float* logit_noise, const float* logits_in,
+                     const void* w_router_terms, const float* router_bias,
+                     const float* selection_bias, const float* logit_noise, const float* logits_in,
                      float* logits_out, float* probs_out, int32_t* topk_ids, float* topk_w,
                      float* mean_prob, float* losses, void* workspace, size_t workspace_bytes,
                      void* stream)
@@ -326,15 +327,37 @@ moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router
     if (topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_ARG;
     if (logits_in == nullptr && (x == nullptr || w_router == nullptr)) return MOE_ERR_ARG;
     if (logits_in == nullptr && !aligned16(x)) return MOE_ERR_ALIGN;
+    if (w_router_terms != nullptr && !aligned16(w_router_terms)) return MOE_ERR_ALIGN;
     const WsLayout L = ws_layout(*cfg);
     st = check_ws(cfg, workspace, workspace_bytes, L.total);
     if (st != MOE_OK) return st;
     const RouterPlan rp = router_plan(*cfg);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return cuda_status(launch_router(*cfg, rp, x, w_router, router_bias, selection_bias,
-                                     logit_noise, logits_in,
+    return cuda_status(launch_router(*cfg, rp, x, w_router, w_router_terms, router_bias,
+                                     selection_bias, logit_noise, logits_in,
                                      logits_out, probs_out, topk_ids, topk_w, mean_prob, losses,
                                      static_cast<char*>(workspace), L, s));
+}
+
+moe_status moe_router_terms_size(const moe_config* cfg, size_t* bytes)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_ARG;
+    *bytes = router_terms_bytes(*cfg);
+    return MOE_OK;
+}
+
+moe_status moe_router_prepare(const moe_config* cfg, const float* w_router, void* w_router_terms,
+                              void* stream)
+{
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (router_terms_bytes(*cfg) == 0) return MOE_ERR_UNSUPPORTED;
+    if (w_router == nullptr || w_router_terms == nullptr) return MOE_ERR_ARG;
+    if (!aligned16(w_router_terms)) return MOE_ERR_ALIGN;
+    return cuda_status(
+        launch_router_prepare(*cfg, w_router, w_router_terms, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* topk_ids,
@@ -398,8 +421,9 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
 // applies the weights, and the routing results stay in the state (copied to
 // the caller's buffers when asked for).
 static cudaError_t run_forward(const moe_config& c, const void* x, const float* w_router,
-                               const float* router_bias, const float* selection_bias,
-                               const float* logit_noise, const void* w_gate, const void* w_up,
+                               const void* w_terms, const float* router_bias,
+                               const float* selection_bias, const float* logit_noise,
+                               const void* w_gate, const void* w_up,
                                const void* w_down, const void* w_gate_shared,
                                const void* w_up_shared, const void* w_down_shared, void* y,
                                float* losses, float* mean_prob, int32_t* counts, int32_t* topk_ids,
@@ -423,8 +447,8 @@ static cudaError_t run_forward(const moe_config& c, const void* x, const float* 
 
     trace(0, s);
     const RouterPlan rp = router_plan(c);
-    cudaError_t e = launch_router(c, rp, x, w_router, router_bias, selection_bias, logit_noise,
-                                  nullptr, logits_keep, nullptr, ids, w, mean_prob, losses, ws,
+    cudaError_t e = launch_router(c, rp, x, w_router, w_terms, router_bias, selection_bias,
+                                  logit_noise, nullptr, logits_keep, nullptr, ids, w, mean_prob, losses, ws,
                                   F.ws, s);
     trace(1, s);
     if (e == cudaSuccess)
@@ -485,8 +509,8 @@ static moe_status check_forward_args(const moe_config* cfg, const void* x, const
 }
 
 moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
-                       const float* router_bias, const float* selection_bias,
-                       const float* logit_noise, const void* w_gate,
+                       const void* w_router_terms, const float* router_bias,
+                       const float* selection_bias, const float* logit_noise, const void* w_gate,
                        const void* w_up, const void* w_down, const void* w_gate_shared,
                        const void* w_up_shared, const void* w_down_shared, void* y, float* losses,
                        float* mean_prob, int32_t* counts, int32_t* topk_ids, float* topk_w,
@@ -495,12 +519,13 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
     moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
                                        w_up_shared, w_down_shared, y);
     if (st != MOE_OK) return st;
+    if (w_router_terms != nullptr && !aligned16(w_router_terms)) return MOE_ERR_ALIGN;
     const FwdLayout F = fwd_layout(*cfg, max_rows_of(*cfg));
     st = check_ws(cfg, workspace, workspace_bytes, F.total);
     if (st != MOE_OK) return st;
-    return cuda_status(run_forward(*cfg, x, w_router, router_bias, selection_bias, logit_noise,
-                                   w_gate, w_up, w_down, w_gate_shared, w_up_shared, w_down_shared,
-                                   y, losses, mean_prob, counts, topk_ids, topk_w,
+    return cuda_status(run_forward(*cfg, x, w_router, w_router_terms, router_bias, selection_bias,
+                                   logit_noise, w_gate, w_up, w_down, w_gate_shared, w_up_shared,
+                                   w_down_shared, y, losses, mean_prob, counts, topk_ids, topk_w,
                                    static_cast<char*>(workspace), F, nullptr,
                                    static_cast<cudaStream_t>(stream)));
 }
@@ -510,7 +535,7 @@ moe_status moe_train_state_size(const moe_config* cfg, size_t* bytes)
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (bytes == nullptr) return MOE_ERR_ARG;
-        *bytes = train_layout(*cfg, max_rows_of(*cfg)).total;
+    *bytes = train_layout(*cfg, max_rows_of(*cfg)).total;
     return MOE_OK;
 }
 
@@ -525,12 +550,13 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const float* 
     moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
                                        w_up_shared, w_down_shared, y);
     if (st != MOE_OK) return st;
-        const TrainLayout TL = train_layout(*cfg, max_rows_of(*cfg));
+    const TrainLayout TL = train_layout(*cfg, max_rows_of(*cfg));
     st = check_ws(cfg, state, state_bytes, TL.total);
     if (st != MOE_OK) return st;
-    return cuda_status(run_forward(*cfg, x, w_router, router_bias, selection_bias, logit_noise,
-                                   w_gate, w_up, w_down, w_gate_shared, w_up_shared, w_down_shared,
-                                   y, losses, mean_prob, counts, topk_ids, topk_w,
+    // the training forward splits the router weight itself (it changes every step)
+    return cuda_status(run_forward(*cfg, x, w_router, nullptr, router_bias, selection_bias,
+                                   logit_noise, w_gate, w_up, w_down, w_gate_shared, w_up_shared,
+                                   w_down_shared, y, losses, mean_prob, counts, topk_ids, topk_w,
                                    static_cast<char*>(state), TL.f, &TL,
                                    static_cast<cudaStream_t>(stream)));
 }
@@ -667,15 +693,16 @@ moe_status moe_clear_device_status(void* workspace, void* stream)
         cudaMemsetAsync(workspace, 0, 64 * sizeof(int), static_cast<cudaStream_t>(stream)));
 }
 
-int32_t moe_forward_kernel_count(const moe_config* cfg)
+int32_t moe_forward_kernel_count(const moe_config* cfg, int32_t router_terms_given)
 {
     if (check_config(cfg) != MOE_OK) return 0;
     const int shared = cfg->F_shared > 0 ? 3 : 0;  // row offsets + two GEMMs
     // dispatch 1 (one cooperative kernel; 3 for more chunks than resident blocks),
-    // gather 1, expert GEMMs 2, combine 1; router: the tensor-core kernel alone,
-    // or logits (tensor-core, or SIMT + its split sum) and the top-k kernel
+    // gather 1, expert GEMMs 2, combine 1; router: the tensor-core kernel (after
+    // the weight split when the caller passes no prepared terms), or the SIMT
+    // logits (+ their split sum) and the top-k kernel
     const int rest = 5 + (dispatch_index_fused(*cfg) ? 0 : 2) + shared;
-    if (router_tc_eligible(*cfg)) return 1 + rest;
+    if (router_tc_eligible(*cfg)) return (router_terms_given ? 1 : 2) + rest;
     return 2 + (router_plan(*cfg).splits > kTopkMaxSplits ? 1 : 0) + rest;
 }
 

@@ -87,6 +87,7 @@ inline bool dispatch_index_fused(const moe_config& c) { return dispatch_chunks(c
 struct WsLayout {
     size_t status;      // int32[64]
     size_t r_part;      // splits * T * E fp32 partial logits of the SIMT router
+    size_t r_terms;     // the tensor-core router's weight terms when the caller has none
     size_t r_mp;        // nb_topk * E fp32
     size_t r_z;         // nb_topk fp32
     size_t r_ent;       // nb_topk fp32 (entropy partials)
@@ -139,21 +140,29 @@ int64_t max_rows_of(const moe_config& c);
 
 // Tensor-core router (router_tc.cu): bf16 layers with E <= 128 and T >= 2048.
 // One kernel: logits, routing, and (when mean_prob or losses is given) the
-// statistics, finished by the CTA that completes last.
+// statistics, finished by the CTA that completes last.  It reads the router
+// weight as its three exact bf16 terms (router_prepare_kernel).
 bool router_tc_eligible(const moe_config& c);
 int router_tc_blocks(const moe_config& c);
 // CTAs per token tile (a cluster splitting d_model; 1: no split)
 int router_tc_splits(const moe_config& c);
+// Bytes of the weight terms, 3 x E16 x D bf16 (0: no tensor-core router for c).
+size_t router_terms_bytes(const moe_config& c);
+cudaError_t launch_router_prepare(const moe_config& c, const float* w_router, void* terms,
+                                  cudaStream_t s);
 cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
-                             const float* w_router, const float* bias, const float* noise,
+                             const void* terms, const float* bias, const float* noise,
                              float* logits_out, float* probs_out, int32_t* ids, float* w,
                              float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
                              float* mean_prob, float* losses, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- launches --
 // Each returns cudaSuccess or the launch error.
+// terms: the prepared router weight or null (the tensor-core router then
+// prepares it in the workspace first).
 cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void* x,
-                          const float* w_router, const float* bias, const float* sel_bias,
+                          const float* w_router, const void* terms, const float* bias,
+                          const float* sel_bias,
                           const float* noise,
                           const float* logits_in, float* logits_out, float* probs_out,
                           int32_t* ids, float* w, float* mean_prob, float* losses, char* ws,

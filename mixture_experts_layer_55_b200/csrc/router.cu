@@ -522,8 +522,8 @@ static cudaError_t launch_topk(const moe_config& c, const RouteOpts& o, const fl
 }
 
 cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void* x,
-                          const float* w_router, const float* bias, const float* sel_bias,
-                          const float* noise, const float* logits_in, float* logits_out,
+                          const float* w_router, const void* terms, const float* bias,
+                          const float* sel_bias, const float* noise, const float* logits_in, float* logits_out,
                           float* probs_out, int32_t* ids, float* w, float* mean_prob,
                           float* losses, char* ws, const WsLayout& L, cudaStream_t s)
 {
@@ -536,11 +536,18 @@ cudaError_t launch_router(const moe_config& c, const RouterPlan& rp, const void*
     int* status = reinterpret_cast<int*>(ws + L.status);
     const float* part;
     int splits = 1;
-    // bf16 layers with enough tokens: the tensor-core router (its bulk copies of W_r
-    // need a 16-byte aligned W_r; an unaligned one takes the SIMT router)
-    if (!logits_in && router_tc_eligible(c) && (reinterpret_cast<uintptr_t>(w_router) & 15u) == 0)
-        return launch_router_tc(c, o, x, w_router, bias, noise, logits_out, probs_out, ids, w, blk_mp,
+    // bf16 layers with enough tokens: the tensor-core router, on the caller's
+    // prepared weight terms or on terms split here into the workspace
+    if (!logits_in && router_tc_eligible(c)) {
+        if (terms == nullptr) {
+            void* own = ws + L.r_terms;
+            const cudaError_t e = launch_router_prepare(c, w_router, own, s);
+            if (e != cudaSuccess) return e;
+            terms = own;
+        }
+        return launch_router_tc(c, o, x, terms, bias, noise, logits_out, probs_out, ids, w, blk_mp,
                                 blk_z, blk_ent, blk_cnt, mean_prob, losses, status, s);
+    }
     if (logits_in) {
         part = logits_in;
         bias = nullptr;

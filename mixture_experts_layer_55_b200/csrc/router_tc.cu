@@ -10,24 +10,26 @@
 // fp32 logits on bf16 tensor cores: x is bf16 already, and each fp32 router
 // weight is split exactly into three bf16 terms w = hi + mid + lo (hi =
 // bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid): 3 x 8 significand
-// bits cover fp32's 24).  Every product x*term is exact in fp32, and the
-// three MMAs of a K step accumulate in fp32 in tensor memory, so the logits
-// carry fp32 accumulation error only (no bf16 rounding of the weights).
+// bits cover fp32's 24).  Every product x*term is exact in fp32 and is
+// accumulated in fp32 in tensor memory, so the logits carry fp32
+// accumulation error only (no bf16 rounding of the weights).  The split is a
+// function of the weight alone: router_prepare_kernel writes the terms once
+// (terms[p][e][d], expert rows of d_model values, rows past E zero), and
+// this kernel reads them by TMA like x.
 //
-// One CTA per 128 tokens (M = 128) and per split of d_model; N = EPN, the
-// expert count rounded up to 16, 32, 64 or 128.  Warps:
+// One CTA per 128 tokens (M = 128) and per split of d_model.  The three
+// terms are stacked along N: one MMA per K step of 16 computes
+// [x.hi | x.mid | x.lo] for all experts at once (N = 3 x EPN, EPN = E rounded
+// up to 16, 32, 64 or 128; two MMAs when that exceeds 256), and the epilogue
+// adds the three partial logits.  Warps:
 //   warp 0      TMA: the x tiles (128 tokens x 64 of d_model, 128-byte
 //               swizzle) into a deep ring (up to 10 stages of 16 KB)
-//   warp 1      tcgen05.mma, three per K step of 16 (one per weight term)
-//   warps 2..5  first the weight split: the 64 x E fp32 slice of W_r of each
-//               K block arrives by bulk copy in a shallow ring of its own,
-//               is split in shared memory into its three bf16 terms and
-//               written K-major (expert rows of 64 d_model values, 128-byte
-//               swizzle) into a shallow ring of weight tiles, so no weight
-//               kernel runs before this one, the weight tiles are E rows
-//               wide, not a padded 64, and the x ring keeps its depth; then
-//               the epilogue, one token row per
-//               thread: logits (+ bias + noise), max and top-K by (logit +
+//   warp 1      tcgen05.mma
+//   warps 2..5  lane 0 of warp 2: TMA of the weight terms of each K block
+//               (3 x EPN rows x 64 of d_model, 128-byte swizzle) into a ring
+//               of their own, so that the x ring keeps its depth; then all
+//               four warps run the epilogue, one token row per thread:
+//               logits (+ bias + noise), max and top-K by (logit +
 //               selection bias desc, id asc, an unrolled insertion network)
 //               in one pass over the experts, softmax sum and entropy
 //               (closed form) and scores in a second, the group limit when
@@ -53,27 +55,26 @@ namespace rtc {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB x tile per stage
-constexpr int NUM_THREADS = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 weights + epilogue
+constexpr int NUM_THREADS = 192;      // warp 0 x TMA, warp 1 MMA, warps 2..5 weight TMA + epilogue
 constexpr int MAX_STAGES = 10;
+constexpr int MAX_WSLOTS = 6;
 constexpr int MAX_SPLITS = 4;
-constexpr int CONVERTER_WARPS = 4;
 
 template <int EPN> struct Geo {
-    static constexpr int TERM_BYTES = EPN * 128;  // EPN expert rows x 64 d_model (bf16)
-    static constexpr int B_BYTES = 3 * TERM_BYTES;
-    static constexpr int TMEM_COLS = EPN < 32 ? 32 : EPN;
+    static constexpr int TERM_BYTES = EPN * 128;       // one term: EPN expert rows x 64 d_model (bf16)
+    static constexpr int W_BYTES = 3 * TERM_BYTES;     // the three terms of one K block
+    static constexpr int NACC = 3 * EPN;               // accumulator columns [hi | mid | lo]
+    static constexpr int N0 = NACC <= 256 ? NACC : 256;  // the first MMA's N
+    static constexpr int N1 = NACC - N0;                 // the second's (EPN = 128: 128)
+    static constexpr int TMEM_COLS = NACC <= 64 ? 64 : NACC <= 128 ? 128 : NACC <= 256 ? 256 : 512;
     static constexpr int LDS = EPN + 1;  // epilogue row stride in floats (odd: conflict-free)
 };
-
-constexpr int WDEPTH = 2;  // slots of the weight rings (fp32 slices and their bf16 terms)
 
 struct Misc {
     uint64_t xfull[MAX_STAGES];   // x tile landed
     uint64_t xempty[MAX_STAGES];  // its MMAs are done
-    uint64_t wl[WDEPTH];          // fp32 weight slice landed
-    uint64_t bfull[WDEPTH];       // its bf16 terms are written
-    uint64_t bempty[WDEPTH];      // their MMAs are done
-    uint64_t wfree[WDEPTH];       // every weight warp is done reading the fp32 slice
+    uint64_t wfull[MAX_WSLOTS];   // weight terms landed
+    uint64_t wempty[MAX_WSLOTS];  // their MMAs are done
     uint64_t tfull;
     uint32_t tmem_base;
     int abort_flag;
@@ -86,7 +87,6 @@ struct Misc {
 
 struct Args {
     RouteOpts o;
-    const float* w;           // W_r (D, E) fp32
     const float* bias;        // E or null
     const float* noise;       // T x E or null
     float* logits_out;        // T x E or null
@@ -105,9 +105,8 @@ struct Args {
     int with_stats;
     int* status;
     int stages;               // depth of the x ring (16 KB stages)
-    uint32_t b_off;           // the bf16 weight-term ring (WDEPTH x 3 x EPN x 128 bytes)
-    uint32_t w_off;           // the fp32 weight-slice ring (WDEPTH x w_slot bytes)
-    uint32_t w_slot;          // bytes per fp32 slice slot (64 x E x 4, rounded up)
+    int wslots;               // depth of the weight-term ring
+    uint32_t w_off;           // the weight-term ring (wslots x W_BYTES), right after the x ring
     int splits;               // CTAs per token tile (cluster size along y)
     int split_kb;             // K blocks per split
     uint32_t misc_off;        // byte offsets in the aligned shared memory
@@ -121,38 +120,84 @@ MOE_DEVICE void st_cluster_f32(uint32_t cluster_addr, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
 }
 
-// The three bf16 terms of two fp32 weights, packed in pairs (a in the low
-// half): hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid), each pair
-// rounded by one paired conversion.
-MOE_DEVICE uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
-MOE_DEVICE void split3(float a, float b, uint32_t& hi, uint32_t& mid, uint32_t& lo)
+// terms[p][e][d] = the p-th bf16 term of W_r[d][e] (p = 0 hi, 1 mid, 2 lo);
+// rows e >= E are zero.  Two consecutive d per thread (D is even).
+__global__ void router_prepare_kernel(const float* __restrict__ w, __nv_bfloat16* __restrict__ terms,
+                                      int D, int E, int EPN)
 {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    const float2 hf = __bfloat1622float2(h);
-    const float ra = a - hf.x, rb = b - hf.y;
-    const __nv_bfloat162 m = __floats2bfloat162_rn(ra, rb);
-    const float2 mf = __bfloat1622float2(m);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(ra - mf.x, rb - mf.y);
-    hi = bf16x2_bits(h);
-    mid = bf16x2_bits(m);
-    lo = bf16x2_bits(l);
+    const int64_t half = (int64_t)D / 2;
+    const int64_t n = (int64_t)EPN * half;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int e = (int)(i / half);
+        const int d = (int)(i % half) * 2;
+        const float a = e < E ? w[(int64_t)d * E + e] : 0.f;
+        const float b = e < E ? w[(int64_t)(d + 1) * E + e] : 0.f;
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
+        const float2 hf = __bfloat1622float2(hi);
+        const float ra = a - hf.x, rb = b - hf.y;  // exact
+        const __nv_bfloat162 mid = __floats2bfloat162_rn(ra, rb);
+        const float2 mf = __bfloat1622float2(mid);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(ra - mf.x, rb - mf.y);
+        const int64_t o = (int64_t)e * D + d;
+        const int64_t plane = (int64_t)EPN * D;
+        *reinterpret_cast<__nv_bfloat162*>(terms + o) = hi;
+        *reinterpret_cast<__nv_bfloat162*>(terms + plane + o) = mid;
+        *reinterpret_cast<__nv_bfloat162*>(terms + 2 * plane + o) = lo;
+    }
+}
+
+// The three partial logits of accumulator columns e, EPN + e and 2 EPN + e,
+// added (hi + mid) + lo.
+template <int EPN>
+MOE_DEVICE void read_logits(uint32_t taddr, bool ok, float* dst_local, uint32_t dst_remote, bool remote)
+{
+    auto put = [&](int e, float v) {
+        if (remote) st_cluster_f32(dst_remote + e * 4, v);
+        else dst_local[e] = v;
+    };
+    if (EPN == 16) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(taddr, v0);       // hi 0..15, mid 0..15
+        tmem_ld_32x32b_x32(taddr + 32, v1);  // lo 0..15 (columns 48..63 unused)
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float L = (__uint_as_float(v0[e]) + __uint_as_float(v0[16 + e])) + __uint_as_float(v1[e]);
+            put(e, ok ? L : 0.f);
+        }
+    } else {
+#pragma unroll 1
+        for (int c = 0; c < EPN / 32; ++c) {
+            uint32_t h[32], m[32], l[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, h);
+            tmem_ld_32x32b_x32(taddr + EPN + c * 32, m);
+            tmem_ld_32x32b_x32(taddr + 2 * EPN + c * 32, l);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float L = (__uint_as_float(h[j]) + __uint_as_float(m[j])) + __uint_as_float(l[j]);
+                put(c * 32 + j, ok ? L : 0.f);
+            }
+        }
+    }
 }
 
 template <int EPN, int KM, int MINB>
 __global__ void __launch_bounds__(NUM_THREADS, MINB)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const Args a)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const Args a)
 {
     using G = Geo<EPN>;
-    constexpr int TERM = G::TERM_BYTES, LDS = G::LDS;
+    constexpr int LDS = G::LDS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* xring = smem;              // S x 16 KB; the whole ring area is the epilogue's scratch
-    uint8_t* bring = smem + a.b_off;    // WDEPTH x B_BYTES
-    uint8_t* wring = smem + a.w_off;    // WDEPTH x w_slot
+    uint8_t* xring = smem;              // S x 16 KB, then the weight ring: together the epilogue's scratch
+    uint8_t* wring = smem + a.w_off;    // WS x W_BYTES
     Misc* m = reinterpret_cast<Misc*>(smem + a.misc_off);
     float* recv = reinterpret_cast<float*>(smem + a.recv_off);
-    const int S = a.stages;
+    const int S = a.stages, WS = a.wslots;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
     const int split = (int)blockIdx.y;  // the CTA's rank in its cluster when splits > 1
@@ -160,7 +205,6 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     const int kb_begin = split * a.split_kb;                // never empty (host guarantee)
     const int kb_end = min(num_kb, kb_begin + a.split_kb);
     const int nkb = kb_end - kb_begin;
-    auto kb_at = [&](int i) { return kb_begin + i; };
     const int E = a.E;
 
     if (threadIdx.x == 0) {
@@ -168,35 +212,18 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             mbar_init(&m->xfull[s], 1);
             mbar_init(&m->xempty[s], 1);
         }
-        for (int j = 0; j < WDEPTH; ++j) {
-            mbar_init(&m->wl[j], 1);
-            mbar_init(&m->bfull[j], CONVERTER_WARPS);
-            mbar_init(&m->bempty[j], 1);
-            mbar_init(&m->wfree[j], CONVERTER_WARPS);
+        for (int j = 0; j < WS; ++j) {
+            mbar_init(&m->wfull[j], 1);
+            mbar_init(&m->wempty[j], 1);
         }
         mbar_init(&m->tfull, 1);
         m->abort_flag = 0;
         m->last = 0;
         fence_mbar_init();
         prefetch_tmap(&tmX);
+        prefetch_tmap(&tmW);
     }
-    if (warp >= 2) {
-        // weight terms: rows E .. EPN-1 (if any) stay zero in every slot
-        const int tid = threadIdx.x - 64;
-        m->cnt[tid] = 0;
-        const int pad = EPN - E;
-        if (pad > 0) {
-            const int per_slot = 3 * pad * 8;  // 16-byte chunks
-            for (int i = tid; i < WDEPTH * per_slot; i += 128) {
-                const int j = i / per_slot;
-                int r = i % per_slot;
-                const int p = r / (pad * 8);
-                r %= pad * 8;
-                uint8_t* dst = bring + (size_t)j * G::B_BYTES + p * TERM + (E + r / 8) * 128 + (r % 8) * 16;
-                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-    }
+    if (warp >= 2) m->cnt[threadIdx.x - 64] = 0;
     if (warp == 1) {
         tmem_alloc(&m->tmem_base, G::TMEM_COLS);
         tmem_relinquish();
@@ -206,14 +233,6 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
     volatile int* abort_flag = &m->abort_flag;
-    // the fp32 weight slice of K block kb into slot j (issued by one converter thread)
-    auto load_w = [&](int kb, int j) {
-        const int d0 = kb * BK;
-        const int rows = min(BK, a.D - d0);  // a multiple of 8 (D % 8 == 0)
-        const uint32_t bytes = (uint32_t)rows * (uint32_t)E * 4u;
-        mbar_arrive_expect_tx(&m->wl[j], bytes);
-        bulk_load_g2s(wring + (size_t)j * a.w_slot, a.w + (size_t)d0 * E, bytes, &m->wl[j]);
-    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -225,7 +244,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             for (int i = 0; i < nkb; ++i) {
                 if (!mbar_wait(&m->xempty[stage], phase ^ 1u, a.status, 510, abort_flag)) break;
                 mbar_arrive_expect_tx(&m->xfull[stage], A_BYTES);
-                tma_load_2d(xring + (size_t)stage * A_BYTES, &tmX, kb_at(i) * BK, (int32_t)t0,
+                tma_load_2d(xring + (size_t)stage * A_BYTES, &tmX, (kb_begin + i) * BK, (int32_t)t0,
                             &m->xfull[stage]);
                 last_phase[stage] = (int)phase;
                 if (++stage == S) {
@@ -241,104 +260,65 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = umma_idesc_bf16(BM, EPN, 0, 0);
+            constexpr uint32_t idesc0 = umma_idesc_bf16(BM, G::N0, 0, 0);
+            constexpr uint32_t idesc1 = umma_idesc_bf16(BM, G::N1 > 0 ? G::N1 : 16, 0, 0);
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % S, j = i % WDEPTH;
+                const int s = i % S, j = i % WS;
                 if (!mbar_wait(&m->xfull[s], (uint32_t)((i / S) & 1), a.status, 520, abort_flag)) break;
-                if (!mbar_wait(&m->bfull[j], (uint32_t)((i / WDEPTH) & 1), a.status, 521, abort_flag)) break;
+                if (!mbar_wait(&m->wfull[j], (uint32_t)((i / WS) & 1), a.status, 521, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t sA = smem_u32(xring + (size_t)s * A_BYTES);
-                const uint32_t sB = smem_u32(bring + (size_t)j * G::B_BYTES);
+                const uint32_t sB = smem_u32(wring + (size_t)j * G::W_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t acc = (i || kk) ? 1u : 0u;
+                    // both operands K-major: 8-row groups 1024 B apart, +32 B per 16-element K step
                     const uint64_t adesc = umma_desc_sw128(sA + kk * 32, 16, 1024);
-#pragma unroll
-                    for (int p = 0; p < 3; ++p) {
-                        const uint64_t bdesc = umma_desc_sw128(sB + p * TERM + kk * 32, 16, 1024);
-                        umma_f16_ss(tmem_base, adesc, bdesc, idesc, (i || kk || p) ? 1u : 0u);
-                    }
+                    umma_f16_ss(tmem_base, adesc, umma_desc_sw128(sB + kk * 32, 16, 1024), idesc0, acc);
+                    if (G::N1 > 0)  // weight rows 256 .. 3 EPN - 1 into columns 256 ..
+                        umma_f16_ss(tmem_base + 256, adesc, umma_desc_sw128(sB + 256 * 128 + kk * 32, 16, 1024),
+                                    idesc1, acc);
                 }
                 umma_commit(&m->xempty[s]);
-                umma_commit(&m->bempty[j]);
+                umma_commit(&m->wempty[j]);
             }
             umma_commit(&m->tfull);  // also the drain: every MMA done once it fires
         }
     } else {
-        // ------------------------------------------------ weight split (warps 2..5)
-        const int tid = threadIdx.x - 64;
-        {
-            int issued = 0;  // fp32 slices issued (slot = index % WDEPTH)
-            if (tid == 0)
-                for (; issued < WDEPTH && issued < nkb; ++issued) load_w(kb_at(issued), issued);
-            const int pairs = E * 8;  // (expert, 8-wide chunk of d_model)
-            int i = 0;
-            for (; i < nkb; ++i) {
-                const int j = i % WDEPTH;
-                const uint32_t ph = (uint32_t)((i / WDEPTH) & 1);
-                if (!mbar_wait(&m->wl[j], ph, a.status, 540, abort_flag)) break;
-                if (!mbar_wait(&m->bempty[j], ph ^ 1u, a.status, 541, abort_flag)) break;
-                uint8_t* sB = bring + (size_t)j * G::B_BYTES;
-                const float* wsm = reinterpret_cast<const float*>(wring + (size_t)j * a.w_slot);
-                const int d0 = kb_at(i) * BK;
-                for (int q = tid; q < pairs; q += 128) {
-                    const int e = q % E, c = q / E;
-                    const bool in = d0 + c * 8 < a.D;  // D % 8 == 0: a chunk is all in or all out
-                    float v[8];
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) v[jj] = in ? wsm[(c * 8 + jj) * E + e] : 0.f;
-                    uint32_t h[4], md[4], l[4];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) split3(v[2 * jj], v[2 * jj + 1], h[jj], md[jj], l[jj]);
-                    const int off = e * 128 + ((c ^ (e & 7)) << 4);
-                    *reinterpret_cast<uint4*>(sB + off) = make_uint4(h[0], h[1], h[2], h[3]);
-                    *reinterpret_cast<uint4*>(sB + TERM + off) = make_uint4(md[0], md[1], md[2], md[3]);
-                    *reinterpret_cast<uint4*>(sB + 2 * TERM + off) = make_uint4(l[0], l[1], l[2], l[3]);
-                }
-                fence_proxy_async_smem();  // visible to the tensor cores
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&m->bfull[j]);
-                    mbar_arrive(&m->wfree[j]);
-                }
-                // refill fp32 slot j once every weight warp is done with it
-                if (tid == 0 && issued < nkb) {
-                    if (!mbar_wait(&m->wfree[j], ph, a.status, 543, abort_flag)) break;
-                    load_w(kb_at(issued), issued % WDEPTH);
-                    ++issued;
+        if (warp == 2 && lane == 0) {
+            // ------------------------------------------------ weight terms, WS slots ahead
+            int slot = 0;
+            uint32_t phase = 0;
+            int last_phase[MAX_WSLOTS];
+            for (int j = 0; j < MAX_WSLOTS; ++j) last_phase[j] = -1;
+            for (int i = 0; i < nkb; ++i) {
+                if (!mbar_wait(&m->wempty[slot], phase ^ 1u, a.status, 540, abort_flag)) break;
+                mbar_arrive_expect_tx(&m->wfull[slot], G::W_BYTES);
+                tma_load_3d(wring + (size_t)slot * G::W_BYTES, &tmW, (kb_begin + i) * BK, 0, 0,
+                            &m->wfull[slot]);
+                last_phase[slot] = (int)phase;
+                if (++slot == WS) {
+                    slot = 0;
+                    phase ^= 1u;
                 }
             }
-            // after an early exit, the slices still in flight land before the CTA goes on
-            if (tid == 0)
-                for (int k = i; k < issued; ++k)
-                    mbar_wait(&m->wl[k % WDEPTH], (uint32_t)((k / WDEPTH) & 1), a.status, 542, nullptr);
+            for (int j = 0; j < WS; ++j)
+                if (last_phase[j] >= 0)
+                    mbar_wait(&m->wfull[j], (uint32_t)last_phase[j], a.status, 541, nullptr);
         }
+        __syncwarp();
         // ------------------------------------------------ accumulators out of tensor memory
         const int quad = warp & 3;        // the lane quadrant this warp may read
         const int r = quad * 32 + lane;   // token row in the tile
         float* Ls = reinterpret_cast<float*>(xring);  // [BM][LDS]
-        const bool ok = mbar_wait(&m->tfull, 0, a.status, 530, abort_flag);
+        // tcgen05.ld is warp-collective: the vote keeps the warp converged
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&m->tfull, 0, a.status, 530, abort_flag));
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
         uint32_t remote = 0;
         if (split > 0)  // this row's slot in the leader's receive buffer
             remote = mapa_shared(smem_u32(recv + ((size_t)(split - 1) * BM + r) * EPN), 0);
-#pragma unroll 1
-        for (int c = 0; c < (EPN + 31) / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(taddr + c * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int e = c * 32 + j;
-                if (e < EPN) {
-                    const float x = ok ? __uint_as_float(v[j]) : 0.f;
-                    if (split > 0)
-                        st_cluster_f32(remote + e * 4, x);
-                    else
-                        Ls[r * LDS + e] = x;
-                }
-            }
-        }
+        read_logits<EPN>(taddr, ok, Ls + r * LDS, remote, split > 0);
     }
     __syncwarp();
     if (a.splits > 1) cluster_sync();  // the other splits' partials are in the leader's buffer
@@ -538,13 +518,12 @@ static EncodeTiledFn encoder()
     return fn;
 }
 
-// Ring depth and shared-memory layout for `ctas_per_sm` CTAs on each SM:
-// [x ring: stages x 16 KB][weight terms: WDEPTH x 3 x EPN x 128][fp32 slices:
-// WDEPTH x w_slot][Misc][split partials]; the rings together are the
-// epilogue's scratch.
+// Ring depths and shared-memory layout for `ctas_per_sm` CTAs on each SM:
+// [x ring: stages x 16 KB][weight terms: wslots x 3 x EPN x 128][Misc][split
+// partials]; the two rings together are the epilogue's scratch.
 struct Plan {
-    int epn, splits, split_kb, ctas_per_sm, stages;
-    uint32_t b_off, w_off, w_slot, misc_off, recv_off;
+    int epn, splits, split_kb, ctas_per_sm, stages, wslots;
+    uint32_t w_off, misc_off, recv_off;
     size_t smem;  // dynamic shared memory, with 1 KB of alignment slack
 };
 
@@ -558,36 +537,45 @@ static Plan make_plan(const moe_config& c)
     const int nkb = (c.D + BK - 1) / BK;
     p.splits = router_tc_splits(c);
     p.split_kb = (nkb + p.splits - 1) / p.splits;
-    const size_t b_bytes = (size_t)3 * p.epn * 128;
-    p.w_slot = (uint32_t)align_up((size_t)64 * c.E * 4, 1024);
+    const size_t w_bytes = (size_t)3 * p.epn * 128;
     const size_t recv = (size_t)(p.splits - 1) * BM * p.epn * sizeof(float);
     const size_t misc = align_up(sizeof(Misc), 1024);
-    const size_t fixed = 1024 + WDEPTH * (b_bytes + p.w_slot) + misc + align_up(recv, 1024);
+    const size_t fixed = 1024 + misc + align_up(recv, 1024);
     // the epilogue scratch (and the statistics' last step) live in the rings
     const size_t epi = (size_t)2 * BM * (p.epn + 1) * sizeof(float);
     const size_t fin = (size_t)kStatD * sizeof(double) + (size_t)kStatC * sizeof(long long);
-    auto stages_for = [&](size_t budget) {
-        if (budget <= fixed) return 0;
-        int st = (int)((budget - fixed) / A_BYTES);
+    // the weight ring takes up to about 45 % of the budget (its tiles come from
+    // L2: a few in flight cover that latency), the x ring the rest
+    auto fit = [&](size_t budget, int& st, int& ws) {
+        st = ws = 0;
+        if (budget <= fixed) return false;
+        const size_t room = budget - fixed;
+        ws = (int)(room * 45 / 100 / w_bytes);
+        if (ws > MAX_WSLOTS) ws = MAX_WSLOTS;
+        if (ws < 2) ws = 2;
+        if ((size_t)ws * w_bytes >= room) return false;
+        st = (int)((room - (size_t)ws * w_bytes) / A_BYTES);
         if (st > MAX_STAGES) st = MAX_STAGES;
-        const size_t rings = (size_t)st * A_BYTES + WDEPTH * (b_bytes + p.w_slot);
-        return (rings >= epi && rings >= fin) ? st : 0;
+        const size_t rings = (size_t)st * A_BYTES + (size_t)ws * w_bytes;
+        return st >= 3 && rings >= epi && rings >= fin;
     };
     // two CTAs per SM when the tiles outnumber the SMs and each still gets 3 x stages
+    int st = 0, ws = 0;
     p.ctas_per_sm = 1;
-    if (tiles * p.splits > 148 && p.epn <= 64 && stages_for(112 * 1024) >= 3) p.ctas_per_sm = 2;
-    p.stages = stages_for(p.ctas_per_sm == 2 ? 112 * 1024 : 226 * 1024);
-    p.b_off = (uint32_t)((size_t)p.stages * A_BYTES);
-    p.w_off = p.b_off + (uint32_t)(WDEPTH * b_bytes);
-    p.misc_off = p.w_off + (uint32_t)(WDEPTH * p.w_slot);
+    if (tiles * p.splits > 148 && p.epn <= 64 && fit(112 * 1024, st, ws)) p.ctas_per_sm = 2;
+    else fit(226 * 1024, st, ws);
+    p.stages = st;
+    p.wslots = ws;
+    p.w_off = (uint32_t)((size_t)p.stages * A_BYTES);
+    p.misc_off = p.w_off + (uint32_t)((size_t)p.wslots * w_bytes);
     p.recv_off = p.misc_off + (uint32_t)misc;
     p.smem = (size_t)p.recv_off + align_up(recv, 1024) + 1024;
     return p;
 }
 
 template <int EPN, int KM, int MINB>
-static cudaError_t launch_t(const moe_config& c, const CUtensorMap& mX, const Args& a, const Plan& p,
-                            cudaStream_t s)
+static cudaError_t launch_t(const moe_config& c, const CUtensorMap& mX, const CUtensorMap& mW, const Args& a,
+                            const Plan& p, cudaStream_t s)
 {
     auto kern = router_tc_kernel<EPN, KM, MINB>;
     static PerDeviceFlag smem_set;
@@ -607,27 +595,27 @@ static cudaError_t launch_t(const moe_config& c, const CUtensorMap& mX, const Ar
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = p.splits > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, mX, a);
+    return cudaLaunchKernelEx(&cfg, kern, mX, mW, a);
 }
 
 template <int EPN>
-static cudaError_t launch_k(const moe_config& c, const CUtensorMap& mX, const Args& a, const Plan& p,
-                            cudaStream_t s)
+static cudaError_t launch_k(const moe_config& c, const CUtensorMap& mX, const CUtensorMap& mW, const Args& a,
+                            const Plan& p, cudaStream_t s)
 {
     const int km = c.K <= 2 ? 2 : c.K <= 4 ? 4 : c.K <= 6 ? 6 : 8;
     if (p.ctas_per_sm == 2) {
         if constexpr (EPN <= 64) {
-            return km == 2 ? launch_t<EPN, 2, 2>(c, mX, a, p, s)
-                 : km == 4 ? launch_t<EPN, 4, 2>(c, mX, a, p, s)
-                 : km == 6 ? launch_t<EPN, 6, 2>(c, mX, a, p, s)
-                           : launch_t<EPN, 8, 2>(c, mX, a, p, s);
+            return km == 2 ? launch_t<EPN, 2, 2>(c, mX, mW, a, p, s)
+                 : km == 4 ? launch_t<EPN, 4, 2>(c, mX, mW, a, p, s)
+                 : km == 6 ? launch_t<EPN, 6, 2>(c, mX, mW, a, p, s)
+                           : launch_t<EPN, 8, 2>(c, mX, mW, a, p, s);
         }
         return cudaErrorInvalidValue;
     }
-    return km == 2 ? launch_t<EPN, 2, 1>(c, mX, a, p, s)
-         : km == 4 ? launch_t<EPN, 4, 1>(c, mX, a, p, s)
-         : km == 6 ? launch_t<EPN, 6, 1>(c, mX, a, p, s)
-                   : launch_t<EPN, 8, 1>(c, mX, a, p, s);
+    return km == 2 ? launch_t<EPN, 2, 1>(c, mX, mW, a, p, s)
+         : km == 4 ? launch_t<EPN, 4, 1>(c, mX, mW, a, p, s)
+         : km == 6 ? launch_t<EPN, 6, 1>(c, mX, mW, a, p, s)
+                   : launch_t<EPN, 8, 1>(c, mX, mW, a, p, s);
 }
 
 }  // namespace rtc
@@ -654,17 +642,34 @@ int router_tc_splits(const moe_config& c)
     return (nkb + per - 1) / per;
 }
 
-cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x,
-                             const float* w_router, const float* bias, const float* noise,
-                             float* logits_out, float* probs_out, int32_t* ids, float* w,
-                             float* blk_mp, float* blk_z, float* blk_ent, int32_t* blk_cnt,
-                             float* mean_prob, float* losses, int* status, cudaStream_t s)
+size_t router_terms_bytes(const moe_config& c)
+{
+    if (c.dtype != MOE_BF16 || c.E > 128) return 0;
+    return (size_t)3 * rtc::epn_of(c.E) * (size_t)c.D * 2;
+}
+
+cudaError_t launch_router_prepare(const moe_config& c, const float* w_router, void* terms, cudaStream_t s)
+{
+    const int epn = rtc::epn_of(c.E);
+    const int64_t n = (int64_t)epn * (c.D / 2);
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    rtc::router_prepare_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+        w_router, static_cast<__nv_bfloat16*>(terms), c.D, c.E, epn);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void* x, const void* terms,
+                             const float* bias, const float* noise, float* logits_out, float* probs_out,
+                             int32_t* ids, float* w, float* blk_mp, float* blk_z, float* blk_ent,
+                             int32_t* blk_cnt, float* mean_prob, float* losses, int* status, cudaStream_t s)
 {
     using namespace rtc;
     const Plan p = make_plan(c);
+    if (p.stages < 3) return cudaErrorInvalidConfiguration;
     EncodeTiledFn enc = encoder();
     if (!enc) return cudaErrorInvalidValue;
-    CUtensorMap mX;
+    CUtensorMap mX, mW;
     {
         cuuint64_t dims[2] = {(cuuint64_t)c.D, (cuuint64_t)c.T};
         cuuint64_t strides[1] = {(cuuint64_t)c.D * 2};
@@ -675,9 +680,20 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
+    {
+        // terms[p][e][d]: box = 64 d_model x EPN experts x 3 terms, stacked in
+        // shared memory as 3 x EPN K-major rows of 128 bytes
+        cuuint64_t dims[3] = {(cuuint64_t)c.D, (cuuint64_t)p.epn, 3};
+        cuuint64_t strides[2] = {(cuuint64_t)c.D * 2, (cuuint64_t)p.epn * c.D * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)p.epn, 3};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&mW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(terms), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     Args a{};
     a.o = o;
-    a.w = w_router;
     a.bias = bias;
     a.noise = noise;
     a.logits_out = logits_out;
@@ -698,18 +714,17 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
     a.with_stats = (mean_prob != nullptr || losses != nullptr) ? 1 : 0;
     a.status = status;
     a.stages = p.stages;
-    a.b_off = p.b_off;
+    a.wslots = p.wslots;
     a.w_off = p.w_off;
-    a.w_slot = p.w_slot;
     a.splits = p.splits;
     a.split_kb = p.split_kb;
     a.misc_off = p.misc_off;
     a.recv_off = p.recv_off;
     switch (p.epn) {
-        case 16: return launch_k<16>(c, mX, a, p, s);
-        case 32: return launch_k<32>(c, mX, a, p, s);
-        case 64: return launch_k<64>(c, mX, a, p, s);
-        default: return launch_k<128>(c, mX, a, p, s);
+        case 16: return launch_k<16>(c, mX, mW, a, p, s);
+        case 32: return launch_k<32>(c, mX, mW, a, p, s);
+        case 64: return launch_k<64>(c, mX, mW, a, p, s);
+        default: return launch_k<128>(c, mX, mW, a, p, s);
     }
 }
 

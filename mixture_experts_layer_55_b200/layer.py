@@ -46,6 +46,21 @@ class MoELayer:
         self.losses = torch.zeros(3, dtype=torch.float32, device=self.device)  # z, balance, entropy
         self.mean_prob = torch.zeros(E, dtype=torch.float32, device=self.device)
         self.counts = torch.zeros(E, dtype=torch.int32, device=self.device)
+        # the router weight split once into the tensor-core router's bf16 terms
+        # (moe_router_prepare); split again when w_router is replaced or changed
+        # in place (tracked by the tensor's version counter)
+        nb = B.router_terms_size(self.cfg)
+        self.router_terms = torch.empty(nb, dtype=torch.uint8, device=self.device) if nb else None
+        self._terms_of = None
+
+    def _terms(self, stream=None):
+        if self.router_terms is None:
+            return None
+        key = (id(self.w_router), self.w_router.data_ptr(), self.w_router._version)
+        if key != self._terms_of:
+            B.moe_router_prepare(self.cfg, self.w_router, self.router_terms, stream=stream)
+            self._terms_of = key
+        return self.router_terms
 
     def forward(self, x, y=None, logit_noise=None, stats: bool = True, stream=None):
         """y = MoE(x) for x (T, D) on the device; returns y.  With stats the
@@ -54,7 +69,8 @@ class MoELayer:
         if y is None:
             y = torch.empty_like(x)
         B.moe_forward(self.cfg, x, self.w_router, self.w_gate, self.w_up, self.w_down, y,
-                      self.workspace, router_bias=self.router_bias, logit_noise=logit_noise,
+                      self.workspace, w_router_terms=self._terms(stream),
+                      router_bias=self.router_bias, logit_noise=logit_noise,
                       selection_bias=self.selection_bias, shared=self.shared,
                       losses=self.losses if stats else None,
                       mean_prob=self.mean_prob if stats else None,

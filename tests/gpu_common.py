@@ -105,6 +105,17 @@ class Bufs:
         assert flags == 0, f"device status flags {flags:#x}"
 
 
+def prepared_terms(cfg, w_router):
+    """The router weight split by moe_router_prepare (None where the layer's
+    router takes no prepared weight)."""
+    nb = B.router_terms_size(cfg)
+    if nb == 0:
+        return None
+    terms = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    B.moe_router_prepare(cfg, w_router, terms)
+    return terms
+
+
 def check_logits(wl, inp_cpu, logits_gpu):
     """fp32 logits against the fp64 ones, within gamma_n * sum|terms|."""
     L64 = oracle.router_logits(inp_cpu["x"], inp_cpu["w_router"], inp_cpu["bias"],

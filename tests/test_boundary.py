@@ -87,10 +87,10 @@ def test_workspace_sizes_grow_with_problem(lib):
 FAKE = 0x10000  # an aligned address the library never dereferences here
 
 
-def _call_route(lib, cfg, x=FAKE, w=FAKE, ids=FAKE, tw=FAKE, ws=FAKE, nbytes=None):
+def _call_route(lib, cfg, x=FAKE, w=FAKE, ids=FAKE, tw=FAKE, ws=FAKE, nbytes=None, terms=None):
     nb = B.workspace_size(cfg) if nbytes is None else nbytes
-    return lib.moe_route(ctypes.byref(cfg), x, w, None, None, None, None, None, None, ids, tw,
-                         None, None, ws, nb, None)
+    return lib.moe_route(ctypes.byref(cfg), x, w, terms, None, None, None, None, None, None, ids,
+                         tw, None, None, ws, nb, None)
 
 
 def test_route_argument_errors(lib):
@@ -99,6 +99,7 @@ def test_route_argument_errors(lib):
     assert _call_route(lib, c, tw=None) == B.MOE_ERR_ARG
     assert _call_route(lib, c, x=None) == B.MOE_ERR_ARG
     assert _call_route(lib, c, x=FAKE + 8) == B.MOE_ERR_ALIGN
+    assert _call_route(lib, c, terms=FAKE + 8) == B.MOE_ERR_ALIGN
     assert _call_route(lib, c, ws=None) == B.MOE_ERR_WORKSPACE
     assert _call_route(lib, c, nbytes=16) == B.MOE_ERR_WORKSPACE
     assert _call_route(lib, c, ws=FAKE + 16) == B.MOE_ERR_ALIGN  # workspace wants 256 B
@@ -128,17 +129,20 @@ def test_dispatch_ffn_combine_forward_argument_errors(lib):
     assert lib.moe_expert_ffn(cr, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nb,
                               None) == B.MOE_ERR_ARG
     fb = B.forward_workspace_size(c)
-    assert lib.moe_forward(cr, FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, None, None, None,
-                           FAKE, None, None, None, None, None, FAKE, fb - 1,
+    assert lib.moe_forward(cr, FAKE, FAKE, None, None, None, None, FAKE, FAKE, FAKE, None, None,
+                           None, FAKE, None, None, None, None, None, FAKE, fb - 1,
                            None) == B.MOE_ERR_WORKSPACE
-    assert lib.moe_forward(cr, FAKE, None, None, None, None, FAKE, FAKE, FAKE, None, None, None,
-                           FAKE, None, None, None, None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+    assert lib.moe_forward(cr, FAKE, None, None, None, None, None, FAKE, FAKE, FAKE, None, None,
+                           None, FAKE, None, None, None, None, None, FAKE, fb, None) == B.MOE_ERR_ARG
+    assert lib.moe_forward(cr, FAKE, FAKE, FAKE + 8, None, None, None, FAKE, FAKE, FAKE, None,
+                           None, None, FAKE, None, None, None, None, None, FAKE, fb,
+                           None) == B.MOE_ERR_ALIGN
     # a shared expert needs its three weights
     cs = _cfg(F_shared=64)
     fbs = B.forward_workspace_size(cs)
     assert fbs > fb
-    assert lib.moe_forward(ctypes.byref(cs), FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE,
-                           None, FAKE, FAKE, None, None, None, None, None, FAKE, fbs,
+    assert lib.moe_forward(ctypes.byref(cs), FAKE, FAKE, None, None, None, None, FAKE, FAKE, FAKE,
+                           FAKE, None, FAKE, FAKE, None, None, None, None, None, FAKE, fbs,
                            None) == B.MOE_ERR_ARG
     assert lib.moe_update_selection_bias(cr, None, ctypes.c_float(0.01), FAKE, None) == B.MOE_ERR_ARG
     assert lib.moe_update_selection_bias(cr, FAKE, ctypes.c_float(float("nan")), FAKE,
@@ -158,15 +162,35 @@ def test_forward_kernel_count(lib):
     # router: SIMT logits GEMM + top-k (the top-k kernel finishes the statistics)
     assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 7
     # tensor-core router: one kernel for routing and statistics, with or without the
-    # d_model split (64 tiles of 128 tokens: a cluster of 2 CTAs per tile)
-    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=16, K=2)) == 6
-    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=64, K=6)) == 6
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 6
+    # d_model split (64 tiles of 128 tokens: a cluster of 2 CTAs per tile), after the
+    # weight split unless the caller passes prepared terms
+    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=16, K=2), True) == 6
+    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=64, K=6), True) == 6
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2), True) == 6
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 7
     assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 8  # split SIMT router
+    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8), True) == 8
     assert B.forward_kernel_count(_cfg(K=0)) == 0
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256)) == 9
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256), True) == 9
     # more chunks of 2048 assignments than SMs: the three-kernel index pass
-    assert B.forward_kernel_count(_cfg(T=160000, D=256, F=256, E=8, K=2)) == 8
+    assert B.forward_kernel_count(_cfg(T=160000, D=256, F=256, E=8, K=2), True) == 8
+
+
+def test_router_terms_size_and_prepare_checks(lib):
+    # 3 terms x E rounded up to 16/32/64/128 x D bf16 for bf16 layers with E <= 128
+    assert B.router_terms_size(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 3 * 16 * 4096 * 2
+    assert B.router_terms_size(_cfg(T=16384, D=2048, F=1408, E=64, K=6)) == 3 * 64 * 2048 * 2
+    assert B.router_terms_size(_cfg(T=64, D=256, F=256, E=100, K=2)) == 3 * 128 * 256 * 2
+    assert B.router_terms_size(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 0
+    assert B.router_terms_size(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 0
+    c = ctypes.byref(_cfg(T=8192, D=4096, F=14336, E=8, K=2))
+    assert lib.moe_router_prepare(c, FAKE, None, None) == B.MOE_ERR_ARG
+    assert lib.moe_router_prepare(c, None, FAKE, None) == B.MOE_ERR_ARG
+    assert lib.moe_router_prepare(c, FAKE, FAKE + 8, None) == B.MOE_ERR_ALIGN
+    c32 = ctypes.byref(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32"))
+    assert lib.moe_router_prepare(c32, FAKE, FAKE, None) == B.MOE_ERR_UNSUPPORTED
+    bad = ctypes.byref(_cfg(K=0))
+    assert lib.moe_router_prepare(bad, FAKE, FAKE, None) != B.MOE_OK
 
 
 def test_status_strings_and_trace_table(lib):

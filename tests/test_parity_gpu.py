@@ -16,7 +16,7 @@ import torch
 import oracle
 from mixture_experts_layer_55_b200 import _binding as B
 from tests.gpu_common import (Bufs, assert_close_out, check_logits, check_routing, check_tokens,
-                              full_size_tokens, to_np)
+                              full_size_tokens, prepared_terms, to_np)
 from workloads import WORKLOADS, Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -124,14 +124,17 @@ def test_small_layers_elementwise(cuda_ok, wl):
             assert (to_np(b.y[none]) == 0).all()
         else:
             assert torch.equal(b.y[none], b.y_shared[none])
-    # the whole layer in one call gives the same bits as the op-by-op path
+    # the whole layer in one call gives the same bits as the op-by-op path (the
+    # latter splits the router weight inside moe_route; here it is prepared once)
     ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
     y2 = torch.empty_like(b.y)
     losses = torch.empty(3, device="cuda")
     counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+    terms = prepared_terms(b.cfg, inp["w_router"])
     B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y2,
                   ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses,
-                  counts=counts, selection_bias=inp["sel_bias"], shared=inp["shared"])
+                  counts=counts, selection_bias=inp["sel_bias"], shared=inp["shared"],
+                  w_router_terms=terms)
     torch.cuda.synchronize()
     assert torch.equal(y2, b.y)
     assert torch.equal(losses, b.losses)
@@ -185,10 +188,10 @@ def test_update_selection_bias_matches_oracle(cuda_ok):
     assert float(b[2]) == float(bias0[2])
 
 
-def test_unaligned_router_weight_takes_the_simt_router(cuda_ok):
-    """A router weight that is not 16-byte aligned cannot be bulk-copied by the
-    tensor-core router; the SIMT router routes instead, with the same results
-    against the oracle."""
+def test_unaligned_router_weight(cuda_ok):
+    """A router weight that is not 16-byte aligned: the weight split reads it
+    with plain loads, so the tensor-core router still serves the layer, with
+    the same results against the oracle."""
     wl = _wl("unaligned_wr", T=2304, D=128, F=32, E=12, K=3, bias="zipf", seed=47)
     inp_cpu = make_inputs(wl, device="cpu")
     inp = _to_dev(inp_cpu)
@@ -273,12 +276,14 @@ def test_full_size_layer(cuda_ok, capsys, name):
     b = Bufs(wl)
     b.run_ops(inp)
     rt = check_routing(wl, b, inp["sel_bias"])
-    # the benchmark's call: the whole layer through moe_forward
+    # the benchmark's call: the whole layer through moe_forward, the router
+    # weight prepared once
     ws = torch.zeros(B.forward_workspace_size(b.cfg), dtype=torch.uint8, device="cuda")
     y = torch.empty_like(b.y)
     losses = torch.empty(3, device="cuda")
     B.moe_forward(b.cfg, inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y,
-                  ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses)
+                  ws, router_bias=inp["bias"], logit_noise=inp["noise"], losses=losses,
+                  w_router_terms=prepared_terms(b.cfg, inp["w_router"]))
     torch.cuda.synchronize()
     assert B.moe_get_device_status(ws) == 0
     assert torch.equal(y, b.y), "moe_forward differs from the op-by-op path"
