@@ -83,6 +83,8 @@ struct Misc {
     float psum[128];  // chunk sums of the normalised scores
     float wz[4];      // per lane-quadrant sums of lse^2
     float wh[4];      // and of the entropy
+    float bias_s[128];  // router bias (0 when none)
+    float sel_s[128];   // selection bias (0 when none)
 };
 
 struct Args {
@@ -334,7 +336,36 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         const RouteOpts& o = a.o;
         float* Ls = reinterpret_cast<float*>(xring);  // logits, then normalised scores
         float* Xs = Ls + BM * LDS;                     // scores: exp(L - max), or sigmoid(L)
+        float* Ns = Xs + BM * LDS;                     // this tile's logit noise
         const int G = o.n_groups, gsz = E / G;
+        const int rows = a.T - t0 < BM ? (int)(a.T - t0) : BM;  // tokens of this tile
+        // the biases, and the tile's noise rows (one contiguous block, read coalesced)
+        for (int e = tid; e < E; e += 128) {
+            m->bias_s[e] = a.bias ? a.bias[e] : 0.f;
+            m->sel_s[e] = o.sel_bias ? o.sel_bias[e] : 0.f;
+        }
+        if (a.noise) {
+            // eight loads in flight per thread, then their stores
+            const float* src = a.noise + t0 * E;
+            const int n = rows * E;
+            for (int i0 = 0; i0 < n; i0 += 8 * 128) {
+                float v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + u * 128 + tid;
+                    v[u] = i < n ? __ldcs(src + i) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + u * 128 + tid;
+                    if (i < n) {
+                        const int rr = i / E;
+                        Ns[rr * LDS + (i - rr * E)] = v[u];
+                    }
+                }
+            }
+        }
+        epi_sync();
         // top-K by (u desc, id asc), u = L + selection bias: an unrolled insertion
         // network of KM >= K slots (a displaced entry carried down keeps that order)
         float tv[KM];
@@ -363,12 +394,19 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         for (int e = 0; e < E; ++e) {
             float L = Ls[r * LDS + e];
             for (int sp = 1; sp < a.splits; ++sp) L += recv[((size_t)(sp - 1) * BM + r) * EPN + e];
-            if (a.bias) L += a.bias[e];
-            if (a.noise && valid) L += a.noise[t * E + e];
-            if (a.logits_out && valid) a.logits_out[t * E + e] = L;
+            if (a.bias) L += m->bias_s[e];
+            if (a.noise && valid) L += Ns[r * LDS + e];
             Ls[r * LDS + e] = L;
             mx = fmaxf(mx, L);
-            if (G == 1) insert(L + (o.sel_bias ? o.sel_bias[e] : 0.f), e);
+            if (G == 1) insert(L + m->sel_s[e], e);
+        }
+        if (a.logits_out) {  // the tile's logits, one contiguous block, written coalesced
+            epi_sync();
+            float* dst = a.logits_out + t0 * E;
+            for (int i = tid; i < rows * E; i += 128) {
+                const int rr = i / E;
+                dst[i] = Ls[rr * LDS + (i - rr * E)];
+            }
         }
         // pass 2: softmax sum, sum of exp(L - max) (L - max) for the entropy, and
         // the scores (sigmoid scores and their sum with score_func sigmoid)
@@ -400,7 +438,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 gm[g] = -INFINITY;
                 if (g < G)
                     for (int e = g * gsz; e < (g + 1) * gsz; ++e)
-                        gm[g] = fmaxf(gm[g], Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f));
+                        gm[g] = fmaxf(gm[g], Ls[r * LDS + e] + m->sel_s[e]);
             }
             uint32_t keep = 0;
             for (int rr = 0; rr < o.topk_groups; ++rr) {
@@ -415,7 +453,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 keep |= 1u << bg;
             }
             for (int e = 0; e < E; ++e)
-                if ((keep >> (e / gsz)) & 1u) insert(Ls[r * LDS + e] + (o.sel_bias ? o.sel_bias[e] : 0.f), e);
+                if ((keep >> (e / gsz)) & 1u) insert(Ls[r * LDS + e] + m->sel_s[e], e);
         }
         // weights from the scores of the selected experts
         float sk[KM];
@@ -440,7 +478,14 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         for (int e = 0; e < E; ++e) {
             const float pn = Xs[r * LDS + e] * scinv;
             Ls[r * LDS + e] = valid ? pn : 0.f;
-            if (a.probs_out && valid) a.probs_out[t * E + e] = pn;
+        }
+        if (a.probs_out) {  // one contiguous block, written coalesced
+            epi_sync();
+            float* dst = a.probs_out + t0 * E;
+            for (int i = tid; i < rows * E; i += 128) {
+                const int rr = i / E;
+                dst[i] = Ls[rr * LDS + (i - rr * E)];
+            }
         }
         if (a.with_stats) {
             // per-CTA statistics, each in a fixed order
@@ -529,7 +574,7 @@ struct Plan {
 
 static int epn_of(int E) { return E <= 16 ? 16 : E <= 32 ? 32 : E <= 64 ? 64 : 128; }
 
-static Plan make_plan(const moe_config& c)
+static Plan make_plan(const moe_config& c, bool noise)
 {
     Plan p{};
     p.epn = epn_of(c.E);
@@ -542,7 +587,7 @@ static Plan make_plan(const moe_config& c)
     const size_t misc = align_up(sizeof(Misc), 1024);
     const size_t fixed = 1024 + misc + align_up(recv, 1024);
     // the epilogue scratch (and the statistics' last step) live in the rings
-    const size_t epi = (size_t)2 * BM * (p.epn + 1) * sizeof(float);
+    const size_t epi = (size_t)(noise ? 3 : 2) * BM * (p.epn + 1) * sizeof(float);
     const size_t fin = (size_t)kStatD * sizeof(double) + (size_t)kStatC * sizeof(long long);
     // the weight ring takes up to about 45 % of the budget (its tiles come from
     // L2: a few in flight cover that latency), the x ring the rest
@@ -665,7 +710,7 @@ cudaError_t launch_router_tc(const moe_config& c, const RouteOpts& o, const void
                              int32_t* blk_cnt, float* mean_prob, float* losses, int* status, cudaStream_t s)
 {
     using namespace rtc;
-    const Plan p = make_plan(c);
+    const Plan p = make_plan(c, noise != nullptr);
     if (p.stages < 3) return cudaErrorInvalidConfiguration;
     EncodeTiledFn enc = encoder();
     if (!enc) return cudaErrorInvalidValue;
