@@ -78,6 +78,18 @@ def barrier(world: int):
         dist.barrier()
 
 
+def materialize_events(event_lists, stream):
+    """Give every torch event its CUDA handle before a timed region: torch
+    creates it lazily at the first record, and the library's trace attach
+    records a handle-less event once to obtain one, which inside the timed
+    region would add an event record per stage boundary and step."""
+    for evs in event_lists:
+        for e in evs:
+            if not e.cuda_event:
+                e.record(stream)
+    torch.cuda.synchronize()
+
+
 def aggregate(ms_total_local: float, world: int, T: int, steps: int, device) -> tuple:
     """(ms per step, tokens/s of the whole job): the slowest rank's device time
     over all ranks' tokens (each rank processes its own T tokens per step)."""
@@ -336,6 +348,8 @@ def measure_forward(M, wl: Workload, args, rank: int, world: int, dev, *, headli
 
     def timed(run_step, per_step_events=None):
         """Device time of `steps` steps (ms, this rank), with the clock record."""
+        if per_step_events is not None:
+            materialize_events(per_step_events, stream)
         clocks = ClockSampler(dev.index if dev.index is not None else 0)
         clocks.start()
         time.sleep(0.3)
@@ -367,7 +381,8 @@ def measure_forward(M, wl: Workload, args, rank: int, world: int, dev, *, headli
         M.moe_trace_attach([])
         return total, clocks.stop()
 
-    # eager: stream launches, with per-stage events
+    # eager: stream launches, with an event at every stage boundary inside the
+    # timed region (the per-kernel times on the launching stream)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(steps)]
     eager_total, eager_clk = timed(lambda i: layer.forward(xs[i % nbuf], y, logit_noise=noise),
                                    evs)
@@ -379,6 +394,10 @@ def measure_forward(M, wl: Workload, args, rank: int, world: int, dev, *, headli
     launch = "stream"
     total, clk = eager_total, eager_clk
     eager_ms_step = max_over_ranks(eager_total, world, dev) / steps
+    # for reference: the same steps without the stage events (each event record
+    # is a command of its own on the stream)
+    plain_total, _ = timed(lambda i: layer.forward(xs[i % nbuf], y, logit_noise=noise))
+    untraced_ms_step = max_over_ranks(plain_total, world, dev) / steps
     if graph:
         # one CUDA graph of the whole forward per input buffer, replayed
         graphs = [layer.capture(xs[i], y, logit_noise=noise) for i in range(nbuf)]
@@ -394,7 +413,7 @@ def measure_forward(M, wl: Workload, args, rank: int, world: int, dev, *, headli
     kept_rows = int(min(sum(min(c, M.capacity(layer.cfg)) for c in counts), M.max_rows(layer.cfg)))
     alg = algorithmic(wl, counts, kept_rows)
     rec = {"value": round(value, 1), "unit": UNIT, "ms_per_step": round(ms_step, 4),
-           "steps": steps, "launch": launch}
+           "steps": steps, "launch": launch, "untraced_ms_per_step": round(untraced_ms_step, 4)}
     if graph:
         rec["stream_ms_per_step"] = round(eager_ms_step, 4)
 
@@ -493,6 +512,7 @@ def run_gpu(args):
         "config": head["config"],
         "e2e": head["e2e"],
         "gpu_launches": head["gpu_launches"],
+        "untraced_ms_per_step": head["untraced_ms_per_step"],
         "roofline": head["roofline"],
         "stages": head["stages"],
         "layer": head["layer"],
@@ -542,6 +562,7 @@ def run_gpu_train(args):
     evf = [[torch.cuda.Event(enable_timing=True) for _ in range(nf)] for _ in range(args.steps)]
     evb = [[torch.cuda.Event(enable_timing=True) for _ in range(nbk)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    materialize_events(evf + evb, stream)
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
