@@ -548,13 +548,23 @@ MOE_API moe_status moe_ep_peer_combine(const moe_config *cfg, int32_t world, con
  *     behind; each call clears what must start at zero.  Calls whose work
  *     overlaps on the GPU (other streams, other threads) race on the array:
  *     order them on one stream.
- *   - Device-side range checks still guard every write, but their flags are
- *     kept in the shared array and are not reported to the caller.
+ *   - Device-side range checks still guard every write; their flags go to a
+ *     status word in the shared array, cleared at the start of every call and
+ *     read back by moe_dispatch_noalloc_status.
  */
 MOE_API moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
                                         const int32_t *topk_ids, int32_t *counts, int32_t *kept,
                                         int32_t *offsets, int32_t *perm, int32_t *row_of,
                                         void *x_perm, void *stream);
+
+/*
+ * The device status of the last moe_dispatch_noalloc on the current device
+ * (the MOE_DEVFLAG_* bits of its static array's status word, read like
+ * moe_get_device_status reads a workspace's): synchronises the stream, stores
+ * the flags in *flags and returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
+ * MOE_ERR_DEVICE_BOUNDS.  Allocates nothing.
+ */
+MOE_API moe_status moe_dispatch_noalloc_status(void *stream, int32_t *flags);
 
 /*
  * Device status of a workspace: synchronises the stream, then reads the

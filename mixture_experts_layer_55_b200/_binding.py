@@ -23,6 +23,8 @@ MOE_ERR_CUDA = -5
 MOE_ERR_DEVICE_TIMEOUT = -6
 MOE_ERR_DEVICE_BOUNDS = -7
 MOE_ERR_WORKSPACE = -8
+MOE_DEVFLAG_TIMEOUT = 0x1  # device status word bits (include/moe.h)
+MOE_DEVFLAG_BOUNDS = 0x2
 
 MOE_F32 = 0
 MOE_BF16 = 1
@@ -80,6 +82,7 @@ _SIG = {
     "moe_route": ([_P] * 15 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch_noalloc": ([_P] * 10, ctypes.c_int32),
+    "moe_dispatch_noalloc_status": ([_P, _P], ctypes.c_int32),
     "moe_expert_ffn": ([_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([_P] * 6, ctypes.c_int32),
     "moe_forward": ([_P] * 20 + [ctypes.c_size_t, _P], ctypes.c_int32),
@@ -249,6 +252,16 @@ def moe_dispatch_noalloc(cfg, x, topk_ids, counts, kept, offsets, perm, row_of, 
                                     _ptr(offsets), _ptr(perm), _ptr(row_of), _ptr(x_perm),
                                     _stream(stream))
     _check(st, "moe_dispatch_noalloc")
+
+
+def moe_dispatch_noalloc_status(stream=None) -> int:
+    """Flags word of the last moe_dispatch_noalloc on the current device
+    (synchronises the stream)."""
+    flags = ctypes.c_int32()
+    st = lib().moe_dispatch_noalloc_status(_stream(stream), ctypes.byref(flags))
+    if st not in (MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS):
+        _check(st, "moe_dispatch_noalloc_status")
+    return flags.value
 
 
 def moe_expert_ffn(cfg, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h, y_perm, workspace,

@@ -81,3 +81,20 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
     }
     return cuda_status(e);
 }
+
+extern "C" moe_status moe_dispatch_noalloc_status(void* stream, int32_t* flags)
+{
+    if (flags == nullptr) return MOE_ERR_ARG;
+    char* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t word = 0;  // word 0 of the status region (offset 0 of the layout)
+    e = cudaMemcpyAsync(&word, scratch, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e);
+    *flags = word;
+    if (word & MOE_DEVFLAG_TIMEOUT) return MOE_ERR_DEVICE_TIMEOUT;
+    if (word & MOE_DEVFLAG_BOUNDS) return MOE_ERR_DEVICE_BOUNDS;
+    return MOE_OK;
+}

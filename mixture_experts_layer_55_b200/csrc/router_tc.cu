@@ -389,16 +389,34 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         };
         // pass 1: logits (own K range + the other splits in order, + bias + noise),
         // their maximum, and (without a group limit) the top-K
-        float mx = -INFINITY;
+        if (a.splits > 1 || a.bias || (a.noise && valid)) {
+            // the complete logits first, so that the top-K loop below stays lean
+            float* Lr = Ls + r * LDS;
+            for (int sp = 1; sp < a.splits; ++sp) {
+                const float* Pr = recv + ((size_t)(sp - 1) * BM + r) * EPN;
 #pragma unroll 4
-        for (int e = 0; e < E; ++e) {
-            float L = Ls[r * LDS + e];
-            for (int sp = 1; sp < a.splits; ++sp) L += recv[((size_t)(sp - 1) * BM + r) * EPN + e];
-            if (a.bias) L += m->bias_s[e];
-            if (a.noise && valid) L += Ns[r * LDS + e];
-            Ls[r * LDS + e] = L;
-            mx = fmaxf(mx, L);
-            if (G == 1) insert(L + m->sel_s[e], e);
+                for (int e = 0; e < E; ++e) Lr[e] += Pr[e];
+            }
+            if (a.bias) {
+#pragma unroll 4
+                for (int e = 0; e < E; ++e) Lr[e] += m->bias_s[e];
+            }
+            if (a.noise && valid) {
+#pragma unroll 4
+                for (int e = 0; e < E; ++e) Lr[e] += Ns[r * LDS + e];
+            }
+        }
+        float mx = -INFINITY;
+        if (G == 1) {
+#pragma unroll 8
+            for (int e = 0; e < E; ++e) {
+                const float L = Ls[r * LDS + e];
+                mx = fmaxf(mx, L);
+                insert(L + m->sel_s[e], e);
+            }
+        } else {
+#pragma unroll 8
+            for (int e = 0; e < E; ++e) mx = fmaxf(mx, Ls[r * LDS + e]);
         }
         if (a.logits_out) {  // the tile's logits, one contiguous block, written coalesced
             epi_sync();

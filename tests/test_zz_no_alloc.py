@@ -7,7 +7,7 @@ array inside the library, so it takes no workspace.
 The GPU test calls it through the C ABI twice in a row, on different routings,
 and checks each result against moe_dispatch (with a workspace): the index
 arrays and the gathered rows are integer or copy work, so they must match
-bit for bit.  This file is collected last on purpose.
+bit for bit; the static array's status word must stay clear.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -38,6 +38,7 @@ def test_rejects_problems_beyond_the_static_scratch():
     st = lib.moe_dispatch_noalloc(ctypes.byref(bad), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                   None, None)
     assert st == B.MOE_ERR_ARG
+    assert lib.moe_dispatch_noalloc_status(None, None) == B.MOE_ERR_ARG
 
 
 def _outputs(cfg, dev):
@@ -73,6 +74,7 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice(cuda_ok):
                                got["perm"], got["row_of"], got["x_perm"])
         torch.cuda.synchronize(dev)
         assert B.moe_get_device_status(ws) == 0
+        assert B.moe_dispatch_noalloc_status() == 0  # the static array's own status word
         R = int(ref["offsets"][-1])
         assert R > 0 and int(ref["kept"].sum()) == R
         assert int((ref["row_of"] < 0).sum()) > 0, "the capacity factor should drop assignments"
@@ -80,3 +82,26 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice(cuda_ok):
             assert torch.equal(got[k], ref[k]), f"call {call}: {k} differs"
         assert torch.equal(got["perm"][:R], ref["perm"][:R]), f"call {call}: perm differs"
         assert torch.equal(got["x_perm"][:R], ref["x_perm"][:R]), f"call {call}: x_perm differs"
+
+
+@pytest.mark.gpu
+def test_noalloc_status_reports_a_corrupt_id_and_clears(cuda_ok):
+    """An expert id out of range is skipped by the device range check, which sets
+    the bounds flag in the static array's status word; the next clean call starts
+    from a cleared word."""
+    build_mod.build()
+    dev = torch.device("cuda", 0)
+    cfg = _cfg(capacity_factor=0.0)
+    g = torch.Generator(device=dev).manual_seed(5)
+    ids = torch.randint(0, cfg.E, (cfg.T, cfg.K), generator=g, device=dev, dtype=torch.int32)
+    bad = ids.clone()
+    bad[17, 1] = cfg.E + 3
+    out = _outputs(cfg, dev)
+    B.moe_dispatch_noalloc(cfg, None, bad, out["counts"], out["kept"], out["offsets"], out["perm"],
+                           out["row_of"], None)
+    assert B.moe_dispatch_noalloc_status() & B.MOE_DEVFLAG_BOUNDS
+    out = _outputs(cfg, dev)
+    B.moe_dispatch_noalloc(cfg, None, ids, out["counts"], out["kept"], out["offsets"], out["perm"],
+                           out["row_of"], None)
+    assert B.moe_dispatch_noalloc_status() == 0
+    assert int(out["offsets"][-1]) == cfg.T * cfg.K
