@@ -55,7 +55,16 @@ namespace rtc {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB x tile per stage
-constexpr int NUM_THREADS = 192;      // warp 0 x TMA, warp 1 MMA, warps 2..5 weight TMA + epilogue
+// Warps: 0 x TMA, 1 MMA, 2.. weight TMA (lane 0 of warp 2) and the epilogue:
+// eight epilogue warps (two per tensor-memory lane quadrant, each taking half
+// of the experts of its 32 tokens) with one CTA per SM, four with two CTAs.
+template <int MINB> struct Threads {
+    static constexpr int EPI_WARPS = MINB == 1 ? 8 : 4;
+    static constexpr int HALVES = EPI_WARPS / 4;
+    static constexpr int NTH = 32 * EPI_WARPS;  // epilogue threads
+    static constexpr int NT = 64 + NTH;         // block size
+};
+constexpr int MAX_KM = 8;
 constexpr int MAX_STAGES = 10;
 constexpr int MAX_WSLOTS = 6;
 constexpr int MAX_SPLITS = 4;
@@ -80,7 +89,7 @@ struct Misc {
     int abort_flag;
     int last;         // this CTA finishes the statistics of the grid
     int cnt[128];     // this CTA's expert counts
-    float psum[128];  // chunk sums of the normalised scores
+    float psum[256];  // chunk sums of the normalised scores
     float wz[4];      // per lane-quadrant sums of lse^2
     float wh[4];      // and of the entropy
     float bias_s[128];  // router bias (0 when none)
@@ -115,7 +124,8 @@ struct Args {
     uint32_t recv_off;        // (splits - 1) x BM x EPN fp32 partial logits (leader)
 };
 
-MOE_DEVICE void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// barrier of the NTH epilogue threads
+template <int NTH> MOE_DEVICE void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NTH) : "memory"); }
 
 MOE_DEVICE void st_cluster_f32(uint32_t cluster_addr, float v)
 {
@@ -186,11 +196,12 @@ MOE_DEVICE void read_logits(uint32_t taddr, bool ok, float* dst_local, uint32_t 
 }
 
 template <int EPN, int KM, int MINB>
-__global__ void __launch_bounds__(NUM_THREADS, MINB)
+__global__ void __launch_bounds__(Threads<MINB>::NT, MINB)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const Args a)
 {
     using G = Geo<EPN>;
+    using TH = Threads<MINB>;
     constexpr int LDS = G::LDS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -225,7 +236,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
     }
-    if (warp >= 2) m->cnt[threadIdx.x - 64] = 0;
+    if (warp >= 2 && threadIdx.x - 64 < 128) m->cnt[threadIdx.x - 64] = 0;
     if (warp == 1) {
         tmem_alloc(&m->tmem_base, G::TMEM_COLS);
         tmem_relinquish();
@@ -309,25 +320,35 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                     mbar_wait(&m->wfull[j], (uint32_t)last_phase[j], a.status, 541, nullptr);
         }
         __syncwarp();
-        // ------------------------------------------------ accumulators out of tensor memory
-        const int quad = warp & 3;        // the lane quadrant this warp may read
-        const int r = quad * 32 + lane;   // token row in the tile
-        float* Ls = reinterpret_cast<float*>(xring);  // [BM][LDS]
-        // tcgen05.ld is warp-collective: the vote keeps the warp converged
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&m->tfull, 0, a.status, 530, abort_flag));
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
-        uint32_t remote = 0;
-        if (split > 0)  // this row's slot in the leader's receive buffer
-            remote = mapa_shared(smem_u32(recv + ((size_t)(split - 1) * BM + r) * EPN), 0);
-        read_logits<EPN>(taddr, ok, Ls + r * LDS, remote, split > 0);
+        if (warp < 6) {
+            // -------------------------------------------- accumulators out of tensor memory
+            const int quad = warp & 3;        // the lane quadrant this warp may read
+            const int r = quad * 32 + lane;   // token row in the tile
+            float* Ls = reinterpret_cast<float*>(xring);  // [BM][LDS]
+            // tcgen05.ld is warp-collective: the vote keeps the warp converged
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&m->tfull, 0, a.status, 530, abort_flag));
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+            uint32_t remote = 0;
+            if (split > 0)  // this row's slot in the leader's receive buffer
+                remote = mapa_shared(smem_u32(recv + ((size_t)(split - 1) * BM + r) * EPN), 0);
+            read_logits<EPN>(taddr, ok, Ls + r * LDS, remote, split > 0);
+        } else {
+            // the second epilogue warp of each quadrant: the rings are the
+            // epilogue's scratch only once every MMA (and so every copy) is done
+            mbar_wait(&m->tfull, 0, a.status, 531, abort_flag);
+        }
     }
     __syncwarp();
     if (a.splits > 1) cluster_sync();  // the other splits' partials are in the leader's buffer
 
     if (warp >= 2 && split == 0) {
         // ------------------------------------------------ epilogue: one token row per thread
+        // (with two warps per lane quadrant, each of the row's two threads takes
+        // half of the experts and the halves meet in shared memory)
+        constexpr int HALVES = TH::HALVES, NTH = TH::NTH;
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
         const int tid = threadIdx.x - 64;
         const int64_t t = t0 + r;
@@ -337,10 +358,17 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         float* Ls = reinterpret_cast<float*>(xring);  // logits, then normalised scores
         float* Xs = Ls + BM * LDS;                     // scores: exp(L - max), or sigmoid(L)
         float* Ns = Xs + BM * LDS;                     // this tile's logit noise
+        float* Xc = Ns + BM * LDS;                     // the halves' exchange (two halves only)
+        float* xm = Xc;                                // [BM] row maximum
+        float* xp = Xc + BM;                           // [3][BM] partial sums, then [BM] scale
+        float* xv = Xc + 4 * BM;                       // [BM][KM] the second half's top-K values
+        int* xi = reinterpret_cast<int*>(Xc + (4 + KM) * BM);  // and ids
         const int G = o.n_groups, gsz = E / G;
         const int rows = a.T - t0 < BM ? (int)(a.T - t0) : BM;  // tokens of this tile
+        const int eh = (E + HALVES - 1) / HALVES;               // this thread's experts [e0, e1)
+        const int e0 = half * eh, e1 = e0 + eh < E ? e0 + eh : E;
         // the biases, and the tile's noise rows (one contiguous block, read coalesced)
-        for (int e = tid; e < E; e += 128) {
+        for (int e = tid; e < E; e += NTH) {
             m->bias_s[e] = a.bias ? a.bias[e] : 0.f;
             m->sel_s[e] = o.sel_bias ? o.sel_bias[e] : 0.f;
         }
@@ -348,16 +376,16 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             // eight loads in flight per thread, then their stores
             const float* src = a.noise + t0 * E;
             const int n = rows * E;
-            for (int i0 = 0; i0 < n; i0 += 8 * 128) {
+            for (int i0 = 0; i0 < n; i0 += 8 * NTH) {
                 float v[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + u * 128 + tid;
+                    const int i = i0 + u * NTH + tid;
                     v[u] = i < n ? __ldcs(src + i) : 0.f;
                 }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + u * 128 + tid;
+                    const int i = i0 + u * NTH + tid;
                     if (i < n) {
                         const int rr = i / E;
                         Ns[rr * LDS + (i - rr * E)] = v[u];
@@ -365,7 +393,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 }
             }
         }
-        epi_sync();
+        epi_sync<NTH>();
         // top-K by (u desc, id asc), u = L + selection bias: an unrolled insertion
         // network of KM >= K slots (a displaced entry carried down keeps that order)
         float tv[KM];
@@ -375,14 +403,14 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             tv[k] = -INFINITY;
             ti[k] = 0x7fffffff;
         }
-        auto insert = [&](float xv, int xi) {
+        auto insert = [&](float xv_, int xi_) {
 #pragma unroll
             for (int k = 0; k < KM; ++k) {
-                const bool gt = xv > tv[k] || (xv == tv[k] && xi < ti[k]);
-                const float nv = gt ? xv : tv[k];
-                const int ni = gt ? xi : ti[k];
-                xv = gt ? tv[k] : xv;
-                xi = gt ? ti[k] : xi;
+                const bool gt = xv_ > tv[k] || (xv_ == tv[k] && xi_ < ti[k]);
+                const float nv = gt ? xv_ : tv[k];
+                const int ni = gt ? xi_ : ti[k];
+                xv_ = gt ? tv[k] : xv_;
+                xi_ = gt ? ti[k] : xi_;
                 tv[k] = nv;
                 ti[k] = ni;
             }
@@ -395,33 +423,57 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             for (int sp = 1; sp < a.splits; ++sp) {
                 const float* Pr = recv + ((size_t)(sp - 1) * BM + r) * EPN;
 #pragma unroll 4
-                for (int e = 0; e < E; ++e) Lr[e] += Pr[e];
+                for (int e = e0; e < e1; ++e) Lr[e] += Pr[e];
             }
             if (a.bias) {
 #pragma unroll 4
-                for (int e = 0; e < E; ++e) Lr[e] += m->bias_s[e];
+                for (int e = e0; e < e1; ++e) Lr[e] += m->bias_s[e];
             }
             if (a.noise && valid) {
 #pragma unroll 4
-                for (int e = 0; e < E; ++e) Lr[e] += Ns[r * LDS + e];
+                for (int e = e0; e < e1; ++e) Lr[e] += Ns[r * LDS + e];
             }
         }
         float mx = -INFINITY;
         if (G == 1) {
 #pragma unroll 8
-            for (int e = 0; e < E; ++e) {
+            for (int e = e0; e < e1; ++e) {
                 const float L = Ls[r * LDS + e];
                 mx = fmaxf(mx, L);
                 insert(L + m->sel_s[e], e);
             }
         } else {
 #pragma unroll 8
-            for (int e = 0; e < E; ++e) mx = fmaxf(mx, Ls[r * LDS + e]);
+            for (int e = e0; e < e1; ++e) mx = fmaxf(mx, Ls[r * LDS + e]);
+        }
+        if (HALVES == 2) {
+            // the second half hands its maximum and its top-K to the first
+            if (half == 1) {
+                xm[r] = mx;
+#pragma unroll
+                for (int k = 0; k < KM; ++k) {
+                    xv[r * KM + k] = tv[k];
+                    xi[r * KM + k] = ti[k];
+                }
+            }
+            epi_sync<NTH>();
+            if (half == 0) {
+                mx = fmaxf(mx, xm[r]);
+                if (G == 1) {
+#pragma unroll
+                    for (int k = 0; k < KM; ++k) insert(xv[r * KM + k], xi[r * KM + k]);
+                }
+            }
+            epi_sync<NTH>();
+            if (half == 0) xm[r] = mx;  // the row maximum back to the second half
+            epi_sync<NTH>();
+            if (half == 1) mx = xm[r];
+        } else if (a.logits_out) {
+            epi_sync<NTH>();
         }
         if (a.logits_out) {  // the tile's logits, one contiguous block, written coalesced
-            epi_sync();
             float* dst = a.logits_out + t0 * E;
-            for (int i = tid; i < rows * E; i += 128) {
+            for (int i = tid; i < rows * E; i += NTH) {
                 const int rr = i / E;
                 dst[i] = Ls[rr * LDS + (i - rr * E)];
             }
@@ -430,7 +482,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
         // the scores (sigmoid scores and their sum with score_func sigmoid)
         float ssum = 0.f, s1 = 0.f, scsum = 0.f;
 #pragma unroll 4
-        for (int e = 0; e < E; ++e) {
+        for (int e = e0; e < e1; ++e) {
             const float L = Ls[r * LDS + e];
             const float x = __expf(L - mx);
             ssum += x;
@@ -442,84 +494,108 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
             }
             Xs[r * LDS + e] = sc;
         }
-        const float inv = 1.0f / ssum;
-        const float lss = logf(ssum);
-        // entropy -sum q log q = log(sum) - sum q (L - max), q = exp(L - max) / sum
-        const float ent = lss - s1 * inv;
-        // softmax scores are Xs * inv, sigmoid scores Xs itself
-        const float sc_mul = o.score_func == 1 ? 1.0f : inv;
-        if (G > 1) {
-            // group limit: a group's score is its best selection score u = L + b
-            float gm[32];
-#pragma unroll
-            for (int g = 0; g < 32; ++g) {
-                gm[g] = -INFINITY;
-                if (g < G)
-                    for (int e = g * gsz; e < (g + 1) * gsz; ++e)
-                        gm[g] = fmaxf(gm[g], Ls[r * LDS + e] + m->sel_s[e]);
+        if (HALVES == 2) {
+            if (half == 1) {
+                xp[r] = ssum;
+                xp[BM + r] = s1;
+                xp[2 * BM + r] = scsum;
             }
-            uint32_t keep = 0;
-            for (int rr = 0; rr < o.topk_groups; ++rr) {
-                float bv = -INFINITY;
-                int bg = 0;
-#pragma unroll
-                for (int g = 0; g < 32; ++g)
-                    if (g < G && !((keep >> g) & 1u) && gm[g] > bv) {  // strict: lower group id on ties
-                        bv = gm[g];
-                        bg = g;
-                    }
-                keep |= 1u << bg;
+            epi_sync<NTH>();
+            if (half == 0) {  // the halves' sums, first half first
+                ssum += xp[r];
+                s1 += xp[BM + r];
+                scsum += xp[2 * BM + r];
             }
-            for (int e = 0; e < E; ++e)
-                if ((keep >> (e / gsz)) & 1u) insert(Ls[r * LDS + e] + m->sel_s[e], e);
         }
-        // weights from the scores of the selected experts
-        float sk[KM];
-        float ssel = 0.f;
+        float scinv = 0.f, lss = 0.f, ent = 0.f;
+        if (half == 0) {
+            const float inv = 1.0f / ssum;
+            lss = logf(ssum);
+            // entropy -sum q log q = log(sum) - sum q (L - max), q = exp(L - max) / sum
+            ent = lss - s1 * inv;
+            // softmax scores are Xs * inv, sigmoid scores Xs itself
+            const float sc_mul = o.score_func == 1 ? 1.0f : inv;
+            if (G > 1) {
+                // group limit: a group's score is its best selection score u = L + b
+                float gm[32];
 #pragma unroll
-        for (int k = 0; k < KM; ++k) {
-            sk[k] = k < K ? Xs[r * LDS + ti[k]] * sc_mul : 0.f;
-            ssel += sk[k];
-        }
-        if (valid) {
-#pragma unroll
-            for (int k = 0; k < KM; ++k)
-                if (k < K) {
-                    a.ids[t * K + k] = ti[k];
-                    a.wout[t * K + k] = (o.renorm ? sk[k] / ssel : sk[k]) * o.route_scale;
-                    if (a.with_stats) atomicAdd(&m->cnt[ti[k]], 1);  // integer: order-free
+                for (int g = 0; g < 32; ++g) {
+                    gm[g] = -INFINITY;
+                    if (g < G)
+                        for (int e = g * gsz; e < (g + 1) * gsz; ++e)
+                            gm[g] = fmaxf(gm[g], Ls[r * LDS + e] + m->sel_s[e]);
                 }
+                uint32_t keep = 0;
+                for (int rr = 0; rr < o.topk_groups; ++rr) {
+                    float bv = -INFINITY;
+                    int bg = 0;
+#pragma unroll
+                    for (int g = 0; g < 32; ++g)
+                        if (g < G && !((keep >> g) & 1u) && gm[g] > bv) {  // strict: lower group id on ties
+                            bv = gm[g];
+                            bg = g;
+                        }
+                    keep |= 1u << bg;
+                }
+                for (int e = 0; e < E; ++e)
+                    if ((keep >> (e / gsz)) & 1u) insert(Ls[r * LDS + e] + m->sel_s[e], e);
+            }
+            // weights from the scores of the selected experts
+            float sk[KM];
+            float ssel = 0.f;
+#pragma unroll
+            for (int k = 0; k < KM; ++k) {
+                sk[k] = k < K ? Xs[r * LDS + ti[k]] * sc_mul : 0.f;
+                ssel += sk[k];
+            }
+            if (valid) {
+#pragma unroll
+                for (int k = 0; k < KM; ++k)
+                    if (k < K) {
+                        a.ids[t * K + k] = ti[k];
+                        a.wout[t * K + k] = (o.renorm ? sk[k] / ssel : sk[k]) * o.route_scale;
+                        if (a.with_stats) atomicAdd(&m->cnt[ti[k]], 1);  // integer: order-free
+                    }
+            }
+            scinv = o.score_func == 1 ? 1.0f / scsum : inv;
+        }
+        if (HALVES == 2) {
+            epi_sync<NTH>();  // the second half has read its partial sums
+            if (half == 0) xp[r] = scinv;
+            epi_sync<NTH>();
+            if (half == 1) scinv = xp[r];
         }
         // pass 3: normalised scores into Ls (and probs_out); rows past T give nothing
-        const float scinv = o.score_func == 1 ? 1.0f / scsum : inv;
 #pragma unroll 4
-        for (int e = 0; e < E; ++e) {
+        for (int e = e0; e < e1; ++e) {
             const float pn = Xs[r * LDS + e] * scinv;
             Ls[r * LDS + e] = valid ? pn : 0.f;
         }
         if (a.probs_out) {  // one contiguous block, written coalesced
-            epi_sync();
+            epi_sync<NTH>();
             float* dst = a.probs_out + t0 * E;
-            for (int i = tid; i < rows * E; i += 128) {
+            for (int i = tid; i < rows * E; i += NTH) {
                 const int rr = i / E;
                 dst[i] = Ls[rr * LDS + (i - rr * E)];
             }
         }
         if (a.with_stats) {
             // per-CTA statistics, each in a fixed order
-            const float lse = mx + lss;
-            float z = valid ? lse * lse : 0.f, h = valid ? ent : 0.f;
+            if (half == 0) {
+                const float lse = mx + lss;
+                float z = valid ? lse * lse : 0.f, h = valid ? ent : 0.f;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                z += __shfl_xor_sync(0xffffffffu, z, off);
-                h += __shfl_xor_sync(0xffffffffu, h, off);
+                for (int off = 16; off > 0; off >>= 1) {
+                    z += __shfl_xor_sync(0xffffffffu, z, off);
+                    h += __shfl_xor_sync(0xffffffffu, h, off);
+                }
+                if (lane == 0) {
+                    m->wz[quad] = z;
+                    m->wh[quad] = h;
+                }
             }
-            if (lane == 0) {
-                m->wz[quad] = z;
-                m->wh[quad] = h;
-            }
-            epi_sync();
-            constexpr int CH = 128 / EPN;  // row chunks per column (EPN x CH = 128 threads)
+            epi_sync<NTH>();
+            constexpr int CH = NTH / EPN;  // row chunks per column (EPN x CH = NTH threads)
             constexpr int RC = BM / CH;
             {
                 const int col = tid % EPN, ch = tid / EPN;
@@ -528,7 +604,7 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                     for (int rr = ch * RC; rr < (ch + 1) * RC; ++rr) sp += Ls[rr * LDS + col];
                 m->psum[ch * EPN + col] = sp;
             }
-            epi_sync();
+            epi_sync<NTH>();
             if (tid < E) {
                 float sp = 0.f;
                 for (int ch = 0; ch < CH; ++ch) sp += m->psum[ch * EPN + tid];
@@ -540,19 +616,19 @@ __global__ void __launch_bounds__(NUM_THREADS, MINB)
                 a.blk_ent[blockIdx.x] = ((m->wh[0] + m->wh[1]) + m->wh[2]) + m->wh[3];
             }
             __threadfence();
-            epi_sync();
+            epi_sync<NTH>();
             if (tid == 0) m->last = atomicAdd(a.counter, 1) == (int)gridDim.x - 1;
         }
     }
     tc_fence_before();
     __syncthreads();
     if (split == 0 && a.with_stats && m->last) {
-        // the last CTA: the statistics of the whole grid (all 192 threads)
+        // the last CTA: the statistics of the whole grid (all its threads)
         __threadfence();
         double* sd = reinterpret_cast<double*>(xring);
         long long* sc = reinterpret_cast<long long*>(sd + kStatD);
         finish_router_stats(a.blk_mp, a.blk_z, a.blk_ent, a.blk_cnt, (int)gridDim.x, a.T, E, a.K,
-                            a.mean_prob, a.losses, sd, sc, NUM_THREADS, (int)threadIdx.x,
+                            a.mean_prob, a.losses, sd, sc, TH::NT, (int)threadIdx.x,
                             [] { __syncthreads(); });
         if (threadIdx.x == 0) *a.counter = 0;
     }
@@ -598,18 +674,17 @@ static Plan make_plan(const moe_config& c, bool noise)
     p.epn = epn_of(c.E);
     const int tiles = router_tc_blocks(c);
     const int nkb = (c.D + BK - 1) / BK;
-    p.splits = router_tc_splits(c);
-    p.split_kb = (nkb + p.splits - 1) / p.splits;
     const size_t w_bytes = (size_t)3 * p.epn * 128;
-    const size_t recv = (size_t)(p.splits - 1) * BM * p.epn * sizeof(float);
     const size_t misc = align_up(sizeof(Misc), 1024);
-    const size_t fixed = 1024 + misc + align_up(recv, 1024);
-    // the epilogue scratch (and the statistics' last step) live in the rings
-    const size_t epi = (size_t)(noise ? 3 : 2) * BM * (p.epn + 1) * sizeof(float);
+    // the epilogue scratch (and the statistics' last step) live in the rings:
+    // logits, scores and noise rows ([BM][EPN + 1] fp32 each), and with one CTA
+    // per SM (two epilogue threads per row) the halves' exchange, (4 + 2 KM) x BM words
+    const size_t epi2 = (size_t)(noise ? 3 : 2) * BM * (p.epn + 1) * sizeof(float);
+    const size_t epi1 = ((size_t)3 * BM * (p.epn + 1) + (size_t)(4 + 2 * MAX_KM) * BM) * sizeof(float);
     const size_t fin = (size_t)kStatD * sizeof(double) + (size_t)kStatC * sizeof(long long);
     // the weight ring takes up to about 45 % of the budget (its tiles come from
     // L2: a few in flight cover that latency), the x ring the rest
-    auto fit = [&](size_t budget, int& st, int& ws) {
+    auto fit = [&](size_t budget, size_t fixed, size_t epi, int& st, int& ws) {
         st = ws = 0;
         if (budget <= fixed) return false;
         const size_t room = budget - fixed;
@@ -622,11 +697,24 @@ static Plan make_plan(const moe_config& c, bool noise)
         const size_t rings = (size_t)st * A_BYTES + (size_t)ws * w_bytes;
         return st >= 3 && rings >= epi && rings >= fin;
     };
-    // two CTAs per SM when the tiles outnumber the SMs and each still gets 3 x stages
+    // the d_model split the token tiles ask for, fewer when its partial logits
+    // (received by each tile's leader) leave the rings too little room; one
+    // split always fits (E <= 128)
+    size_t recv = 0;
     int st = 0, ws = 0;
-    p.ctas_per_sm = 1;
-    if (tiles * p.splits > 148 && p.epn <= 64 && fit(112 * 1024, st, ws)) p.ctas_per_sm = 2;
-    else fit(226 * 1024, st, ws);
+    for (int want = router_tc_splits(c); want >= 1; --want) {
+        const int per = (nkb + want - 1) / want;  // K blocks per split: every split non-empty
+        p.splits = (nkb + per - 1) / per;
+        recv = (size_t)(p.splits - 1) * BM * p.epn * sizeof(float);
+        const size_t fixed = 1024 + misc + align_up(recv, 1024);
+        // two CTAs per SM when the tiles outnumber the SMs and each still gets 3 x stages
+        p.ctas_per_sm = 2;
+        if (tiles * p.splits > 148 && p.epn <= 64 && fit(112 * 1024, fixed, epi2, st, ws)) break;
+        p.ctas_per_sm = 1;
+        if (fit(226 * 1024, fixed, epi1, st, ws)) break;
+        st = 0;  // no fit: the launcher rejects fewer than 3 stages (unreachable for E <= 128)
+    }
+    p.split_kb = (nkb + p.splits - 1) / p.splits;
     p.stages = st;
     p.wslots = ws;
     p.w_off = (uint32_t)((size_t)p.stages * A_BYTES);
@@ -648,7 +736,7 @@ static cudaError_t launch_t(const moe_config& c, const CUtensorMap& mX, const CU
     if (ae != cudaSuccess) return ae;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)router_tc_blocks(c), (unsigned)p.splits, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(Threads<MINB>::NT, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
