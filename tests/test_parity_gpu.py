@@ -55,6 +55,9 @@ SMALL = [
     _wl("tcr_ragged", T=2500, D=136, F=64, E=8, K=2, seed=16),
     _wl("tcr_e100", T=2100, D=264, F=64, E=100, K=4, bias="zipf", noise=True, seed=17),
     _wl("tcr_e128_k8", T=2048, D=128, F=32, E=128, K=8, seed=18),
+    # 16 token tiles would split d_model in two, but the leader's receive buffer for
+    # 128 experts leaves the rings too small: the plan falls back to one split
+    _wl("tcr_e128_split_fit", T=2048, D=1024, F=32, E=128, K=4, bias="zipf", seed=61),
     # more token tiles than SMs: two router CTAs per SM (shallower rings)
     _wl("tcr_two_per_sm", T=19200, D=136, F=32, E=24, K=3, noise=True, seed=44),
     _wl("tcr_two_per_sm_e64", T=19000, D=64, F=32, E=64, K=6, bias="zipf", seed=45),
