@@ -25,17 +25,20 @@
 //   warp 0      TMA: the x tiles (128 tokens x 64 of d_model, 128-byte
 //               swizzle) into a deep ring (up to 10 stages of 16 KB)
 //   warp 1      tcgen05.mma
-//   warps 2..5  lane 0 of warp 2: TMA of the weight terms of each K block
+//   warps 2..   lane 0 of warp 2: TMA of the weight terms of each K block
 //               (3 x EPN rows x 64 of d_model, 128-byte swizzle) into a ring
-//               of their own, so that the x ring keeps its depth; then all
-//               four warps run the epilogue, one token row per thread:
-//               logits (+ bias + noise), max and top-K by (logit +
-//               selection bias desc, id asc, an unrolled insertion network)
-//               in one pass over the experts, softmax sum and entropy
-//               (closed form) and scores in a second, the group limit when
-//               set, weights, normalised scores in a third, and the per-CTA
-//               statistics (counts by shared-memory atomics; column sums
-//               in a fixed order).
+//               of their own, so that the x ring keeps its depth.  Warps 2..5
+//               read the accumulators out of tensor memory (each its lane
+//               quadrant).  Then the epilogue: four warps with two CTAs per
+//               SM (one token row per thread), eight with one CTA per SM (a
+//               token's two threads take half of the experts each and meet
+//               in shared memory): logits (+ partials of the other splits +
+//               bias + noise), max and top-K by (logit + selection bias
+//               desc, id asc, an unrolled insertion network), softmax sum
+//               and entropy (closed form) and scores, the group limit when
+//               set, weights, normalised scores, and the per-CTA statistics
+//               (counts by shared-memory atomics; column sums in a fixed
+//               order).
 // When the token tiles alone leave most SMs idle, d_model is split over a
 // cluster of CTAs along grid y: each non-leader CTA sends its partial logits
 // to the leader's shared memory (distributed shared memory), and the leader
