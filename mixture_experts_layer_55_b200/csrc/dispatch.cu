@@ -67,11 +67,22 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __res
     const int e = threadIdx.x;
     int32_t kp = 0;
     if (e < E) {
+        // sixteen loads in flight at a time (clamped indices), bases in chunk order
         int64_t run = 0;
-        for (int64_t b = 0; b < nchunks; ++b) {
-            int32_t v = blk_cnt[b * E + e];
-            blk_base[b * E + e] = (int32_t)run;
-            run += v;
+        for (int64_t b0 = 0; b0 < nchunks; b0 += 16) {
+            int32_t v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int64_t b = b0 + u < nchunks ? b0 + u : nchunks - 1;
+                v[u] = blk_cnt[b * E + e];
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                if (b0 + u < nchunks) {
+                    blk_base[(b0 + u) * E + e] = (int32_t)run;
+                    run += v[u];
+                }
+            }
         }
         counts[e] = (int32_t)run;
         kp = (int32_t)(run < C ? run : C);
@@ -261,10 +272,23 @@ __global__ void __launch_bounds__(256) dispatch_index_kernel(
         const int e = threadIdx.x;
         int32_t kp = 0;
         if (e < E) {
+            // every chunk's count of expert e, sixteen loads in flight at a time
+            // (issued unconditionally at clamped indices), added in chunk order
             int64_t run = 0, mine = 0;
-            for (int b = 0; b < nch; ++b) {
-                if (b == (int)blockIdx.x) mine = run;
-                run += __ldcg(blk_cnt + (size_t)b * E + e);
+            for (int b0 = 0; b0 < nch; b0 += 16) {
+                int32_t v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int b = b0 + u < nch ? b0 + u : nch - 1;
+                    v[u] = __ldcg(blk_cnt + (size_t)b * E + e);
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    if (b0 + u < nch) {
+                        if (b0 + u == (int)blockIdx.x) mine = run;
+                        run += v[u];
+                    }
+                }
             }
             s_base[e] = (int32_t)mine;
             kp = (int32_t)(run < C ? run : C);
