@@ -58,7 +58,7 @@ typedef enum moe_status {
     MOE_OK = 0,
     MOE_ERR_ARG = -1,            /* K outside [1, min(E, 8)], E > 256, a NULL required pointer, a bad enum */
     MOE_ERR_SHAPE = -2,          /* T, D, F or E below 1, or T*K beyond 2^31 - 1 */
-    MOE_ERR_UNSUPPORTED = -3,    /* an option this build does not implement */
+    MOE_ERR_UNSUPPORTED = -3,    /* an option this library does not implement */
     MOE_ERR_ALIGN = -4,          /* D or F not a multiple of 8, or a buffer not 16-byte aligned */
     MOE_ERR_CUDA = -5,           /* a CUDA runtime call failed */
     MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel gave up a bounded wait (device status) */
