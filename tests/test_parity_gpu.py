@@ -209,6 +209,61 @@ def test_unaligned_router_weight(cuda_ok):
     check_routing(wl, b)
 
 
+def _split3_cpu(w):
+    """The three bf16 terms of fp32 weights, as the pages' fp32 logits need them
+    written exactly: hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid),
+    each rounded to nearest even (torch's float -> bfloat16 conversion)."""
+    hi = w.bfloat16()
+    r = w - hi.float()
+    mid = r.bfloat16()
+    lo = (r - mid.float()).bfloat16()
+    return hi, mid, lo
+
+
+@pytest.mark.parametrize("E", [8, 24, 100])
+def test_router_prepare_writes_the_exact_terms(cuda_ok, E):
+    """moe_router_prepare: terms[p][e][d] (p = hi, mid, lo; e < E16, rows past E
+    zero) equal the exact three-term split of W_r computed on the CPU, bit for bit."""
+    D = 200
+    cfg = B.MoeConfig.make(4096, D, 64, E, 2, "bf16")
+    g = torch.Generator().manual_seed(E)
+    w = torch.randn(D, E, generator=g) * 0.02
+    w[0, 0] = 1.0 + 2.0 ** -9 + 2.0 ** -18  # a value whose split needs all three terms
+    terms = torch.empty(B.router_terms_size(cfg), dtype=torch.uint8, device="cuda")
+    B.moe_router_prepare(cfg, w.cuda(), terms)
+    torch.cuda.synchronize()
+    e16 = B.router_terms_size(cfg) // (3 * D * 2)
+    assert e16 >= E and e16 in (16, 32, 64, 128)
+    got = terms.view(torch.bfloat16).view(3, e16, D).cpu()
+    for p, ref in enumerate(_split3_cpu(w)):
+        assert torch.equal(got[p, :E].view(torch.int16), ref.t().contiguous().view(torch.int16)), p
+        assert (got[p, E:].view(torch.int16) == 0).all()
+    # the three terms add up to the weight exactly (24 significand bits in 3 x 8)
+    s = got[0, :E].double() + got[1, :E].double() + got[2, :E].double()
+    assert torch.equal(s, w.t().double())
+
+
+def test_layer_prepares_the_router_terms_again_after_an_update(cuda_ok):
+    """MoELayer splits w_router once; after the weight is changed in place (its
+    version counter moves) or replaced, the next forward uses the new terms: the
+    same bits as a layer built on the new weight."""
+    from mixture_experts_layer_55_b200 import MoELayer
+    wl = _wl("terms_refresh", T=2304, D=128, F=64, E=16, K=2, seed=62)
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    layer = MoELayer(wl.T, inp["w_router"].clone(), inp["w_gate"], inp["w_up"], inp["w_down"], wl.K)
+    x = inp["x"]
+    y0 = layer.forward(x).clone()
+    layer.w_router.mul_(-1.5)  # in place: new routing
+    y1 = layer.forward(x).clone()
+    ref = MoELayer(wl.T, inp["w_router"] * -1.5, inp["w_gate"], inp["w_up"], inp["w_down"], wl.K)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, ref.forward(x))
+    assert not torch.equal(y0, y1)
+    layer.w_router = inp["w_router"].clone()  # replaced: back to the first routing
+    assert torch.equal(layer.forward(x), y0)
+    assert B.moe_get_device_status(layer.workspace) == 0
+
+
 def test_dispatch_index_three_kernel_path(cuda_ok):
     """More chunks of 2048 assignments than SMs (T*K = 320000): the index pass
     runs as three kernels instead of one cooperative launch; routing, counts,
