@@ -67,11 +67,26 @@ class CudaOps:
         self.src_of = torch.empty(self.max_recv, **i32)
         self.remote_row = None  # peer exchange: row of each slot in its owner's buffer
         self.h_local = None     # peer exchange: the local experts' hidden activations
+        # the router weight's bf16 terms (moe_router_prepare), split again when the
+        # weight is replaced or changed in place (its version counter)
+        nb = B.router_terms_size(self.cfg)
+        self.router_terms = torch.empty(nb, dtype=torch.uint8, device=device) if nb else None
+        self._terms_of = None
+
+    def _terms(self, w_router):
+        if self.router_terms is None:
+            return None
+        key = (id(w_router), w_router.data_ptr(), w_router._version)
+        if key != self._terms_of:
+            B.moe_router_prepare(self.cfg, w_router, self.router_terms)
+            self._terms_of = key
+        return self.router_terms
 
     def route_dispatch(self, x, w_router, router_bias, selection_bias, logit_noise):
         x_perm = torch.empty((self.max_rows, x.shape[1]), dtype=x.dtype, device=x.device)
         B.moe_route(self.cfg, x, w_router, self.ids, self.w, self.ws, router_bias=router_bias,
-                    logit_noise=logit_noise, selection_bias=selection_bias)
+                    logit_noise=logit_noise, selection_bias=selection_bias,
+                    w_router_terms=self._terms(w_router))
         B.moe_dispatch(self.cfg, x, self.ids, self.counts, self.kept, self.offsets, self.perm,
                        self.row_of, x_perm, self.ws)
         return self.kept, self.offsets, x_perm
@@ -117,7 +132,8 @@ class CudaOps:
 
     def route_index(self, x, w_router, router_bias, selection_bias, logit_noise):
         B.moe_route(self.cfg, x, w_router, self.ids, self.w, self.ws, router_bias=router_bias,
-                    logit_noise=logit_noise, selection_bias=selection_bias)
+                    logit_noise=logit_noise, selection_bias=selection_bias,
+                    w_router_terms=self._terms(w_router))
         B.moe_dispatch(self.cfg, None, self.ids, self.counts, self.kept, self.offsets, self.perm,
                        self.row_of, None, self.ws)
         return self.kept
