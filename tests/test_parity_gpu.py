@@ -264,6 +264,65 @@ def test_layer_prepares_the_router_terms_again_after_an_update(cuda_ok):
     assert B.moe_get_device_status(layer.workspace) == 0
 
 
+def _random_router_cases(n=20, seed=2024):
+    """Seeded random shapes for the tensor-core router (bf16, T >= 2048, E <= 128):
+    any E (so E16 = 16, 32, 64 or 128 and ragged expert rows), d_model splits or
+    none, one or two CTAs per SM, and the options (bias, noise, sigmoid scores,
+    no renormalisation, selection bias, group limit)."""
+    import random
+    rng = random.Random(seed)
+    cases = []
+    while len(cases) < n:
+        E = rng.choice([1, 3, 8, 13, 16, 24, 33, 50, 64, 77, 100, 128])
+        K = rng.randint(1, min(E, 8))
+        T = rng.choice([2048, 2049, 3000, 5000, 9000, 19000])
+        D = rng.choice([64, 136, 264, 520, 1032, 2056])
+        if T * D * E > 1_500_000_000:
+            continue
+        kw = dict(T=T, D=D, F=32, E=E, K=K, seed=300 + len(cases))
+        if rng.random() < 0.4:
+            kw["bias"] = "zipf"
+        if rng.random() < 0.4:
+            kw["noise"] = True
+        if rng.random() < 0.3:
+            kw["score_func"] = "sigmoid"
+        if rng.random() < 0.3:
+            kw["renormalize"] = False
+        if rng.random() < 0.3:
+            kw["sel_bias"] = True
+        groups = [g for g in (2, 4, 8) if E % g == 0 and E // g >= 1]
+        if groups and rng.random() < 0.3:
+            g = rng.choice(groups)
+            tg = rng.randint(1, g)
+            if tg * (E // g) >= K:
+                kw["n_groups"], kw["topk_groups"] = g, tg
+        name = "rand_" + "_".join(f"{k}{v}" for k, v in kw.items() if k not in ("F", "seed"))
+        cases.append(_wl(name, **kw))
+    return cases
+
+
+RANDOM_ROUTER = _random_router_cases() + [
+    _wl("rand_T2048_D64_E1_K1", T=2048, D=64, F=32, E=1, K=1, seed=330),
+    _wl("rand_T2100_D136_E3_K3_noise_sigmoid", T=2100, D=136, F=32, E=3, K=3, noise=True,
+        score_func="sigmoid", seed=331),
+]
+
+
+@pytest.mark.parametrize("wl", RANDOM_ROUTER, ids=[w.name for w in RANDOM_ROUTER])
+def test_tensor_core_router_random_shapes(cuda_ok, wl):
+    """Logits within the fp32 bound and every routing output bit-exact (ids,
+    weights and probabilities within 1e-5, statistics, counts) against the
+    oracle, over seeded random shapes and options of the tensor-core router."""
+    assert B.check_config(B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K, wl.dtype,
+                                           wl.capacity_factor, **wl.routing())) == B.MOE_OK
+    inp_cpu = make_inputs(wl, device="cpu")
+    inp = _to_dev(inp_cpu)
+    b = Bufs(wl)
+    b.run_ops(inp)
+    check_logits(wl, inp_cpu, b.logits.cpu().numpy())
+    check_routing(wl, b, inp["sel_bias"])
+
+
 def test_dispatch_index_three_kernel_path(cuda_ok):
     """More chunks of 2048 assignments than SMs (T*K = 320000): the index pass
     runs as three kernels instead of one cooperative launch; routing, counts,
