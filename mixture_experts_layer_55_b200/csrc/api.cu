@@ -129,6 +129,9 @@ BwdLayout bwd_layout(const moe_config& c, int64_t max_rows)
         B.sh_dgu = o; o += align_up((size_t)c.T * 2 * c.F_shared * es);
         B.sh_dx = o;  o += align_up((size_t)c.T * c.D * es);
     }
+    // two launches (dWd, then [dWg | dWu]) of E experts each, one slot apiece
+    B.tmaps = o;    o += c.dtype == MOE_BF16 ? 2 * align_up(wgrad_maps_bytes(c.E)) : 0;
+    B.tmaps_sh = o; o += c.dtype == MOE_BF16 && c.F_shared > 0 ? 2 * align_up(wgrad_maps_bytes(1)) : 0;
     B.total = o;
     return B;
 }
@@ -225,12 +228,12 @@ static cudaError_t launch_dgrad(const moe_config& c, int64_t max_rows, const voi
 }
 
 static cudaError_t launch_wgrad(int32_t dt, int E, int64_t max_rows, const int32_t* offsets, const void* a,
-                                int M, const void* b, int N, int halves, float* out0, float* out1, int* status,
-                                cudaStream_t s)
+                                int M, const void* b, int N, int halves, float* out0, float* out1, void* maps,
+                                int* status, cudaStream_t s)
 {
     if (dt == MOE_F32)
         return launch_wgrad_simt_f32(E, max_rows, offsets, a, M, b, N, halves, out0, out1, status, s);
-    return launch_wgrad_tc_bf16(E, max_rows, offsets, a, M, b, N, halves, out0, out1, status, s);
+    return launch_wgrad_tc_bf16(E, max_rows, offsets, a, M, b, N, halves, out0, out1, maps, status, s);
 }
 
 // the shared expert as a layer of one expert over every token
@@ -566,7 +569,7 @@ moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes)
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (bytes == nullptr) return MOE_ERR_ARG;
-        *bytes = bwd_layout(*cfg, max_rows_of(*cfg)).total;
+    *bytes = bwd_layout(*cfg, max_rows_of(*cfg)).total;
     return MOE_OK;
 }
 
@@ -582,7 +585,7 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
     moe_status st = check_forward_args(cfg, x, w_router, w_gate, w_up, w_down, w_gate_shared,
                                        w_up_shared, w_down_shared, dx);
     if (st != MOE_OK) return st;
-        if (!dy || !dw_router || !dw_gate || !dw_up || !dw_down) return MOE_ERR_ARG;
+    if (!dy || !dw_router || !dw_gate || !dw_up || !dw_down) return MOE_ERR_ARG;
     if (!aligned16(dy) || !aligned16(dw_gate) || !aligned16(dw_up) || !aligned16(dw_down))
         return MOE_ERR_ALIGN;
     if (cfg->F_shared > 0) {
@@ -628,11 +631,11 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
     btrace(4, s);
     if (e == cudaSuccess)  // dWd = h^T dYp
         e = launch_wgrad(c.dtype, c.E, max_rows, offsets, sv + F.h, c.F, ws + B.dyp, c.D, 1, dw_down,
-                                 nullptr, status, s);
+                         nullptr, ws + B.tmaps, status, s);
     btrace(5, s);
     if (e == cudaSuccess)  // [dWg | dWu] = x_perm^T [dg | du]
         e = launch_wgrad(c.dtype, c.E, max_rows, offsets, sv + F.x_perm, c.D, ws + B.dgu, c.F, 2,
-                                 dw_gate, dw_up, status, s);
+                         dw_gate, dw_up, ws + B.tmaps + align_up(wgrad_maps_bytes(c.E)), status, s);
     btrace(6, s);
     const void* dx_shared = nullptr;
     if (e == cudaSuccess && c.F_shared > 0) {
@@ -643,10 +646,11 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
                                  nullptr);
         if (e == cudaSuccess)
             e = launch_wgrad(c.dtype, 1, c.T, sh_off, sv + F.sh_h, c.F_shared, dy, c.D, 1,
-                                     dw_down_shared, nullptr, status, s);
+                             dw_down_shared, nullptr, ws + B.tmaps_sh, status, s);
         if (e == cudaSuccess)
             e = launch_wgrad(c.dtype, 1, c.T, sh_off, x, c.D, ws + B.sh_dgu, c.F_shared, 2,
-                                     dw_gate_shared, dw_up_shared, status, s);
+                             dw_gate_shared, dw_up_shared, ws + B.tmaps_sh + align_up(wgrad_maps_bytes(1)),
+                             status, s);
         dx_shared = ws + B.sh_dx;
     }
     btrace(7, s);
@@ -849,8 +853,10 @@ int32_t moe_backward_kernel_count(const moe_config* cfg)
     if (check_config(cfg) != MOE_OK) return 0;
     // rows, router, two dgrad GEMMs, two wgrad GEMMs, router weight partials,
     // their sum, the bias gradient, dx; the shared expert adds its two dgrad
-    // and two wgrad GEMMs
-    return 10 + (cfg->F_shared > 0 ? 4 : 0);
+    // and two wgrad GEMMs.  In bf16 layers each wgrad GEMM is preceded by the
+    // kernel that writes its experts' operand maps.
+    const int maps = cfg->dtype == MOE_BF16 ? 1 : 0;
+    return 10 + 2 * maps + (cfg->F_shared > 0 ? 4 + 2 * maps : 0);
 }
 
 moe_status moe_trace_attach_backward(void* const* events, int32_t n_events)

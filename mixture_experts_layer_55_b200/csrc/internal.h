@@ -130,6 +130,8 @@ struct BwdLayout {
     size_t db_scratch;  // (E) fp32: the bias gradient when the caller wants none
     size_t sh_dgu;      // (T, 2 F_shared)
     size_t sh_dx;       // (T, D)
+    size_t tmaps;       // the weight-gradient GEMMs' per-expert tensor maps (bf16 layers)
+    size_t tmaps_sh;    // and the shared expert's
     int rw_splits;
     size_t total;
 };
@@ -201,9 +203,12 @@ cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const vo
                                  const void* w_up, const void* w_down, void* dgu, void* dxp,
                                  int* status, cudaStream_t s, StageHook mid, void* mid_ctx);
 // out0 / out1 (E, M, Nh) fp32 = A[block]^T . B[block] per expert block.
+// `maps`: device scratch of wgrad_maps_bytes(E) bytes, 128-byte aligned,
+// rewritten by the launch (each expert's operand tensor maps).
+size_t wgrad_maps_bytes(int E);
 cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets, const void* A,
                                  int M, const void* B, int Nh, int halves, float* out0, float* out1,
-                                 int* status, cudaStream_t s);
+                                 void* maps, int* status, cudaStream_t s);
 cudaError_t launch_bwd_rows(const moe_config& c, const void* dy, const void* o, const int32_t* offsets,
                             const int32_t* perm, const float* topk_w, void* dyp, float* dw_row,
                             int64_t max_rows, int* status, cudaStream_t s);

@@ -12,19 +12,24 @@
 //
 // Both operands are row blocks of row-major (rows, M) and (rows, N) matrices,
 // so both are read MN-major (128-byte swizzle, 64-column boxes); K is the
-// expert's row count, ragged.  A K block that runs past the expert's last row
-// reads the next expert's rows: the MMA warp zeroes those rows of the stage in
-// shared memory before issuing (an expert with no rows writes zeros).  The
-// result is stored in fp32 (the precision weight gradients are accumulated in).
+// expert's row count, ragged.  Each expert reads its operands through its own
+// pair of tensor maps, whose row extent ends at the expert's last row: a K
+// block that runs past it arrives with those rows zero-filled by the copy
+// engine, so nothing has to be fixed up in shared memory before the MMAs.  A
+// small kernel writes the maps before each launch (a host-encoded template,
+// its row extent replaced on the device from the row offsets, which stay on
+// the device).  An expert with no rows writes zeros.  The result is stored in
+// fp32 (the precision weight gradients are accumulated in).
 //
 // Persistent kernel, one CTA per SM, tiles M = 128 x N = 256, 4-stage ring of
-// 48 KB, double-buffered 2 x 256-column accumulators.  11 warps: warp 0 TMA,
-// warp 1 MMA (one thread), warps 2..9 epilogue, warp 10 the tail fixer.  The
-// epilogue stages each warp's 32 x 32 fp32 pieces in shared memory (128-byte
-// swizzle, conflict-free) and writes them with TMA tensor stores over an
-// (E, M, N) map, so the stores are whole lines and the map clips the tile's
-// edges per expert.  (Measured: six operand stages with one staging buffer per
-// warp beat five stages with two.)  Every wait is bounded (device status flag).
+// 48 KB, double-buffered 2 x 256-column accumulators.  10 warps: warp 0 TMA,
+// warp 1 MMA (one thread), warps 2..9 epilogue.  The epilogue stages each
+// warp's 32 x 32 fp32 pieces in shared memory (128-byte swizzle, conflict-free)
+// and writes them with TMA tensor stores over an (E, M, N) map, so the stores
+// are whole lines and the map clips the tile's edges per expert.  (Measured:
+// six operand stages with one staging buffer per warp beat five stages with
+// two; the zero-filling maps beat zeroing the tail rows in shared memory from
+// a dedicated warp by 7-8 %.)  Every wait is bounded (device status flag).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -41,9 +46,8 @@ constexpr int OUT_BYTES = 32 * 32 * 4;  // one staged 32 x 32 fp32 piece
 constexpr int OUT_BUFS = 1;             // staged pieces per epilogue warp
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_THREADS = 352;  // warp 0 TMA, 1 MMA, 2..9 epilogue, 10 tail fixer
+constexpr int NUM_THREADS = 320;  // warp 0 TMA, 1 MMA, 2..9 epilogue
 constexpr int EPI_WARPS = 8;
-constexpr int FIX_WARP = 2 + EPI_WARPS;
 constexpr int MAX_E = 256;
 
 // Single CTA: M = 128 output rows, all 256 columns in this CTA (2 A + 4 B
@@ -63,8 +67,6 @@ template <bool PAIR> struct Geo {
 struct Misc {
     uint64_t full[6];
     uint64_t empty[6];
-    uint64_t pfull[6];  // a partial block's copies have landed (leader; the fixer waits)
-    uint64_t fixed[6];  // a partial block's tail rows are zeroed (leader; the MMA warp waits)
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -82,6 +84,7 @@ static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "sh
 
 struct Args {
     const int32_t* offsets;  // (E + 1) row offsets of the experts' blocks
+    const CUtensorMap* maps; // 2 per expert (A, B): the operands' maps, rows ending at the expert's end
     int E;
     int M;                   // output rows (A's columns)
     int Nh;                  // output columns per half
@@ -115,17 +118,51 @@ MOE_DEVICE void decode(const Args& a, int bm, int t, int& e, int& m0, int& hf, i
     n0 = (j - hf * a.nth) * BN;
 }
 
-MOE_DEVICE void fence_proxy_async_cluster() { asm volatile("fence.proxy.async.shared::cluster;" ::: "memory"); }
-
-MOE_DEVICE void st_cluster_zero16(uint32_t cluster_addr)
+// A tensor map in global memory, rewritten by the generic proxy: its row
+// extent (dimension 1; dimension 0 is the contiguous one) is replaced in place;
+// the writer releases the maps to the copy engine's view, each reader acquires
+// the one it is about to use (which also drops a stale cached copy of it).
+MOE_DEVICE void tmap_set_rows(CUtensorMap* gmap, uint32_t rows)
 {
-    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(cluster_addr), "r"(0) : "memory");
+    asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(gmap), "r"(rows)
+                 : "memory");
+}
+
+MOE_DEVICE void tmap_release() { asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory"); }
+
+MOE_DEVICE void tmap_acquire(const CUtensorMap* gmap)
+{
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
+}
+
+// maps[2e], maps[2e+1] = the A and B templates with the row extent cut to
+// expert e's end (offsets[e+1], clamped to 1 .. max_rows: a malformed offset
+// can only shorten the rows a map reaches, never extend them past the
+// matrices).  One thread per expert.
+__global__ void wgrad_maps_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                  const int32_t* offsets, int E, int64_t max_rows, CUtensorMap* maps)
+{
+    const int e = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    if (e >= E) return;
+    int64_t r1 = offsets[e + 1];
+    r1 = r1 < 1 ? 1 : (r1 > max_rows ? max_rows : r1);
+    const uint4* srcA = reinterpret_cast<const uint4*>(&tmA);
+    const uint4* srcB = reinterpret_cast<const uint4*>(&tmB);
+    uint4* dA = reinterpret_cast<uint4*>(&maps[2 * e]);
+    uint4* dB = reinterpret_cast<uint4*>(&maps[2 * e + 1]);
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(CUtensorMap) / sizeof(uint4)); ++i) {
+        dA[i] = srcA[i];
+        dB[i] = srcB[i];
+    }
+    tmap_set_rows(&maps[2 * e], (uint32_t)r1);
+    tmap_set_rows(&maps[2 * e + 1], (uint32_t)r1);
+    tmap_release();
 }
 
 template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
+    wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                     const Args a)
 {
     using G = Geo<PAIR>;
@@ -146,8 +183,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&m->full[s], 1);
             mbar_init(&m->empty[s], 1);
-            mbar_init(&m->pfull[s], 1);
-            mbar_init(&m->fixed[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&m->tfull[b], 1);
@@ -156,8 +191,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_init(&m->drain, 1);
         m->abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
         prefetch_tmap(&tmO0);
         if (a.halves == 2) prefetch_tmap(&tmO1);
     }
@@ -196,20 +229,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer (each CTA)
-        // A block whose last 16-row step is partial completes on pfull[] (the
-        // fixer zeroes its tail before the MMA warp sees it), every other block
-        // on full[]; each barrier's phases are tracked per stage.
         int stage = 0;
-        uint32_t phase = 0;                 // of empty[]: every block passes through it
-        uint32_t fullph = 0, pfullph = 0;   // per-stage parity of the next full[] / pfull[] phase
-        int last_bar[STAGES];               // per stage: -1 unused, 0 full, 1 pfull
-        uint32_t last_par[STAGES];
-        for (int s = 0; s < STAGES; ++s) last_bar[s] = -1;
+        uint32_t phase = 0;       // of the ring: a stage's n-th use is its full[] phase n
+        int last_par[STAGES];     // per stage: the parity of its last issued phase, -1 unused
+        for (int s = 0; s < STAGES; ++s) last_par[s] = -1;
         bool ok = true;
+        int last_e = -1;
         for (int t = unit; t < total && ok; t += units) {
             int e, m0, hf, n0;
             decode(a, BM, t, e, m0, hf, n0);
             const int r0 = m->off[e], r1 = m->off[e + 1];
+            const CUtensorMap* mA = a.maps + 2 * e;
+            const CUtensorMap* mB = mA + 1;
+            if (e != last_e && r1 > r0) {  // the expert's maps, as the maps kernel wrote them
+                tmap_acquire(mA);
+                tmap_acquire(mB);
+                last_e = e;
+            }
             const int acol = m0 + 128 * (int)rank;                           // this CTA's A columns
             const int bcol = hf * a.Nh + n0 + (PAIR ? 128 * (int)rank : 0);  // and B columns
             for (int k = r0; k < r1; k += BK) {
@@ -217,31 +253,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ok = false;
                     break;
                 }
-                const int valid = r1 - k < BK ? r1 - k : BK;
-                const bool partial = (valid % UK) != 0;
-                uint64_t* bar = partial ? &m->pfull[stage] : &m->full[stage];
-                last_bar[stage] = partial ? 1 : 0;
-                last_par[stage] = ((partial ? pfullph : fullph) >> stage) & 1u;
-                if (partial) pfullph ^= 1u << stage;
-                else fullph ^= 1u << stage;
+                uint64_t* bar = &m->full[stage];
+                last_par[stage] = (int)phase;
                 uint8_t* sA = stages + (size_t)stage * STAGE_BYTES;
                 uint8_t* sB = sA + G::A_BYTES;
+                // rows past the expert's end (and past the matrices) arrive as
+                // zeros; the box's full size is counted either way
                 if (PAIR) {
                     // both CTAs' bytes are counted on the leader's barrier
                     if (rank == 0) mbar_arrive_expect_tx(bar, 2 * STAGE_BYTES);
                     const uint32_t fb = mapa_shared(smem_u32(bar), 0);
 #pragma unroll
                     for (int j = 0; j < G::A_BOXES; ++j)
-                        tma_load_2d_pair(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, fb);
+                        tma_load_2d_pair(sA + j * BOX_BYTES, mA, acol + 64 * j, k, fb);
 #pragma unroll
                     for (int j = 0; j < G::B_BOXES; ++j)
-                        tma_load_2d_pair(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, fb);
+                        tma_load_2d_pair(sB + j * BOX_BYTES, mB, bcol + 64 * j, k, fb);
                 } else {
                     mbar_arrive_expect_tx(bar, STAGE_BYTES);
 #pragma unroll
-                    for (int j = 0; j < G::A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, &tmA, acol + 64 * j, k, bar);
+                    for (int j = 0; j < G::A_BOXES; ++j) tma_load_2d(sA + j * BOX_BYTES, mA, acol + 64 * j, k, bar);
 #pragma unroll
-                    for (int j = 0; j < G::B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, &tmB, bcol + 64 * j, k, bar);
+                    for (int j = 0; j < G::B_BOXES; ++j) tma_load_2d(sB + j * BOX_BYTES, mB, bcol + 64 * j, k, bar);
                 }
                 if (++stage == STAGES) {
                     stage = 0;
@@ -252,18 +285,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // never leave the CTA with a copy in flight (the leader sees every completion)
         if (!PAIR || rank == 0)
             for (int s = 0; s < STAGES; ++s)
-                if (last_bar[s] >= 0)
-                    mbar_wait(last_bar[s] ? &m->pfull[s] : &m->full[s], last_par[s], a.status, 511, nullptr);
+                if (last_par[s] >= 0) mbar_wait(&m->full[s], (uint32_t)last_par[s], a.status, 511, nullptr);
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ---------------------------------------- MMA issuer (leader; one thread)
         // A and B MN-major: 64-column boxes 8 KB apart (LBO), 8-row K groups
         // 1024 B apart (SBO), +2048 B per 16-row K step
         constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, 1, 1);
         int stage = 0;
+        uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        uint32_t fph = 0;     // per-stage parity of the next fixed[] phase
-        uint32_t fullph = 0;  // and of the next full[] phase
         bool ok = true;
         for (int t = unit; t < total && ok; t += units) {
             int e, m0, hf, n0;
@@ -273,21 +304,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * ACC_COLS);
             for (int k = r0; k < r1; k += BK) {
-                // rows of this block that belong to the expert; steps past the
-                // expert's last row are not issued, and a partial step's tail rows
-                // (the next expert's, or rows past the written ones) are zeroed by
-                // the fixer warp first: then this thread waits on fixed[] instead
+                // rows of this block that belong to the expert; steps wholly past
+                // the expert's last row are not issued (a partial step's tail rows
+                // arrived as zeros)
                 const int valid = r1 - k < BK ? r1 - k : BK;
-                const int nsteps = (valid + UK - 1) / UK, rem = valid % UK;
-                bool got;
-                if (rem != 0) {
-                    got = mbar_wait(&m->fixed[stage], (fph >> stage) & 1u, a.status, 523, abort_flag);
-                    fph ^= 1u << stage;
-                } else {
-                    got = mbar_wait(&m->full[stage], (fullph >> stage) & 1u, a.status, 521, abort_flag);
-                    fullph ^= 1u << stage;
-                }
-                if (!got) {
+                const int nsteps = (valid + UK - 1) / UK;
+                if (!mbar_wait(&m->full[stage], phase, a.status, 521, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -306,7 +328,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // frees the stage (in both CTAs) once these MMAs complete
                 if (PAIR) umma_commit_pair_mc(&m->empty[stage], 0x3);
                 else umma_commit(&m->empty[stage]);
-                if (++stage == STAGES) stage = 0;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
             if (!ok) break;
             // accumulator ready for the epilogue (of both CTAs); with no rows: at once
@@ -321,53 +346,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (PAIR) umma_commit_pair_mc(&m->drain, 0x1);
         else umma_commit(&m->drain);
         mbar_wait(&m->drain, 0, a.status, 522, nullptr);
-    } else if (warp == FIX_WARP && rank == 0) {
-        // ------------------------------------ tail fixer (leader; whole warp)
-        // Walks the MMA warp's schedule; for each partial block, once every copy
-        // of the stage has landed (pfull[] counts both CTAs' bytes), it
-        // zeroes the partial step's tail rows in every box of the stage, in both
-        // CTAs of a pair (the peer's through its shared::cluster address), makes
-        // the writes visible to the tensor cores, and signals fixed[].  It runs
-        // ahead of the MMA warp, so the zeroing is off the MMA issue path.
-        int stage = 0;
-        uint32_t pfullph = 0;  // per-stage parity of the next pfull[] phase
-        bool ok = true;
-        for (int t = unit; t < total && ok; t += units) {
-            int e, m0, hf, n0;
-            decode(a, BM, t, e, m0, hf, n0);
-            const int r0 = m->off[e], r1 = m->off[e + 1];
-            for (int k = r0; k < r1; k += BK) {
-                const int valid = r1 - k < BK ? r1 - k : BK;
-                const int nsteps = (valid + UK - 1) / UK, rem = valid % UK;
-                if (rem != 0) {
-                    // only partial blocks advance pfull[stage], and the next one
-                    // cannot land before the MMA warp has used this one (which
-                    // waits for fixed[]): each wait is on the very next phase
-                    const bool got = mbar_wait(&m->pfull[stage], (pfullph >> stage) & 1u, a.status, 540,
-                                               abort_flag);
-                    pfullph ^= 1u << stage;
-                    if (!__all_sync(0xffffffffu, got)) {
-                        ok = false;
-                        break;
-                    }
-                    const int n16 = (UK - rem) * 8;  // 16-byte words per box
-                    const uint32_t base = smem_u32(stages + (size_t)stage * STAGE_BYTES) +
-                                          (uint32_t)(((nsteps - 1) * UK + rem) * 128);
-#pragma unroll 1
-                    for (uint32_t cta = 0; cta < (uint32_t)G::CTAS; ++cta) {
-                        const uint32_t cbase = PAIR ? mapa_shared(base, cta) : base;
-#pragma unroll 1
-                        for (int bx = 0; bx < G::A_BOXES + G::B_BOXES; ++bx)
-                            for (int i = lane; i < n16; i += 32)
-                                st_cluster_zero16(cbase + (uint32_t)(bx * BOX_BYTES + i * 16));
-                    }
-                    fence_proxy_async_cluster();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&m->fixed[stage]);
-                }
-                if (++stage == STAGES) stage = 0;
-            }
-        }
     } else if (warp >= 2 && warp < 2 + EPI_WARPS) {
         // -------------------------------------------------------- epilogue
         // warp w: tensor-memory lanes 32*(w%4) .. +31 (this CTA's output rows),
@@ -528,8 +506,7 @@ template <bool PAIR> static cudaError_t prepare(int* units_out)
 }
 
 template <bool PAIR>
-static cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mO0,
-                               const CUtensorMap& mO1, Args a, cudaStream_t s)
+static cudaError_t launch_mode(const CUtensorMap& mO0, const CUtensorMap& mO1, Args a, cudaStream_t s)
 {
     int units = 0;
     cudaError_t e = prepare<PAIR>(&units);
@@ -539,7 +516,7 @@ static cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, con
     const int n = (int)(total < units ? total : units);
     constexpr size_t smem = smem_bytes<PAIR>();
     if (!PAIR) {
-        wgrad_tc_kernel<false><<<n, NUM_THREADS, smem, s>>>(mA, mB, mO0, mO1, a);
+        wgrad_tc_kernel<false><<<n, NUM_THREADS, smem, s>>>(mO0, mO1, a);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
@@ -554,20 +531,25 @@ static cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, con
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, wgrad_tc_kernel<true>, mA, mB, mO0, mO1, a);
+    return cudaLaunchKernelEx(&cfg, wgrad_tc_kernel<true>, mO0, mO1, a);
 }
 
 }  // namespace wg
 
+size_t wgrad_maps_bytes(int E) { return (size_t)2 * E * sizeof(CUtensorMap); }
+
 // out0/out1 (E, M, Nh) fp32 = for each expert, A[block]^T . B[block] with A
 // (max_rows, M) and B (max_rows, halves * Nh) bf16 row-major.  CTA pairs
-// (256-row output tiles) when M >= 256, single CTAs otherwise.
+// (256-row output tiles) when M >= 256, single CTAs otherwise.  `maps`: device
+// scratch of wgrad_maps_bytes(E), 128-byte aligned, that the launch rewrites
+// (the experts' operand maps).
 cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets, const void* A,
                                  int M, const void* B, int Nh, int halves, float* out0, float* out1,
-                                 int* status, cudaStream_t s)
+                                 void* maps, int* status, cudaStream_t s)
 {
     using namespace wg;
     if (E < 1 || E > MAX_E || M < 1 || Nh < 1 || (halves != 1 && halves != 2)) return cudaErrorInvalidValue;
+    if (maps == nullptr || ((uintptr_t)maps & 127) != 0) return cudaErrorInvalidValue;
     CUtensorMap mA, mB, mO0, mO1;
     if (!map_rows(&mA, A, (uint64_t)M, (uint64_t)max_rows) ||
         !map_rows(&mB, B, (uint64_t)Nh * halves, (uint64_t)max_rows) ||
@@ -577,8 +559,12 @@ cudaError_t launch_wgrad_tc_bf16(int E, int64_t max_rows, const int32_t* offsets
     // the A block of an expert (M columns) larger than its B block (halves * Nh):
     // walk the n tiles fastest (e.g. the down projection's gradient, M = F)
     const int n_fast = (int64_t)M > (int64_t)Nh * halves ? 1 : 0;
-    Args a{offsets, E, M, Nh, halves, 0, (Nh + BN - 1) / BN, n_fast, max_rows, status};
-    return M >= 256 ? launch_mode<true>(mA, mB, mO0, mO1, a, s) : launch_mode<false>(mA, mB, mO0, mO1, a, s);
+    CUtensorMap* gmaps = static_cast<CUtensorMap*>(maps);
+    wgrad_maps_kernel<<<(E + 127) / 128, 128, 0, s>>>(mA, mB, offsets, E, max_rows, gmaps);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    Args a{offsets, gmaps, E, M, Nh, halves, 0, (Nh + BN - 1) / BN, n_fast, max_rows, status};
+    return M >= 256 ? launch_mode<true>(mO0, mO1, a, s) : launch_mode<false>(mO0, mO1, a, s);
 }
 
 }  // namespace moe
