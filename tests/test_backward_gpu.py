@@ -144,6 +144,10 @@ SMALL = {
     "shared_bias_noise": Workload("shared_bias_noise", T=600, D=256, F=320, E=8, K=2,
                                   bias="zipf", noise=True, F_shared=192, capacity_factor=1.0),
     "many_experts_top1": Workload("many_experts_top1", T=256, D=128, F=128, E=64, K=1),
+    # more than 128 experts: the operand tensor maps of the weight-gradient GEMMs are written
+    # by two blocks; a few rows per expert (single CTAs, and CTA pairs for M >= 256)
+    "e256_single": Workload("e256_single", T=512, D=128, F=128, E=256, K=4),
+    "e200_pair": Workload("e200_pair", T=600, D=256, F=320, E=200, K=3, bias="zipf"),
     "single_expert": Workload("single_expert", T=100, D=128, F=192, E=1, K=1),
     "one_token": Workload("one_token", T=1, D=128, F=128, E=8, K=2),
     # few tokens and a long d_model: the combine splits each row over several warps
