@@ -98,7 +98,55 @@ def _to_dev(inp):
     return {k: dev(v) for k, v in inp.items()}
 
 
-@pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
+def _random_layer_cases(n=32, seed=77):
+    """Seeded random layers for the whole forward: bf16 and fp32, T from 1 token to
+    past the tensor-core router's threshold, d_model and d_hidden any multiple of 8
+    (ragged K and N tiles), 1 to 256 experts (single CTAs and CTA pairs), capacity
+    drops, every routing option, sometimes a shared expert."""
+    import random
+    rng = random.Random(seed)
+    cases = []
+    while len(cases) < n:
+        dtype = "f32" if rng.random() < 0.25 else "bf16"
+        E = rng.choice([1, 2, 3, 5, 8, 13, 16, 32, 64, 100, 256])
+        K = rng.randint(1, min(E, 8))
+        T = rng.choice([1, 7, 100, 333, 1000, 2049, 3000])
+        D = 8 * rng.randint(1, 66)
+        F = 8 * rng.randint(1, 66)
+        if T * K * D * F > 2_000_000_000:
+            continue
+        kw = dict(T=T, D=D, F=F, E=E, K=K, dtype=dtype, seed=500 + len(cases))
+        if rng.random() < 0.35:
+            kw["capacity_factor"] = rng.choice([0.5, 1.0, 1.25])
+        if rng.random() < 0.3:
+            kw["bias"] = "zipf"
+        if rng.random() < 0.3:
+            kw["noise"] = True
+        if rng.random() < 0.25:
+            kw["score_func"] = "sigmoid"
+        if rng.random() < 0.25:
+            kw["renormalize"] = False
+        if rng.random() < 0.2:
+            kw["route_scale"] = 1.5
+        if rng.random() < 0.25:
+            kw["sel_bias"] = True
+        groups = [g for g in (2, 4, 8) if E % g == 0]
+        if groups and rng.random() < 0.25:
+            g = rng.choice(groups)
+            tg = rng.randint(1, g)
+            if tg * (E // g) >= K:
+                kw["n_groups"], kw["topk_groups"] = g, tg
+        if rng.random() < 0.2:
+            kw["F_shared"] = 8 * rng.randint(1, 40)
+        name = "rand_" + "_".join(f"{k}{v}" for k, v in kw.items() if k != "seed")
+        cases.append(_wl(name, **kw))
+    return cases
+
+
+RANDOM_LAYERS = _random_layer_cases()
+
+
+@pytest.mark.parametrize("wl", SMALL + RANDOM_LAYERS, ids=[w.name for w in SMALL + RANDOM_LAYERS])
 def test_small_layers_elementwise(cuda_ok, wl):
     inp_cpu = make_inputs(wl, device="cpu")
     inp = _to_dev(inp_cpu)
