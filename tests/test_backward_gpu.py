@@ -163,6 +163,61 @@ SMALL = {
 }
 
 
+def _random_backward_cases(n=24, seed=91):
+    """Seeded random layers for the backward: bf16 and fp32, a few to a thousand tokens,
+    d_model and d_hidden any multiple of 8 (ragged K tails in the weight-gradient GEMMs,
+    ragged N tiles in dH and dX), 1 to 256 experts, drops, every routing option, some
+    with a shared expert."""
+    import random
+    rng = random.Random(seed)
+    cases = {}
+    while len(cases) < n:
+        dtype = "f32" if rng.random() < 0.3 else "bf16"
+        E = rng.choice([1, 2, 3, 5, 8, 16, 32, 64, 200, 256])
+        K = rng.randint(1, min(E, 8))
+        T = rng.choice([3, 50, 257, 600, 1000])
+        D = 8 * rng.randint(1, 40)
+        F = 8 * rng.randint(1, 40)
+        kw = dict(T=T, D=D, F=F, E=E, K=K, dtype=dtype, seed=900 + len(cases))
+        if rng.random() < 0.35:
+            kw["capacity_factor"] = rng.choice([0.5, 1.0, 1.25])
+        if rng.random() < 0.3:
+            kw["bias"] = "zipf"
+        if rng.random() < 0.3:
+            kw["noise"] = True
+        if rng.random() < 0.25:
+            kw["score_func"] = "sigmoid"
+        if rng.random() < 0.25:
+            kw["renormalize"] = False
+        if rng.random() < 0.2:
+            kw["route_scale"] = 1.5
+        if rng.random() < 0.25:
+            kw["sel_bias"] = True
+        groups = [g for g in (2, 4, 8) if E % g == 0]
+        if groups and rng.random() < 0.25:
+            g = rng.choice(groups)
+            tg = rng.randint(1, g)
+            if tg * (E // g) >= K:
+                kw["n_groups"], kw["topk_groups"] = g, tg
+        if rng.random() < 0.2:
+            kw["F_shared"] = 8 * rng.randint(1, 24)
+        name = "rand_" + "_".join(f"{k}{v}" for k, v in kw.items() if k != "seed")
+        cases[name] = Workload(name, **kw)
+    return cases
+
+
+RANDOM = _random_backward_cases()
+
+
+@pytest.mark.parametrize("name", sorted(RANDOM))
+def test_backward_random(name):
+    wl = RANDOM[name]
+    inp = make_inputs(wl)
+    dy = make_output_grad(wl)
+    got = run_train(wl, inp, dy)
+    compare_all(wl, inp, dy, got)
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_backward_small(name):
     wl = SMALL[name]
