@@ -205,6 +205,33 @@ PEER_CASES = {
 }
 
 
+
+def _random_peer_cases(n=8, seed=53):
+    """Seeded random layers over emulated ranks: 2, 4 or 8 ranks, any number of local
+    experts, K up to 8, ragged d_model and d_hidden, drops, a router bias."""
+    import random
+    rng = random.Random(seed)
+    out = {}
+    while len(out) < n:
+        W = rng.choice([2, 4, 8])
+        E = W * rng.choice([1, 2, 3, 4, 8])
+        K = rng.randint(1, min(E, 8))
+        T = rng.choice([1, 17, 100, 257])
+        D = 8 * rng.randint(2, 48)
+        F = 8 * rng.randint(2, 48)
+        kw = dict(T=T, D=D, F=F, E=E, K=K, seed=700 + len(out))
+        if rng.random() < 0.4:
+            kw["capacity_factor"] = rng.choice([0.5, 1.0])
+        if rng.random() < 0.4:
+            kw["bias"] = "zipf"
+        name = f"rand_w{W}_" + "_".join(f"{k}{v}" for k, v in kw.items() if k != "seed")
+        out[name] = (W, Workload(name, **kw), None)
+    return out
+
+
+PEER_CASES.update(_random_peer_cases())
+
+
 @pytest.mark.parametrize("name", sorted(PEER_CASES))
 def test_peer_exchange_emulated_ranks(name):
     W, wl, skew = PEER_CASES[name]
