@@ -399,6 +399,41 @@ def test_determinism_bitwise(cuda_ok):
         assert torch.equal(a, c)
 
 
+@pytest.mark.parametrize("wl", [
+    _wl("inv_tcr_pairs", T=4096, D=256, F=512, E=8, K=2, bias="zipf", seed=81),
+    _wl("inv_simt_single", T=600, D=136, F=200, E=16, K=4, seed=82),
+    _wl("inv_f32", T=512, D=64, F=96, E=8, K=2, dtype="f32", seed=83),
+    _wl("inv_shared", T=2048, D=128, F=256, E=4, K=2, F_shared=128, seed=84),
+], ids=lambda w: w.name)
+def test_batch_invariance_at_a_fixed_batch_size(cuda_ok, wl):
+    """Dropless layers: a token's output depends on that token alone, and the
+    kernels sum every output element in an order fixed by the shape, so the
+    same token gives the same bits whatever the other tokens of a batch of the
+    same size are (they change every expert's row count and so the tiles its
+    rows land in)."""
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    cfg = B.MoeConfig.make(wl.T, wl.D, wl.F, wl.E, wl.K, wl.dtype, wl.capacity_factor,
+                           F_shared=wl.F_shared, **wl.routing())
+    ws = torch.zeros(B.forward_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    terms = prepared_terms(cfg, inp["w_router"])
+    half = wl.T // 2
+    x1 = inp["x"]
+    g = torch.Generator(device="cuda").manual_seed(wl.seed + 1000)
+    x2 = x1.clone()
+    x2[half:] = (torch.randn(wl.T - half, wl.D, generator=g, device="cuda") * 3.0).to(x1.dtype)
+    x2[:half] = x1[:half].flip(0)  # the shared tokens also move to other rows
+    ys = []
+    for x in (x1, x2):
+        y = torch.empty_like(x)
+        B.moe_forward(cfg, x, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], y, ws,
+                      router_bias=inp["bias"], shared=inp["shared"], w_router_terms=terms)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status(ws) == 0
+    assert torch.equal(ys[1][:half].flip(0), ys[0][:half])
+    assert not torch.equal(ys[1][half:], ys[0][half:])
+
+
 def test_out_of_range_ids_raise_bounds_flag(cuda_ok):
     """Corrupt ids are caught by the dispatch kernels' own bounds checks: the
     status word gets the bounds flag and nothing is written out of range."""
