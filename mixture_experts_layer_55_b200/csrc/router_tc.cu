@@ -480,6 +480,9 @@ __global__ void __launch_bounds__(Threads<MINB>::NT, MINB)
                 const int rr = i / E;
                 dst[i] = Ls[rr * LDS + (i - rr * E)];
             }
+            // every row is copied before pass 3 rewrites its logits (with two halves
+            // the exchange's barriers below already order the two)
+            if (HALVES == 1) epi_sync<NTH>();
         }
         // pass 2: softmax sum, sum of exp(L - max) (L - max) for the entropy, and
         // the scores (sigmoid scores and their sum with score_func sigmoid)
