@@ -17,7 +17,7 @@ cudaError_t launch_ffn_simt_f32(const moe_config& c, int64_t max_rows, const voi
 cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                const void* w_gate, const void* w_up, const void* w_down, void* h,
-                               void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                               void* y_perm, void* gu_keep, void* amaps, int* status, cudaStream_t s,
                                StageHook mid, void* mid_ctx);
 
 int64_t capacity_of(const moe_config& c)
@@ -63,6 +63,8 @@ WsLayout ws_layout(const moe_config& c)
     o += align_up((size_t)nch * c.E * sizeof(int32_t));
     L.d_base = o;
     o += align_up((size_t)nch * c.E * sizeof(int32_t));
+    L.f_amaps = o;
+    o += c.dtype == MOE_BF16 ? align_up(2 * (size_t)c.E * kTensorMapBytes) : 0;
     L.total = o;
     return L;
 }
@@ -205,14 +207,14 @@ __global__ void set_row_range_kernel(int32_t* off, int32_t n)
 cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
                               const void* w_gate, const void* w_up, const void* w_down, void* h,
-                              void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                              void* y_perm, void* gu_keep, void* amaps, int* status, cudaStream_t s,
                               StageHook mid, void* mid_ctx)
 {
     if (c.dtype == MOE_F32)
         return launch_ffn_simt_f32(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up,
                                    w_down, h, y_perm, gu_keep, status, s, mid, mid_ctx);
     return launch_ffn_tc_bf16(c, max_rows, x_perm, offsets, perm, topk_w, w_gate, w_up, w_down, h,
-                              y_perm, gu_keep, status, s, mid, mid_ctx);
+                              y_perm, gu_keep, amaps, status, s, mid, mid_ctx);
 }
 
 // the backward's GEMMs in the layer's dtype: tensor cores for bf16, fp32 SIMT for fp32
@@ -404,7 +406,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + L.status);
     return cuda_status(launch_expert_ffn(*cfg, max_rows_of(*cfg), x_perm, offsets, perm, topk_w,
-                                         w_gate, w_up, w_down, h, y_perm, nullptr, status, s,
+                                         w_gate, w_up, w_down, h, y_perm, nullptr,
+                                         static_cast<char*>(workspace) + L.f_amaps, status, s,
                                          nullptr, nullptr));
 }
 
@@ -463,7 +466,8 @@ static cudaError_t run_forward(const moe_config& c, const void* x, const float* 
     if (e == cudaSuccess)
         e = launch_expert_ffn(c, max_rows, x_perm, offsets, train ? nullptr : perm,
                               train ? nullptr : w, w_gate, w_up, w_down, h, y_perm,
-                              train ? ws + TL->gu : nullptr, status, s, trace_mid_ffn, nullptr);
+                              train ? ws + TL->gu : nullptr, ws + F.ws.f_amaps, status, s, trace_mid_ffn,
+                              nullptr);
     trace(5, s);
     const void* y_add = nullptr;
     if (e == cudaSuccess && c.F_shared > 0) {
@@ -475,7 +479,7 @@ static cudaError_t run_forward(const moe_config& c, const void* x, const float* 
         if (e == cudaSuccess)
             e = launch_expert_ffn(cs, c.T, x, sh_off, nullptr, nullptr, w_gate_shared, w_up_shared,
                                   w_down_shared, ws + F.sh_h, ws + F.sh_y,
-                                  train ? ws + TL->sh_gu : nullptr, status, s, nullptr, nullptr);
+                                  train ? ws + TL->sh_gu : nullptr, nullptr, status, s, nullptr, nullptr);
         y_add = ws + F.sh_y;
     }
     trace(6, s);
@@ -705,7 +709,8 @@ int32_t moe_forward_kernel_count(const moe_config* cfg, int32_t router_terms_giv
     // gather 1, expert GEMMs 2, combine 1; router: the tensor-core kernel (after
     // the weight split when the caller passes no prepared terms), or the SIMT
     // logits (+ their split sum) and the top-k kernel
-    const int rest = 5 + (dispatch_index_fused(*cfg) ? 0 : 2) + shared;
+    // (bf16: and the kernel that writes the experts' A maps before the GEMMs)
+    const int rest = 5 + (cfg->dtype == MOE_BF16 ? 1 : 0) + (dispatch_index_fused(*cfg) ? 0 : 2) + shared;
     if (router_tc_eligible(*cfg)) return (router_terms_given ? 1 : 2) + rest;
     return 2 + (router_plan(*cfg).splits > kTopkMaxSplits ? 1 : 0) + rest;
 }

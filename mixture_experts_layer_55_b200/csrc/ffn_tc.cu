@@ -116,7 +116,51 @@ struct Args {
     __nv_bfloat16* gu_out;       // gate/up: keep [g | u] here, row stride 2N (null: do not)
     const __nv_bfloat16* gu_in;  // dgrad-h: the kept [g | u], row stride 2N
     int* status;
+    const CUtensorMap* amaps;    // forward modes: A's map per expert, rows ending at its end (null: tmA)
 };
+
+// A tensor map in global memory, rewritten by the generic proxy: its row extent
+// (dimension 1; dimension 0 is the contiguous one) is replaced in place; the
+// writer releases the maps to the copy engine's view, each reader acquires the
+// one it is about to use (which also drops a stale cached copy of it).
+MOE_DEVICE void tmap_set_rows(CUtensorMap* gmap, uint32_t rows)
+{
+    asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(gmap), "r"(rows)
+                 : "memory");
+}
+
+MOE_DEVICE void tmap_release() { asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory"); }
+
+MOE_DEVICE void tmap_acquire(const CUtensorMap* gmap)
+{
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
+}
+
+// maps[e] = tmX, maps[E + e] = tmH, each with the row extent cut to expert e's
+// end (offsets[e+1], clamped to 1 .. max_rows: a malformed offset can only
+// shorten the rows a map reaches).  A tile's rows past its expert's end then
+// arrive as zeros from the copy engine instead of being read (their results are
+// never stored).  One thread per expert.
+__global__ void ffn_amaps_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmH,
+                                 const int32_t* offsets, int E, int64_t max_rows, CUtensorMap* maps)
+{
+    const int e = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    if (e >= E) return;
+    int64_t r1 = offsets[e + 1];
+    r1 = r1 < 1 ? 1 : (r1 > max_rows ? max_rows : r1);
+    const uint4* sx = reinterpret_cast<const uint4*>(&tmX);
+    const uint4* sh = reinterpret_cast<const uint4*>(&tmH);
+    uint4* dx = reinterpret_cast<uint4*>(&maps[e]);
+    uint4* dh = reinterpret_cast<uint4*>(&maps[E + e]);
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(CUtensorMap) / sizeof(uint4)); ++i) {
+        dx[i] = sx[i];
+        dh[i] = sh[i];
+    }
+    tmap_set_rows(&maps[e], (uint32_t)r1);
+    tmap_set_rows(&maps[E + e], (uint32_t)r1);
+    tmap_release();
+}
 
 MOE_DEVICE void decode_tile(const Misc* m, int E, int bm, int bn, int t, int& e, int& m_row0,
                             int& row_end, int& n0)
@@ -256,10 +300,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int last_phase[STAGES];
         for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
         bool ok = true;
+        int last_e = -1;
         for (int t = unit; t < total && ok; t += units) {
             int e, m_row0, row_end, n0;
             decode_tile(m, E, BM, BN, t, e, m_row0, row_end, n0);
             const int a_row = m_row0 + (int)rank * 128;
+            // forward modes: the expert's own A map (rows past its end read as zeros)
+            const CUtensorMap* mA = &tmA;
+            if ((MODE == kGateUp || MODE == kDown) && a.amaps != nullptr) {
+                mA = a.amaps + e;
+                if (e != last_e) {
+                    tmap_acquire(mA);
+                    last_e = e;
+                }
+            }
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!mbar_wait(&m->empty[stage], phase ^ 1u, a.status, 410, abort_flag)) {
                     ok = false;
@@ -301,7 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     // both CTAs' bytes are counted on the leader's full barrier
                     if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
                     const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
-                    tma_load_2d_pair(sA, &tmA, k0, a_row, fb);
+                    tma_load_2d_pair(sA, mA, k0, a_row, fb);
                     if (GATEUP) {  // this CTA's [gate 64 | up 64] columns
                         tma_load_3d_pair(sB, &tmB0, n0 + 64 * (int)rank, k0, e, fb);
                         tma_load_3d_pair(sB + BOX_BYTES, &tmB1, n0 + 64 * (int)rank, k0, e, fb);
@@ -312,7 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 } else {
                     uint64_t* fb = &m->full[stage];
                     mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(sA, &tmA, k0, a_row, fb);
+                    tma_load_2d(sA, mA, k0, a_row, fb);
                     if (GATEUP) {  // [gate n0 | up n0 | gate n0+64 | up n0+64]
                         tma_load_3d(sB, &tmB0, n0, k0, e, fb);
                         tma_load_3d(sB + BOX_BYTES, &tmB1, n0, k0, e, fb);
@@ -792,7 +846,7 @@ static bool use_pairs(const moe_config& c, int64_t max_rows) { return max_rows >
 cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void* x_perm,
                                const int32_t* offsets, const int32_t* perm, const float* topk_w,
                                const void* w_gate, const void* w_up, const void* w_down, void* h,
-                               void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                               void* y_perm, void* gu_keep, void* amaps, int* status, cudaStream_t s,
                                StageHook mid, void* mid_ctx)
 {
     using namespace tc;
@@ -813,15 +867,24 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
     const int64_t bm = pair ? 256 : 128;
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
 
+    // each expert's A maps (x_perm for gate/up, h for down), rows ending at the expert's end
+    CUtensorMap* gmaps = nullptr;
+    if (amaps != nullptr && (reinterpret_cast<uintptr_t>(amaps) & 127u) == 0) {
+        gmaps = static_cast<CUtensorMap*>(amaps);
+        ffn_amaps_kernel<<<(c.E + 127) / 128, 128, 0, s>>>(mA, mH, offsets, c.E, max_rows, gmaps);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     Args a1{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(h), c.E, c.D, c.F,
             (c.F + 127) / 128, c.F, max_rows, c.T * c.K,
-            static_cast<__nv_bfloat16*>(gu_keep), nullptr, status};
+            static_cast<__nv_bfloat16*>(gu_keep), nullptr, status, gmaps};
     cudaError_t err = pair ? launch_one<kGateUp, true>(mA, mG, mU, mHo, mGUo, a1, mtiles_bound * a1.n_tiles, s)
                            : launch_one<kGateUp, false>(mA, mG, mU, mHo, mGUo, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     Args a2{offsets, perm, topk_w, static_cast<__nv_bfloat16*>(y_perm), c.E, c.F, c.D,
-            (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status};
+            (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status,
+            gmaps ? gmaps + c.E : nullptr};
     return pair ? launch_one<kDown, true>(mH, mD, mD, mYo, mYo, a2, mtiles_bound * a2.n_tiles, s)
                 : launch_one<kDown, false>(mH, mD, mD, mYo, mYo, a2, mtiles_bound * a2.n_tiles, s);
 }

@@ -94,9 +94,11 @@ struct WsLayout {
     size_t r_cnt;       // nb_topk * E int32
     size_t d_cnt;       // chunks * E int32
     size_t d_base;      // chunks * E int32
+    size_t f_amaps;     // bf16 layers: the expert GEMMs' per-expert A maps (2 E tensor maps)
     size_t total;
 };
 WsLayout ws_layout(const moe_config& c);
+constexpr size_t kTensorMapBytes = 128;  // one CUtensorMap
 
 struct FwdLayout {
     WsLayout ws;        // scratch at offset 0
@@ -190,10 +192,13 @@ cudaError_t launch_combine(const moe_config& c, const void* y_perm, const int32_
 // null): it is called after the gate/up launch.
 typedef void (*StageHook)(void* ctx, cudaStream_t s);
 // gu_keep (max_rows, 2F) or null: where the gate/up GEMM keeps [g | u] (bf16 only).
+// amaps: null, or 2 E * kTensorMapBytes of device scratch, 128-byte aligned, where
+// the bf16 GEMMs write each expert's A maps (rows past the expert's end then read
+// as zeros instead of being fetched).
 cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void* x_perm,
                               const int32_t* offsets, const int32_t* perm, const float* topk_w,
                               const void* w_gate, const void* w_up, const void* w_down, void* h,
-                              void* y_perm, void* gu_keep, int* status, cudaStream_t s,
+                              void* y_perm, void* gu_keep, void* amaps, int* status, cudaStream_t s,
                               StageHook mid, void* mid_ctx);
 
 // ---------------------------------------------------------------- backward --

@@ -163,17 +163,18 @@ def test_forward_kernel_count(lib):
     assert B.forward_kernel_count(_cfg(T=512, D=256, F=512, E=8, K=2, dtype="f32")) == 7
     # tensor-core router: one kernel for routing and statistics, with or without the
     # d_model split (64 tiles of 128 tokens: a cluster of 2 CTAs per tile), after the
-    # weight split unless the caller passes prepared terms
-    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=16, K=2), True) == 6
-    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=64, K=6), True) == 6
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2), True) == 6
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 7
-    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 8  # split SIMT router
-    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8), True) == 8
+    # weight split unless the caller passes prepared terms; bf16 layers also write the
+    # experts' A maps before the GEMMs (one kernel)
+    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=16, K=2), True) == 7
+    assert B.forward_kernel_count(_cfg(T=16384, D=2048, F=1408, E=64, K=6), True) == 7
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2), True) == 7
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2)) == 8
+    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8)) == 9  # split SIMT router
+    assert B.forward_kernel_count(_cfg(T=128, D=7168, F=2048, E=256, K=8), True) == 9
     assert B.forward_kernel_count(_cfg(K=0)) == 0
-    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256), True) == 9
+    assert B.forward_kernel_count(_cfg(T=8192, D=4096, F=14336, E=8, K=2, F_shared=256), True) == 10
     # more chunks of 2048 assignments than SMs: the three-kernel index pass
-    assert B.forward_kernel_count(_cfg(T=160000, D=256, F=256, E=8, K=2), True) == 8
+    assert B.forward_kernel_count(_cfg(T=160000, D=256, F=256, E=8, K=2), True) == 9
 
 
 def test_router_terms_size_and_prepare_checks(lib):
