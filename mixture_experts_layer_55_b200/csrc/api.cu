@@ -134,6 +134,7 @@ BwdLayout bwd_layout(const moe_config& c, int64_t max_rows)
     // two launches (dWd, then [dWg | dWu]) of E experts each, one slot apiece
     B.tmaps = o;    o += c.dtype == MOE_BF16 ? 2 * align_up(wgrad_maps_bytes(c.E)) : 0;
     B.tmaps_sh = o; o += c.dtype == MOE_BF16 && c.F_shared > 0 ? 2 * align_up(wgrad_maps_bytes(1)) : 0;
+    B.dmaps = o;    o += c.dtype == MOE_BF16 ? align_up(2 * (size_t)c.E * kTensorMapBytes) : 0;
     B.total = o;
     return B;
 }
@@ -220,13 +221,14 @@ cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void*
 // the backward's GEMMs in the layer's dtype: tensor cores for bf16, fp32 SIMT for fp32
 static cudaError_t launch_dgrad(const moe_config& c, int64_t max_rows, const void* dyp, const int32_t* offsets,
                                 const void* gu, const void* w_gate, const void* w_up, const void* w_down,
-                                void* dgu, void* dxp, int* status, cudaStream_t s, StageHook mid, void* mid_ctx)
+                                void* dgu, void* dxp, void* amaps, int* status, cudaStream_t s, StageHook mid,
+                                void* mid_ctx)
 {
     if (c.dtype == MOE_F32)
         return launch_dgrad_simt_f32(c, max_rows, dyp, offsets, gu, w_gate, w_up, w_down, dgu, dxp, status, s,
                                      mid, mid_ctx);
-    return launch_dgrad_tc_bf16(c, max_rows, dyp, offsets, gu, w_gate, w_up, w_down, dgu, dxp, status, s, mid,
-                                mid_ctx);
+    return launch_dgrad_tc_bf16(c, max_rows, dyp, offsets, gu, w_gate, w_up, w_down, dgu, dxp, amaps, status, s,
+                                mid, mid_ctx);
 }
 
 static cudaError_t launch_wgrad(int32_t dt, int E, int64_t max_rows, const int32_t* offsets, const void* a,
@@ -631,7 +633,7 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
     btrace(2, s);
     if (e == cudaSuccess)  // dH -> [dg | du], then dXp (boundary 3 between the two)
         e = launch_dgrad(c, max_rows, ws + B.dyp, offsets, sv + TL.gu, w_gate, w_up, w_down,
-                                 ws + B.dgu, ws + B.dxp, status, s, btrace_mid_dgrad, nullptr);
+                         ws + B.dgu, ws + B.dxp, ws + B.dmaps, status, s, btrace_mid_dgrad, nullptr);
     btrace(4, s);
     if (e == cudaSuccess)  // dWd = h^T dYp
         e = launch_wgrad(c.dtype, c.E, max_rows, offsets, sv + F.h, c.F, ws + B.dyp, c.D, 1, dw_down,
@@ -646,8 +648,8 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const float* w_rou
         const moe_config cs = shared_config(c);
         const int32_t* sh_off = reinterpret_cast<const int32_t*>(sv + F.sh_offsets);
         e = launch_dgrad(cs, c.T, dy, sh_off, sv + TL.sh_gu, w_gate_shared, w_up_shared,
-                                 w_down_shared, ws + B.sh_dgu, ws + B.sh_dx, status, s, nullptr,
-                                 nullptr);
+                         w_down_shared, ws + B.sh_dgu, ws + B.sh_dx, nullptr, status, s, nullptr,
+                         nullptr);
         if (e == cudaSuccess)
             e = launch_wgrad(c.dtype, 1, c.T, sh_off, sv + F.sh_h, c.F_shared, dy, c.D, 1,
                              dw_down_shared, nullptr, ws + B.tmaps_sh, status, s);
@@ -859,9 +861,10 @@ int32_t moe_backward_kernel_count(const moe_config* cfg)
     // rows, router, two dgrad GEMMs, two wgrad GEMMs, router weight partials,
     // their sum, the bias gradient, dx; the shared expert adds its two dgrad
     // and two wgrad GEMMs.  In bf16 layers each wgrad GEMM is preceded by the
-    // kernel that writes its experts' operand maps.
+    // kernel that writes its experts' operand maps, and the dgrad GEMMs by one
+    // that writes their experts' A maps.
     const int maps = cfg->dtype == MOE_BF16 ? 1 : 0;
-    return 10 + 2 * maps + (cfg->F_shared > 0 ? 4 + 2 * maps : 0);
+    return 10 + 3 * maps + (cfg->F_shared > 0 ? 4 + 2 * maps : 0);
 }
 
 moe_status moe_trace_attach_backward(void* const* events, int32_t n_events)

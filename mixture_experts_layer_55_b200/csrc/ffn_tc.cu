@@ -116,7 +116,7 @@ struct Args {
     __nv_bfloat16* gu_out;       // gate/up: keep [g | u] here, row stride 2N (null: do not)
     const __nv_bfloat16* gu_in;  // dgrad-h: the kept [g | u], row stride 2N
     int* status;
-    const CUtensorMap* amaps;    // forward modes: A's map per expert, rows ending at its end (null: tmA)
+    const CUtensorMap* amaps;    // A's map per expert, rows ending at the expert's end (null: tmA)
 };
 
 // A tensor map in global memory, rewritten by the generic proxy: its row extent
@@ -126,6 +126,13 @@ struct Args {
 MOE_DEVICE void tmap_set_rows(CUtensorMap* gmap, uint32_t rows)
 {
     asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(gmap), "r"(rows)
+                 : "memory");
+}
+
+// the same for a 3-D map whose rows are dimension 2 ([dg | du] viewed as (rows, 2, F))
+MOE_DEVICE void tmap_set_rows_dim2(CUtensorMap* gmap, uint32_t rows)
+{
+    asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 2, %1;" ::"l"(gmap), "r"(rows)
                  : "memory");
 }
 
@@ -140,9 +147,12 @@ MOE_DEVICE void tmap_acquire(const CUtensorMap* gmap)
 // end (offsets[e+1], clamped to 1 .. max_rows: a malformed offset can only
 // shorten the rows a map reaches).  A tile's rows past its expert's end then
 // arrive as zeros from the copy engine instead of being read (their results are
-// never stored).  One thread per expert.
+// never stored).  The forward's pair is (x_perm, h), both 2-D; the backward's
+// (dYp, [dg | du]), the second 3-D with its rows in dimension 2 (h_rows_dim2).
+// One thread per expert.
 __global__ void ffn_amaps_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmH,
-                                 const int32_t* offsets, int E, int64_t max_rows, CUtensorMap* maps)
+                                 const int32_t* offsets, int E, int64_t max_rows, int h_rows_dim2,
+                                 CUtensorMap* maps)
 {
     const int e = (int)(blockIdx.x * blockDim.x + threadIdx.x);
     if (e >= E) return;
@@ -158,7 +168,8 @@ __global__ void ffn_amaps_kernel(const __grid_constant__ CUtensorMap tmX, const 
         dh[i] = sh[i];
     }
     tmap_set_rows(&maps[e], (uint32_t)r1);
-    tmap_set_rows(&maps[E + e], (uint32_t)r1);
+    if (h_rows_dim2) tmap_set_rows_dim2(&maps[E + e], (uint32_t)r1);
+    else tmap_set_rows(&maps[E + e], (uint32_t)r1);
     tmap_release();
 }
 
@@ -305,9 +316,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int e, m_row0, row_end, n0;
             decode_tile(m, E, BM, BN, t, e, m_row0, row_end, n0);
             const int a_row = m_row0 + (int)rank * 128;
-            // forward modes: the expert's own A map (rows past its end read as zeros)
+            // the expert's own A map (rows past its end read as zeros)
             const CUtensorMap* mA = &tmA;
-            if ((MODE == kGateUp || MODE == kDown) && a.amaps != nullptr) {
+            if (a.amaps != nullptr) {
                 mA = a.amaps + e;
                 if (e != last_e) {
                     tmap_acquire(mA);
@@ -330,12 +341,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (PAIR) {
                         if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
                         const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
-                        tma_load_3d_pair(sA, &tmA, kk0, hf, a_row, fb);
+                        tma_load_3d_pair(sA, mA, kk0, hf, a_row, fb);
                         tma_load_3d_pair(sB, mb, kk0, n0 + 128 * (int)rank, e, fb);
                     } else {
                         uint64_t* fb = &m->full[stage];
                         mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                        tma_load_3d(sA, &tmA, kk0, hf, a_row, fb);
+                        tma_load_3d(sA, mA, kk0, hf, a_row, fb);
                         tma_load_3d(sB, mb, kk0, n0, e, fb);
                     }
                 } else if (MODE == kDgradH) {
@@ -343,12 +354,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (PAIR) {
                         if (rank == 0) mbar_arrive_expect_tx(&m->full[stage], 2 * STAGE_BYTES);
                         const uint32_t fb = mapa_shared(smem_u32(&m->full[stage]), 0);
-                        tma_load_2d_pair(sA, &tmA, k0, a_row, fb);
+                        tma_load_2d_pair(sA, mA, k0, a_row, fb);
                         tma_load_3d_pair(sB, &tmB0, k0, n0 + 128 * (int)rank, e, fb);
                     } else {
                         uint64_t* fb = &m->full[stage];
                         mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                        tma_load_2d(sA, &tmA, k0, a_row, fb);
+                        tma_load_2d(sA, mA, k0, a_row, fb);
                         tma_load_3d(sB, &tmB0, k0, n0, e, fb);
                     }
                 } else if (PAIR) {
@@ -871,7 +882,7 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
     CUtensorMap* gmaps = nullptr;
     if (amaps != nullptr && (reinterpret_cast<uintptr_t>(amaps) & 127u) == 0) {
         gmaps = static_cast<CUtensorMap*>(amaps);
-        ffn_amaps_kernel<<<(c.E + 127) / 128, 128, 0, s>>>(mA, mH, offsets, c.E, max_rows, gmaps);
+        ffn_amaps_kernel<<<(c.E + 127) / 128, 128, 0, s>>>(mA, mH, offsets, c.E, max_rows, 0, gmaps);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -892,7 +903,7 @@ cudaError_t launch_ffn_tc_bf16(const moe_config& c, int64_t max_rows, const void
 cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const void* dyp,
                                  const int32_t* offsets, const void* gu, const void* w_gate,
                                  const void* w_up, const void* w_down, void* dgu, void* dxp,
-                                 int* status, cudaStream_t s, StageHook mid, void* mid_ctx)
+                                 void* amaps, int* status, cudaStream_t s, StageHook mid, void* mid_ctx)
 {
     using namespace tc;
     const bool pair = use_pairs(c, max_rows);
@@ -911,17 +922,26 @@ cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const vo
         return cudaErrorInvalidValue;
     const int64_t bm = pair ? 256 : 128;
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
+    // each expert's A maps (dYp for dH, [dg | du] for dX), rows ending at the expert's end
+    CUtensorMap* gmaps = nullptr;
+    if (amaps != nullptr && (reinterpret_cast<uintptr_t>(amaps) & 127u) == 0) {
+        gmaps = static_cast<CUtensorMap*>(amaps);
+        ffn_amaps_kernel<<<(c.E + 127) / 128, 128, 0, s>>>(mA, mDGU, offsets, c.E, max_rows, 1, gmaps);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     // dH = dYp . Wd^T (K = D), epilogue through SwiGLU into [dg | du]
     Args a1{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dgu), c.E, c.D, c.F,
             (c.F + 255) / 256, 2 * (int64_t)c.F, max_rows, c.T * c.K, nullptr,
-            static_cast<const __nv_bfloat16*>(gu), status};
+            static_cast<const __nv_bfloat16*>(gu), status, gmaps};
     cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mWd, mOut, mOut, a1, mtiles_bound * a1.n_tiles, s)
                            : launch_one<kDgradH, false>(mA, mWd, mWd, mOut, mOut, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     // dXp = [dg | du] . [Wg | Wu]^T (K = 2F), unit weights
     Args a2{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dxp), c.E, c.F, c.D,
-            (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status};
+            (c.D + 255) / 256, c.D, max_rows, c.T * c.K, nullptr, nullptr, status,
+            gmaps ? gmaps + c.E : nullptr};
     return pair ? launch_one<kDgradX, true>(mDGU, mG, mU, mXo, mXo, a2, mtiles_bound * a2.n_tiles, s)
                 : launch_one<kDgradX, false>(mDGU, mG, mU, mXo, mXo, a2, mtiles_bound * a2.n_tiles, s);
 }

@@ -133,6 +133,7 @@ struct BwdLayout {
     size_t sh_dgu;      // (T, 2 F_shared)
     size_t sh_dx;       // (T, D)
     size_t tmaps;       // the weight-gradient GEMMs' per-expert tensor maps (bf16 layers)
+    size_t dmaps;       // the dgrad GEMMs' per-expert A maps (bf16 layers)
     size_t tmaps_sh;    // and the shared expert's
     int rw_splits;
     size_t total;
@@ -203,10 +204,12 @@ cudaError_t launch_expert_ffn(const moe_config& c, int64_t max_rows, const void*
 
 // ---------------------------------------------------------------- backward --
 // dH = dYp . Wd^T through SwiGLU into dgu = [dg | du], then dXp = dgu . [Wg | Wu]^T.
+// amaps: null, or 2 E * kTensorMapBytes of device scratch (128-byte aligned) for
+// each expert's A maps, as for the forward's expert GEMMs.
 cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const void* dyp,
                                  const int32_t* offsets, const void* gu, const void* w_gate,
                                  const void* w_up, const void* w_down, void* dgu, void* dxp,
-                                 int* status, cudaStream_t s, StageHook mid, void* mid_ctx);
+                                 void* amaps, int* status, cudaStream_t s, StageHook mid, void* mid_ctx);
 // out0 / out1 (E, M, Nh) fp32 = A[block]^T . B[block] per expert block.
 // `maps`: device scratch of wgrad_maps_bytes(E) bytes, 128-byte aligned,
 // rewritten by the launch (each expert's operand tensor maps).

@@ -209,9 +209,10 @@ def test_backward_sizes_counts_and_trace(lib):
     c = _cfg(T=1200, D=256, F=384, E=4, K=2)
     assert B.train_state_size(c) > B.forward_workspace_size(c)
     assert B.backward_workspace_size(c) > 0
-    # bf16: each weight-gradient GEMM is preceded by its operand-map kernel
-    assert B.backward_kernel_count(c) == 12
-    assert B.backward_kernel_count(_cfg(T=600, F=320, F_shared=192, capacity_factor=1.0)) == 18
+    # bf16: each weight-gradient GEMM is preceded by its operand-map kernel, and the
+    # dgrad GEMMs by one that writes their experts' A maps
+    assert B.backward_kernel_count(c) == 13
+    assert B.backward_kernel_count(_cfg(T=600, F=320, F_shared=192, capacity_factor=1.0)) == 19
     cf = _cfg(dtype="f32")  # fp32 layers: SIMT GEMMs, no tensor maps
     assert B.backward_kernel_count(cf) == 10
     assert B.train_state_size(cf) > B.train_state_size(_cfg())  # 4-byte activations
