@@ -434,6 +434,38 @@ def test_batch_invariance_at_a_fixed_batch_size(cuda_ok, wl):
     assert not torch.equal(ys[1][half:], ys[0][half:])
 
 
+@pytest.mark.parametrize("wl", [
+    _wl("bad_offsets_pair", T=600, D=128, F=136, E=4, K=2, seed=85),
+    _wl("bad_offsets_single", T=100, D=72, F=64, E=8, K=2, seed=86),
+    _wl("bad_offsets_f32", T=200, D=64, F=64, E=4, K=2, dtype="f32", seed=87),
+], ids=lambda w: w.name)
+def test_malformed_offsets_raise_bounds_flag(cuda_ok, wl):
+    """Row offsets that decrease or run past max_rows, handed straight to
+    moe_expert_ffn: the GEMM kernels' own checks treat those expert blocks as
+    empty and raise the bounds flag (the per-expert A maps are clamped to the
+    buffer as well); after the flag is cleared a well-formed call runs clean."""
+    inp = _to_dev(make_inputs(wl, device="cpu"))
+    b = Bufs(wl)
+    b.run_ops(inp)
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status(b.ws) == 0
+    R = b.max_rows
+    good = b.offsets.clone()
+    bad = good.clone()
+    bad[1] = min(int(good[2]) + 5, R)     # expert 0 runs past expert 1's start...
+    bad[2] = max(int(good[1]) - 3, 0)     # ...and expert 1's block ends before it begins
+    bad[wl.E - 1] = R + 77                # past the buffers
+    B.moe_expert_ffn(b.cfg, b.x_perm, bad, b.perm, b.w, inp["w_gate"], inp["w_up"], inp["w_down"],
+                     b.h, b.y_perm, b.ws)
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status(b.ws) & 0x2
+    B.moe_clear_device_status(b.ws)
+    B.moe_expert_ffn(b.cfg, b.x_perm, good, b.perm, b.w, inp["w_gate"], inp["w_up"], inp["w_down"],
+                     b.h, b.y_perm, b.ws)
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status(b.ws) == 0
+
+
 def test_out_of_range_ids_raise_bounds_flag(cuda_ok):
     """Corrupt ids are caught by the dispatch kernels' own bounds checks: the
     status word gets the bounds flag and nothing is written out of range."""
