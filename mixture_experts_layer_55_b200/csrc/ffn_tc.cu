@@ -87,6 +87,7 @@ struct Misc {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
+    uint64_t gbar[8];     // dgrad-h: an epilogue warp's [g | u] piece has landed (one per warp)
     uint32_t tmem_base;
     int abort_flag;
     int row0[MAX_E];
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&m->tempty[b], G::EPI_ARRIVALS);
         }
         mbar_init(&m->drain, 1);
+        for (int w = 0; w < 8; ++w) mbar_init(&m->gbar[w], 1);
         m->abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -465,6 +467,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m->tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m->tempty[1]), 0);
         uint8_t* obuf = outbuf + (size_t)(warp - 2) * G::OUT_BYTES;  // staging (dgrad-h: [dg | du])
+        uint64_t* gbar = &m->gbar[warp - 2];
+        uint32_t gphase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = unit; t < total; t += units) {
@@ -534,21 +538,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             } else if (MODE == kDgradH) {
 #pragma unroll 1
                 for (int c = 4 * half; c < 4 * half + 4; ++c) {
+                    const int col = n0 + c * 32;
+                    // a warp whose 32 rows all belong to the expert has its [g | u]
+                    // piece copied into its staging buffer by TMA (tmO1 maps the kept
+                    // [g | u] like the [dg | du] stores, 64-byte swizzle), once the
+                    // last stores have read the buffer; the others load by lane
+                    const bool tma_in = warp_full && col < a.N;
+                    if (tma_in) {
+                        if (lane == 0) {
+                            bulk_wait_read<0>();
+                            mbar_arrive_expect_tx(gbar, 4096);
+                            tma_load_3d(obuf, &tmO1, col, 0, (int)warp_row0, gbar);
+                            tma_load_3d(obuf + 2048, &tmO1, col, 1, (int)warp_row0, gbar);
+                        }
+                        __syncwarp();
+                    }
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
                     tmem_ld_wait();
-                    const int col = n0 + c * 32;
-                    if (warp_full && col < a.N) {
-                        if (lane == 0) bulk_wait_read<0>();  // the last stores have read the buffer
+                    if (tma_in) {
+                        // an abort elsewhere ends the first wait early: the copy is still
+                        // let land (bounded) before the buffer is touched or the CTA exits
+                        if (!__all_sync(0xffffffffu, mbar_wait(gbar, gphase, a.status, 432, abort_flag)))
+                            mbar_wait(gbar, gphase, a.status, 433, nullptr);
                         __syncwarp();
+                        gphase ^= 1u;
                     }
                     if (valid && col < a.N) {
                         const __nv_bfloat16* grow = a.gu_in + row * 2 * (int64_t)a.N + col;
+                        const uint4* gsrc = reinterpret_cast<const uint4*>(obuf + lane * 64);
+                        const uint4* usrc = reinterpret_cast<const uint4*>(obuf + 2048 + lane * 64);
+                        const int swz = (lane >> 1) & 3;
                         uint32_t dg[16], du[16];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             uint4 gq = make_uint4(0, 0, 0, 0), uq = make_uint4(0, 0, 0, 0);
-                            if (col + 8 * q < a.N) {
+                            if (tma_in) {  // columns past F arrived as zeros
+                                gq = gsrc[q ^ swz];
+                                uq = usrc[q ^ swz];
+                            } else if (col + 8 * q < a.N) {
                                 gq = *reinterpret_cast<const uint4*>(grow + 8 * q);
                                 uq = *reinterpret_cast<const uint4*>(grow + a.N + 8 * q);
                             }
@@ -915,10 +943,12 @@ cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const vo
         !map_3d_kmajor(&mG, w_gate, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows) ||
         !map_3d_kmajor(&mU, w_up, (uint64_t)c.F, (uint64_t)c.D, (uint64_t)c.E, brows))
         return cudaErrorInvalidValue;
-    // the epilogues' stores: [dg | du] viewed as (rows, 2, F), dXp (rows, D)
-    CUtensorMap mOut, mXo;
+    // the epilogues' stores: [dg | du] viewed as (rows, 2, F), dXp (rows, D); and the dH
+    // epilogue's loads of the kept [g | u] pieces, laid out like the [dg | du] stores
+    CUtensorMap mOut, mXo, mGUin;
     if (!map_halves_store(&mOut, dgu, (uint64_t)c.F, (uint64_t)max_rows) ||
-        !map_store_2d(&mXo, dxp, (uint64_t)c.D, (uint64_t)max_rows))
+        !map_store_2d(&mXo, dxp, (uint64_t)c.D, (uint64_t)max_rows) ||
+        !map_halves_store(&mGUin, gu, (uint64_t)c.F, (uint64_t)max_rows))
         return cudaErrorInvalidValue;
     const int64_t bm = pair ? 256 : 128;
     const int64_t mtiles_bound = (max_rows + bm - 1) / bm + c.E;
@@ -934,8 +964,8 @@ cudaError_t launch_dgrad_tc_bf16(const moe_config& c, int64_t max_rows, const vo
     Args a1{offsets, nullptr, nullptr, static_cast<__nv_bfloat16*>(dgu), c.E, c.D, c.F,
             (c.F + 255) / 256, 2 * (int64_t)c.F, max_rows, c.T * c.K, nullptr,
             static_cast<const __nv_bfloat16*>(gu), status, gmaps};
-    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mWd, mOut, mOut, a1, mtiles_bound * a1.n_tiles, s)
-                           : launch_one<kDgradH, false>(mA, mWd, mWd, mOut, mOut, a1, mtiles_bound * a1.n_tiles, s);
+    cudaError_t err = pair ? launch_one<kDgradH, true>(mA, mWd, mWd, mOut, mGUin, a1, mtiles_bound * a1.n_tiles, s)
+                           : launch_one<kDgradH, false>(mA, mWd, mWd, mOut, mGUin, a1, mtiles_bound * a1.n_tiles, s);
     if (err != cudaSuccess) return err;
     if (mid) mid(mid_ctx, s);
     // dXp = [dg | du] . [Wg | Wu]^T (K = 2F), unit weights
